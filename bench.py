@@ -1,0 +1,513 @@
+"""Throughput of the GPTQ hot path: weights quantized per second.
+
+One step = one pass of the whole path over one decoder layer's problems:
+  for every Hessian of the layer: zero H, gptq_hessian_accumulate (K1),
+  gptq_prepare (K2), gptq_quantize (ingest, K3/K4 per block, K5).
+Default workload: one SmolLM-135M-shaped decoder layer (q/k/v/o/gate/up
+4608×576 on one H, down 576×1536 on another), 2048 cone-structured
+calibration tokens, 4-bit, group 128, block 128, damp 0.01.
+
+    python bench.py --gpus N --steps K --warmup W [--config C] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank quantizes its own,
+independent layer (no collective on the data path: weak scaling); timing is
+the max over ranks of the device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import CONFIGS, problems_for  # noqa: E402
+
+METRIC = "GPTQ weights quantized/sec (params/s incl. Hessian) & % of roofline, 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------- host helpers
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def layer_for_rank(rank: int) -> int:
+    """Each rank quantizes its own, independent layer (seed block = rank)."""
+    return rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def workload_name(cid: int, bits: int) -> str:
+    c = CONFIGS[cid]
+    if c["kind"] == "decoder":
+        h, kv, it = c["hidden"], c["kv"], c["inter"]
+        rows = 2 * h + 2 * kv + 2 * it
+        return (f"{c['name']}: q/k/v/o/gate/up {rows}x{h} on one H + down {h}x{it}, "
+                f"T={c['T']} cone tokens, {bits}-bit g128 b128 damp0.01, per layer")
+    return f"{c['name']}: W {c['m']}x{c['n']}, T={c['T']}, {bits}-bit g128 b128 damp0.01"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of the GPU's clocks during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- roofline
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def fp64_peak_tflops(sm_mhz: float) -> float:
+    """B200 float64: 148 SMs × 64 FP64 FMA lanes × 2 flops × clock."""
+    return 148 * 64 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def kernel_work(probs, block: int):
+    """Algorithmic work per kernel kind for one step: {kind: (unit, amount)}.
+
+    hessian   flops T·n·(n+1)               (upper triangle incl. diagonal)
+    chol_*    flops of the executed float64 tile products (Σ_k tiles·2·64³)
+    sweep     bytes: strip read + Err write (4+4 B) + codes (1 B) per element,
+              U panel 4·bw², scale+zero 5 B per (row, group)
+    trailing  bytes: W read+write 8 B per trailing element, Err 4·m·bw,
+              U panel 4·bw·N2
+    pack      bytes: codes 1 B + packed bits/8 B per element, scale/zero
+    ingest    bytes: W in (2 or 4 B) + float32 out per element
+    """
+    w = {k: 0.0 for k in ("hessian", "chol_trail", "chol_panel", "sweep", "trailing",
+                          "pack", "ingest")}
+    for p in probs:
+        m, n, T = p.m, p.n, p.T
+        w["hessian"] += T * n * (n + 1)
+        N = -(-n // 64)
+        for k in range(N):
+            r = N - k - 1
+            w["chol_trail"] += (r * (r + 1) // 2 + r * (k + 1)) * 2 * 64 ** 3
+            w["chol_panel"] += (r + k) * 2 * 64 ** 3
+        ng = -(-n // p.group)
+        for j0 in range(0, n, block):
+            bw = min(block, n - j0)
+            n2 = n - j0 - bw
+            w["sweep"] += 9 * m * bw + 4 * bw * bw + 5 * m * (-(-bw // p.group))
+            if n2 > 0:
+                w["trailing"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
+        w["pack"] += m * n + m * n * p.bits / 8 + 5 * m * ng
+        w["ingest"] += m * n * (p.W.element_size() + 4)
+    units = {"hessian": "TFLOP/s", "chol_trail": "TFLOP/s", "chol_panel": "TFLOP/s",
+             "sweep": "GB/s", "trailing": "GB/s", "pack": "GB/s", "ingest": "GB/s"}
+    return {k: (units[k], v) for k, v in w.items()}
+
+
+def traffic_for(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary, if still current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if not e or e.get("workload") != workload:
+            return None
+        import hashlib
+        src = os.path.join(ROOT, "post_weight_quantization_08_b200", "csrc", e["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return e["bytes_per_launch"] if h == e.get("source_sha") else None
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+class Layer:
+    """Device buffers of one layer's problems, allocated once."""
+
+    def __init__(self, probs, device):
+        import post_weight_quantization_08_b200 as g
+        self.g = g
+        self.probs = probs
+        self.dev = device
+        self.items = []
+        for p in probs:
+            m, n = p.m, p.n
+            ng = -(-n // p.group)
+            nw = -(-n * p.bits // 32)
+            it = {
+                "p": p,
+                "X": p.X.to(device).contiguous(),
+                "W": p.W.to(device).contiguous(),
+                "H": torch.zeros(n, n, dtype=torch.float32, device=device),
+                "perm": torch.empty(n, dtype=torch.int32, device=device),
+                "U": torch.empty(n, n, dtype=torch.float32, device=device),
+                "dead": torch.empty(n, dtype=torch.uint8, device=device),
+                "info_p": torch.zeros(2, dtype=torch.int32, device=device),
+                "info_q": torch.zeros(2, dtype=torch.int32, device=device),
+                "ws_p": g.workspace(g.gptq_prepare_workspace_bytes(n), device),
+                "ws_q": g.workspace(g.gptq_quantize_workspace_bytes(m, n, p.block), device),
+                "qweight": torch.empty(m, nw, dtype=torch.int32, device=device),
+                "scale": torch.empty(m, ng, dtype=torch.float32, device=device),
+                "zero": torch.empty(m, ng, dtype=torch.uint8, device=device),
+                "g_idx": torch.empty(n, dtype=torch.int32, device=device),
+                "loss": torch.empty(m, dtype=torch.float32, device=device),
+                "stream": torch.cuda.Stream(device=device),
+            }
+            self.items.append(it)
+
+    def run_problem(self, it):
+        g, p, s = self.g, it["p"], it["stream"]
+        with torch.cuda.stream(s):
+            it["H"].zero_()
+        g.gptq_hessian_accumulate(it["X"], it["H"], s)
+        g.gptq_prepare(it["H"], p.damp, p.order, it["perm"], it["U"], it["dead"],
+                       it["info_p"], it["ws_p"], s)
+        g.gptq_quantize(it["W"], it["U"], it["perm"], it["dead"], p.bits, p.group, p.block,
+                        it["qweight"], it["scale"], it["zero"], it["g_idx"], it["loss"],
+                        None, it["info_q"], it["ws_q"], s)
+
+    def step(self, main):
+        """Fork the layer's problems onto their own streams, join on `main`."""
+        fork = torch.cuda.Event()
+        fork.record(main)
+        joins = []
+        for it in self.items:
+            it["stream"].wait_event(fork)
+            self.run_problem(it)
+            e = torch.cuda.Event()
+            e.record(it["stream"])
+            joins.append(e)
+        for e in joins:
+            main.wait_event(e)
+
+    def check(self):
+        for it in self.items:
+            for key in ("info_p", "info_q"):
+                st, idx = self.g.gptq_check(it[key], it["stream"])
+                if st != 0:
+                    raise RuntimeError(f"device reported status {st} at {idx}")
+
+
+def run_ours(args, rank, world, local):
+    import post_weight_quantization_08_b200 as g
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = CONFIGS[args.config]
+    bits = args.bits or cfg["bits"][0]
+    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits)
+    layer = Layer(probs, device)
+    params = sum(p.params for p in probs)
+    main = torch.cuda.current_stream(device)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    for _ in range(args.warmup):
+        layer.step(main)
+    torch.cuda.synchronize(device)
+    layer.check()
+
+    # ---- device-resident timed region
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = g.gptq_launch_count()
+    g.gptq_profile_start(1 << 16)
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)                       # evict L2 between steps
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        layer.step(main)
+        b.record(main)
+        evs.append((a, b))
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    kprof = g.gptq_profile_stop()
+    launches = g.gptq_launch_count() - launches0
+    clk = clocks.stop()
+    layer.check()
+    dev_ms = sum(a.elapsed_time(b) for a, b in evs)
+    dev_ms = max_over_ranks(dev_ms, world, device)
+    total_params = sum_over_ranks(params * args.steps, world, device)
+    value = total_params / (dev_ms / 1e3)
+
+    # ---- end to end: pinned host inputs in, packed results out, every step
+    host_in = [(it, it["X"].cpu().pin_memory(), it["W"].cpu().pin_memory()) for it in layer.items]
+    host_out = [{k: torch.empty(it[k].shape, dtype=it[k].dtype).pin_memory()
+                 for k in ("qweight", "scale", "zero", "g_idx", "loss")} for it in layer.items]
+    h2d = sum(x.numel() * x.element_size() + w.numel() * w.element_size() for _, x, w in host_in)
+    d2h = sum(t.numel() * t.element_size() for o in host_out for t in o.values())
+
+    def e2e_step():
+        for (it, x, w) in host_in:
+            it["X"].copy_(x, non_blocking=True)
+            it["W"].copy_(w, non_blocking=True)
+        layer.step(main)
+        for it, o in zip(layer.items, host_out):
+            for k, t in o.items():
+                t.copy_(it[k], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    e2e_ms = 0.0
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        e2e_step()
+        b.record(main)
+        torch.cuda.synchronize(device)
+        e2e_ms += a.elapsed_time(b)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    layer.check()
+
+    # ---- roofline of the dominant kernel
+    work = kernel_work(probs, probs[0].block)
+    tot = {k: v[0] for k, v in kprof.items()}
+    dom = max(tot, key=lambda k: tot[k])
+    peaks, src = _peaks()
+    sm_mhz = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    roof = None
+    if dom in work and kprof[dom][1] > 0:
+        unit, amount = work[dom]
+        per_step_ms = tot[dom] / args.steps
+        if unit == "TFLOP/s":
+            achieved = amount / (per_step_ms / 1e3) / 1e12
+            if dom == "hessian":
+                bound, peak, note = "tensor", peaks["bf16_tflops"], f"bf16 {src}"
+            else:
+                bound, peak = "alu", fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+                note = "fp64 148 SMs x 64 FMA x 2 x max clock"
+        else:
+            achieved = amount / (per_step_ms / 1e3) / 1e9
+            bound, peak, note = "hbm", peaks["hbm_gbs"], f"copy bandwidth, {src}"
+        launches_per_step = kprof[dom][1] / args.steps
+        roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2),
+                "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+                "peak_source": note,
+                "traffic": traffic_for(dom, workload_name(args.config, bits)),
+                "launches_per_step": launches_per_step,
+                "share": round(tot[dom] / max(1e-9, sum(tot.values())), 4)}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "params/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep",
+        "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
+        "config": {"workload": workload_name(args.config, bits), "params_per_step_per_gpu": params,
+                   "global_batch": len(probs) * world, "seq_len": probs[0].T,
+                   "parallelism": f"independent layers x{world}",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "e2e": {"value": round(total_params / (e2e_ms / 1e3), 1), "unit": "params/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "roofline": roof,
+        "kernels_ms_per_step": {k: round(v / args.steps, 4) for k, v in tot.items() if v > 0},
+        "clocks": clk,
+    }
+    return out, probs, params
+
+
+# ---------------------------------------------------------------- CPU oracle arm
+
+def oracle_pass(probs):
+    """One pass of the float64 oracle over the problems (test infrastructure)."""
+    import numpy as np
+    from oracle import gptq as og
+    for p in probs:
+        X = p.X.to(torch.float64).numpy()
+        W = p.W.to(torch.float64).numpy()
+        H = og.hessian(X)
+        og.gptq_layer(W, H, p.bits, p.group, p.block, p.damp, p.order)
+    return sum(p.params for p in probs)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(probs, budget_s: float = 12.0):
+    done, t0 = 0, time.perf_counter()
+    passes = 0
+    while True:
+        done += oracle_pass(probs)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or passes >= 50:
+            break
+    return {"value": round(done / el, 1), "unit": "params/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{passes} full passes of the layer's problems ({el:.1f} s, float64 numpy)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = CONFIGS[args.config]
+    bits = args.bits or cfg["bits"][0]
+    probs = problems_for(args.config, layer=0, bits=bits)
+    for _ in range(args.warmup):
+        oracle_pass(probs)
+    t0 = time.perf_counter()
+    params = 0
+    for _ in range(args.steps):
+        params += oracle_pass(probs)
+    el = time.perf_counter() - t0
+    value = params / el
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "params/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
+        "config": {"workload": workload_name(args.config, bits)},
+        "cpu_baseline": {"value": round(value, 1), "unit": "params/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{args.steps} timed passes of one layer on the host cores"},
+        "e2e": {"value": round(value, 1), "unit": "params/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--bits", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        out, probs, _ = run_ours(args, rank, world, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(probs)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

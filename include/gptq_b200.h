@@ -1,0 +1,196 @@
+/*
+ * gptq_b200.h — C ABI of the B200 (sm_100a) GPTQ library.
+ *
+ * GPTQ quantizes a linear layer's weights column by column and pushes each
+ * column's rounding error onto the columns not yet quantized, weighted by the
+ * inverse Hessian of the layer inputs:
+ *   "Warum Geometrie Gewichte nicht komprimiert" (nonndazone.ru), section
+ *   "Methodik. Was ist CHMC", Schritt 2 — H = XᵀX/n + λ·mean(diag H)·I, the
+ *   inverse through the Cholesky factorisation, act-order, and per column j:
+ *   err_j = (col_j − q_j)/H⁻¹[j,j],  R[:, j+1:] −= err_j·H⁻¹[j, j+1:].
+ *   "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+ *   Algorithm" (gist.science summary), §2.1–§2.3 — the same loop is Babai's
+ *   nearest-plane algorithm on the lattice that the Hessian defines.
+ *
+ * Three calls follow that statement of the problem:
+ *   gptq_hessian_accumulate(X)                 H += 2·XᵀX
+ *   gptq_prepare(H, damp)                      U = upper Cholesky factor of
+ *                                              (P·(H + damp·mean(diag H)·I)·Pᵀ)⁻¹
+ *   gptq_quantize(W, U, bits, group, block)    packed codes + scale + zero
+ *
+ * Conventions shared by every call
+ *   - Every array pointer is a DEVICE pointer unless stated otherwise; the
+ *     caller owns all memory (outputs and workspaces).  The library never
+ *     allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it.
+ *   - Arrays are dense and row-major (C order).
+ *   - Host-detectable argument errors return before anything is enqueued.
+ *     Errors found on the device (non-positive pivot, NaN/Inf input) are
+ *     written to the caller's `info` array (two int32 on the device:
+ *     info[0] = gptq_status, info[1] = index) and reported by gptq_check().
+ *   - A CUDA launch error returns GPTQ_ERR_CUDA; gptq_last_error() gives the
+ *     message of the last failure on the calling thread.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, workspace too small   */
+  GPTQ_ERR_NOT_PD = 2,       /* damped, permuted H not positive definite     */
+  GPTQ_ERR_NONFINITE = 3,    /* NaN or Inf in H or W                         */
+  GPTQ_ERR_UNSUPPORTED = 4,  /* bits/group/block combination not implemented */
+  GPTQ_ERR_TIMEOUT = 5,      /* a bounded device wait ran out                */
+  GPTQ_ERR_CUDA = 6          /* a CUDA runtime call failed                   */
+} gptq_status;
+
+typedef enum {
+  GPTQ_ORDER_NATURAL = 0,  /* columns 0..n−1                                  */
+  GPTQ_ORDER_ACT = 1,      /* descending diag(H); equal entries keep index order
+                              ("act-order": Schritt 2 of the CHMC page; the
+                              Babai page, §2.3, defines it by the diagonal)   */
+  GPTQ_ORDER_REVERSE = 2,  /* columns n−1..0: back to front, the order in which
+                              GPTQ is Babai's algorithm (Babai page, §2.2)    */
+  GPTQ_ORDER_CUSTOM = 3    /* caller's permutation, read from `perm`          */
+} gptq_order;
+
+typedef enum {
+  GPTQ_DTYPE_F32 = 0,
+  GPTQ_DTYPE_BF16 = 1
+} gptq_dtype;
+
+/*
+ * H += 2·XᵀX.
+ *   X  T×n bfloat16, row-major (one row per calibration token), device.
+ *   H  n×n float32, row-major, device; read and written (accumulates, so a
+ *      calibration set may arrive in several calls).  The caller zeroes H
+ *      before the first call.  Both triangles are written (H stays symmetric).
+ *   T  may be 0 (no-op).  n ≥ 1.
+ * Source: CHMC page, Schritt 2 ("Hesse-Matrix aus den
+ * Kalibrierungsaktivierungen", XᵀX/n); the factor 2 instead of 1/n leaves the
+ * codes unchanged because the damping is relative.  Babai page, §2.1: XᵀX is
+ * the Gram matrix of the lattice basis.
+ * Errors: INVALID_ARG (null pointer, T < 0, n < 1), CUDA.
+ */
+gptq_status gptq_hessian_accumulate(const void* X, int64_t T, int64_t n,
+                                    float* H, void* stream);
+
+/* Bytes of device workspace gptq_prepare needs for size n (256-byte aligned). */
+size_t gptq_prepare_workspace_bytes(int64_t n);
+
+/*
+ * Damp, order and factor.
+ *   H      n×n float32 from gptq_hessian_accumulate, device, read only.
+ *   damp   relative damping λ ≥ 0 (float64): H_d = H + λ·mean(diag H)·I.  The mean is
+ *          taken before the dead-column fix.  Dead columns (H_jj == 0) get
+ *          H_jj := 1 (and gptq_quantize zeroes their weights).
+ *   order  a gptq_order value.
+ *   perm   int32[n], device.  Output (processing position p → original column
+ *          perm[p]) unless order == CUSTOM, where it is the input.
+ *   U      n×n float32, device, output: upper triangular, UᵀU = (P·H_d·Pᵀ)⁻¹
+ *          with P the processing-order permutation; the strict lower triangle
+ *          is written as 0.  Computed in float64 and rounded once.
+ *   dead   uint8[n], device, output: 1 where H_jj == 0.
+ *   info   int32[2], device, output: {status, index}; NOT_PD sets index to
+ *          the failing pivot (processing position) + 1; NONFINITE to the
+ *          flattened index + 1 of a NaN/Inf entry of H.
+ *   ws     device workspace of at least gptq_prepare_workspace_bytes(n),
+ *          256-byte aligned.
+ * Source: CHMC page, Schritt 2 (damping, act-order, "H⁻¹ über die
+ * Cholesky-Zerlegung"); Babai page, §2.3 (ordering by the Hessian diagonal).
+ * Errors: INVALID_ARG (null pointer, n < 1, damp < 0 or not finite, bad
+ * order, workspace too small; a CUSTOM perm that is not a permutation is
+ * reported through info), CUDA; NOT_PD / NONFINITE through info.
+ */
+gptq_status gptq_prepare(const float* H, int64_t n, double damp, int order,
+                         int32_t* perm, float* U, uint8_t* dead, int32_t* info,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace gptq_quantize needs (256-byte aligned). */
+size_t gptq_quantize_workspace_bytes(int64_t m, int64_t n, int block);
+
+/*
+ * Quantize W (m×n) column by column with error compensation.
+ *   W        m×n, device, bfloat16 or float32 (w_dtype), row-major; not
+ *            modified.  Rows are output channels, columns input channels.
+ *   U, perm, dead   from gptq_prepare for this W's Hessian.
+ *   bits     2, 3, 4 or 8.  Asymmetric min-max grid with an integer zero
+ *            point; the range contains 0; all-zero group → [−1, 1].
+ *   group    columns per scale group, along the input channels, counted in
+ *            processing order (CHMC page, Schritt 3: GPTQ keeps o·⌈i/gs⌉
+ *            scales).  A multiple of 32.
+ *   block    lazy-batch width: a multiple of group, at most 128.  The block
+ *            changes rounding order only, not the algorithm.
+ *   qweight  m × ceil(n·bits/32) uint32, output: per row an LSB-first bit
+ *            stream of the codes in ORIGINAL column order (column c in bits
+ *            [c·bits, (c+1)·bits) of the row's stream).
+ *   scale    m × ceil(n/group) float32, output; zero: same shape, uint8.
+ *            Group g covers processing positions [g·group, (g+1)·group).
+ *   g_idx    int32[n], output: group of each original column.
+ *   loss_row float32[m] or NULL: Σ_j e_j² with e_j = (w_j − q̂_j)/U_jj, the
+ *            damped layer loss of the row.
+ *   Qdq      m×n float32 or NULL: dequantized weights s·(q − z), original
+ *            column order.
+ *   info     int32[2], device, output (NONFINITE: flattened index + 1 of the
+ *            first NaN/Inf weight found).
+ *   ws       device workspace of at least gptq_quantize_workspace_bytes().
+ * Per column j (processing order):  q = clamp(rint(w/s) + z, 0, 2^bits − 1),
+ *   e = (w − s·(q − z))/U_jj,  w[j+1:] −= e·U[j, j+1:]   (CHMC page, Schritt 2;
+ *   scale and zero from the group's current values at its first column.)
+ * Errors: INVALID_ARG, UNSUPPORTED (bits, group, block), CUDA; NONFINITE
+ * through info.
+ */
+gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
+                          const float* U, const int32_t* perm,
+                          const uint8_t* dead, int bits, int group, int block,
+                          uint32_t* qweight, float* scale, uint8_t* zero,
+                          int32_t* g_idx, float* loss_row, float* Qdq,
+                          int32_t* info, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Synchronize `stream`, read info[0..1] and return info[0] (a gptq_status).
+ * If `index` is not NULL it receives info[1].  `info` is a device pointer.
+ */
+gptq_status gptq_check(const int32_t* info, int32_t* index, void* stream);
+
+/* Message of the last failure on the calling thread ("" if none). */
+const char* gptq_last_error(void);
+
+/* Name of a status code. */
+const char* gptq_status_string(int status);
+
+/* ---- instrumentation (host-side; no device memory) ---------------------- */
+
+/* Number of kernels this library has launched in this process. */
+uint64_t gptq_launch_count(void);
+
+/* Number of kernel kinds, and the name of kind k (e.g. "hessian_tc"). */
+int gptq_kernel_kinds(void);
+const char* gptq_kernel_name(int kind);
+
+/*
+ * Kernel timing: after gptq_profile_start(capacity) every launch (up to
+ * `capacity`) is bracketed by a pair of CUDA events recorded on the stream it
+ * is launched on.  gptq_profile_stop() waits for those events and sums the
+ * elapsed times per kernel kind; gptq_profile_get() returns the sum (ms) and
+ * the number of timed launches of kind k.  Events are host objects; no device
+ * memory is allocated.
+ */
+gptq_status gptq_profile_start(int capacity);
+gptq_status gptq_profile_stop(void);
+gptq_status gptq_profile_get(int kind, double* total_ms, int64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

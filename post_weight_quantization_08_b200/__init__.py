@@ -1,0 +1,91 @@
+"""B200-native GPTQ: Hessian → inverse-Cholesky → column sweep → packed codes.
+
+The C ABI (include/gptq_b200.h) is exposed under the same names by
+:mod:`._binding`.  The helpers below only allocate the output tensors with
+torch (device memory is the caller's) and call those functions; every step of
+the path runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from ._binding import (DTYPES, ORDERS, GptqError, exported_symbols,
+                       gptq_check, gptq_hessian_accumulate, gptq_launch_count,
+                       gptq_prepare, gptq_prepare_workspace_bytes,
+                       gptq_profile_start, gptq_profile_stop, gptq_quantize,
+                       gptq_quantize_workspace_bytes, kernel_names, lib)
+
+__all__ = [
+    "GptqError", "ORDERS", "DTYPES", "lib", "exported_symbols", "kernel_names",
+    "gptq_hessian_accumulate", "gptq_prepare", "gptq_quantize", "gptq_check",
+    "gptq_prepare_workspace_bytes", "gptq_quantize_workspace_bytes",
+    "gptq_launch_count", "gptq_profile_start", "gptq_profile_stop",
+    "hessian", "prepare", "quantize", "workspace",
+]
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A device byte buffer for the library's workspace (256-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _raise_info(info, stream, what):
+    st, idx = gptq_check(info, stream)
+    if st != 0:
+        raise GptqError(st, f"{what}: device reported index {idx}")
+
+
+def hessian(X: torch.Tensor, H: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H += 2·XᵀX; allocates a zero H when none is given."""
+    if H is None:
+        n = X.shape[1]
+        H = torch.zeros(n, n, dtype=torch.float32, device=X.device)
+    gptq_hessian_accumulate(X, H, stream)
+    return H
+
+
+def prepare(H: torch.Tensor, damp: float = 0.01, order: str = "natural",
+            perm: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+            stream=None, check: bool = True) -> dict:
+    """Returns {"U", "perm", "dead", "info"} on H's device."""
+    n = H.shape[0]
+    dev = H.device
+    if perm is None:
+        perm = torch.empty(n, dtype=torch.int32, device=dev)
+    U = torch.empty(n, n, dtype=torch.float32, device=dev)
+    dead = torch.empty(n, dtype=torch.uint8, device=dev)
+    info = torch.zeros(2, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(gptq_prepare_workspace_bytes(n), dev)
+    gptq_prepare(H, damp, order, perm, U, dead, info, ws, stream)
+    if check:
+        _raise_info(info, stream, "gptq_prepare")
+    return {"U": U, "perm": perm, "dead": dead, "info": info}
+
+
+def quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
+             block: int = 128, want_loss: bool = True, want_qdq: bool = False,
+             ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+    """Returns qweight (int32 bit patterns of the uint32 words), scale, zero,
+    g_idx and optionally loss_row / Qdq."""
+    m, n = W.shape
+    dev = W.device
+    ng = -(-n // group)
+    nwords = -(-n * bits // 32)
+    out = {
+        "qweight": torch.empty(m, nwords, dtype=torch.int32, device=dev),
+        "scale": torch.empty(m, ng, dtype=torch.float32, device=dev),
+        "zero": torch.empty(m, ng, dtype=torch.uint8, device=dev),
+        "g_idx": torch.empty(n, dtype=torch.int32, device=dev),
+        "loss_row": torch.empty(m, dtype=torch.float32, device=dev) if want_loss else None,
+        "Qdq": torch.empty(m, n, dtype=torch.float32, device=dev) if want_qdq else None,
+        "info": torch.zeros(2, dtype=torch.int32, device=dev),
+    }
+    if ws is None:
+        ws = workspace(gptq_quantize_workspace_bytes(m, n, block), dev)
+    gptq_quantize(W, prep["U"], prep["perm"], prep["dead"], bits, group, block,
+                  out["qweight"], out["scale"], out["zero"], out["g_idx"],
+                  out["loss_row"], out["Qdq"], out["info"], ws, stream)
+    if check:
+        _raise_info(out["info"], stream, "gptq_quantize")
+    return out

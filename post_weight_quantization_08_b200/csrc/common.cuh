@@ -1,0 +1,64 @@
+// Shared plumbing of the GPTQ kernels: kernel kinds, launch bookkeeping,
+// error reporting through the caller's device `info` words.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstddef>
+
+#include "../../include/gptq_b200.h"
+
+namespace gptq {
+
+// Kernel kinds, for the launch counter and the event profiler.
+enum KernelKind : int {
+  KK_HESSIAN = 0,     // H += 2·XᵀX
+  KK_PREP_STATS,      // mean(diag H), dead columns, order keys
+  KK_PREP_ORDER,      // processing permutation
+  KK_PREP_GATHER,     // reversed, permuted, damped float64 copy of H
+  KK_CHOL_DIAG,       // diagonal block: Cholesky + triangular inverse
+  KK_CHOL_PANEL,      // panel solve and finished rows of L⁻¹
+  KK_CHOL_TRAIL,      // trailing update of A and of the L⁻¹ accumulator
+  KK_PREP_OUT,        // U = reversed L⁻¹, rounded to float32
+  KK_INGEST,          // W → float32 working copy in processing order
+  KK_SWEEP,           // one block of the column sweep
+  KK_TRAIL,           // lazy-batch trailing update W −= Err·U
+  KK_PACK,            // codes → packed words, g_idx, dequantized copy
+  KK_COUNT
+};
+
+const char* kernel_kind_name(int k);
+
+// Launch bookkeeping (counter always; CUDA events when profiling is on).
+void launch_begin(int kind, cudaStream_t s);
+void launch_end(int kind, cudaStream_t s);
+
+// Record a failure message for gptq_last_error() and return `st`.
+gptq_status fail(gptq_status st, const char* fmt, ...);
+gptq_status cuda_fail(cudaError_t e, const char* what);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Device-side error report: first error wins (status word goes 0 → st).
+__device__ __forceinline__ void report(int32_t* info, int32_t st, int64_t index) {
+  if (info == nullptr) return;
+  if (atomicCAS(info, 0, st) == 0) info[1] = (int32_t)(index + 1);
+}
+
+}  // namespace gptq
+
+#define GPTQ_LAUNCH(kind, stream, kernel, grid, block, smem, ...)              \
+  do {                                                                         \
+    gptq::launch_begin((kind), (stream));                                      \
+    kernel<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+    gptq::launch_end((kind), (stream));                                        \
+    cudaError_t e__ = cudaGetLastError();                                      \
+    if (e__ != cudaSuccess) return gptq::cuda_fail(e__, #kernel);              \
+  } while (0)
+
+#define GPTQ_CUDA(call)                                                        \
+  do {                                                                         \
+    cudaError_t e__ = (call);                                                  \
+    if (e__ != cudaSuccess) return gptq::cuda_fail(e__, #call);                \
+  } while (0)

@@ -1,0 +1,206 @@
+// gptq_quantize: ingest (W → float32, processing order), the block loop of
+// sweep (K3) and trailing update (K4), and K5: packing the codes back into the
+// original column order, g_idx and the optional dequantized copy.
+//
+// "Warum Geometrie Gewichte nicht komprimiert", Methodik, Schritt 2 (the
+// column loop) and Table 1 (GPTQ stores integer indices plus group scales);
+// Schritt 3 (GPTQ's groups run along the input channels).
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+
+namespace gptq {
+namespace {
+
+struct QuantWs {
+  float* Wp;        // m × n working copy, processing order
+  uint8_t* codes;   // m × n codes, processing order
+  float* Err;       // m × block scaled errors of the current block
+  int32_t* pinv;    // n: processing position of each original column
+};
+
+size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  size_t o_wp = take(sizeof(float) * (size_t)m * (size_t)n);
+  size_t o_codes = take((size_t)m * (size_t)n);
+  size_t o_err = take(sizeof(float) * (size_t)m * (size_t)block);
+  size_t o_pinv = take(sizeof(int32_t) * (size_t)n);
+  if (w && base) {
+    w->Wp = reinterpret_cast<float*>(base + o_wp);
+    w->codes = reinterpret_cast<uint8_t*>(base + o_codes);
+    w->Err = reinterpret_cast<float*>(base + o_err);
+    w->pinv = reinterpret_cast<int32_t*>(base + o_pinv);
+  }
+  return off;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// pinv[perm[p]] = p and g_idx[perm[p]] = p / group.
+__global__ void __launch_bounds__(256)
+pinv_kernel(const int32_t* __restrict__ perm, int64_t n, int group,
+            int32_t* __restrict__ pinv, int32_t* __restrict__ g_idx, int32_t* info) {
+  const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (p >= n) return;
+  const int32_t c = perm[p];
+  if (c < 0 || c >= n) { report(info, GPTQ_ERR_INVALID_ARG, p); return; }
+  pinv[c] = (int32_t)p;
+  g_idx[c] = (int32_t)(p / group);
+}
+
+// Wp[r][p] = W[r][perm[p]] as float32; dead columns read as 0.
+template <typename T>
+__global__ void __launch_bounds__(256)
+ingest_kernel(const T* __restrict__ W, int64_t m, int64_t n,
+              const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
+              float* __restrict__ Wp, int32_t* info) {
+  const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (e >= m * n) return;
+  const int64_t r = e / n, p = e % n;
+  const int32_t c = perm[p];
+  float v = 0.f;
+  if (c >= 0 && c < n) {
+    v = to_f32(W[r * n + c]);
+    if (!isfinite(v)) { report(info, GPTQ_ERR_NONFINITE, r * n + c); v = 0.f; }
+    if (dead[c]) v = 0.f;
+  }
+  Wp[e] = v;
+}
+
+// One thread packs 32 consecutive original columns of one row into BITS words.
+template <int BITS>
+__global__ void __launch_bounds__(256)
+pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
+            const int32_t* __restrict__ pinv, int group, int64_t ngroups,
+            const float* __restrict__ scale, const uint8_t* __restrict__ zero,
+            uint32_t* __restrict__ qweight, int64_t nwords,
+            float* __restrict__ Qdq, int32_t* info) {
+  const int64_t chunks = (n + 31) / 32;
+  const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (e >= m * chunks) return;
+  const int64_t r = e / chunks, ch = e % chunks;
+  uint32_t w[BITS];
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) w[i] = 0u;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int64_t c = ch * 32 + k;
+    if (c < n) {
+      const int32_t p = pinv[c];
+      uint32_t q = 0;
+      if (p < 0 || p >= n) {
+        report(info, GPTQ_ERR_INVALID_ARG, c);
+      } else {
+        q = codes[r * n + p];
+        if (Qdq != nullptr) {
+          const int64_t g = p / group;
+          Qdq[r * n + c] = scale[r * ngroups + g] * ((float)q - (float)zero[r * ngroups + g]);
+        }
+      }
+      const int off = k * BITS, wi = off >> 5, sh = off & 31;
+      w[wi] |= q << sh;
+      if (sh + BITS > 32) w[wi + 1] |= q >> (32 - sh);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) {
+    const int64_t word = ch * BITS + i;
+    if (word < nwords) qweight[r * nwords + word] = w[i];
+  }
+}
+
+}  // namespace
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" size_t gptq_quantize_workspace_bytes(int64_t m, int64_t n, int block) {
+  if (m < 1 || n < 1 || block < 1) return 0;
+  return quant_ws_layout(m, n, block, nullptr, nullptr);
+}
+
+extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
+                                     int64_t n, const float* U,
+                                     const int32_t* perm, const uint8_t* dead,
+                                     int bits, int group, int block,
+                                     uint32_t* qweight, float* scale,
+                                     uint8_t* zero, int32_t* g_idx,
+                                     float* loss_row, float* Qdq, int32_t* info,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !U || !perm || !dead || !qweight || !scale || !zero || !g_idx || !info || !ws)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: null pointer");
+  if (m < 1 || n < 1 || m > ((int64_t)1 << 31) || n > ((int64_t)1 << 20))
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: m=%lld n=%lld", (long long)m,
+                (long long)n);
+  if (w_dtype != GPTQ_DTYPE_F32 && w_dtype != GPTQ_DTYPE_BF16)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: w_dtype=%d", w_dtype);
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+    return fail(GPTQ_ERR_UNSUPPORTED, "gptq_quantize: bits=%d (2, 3, 4, 8)", bits);
+  if (group < 32 || group % 32 != 0 || block < group || block > 128 || block % group != 0)
+    return fail(GPTQ_ERR_UNSUPPORTED,
+                "gptq_quantize: group=%d block=%d (group a multiple of 32, block a "
+                "multiple of group, block <= 128)", group, block);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: workspace not 256-byte aligned");
+  const size_t need = quant_ws_layout(m, n, block, nullptr, nullptr);
+  if (ws_bytes < need)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: workspace %zu < %zu bytes",
+                ws_bytes, need);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  QuantWs w;
+  quant_ws_layout(m, n, block, &w, static_cast<char*>(ws));
+  const int64_t ngroups = ceil_div(n, group);
+  const int64_t nwords = ceil_div(n * bits, 32);
+
+  GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
+  GPTQ_CUDA(cudaMemsetAsync(w.pinv, 0xFF, sizeof(int32_t) * n, s));
+  if (loss_row) GPTQ_CUDA(cudaMemsetAsync(loss_row, 0, sizeof(float) * m, s));
+  GPTQ_LAUNCH(KK_INGEST, s, pinv_kernel, (unsigned)ceil_div(n, 256), 256, 0, perm, n,
+              group, w.pinv, g_idx, info);
+  const unsigned gin = (unsigned)ceil_div(m * n, 256);
+  if (w_dtype == GPTQ_DTYPE_BF16)
+    GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<__nv_bfloat16>, gin, 256, 0,
+                static_cast<const __nv_bfloat16*>(W), m, n, perm, dead, w.Wp, info);
+  else
+    GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<float>, gin, 256, 0,
+                static_cast<const float*>(W), m, n, perm, dead, w.Wp, info);
+
+  for (int64_t j0 = 0; j0 < n; j0 += block) {
+    const int bw = (int)((n - j0 < block) ? (n - j0) : block);
+    gptq_status st = launch_sweep(w.Wp, m, n, j0, bw, U, bits, group, ngroups,
+                                  w.codes, scale, zero, w.Err, block, loss_row, s);
+    if (st != GPTQ_OK) return st;
+    if (j0 + bw < n) {
+      st = launch_trailing(w.Wp, m, n, j0 + bw, w.Err, block, j0, bw, U, s);
+      if (st != GPTQ_OK) return st;
+    }
+  }
+
+  const unsigned gpk = (unsigned)ceil_div(m * ceil_div(n, 32), 256);
+  switch (bits) {
+    case 2:
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
+                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+      break;
+    case 3:
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
+                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+      break;
+    case 4:
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
+                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+      break;
+    default:
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
+                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+      break;
+  }
+  return GPTQ_OK;
+}

@@ -1,0 +1,177 @@
+"""GPU parity: every stage of the CUDA path against the float64 oracle.
+
+Sizes span several tiles and a ragged tail (n = 576 is 4½ groups of 128;
+m = 300 is not a multiple of the 64-row CTA) and stay small enough for the
+oracle to finish in seconds.  Edge cases: n = 1 / 8 / 64, m = 1 / 7, every bit
+width, groups of 32/64/128, all four orders, dead columns, and the error paths.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gptq as og
+from oracle import lattice as ol
+from workloads import cone_activations, gaussian_weights, problems_for
+
+from . import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _layer(T, n, m, seed, wdtype=torch.bfloat16):
+    X = cone_activations(T, n, seed).to(torch.bfloat16)
+    W = gaussian_weights(m, n, seed + 1).to(wdtype)
+    return X, W
+
+
+def _full_check(X, W, bits, group, block, order="natural", damp=0.01, perm=None):
+    out = P.run_gpu(X, W, bits, group, block, damp, order, perm, DEV)
+    stats = P.check_hessian(X, out["H"])
+    _, s2 = P.check_prepare(out["H"], out, damp, order, perm)
+    stats.update(s2)
+    stats.update(P.check_quantize(W, out, None, bits, group, block))
+    stats.update(P.check_layer_loss(X, W, out, bits, group, block, damp, order, perm))
+    return out, stats
+
+
+def test_single_layer_576():
+    """The single-layer workload: 576×576 float32 W, 2048 cone tokens."""
+    p = problems_for(0)[0]
+    out, st = _full_check(p.X, p.W, 4, 128, 128)
+    assert st["code_diff"] <= 1e-3 * st["codes"]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_bits(bits):
+    X, W = _layer(1024, 576, 300, 100 + bits)
+    _full_check(X, W, bits, 128, 128)
+
+
+@pytest.mark.parametrize("group,block", [(32, 32), (32, 128), (64, 64), (64, 128), (128, 128)])
+def test_group_block(group, block):
+    X, W = _layer(512, 320, 130, 7)
+    _full_check(X, W, 4, group, block)
+
+
+@pytest.mark.parametrize("order", ["natural", "act", "reverse"])
+def test_orders(order):
+    X, W = _layer(768, 448, 96, 11)
+    _full_check(X, W, 4, 64, 128, order)
+
+
+def test_custom_order():
+    X, W = _layer(512, 200, 40, 12)
+    perm = np.random.default_rng(0).permutation(200)
+    _full_check(X, W, 3, 32, 64, "custom", perm=perm)
+
+
+@pytest.mark.parametrize("m,n", [(1, 1), (7, 8), (1, 64), (7, 130), (65, 33)])
+def test_small_and_ragged(m, n):
+    X, W = _layer(256, n, m, 13 + m + n)
+    _full_check(X, W, 4, 32, 64)
+
+
+def test_float32_weights():
+    X, W = _layer(512, 256, 70, 14, torch.float32)
+    _full_check(X, W, 4, 128, 128)
+
+
+def test_identity_hessian_is_rtn():
+    """H = I (prepare fed directly): codes, scales and zeros equal RTN bit for bit."""
+    import post_weight_quantization_08_b200 as g
+    n, m = 300, 50
+    W = gaussian_weights(m, n, 15)
+    H = torch.eye(n, dtype=torch.float32, device=DEV)
+    prep = g.prepare(H, 0.01, "natural")
+    q = g.quantize(W.to(DEV), prep, 4, 64, 128)
+    codes = P.unpack_rows(q["qweight"].cpu().numpy(), 4, n)
+    c, s, z, _ = ol.rtn(W.double().numpy(), 4, 64)
+    assert np.array_equal(codes, c)
+    assert np.array_equal(q["scale"].cpu().numpy(), s)
+    assert np.array_equal(q["zero"].cpu().numpy().astype(np.float32), z)
+
+
+def test_dead_columns():
+    X, W = _layer(300, 100, 20, 16)
+    X[:, [3, 50]] = 0
+    out, _ = _full_check(X, W, 4, 32, 64, "act")
+    assert out["dead"][3] and out["dead"][50] and out["dead"].sum() == 2
+
+
+def test_hessian_accumulates_across_calls():
+    import post_weight_quantization_08_b200 as g
+    X = cone_activations(1000, 200, 17).to(torch.bfloat16).to(DEV)
+    H1 = g.hessian(X)
+    H2 = g.hessian(X[:400].contiguous())
+    g.hessian(X[400:].contiguous(), H2)
+    torch.cuda.synchronize()
+    ref = og.hessian(X.cpu().double().numpy())
+    S = 2.0 * np.abs(X.cpu().double().numpy()).T @ np.abs(X.cpu().double().numpy())
+    for H in (H1, H2):
+        assert np.all(np.abs(H.cpu().double().numpy() - ref) <= 2 * 1000 * 2 ** -24 * S + 1e-30)
+    # T = 0 is a no-op
+    g.hessian(X[:0], H1)
+    torch.cuda.synchronize()
+
+
+def test_repeatable():
+    X, W = _layer(512, 256, 64, 18)
+    a = P.run_gpu(X, W, 4, 128, 128)
+    b = P.run_gpu(X, W, 4, 128, 128)
+    for k in ("H", "U", "qweight", "scale", "zero"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+# ---------------------------------------------------------------- error paths
+
+def test_not_positive_definite():
+    import post_weight_quantization_08_b200 as g
+    n = 70
+    H = torch.eye(n, device=DEV)
+    H[5, 5] = -4.0
+    with pytest.raises(g.GptqError) as e:
+        g.prepare(H, 0.0)
+    assert e.value.status == 2
+
+
+def test_nonfinite_inputs():
+    import post_weight_quantization_08_b200 as g
+    n = 40
+    H = torch.eye(n, device=DEV)
+    H[2, 7] = float("nan")
+    with pytest.raises(g.GptqError) as e:
+        g.prepare(H, 0.01)
+    assert e.value.status == 3
+    prep = g.prepare(torch.eye(n, device=DEV), 0.01)
+    W = torch.zeros(4, n, device=DEV)
+    W[1, 3] = float("inf")
+    with pytest.raises(g.GptqError) as e:
+        g.quantize(W, prep, 4, 32, 32)
+    assert e.value.status == 3
+
+
+def test_bad_custom_order():
+    import post_weight_quantization_08_b200 as g
+    n = 10
+    perm = torch.arange(n, dtype=torch.int32, device=DEV)
+    perm[3] = 4            # duplicate
+    with pytest.raises(g.GptqError) as e:
+        g.prepare(torch.eye(n, device=DEV), 0.01, "custom", perm=perm)
+    assert e.value.status == 1
+
+
+def test_host_side_argument_errors():
+    import post_weight_quantization_08_b200 as g
+    n = 64
+    prep = g.prepare(torch.eye(n, device=DEV), 0.01)
+    W = torch.randn(8, n, device=DEV)
+    for bits, group, block in ((5, 32, 32), (4, 48, 96), (4, 64, 32), (4, 64, 256)):
+        with pytest.raises(g.GptqError) as e:
+            g.quantize(W, prep, bits, group, block)
+        assert e.value.status == 4
+    small = torch.empty(256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(g.GptqError) as e:
+        g.quantize(W, prep, 4, 32, 32, ws=small)
+    assert e.value.status == 1
