@@ -163,8 +163,8 @@ def kernel_work(probs, block: int):
     pack      bytes: codes 1 B + packed bits/8 B per element, scale/zero
     ingest    bytes: W in (2 or 4 B) + float32 out per element
     """
-    w = {k: 0.0 for k in ("hessian", "chol_trail", "chol_panel", "sweep", "trailing",
-                          "pack", "ingest")}
+    w = {k: 0.0 for k in ("hessian", "chol_diag", "chol_trail", "chol_panel", "sweep",
+                          "trailing", "pack", "ingest")}
     for p in probs:
         m, n, T = p.m, p.n, p.T
         w["hessian"] += T * n * (n + 1)
@@ -173,6 +173,7 @@ def kernel_work(probs, block: int):
             r = N - k - 1
             w["chol_trail"] += (r * (r + 1) // 2 + r * (k + 1)) * 2 * 64 ** 3
             w["chol_panel"] += (r + k) * 2 * 64 ** 3
+            w["chol_diag"] += 2 * 64 ** 3 / 3        # Cholesky + inverse of a tile
         ng = -(-n // p.group)
         for j0 in range(0, n, block):
             bw = min(block, n - j0)
@@ -182,7 +183,8 @@ def kernel_work(probs, block: int):
                 w["trailing"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
         w["pack"] += m * n + m * n * p.bits / 8 + 5 * m * ng
         w["ingest"] += m * n * (p.W.element_size() + 4)
-    units = {"hessian": "TFLOP/s", "chol_trail": "TFLOP/s", "chol_panel": "TFLOP/s",
+    units = {"hessian": "TFLOP/s", "chol_diag": "TFLOP/s", "chol_trail": "TFLOP/s",
+             "chol_panel": "TFLOP/s",
              "sweep": "GB/s", "trailing": "GB/s", "pack": "GB/s", "ingest": "GB/s"}
     return {k: (units[k], v) for k, v in w.items()}
 
@@ -229,6 +231,7 @@ class Layer:
                 "perm": torch.empty(n, dtype=torch.int32, device=device),
                 "U": torch.empty(n, n, dtype=torch.float32, device=device),
                 "dead": torch.empty(n, dtype=torch.uint8, device=device),
+                "info_h": torch.zeros(2, dtype=torch.int32, device=device),
                 "info_p": torch.zeros(2, dtype=torch.int32, device=device),
                 "info_q": torch.zeros(2, dtype=torch.int32, device=device),
                 "ws_p": g.workspace(g.gptq_prepare_workspace_bytes(n), device),
@@ -246,7 +249,7 @@ class Layer:
         g, p, s = self.g, it["p"], it["stream"]
         with torch.cuda.stream(s):
             it["H"].zero_()
-        g.gptq_hessian_accumulate(it["X"], it["H"], s)
+        g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
         g.gptq_prepare(it["H"], p.damp, p.order, it["perm"], it["U"], it["dead"],
                        it["info_p"], it["ws_p"], s)
         g.gptq_quantize(it["W"], it["U"], it["perm"], it["dead"], p.bits, p.group, p.block,
@@ -267,9 +270,19 @@ class Layer:
         for e in joins:
             main.wait_event(e)
 
+    def step_serial(self, main):
+        """Every problem on `main`, one after the other (for kernel timing)."""
+        for it in self.items:
+            s = it["stream"]
+            it["stream"] = main
+            try:
+                self.run_problem(it)
+            finally:
+                it["stream"] = s
+
     def check(self):
         for it in self.items:
-            for key in ("info_p", "info_q"):
+            for key in ("info_h", "info_p", "info_q"):
                 st, idx = self.g.gptq_check(it[key], it["stream"])
                 if st != 0:
                     raise RuntimeError(f"device reported status {st} at {idx}")
@@ -284,13 +297,34 @@ def run_ours(args, rank, world, local):
     probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits)
     layer = Layer(probs, device)
     params = sum(p.params for p in probs)
-    main = torch.cuda.current_stream(device)
+    main = torch.cuda.Stream(device=device)     # non-default: graphs capture here
+    torch.cuda.set_stream(main)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
     for _ in range(args.warmup):
         layer.step(main)
     torch.cuda.synchronize(device)
     layer.check()
+
+    # ---- one step captured as a CUDA graph (both problems, forked streams)
+    graph = None
+    launches_per_step = 0
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        c0 = g.gptq_launch_count()
+        with torch.cuda.graph(graph, stream=main):
+            layer.step(main)
+        launches_per_step = g.gptq_launch_count() - c0
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize(device)
+        layer.check()
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            layer.step(main)
 
     # ---- device-resident timed region
     if world > 1:
@@ -299,27 +333,36 @@ def run_ours(args, rank, world, local):
     clocks = ClockSampler(local)
     clocks.start()
     launches0 = g.gptq_launch_count()
-    g.gptq_profile_start(1 << 16)
     evs = []
     for _ in range(args.steps):
         flush.fill_(1.0)                       # evict L2 between steps
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(main)
-        layer.step(main)
+        run_step()
         b.record(main)
         evs.append((a, b))
     torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
-    kprof = g.gptq_profile_stop()
-    launches = g.gptq_launch_count() - launches0
+    launches = (g.gptq_launch_count() - launches0) if graph is None else launches_per_step * args.steps
     clk = clocks.stop()
     layer.check()
     dev_ms = sum(a.elapsed_time(b) for a, b in evs)
     dev_ms = max_over_ranks(dev_ms, world, device)
     total_params = sum_over_ranks(params * args.steps, world, device)
     value = total_params / (dev_ms / 1e3)
+
+    # ---- per-kernel durations: the same K steps launched eagerly, every
+    # launch bracketed by CUDA events on its own stream
+    # (problems one after the other on one stream, so that no kernel's
+    # interval includes time spent waiting for the other problem's kernels)
+    g.gptq_profile_start(1 << 16)
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        layer.step_serial(main)
+    torch.cuda.synchronize(device)
+    kprof = g.gptq_profile_stop()
 
     # ---- end to end: pinned host inputs in, packed results out, every step
     host_in = [(it, it["X"].cpu().pin_memory(), it["W"].cpu().pin_memory()) for it in layer.items]
@@ -332,7 +375,7 @@ def run_ours(args, rank, world, local):
         for (it, x, w) in host_in:
             it["X"].copy_(x, non_blocking=True)
             it["W"].copy_(w, non_blocking=True)
-        layer.step(main)
+        run_step()
         for it, o in zip(layer.items, host_out):
             for k, t in o.items():
                 t.copy_(it[k], non_blocking=True)
@@ -391,7 +434,8 @@ def run_ours(args, rank, world, local):
         "config": {"workload": workload_name(args.config, bits), "params_per_step_per_gpu": params,
                    "global_batch": len(probs) * world, "seq_len": probs[0].T,
                    "parallelism": f"independent layers x{world}",
-                   "l2": "flushed between timed steps (256 MB write)"},
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "launch": "CUDA graph replay per step" if graph is not None else "eager launches"},
         "e2e": {"value": round(total_params / (e2e_ms / 1e3), 1), "unit": "params/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
@@ -480,6 +524,7 @@ def main(argv=None):
     ap.add_argument("--bits", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -74,14 +74,20 @@ typedef enum {
  *      calibration set may arrive in several calls).  The caller zeroes H
  *      before the first call.  Both triangles are written (H stays symmetric).
  *   T  may be 0 (no-op).  n ≥ 1.
+ *   info  int32[2] on the device, or NULL: a bounded wait inside the kernel
+ *      that runs out is reported there as GPTQ_ERR_TIMEOUT (it is not reset
+ *      by this call, so several calls may share one info pair).
+ * Kernel: for n a multiple of 8 (and X 16-byte aligned) a TMA → tcgen05
+ * pipeline (bf16 operands, float32 accumulator in tensor memory, 128×128
+ * tiles on or above the diagonal); otherwise a float32 SIMT tile kernel.
  * Source: CHMC page, Schritt 2 ("Hesse-Matrix aus den
  * Kalibrierungsaktivierungen", XᵀX/n); the factor 2 instead of 1/n leaves the
  * codes unchanged because the damping is relative.  Babai page, §2.1: XᵀX is
  * the Gram matrix of the lattice basis.
- * Errors: INVALID_ARG (null pointer, T < 0, n < 1), CUDA.
+ * Errors: INVALID_ARG (null pointer, T < 0, n < 1), CUDA; TIMEOUT via info.
  */
 gptq_status gptq_hessian_accumulate(const void* X, int64_t T, int64_t n,
-                                    float* H, void* stream);
+                                    float* H, int32_t* info, void* stream);
 
 /* Bytes of device workspace gptq_prepare needs for size n (256-byte aligned). */
 size_t gptq_prepare_workspace_bytes(int64_t n);

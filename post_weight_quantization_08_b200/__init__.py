@@ -35,12 +35,16 @@ def _raise_info(info, stream, what):
         raise GptqError(st, f"{what}: device reported index {idx}")
 
 
-def hessian(X: torch.Tensor, H: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+def hessian(X: torch.Tensor, H: torch.Tensor | None = None, stream=None,
+            check: bool = True) -> torch.Tensor:
     """H += 2·XᵀX; allocates a zero H when none is given."""
     if H is None:
         n = X.shape[1]
         H = torch.zeros(n, n, dtype=torch.float32, device=X.device)
-    gptq_hessian_accumulate(X, H, stream)
+    info = torch.zeros(2, dtype=torch.int32, device=X.device) if check else None
+    gptq_hessian_accumulate(X, H, info, stream)
+    if check:
+        _raise_info(info, stream, "gptq_hessian_accumulate")
     return H
 
 

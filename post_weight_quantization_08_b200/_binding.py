@@ -24,7 +24,8 @@ DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 # name: (restype, argtypes)
 _SIGS = {
-    "gptq_hessian_accumulate": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]),
+    "gptq_hessian_accumulate": (C.c_int, [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p,
+                                          C.c_void_p, C.c_void_p]),
     "gptq_prepare_workspace_bytes": (C.c_size_t, [C.c_int64]),
     "gptq_prepare": (C.c_int, [C.c_void_p, C.c_int64, C.c_double, C.c_int, C.c_void_p,
                                C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
@@ -110,12 +111,15 @@ def _need(t, name, dtype, shape=None, device=None):
 
 # ---------------------------------------------------------------- C calls
 
-def gptq_hessian_accumulate(X, H, stream=None):
+def gptq_hessian_accumulate(X, H, info=None, stream=None):
     """H += 2·XᵀX (X: T×n bf16, H: n×n float32; both on the same GPU)."""
     _need(X, "X", torch.bfloat16)
     T, n = X.shape
     _need(H, "H", torch.float32, (n, n), X.device)
-    _raise(lib().gptq_hessian_accumulate(_ptr(X), T, n, _ptr(H), _stream(stream, X.device)))
+    if info is not None:
+        _need(info, "info", torch.int32, (2,), X.device)
+    _raise(lib().gptq_hessian_accumulate(_ptr(X), T, n, _ptr(H), _ptr(info),
+                                         _stream(stream, X.device)))
 
 
 def gptq_prepare_workspace_bytes(n: int) -> int:

@@ -5,19 +5,41 @@
 
 namespace gptq {
 
+// Largest block width, and the bytes of one pre-transposed U panel
+// (UT[128][132] floats plus 128 reciprocal diagonals).
+constexpr int SWEEP_BLOCK_MAX = 128;
+constexpr size_t PANEL_BYTES = (size_t)(128 * 132 + 128) * sizeof(float);
+
+size_t panel_workspace_bytes(int64_t n, int block);
+
+// One panel per block of U, laid out for the sweep's bulk copy.
+gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
+                          cudaStream_t s);
+
 // Columns [j0, j0+bw) of the float32 working copy Wp (m×n, processing order):
 // quantize column by column with in-block error propagation.  Writes codes
-// (m×n u8, processing order), scale/zero (m×ngroups), the scaled errors
-// Err (m×bw, leading dimension ldE) and adds Σe² to loss_row (may be NULL).
-gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0,
-                         int bw, const float* U, int bits, int group,
-                         int64_t ngroups, uint8_t* codes, float* scale,
-                         uint8_t* zero, float* Err, int ldE, float* loss_row,
-                         cudaStream_t s);
+// (m×n u8, processing order), scale/zero (m×ngroups), the scaled errors as a
+// TF32 split Ehi + Elo (each m×128, Ehi = TF32(e), Elo = e − Ehi exactly) and
+// adds Σe² to loss_row (may be NULL).
+gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
+                         const float* panel, int bits, int group, int64_t ngroups,
+                         uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
+                         float* Elo, float* loss_row, int32_t* info, cudaStream_t s);
 
-// Wp[:, c0:n] −= Err[:, 0:kw]·U[k0:k0+kw, c0:n]   (lazy-batch update).
-gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0,
-                            const float* Err, int ldE, int64_t k0, int kw,
-                            const float* U, cudaStream_t s);
+// Whether the trailing update runs on the tensor cores for this shape.
+bool trailing_uses_tensor_cores(int64_t n, int block);
+
+// TF32 split of the n×n matrix x, transposed: hiT[c][r] = TF32(x[r][c]),
+// loT[c][r] = x[r][c] − hiT[c][r].
+gptq_status launch_split_tf32_t(const float* x, int64_t n, float* hiT, float* loT,
+                                cudaStream_t s);
+
+// Wp[:, c0:n] −= (Ehi+Elo)[:, 0:kw]·U[k0:k0+kw, c0:n]   (lazy-batch update).
+// With UhiT/UloT (the transposed TF32 split of U) the product runs on the
+// tensor cores.
+gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, const float* Ehi,
+                            const float* Elo, int64_t k0, int kw, const float* U,
+                            const float* Uhi, const float* Ulo, int32_t* info,
+                            cudaStream_t s);
 
 }  // namespace gptq

@@ -171,10 +171,33 @@ prep_gather_kernel(const float* __restrict__ H, int64_t n, int64_t np,
   A[e] = v;
 }
 
-// Diagonal tile: L_kk = chol(A_kk) and D = L_kk⁻¹, fused right-looking, one
-// barrier per column.  Column c's scaled entries are written one step late,
-// when nothing reads them any more.
-__global__ void __launch_bounds__(256)
+// Diagonal tile: L_kk = chol(A_kk) and D = L_kk⁻¹, blocked by panels of 8
+// columns so that the 64 dependent pivots cost 16 barriers instead of 64:
+//   phase 1 (warp 0): factor the 8-column panel in registers (lane l owns rows
+//            l and l + 32), pivots and multipliers exchanged by shuffles, and
+//            finish the panel's 8 rows of D by forward substitution (lanes
+//            over columns);
+//   phase 2 (8 warps): rank-8 update of the trailing block of A and of the
+//            rows of D below the panel.
+// Pivots use rsqrt_pivot (Newton steps from the float32 estimate).
+constexpr int DIAG_THREADS = 256;
+constexpr int PW = 8;                         // panel width
+
+// 1/sqrt(d) for a pivot d > 0 by Newton–Raphson on f(y) = y⁻² − d,
+// y ← y·(3 − d·y²)/2, started from the float32 reciprocal-square-root estimate
+// (≈ 2⁻²² relative); quadratic convergence gives float64 precision after two
+// steps.  Much shorter on the critical path than a correctly rounded float64
+// sqrt followed by a division.  Pivots outside the float32 range take the
+// exact route.
+__device__ __forceinline__ double rsqrt_pivot(double d) {
+  if (d < 1e-30 || d > 1e30) return 1.0 / sqrt(d);
+  double y = (double)rsqrtf((float)d);
+  y = y * (1.5 - 0.5 * d * y * y);
+  y = y * (1.5 - 0.5 * d * y * y);
+  return y;
+}
+
+__global__ void __launch_bounds__(DIAG_THREADS)
 chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
                  double* __restrict__ D, int64_t n, int64_t np, int k,
                  int32_t* info) {
@@ -182,64 +205,110 @@ chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
   extern __shared__ double sm[];
   double (*a)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);
   double (*b)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  __shared__ int bad_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t base = (int64_t)k * NB;
-  for (int e = tid; e < NB * NB; e += 256) {
+  for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
     const int r = e / NB, c = e % NB;
     a[r][c] = (c <= r) ? A[(base + r) * np + base + c] : 0.0;
     b[r][c] = (r == c) ? 1.0 : 0.0;
   }
+  if (tid == 0) bad_s = 0;
   __syncthreads();
-  double prev_piv = 0.0, prev_rp = 0.0;
-  bool bad = false;
-  for (int c = 0; c < NB; ++c) {
-    const double d = a[c][c];
-    if (!(d > 0.0) || !isfinite(d)) {
-      if (tid == 0) {
-        const int64_t apos = base + c;                // index in A
-        report(info, isfinite(d) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE,
-               n - 1 - apos);                         // processing position
+
+  for (int c0 = 0; c0 < NB; c0 += PW) {
+    if (warp == 0) {
+      // ---- phase 1: the panel, rows c0..63, columns c0..c0+7
+      double v0[PW], v1[PW];                 // rows lane and lane + 32
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        v0[c] = a[lane][c0 + c];
+        v1[c] = a[lane + 32][c0 + c];
       }
-      bad = true;
-      break;
-    }
-    const double piv = sqrt(d);
-    const double rp = 1.0 / piv;
-    // deferred scaling of column c−1 of a and row c−1 of b
-    if (c > 0) {
-      for (int r = c + tid; r < NB; r += 256) a[r][c - 1] *= prev_rp;
-      for (int x = tid; x < c; x += 256) b[c - 1][x] *= prev_rp;
-      if (tid == 0) a[c - 1][c - 1] = prev_piv;
-    }
-    // rank-1 updates with l = column c scaled by 1/piv
+      double ys[PW];
+      bool bad = false;
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      const int r = ty * 4 + rr;
-      if (r <= c) continue;
-      const double lr = a[r][c] * rp;
+      for (int c = 0; c < PW; ++c) {
+        const int pr = c0 + c;
+        const double mine = (pr < 32) ? v0[c] : v1[c];
+        const double d = __shfl_sync(0xffffffffu, mine, pr & 31);
+        if (!(d > 0.0) || !isfinite(d)) bad = true;
+        const double y = (d > 0.0) ? rsqrt_pivot(d) : 0.0;
+        ys[c] = y;
+        // scale column c below the pivot; the pivot becomes sqrt(d)
+        if (lane > pr) v0[c] *= y;
+        else if (lane == pr) v0[c] = d * y;
+        if (lane + 32 > pr) v1[c] *= y;
+        else if (lane + 32 == pr) v1[c] = d * y;
+        // update the panel's later columns
 #pragma unroll
-      for (int xx = 0; xx < 4; ++xx) {
-        const int x = tx * 4 + xx;
-        if (x > c) {
-          if (x <= r) a[r][x] -= lr * (a[x][c] * rp);
+        for (int cc = c + 1; cc < PW; ++cc) {
+          const int rr = c0 + cc;                     // row whose multiplier we need
+          const double own = (rr < 32) ? v0[c] : v1[c];
+          const double lk = __shfl_sync(0xffffffffu, own, rr & 31);
+          if (lane >= rr) v0[cc] -= v0[c] * lk;
+          if (lane + 32 >= rr) v1[cc] -= v1[c] * lk;
+        }
+      }
+      if (bad) {
+        if (lane == 0) {
+          bad_s = 1;
+          report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + c0));
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        if (lane >= c0) a[lane][c0 + c] = v0[c];
+        if (lane + 32 >= c0) a[lane + 32][c0 + c] = v1[c];
+      }
+      __syncwarp();
+      // panel rows of D: forward substitution over the panel, lanes over x
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        const int pr = c0 + c;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int x = lane + 32 * h;
+          if (x <= pr) {
+            double acc = b[pr][x];
+#pragma unroll
+            for (int cp = 0; cp < c; ++cp) acc -= a[pr][c0 + cp] * b[c0 + cp][x];
+            b[pr][x] = acc * ys[c];
+          }
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    if (bad_s) return;
+    // ---- phase 2: rank-8 update of rows below the panel
+    const int rs = c0 + PW;
+    for (int r = rs + warp; r < NB; r += DIAG_THREADS / 32) {
+      double lr[PW];
+#pragma unroll
+      for (int c = 0; c < PW; ++c) lr[c] = a[r][c0 + c];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int x = lane + 32 * h;
+        if (x >= rs) {
+          if (x <= r) {
+            double acc = a[r][x];
+#pragma unroll
+            for (int c = 0; c < PW; ++c) acc -= lr[c] * a[x][c0 + c];
+            a[r][x] = acc;
+          }
         } else {
-          b[r][x] -= lr * (b[c][x] * rp);
+          double acc = b[r][x];
+#pragma unroll
+          for (int c = 0; c < PW; ++c) acc -= lr[c] * b[c0 + c][x];
+          b[r][x] = acc;
         }
       }
     }
-    prev_piv = piv;
-    prev_rp = rp;
     __syncthreads();
   }
-  if (bad) return;
-  // last column's deferred scaling
-  for (int x = tid; x < NB - 1; x += 256) b[NB - 1][x] *= prev_rp;
-  if (tid == 0) {
-    a[NB - 1][NB - 1] = prev_piv;
-    b[NB - 1][NB - 1] *= prev_rp;
-  }
-  __syncthreads();
-  for (int e = tid; e < NB * NB; e += 256) {
+
+  for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
     const int r = e / NB, c = e % NB;
     if (c <= r) A[(base + r) * np + base + c] = a[r][c];
     M[(base + r) * np + base + c] = b[r][c];
@@ -247,31 +316,82 @@ chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
   }
 }
 
-// 64×64 float64 tile product C = X·Y on shared-memory tiles; each of the 256
-// threads owns a 4×4 block of C.
-__device__ __forceinline__ void tile_mm(const double (*x)[LDT], const double (*y)[LDT],
-                                        double acc[4][4], int tx, int ty) {
+// 64×64 float64 tile products on the float64 tensor cores (DMMA,
+// mma.sync m8n8k4).  Tiles sit in shared memory with a row stride of 68
+// doubles, which spreads the fragment reads over all banks.  Warp w owns rows
+// 16·(w/2) .. +16 and columns 32·(w%2) .. +32 of C: 2 × 4 accumulator tiles
+// of 8×8, two doubles per thread each (row g = lane/4, columns 2·(lane%4)+{0,1}).
+constexpr int LDM = 68;
+
+__device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ void tile_mm(const double (*x)[LDM], const double (*y)[LDM],
+                                        double acc[2][4][2], int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
 #pragma unroll 4
-  for (int q = 0; q < NB; ++q) {
-    double xv[4], yv[4];
+  for (int q = 0; q < NB; q += 4) {
+    double a[2], b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      xv[i] = x[ty * 4 + i][q];
-      yv[i] = y[q][tx * 4 + i];
-    }
+    for (int i = 0; i < 2; ++i) a[i] = x[rb + 8 * i + g][q + t];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 4; ++j) b[j] = y[q + t][cb + 8 * j + g];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv[i], yv[j], acc[i][j]);
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dmma_884(acc[i][j], a[i], b[j]);
   }
 }
 
-__device__ __forceinline__ void load_tile(double (*dst)[LDT], const double* src,
+// out ±= C (sign = +1 stores C, −1 subtracts it), leading dimension ld.
+template <bool SUBTRACT>
+__device__ __forceinline__ void tile_store(double* out, int64_t ld, const double acc[2][4][2],
+                                           int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double2* p = reinterpret_cast<double2*>(out + (int64_t)(rb + 8 * i + g) * ld + cb + 8 * j + 2 * t);
+      double2 v;
+      if (SUBTRACT) {
+        v = *p;
+        v.x -= acc[i][j][0];
+        v.y -= acc[i][j][1];
+      } else {
+        v = make_double2(acc[i][j][0], acc[i][j][1]);
+      }
+      *p = v;
+    }
+}
+
+// 64×64 float64 tile from global (leading dimension ld) into shared memory,
+// optionally transposed; 16-byte loads, all issued before the stores.
+__device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
                                           int64_t ld, bool transpose, int tid) {
-  for (int e = tid; e < NB * NB; e += 256) {
-    const int r = e / NB, c = e % NB;
-    const double v = src[(int64_t)r * ld + c];
-    if (transpose) dst[c][r] = v; else dst[r][c] = v;
+  double2 buf[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = tid + 256 * k;            // 2048 pairs
+    const int r = e >> 5, c2 = (e & 31) * 2;
+    buf[k] = *reinterpret_cast<const double2*>(src + (int64_t)r * ld + c2);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = tid + 256 * k;
+    const int r = e >> 5, c2 = (e & 31) * 2;
+    if (transpose) {
+      dst[c2][r] = buf[k].x;
+      dst[c2 + 1][r] = buf[k].y;
+    } else {
+      dst[r][c2] = buf[k].x;
+      dst[r][c2 + 1] = buf[k].y;
+    }
   }
 }
 
@@ -282,9 +402,9 @@ chol_panel_kernel(double* __restrict__ A, double* __restrict__ M,
                   int32_t* info) {
   if (info[0] != 0) return;
   extern __shared__ double sm[];
-  double (*x)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);
-  double (*y)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
+  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nlow = N - k - 1;
   double* out;
   if ((int)blockIdx.x < nlow) {
@@ -299,12 +419,9 @@ chol_panel_kernel(double* __restrict__ A, double* __restrict__ M,
     load_tile(y, out, np, false, tid);
   }
   __syncthreads();
-  double acc[4][4] = {};
-  tile_mm(x, y, acc, tx, ty);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) out[(int64_t)(ty * 4 + i) * np + tx * 4 + j] = acc[i][j];
+  double acc[2][4][2] = {};
+  tile_mm(x, y, acc, warp, lane);
+  tile_store<false>(out, np, acc, warp, lane);
 }
 
 // trail(k): first r(r+1)/2 blocks are (i, j), k < j ≤ i: A_ij −= L_ik·L_jkᵀ;
@@ -314,9 +431,9 @@ chol_trail_kernel(double* __restrict__ A, double* __restrict__ M, int64_t np,
                   int N, int k, int32_t* info) {
   if (info[0] != 0) return;
   extern __shared__ double sm[];
-  double (*x)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);
-  double (*y)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
+  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = N - k - 1;
   const int ntri = r * (r + 1) / 2;
   int lin = blockIdx.x;
@@ -337,12 +454,9 @@ chol_trail_kernel(double* __restrict__ A, double* __restrict__ M, int64_t np,
     load_tile(y, M + (int64_t)k * NB * np + (int64_t)c * NB, np, false, tid);
   }
   __syncthreads();
-  double acc[4][4] = {};
-  tile_mm(x, y, acc, tx, ty);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) out[(int64_t)(ty * 4 + i) * np + tx * 4 + j] -= acc[i][j];
+  double acc[2][4][2] = {};
+  tile_mm(x, y, acc, warp, lane);
+  tile_store<true>(out, np, acc, warp, lane);
 }
 
 // U[i][j] = L⁻¹[n−1−i][n−1−j] for j ≥ i, 0 below the diagonal.
@@ -390,7 +504,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  const size_t tile_smem = 2 * NB * LDT * sizeof(double);
+  const size_t tile_smem = 2 * NB * LDM * sizeof(double);   // ≥ the diagonal kernel's 2·NB·LDT
   if (!g_smem_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(chol_diag_kernel,
               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
@@ -411,7 +525,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);
   for (int k = 0; k < N; ++k) {
-    GPTQ_LAUNCH(KK_CHOL_DIAG, s, chol_diag_kernel, 1, 256, tile_smem, w.A, w.M, w.D, n, np, k, info);
+    GPTQ_LAUNCH(KK_CHOL_DIAG, s, chol_diag_kernel, 1, DIAG_THREADS, tile_smem, w.A, w.M, w.D, n, np, k, info);
     const int r = N - k - 1;
     if (r + k > 0)
       GPTQ_LAUNCH(KK_CHOL_PANEL, s, chol_panel_kernel, r + k, 256, tile_smem,

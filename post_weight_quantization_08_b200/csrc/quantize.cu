@@ -15,8 +15,12 @@ namespace {
 struct QuantWs {
   float* Wp;        // m × n working copy, processing order
   uint8_t* codes;   // m × n codes, processing order
-  float* Err;       // m × block scaled errors of the current block
+  float* Ehi;       // m × 128 scaled errors of the current block, TF32 part
+  float* Elo;       // m × 128 remainder e − Ehi
   int32_t* pinv;    // n: processing position of each original column
+  float* panels;    // pre-transposed U panels, one per block
+  float* Uhi;       // n × n TF32 part of Uᵀ (tensor-core trailing update only)
+  float* Ulo;       // n × n remainder, transposed likewise
 };
 
 size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) {
@@ -28,13 +32,22 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   };
   size_t o_wp = take(sizeof(float) * (size_t)m * (size_t)n);
   size_t o_codes = take((size_t)m * (size_t)n);
-  size_t o_err = take(sizeof(float) * (size_t)m * (size_t)block);
+  size_t o_ehi = take(sizeof(float) * (size_t)m * SWEEP_BLOCK_MAX);
+  size_t o_elo = take(sizeof(float) * (size_t)m * SWEEP_BLOCK_MAX);
   size_t o_pinv = take(sizeof(int32_t) * (size_t)n);
+  size_t o_pan = take(panel_workspace_bytes(n, block));
+  const bool tc = trailing_uses_tensor_cores(n, block);
+  size_t o_uhi = tc ? take(sizeof(float) * (size_t)n * (size_t)n) : 0;
+  size_t o_ulo = tc ? take(sizeof(float) * (size_t)n * (size_t)n) : 0;
   if (w && base) {
     w->Wp = reinterpret_cast<float*>(base + o_wp);
     w->codes = reinterpret_cast<uint8_t*>(base + o_codes);
-    w->Err = reinterpret_cast<float*>(base + o_err);
+    w->Ehi = reinterpret_cast<float*>(base + o_ehi);
+    w->Elo = reinterpret_cast<float*>(base + o_elo);
     w->pinv = reinterpret_cast<int32_t*>(base + o_pinv);
+    w->panels = reinterpret_cast<float*>(base + o_pan);
+    w->Uhi = tc ? reinterpret_cast<float*>(base + o_uhi) : nullptr;
+    w->Ulo = tc ? reinterpret_cast<float*>(base + o_ulo) : nullptr;
   }
   return off;
 }
@@ -172,13 +185,21 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
     GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<float>, gin, 256, 0,
                 static_cast<const float*>(W), m, n, perm, dead, w.Wp, info);
 
+  gptq_status st = launch_panels(U, n, block, w.panels, s);
+  if (st != GPTQ_OK) return st;
+  if (w.Uhi != nullptr && n > block) {
+    st = launch_split_tf32_t(U, n, w.Uhi, w.Ulo, s);
+    if (st != GPTQ_OK) return st;
+  }
   for (int64_t j0 = 0; j0 < n; j0 += block) {
     const int bw = (int)((n - j0 < block) ? (n - j0) : block);
-    gptq_status st = launch_sweep(w.Wp, m, n, j0, bw, U, bits, group, ngroups,
-                                  w.codes, scale, zero, w.Err, block, loss_row, s);
+    const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
+    st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes, scale,
+                      zero, w.Ehi, w.Elo, loss_row, info, s);
     if (st != GPTQ_OK) return st;
     if (j0 + bw < n) {
-      st = launch_trailing(w.Wp, m, n, j0 + bw, w.Err, block, j0, bw, U, s);
+      st = launch_trailing(w.Wp, m, n, j0 + bw, w.Ehi, w.Elo, j0, bw, U, w.Uhi, w.Ulo, info,
+                           s);
       if (st != GPTQ_OK) return st;
     }
   }

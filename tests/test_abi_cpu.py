@@ -57,8 +57,8 @@ FAKE = C.c_void_p(0x100000)   # never dereferenced: validation returns first
 
 def test_host_validation_without_gpu(lib):
     # null pointers
-    assert lib.gptq_hessian_accumulate(None, 10, 10, None, None) == 1
-    assert lib.gptq_hessian_accumulate(FAKE, -1, 10, FAKE, None) == 1
+    assert lib.gptq_hessian_accumulate(None, 10, 10, None, None, None) == 1
+    assert lib.gptq_hessian_accumulate(FAKE, -1, 10, FAKE, None, None) == 1
     assert lib.gptq_prepare(None, 10, 0.01, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 1
     assert lib.gptq_prepare(FAKE, 10, -1.0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 1
     assert lib.gptq_prepare(FAKE, 10, 0.01, 9, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 1
