@@ -120,6 +120,33 @@ gptq_status gptq_prepare(const float* H, int64_t n, double damp, int order,
                          int32_t* perm, float* U, uint8_t* dead, int32_t* info,
                          void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * gptq_prepare without a workspace argument: the same operation, arguments
+ * and results as gptq_prepare, for callers that cannot hand this library a
+ * block of device memory — for example code that runs while another
+ * framework owns every allocation on the device, a plugin with no allocator
+ * of its own, or a caller that must not call cudaMalloc/cudaFree (which
+ * synchronise the device) on a latency-sensitive path.  The pages have no
+ * counterpart to this entry point.
+ *   The scratch is a fixed array inside the library (about 16 MB for the
+ *   limit below), reserved on every GPU that loads the library until the
+ *   process exits.  This call allocates nothing: no cudaMalloc, no cudaFree,
+ *   no allocating library routine.
+ *   n must be at most GPTQ_NOALLOC_MAX_N; larger n returns
+ *   GPTQ_ERR_INVALID_ARG with a message (use gptq_prepare instead).
+ *   The first call on each device looks up the array's device address
+ *   (with that device current); make that first call before any stream
+ *   capture.
+ *   All calls on one device share the array and it keeps the last call's
+ *   contents; the call initialises every part it reads.  Calls whose work
+ *   overlaps on the GPU (different streams, or different host threads, on
+ *   the same device) race on the array: serialise them.
+ */
+#define GPTQ_NOALLOC_MAX_N 1024
+gptq_status gptq_prepare_noalloc(const float* H, int64_t n, double damp, int order,
+                                 int32_t* perm, float* U, uint8_t* dead, int32_t* info,
+                                 void* stream);
+
 /* Bytes of device workspace gptq_quantize needs (256-byte aligned). */
 size_t gptq_quantize_workspace_bytes(int64_t m, int64_t n, int block);
 

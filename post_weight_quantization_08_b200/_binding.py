@@ -30,6 +30,9 @@ _SIGS = {
     "gptq_prepare": (C.c_int, [C.c_void_p, C.c_int64, C.c_double, C.c_int, C.c_void_p,
                                C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
                                C.c_void_p]),
+    "gptq_prepare_noalloc": (C.c_int, [C.c_void_p, C.c_int64, C.c_double, C.c_int,
+                                       C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.c_void_p]),
     "gptq_quantize_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int]),
     "gptq_quantize": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
                                 C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,

@@ -539,3 +539,61 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
               w.M, n, np, U);
   return GPTQ_OK;
 }
+
+// ---------------------------------------------------------------------------
+// gptq_prepare_noalloc: gptq_prepare on a scratch area that lives in the
+// library itself, for callers that cannot hand over device memory.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace gptq {
+namespace {
+
+constexpr int64_t kNoAllocMaxN = GPTQ_NOALLOC_MAX_N;
+constexpr size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+// Same arithmetic as prep_ws_layout() for n = kNoAllocMaxN (a multiple of 64).
+constexpr size_t kNoAllocBytes =
+    up256(sizeof(double)) + up256(sizeof(int32_t) * kNoAllocMaxN) +
+    2 * up256(sizeof(double) * kNoAllocMaxN * kNoAllocMaxN) + up256(sizeof(double) * NB * NB);
+static_assert(kNoAllocMaxN % NB == 0, "the fixed limit is a whole number of tiles");
+
+// The scratch itself: every GPU that loads this library holds it until the
+// process exits.  All calls on one device share it.
+static __device__ __align__(256) unsigned char g_prepare_scratch[kNoAllocBytes];
+
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 128;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+}  // namespace gptq
+
+extern "C" gptq_status gptq_prepare_noalloc(const float* H, int64_t n, double damp, int order,
+                                            int32_t* perm, float* U, uint8_t* dead,
+                                            int32_t* info, void* stream) {
+  if (n < 1 || n > kNoAllocMaxN)
+    return fail(GPTQ_ERR_INVALID_ARG,
+                "gptq_prepare_noalloc: n=%lld is outside 1..%lld, the size of the library's "
+                "fixed scratch; use gptq_prepare with a caller workspace",
+                (long long)n, (long long)kNoAllocMaxN);
+  if (prep_ws_layout(n, nullptr, nullptr) > sizeof(g_prepare_scratch))
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare_noalloc: scratch layout exceeds the array");
+  int dev = 0;
+  GPTQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare_noalloc: device ordinal %d", dev);
+  void* scratch = nullptr;
+  {
+    // Once per device, with that device current: the device address of the
+    // array (host code only sees a stand-in symbol, not a device pointer).
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    scratch = g_noalloc_ptr[dev];
+    if (scratch == nullptr) {
+      cudaError_t e = cudaGetSymbolAddress(&scratch, g_prepare_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_prepare_scratch)");
+      g_noalloc_ptr[dev] = scratch;
+    }
+  }
+  return gptq_prepare(H, n, damp, order, perm, U, dead, info, scratch,
+                      sizeof(g_prepare_scratch), stream);
+}
