@@ -5,10 +5,12 @@
 
 namespace gptq {
 
-// Largest block width, and the bytes of one pre-transposed U panel
-// (UT[128][132] floats plus 128 reciprocal diagonals).
+// Largest block width, and the bytes of the per-block package of U that the
+// sweep fetches with one bulk copy: 12 swizzled 32×32 TF32 boxes (hi and lo
+// of the 6 off-diagonal pieces), 4 diagonal 32×32 pieces, 128 reciprocal
+// diagonals.
 constexpr int SWEEP_BLOCK_MAX = 128;
-constexpr size_t PANEL_BYTES = (size_t)(128 * 132 + 128) * sizeof(float);
+constexpr size_t PANEL_BYTES = (size_t)16 * 4096 + 128 * sizeof(float);
 
 size_t panel_workspace_bytes(int64_t n, int block);
 

@@ -8,21 +8,26 @@
 // block's later columns; the columns after the block receive the block's
 // errors in one product afterwards (trailing.cu).
 //
-// Rows are independent (U is shared), so one thread owns one row and a CTA
-// owns 128 rows.  The block's U panel is pre-transposed once per call
-// (panel_kernel: UT[c][i] = U[j0+i][j0+c] plus 1/U_jj) so that each CTA
-// fetches it with a single bulk (TMA) copy into shared memory while its
-// threads load their rows.  The block is walked in sub-blocks of 32 columns
-// held in registers: the 32 dependent column steps run fully unrolled, then
-// the sub-block's 32 errors update the block's later columns (four columns
-// at a time for instruction-level parallelism) with vectorised panel reads.
+// One thread owns one row; a CTA owns 128 rows and walks the block in
+// sub-blocks of 32 columns:
+//   * the 32 dependent column steps of a sub-block run unrolled in registers,
+//     each step updating the sub-block's later columns in float32 with the
+//     sub-block's diagonal 32×32 piece of U (row-major, vector reads);
+//   * the sub-block's errors E (128 rows × 32) then update the block's later
+//     columns on the tensor core: D[rows, later] += E·U[sub-block rows, later]
+//     with tcgen05.mma kind::tf32 and the same three-term TF32 split as the
+//     trailing update (E = E_hi + E_lo, U = U_hi + U_lo, lo·lo dropped).  D
+//     lives in tensor memory (TMEM lane = row = thread) and accumulates over
+//     the sub-blocks; a sub-block's current values are its loaded values
+//     minus D, read back with tcgen05.ld.
+// Everything U-derived a CTA needs (the B operands in K-major, 128-byte
+// swizzled boxes, the diagonal pieces and 1/U_jj) is packed once per call by
+// package_kernel and fetched with one bulk (TMA) copy per CTA.
 //
 // Scale and zero: min-max over the group's current values at the group's
 // first column, the range always containing 0; decisions in IEEE float32
-// (correctly rounded division and rint, no fast-math).
-//
-// The block's errors leave as a TF32 split (Ehi = TF32(e), Elo = e − Ehi) for
-// the tensor-core trailing update.
+// (correctly rounded division and rint, no fast-math).  The block's errors
+// also leave as a TF32 split (Ehi, Elo) for the trailing update.
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -30,73 +35,126 @@ namespace gptq {
 namespace {
 
 constexpr int SB = 128;       // largest block width
-constexpr int SS = 32;        // register sub-block
-constexpr int LDU = SB + 4;   // transposed-panel row stride (floats; 16-byte rows)
+constexpr int SS = 32;        // sub-block
 constexpr int RT = 128;       // rows (threads) per CTA
 constexpr int LDV = SB + 1;   // row-major values, odd stride: conflict-free columns
 constexpr int LDB = SB + 4;   // bytes per staged code row
-constexpr size_t PANEL_FLOATS = (size_t)SB * LDU + SB;
-constexpr size_t SMEM_BYTES = PANEL_BYTES + sizeof(float) * RT * LDV + (size_t)RT * LDB + 16;
-static_assert(PANEL_BYTES == PANEL_FLOATS * sizeof(float), "panel layout");
-static_assert(PANEL_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
 
-// Panel of block b: UT[c][i] = U[j0+i][j0+c] (zero outside the block), and
-// rdiag[c] = 1/U[j0+c][j0+c].  32×32 tiles through shared memory.
+// package layout (bytes)
+constexpr uint32_t BOX = 32 * 128;                 // 32 rows × 32 TF32 (K-major, swizzled)
+constexpr uint32_t PK_BHI = 0;                     // 6 boxes: (s,t) for s < t ≤ 3
+constexpr uint32_t PK_BLO = 6 * BOX;
+constexpr uint32_t PK_UD = 12 * BOX;               // 4 diagonal 32×32 pieces, row-major
+constexpr uint32_t PK_RD = PK_UD + 4 * 32 * 32 * 4;// 128 reciprocal diagonals
+constexpr uint32_t PK_BYTES = PK_RD + SB * 4;
+static_assert(PK_BYTES == PANEL_BYTES, "package size");
+static_assert(PK_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
+
+__host__ __device__ constexpr int box_index(int s, int t) {   // s < t
+  return s == 0 ? t - 1 : (s == 1 ? t + 1 : 5);
+}
+
+// smem layout (bytes from a 1024-aligned base)
+constexpr uint32_t SM_PKG = 0;
+constexpr uint32_t SM_AHI = 66560;                 // 65 KB, 1024-aligned
+constexpr uint32_t SM_ALO = SM_AHI + RT * 128;
+constexpr uint32_t SM_VALS = SM_ALO + RT * 128;
+constexpr uint32_t SM_CODES = SM_VALS + RT * LDV * 4;
+constexpr uint32_t SM_BARS = (SM_CODES + RT * LDB + 15) / 16 * 16;
+constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 32;
+static_assert(SM_AHI >= PK_BYTES && SM_AHI % 1024 == 0, "A operand placement");
+
+// Package of block b.  blockIdx.y: 0..5 a B box (hi and lo), 6..9 a diagonal
+// piece, 10 the reciprocal diagonals.  Box (s,t) holds, in K-major 128-byte
+// swizzled layout, row nn = column j0+32t+nn of U and, along K, kk = rows
+// j0+32s+kk: element at byte nn·128 + ((kk/4) ^ (nn mod 8))·16 + (kk mod 4)·4.
 __global__ void __launch_bounds__(256)
-panel_kernel(const float* __restrict__ U, int64_t n, int block,
-             float* __restrict__ panels) {
+package_kernel(const float* __restrict__ U, int64_t n, int block,
+               unsigned char* __restrict__ pkgs) {
   __shared__ float tile[32][33];
-  const int b = blockIdx.x, ci = blockIdx.y, ii = blockIdx.z;
+  const int b = blockIdx.x, part = blockIdx.y;
   const int64_t j0 = (int64_t)b * block;
   const int bw = (int)((n - j0 < block) ? (n - j0) : block);
-  float* P = panels + (size_t)b * PANEL_FLOATS;
+  unsigned char* P = pkgs + (size_t)b * PK_BYTES;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  if (part < 6) {
+    const int s = part < 3 ? 0 : (part < 5 ? 1 : 2);
+    const int t = part < 3 ? part + 1 : (part < 5 ? part - 1 : 3);
+    // tile[kk][nn] = U[j0+32s+kk][j0+32t+nn]
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int i = ii * 32 + ty + 8 * k, c = ci * 32 + tx;
-    tile[ty + 8 * k][tx] = (i < bw && c < bw) ? U[(j0 + i) * n + j0 + c] : 0.f;
-  }
-  __syncthreads();
+    for (int q = 0; q < 4; ++q) {
+      const int kk = ty + 8 * q, nn = tx;
+      const int r = 32 * s + kk, c = 32 * t + nn;
+      tile[kk][nn] = (r < bw && c < bw) ? U[(j0 + r) * n + j0 + c] : 0.f;
+    }
+    __syncthreads();
+    float* hi = reinterpret_cast<float*>(P + PK_BHI + box_index(s, t) * BOX);
+    float* lo = reinterpret_cast<float*>(P + PK_BLO + box_index(s, t) * BOX);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = ci * 32 + ty + 8 * k, i = ii * 32 + tx;
-    P[c * LDU + i] = tile[tx][ty + 8 * k];
-  }
-  if (ii == 3 && threadIdx.x < 32 * (LDU - SB)) {       // zero the row padding
-    const int c = ci * 32 + (threadIdx.x >> 2), p = SB + (threadIdx.x & 3);
-    P[c * LDU + p] = 0.f;
-  }
-  if (ii == ci && ty == 0) {
-    const int c = ci * 32 + tx;
-    P[SB * LDU + c] = (c < bw) ? 1.0f / U[(j0 + c) * n + j0 + c] : 0.f;
+    for (int q = 0; q < 4; ++q) {
+      const int nn = ty + 8 * q, kk = tx;
+      const float v = tile[kk][nn];
+      const float h = to_tf32(v);
+      const int off = nn * 32 + (((kk >> 2) ^ (nn & 7)) << 2) + (kk & 3);   // floats
+      hi[off] = h;
+      lo[off] = v - h;
+    }
+  } else if (part < 10) {
+    const int s = part - 6;
+    float* ud = reinterpret_cast<float*>(P + PK_UD) + s * 32 * 32;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = ty + 8 * q, kk = tx;
+      const int r = 32 * s + i, c = 32 * s + kk;
+      ud[i * 32 + kk] = (r < bw && c < bw) ? U[(j0 + r) * n + j0 + c] : 0.f;
+    }
+  } else if (threadIdx.x < SB) {
+    const int c = threadIdx.x;
+    float* rd = reinterpret_cast<float*>(P + PK_RD);
+    rd[c] = (c < bw) ? 1.0f / U[(j0 + c) * n + j0 + c] : 0.f;
   }
 }
 
-__global__ void __launch_bounds__(RT)
+__global__ void __launch_bounds__(RT, 1)
 sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
-             const float* __restrict__ panel, int bits, int group, int64_t ngroups,
+             const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
              uint8_t* __restrict__ codes, float* __restrict__ scale,
              uint8_t* __restrict__ zero, float* __restrict__ Ehi,
              float* __restrict__ Elo, float* __restrict__ loss_row, int32_t* info) {
-  extern __shared__ __align__(128) unsigned char smraw[];
-  float* UT = reinterpret_cast<float*>(smraw);
-  const float* rdiag = UT + SB * LDU;
-  float* vals = reinterpret_cast<float*>(smraw + PANEL_BYTES);
-  uint8_t* cs = reinterpret_cast<uint8_t*>(vals + RT * LDV);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(cs + RT * LDB);
+  extern __shared__ unsigned char smraw[];
+  const uint32_t raw = smem_addr(smraw);
+  unsigned char* sm = smraw + ((1024 - (raw & 1023)) & 1023);
+  const float* Ud = reinterpret_cast<const float*>(sm + SM_PKG + PK_UD);
+  const float* rdiag = reinterpret_cast<const float*>(sm + SM_PKG + PK_RD);
+  unsigned char* ahi = sm + SM_AHI;
+  unsigned char* alo = sm + SM_ALO;
+  float* vals = reinterpret_cast<float*>(sm + SM_VALS);
+  uint8_t* cs = sm + SM_CODES;
+  uint64_t* pkg_bar = reinterpret_cast<uint64_t*>(sm + SM_BARS);
+  uint64_t* mma_bar = pkg_bar + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(mma_bar + 1);
 
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t r0 = (int64_t)blockIdx.x * RT;
   const int64_t row = r0 + t;
 
   if (t == 0) {
-    mbar_init(bar, 1);
+    mbar_init(pkg_bar, 1);
+    mbar_init(mma_bar, 1);
     fence_barrier_init();
   }
+  if (warp == 0) {
+    tmem_alloc(tslot, SB);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
   if (t == 0) {
-    mbar_arrive_expect_tx(bar, (uint32_t)PANEL_BYTES);
-    bulk_g2s(UT, panel, (uint32_t)PANEL_BYTES, bar);
+    mbar_arrive_expect_tx(pkg_bar, PK_BYTES);
+    bulk_g2s(sm + SM_PKG, pkg, PK_BYTES, pkg_bar);
   }
 
   // this thread's row of the block → vals (row-major, odd stride)
@@ -125,25 +183,55 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
     for (int c = 0; c < SB; ++c) vr[c] = 0.f;
   }
 
-  if (!mbar_wait_bounded(bar, 0)) {
+  bool abort = !mbar_wait_bounded(pkg_bar, 0);
+  if (abort) {
     report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
-    if (t == 0) mbar_wait_bounded(bar, 0);   // let our own copy land first
-    return;
+    if (t == 0) mbar_wait_bounded(pkg_bar, 0);   // let our own copy land first
   }
 
   const float maxq = (float)((1 << bits) - 1);
   float s = 1.f, z = 0.f, loss = 0.f;
   uint8_t* cr = cs + t * LDB;
   const int nsb = (bw + SS - 1) / SS;
-  for (int sb = 0; sb < nsb; ++sb) {
+  int issued = 0;                       // MMA groups committed to mma_bar
+  for (int sb = 0; sb < nsb && !abort; ++sb) {
     const int c0 = sb * SS;
+    float v[SS], e[SS];
+    if (sb == 0) {
+#pragma unroll
+      for (int k = 0; k < SS; ++k) v[k] = vr[k];
+    } else {
+      const bool ok = mbar_wait_bounded(mma_bar, (sb - 1) & 1);
+      if (__syncthreads_or(!ok)) {
+        report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+        abort = true;
+        break;
+      }
+      tc_fence_after();
+      float d[32];
+      tmem_ld_32x32b_x32(trow + c0, d);
+#pragma unroll
+      for (int k = 0; k < SS; ++k) v[k] = vr[c0 + k] - d[k];
+    }
     if (c0 % group == 0) {
-      const int cend = min(c0 + group, bw);
+      // the group's current values: this sub-block, then later ones in the group
       float xmin = 0.f, xmax = 0.f;
-      for (int c = c0; c < cend; ++c) {
-        const float x = vr[c];
+#pragma unroll
+      for (int k = 0; k < SS; ++k) {
+        const float x = (c0 + k < bw) ? v[k] : 0.f;
         xmin = fminf(xmin, x);
         xmax = fmaxf(xmax, x);
+      }
+      const int gend = min(c0 + group, bw);
+      for (int cs0 = c0 + SS; cs0 < gend; cs0 += SS) {
+        float d[32];
+        if (sb > 0) tmem_ld_32x32b_x32(trow + cs0, d);
+#pragma unroll
+        for (int k = 0; k < SS; ++k) {
+          const float x = (cs0 + k < gend) ? vr[cs0 + k] - (sb > 0 ? d[k] : 0.f) : 0.f;
+          xmin = fminf(xmin, x);
+          xmax = fmaxf(xmax, x);
+        }
       }
       if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
       s = __fdiv_rn(xmax - xmin, maxq);
@@ -154,9 +242,8 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
         zero[row * ngroups + g] = (uint8_t)z;
       }
     }
-    float v[SS], e[SS];
-#pragma unroll
-    for (int k = 0; k < SS; ++k) v[k] = vr[c0 + k];
+    // ---- the 32 dependent column steps
+    const float* ud = Ud + sb * SS * SS;
 #pragma unroll
     for (int i = 0; i < SS; ++i) {
       const int c = c0 + i;
@@ -166,53 +253,89 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
       e[i] = ei;
       loss = fmaf(ei, ei, loss);
       cr[c] = (uint8_t)q;
+      const float4* ur = reinterpret_cast<const float4*>(ud + i * SS);
 #pragma unroll
-      for (int k = i + 1; k < SS; ++k) v[k] = fmaf(-ei, UT[(c0 + k) * LDU + c], v[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < SS; ++k) vr[c0 + k] = e[k];
-    for (int c = c0 + SS; c < bw; c += 4) {
-      float a0 = vr[c], a1 = vr[c + 1], a2 = vr[c + 2], a3 = vr[c + 3];
-      const float4* u0 = reinterpret_cast<const float4*>(UT + (c + 0) * LDU + c0);
-      const float4* u1 = reinterpret_cast<const float4*>(UT + (c + 1) * LDU + c0);
-      const float4* u2 = reinterpret_cast<const float4*>(UT + (c + 2) * LDU + c0);
-      const float4* u3 = reinterpret_cast<const float4*>(UT + (c + 3) * LDU + c0);
-#pragma unroll
-      for (int q4 = 0; q4 < SS / 4; ++q4) {
-        const float4 x0 = u0[q4], x1 = u1[q4], x2 = u2[q4], x3 = u3[q4];
-        const float e0 = e[4 * q4], e1 = e[4 * q4 + 1], e2 = e[4 * q4 + 2], e3 = e[4 * q4 + 3];
-        a0 = fmaf(-e0, x0.x, a0); a1 = fmaf(-e0, x1.x, a1);
-        a2 = fmaf(-e0, x2.x, a2); a3 = fmaf(-e0, x3.x, a3);
-        a0 = fmaf(-e1, x0.y, a0); a1 = fmaf(-e1, x1.y, a1);
-        a2 = fmaf(-e1, x2.y, a2); a3 = fmaf(-e1, x3.y, a3);
-        a0 = fmaf(-e2, x0.z, a0); a1 = fmaf(-e2, x1.z, a1);
-        a2 = fmaf(-e2, x2.z, a2); a3 = fmaf(-e2, x3.z, a3);
-        a0 = fmaf(-e3, x0.w, a0); a1 = fmaf(-e3, x1.w, a1);
-        a2 = fmaf(-e3, x2.w, a2); a3 = fmaf(-e3, x3.w, a3);
+      for (int q4 = (i + 1) / 4; q4 < SS / 4; ++q4) {
+        const float4 u = ur[q4];
+        if (4 * q4 + 0 > i) v[4 * q4 + 0] = fmaf(-ei, u.x, v[4 * q4 + 0]);
+        if (4 * q4 + 1 > i) v[4 * q4 + 1] = fmaf(-ei, u.y, v[4 * q4 + 1]);
+        if (4 * q4 + 2 > i) v[4 * q4 + 2] = fmaf(-ei, u.z, v[4 * q4 + 2]);
+        if (4 * q4 + 3 > i) v[4 * q4 + 3] = fmaf(-ei, u.w, v[4 * q4 + 3]);
       }
-      vr[c] = a0; vr[c + 1] = a1; vr[c + 2] = a2; vr[c + 3] = a3;
+    }
+    // ---- errors out: TF32 split to global (trailing update) and to the
+    // K-major swizzled A operand in shared memory (in-block far update)
+    float eh[SS], el[SS];
+#pragma unroll
+    for (int k = 0; k < SS; ++k) {
+      eh[k] = to_tf32(e[k]);
+      el[k] = e[k] - eh[k];
+    }
+    if (row < m) {
+      float4* gh = reinterpret_cast<float4*>(Ehi + row * SB + c0);
+      float4* gl = reinterpret_cast<float4*>(Elo + row * SB + c0);
+#pragma unroll
+      for (int q = 0; q < SS / 4; ++q) {
+        gh[q] = make_float4(eh[4 * q], eh[4 * q + 1], eh[4 * q + 2], eh[4 * q + 3]);
+        gl[q] = make_float4(el[4 * q], el[4 * q + 1], el[4 * q + 2], el[4 * q + 3]);
+      }
+    }
+    if (sb + 1 < nsb) {
+#pragma unroll
+      for (int q = 0; q < SS / 4; ++q) {
+        const uint32_t off = t * 128 + ((q ^ (t & 7)) << 4);
+        *reinterpret_cast<float4*>(ahi + off) =
+            make_float4(eh[4 * q], eh[4 * q + 1], eh[4 * q + 2], eh[4 * q + 3]);
+        *reinterpret_cast<float4*>(alo + off) =
+            make_float4(el[4 * q], el[4 * q + 1], el[4 * q + 2], el[4 * q + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (t == 0) {
+        tc_fence_after();
+        // D[:, 32(sb+1) : 128] += E·U[c0:c0+32, 32(sb+1):128]
+        const uint32_t N = (uint32_t)(SB - SS * (sb + 1));
+        const uint32_t idesc = idesc_f32acc(2, 2, 0, 0, RT, N);
+        const uint32_t bhi = smem_addr(sm + SM_PKG + PK_BHI + box_index(sb, sb + 1) * BOX);
+        const uint32_t blo = smem_addr(sm + SM_PKG + PK_BLO + box_index(sb, sb + 1) * BOX);
+        const uint32_t ah = smem_addr(ahi), al = smem_addr(alo);
+        const uint32_t dcol = tmem + (uint32_t)(SS * (sb + 1));
+#pragma unroll
+        for (int ks = 0; ks < SS / 8; ++ks) {
+          const uint64_t dah = sdesc_sw128(ah + ks * 32, SW128_KMAJOR_LBO, 1024);
+          const uint64_t dal = sdesc_sw128(al + ks * 32, SW128_KMAJOR_LBO, 1024);
+          const uint64_t dbh = sdesc_sw128(bhi + ks * 32, SW128_KMAJOR_LBO, 1024);
+          const uint64_t dbl = sdesc_sw128(blo + ks * 32, SW128_KMAJOR_LBO, 1024);
+          umma_tf32_ss(dcol, dah, dbh, idesc, (sb > 0 || ks > 0) ? 1u : 0u);
+          umma_tf32_ss(dcol, dah, dbl, idesc, 1u);
+          umma_tf32_ss(dcol, dal, dbh, idesc, 1u);
+        }
+        umma_commit(mma_bar);
+      }
+      ++issued;
     }
   }
-  if (row < m && loss_row != nullptr) loss_row[row] += loss;
+  if (!abort && row < m && loss_row != nullptr) loss_row[row] += loss;
+  tc_fence_before();
   __syncthreads();
 
-  // errors and codes out, one warp per row, coalesced
-  const int lane = t & 31, warp = t >> 5;
-  for (int rr = warp; rr < RT; rr += RT / 32) {
-    const int64_t r = r0 + rr;
-    if (r >= m) break;
+  // codes out, one warp per row, coalesced
+  if (!abort) {
+    for (int rr = warp; rr < RT; rr += RT / 32) {
+      const int64_t r = r0 + rr;
+      if (r >= m) break;
 #pragma unroll
-    for (int it = 0; it < SB / 32; ++it) {
-      const int c = lane + 32 * it;
-      if (c < bw) {
-        const float e = vals[rr * LDV + c];
-        const float h = to_tf32(e);
-        Ehi[r * SB + c] = h;
-        Elo[r * SB + c] = e - h;
-        codes[r * n + j0 + c] = cs[rr * LDB + c];
+      for (int it = 0; it < SB / 32; ++it) {
+        const int c = lane + 32 * it;
+        if (c < bw) codes[r * n + j0 + c] = cs[rr * LDB + c];
       }
     }
   }
+  if (abort && t == 0 && issued > 0)            // no MMA may still write TMEM
+    mbar_wait_bounded(mma_bar, (issued - 1) & 1, 1u << 16);
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, SB);
 }
 
 bool g_attr_set = false;
@@ -225,8 +348,9 @@ size_t panel_workspace_bytes(int64_t n, int block) {
 
 gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
                           cudaStream_t s) {
-  const dim3 grid((unsigned)ceil_div(n, block), SB / 32, SB / 32);
-  GPTQ_LAUNCH(KK_INGEST, s, panel_kernel, grid, 256, 0, U, n, block, panels);
+  const dim3 grid((unsigned)ceil_div(n, block), 11);
+  GPTQ_LAUNCH(KK_INGEST, s, package_kernel, grid, 256, 0, U, n, block,
+              reinterpret_cast<unsigned char*>(panels));
   return GPTQ_OK;
 }
 
@@ -240,8 +364,9 @@ gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int 
     g_attr_set = true;
   }
   const unsigned grid = (unsigned)ceil_div(m, RT);
-  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, Wp, m, n, j0, bw, panel,
-              bits, group, ngroups, codes, scale, zero, Ehi, Elo, loss_row, info);
+  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, Wp, m, n, j0, bw,
+              reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
+              scale, zero, Ehi, Elo, loss_row, info);
   return GPTQ_OK;
 }
 

@@ -1,0 +1,81 @@
+"""GPU parity at the workloads' full sizes, through the same calls bench.py makes.
+
+The single 576×576 layer and the SmolLM-135M layer are checked in full (every
+row).  For the Qwen2.5-0.5B and TinyLlama-1.1B layers and the 8192² stress
+layer the GPU runs the whole problem and the oracle checks the Hessian and U
+in full (float64 on the GPU's own H) and the sweep on sampled rows — a row's
+result depends only on that row and U, so sampled rows are exact checks.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import gptq as og
+from workloads import problems_for
+
+from . import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+SAMPLE_ROWS = 96
+
+
+def _rows(m, seed):
+    rng = np.random.default_rng(seed)
+    k = min(m, SAMPLE_ROWS)
+    return np.sort(rng.choice(m, size=k, replace=False))
+
+
+def _check_problem(p, full_rows: bool, order=None, seed=0, hessian_full=True):
+    order = order or p.order
+    out = P.run_gpu(p.X, p.W, p.bits, p.group, p.block, p.damp, order, None, DEV,
+                    qdq=full_rows)
+    stats = {}
+    if hessian_full:
+        stats.update(P.check_hessian(p.X, out["H"]))
+    _, s2 = P.check_prepare(out["H"], out, p.damp, order)
+    stats.update(s2)
+    rows = None if full_rows else _rows(p.m, seed)
+    stats.update(P.check_quantize(p.W, out, None, p.bits, p.group, p.block, rows=rows))
+    if full_rows:
+        stats.update(P.check_layer_loss(p.X, p.W, out, p.bits, p.group, p.block, p.damp, order))
+    return stats, out
+
+
+def test_single_layer_full():
+    p = problems_for(0)[0]
+    st, _ = _check_problem(p, full_rows=True)
+    assert st["code_diff"] <= 1e-3 * st["codes"]
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_smollm_layer_full(which):
+    p = problems_for(1)[which]
+    st, _ = _check_problem(p, full_rows=True)
+    assert st["code_diff"] <= 1e-3 * st["codes"]
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_qwen_layer_sampled(which):
+    p = problems_for(2, layer=3)[which]
+    _check_problem(p, full_rows=False, seed=which)
+
+
+@pytest.mark.parametrize("bits,which", [(4, 0), (4, 1), (3, 1)])
+def test_tinyllama_layer_sampled(bits, which):
+    p = problems_for(3, layer=5, bits=bits)[which]
+    _check_problem(p, full_rows=False, seed=bits * 10 + which)
+
+
+@pytest.mark.parametrize("order", ["act", "reverse"])
+def test_stress_layer_sampled(order):
+    p = problems_for(4, order=order)[0]
+    # the float64 Hessian of 16384×8192 is checked on a block of entries
+    _, out = _check_problem(p, full_rows=False, order=order, seed=7, hessian_full=False)
+    Xs = p.X[:, :256].to(torch.float64).numpy()
+    H = out["H"]
+    Hr = og.hessian(Xs)
+    S = 2.0 * (np.abs(Xs).T @ np.abs(Xs))
+    T = Xs.shape[0]
+    assert np.all(np.abs(H[:256, :256] - Hr) <= 2.0 * T * 2.0 ** -24 * S + 1e-30)
