@@ -18,7 +18,10 @@
 //   warp 1 lane 0   MMA issuer: tcgen05.mma kind::f16 (bf16 in, f32 in TMEM),
 //                   M = N = 128, K = 16 per instruction, both operands
 //                   MN-major (X is token-major, so columns of H are contiguous);
-//   all 4 warps     epilogue: tcgen05.ld of the 128×128 accumulator, H += 2·D.
+//   all 4 warps     epilogue: tcgen05.ld of the 128×128 accumulator into
+//                   128-byte-swizzled shared boxes (2·D, and for off-diagonal
+//                   tiles also 2·Dᵀ), then TMA reduce-adds into H — no
+//                   read-modify-write round trips from the threads.
 // Every wait is bounded; a time-out is reported through `info`.
 // Fallback (n not a multiple of 8): a float32 SIMT tile kernel.
 #include <cuda_bf16.h>
@@ -105,10 +108,12 @@ constexpr uint32_t TC_OPER_BYTES = 2 * TC_BOX_BYTES;        // 128 columns
 constexpr uint32_t TC_STAGE_BYTES = 2 * TC_OPER_BYTES;      // A and B
 constexpr uint32_t TC_IDESC = idesc_f32acc(1, 1, 1, 1, TC_TILE, TC_TILE);   // bf16, MN-major
 constexpr size_t TC_SMEM = 1024 + TC_STAGES * TC_STAGE_BYTES + 256;
+constexpr uint32_t EP_BOX = 32 * TC_TILE * 4;               // 32 columns × 128 rows f32
+static_assert(8 * EP_BOX <= TC_STAGES * TC_STAGE_BYTES, "epilogue boxes reuse the ring");
 
 __global__ void __launch_bounds__(128, 1)
-hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, int64_t T, int64_t n, int nt,
-                  float* __restrict__ H, int32_t* info) {
+hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmH,
+                  int64_t T, int64_t n, int nt, int32_t* info) {
   extern __shared__ unsigned char smraw[];
   // 1024-byte aligned operand ring (128-byte swizzle atoms are 1 KB)
   const uint32_t raw = smem_addr(smraw);
@@ -192,40 +197,47 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, int64_t T, int64_t n,
   }
   __syncwarp();
 
-  // ---- epilogue: all four warps, one accumulator row per thread
+  // ---- epilogue: all four warps, one accumulator row per thread.  The ring
+  // is free again (every load was consumed, every MMA has retired): boxes
+  // 0..3 take 2·D (row r, columns 32b..32b+31), boxes 4..7 take 2·Dᵀ.
   const bool ok = mbar_wait_bounded(done, 0);
   if (!ok) report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
   tc_fence_after();
-  if (ok && !*abort_flag) {
-    const int64_t row = i0 + warp * 32 + lane;
+  const bool write = ok && !*abort_flag;
+  if (write) {
+    const int r = warp * 32 + lane;
 #pragma unroll 1
     for (int ch = 0; ch < TC_TILE / 32; ++ch) {
       float v[32];
       tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + ch * 32, v);
-      const int64_t jb = j0 + ch * 32;
-      if (row < n) {
-        float* hr = H + row * n + jb;
-        if (jb + 32 <= n) {
+      unsigned char* box = ring + ch * EP_BOX + r * 128;
 #pragma unroll
-          for (int k = 0; k < 32; k += 4) {
-            float4 h = *reinterpret_cast<float4*>(hr + k);
-            h.x += 2.f * v[k]; h.y += 2.f * v[k + 1]; h.z += 2.f * v[k + 2]; h.w += 2.f * v[k + 3];
-            *reinterpret_cast<float4*>(hr + k) = h;
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (jb + k < n) hr[k] += 2.f * v[k];
-        }
-      }
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(box + ((q ^ (r & 7)) << 4)) =
+            make_float4(2.f * v[4 * q], 2.f * v[4 * q + 1], 2.f * v[4 * q + 2], 2.f * v[4 * q + 3]);
       if (!diag) {
+        // Dᵀ: row c = 32·ch + k of the mirrored tile, column r
+        unsigned char* mbox = ring + (4 + warp) * EP_BOX;
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const int64_t j = jb + k;
-          if (row < n && j < n) H[j * n + row] += 2.f * v[k];
+          const int c = 32 * ch + k;
+          *reinterpret_cast<float*>(mbox + c * 128 + (((lane >> 2) ^ (c & 7)) << 4) + (lane & 3) * 4) =
+              2.f * v[k];
         }
       }
     }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (write && tid == 0) {
+#pragma unroll 1
+    for (int b = 0; b < TC_TILE / 32; ++b) {
+      if (j0 + 32 * b < n) tma_reduce_add_2d(&tmH, j0 + 32 * b, i0, ring + b * EP_BOX);
+      if (!diag && i0 + 32 * b < n) tma_reduce_add_2d(&tmH, i0 + 32 * b, j0, ring + (4 + b) * EP_BOX);
+    }
+    bulk_commit();
+    bulk_wait_all();
   }
   // ---- teardown: no copy or MMA may still be in flight when TMEM goes
   if (tid == 0) {
@@ -252,6 +264,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(tm, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool g_tc_attr = false;
 
 }  // namespace
@@ -268,29 +293,21 @@ extern "C" gptq_status gptq_hessian_accumulate(const void* X, int64_t T, int64_t
                 (long long)T, (long long)n);
   if (T == 0) return GPTQ_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool tma_ok = (n % 8 == 0) && (reinterpret_cast<uintptr_t>(X) % 16 == 0);
+  const bool tma_ok = (n % 8 == 0) && (reinterpret_cast<uintptr_t>(X) % 16 == 0) &&
+                      (reinterpret_cast<uintptr_t>(H) % 16 == 0);
   if (tma_ok) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
-    if (enc == nullptr) return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    CUtensorMap tm;
-    cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)T};
-    cuuint64_t strides[1] = {(cuuint64_t)n * 2};
-    cuuint32_t box[2] = {64, TC_KT};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
-      return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    CUtensorMap tm, th;
+    if (!encode_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, n, T, n * 2, 64, TC_KT) ||
+        !encode_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, H, n, n, n * 4, 32, TC_TILE))
+      return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the Hessian");
     if (!g_tc_attr) {
       GPTQ_CUDA(cudaFuncSetAttribute(hessian_tc_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM));
       g_tc_attr = true;
     }
     const int nt = (int)ceil_div(n, TC_TILE);
-    GPTQ_LAUNCH(KK_HESSIAN, s, hessian_tc_kernel, nt * (nt + 1) / 2, 128, TC_SMEM, tm, T, n,
-                nt, H, info);
+    GPTQ_LAUNCH(KK_HESSIAN, s, hessian_tc_kernel, nt * (nt + 1) / 2, 128, TC_SMEM, tm, th, T, n,
+                nt, info);
     return GPTQ_OK;
   }
   const int nt = (int)ceil_div(n, HT);

@@ -171,6 +171,18 @@ prep_gather_kernel(const float* __restrict__ H, int64_t n, int64_t np,
   A[e] = v;
 }
 
+// Diagonal tile: L_kk = chol(A_kk) and D = L_kk⁻¹, blocked by panels of 8
+// columns so that the 64 dependent pivots cost 16 barriers instead of 64:
+//   phase 1 (warp 0): factor the 8-column panel in registers (lane l owns rows
+//            l and l + 32), pivots and multipliers exchanged by shuffles, and
+//            finish the panel's 8 rows of D by forward substitution (lanes
+//            over columns);
+//   phase 2 (8 warps): rank-8 update of the trailing block of A and of the
+//            rows of D below the panel.
+// Pivots use rsqrt_pivot (Newton steps from the float32 estimate).
+constexpr int DIAG_THREADS = 256;
+constexpr int PW = 8;                         // panel width
+
 // 1/sqrt(d) for a pivot d > 0 by Newton–Raphson on f(y) = y⁻² − d,
 // y ← y·(3 − d·y²)/2, started from the float32 reciprocal-square-root estimate
 // (≈ 2⁻²² relative); quadratic convergence gives float64 precision after two
@@ -185,155 +197,116 @@ __device__ __forceinline__ double rsqrt_pivot(double d) {
   return y;
 }
 
-constexpr unsigned kFull = 0xffffffffu;
-
-// Cholesky of a 32×32 SPD block held by one warp, lane l owning row l in
-// r[0..31] (entries right of the diagonal are ignored).  On return r is row l
-// of L, ys[c] = 1/L_cc (the same in every lane), `bad` flags a pivot that is
-// not positive and finite.  Multipliers travel by shuffles; no barrier.
-__device__ __forceinline__ void chol32_regs(double (&r)[32], double (&ys)[32], int lane,
-                                            bool& bad) {
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    const double d = __shfl_sync(kFull, r[c], c);
-    if (!(d > 0.0) || !isfinite(d)) bad = true;
-    const double y = (d > 0.0) ? rsqrt_pivot(d) : 0.0;
-    ys[c] = y;
-    if (lane > c) r[c] *= y;
-    else if (lane == c) r[c] = d * y;
-#pragma unroll
-    for (int k = c + 1; k < 32; ++k) {
-      const double lk = __shfl_sync(kFull, r[c], k);   // L[k][c], lane k
-      if (lane >= k) r[k] = fma(-r[c], lk, r[k]);
-    }
-  }
-}
-
-// Column `lane` of L⁻¹ for the 32×32 lower factor held as in chol32_regs:
-// forward substitution x_i = (δ_i,lane − Σ_{k<i} L_ik x_k)·(1/L_ii), the row
-// L_i· broadcast from lane i.
-__device__ __forceinline__ void inv32_regs(const double (&r)[32], const double (&ys)[32],
-                                           int lane, double (&x)[32]) {
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    double acc0 = (i == lane) ? 1.0 : 0.0, acc1 = 0.0;
-#pragma unroll
-    for (int k = 0; k < i; ++k) {
-      const double lik = __shfl_sync(kFull, r[k], i);
-      if (k & 1) acc1 = fma(-lik, x[k], acc1);
-      else acc0 = fma(-lik, x[k], acc0);
-    }
-    x[i] = (acc0 + acc1) * ys[i];
-  }
-}
-
-// Diagonal tile: L_kk = chol(A_kk) and D = L_kk⁻¹ by a 2×2 block recursion on
-// 32-column halves:
-//   warp 0: L11 = chol(A11), L11⁻¹            (registers)
-//   all:    L21 = A21·L11⁻ᵀ;  A22 −= L21·L21ᵀ
-//   warp 0: L22 = chol(A22), L22⁻¹            (registers)
-//   all:    (L⁻¹)21 = −L22⁻¹·(L21·L11⁻¹)
-// The dependent pivot chain runs inside one warp with shuffles; the block
-// products are spread over all 8 warps.
-constexpr int DIAG_THREADS = 256;
-constexpr int LDH = 33;                      // 32-column halves in shared memory
-constexpr size_t DIAG_SMEM = sizeof(double) * (2 * NB * LDT + 2 * 32 * LDH);
-
 __global__ void __launch_bounds__(DIAG_THREADS)
 chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
                  double* __restrict__ D, int64_t n, int64_t np, int k,
                  int32_t* info) {
   if (info[0] != 0) return;
   extern __shared__ double sm[];
-  double (*a)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);             // A, then L
-  double (*b)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);  // L⁻¹
-  double (*t21)[LDH] = reinterpret_cast<double (*)[LDH]>(sm + 2 * NB * LDT);
-  double (*t2)[LDH] = reinterpret_cast<double (*)[LDH]>(sm + 2 * NB * LDT + 32 * LDH);
+  double (*a)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);
+  double (*b)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);
   __shared__ int bad_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t base = (int64_t)k * NB;
   for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
     const int r = e / NB, c = e % NB;
     a[r][c] = (c <= r) ? A[(base + r) * np + base + c] : 0.0;
-    b[r][c] = 0.0;
+    b[r][c] = (r == c) ? 1.0 : 0.0;
   }
   if (tid == 0) bad_s = 0;
   __syncthreads();
 
-  // ---- L11, L11⁻¹
-  if (warp == 0) {
-    double r[32], ys[32], x[32];
-    bool bad = false;
+  for (int c0 = 0; c0 < NB; c0 += PW) {
+    if (warp == 0) {
+      // ---- phase 1: the panel, rows c0..63, columns c0..c0+7
+      double v0[PW], v1[PW];                 // rows lane and lane + 32
 #pragma unroll
-    for (int c = 0; c < 32; ++c) r[c] = a[lane][c];
-    chol32_regs(r, ys, lane, bad);
-    if (bad && lane == 0) {
-      bad_s = 1;
-      report(info, GPTQ_ERR_NOT_PD, n - 1 - base);
+      for (int c = 0; c < PW; ++c) {
+        v0[c] = a[lane][c0 + c];
+        v1[c] = a[lane + 32][c0 + c];
+      }
+      double ys[PW];
+      bool bad = false;
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        const int pr = c0 + c;
+        const double mine = (pr < 32) ? v0[c] : v1[c];
+        const double d = __shfl_sync(0xffffffffu, mine, pr & 31);
+        if (!(d > 0.0) || !isfinite(d)) bad = true;
+        const double y = (d > 0.0) ? rsqrt_pivot(d) : 0.0;
+        ys[c] = y;
+        // scale column c below the pivot; the pivot becomes sqrt(d)
+        if (lane > pr) v0[c] *= y;
+        else if (lane == pr) v0[c] = d * y;
+        if (lane + 32 > pr) v1[c] *= y;
+        else if (lane + 32 == pr) v1[c] = d * y;
+        // update the panel's later columns
+#pragma unroll
+        for (int cc = c + 1; cc < PW; ++cc) {
+          const int rr = c0 + cc;                     // row whose multiplier we need
+          const double own = (rr < 32) ? v0[c] : v1[c];
+          const double lk = __shfl_sync(0xffffffffu, own, rr & 31);
+          if (lane >= rr) v0[cc] -= v0[c] * lk;
+          if (lane + 32 >= rr) v1[cc] -= v1[c] * lk;
+        }
+      }
+      if (bad) {
+        if (lane == 0) {
+          bad_s = 1;
+          report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + c0));
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        if (lane >= c0) a[lane][c0 + c] = v0[c];
+        if (lane + 32 >= c0) a[lane + 32][c0 + c] = v1[c];
+      }
+      __syncwarp();
+      // panel rows of D: forward substitution over the panel, lanes over x
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        const int pr = c0 + c;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int x = lane + 32 * h;
+          if (x <= pr) {
+            double acc = b[pr][x];
+#pragma unroll
+            for (int cp = 0; cp < c; ++cp) acc -= a[pr][c0 + cp] * b[c0 + cp][x];
+            b[pr][x] = acc * ys[c];
+          }
+        }
+        __syncwarp();
+      }
     }
+    __syncthreads();
+    if (bad_s) return;
+    // ---- phase 2: rank-8 update of rows below the panel
+    const int rs = c0 + PW;
+    for (int r = rs + warp; r < NB; r += DIAG_THREADS / 32) {
+      double lr[PW];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) a[lane][c] = (c <= lane) ? r[c] : 0.0;
-    inv32_regs(r, ys, lane, x);
+      for (int c = 0; c < PW; ++c) lr[c] = a[r][c0 + c];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) b[i][lane] = x[i];
-  }
-  __syncthreads();
-  if (bad_s) return;
-  // ---- L21 = A21·L11⁻ᵀ: L21[i][j] = Σ_{q ≤ j} A21[i][q]·L11⁻¹[j][q]
-  for (int e = tid; e < 32 * 32; e += DIAG_THREADS) {
-    const int i = e >> 5, j = e & 31;
-    double acc = 0.0;
-    for (int q = 0; q <= j; ++q) acc = fma(a[32 + i][q], b[j][q], acc);
-    t21[i][j] = acc;
-  }
-  __syncthreads();
-  // ---- A22 −= L21·L21ᵀ (lower part)
-  for (int e = tid; e < 32 * 32; e += DIAG_THREADS) {
-    const int i = e >> 5, j = e & 31;
-    if (j <= i) {
-      double acc = a[32 + i][32 + j];
-#pragma unroll 8
-      for (int q = 0; q < 32; ++q) acc = fma(-t21[i][q], t21[j][q], acc);
-      a[32 + i][32 + j] = acc;
+      for (int h = 0; h < 2; ++h) {
+        const int x = lane + 32 * h;
+        if (x >= rs) {
+          if (x <= r) {
+            double acc = a[r][x];
+#pragma unroll
+            for (int c = 0; c < PW; ++c) acc -= lr[c] * a[x][c0 + c];
+            a[r][x] = acc;
+          }
+        } else {
+          double acc = b[r][x];
+#pragma unroll
+          for (int c = 0; c < PW; ++c) acc -= lr[c] * b[c0 + c][x];
+          b[r][x] = acc;
+        }
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
-  // ---- L22, L22⁻¹
-  if (warp == 0) {
-    double r[32], ys[32], x[32];
-    bool bad = false;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) r[c] = a[32 + lane][32 + c];
-    chol32_regs(r, ys, lane, bad);
-    if (bad && lane == 0) {
-      bad_s = 1;
-      report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + 32));
-    }
-#pragma unroll
-    for (int c = 0; c < 32; ++c) a[32 + lane][32 + c] = (c <= lane) ? r[c] : 0.0;
-    inv32_regs(r, ys, lane, x);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) b[32 + i][32 + lane] = x[i];
-  }
-  __syncthreads();
-  if (bad_s) return;
-  // ---- T = L21·L11⁻¹ (T[i][j] = Σ_{q ≥ j} L21[i][q]·L11⁻¹[q][j]), L21 into A
-  for (int e = tid; e < 32 * 32; e += DIAG_THREADS) {
-    const int i = e >> 5, j = e & 31;
-    double acc = 0.0;
-    for (int q = j; q < 32; ++q) acc = fma(t21[i][q], b[q][j], acc);
-    t2[i][j] = acc;
-    a[32 + i][j] = t21[i][j];
-  }
-  __syncthreads();
-  // ---- (L⁻¹)21 = −L22⁻¹·T
-  for (int e = tid; e < 32 * 32; e += DIAG_THREADS) {
-    const int i = e >> 5, j = e & 31;
-    double acc = 0.0;
-    for (int q = 0; q <= i; ++q) acc = fma(b[32 + i][32 + q], t2[q][j], acc);
-    b[32 + i][j] = -acc;
-  }
-  __syncthreads();
 
   for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
     const int r = e / NB, c = e % NB;
@@ -534,7 +507,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   const size_t tile_smem = 2 * NB * LDM * sizeof(double);   // ≥ the diagonal kernel's 2·NB·LDT
   if (!g_smem_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(chol_diag_kernel,
-              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DIAG_SMEM));
+              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
     GPTQ_CUDA(cudaFuncSetAttribute(chol_panel_kernel,
               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
     GPTQ_CUDA(cudaFuncSetAttribute(chol_trail_kernel,
@@ -552,7 +525,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);
   for (int k = 0; k < N; ++k) {
-    GPTQ_LAUNCH(KK_CHOL_DIAG, s, chol_diag_kernel, 1, DIAG_THREADS, DIAG_SMEM, w.A, w.M, w.D, n, np, k, info);
+    GPTQ_LAUNCH(KK_CHOL_DIAG, s, chol_diag_kernel, 1, DIAG_THREADS, tile_smem, w.A, w.M, w.D, n, np, k, info);
     const int r = N - k - 1;
     if (r + k > 0)
       GPTQ_LAUNCH(KK_CHOL_PANEL, s, chol_panel_kernel, r + k, 256, tile_smem,
