@@ -155,7 +155,8 @@ def kernel_work(probs, block: int):
     """Algorithmic work per kernel kind for one step: {kind: (unit, amount)}.
 
     hessian   flops T·n·(n+1)               (upper triangle incl. diagonal)
-    chol_*    flops of the executed float64 tile products (Σ_k tiles·2·64³)
+    cholesky  flops of the executed float64 tile products (Σ_k tiles·2·64³)
+              plus the diagonal tiles' Cholesky and inverse (2·64³/3 each)
     sweep     bytes: strip read + Err write (4+4 B) + codes (1 B) per element,
               U panel 4·bw², scale+zero 5 B per (row, group)
     trailing  bytes: W read+write 8 B per trailing element, Err 4·m·bw,
@@ -163,17 +164,15 @@ def kernel_work(probs, block: int):
     pack      bytes: codes 1 B + packed bits/8 B per element, scale/zero
     ingest    bytes: W in (2 or 4 B) + float32 out per element
     """
-    w = {k: 0.0 for k in ("hessian", "chol_diag", "chol_trail", "chol_panel", "sweep",
-                          "trailing", "pack", "ingest")}
+    w = {k: 0.0 for k in ("hessian", "cholesky", "sweep", "trailing", "pack", "ingest")}
     for p in probs:
         m, n, T = p.m, p.n, p.T
         w["hessian"] += T * n * (n + 1)
         N = -(-n // 64)
         for k in range(N):
             r = N - k - 1
-            w["chol_trail"] += (r * (r + 1) // 2 + r * (k + 1)) * 2 * 64 ** 3
-            w["chol_panel"] += (r + k) * 2 * 64 ** 3
-            w["chol_diag"] += 2 * 64 ** 3 / 3        # Cholesky + inverse of a tile
+            w["cholesky"] += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
+            w["cholesky"] += 2 * 64 ** 3 / 3         # Cholesky + inverse of a tile
         ng = -(-n // p.group)
         for j0 in range(0, n, block):
             bw = min(block, n - j0)
@@ -183,8 +182,7 @@ def kernel_work(probs, block: int):
                 w["trailing"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
         w["pack"] += m * n + m * n * p.bits / 8 + 5 * m * ng
         w["ingest"] += m * n * (p.W.element_size() + 4)
-    units = {"hessian": "TFLOP/s", "chol_diag": "TFLOP/s", "chol_trail": "TFLOP/s",
-             "chol_panel": "TFLOP/s",
+    units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s",
              "sweep": "GB/s", "trailing": "GB/s", "pack": "GB/s", "ingest": "GB/s"}
     return {k: (units[k], v) for k, v in w.items()}
 

@@ -16,9 +16,7 @@ enum KernelKind : int {
   KK_PREP_STATS,      // mean(diag H), dead columns, order keys
   KK_PREP_ORDER,      // processing permutation
   KK_PREP_GATHER,     // reversed, permuted, damped float64 copy of H
-  KK_CHOL_DIAG,       // diagonal block: Cholesky + triangular inverse
-  KK_CHOL_PANEL,      // panel solve and finished rows of L⁻¹
-  KK_CHOL_TRAIL,      // trailing update of A and of the L⁻¹ accumulator
+  KK_CHOL,            // blocked Cholesky + triangular inverse (one dataflow launch)
   KK_PREP_OUT,        // U = reversed L⁻¹, rounded to float32
   KK_INGEST,          // W → float32 working copy in processing order
   KK_SWEEP,           // one block of the column sweep

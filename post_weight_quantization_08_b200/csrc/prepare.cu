@@ -33,11 +33,16 @@ struct PrepWs {
   int32_t* seen;  // n (custom-order check)
   double* A;      // np × np
   double* M;      // np × np
-  double* D;      // NB × NB (L_kk⁻¹ of the current step)
+  double* D;      // N × NB × NB: L_kk⁻¹ of every diagonal tile
+  int* sync;      // flags and counters of the dataflow factorisation
+  size_t sync_bytes;
 };
+
+inline size_t sync_ints(int64_t N) { return 4 + (size_t)N + 4 * (size_t)N * (size_t)N; }
 
 size_t prep_ws_layout(int64_t n, PrepWs* w, char* base) {
   const int64_t np = ceil_div(n, NB) * NB;
+  const int64_t N = np / NB;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -48,13 +53,16 @@ size_t prep_ws_layout(int64_t n, PrepWs* w, char* base) {
   size_t o_seen = take(sizeof(int32_t) * (size_t)n);
   size_t o_A = take(sizeof(double) * (size_t)np * (size_t)np);
   size_t o_M = take(sizeof(double) * (size_t)np * (size_t)np);
-  size_t o_D = take(sizeof(double) * NB * NB);
+  size_t o_D = take(sizeof(double) * NB * NB * (size_t)N);
+  size_t o_S = take(sizeof(int) * sync_ints(N));
   if (w && base) {
     w->mean = reinterpret_cast<double*>(base + o_mean);
     w->seen = reinterpret_cast<int32_t*>(base + o_seen);
     w->A = reinterpret_cast<double*>(base + o_A);
     w->M = reinterpret_cast<double*>(base + o_M);
     w->D = reinterpret_cast<double*>(base + o_D);
+    w->sync = reinterpret_cast<int*>(base + o_S);
+    w->sync_bytes = sizeof(int) * sync_ints(N);
   }
   return off;
 }
@@ -197,12 +205,11 @@ __device__ __forceinline__ double rsqrt_pivot(double d) {
   return y;
 }
 
-__global__ void __launch_bounds__(DIAG_THREADS)
-chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
-                 double* __restrict__ D, int64_t n, int64_t np, int k,
-                 int32_t* info) {
-  if (info[0] != 0) return;
-  extern __shared__ double sm[];
+// Returns false (after reporting through info) when a pivot is not positive.
+// Called by a whole CTA of DIAG_THREADS threads; sm holds 2·NB·LDT doubles.
+__device__ bool diag_tile(double* __restrict__ A, double* __restrict__ M,
+                          double* __restrict__ D, int64_t n, int64_t np, int k,
+                          int32_t* info, double* sm) {
   double (*a)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);
   double (*b)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);
   __shared__ int bad_s;
@@ -210,7 +217,7 @@ chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
   const int64_t base = (int64_t)k * NB;
   for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
     const int r = e / NB, c = e % NB;
-    a[r][c] = (c <= r) ? A[(base + r) * np + base + c] : 0.0;
+    a[r][c] = (c <= r) ? __ldcg(A + (base + r) * np + base + c) : 0.0;
     b[r][c] = (r == c) ? 1.0 : 0.0;
   }
   if (tid == 0) bad_s = 0;
@@ -280,7 +287,7 @@ chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
       }
     }
     __syncthreads();
-    if (bad_s) return;
+    if (bad_s) return false;
     // ---- phase 2: rank-8 update of rows below the panel
     const int rs = c0 + PW;
     for (int r = rs + warp; r < NB; r += DIAG_THREADS / 32) {
@@ -314,6 +321,7 @@ chol_diag_kernel(double* __restrict__ A, double* __restrict__ M,
     M[(base + r) * np + base + c] = b[r][c];
     D[e] = b[r][c];
   }
+  return true;
 }
 
 // 64×64 float64 tile products on the float64 tensor cores (DMMA,
@@ -360,7 +368,7 @@ __device__ __forceinline__ void tile_store(double* out, int64_t ld, const double
       double2* p = reinterpret_cast<double2*>(out + (int64_t)(rb + 8 * i + g) * ld + cb + 8 * j + 2 * t);
       double2 v;
       if (SUBTRACT) {
-        v = *p;
+        v = __ldcg(p);
         v.x -= acc[i][j][0];
         v.y -= acc[i][j][1];
       } else {
@@ -371,7 +379,8 @@ __device__ __forceinline__ void tile_store(double* out, int64_t ld, const double
 }
 
 // 64×64 float64 tile from global (leading dimension ld) into shared memory,
-// optionally transposed; 16-byte loads, all issued before the stores.
+// optionally transposed; 16-byte loads (L2 only: tiles are rewritten by other
+// CTAs of the same launch), all issued before the stores.
 __device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
                                           int64_t ld, bool transpose, int tid) {
   double2 buf[8];
@@ -379,7 +388,7 @@ __device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
   for (int k = 0; k < 8; ++k) {
     const int e = tid + 256 * k;            // 2048 pairs
     const int r = e >> 5, c2 = (e & 31) * 2;
-    buf[k] = *reinterpret_cast<const double2*>(src + (int64_t)r * ld + c2);
+    buf[k] = __ldcg(reinterpret_cast<const double2*>(src + (int64_t)r * ld + c2));
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -395,68 +404,212 @@ __device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
   }
 }
 
-// panel(k): blocks [0, N−k−1): L_ik = A_ik·Dᵀ; blocks [N−k−1, N−1): M_kc = D·M_kc.
-__global__ void __launch_bounds__(256)
-chol_panel_kernel(double* __restrict__ A, double* __restrict__ M,
-                  const double* __restrict__ D, int64_t np, int N, int k,
-                  int32_t* info) {
-  if (info[0] != 0) return;
-  extern __shared__ double sm[];
-  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
-  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nlow = N - k - 1;
-  double* out;
-  if ((int)blockIdx.x < nlow) {
-    const int i = k + 1 + blockIdx.x;
-    out = A + (int64_t)i * NB * np + (int64_t)k * NB;
-    load_tile(x, out, np, false, tid);
-    load_tile(y, D, NB, true, tid);
-  } else {
-    const int c = blockIdx.x - nlow;
-    out = M + (int64_t)k * NB * np + (int64_t)c * NB;
-    load_tile(x, D, NB, false, tid);
-    load_tile(y, out, np, false, tid);
-  }
-  __syncthreads();
-  double acc[2][4][2] = {};
-  tile_mm(x, y, acc, warp, lane);
-  tile_store<false>(out, np, acc, warp, lane);
+// ---------------------------------------------------------------------------
+// The factorisation as one persistent, dataflow launch.
+//
+// Tasks of step k (64-column block k), in the fixed global order in which the
+// workers take them (critical ones first, so step k+1 can start while step k
+// is still updating far tiles):
+//   PANEL(k,k+1), TRAIL(k,k+1,k+1), PANEL(k,i) i > k+1, TRAIL(k,i,k+1),
+//   MROW(k,c) c < k, MTRAIL(k,k+1,c), TRAIL(k,i,j) k+1 < j ≤ i, MTRAIL(k,i,c)
+// with PANEL:  L_ik = A_ik·D_kᵀ          (needs D_k and tile (i,k) updated k times)
+//      MROW:   M_kc = D_k·M_kc           (needs D_k and M_kc updated k−c times)
+//      TRAIL:  A_ij −= L_ik·L_jkᵀ         (needs L_ik, L_jk, tile (i,j) updated k times)
+//      MTRAIL: M_ic −= L_ik·M_kc          (needs L_ik, final M_kc, M_ic updated k−c times)
+// and DIAG(k) — L_kk = chol(A_kk), D_k = L_kk⁻¹ — run by the first CTA to
+// arrive (its instruction cache stays warm across the chain of diagonal
+// tiles) once tile (k,k) has received its k updates.  Every dependency of a
+// task is an earlier task, and tasks are taken in order only by running
+// CTAs, so the launch needs no co-residency guarantee.  Flags are set with
+// release stores after a fence and polled with acquire loads; every wait is
+// bounded and a time-out (or a bad pivot) raises a shared abort flag.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kSpinLimit = 1u << 22;   // ≈ a few seconds with the back-off below
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// trail(k): first r(r+1)/2 blocks are (i, j), k < j ≤ i: A_ij −= L_ik·L_jkᵀ;
-// the next r·(k+1) are (i, c), i > k, c ≤ k: M_ic −= L_ik·M_kc.
-__global__ void __launch_bounds__(256)
-chol_trail_kernel(double* __restrict__ A, double* __restrict__ M, int64_t np,
-                  int N, int k, int32_t* info) {
-  if (info[0] != 0) return;
-  extern __shared__ double sm[];
-  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
-  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r = N - k - 1;
-  const int ntri = r * (r + 1) / 2;
-  int lin = blockIdx.x;
-  double* out;
-  if (lin < ntri) {
-    // decode (ii, jj) with 0 <= jj <= ii < r
-    int ii = 0;
-    while (lin >= ii + 1) { lin -= ii + 1; ++ii; }
-    const int i = k + 1 + ii, j = k + 1 + lin;
-    out = A + (int64_t)i * NB * np + (int64_t)j * NB;
-    load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
-    load_tile(y, A + (int64_t)j * NB * np + (int64_t)k * NB, np, true, tid);
-  } else {
-    lin -= ntri;
-    const int i = k + 1 + lin / (k + 1), c = lin % (k + 1);
-    out = M + (int64_t)i * NB * np + (int64_t)c * NB;
-    load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
-    load_tile(y, M + (int64_t)k * NB * np + (int64_t)c * NB, np, false, tid);
+struct CholSync {
+  int* ctrl;        // [0] next task, [1] arrivals, [2] abort
+  int* diag_done;   // N
+  int* pdone;       // N·N: pdone[k·N + i], L_ik final
+  int* mdone;       // N·N: mdone[k·N + c], M_kc final
+  int* upd;         // N·N: updates applied to A tile (i, j)
+  int* mupd;        // N·N: updates applied to M tile (i, c)
+};
+
+__device__ CholSync sync_view(int* base, int N) {
+  CholSync s;
+  s.ctrl = base;
+  s.diag_done = base + 4;
+  s.pdone = s.diag_done + N;
+  s.mdone = s.pdone + N * N;
+  s.upd = s.mdone + N * N;
+  s.mupd = s.upd + N * N;
+  return s;
+}
+
+// Whole-CTA bounded wait for *flag ≥ target; false on abort or time-out.
+__device__ bool cta_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok) {
+  if (threadIdx.x == 0) {
+    bool ok = false;
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+      if (ld_acquire(flag) >= target) { ok = true; break; }
+      if (*reinterpret_cast<volatile int*>(abortp)) break;
+      if (it > 32) __nanosleep(64);
+    }
+    if (!ok && !*reinterpret_cast<volatile int*>(abortp)) {
+      report(info, GPTQ_ERR_TIMEOUT, target);
+      atomicExch(abortp, 1);
+    }
+    *s_ok = ok ? 1 : 0;
   }
   __syncthreads();
-  double acc[2][4][2] = {};
-  tile_mm(x, y, acc, warp, lane);
-  tile_store<true>(out, np, acc, warp, lane);
+  const bool ok = *s_ok != 0;
+  __syncthreads();
+  return ok;
+}
+
+__device__ __forceinline__ void cta_signal(int* flag, int value) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    st_release(flag, value);
+  }
+}
+
+__host__ __device__ inline int step_tasks(int N, int k) {
+  const int r = N - k - 1;
+  if (r <= 0) return k;                              // MROW only
+  return 2 + 2 * (r - 1) + k + (k + 1) + (r - 1) * r / 2 + (r - 1) * (k + 1);
+}
+
+int total_tasks(int N) {
+  int t = 0;
+  for (int k = 0; k < N; ++k) t += step_tasks(N, k);
+  return t;
+}
+
+enum TaskKind { T_PANEL = 0, T_MROW, T_TRAIL, T_MTRAIL };
+
+__device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) {
+  k = 0;
+  while (task >= step_tasks(N, k)) { task -= step_tasks(N, k); ++k; }
+  const int r = N - k - 1;
+  if (r <= 0) { kind = T_MROW; i = k; j = task; return; }
+  if (task < 1) { kind = T_PANEL; i = k + 1; j = k; return; }
+  task -= 1;
+  if (task < 1) { kind = T_TRAIL; i = k + 1; j = k + 1; return; }
+  task -= 1;
+  if (task < r - 1) { kind = T_PANEL; i = k + 2 + task; j = k; return; }
+  task -= r - 1;
+  if (task < r - 1) { kind = T_TRAIL; i = k + 2 + task; j = k + 1; return; }
+  task -= r - 1;
+  if (task < k) { kind = T_MROW; i = k; j = task; return; }
+  task -= k;
+  if (task < k + 1) { kind = T_MTRAIL; i = k + 1; j = task; return; }
+  task -= k + 1;
+  if (task < (r - 1) * r / 2) {
+    int ii = 0;
+    while (task >= ii + 1) { task -= ii + 1; ++ii; }
+    kind = T_TRAIL; i = k + 2 + ii; j = k + 2 + task; return;
+  }
+  task -= (r - 1) * r / 2;
+  kind = T_MTRAIL; i = k + 2 + task / (k + 1); j = task % (k + 1);
+}
+
+__global__ void __launch_bounds__(256)
+chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
+                       double* __restrict__ Dall, int64_t n, int64_t np, int N,
+                       int ntasks, int* sync_base, int32_t* info) {
+  extern __shared__ double sm[];
+  __shared__ int s_role, s_task, s_ok;
+  const CholSync S = sync_view(sync_base, N);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) s_role = atomicAdd(&S.ctrl[1], 1);
+  __syncthreads();
+  if (*reinterpret_cast<volatile int32_t*>(info) != 0) return;
+
+  if (s_role == 0) {
+    // ---- the chain of diagonal tiles
+    for (int k = 0; k < N; ++k) {
+      if (!cta_wait(&S.upd[k * N + k], k, &S.ctrl[2], info, &s_ok)) return;
+      if (!diag_tile(A, M, Dall + (size_t)k * NB * NB, n, np, k, info, sm)) {
+        if (tid == 0) atomicExch(&S.ctrl[2], 1);
+        return;
+      }
+      cta_signal(&S.diag_done[k], 1);
+    }
+    return;
+  }
+
+  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
+  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
+  for (;;) {
+    if (tid == 0) s_task = atomicAdd(&S.ctrl[0], 1);
+    __syncthreads();
+    const int task = s_task;
+    __syncthreads();
+    if (task >= ntasks || *reinterpret_cast<volatile int*>(&S.ctrl[2])) return;
+    int kind, k, i, j;
+    decode_task(task, N, kind, k, i, j);
+    double acc[2][4][2] = {};
+    if (kind == T_PANEL) {
+      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.upd[i * N + k], k, &S.ctrl[2], info, &s_ok)) return;
+      double* out = A + (int64_t)i * NB * np + (int64_t)k * NB;
+      load_tile(x, out, np, false, tid);
+      load_tile(y, Dall + (size_t)k * NB * NB, NB, true, tid);
+      __syncthreads();
+      tile_mm(x, y, acc, warp, lane);
+      tile_store<false>(out, np, acc, warp, lane);
+      cta_signal(&S.pdone[k * N + i], 1);
+    } else if (kind == T_MROW) {
+      const int c = j;
+      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.mupd[k * N + c], k - c, &S.ctrl[2], info, &s_ok)) return;
+      double* out = M + (int64_t)k * NB * np + (int64_t)c * NB;
+      load_tile(x, Dall + (size_t)k * NB * NB, NB, false, tid);
+      load_tile(y, out, np, false, tid);
+      __syncthreads();
+      tile_mm(x, y, acc, warp, lane);
+      tile_store<false>(out, np, acc, warp, lane);
+      cta_signal(&S.mdone[k * N + c], 1);
+    } else if (kind == T_TRAIL) {
+      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok)) return;
+      if (j != i && !cta_wait(&S.pdone[k * N + j], 1, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.upd[i * N + j], k, &S.ctrl[2], info, &s_ok)) return;
+      double* out = A + (int64_t)i * NB * np + (int64_t)j * NB;
+      load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
+      load_tile(y, A + (int64_t)j * NB * np + (int64_t)k * NB, np, true, tid);
+      __syncthreads();
+      tile_mm(x, y, acc, warp, lane);
+      tile_store<true>(out, np, acc, warp, lane);
+      cta_signal(&S.upd[i * N + j], k + 1);
+    } else {   // T_MTRAIL
+      const int c = j;
+      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok)) return;
+      if (c < k) {
+        if (!cta_wait(&S.mdone[k * N + c], 1, &S.ctrl[2], info, &s_ok)) return;
+      } else if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) {
+        return;
+      }
+      if (!cta_wait(&S.mupd[i * N + c], k - c, &S.ctrl[2], info, &s_ok)) return;
+      double* out = M + (int64_t)i * NB * np + (int64_t)c * NB;
+      load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
+      load_tile(y, M + (int64_t)k * NB * np + (int64_t)c * NB, np, false, tid);
+      __syncthreads();
+      tile_mm(x, y, acc, warp, lane);
+      tile_store<true>(out, np, acc, warp, lane);
+      cta_signal(&S.mupd[i * N + c], k - c + 1);
+    }
+  }
 }
 
 // U[i][j] = L⁻¹[n−1−i][n−1−j] for j ≥ i, 0 below the diagonal.
@@ -470,6 +623,7 @@ prep_out_kernel(const double* __restrict__ M, int64_t n, int64_t np,
 }
 
 bool g_smem_set = false;
+int g_num_sms = 148;
 
 }  // namespace
 }  // namespace gptq
@@ -504,18 +658,18 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  const size_t tile_smem = 2 * NB * LDM * sizeof(double);   // ≥ the diagonal kernel's 2·NB·LDT
+  const size_t tile_smem = 2 * NB * LDM * sizeof(double);   // ≥ the diagonal tile's 2·NB·LDT
   if (!g_smem_set) {
-    GPTQ_CUDA(cudaFuncSetAttribute(chol_diag_kernel,
+    GPTQ_CUDA(cudaFuncSetAttribute(chol_persistent_kernel,
               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
-    GPTQ_CUDA(cudaFuncSetAttribute(chol_panel_kernel,
-              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
-    GPTQ_CUDA(cudaFuncSetAttribute(chol_trail_kernel,
-              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
+    int dev = 0;
+    GPTQ_CUDA(cudaGetDevice(&dev));
+    GPTQ_CUDA(cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev));
     g_smem_set = true;
   }
 
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
+  GPTQ_CUDA(cudaMemsetAsync(w.sync, 0, w.sync_bytes, s));
   if (order == GPTQ_ORDER_CUSTOM)
     GPTQ_CUDA(cudaMemsetAsync(w.seen, 0, sizeof(int32_t) * n, s));
   GPTQ_LAUNCH(KK_PREP_STATS, s, prep_stats_kernel, 1, 1024, 0, H, n, dead, w.mean, info);
@@ -524,17 +678,10 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   GPTQ_LAUNCH(KK_PREP_GATHER, s, prep_gather_kernel, (unsigned)ceil_div(np * np, 256),
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);
-  for (int k = 0; k < N; ++k) {
-    GPTQ_LAUNCH(KK_CHOL_DIAG, s, chol_diag_kernel, 1, DIAG_THREADS, tile_smem, w.A, w.M, w.D, n, np, k, info);
-    const int r = N - k - 1;
-    if (r + k > 0)
-      GPTQ_LAUNCH(KK_CHOL_PANEL, s, chol_panel_kernel, r + k, 256, tile_smem,
-                  w.A, w.M, w.D, np, N, k, info);
-    const int tiles = r * (r + 1) / 2 + r * (k + 1);
-    if (tiles > 0)
-      GPTQ_LAUNCH(KK_CHOL_TRAIL, s, chol_trail_kernel, tiles, 256, tile_smem,
-                  w.A, w.M, np, N, k, info);
-  }
+  const int ntasks = total_tasks(N);
+  const int grid = (ntasks + 1 < 2 * g_num_sms) ? ntasks + 1 : 2 * g_num_sms;
+  GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, w.D, n, np,
+              N, ntasks, w.sync, info);
   GPTQ_LAUNCH(KK_PREP_OUT, s, prep_out_kernel, (unsigned)ceil_div(n * n, 256), 256, 0,
               w.M, n, np, U);
   return GPTQ_OK;
@@ -552,9 +699,12 @@ namespace {
 constexpr int64_t kNoAllocMaxN = GPTQ_NOALLOC_MAX_N;
 constexpr size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 // Same arithmetic as prep_ws_layout() for n = kNoAllocMaxN (a multiple of 64).
+constexpr int64_t kNoAllocN = kNoAllocMaxN / NB;
 constexpr size_t kNoAllocBytes =
     up256(sizeof(double)) + up256(sizeof(int32_t) * kNoAllocMaxN) +
-    2 * up256(sizeof(double) * kNoAllocMaxN * kNoAllocMaxN) + up256(sizeof(double) * NB * NB);
+    2 * up256(sizeof(double) * kNoAllocMaxN * kNoAllocMaxN) +
+    up256(sizeof(double) * NB * NB * kNoAllocN) +
+    up256(sizeof(int) * (4 + kNoAllocN + 4 * kNoAllocN * kNoAllocN));
 static_assert(kNoAllocMaxN % NB == 0, "the fixed limit is a whole number of tiles");
 
 // The scratch itself: every GPU that loads this library holds it until the

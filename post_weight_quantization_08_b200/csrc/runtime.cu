@@ -16,9 +16,8 @@ thread_local char g_last_error[512] = "";
 std::atomic<uint64_t> g_launches{0};
 
 const char* const kKindNames[KK_COUNT] = {
-    "hessian",     "prep_stats",  "prep_order", "prep_gather",
-    "chol_diag",   "chol_panel",  "chol_trail", "prep_out",
-    "ingest",      "sweep",       "trailing",   "pack"};
+    "hessian",  "prep_stats", "prep_order", "prep_gather", "cholesky",
+    "prep_out", "ingest",     "sweep",      "trailing",    "pack"};
 
 struct Profiler {
   std::mutex mu;

@@ -66,7 +66,7 @@ def test_kernel_work_accounting():
     n0, n1 = probs[0].n, probs[1].n
     assert work["hessian"][1] == T * n0 * (n0 + 1) + T * n1 * (n1 + 1)
     # float64 tile work approaches 2n³/3 from above (tiles are 64 wide)
-    tiles = work["chol_trail"][1] + work["chol_panel"][1]
+    tiles = work["cholesky"][1]
     assert 0.9 * (2 * (n0 ** 3 + n1 ** 3) / 3) < tiles < 1.6 * (2 * (n0 ** 3 + n1 ** 3) / 3)
     assert work["sweep"][0] == "GB/s"
 
