@@ -26,14 +26,12 @@ namespace gptq {
 namespace {
 
 constexpr int NB = 64;          // float64 tile edge
-constexpr int LDT = NB + 1;     // padded shared-memory row (doubles)
 
 struct PrepWs {
   double* mean;   // 1
   int32_t* seen;  // n (custom-order check)
   double* A;      // np × np
   double* M;      // np × np
-  double* D;      // N × NB × NB: L_kk⁻¹ of every diagonal tile
   int* sync;      // flags and counters of the dataflow factorisation
   size_t sync_bytes;
 };
@@ -53,14 +51,12 @@ size_t prep_ws_layout(int64_t n, PrepWs* w, char* base) {
   size_t o_seen = take(sizeof(int32_t) * (size_t)n);
   size_t o_A = take(sizeof(double) * (size_t)np * (size_t)np);
   size_t o_M = take(sizeof(double) * (size_t)np * (size_t)np);
-  size_t o_D = take(sizeof(double) * NB * NB * (size_t)N);
   size_t o_S = take(sizeof(int) * sync_ints(N));
   if (w && base) {
     w->mean = reinterpret_cast<double*>(base + o_mean);
     w->seen = reinterpret_cast<int32_t*>(base + o_seen);
     w->A = reinterpret_cast<double*>(base + o_A);
     w->M = reinterpret_cast<double*>(base + o_M);
-    w->D = reinterpret_cast<double*>(base + o_D);
     w->sync = reinterpret_cast<int*>(base + o_S);
     w->sync_bytes = sizeof(int) * sync_ints(N);
   }
@@ -179,156 +175,10 @@ prep_gather_kernel(const float* __restrict__ H, int64_t n, int64_t np,
   A[e] = v;
 }
 
-// Diagonal tile: L_kk = chol(A_kk) and D = L_kk⁻¹, blocked by panels of 8
-// columns so that the 64 dependent pivots cost 16 barriers instead of 64:
-//   phase 1 (warp 0): factor the 8-column panel in registers (lane l owns rows
-//            l and l + 32), pivots and multipliers exchanged by shuffles, and
-//            finish the panel's 8 rows of D by forward substitution (lanes
-//            over columns);
-//   phase 2 (8 warps): rank-8 update of the trailing block of A and of the
-//            rows of D below the panel.
-// Pivots use rsqrt_pivot (Newton steps from the float32 estimate).
-constexpr int DIAG_THREADS = 256;
-constexpr int PW = 8;                         // panel width
-
-// 1/sqrt(d) for a pivot d > 0 by Newton–Raphson on f(y) = y⁻² − d,
-// y ← y·(3 − d·y²)/2, started from the float32 reciprocal-square-root estimate
-// (≈ 2⁻²² relative); quadratic convergence gives float64 precision after two
-// steps.  Much shorter on the critical path than a correctly rounded float64
-// sqrt followed by a division.  Pivots outside the float32 range take the
-// exact route.
-__device__ __forceinline__ double rsqrt_pivot(double d) {
-  if (d < 1e-30 || d > 1e30) return 1.0 / sqrt(d);
-  double y = (double)rsqrtf((float)d);
-  y = y * (1.5 - 0.5 * d * y * y);
-  y = y * (1.5 - 0.5 * d * y * y);
-  return y;
-}
-
-// Returns false (after reporting through info) when a pivot is not positive.
-// Called by a whole CTA of DIAG_THREADS threads; sm holds 2·NB·LDT doubles.
-__device__ bool diag_tile(double* __restrict__ A, double* __restrict__ M,
-                          double* __restrict__ D, int64_t n, int64_t np, int k,
-                          int32_t* info, double* sm) {
-  double (*a)[LDT] = reinterpret_cast<double (*)[LDT]>(sm);
-  double (*b)[LDT] = reinterpret_cast<double (*)[LDT]>(sm + NB * LDT);
-  __shared__ int bad_s;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t base = (int64_t)k * NB;
-  for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
-    const int r = e / NB, c = e % NB;
-    a[r][c] = (c <= r) ? __ldcg(A + (base + r) * np + base + c) : 0.0;
-    b[r][c] = (r == c) ? 1.0 : 0.0;
-  }
-  if (tid == 0) bad_s = 0;
-  __syncthreads();
-
-  for (int c0 = 0; c0 < NB; c0 += PW) {
-    if (warp == 0) {
-      // ---- phase 1: the panel, rows c0..63, columns c0..c0+7
-      double v0[PW], v1[PW];                 // rows lane and lane + 32
-#pragma unroll
-      for (int c = 0; c < PW; ++c) {
-        v0[c] = a[lane][c0 + c];
-        v1[c] = a[lane + 32][c0 + c];
-      }
-      double ys[PW];
-      bool bad = false;
-#pragma unroll
-      for (int c = 0; c < PW; ++c) {
-        const int pr = c0 + c;
-        const double mine = (pr < 32) ? v0[c] : v1[c];
-        const double d = __shfl_sync(0xffffffffu, mine, pr & 31);
-        if (!(d > 0.0) || !isfinite(d)) bad = true;
-        const double y = (d > 0.0) ? rsqrt_pivot(d) : 0.0;
-        ys[c] = y;
-        // scale column c below the pivot; the pivot becomes sqrt(d)
-        if (lane > pr) v0[c] *= y;
-        else if (lane == pr) v0[c] = d * y;
-        if (lane + 32 > pr) v1[c] *= y;
-        else if (lane + 32 == pr) v1[c] = d * y;
-        // update the panel's later columns
-#pragma unroll
-        for (int cc = c + 1; cc < PW; ++cc) {
-          const int rr = c0 + cc;                     // row whose multiplier we need
-          const double own = (rr < 32) ? v0[c] : v1[c];
-          const double lk = __shfl_sync(0xffffffffu, own, rr & 31);
-          if (lane >= rr) v0[cc] -= v0[c] * lk;
-          if (lane + 32 >= rr) v1[cc] -= v1[c] * lk;
-        }
-      }
-      if (bad) {
-        if (lane == 0) {
-          bad_s = 1;
-          report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + c0));
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < PW; ++c) {
-        if (lane >= c0) a[lane][c0 + c] = v0[c];
-        if (lane + 32 >= c0) a[lane + 32][c0 + c] = v1[c];
-      }
-      __syncwarp();
-      // panel rows of D: forward substitution over the panel, lanes over x
-#pragma unroll
-      for (int c = 0; c < PW; ++c) {
-        const int pr = c0 + c;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int x = lane + 32 * h;
-          if (x <= pr) {
-            double acc = b[pr][x];
-#pragma unroll
-            for (int cp = 0; cp < c; ++cp) acc -= a[pr][c0 + cp] * b[c0 + cp][x];
-            b[pr][x] = acc * ys[c];
-          }
-        }
-        __syncwarp();
-      }
-    }
-    __syncthreads();
-    if (bad_s) return false;
-    // ---- phase 2: rank-8 update of rows below the panel
-    const int rs = c0 + PW;
-    for (int r = rs + warp; r < NB; r += DIAG_THREADS / 32) {
-      double lr[PW];
-#pragma unroll
-      for (int c = 0; c < PW; ++c) lr[c] = a[r][c0 + c];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int x = lane + 32 * h;
-        if (x >= rs) {
-          if (x <= r) {
-            double acc = a[r][x];
-#pragma unroll
-            for (int c = 0; c < PW; ++c) acc -= lr[c] * a[x][c0 + c];
-            a[r][x] = acc;
-          }
-        } else {
-          double acc = b[r][x];
-#pragma unroll
-          for (int c = 0; c < PW; ++c) acc -= lr[c] * b[c0 + c][x];
-          b[r][x] = acc;
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  for (int e = tid; e < NB * NB; e += DIAG_THREADS) {
-    const int r = e / NB, c = e % NB;
-    if (c <= r) A[(base + r) * np + base + c] = a[r][c];
-    M[(base + r) * np + base + c] = b[r][c];
-    D[e] = b[r][c];
-  }
-  return true;
-}
-
-// 64×64 float64 tile products on the float64 tensor cores (DMMA,
-// mma.sync m8n8k4).  Tiles sit in shared memory with a row stride of 68
-// doubles, which spreads the fragment reads over all banks.  Warp w owns rows
-// 16·(w/2) .. +16 and columns 32·(w%2) .. +32 of C: 2 × 4 accumulator tiles
-// of 8×8, two doubles per thread each (row g = lane/4, columns 2·(lane%4)+{0,1}).
+// Float64 tensor-core products (DMMA, mma.sync m8n8k4).  Shared-memory tiles
+// have a row stride of 68 doubles, which spreads the fragment reads of a warp
+// over all banks and keeps every row 16-byte aligned.  Fragment layout of an
+// 8×8×4 product: lane = 4·g + t holds A[g][t], B[t][g] and C[g][2t], C[g][2t+1].
 constexpr int LDM = 68;
 
 __device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
@@ -336,6 +186,311 @@ __device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
                : "+d"(d[0]), "+d"(d[1])
                : "d"(a), "d"(b));
 }
+
+// Lower-triangle block pairs (I, J), J ≤ I, in the order e = I·(I+1)/2 + J.
+__constant__ unsigned char kTriI[28] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3, 4, 4, 4, 4,
+                                        4, 5, 5, 5, 5, 5, 5, 6, 6, 6, 6, 6, 6, 6};
+__constant__ unsigned char kTriJ[28] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3, 0, 1, 2, 3,
+                                        4, 0, 1, 2, 3, 4, 5, 0, 1, 2, 3, 4, 5, 6};
+
+// Named barriers of the diagonal tile (0 is __syncthreads): 1 joins warps
+// 1–7; 2 hands X and the next panel block from warp 0 to warps 1–7; 3 hands
+// finished trailing updates from warps 1–7 back to warp 0.
+constexpr int kBarRest = 1, kBarX = 2, kBarDone = 3;
+
+__device__ __forceinline__ void bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(int id, int count) {
+  __threadfence_block();
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// C (8×8 at c, row stride LDM) ±= X·Yᵀ for 8×8 blocks X, Y at x, y (row stride
+// ldx, ldy): two k-steps of the float64 tensor-core product.  Operands are
+// loaded before the products, so C may alias X.
+template <bool SUBTRACT, bool ACCUMULATE>
+__device__ __forceinline__ void block8_nt(double* c, const double* x, int ldx,
+                                          const double* y, int ldy, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  double2* cp = reinterpret_cast<double2*>(c + g * LDM + 2 * t);
+  double acc[2] = {0.0, 0.0};
+  if (ACCUMULATE) {
+    const double2 cv = *cp;
+    acc[0] = cv.x;
+    acc[1] = cv.y;
+  }
+  const double x0 = x[g * ldx + t], x1 = x[g * ldx + 4 + t];
+  const double y0 = y[g * ldy + t], y1 = y[g * ldy + 4 + t];
+  dmma_884(acc, SUBTRACT ? -x0 : x0, y0);
+  dmma_884(acc, SUBTRACT ? -x1 : x1, y1);
+  *cp = make_double2(acc[0], acc[1]);
+}
+
+// C (8×8 at c) = X·B for X 8×8 row-major with stride 8 and B 8×8 at b (row
+// stride LDM); C may alias B.
+__device__ __forceinline__ void block8_xb(double* c, const double* X, const double* b, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  double acc[2] = {0.0, 0.0};
+  const double b0 = b[t * LDM + g], b1 = b[(4 + t) * LDM + g];
+  dmma_884(acc, X[g * 8 + t], b0);
+  dmma_884(acc, X[g * 8 + 4 + t], b1);
+  *reinterpret_cast<double2*>(c + g * LDM + 2 * t) = make_double2(acc[0], acc[1]);
+}
+
+constexpr double kMinNormal = 2.2250738585072014e-308;
+constexpr double kMaxFinite = 1.7976931348623157e308;
+
+// Cholesky of an 8×8 block held (lower triangle, packed row by row) in the
+// registers of every lane of one warp, two pivots at a time: for the leading
+// 2×2 block [[d, b], [b, c]] with det = d·c − b², the two reciprocal square
+// roots 1/√d and 1/√det are independent, and 1/L₁₁ = √d/√det.  Lane j also
+// builds column j (j = lane mod 8) of X = L⁻¹ by forward substitution as the
+// pivots appear, X[i][j] = −(1/L_ii)·Σ_{j≤m<i} L[i][m]·X[m][j].  Returns the
+// first pivot position whose pivot (or 2×2 determinant) is not a positive
+// normal float64, else 8.
+__device__ __forceinline__ int chol8_pairs(double (&l)[36], double (&x)[8], int lane) {
+  const int jc = lane & 7;
+  int badp = 8;
+#pragma unroll
+  for (int p = 0; p < 8; p += 2) {
+    const int P0 = p * (p + 1) / 2, P1 = (p + 1) * (p + 2) / 2;
+    const double d1 = l[P0 + p], bb = l[P1 + p], cc = l[P1 + p + 1];
+    const double det = fma(d1, cc, -bb * bb);
+    const bool ok1 = d1 >= kMinNormal && d1 <= kMaxFinite;
+    const bool ok2 = det >= kMinNormal && det <= kMaxFinite;
+    badp = (badp == 8 && !ok1) ? p : ((badp == 8 && !ok2) ? p + 1 : badp);
+    const double y1 = ok1 ? rsqrt(d1) : 0.0;
+    const double z = ok2 ? rsqrt(det) : 0.0;
+    const double s1 = d1 * y1;
+    const double lb = bb * y1;
+    const double y2 = s1 * z;
+    double s = 0.0;
+#pragma unroll
+    for (int m = 0; m < p; ++m) s = fma(l[P0 + m], x[m], s);
+    x[p] = (p == jc) ? y1 : ((p < jc) ? 0.0 : -y1 * s);
+    double s2 = lb * x[p];
+#pragma unroll
+    for (int m = 0; m < p; ++m) s2 = fma(l[P1 + m], x[m], s2);
+    x[p + 1] = (p + 1 == jc) ? y2 : ((p + 1 < jc) ? 0.0 : -y2 * s2);
+    l[P0 + p] = s1;
+    l[P1 + p] = lb;
+    l[P1 + p + 1] = (det * z) * y1;
+#pragma unroll
+    for (int i = p + 2; i < 8; ++i) {
+      const int I = i * (i + 1) / 2;
+      const double li0 = l[I + p] * y1;
+      l[I + p] = li0;
+      l[I + p + 1] = fma(-li0, lb, l[I + p + 1]) * y2;
+    }
+#pragma unroll
+    for (int i = p + 2; i < 8; ++i)
+#pragma unroll
+      for (int j = p + 2; j <= i; ++j) {
+        const int I = i * (i + 1) / 2, J = j * (j + 1) / 2;
+        l[I + j] = fma(-l[I + p], l[J + p], fma(-l[I + p + 1], l[J + p + 1], l[I + j]));
+      }
+  }
+  return badp;
+}
+
+// Diagonal tile: D = L⁻¹ with L = chol(A) for a 64×64 tile in shared memory
+// (a: lower triangle of A on entry, overwritten; b: zero on entry, D on
+// exit; xs: 3 × 64 doubles), blocked by 8 columns and software-pipelined:
+//   warp 0, step kb: Cholesky of the diagonal block kb (registers), X_kb =
+//     its inverse; then, once warps 1–7 have applied step kb−1 to block row
+//     kb+1, the panel block L_{kb+1,kb} = A_{kb+1,kb}·X_kbᵀ and the diagonal
+//     block A_{kb+1,kb+1} −= L_{kb+1,kb}·L_{kb+1,kb}ᵀ, so that step kb+1 can
+//     start at once;
+//   warps 1–7, step kb: the other panel blocks L_{I,kb} (I ≥ kb+2), the
+//     other trailing blocks A_{IJ} −= L_{I,kb}·L_{J,kb}ᵀ, and block row kb of
+//     D: D_{kb,J} = X_kb·D_{kb,J} (J < kb), D_{kb,kb} = X_kb, then
+//     D_{IJ} −= L_{I,kb}·D_{kb,J} for I > kb, J ≤ kb (the elimination applied
+//     to an identity matrix).
+// All products are 8×8 blocks on the float64 tensor cores.  A bad pivot is
+// reported through info (the factorisation runs to the end on zeros, so that
+// every barrier is met) and makes the function return false.  Called by a
+// whole CTA of 256 threads.
+__device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
+                               int64_t n, int64_t base, int32_t* info, int* bad_s) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, q = lane & 3;
+  if (warp == 0) {
+    double l[36];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j <= i; ++j) l[i * (i + 1) / 2 + j] = a[i][j];
+    int bad = 8 * 8;
+    for (int kb = 0; kb < 8; ++kb) {
+      const int c0 = 8 * kb;
+      double x[8];
+      const int badp = chol8_pairs(l, x, lane);
+      bad = (bad == 64 && badp < 8) ? c0 + badp : bad;
+      double* X = xs + 64 * (kb % 3);   // warp 0 runs up to two steps ahead of the readers
+      if (lane < 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) X[i * 8 + lane] = x[i];
+      }
+      __syncwarp();
+      // warps 1–7 have applied step kb−1 (and so have all passed barrier X
+      // of step kb−1: no arrival below can fall into an older generation)
+      if (kb > 0) bar_sync(kBarDone, 256);
+      if (kb < 7) {
+        const int r1 = c0 + 8;
+        block8_nt<false, false>(&a[r1][c0], &a[r1][c0], LDM, X, 8, lane);
+        __syncwarp();
+        block8_nt<true, true>(&a[r1][r1], &a[r1][c0], LDM, &a[r1][c0], LDM, lane);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j <= i; ++j) l[i * (i + 1) / 2 + j] = a[r1 + i][r1 + j];
+      }
+      bar_arrive(kBarX, 256);                          // X_kb and L_{kb+1,kb} ready
+    }
+    if (lane == 0 && bad < 64) {
+      *bad_s = 1;
+      report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + bad));
+    }
+  } else {
+    const int w = warp - 1;                            // 0..6
+    for (int kb = 0; kb < 8; ++kb) {
+      const int c0 = 8 * kb;
+      const double* X = xs + 64 * (kb % 3);
+      bar_sync(kBarX, 256);
+      // panel blocks I ≥ kb + 2
+      if (kb + 2 + w < 8) {
+        const int r = 8 * (kb + 2 + w);
+        block8_nt<false, false>(&a[r][c0], &a[r][c0], LDM, X, 8, lane);
+      }
+      bar_sync(kBarRest, 224);
+      // trailing blocks kb+1 ≤ J ≤ I ≤ 7 except (kb+1, kb+1); operands first
+      const int rem = 7 - kb;
+      const int nblk = rem * (rem + 1) / 2;
+      double2 cv[4];
+      double f[4][4];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int e = 1 + w + 7 * s;
+        if (e < nblk) {
+          const int bi = kb + 1 + kTriI[e], bj = kb + 1 + kTriJ[e];
+          cv[s] = *reinterpret_cast<const double2*>(&a[8 * bi + g][8 * bj + 2 * q]);
+          f[s][0] = a[8 * bi + g][c0 + q];
+          f[s][1] = a[8 * bi + g][c0 + 4 + q];
+          f[s][2] = a[8 * bj + g][c0 + q];
+          f[s][3] = a[8 * bj + g][c0 + 4 + q];
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int e = 1 + w + 7 * s;
+        if (e < nblk) {
+          const int bi = kb + 1 + kTriI[e], bj = kb + 1 + kTriJ[e];
+          double acc[2] = {cv[s].x, cv[s].y};
+          dmma_884(acc, -f[s][0], f[s][2]);
+          dmma_884(acc, -f[s][1], f[s][3]);
+          *reinterpret_cast<double2*>(&a[8 * bi + g][8 * bj + 2 * q]) = make_double2(acc[0], acc[1]);
+        }
+      }
+      if (kb < 7) bar_arrive(kBarDone, 256);           // warp 0 waits for steps 0..6
+      // block row kb of D
+      if (w < kb) block8_xb(&b[c0][8 * w], X, &b[c0][8 * w], lane);
+      if (w == 6) {
+        for (int e = lane; e < 64; e += 32) b[c0 + (e >> 3)][c0 + (e & 7)] = X[e];
+      }
+      bar_sync(kBarRest, 224);
+      // D_{IJ} −= L_{I,kb}·D_{kb,J}, I > kb, J ≤ kb
+      const int ncol = kb + 1;
+      for (int e = w; e < rem * ncol; e += 7) {
+        const int I = kb + 1 + e / ncol, J = e % ncol;
+        double2* cp = reinterpret_cast<double2*>(&b[8 * I + g][8 * J + 2 * q]);
+        const double2 c2 = *cp;
+        double acc[2] = {c2.x, c2.y};
+        dmma_884(acc, -a[8 * I + g][c0 + q], b[c0 + q][8 * J + g]);
+        dmma_884(acc, -a[8 * I + g][c0 + 4 + q], b[c0 + 4 + q][8 * J + g]);
+        *cp = make_double2(acc[0], acc[1]);
+      }
+    }
+  }
+  __syncthreads();
+  return *bad_s == 0;
+}
+
+// 64×64 tile loads into shared memory: the lower triangle (zeros above), and
+// zeros.  16-byte loads through L2 only (tiles are rewritten by other CTAs of
+// the same launch).
+__device__ __forceinline__ void load_lower(double (*dst)[LDM], const double* src, int64_t ld,
+                                           int tid) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int e = tid + 256 * s;              // 2048 pairs
+    const int r = e >> 5, c = (e & 31) * 2;
+    const double2 v = __ldcg(reinterpret_cast<const double2*>(src + (int64_t)r * ld + c));
+    *reinterpret_cast<double2*>(&dst[r][c]) = make_double2(c <= r ? v.x : 0.0, c + 1 <= r ? v.y : 0.0);
+  }
+}
+__device__ __forceinline__ void zero_tile(double (*dst)[LDM], int tid) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int e = tid + 256 * s;
+    *reinterpret_cast<double2*>(&dst[e >> 5][(e & 31) * 2]) = make_double2(0.0, 0.0);
+  }
+}
+__device__ __forceinline__ void store_tile(double* dst, int64_t ld, const double (*src)[LDM],
+                                           int tid) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int e = tid + 256 * s;
+    const int r = e >> 5, c = (e & 31) * 2;
+    *reinterpret_cast<double2*>(dst + (int64_t)r * ld + c) =
+        *reinterpret_cast<const double2*>(&src[r][c]);
+  }
+}
+
+// C = X·Yᵀ for 64×64 shared-memory tiles, Y given row-major (C[r][c] =
+// Σ_q X[r][q]·Y[c][q]).  Warp w owns rows 16·(w/2) .. +16 and columns
+// 32·(w%2) .. +32 of C: 2 × 4 accumulator blocks of 8×8.
+__device__ __forceinline__ void tile_mm_nt(const double (*x)[LDM], const double (*y)[LDM],
+                                           double acc[2][4][2], int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+#pragma unroll 4
+  for (int q = 0; q < NB; q += 4) {
+    double a[2], b[4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) a[i] = x[rb + 8 * i + g][q + t];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = y[cb + 8 * j + g][q + t];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dmma_884(acc[i][j], a[i], b[j]);
+  }
+}
+
+// Shared-memory tile ±= / = the accumulators of tile_mm_nt.
+template <bool SUBTRACT>
+__device__ __forceinline__ void tile_acc_smem(double (*dst)[LDM], const double acc[2][4][2],
+                                              int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double2* p = reinterpret_cast<double2*>(&dst[rb + 8 * i + g][cb + 8 * j + 2 * t]);
+      double2 v = make_double2(acc[i][j][0], acc[i][j][1]);
+      if (SUBTRACT) {
+        const double2 o = *p;
+        v = make_double2(o.x - v.x, o.y - v.y);
+      }
+      *p = v;
+    }
+}
+
+// 64×64 float64 tile products.  Warp w owns rows 16·(w/2) .. +16 and columns
+// 32·(w%2) .. +32 of C: 2 × 4 accumulator blocks of 8×8.
 
 __device__ __forceinline__ void tile_mm(const double (*x)[LDM], const double (*y)[LDM],
                                         double acc[2][4][2], int warp, int lane) {
@@ -407,22 +562,25 @@ __device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
 // ---------------------------------------------------------------------------
 // The factorisation as one persistent, dataflow launch.
 //
-// Tasks of step k (64-column block k), in the fixed global order in which the
-// workers take them (critical ones first, so step k+1 can start while step k
-// is still updating far tiles):
-//   PANEL(k,k+1), TRAIL(k,k+1,k+1), PANEL(k,i) i > k+1, TRAIL(k,i,k+1),
-//   MROW(k,c) c < k, MTRAIL(k,k+1,c), TRAIL(k,i,j) k+1 < j ≤ i, MTRAIL(k,i,c)
+// The first CTA to arrive runs the critical chain, keeping the diagonal tile
+// in shared memory from one step to the next (and its instruction cache
+// warm): DIAG(k) — D_k = L_kk⁻¹ —, then PANEL(k,k+1) — L_{k+1,k} =
+// A_{k+1,k}·D_kᵀ — and the last update of tile (k+1,k+1), once those two
+// tiles have received their first k updates from the workers.
+// The other CTAs take the remaining tasks of step k (64-column block k) in
+// a fixed global order (those the next steps wait for first):
+//   PANEL(k,i) i > k+1, TRAIL(k,i,k+1) i > k+1, MROW(k,c) c < k,
+//   MTRAIL(k,k+1,c), TRAIL(k,i,j) k+1 < j ≤ i, MTRAIL(k,i,c) i > k+1
 // with PANEL:  L_ik = A_ik·D_kᵀ          (needs D_k and tile (i,k) updated k times)
 //      MROW:   M_kc = D_k·M_kc           (needs D_k and M_kc updated k−c times)
 //      TRAIL:  A_ij −= L_ik·L_jkᵀ         (needs L_ik, L_jk, tile (i,j) updated k times)
 //      MTRAIL: M_ic −= L_ik·M_kc          (needs L_ik, final M_kc, M_ic updated k−c times)
-// and DIAG(k) — L_kk = chol(A_kk), D_k = L_kk⁻¹ — run by the first CTA to
-// arrive (its instruction cache stays warm across the chain of diagonal
-// tiles) once tile (k,k) has received its k updates.  Every dependency of a
-// task is an earlier task, and tasks are taken in order only by running
-// CTAs, so the launch needs no co-residency guarantee.  Flags are set with
-// release stores after a fence and polled with acquire loads; every wait is
-// bounded and a time-out (or a bad pivot) raises a shared abort flag.
+// Every dependency of a task is an earlier task or a step of the chain, the
+// chain at step k waits only for tasks of step k−1, and tasks are taken in
+// order only by running CTAs, so the launch needs no co-residency guarantee.
+// Flags are set with release stores after a fence and polled with acquire
+// loads; every wait is bounded and a time-out (or a bad pivot) raises a
+// shared abort flag.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kSpinLimit = 1u << 22;   // ≈ a few seconds with the back-off below
 
@@ -487,7 +645,7 @@ __device__ __forceinline__ void cta_signal(int* flag, int value) {
 __host__ __device__ inline int step_tasks(int N, int k) {
   const int r = N - k - 1;
   if (r <= 0) return k;                              // MROW only
-  return 2 + 2 * (r - 1) + k + (k + 1) + (r - 1) * r / 2 + (r - 1) * (k + 1);
+  return 2 * (r - 1) + k + (k + 1) + (r - 1) * r / 2 + (r - 1) * (k + 1);
 }
 
 int total_tasks(int N) {
@@ -503,10 +661,6 @@ __device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) 
   while (task >= step_tasks(N, k)) { task -= step_tasks(N, k); ++k; }
   const int r = N - k - 1;
   if (r <= 0) { kind = T_MROW; i = k; j = task; return; }
-  if (task < 1) { kind = T_PANEL; i = k + 1; j = k; return; }
-  task -= 1;
-  if (task < 1) { kind = T_TRAIL; i = k + 1; j = k + 1; return; }
-  task -= 1;
   if (task < r - 1) { kind = T_PANEL; i = k + 2 + task; j = k; return; }
   task -= r - 1;
   if (task < r - 1) { kind = T_TRAIL; i = k + 2 + task; j = k + 1; return; }
@@ -524,12 +678,12 @@ __device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) 
   kind = T_MTRAIL; i = k + 2 + task / (k + 1); j = task % (k + 1);
 }
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
 chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
-                       double* __restrict__ Dall, int64_t n, int64_t np, int N,
+                       int64_t n, int64_t np, int N,
                        int ntasks, int* sync_base, int32_t* info) {
   extern __shared__ double sm[];
-  __shared__ int s_role, s_task, s_ok;
+  __shared__ int s_role, s_task, s_ok, s_bad;
   const CholSync S = sync_view(sync_base, N);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) s_role = atomicAdd(&S.ctrl[1], 1);
@@ -537,14 +691,45 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   if (*reinterpret_cast<volatile int32_t*>(info) != 0) return;
 
   if (s_role == 0) {
-    // ---- the chain of diagonal tiles
+    // ---- the critical chain: DIAG(k), then PANEL(k, k+1) and the last
+    // update of tile (k+1, k+1), which stays in shared memory for DIAG(k+1)
+    double (*a)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
+    double (*b)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
+    double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * NB * LDM);
+    double* xs = sm + 3 * NB * LDM;
+    load_lower(a, A, np, tid);
+    zero_tile(b, tid);
+    if (tid == 0) s_bad = 0;
+    __syncthreads();
     for (int k = 0; k < N; ++k) {
-      if (!cta_wait(&S.upd[k * N + k], k, &S.ctrl[2], info, &s_ok)) return;
-      if (!diag_tile(A, M, Dall + (size_t)k * NB * NB, n, np, k, info, sm)) {
+      const int64_t base = (int64_t)k * NB;
+      if (!diag_tile_smem(a, b, xs, n, base, info, &s_bad)) {
         if (tid == 0) atomicExch(&S.ctrl[2], 1);
         return;
       }
+      store_tile(M + base * np + base, np, b, tid);
       cta_signal(&S.diag_done[k], 1);
+      if (k + 1 == N) break;
+      // L_{k+1,k} = A_{k+1,k}·D_kᵀ
+      if (!cta_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok)) return;
+      double* Lp = A + (base + NB) * np + base;
+      load_tile(x, Lp, np, false, tid);
+      __syncthreads();
+      double acc[2][4][2] = {};
+      tile_mm_nt(x, b, acc, warp, lane);
+      __syncthreads();
+      tile_acc_smem<false>(x, acc, warp, lane);
+      tile_store<false>(Lp, np, acc, warp, lane);
+      cta_signal(&S.pdone[k * N + k + 1], 1);
+      // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
+      if (!cta_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok)) return;
+      load_lower(a, A + (base + NB) * np + base + NB, np, tid);
+      zero_tile(b, tid);
+      __syncthreads();
+      double acc2[2][4][2] = {};
+      tile_mm_nt(x, x, acc2, warp, lane);
+      tile_acc_smem<true>(a, acc2, warp, lane);
+      __syncthreads();
     }
     return;
   }
@@ -565,7 +750,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       if (!cta_wait(&S.upd[i * N + k], k, &S.ctrl[2], info, &s_ok)) return;
       double* out = A + (int64_t)i * NB * np + (int64_t)k * NB;
       load_tile(x, out, np, false, tid);
-      load_tile(y, Dall + (size_t)k * NB * NB, NB, true, tid);
+      load_tile(y, M + (int64_t)k * NB * np + (int64_t)k * NB, np, true, tid);
       __syncthreads();
       tile_mm(x, y, acc, warp, lane);
       tile_store<false>(out, np, acc, warp, lane);
@@ -575,7 +760,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) return;
       if (!cta_wait(&S.mupd[k * N + c], k - c, &S.ctrl[2], info, &s_ok)) return;
       double* out = M + (int64_t)k * NB * np + (int64_t)c * NB;
-      load_tile(x, Dall + (size_t)k * NB * NB, NB, false, tid);
+      load_tile(x, M + (int64_t)k * NB * np + (int64_t)k * NB, np, false, tid);
       load_tile(y, out, np, false, tid);
       __syncthreads();
       tile_mm(x, y, acc, warp, lane);
@@ -658,7 +843,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  const size_t tile_smem = 2 * NB * LDM * sizeof(double);   // ≥ the diagonal tile's 2·NB·LDT
+  const size_t tile_smem = (3 * NB * LDM + 192) * sizeof(double);
   if (!g_smem_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(chol_persistent_kernel,
               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
@@ -680,7 +865,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
               w.mean, damp, w.A, w.M, info);
   const int ntasks = total_tasks(N);
   const int grid = (ntasks + 1 < 2 * g_num_sms) ? ntasks + 1 : 2 * g_num_sms;
-  GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, w.D, n, np,
+  GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, n, np,
               N, ntasks, w.sync, info);
   GPTQ_LAUNCH(KK_PREP_OUT, s, prep_out_kernel, (unsigned)ceil_div(n * n, 256), 256, 0,
               w.M, n, np, U);
@@ -703,7 +888,6 @@ constexpr int64_t kNoAllocN = kNoAllocMaxN / NB;
 constexpr size_t kNoAllocBytes =
     up256(sizeof(double)) + up256(sizeof(int32_t) * kNoAllocMaxN) +
     2 * up256(sizeof(double) * kNoAllocMaxN * kNoAllocMaxN) +
-    up256(sizeof(double) * NB * NB * kNoAllocN) +
     up256(sizeof(int) * (4 + kNoAllocN + 4 * kNoAllocN * kNoAllocN));
 static_assert(kNoAllocMaxN % NB == 0, "the fixed limit is a whole number of tiles");
 
