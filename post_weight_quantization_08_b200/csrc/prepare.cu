@@ -187,11 +187,11 @@ __device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
                : "d"(a), "d"(b));
 }
 
-// Lower-triangle block pairs (I, J), J ≤ I, in the order e = I·(I+1)/2 + J.
-__constant__ unsigned char kTriI[28] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3, 4, 4, 4, 4,
-                                        4, 5, 5, 5, 5, 5, 5, 6, 6, 6, 6, 6, 6, 6};
-__constant__ unsigned char kTriJ[28] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3, 0, 1, 2, 3,
-                                        4, 0, 1, 2, 3, 4, 5, 0, 1, 2, 3, 4, 5, 6};
+// Lower-triangle 8×8 blocks (I, J), J ≤ I < 8, row by row (e = I·(I+1)/2 + J).
+__constant__ unsigned char kTri8I[36] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3, 4, 4, 4, 4, 4, 5, 5, 5,
+                                         5, 5, 5, 6, 6, 6, 6, 6, 6, 6, 7, 7, 7, 7, 7, 7, 7, 7};
+__constant__ unsigned char kTri8J[36] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3, 0, 1, 2, 3, 4, 0, 1, 2,
+                                         3, 4, 5, 0, 1, 2, 3, 4, 5, 6, 0, 1, 2, 3, 4, 5, 6, 7};
 
 // Named barriers of the diagonal tile (0 is __syncthreads): 1 joins warps
 // 1–7; 2 hands X and the next panel block from warp 0 to warps 1–7; 3 hands
@@ -307,12 +307,14 @@ __device__ __forceinline__ int chol8_pairs(double (&l)[36], double (&x)[8], int 
 //     D: D_{kb,J} = X_kb·D_{kb,J} (J < kb), D_{kb,kb} = X_kb, then
 //     D_{IJ} −= L_{I,kb}·D_{kb,J} for I > kb, J ≤ kb (the elimination applied
 //     to an identity matrix).
-// All products are 8×8 blocks on the float64 tensor cores.  A bad pivot is
+// Each block row of D goes out to dout (leading dimension ld) as soon as it is
+// final.  All products are 8×8 blocks on the float64 tensor cores.  A bad pivot is
 // reported through info (the factorisation runs to the end on zeros, so that
 // every barrier is met) and makes the function return false.  Called by a
 // whole CTA of 256 threads.
 __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
-                               int64_t n, int64_t base, int32_t* info, int* bad_s) {
+                               double* __restrict__ dout, int64_t ld, int64_t n, int64_t base,
+                               int32_t* info, int* bad_s) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q = lane & 3;
   if (warp == 0) {
@@ -354,27 +356,29 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
       report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + bad));
     }
   } else {
-    const int w = warp - 1;                            // 0..6
+    // Warp 4 shares a scheduler (and its float64 pipe) with warp 0, so it
+    // takes no work: v numbers the six working warps.
+    const int v = (warp < 4) ? warp - 1 : ((warp > 4) ? warp - 2 : -1);
     for (int kb = 0; kb < 8; ++kb) {
       const int c0 = 8 * kb;
       const double* X = xs + 64 * (kb % 3);
       bar_sync(kBarX, 256);
       // panel blocks I ≥ kb + 2
-      if (kb + 2 + w < 8) {
-        const int r = 8 * (kb + 2 + w);
+      if (v >= 0 && kb + 2 + v < 8) {
+        const int r = 8 * (kb + 2 + v);
         block8_nt<false, false>(&a[r][c0], &a[r][c0], LDM, X, 8, lane);
       }
       bar_sync(kBarRest, 224);
       // trailing blocks kb+1 ≤ J ≤ I ≤ 7 except (kb+1, kb+1); operands first
       const int rem = 7 - kb;
       const int nblk = rem * (rem + 1) / 2;
-      double2 cv[4];
-      double f[4][4];
+      double2 cv[5];
+      double f[5][4];
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int e = 1 + w + 7 * s;
-        if (e < nblk) {
-          const int bi = kb + 1 + kTriI[e], bj = kb + 1 + kTriJ[e];
+      for (int s = 0; s < 5; ++s) {
+        const int e = 1 + v + 6 * s;
+        if (v >= 0 && e < nblk) {
+          const int bi = kb + 1 + kTri8I[e], bj = kb + 1 + kTri8J[e];
           cv[s] = *reinterpret_cast<const double2*>(&a[8 * bi + g][8 * bj + 2 * q]);
           f[s][0] = a[8 * bi + g][c0 + q];
           f[s][1] = a[8 * bi + g][c0 + 4 + q];
@@ -383,10 +387,10 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
         }
       }
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int e = 1 + w + 7 * s;
-        if (e < nblk) {
-          const int bi = kb + 1 + kTriI[e], bj = kb + 1 + kTriJ[e];
+      for (int s = 0; s < 5; ++s) {
+        const int e = 1 + v + 6 * s;
+        if (v >= 0 && e < nblk) {
+          const int bi = kb + 1 + kTri8I[e], bj = kb + 1 + kTri8J[e];
           double acc[2] = {cv[s].x, cv[s].y};
           dmma_884(acc, -f[s][0], f[s][2]);
           dmma_884(acc, -f[s][1], f[s][3]);
@@ -395,14 +399,25 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
       }
       if (kb < 7) bar_arrive(kBarDone, 256);           // warp 0 waits for steps 0..6
       // block row kb of D
-      if (w < kb) block8_xb(&b[c0][8 * w], X, &b[c0][8 * w], lane);
-      if (w == 6) {
+      if (v >= 0) {
+        for (int J = v; J < kb; J += 6) block8_xb(&b[c0][8 * J], X, &b[c0][8 * J], lane);
+      }
+      if (v == 5) {
         for (int e = lane; e < 64; e += 32) b[c0 + (e >> 3)][c0 + (e & 7)] = X[e];
       }
       bar_sync(kBarRest, 224);
+      // block row kb of D is final: out to global memory now, so that little
+      // is left in flight when the tile is published
+      if (v >= 0) {
+        for (int e = 32 * v + lane; e < 256; e += 192) {
+          const int r = c0 + (e >> 5), c = (e & 31) * 2;
+          *reinterpret_cast<double2*>(dout + (int64_t)r * ld + c) =
+              *reinterpret_cast<const double2*>(&b[r][c]);
+        }
+      }
       // D_{IJ} −= L_{I,kb}·D_{kb,J}, I > kb, J ≤ kb
       const int ncol = kb + 1;
-      for (int e = w; e < rem * ncol; e += 7) {
+      for (int e = (v >= 0 ? v : rem * ncol); e < rem * ncol; e += 6) {
         const int I = kb + 1 + e / ncol, J = e % ncol;
         double2* cp = reinterpret_cast<double2*>(&b[8 * I + g][8 * J + 2 * q]);
         const double2 c2 = *cp;
@@ -448,45 +463,93 @@ __device__ __forceinline__ void store_tile(double* dst, int64_t ld, const double
   }
 }
 
-// C = X·Yᵀ for 64×64 shared-memory tiles, Y given row-major (C[r][c] =
-// Σ_q X[r][q]·Y[c][q]).  Warp w owns rows 16·(w/2) .. +16 and columns
-// 32·(w%2) .. +32 of C: 2 × 4 accumulator blocks of 8×8.
-__device__ __forceinline__ void tile_mm_nt(const double (*x)[LDM], const double (*y)[LDM],
-                                           double acc[2][4][2], int warp, int lane) {
+// Asynchronous 64×64 tile copy global → shared memory (16-byte cp.async
+// through L2 only; tiles are rewritten by other CTAs of the same launch).
+__device__ __forceinline__ void copy_tile_async(double (*dst)[LDM], const double* src, int64_t ld,
+                                                int tid) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int e = tid + 256 * s;
+    const int r = e >> 5, c = (e & 31) * 2;
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&dst[r][c]));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + (int64_t)r * ld + c)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void copy_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// L = A·Dᵀ for 64×64 shared-memory tiles with D lower triangular, so block
+// column J of L needs only q < 8·(J+1).  Warp w owns row blocks 4·(w/4) .. +4
+// and block columns J = w mod 4 and 7 − J, which gives every warp the same
+// number of products (and every scheduler the same load).  acc[i][c] is
+// block (4·(w/4) + i, c ? 7 − J : J).
+__device__ __forceinline__ void panel_mm(const double (*x)[LDM], const double (*d)[LDM],
+                                         double acc[4][2][2], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
-#pragma unroll 4
-  for (int q = 0; q < NB; q += 4) {
-    double a[2], b[4];
+  const int rb = 32 * (warp >> 2), J = warp & 3, J1 = 7 - J;
+  const int qlo = 8 * (J + 1), qhi = 8 * (J1 + 1);
+  for (int q = 0; q < qhi; q += 4) {
+    double a[4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    const double b1 = d[8 * J1 + g][q + t];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = y[cb + 8 * j + g][q + t];
+    for (int i = 0; i < 4; ++i) dmma_884(acc[i][1], a[i], b1);
+    if (q < qlo) {
+      const double b0 = d[8 * J + g][q + t];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dmma_884(acc[i][j], a[i], b[j]);
+      for (int i = 0; i < 4; ++i) dmma_884(acc[i][0], a[i], b0);
+    }
   }
 }
 
-// Shared-memory tile ±= / = the accumulators of tile_mm_nt.
-template <bool SUBTRACT>
-__device__ __forceinline__ void tile_acc_smem(double (*dst)[LDM], const double acc[2][4][2],
-                                              int warp, int lane) {
+// Writes the panel accumulators to a shared-memory tile and to global memory.
+__device__ __forceinline__ void panel_store(double (*xs_)[LDM], double* out, int64_t ld,
+                                            const double acc[4][2][2], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+  const int rb = 32 * (warp >> 2), J = warp & 3;
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      double2* p = reinterpret_cast<double2*>(&dst[rb + 8 * i + g][cb + 8 * j + 2 * t]);
-      double2 v = make_double2(acc[i][j][0], acc[i][j][1]);
-      if (SUBTRACT) {
-        const double2 o = *p;
-        v = make_double2(o.x - v.x, o.y - v.y);
-      }
-      *p = v;
+    for (int c = 0; c < 2; ++c) {
+      const int r = rb + 8 * i + g, col = 8 * (c ? 7 - J : J) + 2 * t;
+      const double2 v = make_double2(acc[i][c][0], acc[i][c][1]);
+      *reinterpret_cast<double2*>(&xs_[r][col]) = v;
+      *reinterpret_cast<double2*>(out + (int64_t)r * ld + col) = v;
     }
+}
+
+// T −= L·Lᵀ on the 36 lower 8×8 blocks of a 64×64 shared-memory tile (the
+// blocks above the diagonal are never read).  Warp w takes blocks w + 8·s, so
+// the two warps of each scheduler share nine blocks.
+__device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[LDM], int warp,
+                                           int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  double acc[5][2] = {};
+  int bi[5], bj[5];
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int e = warp + 8 * s;
+    bi[s] = (e < 36) ? kTri8I[e] : 0;
+    bj[s] = (e < 36) ? kTri8J[e] : 0;
+  }
+#pragma unroll 2
+  for (int q = 0; q < NB; q += 4) {
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+      if (warp + 8 * s < 36)
+        dmma_884(acc[s], l[8 * bi[s] + g][q + t], l[8 * bj[s] + g][q + t]);
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    if (warp + 8 * s < 36) {
+      double2* p = reinterpret_cast<double2*>(&tt[8 * bi[s] + g][8 * bj[s] + 2 * t]);
+      const double2 o = *p;
+      *p = make_double2(o.x - acc[s][0], o.y - acc[s][1]);
+    }
+  }
 }
 
 // 64×64 float64 tile products.  Warp w owns rows 16·(w/2) .. +16 and columns
@@ -692,44 +755,56 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
 
   if (s_role == 0) {
     // ---- the critical chain: DIAG(k), then PANEL(k, k+1) and the last
-    // update of tile (k+1, k+1), which stays in shared memory for DIAG(k+1)
-    double (*a)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
-    double (*b)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
-    double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * NB * LDM);
-    double* xs = sm + 3 * NB * LDM;
-    load_lower(a, A, np, tid);
+    // update of tile (k+1, k+1), which stays in shared memory for DIAG(k+1).
+    // Two buffers alternate as the diagonal tile.  D_k leaves block row by
+    // block row during DIAG(k), and L_{k+1,k} is published only after the
+    // update that follows it, so neither signal waits long for its stores.
+    double (*t0)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
+    double (*t1)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
+    double (*b)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * NB * LDM);
+    double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 3 * NB * LDM);
+    double* xs = sm + 4 * NB * LDM;
+    load_lower(t0, A, np, tid);
     zero_tile(b, tid);
     if (tid == 0) s_bad = 0;
     __syncthreads();
     for (int k = 0; k < N; ++k) {
       const int64_t base = (int64_t)k * NB;
-      if (!diag_tile_smem(a, b, xs, n, base, info, &s_bad)) {
+      double (*a)[LDM] = (k & 1) ? t1 : t0;
+      double (*an)[LDM] = (k & 1) ? t0 : t1;
+      const bool more = k + 1 < N;
+      double* Lp = A + (base + NB) * np + base;          // tile (k+1, k)
+      const double* An = A + (base + NB) * np + base + NB;   // tile (k+1, k+1)
+      if (!diag_tile_smem(a, b, xs, M + base * np + base, np, n, base, info, &s_bad)) {
         if (tid == 0) atomicExch(&S.ctrl[2], 1);
         return;
       }
-      store_tile(M + base * np + base, np, b, tid);
-      cta_signal(&S.diag_done[k], 1);
-      if (k + 1 == N) break;
+      if (tid == 0) {                 // D_k is out (the diagonal tile ended with a barrier)
+        __threadfence();
+        st_release(&S.diag_done[k], 1);
+      }
+      if (!more) break;
       // L_{k+1,k} = A_{k+1,k}·D_kᵀ
       if (!cta_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok)) return;
-      double* Lp = A + (base + NB) * np + base;
-      load_tile(x, Lp, np, false, tid);
+      copy_tile_async(x, Lp, np, tid);
+      copy_wait_all();
       __syncthreads();
-      double acc[2][4][2] = {};
-      tile_mm_nt(x, b, acc, warp, lane);
+      double acc[4][2][2] = {};
+      panel_mm(x, b, acc, warp, lane);
       __syncthreads();
-      tile_acc_smem<false>(x, acc, warp, lane);
-      tile_store<false>(Lp, np, acc, warp, lane);
-      cta_signal(&S.pdone[k * N + k + 1], 1);
+      panel_store(x, Lp, np, acc, warp, lane);
+      zero_tile(b, tid);
       // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
       if (!cta_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok)) return;
-      load_lower(a, A + (base + NB) * np + base + NB, np, tid);
-      zero_tile(b, tid);
+      copy_tile_async(an, An, np, tid);
+      copy_wait_all();
       __syncthreads();
-      double acc2[2][4][2] = {};
-      tile_mm_nt(x, x, acc2, warp, lane);
-      tile_acc_smem<true>(a, acc2, warp, lane);
+      lower_syrk(an, x, warp, lane);
       __syncthreads();
+      if (tid == 0) {                 // L_{k+1,k} is out (its stores drained meanwhile)
+        __threadfence();
+        st_release(&S.pdone[k * N + k + 1], 1);
+      }
     }
     return;
   }
@@ -843,7 +918,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  const size_t tile_smem = (3 * NB * LDM + 192) * sizeof(double);
+  const size_t tile_smem = (4 * NB * LDM + 192) * sizeof(double);
   if (!g_smem_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(chol_persistent_kernel,
               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
