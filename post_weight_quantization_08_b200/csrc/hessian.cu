@@ -25,7 +25,6 @@
 // Every wait is bounded; a time-out is reported through `info`.
 // Fallback (n not a multiple of 8): a float32 SIMT tile kernel.
 #include <cuda_bf16.h>
-#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -251,32 +250,6 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
   if (warp == 0) tmem_dealloc(tmem, TC_TILE);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner,
-               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return enc(tm, dt, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool g_tc_attr = false;
 
 }  // namespace
@@ -297,8 +270,8 @@ extern "C" gptq_status gptq_hessian_accumulate(const void* X, int64_t T, int64_t
                       (reinterpret_cast<uintptr_t>(H) % 16 == 0);
   if (tma_ok) {
     CUtensorMap tm, th;
-    if (!encode_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, n, T, n * 2, 64, TC_KT) ||
-        !encode_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, H, n, n, n * 4, 32, TC_TILE))
+    if (!encode_tiled_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, n, T, n * 2, 64, TC_KT) ||
+        !encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, H, n, n, n * 4, 32, TC_TILE))
       return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the Hessian");
     if (!g_tc_attr) {
       GPTQ_CUDA(cudaFuncSetAttribute(hessian_tc_kernel,

@@ -14,6 +14,11 @@ constexpr size_t PANEL_BYTES = (size_t)16 * 4096 + 128 * sizeof(float);
 
 size_t panel_workspace_bytes(int64_t n, int block);
 
+// Rows of the working copy Wp and of the error buffers Ehi/Elo: m rounded up
+// to whole 128-row boxes, so that no box store or reduction is clipped (a
+// clipped one is several times slower).  Rows ≥ m are never read back.
+inline int64_t error_rows(int64_t m) { return (m + 127) / 128 * 128; }
+
 // One panel per block of U, laid out for the sweep's bulk copy.
 gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
                           cudaStream_t s);
@@ -21,7 +26,8 @@ gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
 // Columns [j0, j0+bw) of the float32 working copy Wp (m×n, processing order):
 // quantize column by column with in-block error propagation.  Writes codes
 // (m×n u8, processing order), scale/zero (m×ngroups), the scaled errors as a
-// TF32 split Ehi + Elo (each m×128, Ehi = TF32(e), Elo = e − Ehi exactly) and
+// TF32 split Ehi + Elo (each error_rows(m)×128, Ehi = TF32(e), Elo = e − Ehi
+// exactly) and
 // adds Σe² to loss_row (may be NULL).
 gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,

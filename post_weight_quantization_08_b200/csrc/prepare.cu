@@ -939,7 +939,13 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);
   const int ntasks = total_tasks(N);
-  const int grid = (ntasks + 1 < 2 * g_num_sms) ? ntasks + 1 : 2 * g_num_sms;
+  // Workers: about as many as the dataflow keeps busy (a step offers ≈ N²/2
+  // tile tasks, each ≈ a third of the chain's step), never more than one CTA
+  // per SM besides the chain's, so that work on other streams finds SMs.
+  int workers = N * N / 6 + 2;
+  if (workers > g_num_sms - 1) workers = g_num_sms - 1;
+  if (workers > ntasks) workers = ntasks;
+  const int grid = 1 + workers;
   GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, n, np,
               N, ntasks, w.sync, info);
   GPTQ_LAUNCH(KK_PREP_OUT, s, prep_out_kernel, (unsigned)ceil_div(n * n, 256), 256, 0,

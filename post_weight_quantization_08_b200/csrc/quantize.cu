@@ -13,7 +13,7 @@ namespace gptq {
 namespace {
 
 struct QuantWs {
-  float* Wp;        // m × n working copy, processing order
+  float* Wp;        // error_rows(m) × n working copy, processing order
   uint8_t* codes;   // m × n codes, processing order
   float* Ehi;       // m × 128 scaled errors of the current block, TF32 part
   float* Elo;       // m × 128 remainder e − Ehi
@@ -30,10 +30,13 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
     off = align_up(off + bytes, 256);
     return o;
   };
-  size_t o_wp = take(sizeof(float) * (size_t)m * (size_t)n);
+  // Wp and the error buffers hold whole 128-row boxes, so that no box store
+  // or reduction is clipped (rows ≥ m are never read back)
+  const size_t mrows = (size_t)error_rows(m);
+  size_t o_wp = take(sizeof(float) * mrows * (size_t)n);
   size_t o_codes = take((size_t)m * (size_t)n);
-  size_t o_ehi = take(sizeof(float) * (size_t)m * SWEEP_BLOCK_MAX);
-  size_t o_elo = take(sizeof(float) * (size_t)m * SWEEP_BLOCK_MAX);
+  size_t o_ehi = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
+  size_t o_elo = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
   size_t o_pinv = take(sizeof(int32_t) * (size_t)n);
   size_t o_pan = take(panel_workspace_bytes(n, block));
   const bool tc = trailing_uses_tensor_cores(n, block);

@@ -199,6 +199,21 @@ __device__ __forceinline__ void bulk_commit() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// Wait until every committed bulk group of this thread has finished reading
+// its shared-memory source (the buffers may then be rewritten).
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// 2-D tiled TMA store of one shared-memory box to (x = inner coordinate, y);
+// rows or columns outside the tensor are not written.  x, y ≥ 0.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y,
+                                             const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(x), "r"(y), "r"(smem_addr(src))
+               : "memory");
+}
 
 // float32 → TF32 (round to nearest, ties away), returned in a float container
 // whose low 13 mantissa bits are zero.
@@ -210,5 +225,11 @@ __device__ __forceinline__ float to_tf32(float x) {
 
 // Sanity: "K-major" 128-byte-swizzle descriptors ignore LBO; 16 B by convention.
 constexpr uint32_t SW128_KMAJOR_LBO = 16;
+
+// Host: a 2-D tiled tensor map with 128-byte swizzle (inner extent and box
+// inner size in elements, row pitch in bytes); false when the driver's encoder
+// is unavailable or rejects the arguments.
+bool encode_tiled_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                     uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace gptq

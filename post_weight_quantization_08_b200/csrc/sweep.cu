@@ -115,12 +115,20 @@ package_kernel(const float* __restrict__ U, int64_t n, int block,
   }
 }
 
+// x/s correctly rounded, for s > 0.  A zero numerator is answered directly
+// (the quotient is that same signed zero): the division's general route is
+// many times slower for it, and zero rows (padding, dead columns) are common.
+__device__ __forceinline__ float div_rn(float x, float s) {
+  const float q = __fdiv_rn(x == 0.f ? 1.f : x, s);
+  return x == 0.f ? x : q;
+}
+
 __global__ void __launch_bounds__(RT, 1)
-sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
+sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
+             const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
              const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
              uint8_t* __restrict__ codes, float* __restrict__ scale,
-             uint8_t* __restrict__ zero, float* __restrict__ Ehi,
-             float* __restrict__ Elo, float* __restrict__ loss_row, int32_t* info) {
+             uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info) {
   extern __shared__ unsigned char smraw[];
   const uint32_t raw = smem_addr(smraw);
   unsigned char* sm = smraw + ((1024 - (raw & 1023)) & 1023);
@@ -157,31 +165,29 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
     bulk_g2s(sm + SM_PKG, pkg, PK_BYTES, pkg_bar);
   }
 
-  // this thread's row of the block → vals (row-major, odd stride)
-  float* vr = vals + t * LDV;
-  if (row < m) {
-    const float* src = Wp + row * n + j0;
-    if ((n & 3) == 0 && bw == SB) {
-      const float4* s4 = reinterpret_cast<const float4*>(src);
+  // the CTA's rows of the block → vals (row-major, odd stride): warp w
+  // reads rows 32w .. 32w+31 with lanes along the columns (coalesced 128-byte
+  // reads, conflict-free shared-memory writes); rows past m and columns past
+  // the block are zero
+#pragma unroll 1
+  for (int i0 = 0; i0 < 32; i0 += 8) {
+    float buf[8][4];
 #pragma unroll
-      for (int b4 = 0; b4 < SB / 4; b4 += 8) {
-        float4 buf[8];
+    for (int i = 0; i < 8; ++i) {
+      const int64_t r = r0 + 32 * warp + i0 + i;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) buf[k] = s4[b4 + k];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          vr[4 * (b4 + k) + 0] = buf[k].x;
-          vr[4 * (b4 + k) + 1] = buf[k].y;
-          vr[4 * (b4 + k) + 2] = buf[k].z;
-          vr[4 * (b4 + k) + 3] = buf[k].w;
-        }
+      for (int j = 0; j < 4; ++j) {
+        const int c = lane + 32 * j;
+        buf[i][j] = (r < m && c < bw) ? __ldg(Wp + r * n + j0 + c) : 0.f;
       }
-    } else {
-      for (int c = 0; c < SB; ++c) vr[c] = (c < bw) ? src[c] : 0.f;
     }
-  } else {
-    for (int c = 0; c < SB; ++c) vr[c] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) vals[(32 * warp + i0 + i) * LDV + lane + 32 * j] = buf[i][j];
   }
+  __syncwarp();
+  float* vr = vals + t * LDV;
 
   bool abort = !mbar_wait_bounded(pkg_bar, 0);
   if (abort) {
@@ -202,6 +208,7 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
       for (int k = 0; k < SS; ++k) v[k] = vr[k];
     } else {
       const bool ok = mbar_wait_bounded(mma_bar, (sb - 1) & 1);
+      if (t == 0) bulk_wait_read_all();   // the previous errors have left the A buffers
       if (__syncthreads_or(!ok)) {
         report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
         abort = true;
@@ -235,7 +242,7 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
       }
       if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
       s = __fdiv_rn(xmax - xmin, maxq);
-      z = rintf(__fdiv_rn(-xmin, s));
+      z = rintf(div_rn(-xmin, s));
       if (row < m) {
         const int64_t g = (j0 + c0) / group;
         scale[row * ngroups + g] = s;
@@ -247,7 +254,7 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
 #pragma unroll
     for (int i = 0; i < SS; ++i) {
       const int c = c0 + i;
-      float q = rintf(__fdiv_rn(v[i], s)) + z;
+      float q = rintf(div_rn(v[i], s)) + z;
       q = fminf(fmaxf(q, 0.f), maxq);
       const float ei = (v[i] - s * (q - z)) * rdiag[c];
       e[i] = ei;
@@ -263,36 +270,28 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
         if (4 * q4 + 3 > i) v[4 * q4 + 3] = fmaf(-ei, u.w, v[4 * q4 + 3]);
       }
     }
-    // ---- errors out: TF32 split to global (trailing update) and to the
-    // K-major swizzled A operand in shared memory (in-block far update)
+    // ---- errors out: TF32 split into the K-major swizzled A operand in
+    // shared memory, which feeds the in-block far update (tensor cores) and
+    // leaves for the trailing update as two TMA box stores
     float eh[SS], el[SS];
 #pragma unroll
     for (int k = 0; k < SS; ++k) {
       eh[k] = to_tf32(e[k]);
       el[k] = e[k] - eh[k];
     }
-    if (row < m) {
-      float4* gh = reinterpret_cast<float4*>(Ehi + row * SB + c0);
-      float4* gl = reinterpret_cast<float4*>(Elo + row * SB + c0);
 #pragma unroll
-      for (int q = 0; q < SS / 4; ++q) {
-        gh[q] = make_float4(eh[4 * q], eh[4 * q + 1], eh[4 * q + 2], eh[4 * q + 3]);
-        gl[q] = make_float4(el[4 * q], el[4 * q + 1], el[4 * q + 2], el[4 * q + 3]);
-      }
+    for (int q = 0; q < SS / 4; ++q) {
+      const uint32_t off = t * 128 + ((q ^ (t & 7)) << 4);
+      *reinterpret_cast<float4*>(ahi + off) =
+          make_float4(eh[4 * q], eh[4 * q + 1], eh[4 * q + 2], eh[4 * q + 3]);
+      *reinterpret_cast<float4*>(alo + off) =
+          make_float4(el[4 * q], el[4 * q + 1], el[4 * q + 2], el[4 * q + 3]);
     }
-    if (sb + 1 < nsb) {
-#pragma unroll
-      for (int q = 0; q < SS / 4; ++q) {
-        const uint32_t off = t * 128 + ((q ^ (t & 7)) << 4);
-        *reinterpret_cast<float4*>(ahi + off) =
-            make_float4(eh[4 * q], eh[4 * q + 1], eh[4 * q + 2], eh[4 * q + 3]);
-        *reinterpret_cast<float4*>(alo + off) =
-            make_float4(el[4 * q], el[4 * q + 1], el[4 * q + 2], el[4 * q + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (t == 0) {
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (t == 0) {
+      if (sb + 1 < nsb) {
         tc_fence_after();
         // D[:, 32(sb+1) : 128] += E·U[c0:c0+32, 32(sb+1):128]
         const uint32_t N = (uint32_t)(SB - SS * (sb + 1));
@@ -313,25 +312,39 @@ sweep_kernel(const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int
         }
         umma_commit(mma_bar);
       }
-      ++issued;
+      // the error buffers hold whole 128-row boxes (rows past m are zeros)
+      tma_store_2d(&tmEhi, c0, (int)r0, ahi);
+      tma_store_2d(&tmElo, c0, (int)r0, alo);
+      bulk_commit();
     }
+    if (sb + 1 < nsb) ++issued;
   }
   if (!abort && row < m && loss_row != nullptr) loss_row[row] += loss;
   tc_fence_before();
   __syncthreads();
 
-  // codes out, one warp per row, coalesced
+  // codes out, one warp per row, coalesced (four codes per lane and store
+  // when rows and the block width allow it; j0 is a multiple of 32)
   if (!abort) {
+    const bool wide = ((n & 3) == 0) && ((bw & 3) == 0);
     for (int rr = warp; rr < RT; rr += RT / 32) {
       const int64_t r = r0 + rr;
       if (r >= m) break;
+      if (wide) {
+        const int c = 4 * lane;
+        if (c < bw)
+          *reinterpret_cast<uint32_t*>(codes + r * n + j0 + c) =
+              *reinterpret_cast<const uint32_t*>(cs + rr * LDB + c);
+      } else {
 #pragma unroll
-      for (int it = 0; it < SB / 32; ++it) {
-        const int c = lane + 32 * it;
-        if (c < bw) codes[r * n + j0 + c] = cs[rr * LDB + c];
+        for (int it = 0; it < SB / 32; ++it) {
+          const int c = lane + 32 * it;
+          if (c < bw) codes[r * n + j0 + c] = cs[rr * LDB + c];
+        }
       }
     }
   }
+  if (t == 0) bulk_wait_all();          // the error boxes are in global memory
   if (abort && t == 0 && issued > 0)            // no MMA may still write TMEM
     mbar_wait_bounded(mma_bar, (issued - 1) & 1, 1u << 16);
   __syncthreads();
@@ -363,10 +376,15 @@ gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int 
                                    (int)SMEM_BYTES));
     g_attr_set = true;
   }
+  CUtensorMap th, tl;
+  const int64_t mr = error_rows(m);     // whole boxes: a clipped box store is slow
+  if (!encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ehi, SB, mr, SB * 4, SS, RT) ||
+      !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, SB * 4, SS, RT))
+    return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const unsigned grid = (unsigned)ceil_div(m, RT);
-  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, Wp, m, n, j0, bw,
+  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, Wp, m, n, j0, bw,
               reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
-              scale, zero, Ehi, Elo, loss_row, info);
+              scale, zero, loss_row, info);
   return GPTQ_OK;
 }
 

@@ -26,7 +26,6 @@
 //   4 warps        drain TMEM into swizzled shared boxes, then one TMA
 //                  reduce-add per 32-column box adds them into W.
 // Fallback: float32 SIMT tiles.
-#include <cudaTypedefs.h>
 
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -247,31 +246,10 @@ trailing_tc_kernel(const __grid_constant__ TrailMaps maps, int64_t m, int64_t n,
   if (warp == 0) tmem_dealloc(tmem, QN);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 bool encode_f32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
-             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  return encode_tiled_2d(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, inner, outer, row_bytes,
+                         box_inner, box_outer);
 }
 
 bool g_attr = false;
@@ -296,11 +274,12 @@ gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, const f
   if (c0 >= n || kw <= 0 || m <= 0) return GPTQ_OK;
   if (Uhi != nullptr && trailing_uses_tensor_cores(n, kw)) {
     TrailMaps maps;
-    bool ok = encode_f32(&maps.ahi, Ehi, SWEEP_BLOCK_MAX, m, SWEEP_BLOCK_MAX * 4, QK, QM) &&
-              encode_f32(&maps.alo, Elo, SWEEP_BLOCK_MAX, m, SWEEP_BLOCK_MAX * 4, QK, QM) &&
+    const int64_t mr = error_rows(m);
+    bool ok = encode_f32(&maps.ahi, Ehi, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
+              encode_f32(&maps.alo, Elo, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
               encode_f32(&maps.bhi, Uhi, n, n, n * 4, QK, QN) &&
               encode_f32(&maps.blo, Ulo, n, n, n * 4, QK, QN) &&
-              encode_f32(&maps.c, Wp, n, m, n * 4, 32, QM);
+              encode_f32(&maps.c, Wp, n, mr, n * 4, 32, QM);
     if (!ok) return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the trailing update");
     if (!g_attr) {
       GPTQ_CUDA(cudaFuncSetAttribute(trailing_tc_kernel,
