@@ -423,6 +423,26 @@ def run_ours(args, rank, world, local):
                 "launches_per_step": launches_per_step,
                 "share": round(tot[dom] / max(1e-9, sum(tot.values())), 4)}
 
+    # ---- the same figures for every kernel kind with a work model
+    kernels = {}
+    for k, (unit, amount) in work.items():
+        if k not in kprof or kprof[k][1] <= 0 or amount <= 0:
+            continue
+        per_step_ms = kprof[k][0] / args.steps
+        if unit == "TFLOP/s":
+            ach = amount / (per_step_ms / 1e3) / 1e12
+            if k == "hessian":
+                bound, peak = "tensor", peaks["bf16_tflops"]
+            else:
+                bound, peak = "alu", fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+        else:
+            ach = amount / (per_step_ms / 1e3) / 1e9
+            bound, peak = "hbm", peaks["hbm_gbs"]
+        kernels[k] = {"ms_per_step": round(per_step_ms, 4),
+                      "launches_per_step": kprof[k][1] / args.steps,
+                      "bound": bound, "achieved": round(ach, 2), "unit": unit,
+                      "peak": round(peak, 1), "frac": round(ach / peak, 4)}
+
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "params/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -438,6 +458,7 @@ def run_ours(args, rank, world, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "roofline": roof,
+        "kernels": kernels,
         "kernels_ms_per_step": {k: round(v / args.steps, 4) for k, v in tot.items() if v > 0},
         "clocks": clk,
     }

@@ -136,6 +136,33 @@ def test_not_positive_definite():
     assert e.value.status == 2
 
 
+@pytest.mark.parametrize("n,col", [(70, 5), (200, 3), (200, 190), (130, 64)])
+def test_not_positive_definite_index(n, col):
+    """The reported index is the processing position of the first bad pivot.
+
+    The factorisation runs on the reversed matrix, so the first pivot it meets
+    is the last processed column; with natural order a single negative
+    diagonal entry at `col` (and an identity elsewhere) is bad exactly there.
+    """
+    import post_weight_quantization_08_b200 as g
+    H = torch.eye(n, device=DEV)
+    H[col, col] = -1.0
+    out = g.prepare(H, 0.0, "natural", check=False)
+    st, idx = g.gptq_check(out["info"])
+    assert st == 2 and idx == col + 1
+
+
+def test_singular_block_is_not_positive_definite():
+    """Two identical columns with no damping: the second pivot is exactly 0."""
+    import post_weight_quantization_08_b200 as g
+    n = 96
+    H = torch.eye(n, device=DEV)
+    H[10, 10] = H[11, 11] = H[10, 11] = H[11, 10] = 2.0
+    out = g.prepare(H, 0.0, "natural", check=False)
+    st, idx = g.gptq_check(out["info"])
+    assert st == 2 and idx == 10 + 1
+
+
 def test_nonfinite_inputs():
     import post_weight_quantization_08_b200 as g
     n = 40
