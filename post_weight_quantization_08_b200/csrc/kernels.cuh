@@ -42,12 +42,12 @@ bool trailing_uses_tensor_cores(int64_t n, int block);
 gptq_status launch_split_tf32_t(const float* x, int64_t n, float* hiT, float* loT,
                                 cudaStream_t s);
 
-// Wp[:, c0:n] −= (Ehi+Elo)[:, 0:kw]·U[k0:k0+kw, c0:n]   (lazy-batch update).
-// With UhiT/UloT (the transposed TF32 split of U) the product runs on the
-// tensor cores.
-gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, const float* Ehi,
-                            const float* Elo, int64_t k0, int kw, const float* U,
-                            const float* Uhi, const float* Ulo, int32_t* info,
+// Wp[:, c0:c1] −= (Ehi+Elo)[:, 0:kw]·U[k0:k0+kw, c0:c1]   (lazy-batch update;
+// c1 is clipped to n).  With UhiT/UloT (the transposed TF32 split of U) the
+// product runs on the tensor cores.
+gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, int64_t c1,
+                            const float* Ehi, const float* Elo, int64_t k0, int kw,
+                            const float* U, const float* Uhi, const float* Ulo, int32_t* info,
                             cudaStream_t s);
 
 }  // namespace gptq

@@ -7,6 +7,10 @@
 // Schritt 3 (GPTQ's groups run along the input channels).
 #include <cuda_bf16.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "kernels.cuh"
 
 namespace gptq {
@@ -15,8 +19,8 @@ namespace {
 struct QuantWs {
   float* Wp;        // error_rows(m) × n working copy, processing order
   uint8_t* codes;   // m × n codes, processing order
-  float* Ehi;       // m × 128 scaled errors of the current block, TF32 part
-  float* Elo;       // m × 128 remainder e − Ehi
+  float* Ehi[2];    // error_rows(m) × 128 scaled errors of a block, TF32 part
+  float* Elo[2];    // remainder e − Ehi; two sets, alternating by block
   int32_t* pinv;    // n: processing position of each original column
   float* panels;    // pre-transposed U panels, one per block
   float* Uhi;       // n × n TF32 part of Uᵀ (tensor-core trailing update only)
@@ -35,8 +39,8 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   const size_t mrows = (size_t)error_rows(m);
   size_t o_wp = take(sizeof(float) * mrows * (size_t)n);
   size_t o_codes = take((size_t)m * (size_t)n);
-  size_t o_ehi = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
-  size_t o_elo = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
+  size_t o_e[4];
+  for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
   size_t o_pinv = take(sizeof(int32_t) * (size_t)n);
   size_t o_pan = take(panel_workspace_bytes(n, block));
   const bool tc = trailing_uses_tensor_cores(n, block);
@@ -45,8 +49,10 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   if (w && base) {
     w->Wp = reinterpret_cast<float*>(base + o_wp);
     w->codes = reinterpret_cast<uint8_t*>(base + o_codes);
-    w->Ehi = reinterpret_cast<float*>(base + o_ehi);
-    w->Elo = reinterpret_cast<float*>(base + o_elo);
+    for (int k = 0; k < 2; ++k) {
+      w->Ehi[k] = reinterpret_cast<float*>(base + o_e[2 * k]);
+      w->Elo[k] = reinterpret_cast<float*>(base + o_e[2 * k + 1]);
+    }
     w->pinv = reinterpret_cast<int32_t*>(base + o_pinv);
     w->panels = reinterpret_cast<float*>(base + o_pan);
     w->Uhi = tc ? reinterpret_cast<float*>(base + o_uhi) : nullptr;
@@ -57,6 +63,32 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// The far part of each trailing update runs on a side stream of the caller's
+// stream, so that it overlaps the next block's sweep; one side stream and two
+// events per (device, caller stream), created on first use and kept for the
+// life of the process.
+struct SideStream {
+  cudaStream_t s2 = nullptr;
+  cudaEvent_t swept = nullptr;   // recorded on the caller's stream after a sweep
+  cudaEvent_t far = nullptr;     // recorded on the side stream after a far update
+};
+
+gptq_status side_stream_for(cudaStream_t s, SideStream** out) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, SideStream> reg;
+  int dev = 0;
+  GPTQ_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(mu);
+  SideStream& e = reg[{dev, s}];
+  if (e.s2 == nullptr) {
+    GPTQ_CUDA(cudaStreamCreateWithFlags(&e.s2, cudaStreamNonBlocking));
+    GPTQ_CUDA(cudaEventCreateWithFlags(&e.swept, cudaEventDisableTiming));
+    GPTQ_CUDA(cudaEventCreateWithFlags(&e.far, cudaEventDisableTiming));
+  }
+  *out = &e;
+  return GPTQ_OK;
+}
 
 // pinv[perm[p]] = p and g_idx[perm[p]] = p / group.
 __global__ void __launch_bounds__(256)
@@ -188,24 +220,54 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
     GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<float>, gin, 256, 0,
                 static_cast<const float*>(W), m, n, perm, dead, w.Wp, info);
 
+  // padding rows of the working copy: zero, so that the last row box of
+  // every sweep and trailing update reads defined values
+  if (error_rows(m) > m)
+    GPTQ_CUDA(cudaMemsetAsync(w.Wp + m * n, 0, sizeof(float) * (size_t)(error_rows(m) - m) * n, s));
   gptq_status st = launch_panels(U, n, block, w.panels, s);
   if (st != GPTQ_OK) return st;
   if (w.Uhi != nullptr && n > block) {
     st = launch_split_tf32_t(U, n, w.Uhi, w.Ulo, s);
     if (st != GPTQ_OK) return st;
   }
-  for (int64_t j0 = 0; j0 < n; j0 += block) {
+  // Block b: sweep, then the update of block b+1's columns on the caller's
+  // stream (the next sweep waits for it), and the update of the columns after
+  // that on the side stream, overlapping sweep b+1.  Every column still
+  // receives the blocks' contributions in block order: the update of block
+  // b+1's columns by block b waits for the far update of block b−1, and the
+  // two error buffers alternate so that a far update's input is not
+  // overwritten by the next sweep.
+  SideStream* side = nullptr;
+  st = side_stream_for(s, &side);
+  if (st != GPTQ_OK) return st;
+  bool far_pending = false;
+  for (int64_t j0 = 0, b = 0; j0 < n; j0 += block, ++b) {
     const int bw = (int)((n - j0 < block) ? (n - j0) : block);
+    float* ehi = w.Ehi[b & 1];
+    float* elo = w.Elo[b & 1];
     const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
     st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes, scale,
-                      zero, w.Ehi, w.Elo, loss_row, info, s);
+                      zero, ehi, elo, loss_row, info, s);
     if (st != GPTQ_OK) return st;
-    if (j0 + bw < n) {
-      st = launch_trailing(w.Wp, m, n, j0 + bw, w.Ehi, w.Elo, j0, bw, U, w.Uhi, w.Ulo, info,
-                           s);
+    const int64_t c0 = j0 + bw, c1 = c0 + block;
+    if (c0 >= n) break;
+    if (c1 < n) {
+      GPTQ_CUDA(cudaEventRecord(side->swept, s));
+      GPTQ_CUDA(cudaStreamWaitEvent(side->s2, side->swept, 0));
+    }
+    if (far_pending) GPTQ_CUDA(cudaStreamWaitEvent(s, side->far, 0));
+    st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info, s);
+    if (st != GPTQ_OK) return st;
+    far_pending = false;
+    if (c1 < n) {
+      st = launch_trailing(w.Wp, m, n, c1, n, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info,
+                           side->s2);
       if (st != GPTQ_OK) return st;
+      GPTQ_CUDA(cudaEventRecord(side->far, side->s2));
+      far_pending = true;
     }
   }
+  if (far_pending) GPTQ_CUDA(cudaStreamWaitEvent(s, side->far, 0));
 
   const unsigned gpk = (unsigned)ceil_div(m * ceil_div(n, 32), 256);
   switch (bits) {

@@ -28,6 +28,8 @@
 // first column, the range always containing 0; decisions in IEEE float32
 // (correctly rounded division and rint, no fast-math).  The block's errors
 // also leave as a TF32 split (Ehi, Elo) for the trailing update.
+#include <cstring>
+
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -37,7 +39,6 @@ namespace {
 constexpr int SB = 128;       // largest block width
 constexpr int SS = 32;        // sub-block
 constexpr int RT = 128;       // rows (threads) per CTA
-constexpr int LDV = SB + 1;   // row-major values, odd stride: conflict-free columns
 constexpr int LDB = SB + 4;   // bytes per staged code row
 
 // package layout (bytes)
@@ -59,10 +60,19 @@ constexpr uint32_t SM_PKG = 0;
 constexpr uint32_t SM_AHI = 66560;                 // 65 KB, 1024-aligned
 constexpr uint32_t SM_ALO = SM_AHI + RT * 128;
 constexpr uint32_t SM_VALS = SM_ALO + RT * 128;
-constexpr uint32_t SM_CODES = SM_VALS + RT * LDV * 4;
+constexpr uint32_t VBOX = RT * 128;                // 128 rows × 32 floats, swizzled
+constexpr uint32_t SM_CODES = SM_VALS + 4 * VBOX;
 constexpr uint32_t SM_BARS = (SM_CODES + RT * LDB + 15) / 16 * 16;
 constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 32;
 static_assert(SM_AHI >= PK_BYTES && SM_AHI % 1024 == 0, "A operand placement");
+static_assert(SM_VALS % 1024 == 0, "the strip's boxes use the 128-byte swizzle");
+
+// The block's strip of Wp in shared memory: four boxes of 32 columns × 128
+// rows with the TMA 128-byte swizzle, the 16-byte chunk j of row r at
+// r·128 + ((j ^ (r mod 8))·16).  Chunk j of row r, box q:
+__device__ __forceinline__ float4 strip_chunk(const unsigned char* vals, int q, int r, int j) {
+  return *reinterpret_cast<const float4*>(vals + q * VBOX + r * 128 + ((j ^ (r & 7)) << 4));
+}
 
 // Package of block b.  blockIdx.y: 0..5 a B box (hi and lo), 6..9 a diagonal
 // piece, 10 the reciprocal diagonals.  Box (s,t) holds, in K-major 128-byte
@@ -123,8 +133,22 @@ __device__ __forceinline__ float div_rn(float x, float s) {
   return x == 0.f ? x : q;
 }
 
+// x/s correctly rounded from rs = RN(1/s) by Markstein's FMA correction
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", 1990): q0 = RN(x·rs), r = x − q0·s (exact by FMA),
+// RN(q0 + r·rs) = RN(x/s) when the reciprocal is correctly rounded and nothing
+// under- or overflows.  Three dependent operations and no branch, where the
+// column chain needs it most.  rs is capped at the largest float, so a zero x
+// still gives a zero quotient for a pathologically small s.
+__device__ __forceinline__ float div_fma(float x, float s, float rs) {
+  const float q0 = x * rs;
+  const float r = fmaf(-q0, s, x);
+  return fmaf(r, rs, q0);
+}
+
 __global__ void __launch_bounds__(RT, 1)
 sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
+             const __grid_constant__ CUtensorMap tmW, int strip_tma,
              const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
              const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
              uint8_t* __restrict__ codes, float* __restrict__ scale,
@@ -136,7 +160,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   const float* rdiag = reinterpret_cast<const float*>(sm + SM_PKG + PK_RD);
   unsigned char* ahi = sm + SM_AHI;
   unsigned char* alo = sm + SM_ALO;
-  float* vals = reinterpret_cast<float*>(sm + SM_VALS);
+  unsigned char* vals = sm + SM_VALS;
   uint8_t* cs = sm + SM_CODES;
   uint64_t* pkg_bar = reinterpret_cast<uint64_t*>(sm + SM_BARS);
   uint64_t* mma_bar = pkg_bar + 1;
@@ -161,33 +185,47 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   const uint32_t tmem = *tslot;
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
   if (t == 0) {
-    mbar_arrive_expect_tx(pkg_bar, PK_BYTES);
+    // the package and, when the rows allow a tensor map, the strip: four
+    // boxes at (j0 + 32q, r0); columns past n read as zero, and Wp holds whole
+    // 128-row boxes
+    mbar_arrive_expect_tx(pkg_bar, PK_BYTES + (strip_tma ? 4 * VBOX : 0));
     bulk_g2s(sm + SM_PKG, pkg, PK_BYTES, pkg_bar);
+    if (strip_tma) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tma_load_2d(vals + q * VBOX, &tmW, (int)j0 + 32 * q, (int)r0, pkg_bar);
+    }
   }
 
-  // the CTA's rows of the block → vals (row-major, odd stride): warp w
-  // reads rows 32w .. 32w+31 with lanes along the columns (coalesced 128-byte
-  // reads, conflict-free shared-memory writes); rows past m and columns past
-  // the block are zero
+  if (!strip_tma) {
+    // rows of n % 4 ≠ 0 floats: warp w reads rows 32w .. 32w+31 with lanes
+    // along the columns (coalesced) into the same swizzled layout; rows past
+    // m and columns past the block are zero
 #pragma unroll 1
-  for (int i0 = 0; i0 < 32; i0 += 8) {
-    float buf[8][4];
+    for (int i0 = 0; i0 < 32; i0 += 8) {
+      float buf[8][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t r = r0 + 32 * warp + i0 + i;
+      for (int i = 0; i < 8; ++i) {
+        const int64_t r = r0 + 32 * warp + i0 + i;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = lane + 32 * j;
-        buf[i][j] = (r < m && c < bw) ? __ldg(Wp + r * n + j0 + c) : 0.f;
+        for (int j = 0; j < 4; ++j) {
+          const int c = lane + 32 * j;
+          buf[i][j] = (r < m && c < bw) ? __ldg(Wp + r * n + j0 + c) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 32 * warp + i0 + i;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int cc = lane;       // column 32j + lane: box j, chunk lane/4
+          *reinterpret_cast<float*>(vals + j * VBOX + rr * 128 + (((cc >> 2) ^ (rr & 7)) << 4) +
+                                    (cc & 3) * 4) = buf[i][j];
+        }
       }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) vals[(32 * warp + i0 + i) * LDV + lane + 32 * j] = buf[i][j];
+    __syncthreads();
   }
-  __syncwarp();
-  float* vr = vals + t * LDV;
 
   bool abort = !mbar_wait_bounded(pkg_bar, 0);
   if (abort) {
@@ -196,7 +234,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   }
 
   const float maxq = (float)((1 << bits) - 1);
-  float s = 1.f, z = 0.f, loss = 0.f;
+  float s = 1.f, z = 0.f, loss = 0.f, rs = 1.f, klo = 0.f, khi = maxq;
   uint8_t* cr = cs + t * LDB;
   const int nsb = (bw + SS - 1) / SS;
   int issued = 0;                       // MMA groups committed to mma_bar
@@ -205,7 +243,13 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
     float v[SS], e[SS];
     if (sb == 0) {
 #pragma unroll
-      for (int k = 0; k < SS; ++k) v[k] = vr[k];
+      for (int j = 0; j < SS / 4; ++j) {
+        const float4 f = strip_chunk(vals, 0, t, j);
+        v[4 * j] = f.x;
+        v[4 * j + 1] = f.y;
+        v[4 * j + 2] = f.z;
+        v[4 * j + 3] = f.w;
+      }
     } else {
       const bool ok = mbar_wait_bounded(mma_bar, (sb - 1) & 1);
       if (t == 0) bulk_wait_read_all();   // the previous errors have left the A buffers
@@ -218,7 +262,13 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
       float d[32];
       tmem_ld_32x32b_x32(trow + c0, d);
 #pragma unroll
-      for (int k = 0; k < SS; ++k) v[k] = vr[c0 + k] - d[k];
+      for (int j = 0; j < SS / 4; ++j) {
+        const float4 f = strip_chunk(vals, sb, t, j);
+        v[4 * j] = f.x - d[4 * j];
+        v[4 * j + 1] = f.y - d[4 * j + 1];
+        v[4 * j + 2] = f.z - d[4 * j + 2];
+        v[4 * j + 3] = f.w - d[4 * j + 3];
+      }
     }
     if (c0 % group == 0) {
       // the group's current values: this sub-block, then later ones in the group
@@ -234,15 +284,24 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
         float d[32];
         if (sb > 0) tmem_ld_32x32b_x32(trow + cs0, d);
 #pragma unroll
-        for (int k = 0; k < SS; ++k) {
-          const float x = (cs0 + k < gend) ? vr[cs0 + k] - (sb > 0 ? d[k] : 0.f) : 0.f;
-          xmin = fminf(xmin, x);
-          xmax = fmaxf(xmax, x);
+        for (int j = 0; j < SS / 4; ++j) {
+          const float4 f = strip_chunk(vals, cs0 / SS, t, j);
+          const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int k = 4 * j + k4;
+            const float x = (cs0 + k < gend) ? fv[k4] - (sb > 0 ? d[k] : 0.f) : 0.f;
+            xmin = fminf(xmin, x);
+            xmax = fmaxf(xmax, x);
+          }
         }
       }
       if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
       s = __fdiv_rn(xmax - xmin, maxq);
+      rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
       z = rintf(div_rn(-xmin, s));
+      klo = -z;
+      khi = maxq - z;
       if (row < m) {
         const int64_t g = (j0 + c0) / group;
         scale[row * ngroups + g] = s;
@@ -254,12 +313,13 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
 #pragma unroll
     for (int i = 0; i < SS; ++i) {
       const int c = c0 + i;
-      float q = rintf(div_rn(v[i], s)) + z;
-      q = fminf(fmaxf(q, 0.f), maxq);
-      const float ei = (v[i] - s * (q - z)) * rdiag[c];
+      // q − z = clamp(rint(v/s), −z, maxq − z) exactly (small integers), so
+      // the clamp works on k = q − z and the error takes one FMA
+      const float k = fminf(fmaxf(rintf(div_fma(v[i], s, rs)), klo), khi);
+      const float ei = fmaf(-s, k, v[i]) * rdiag[c];
       e[i] = ei;
       loss = fmaf(ei, ei, loss);
-      cr[c] = (uint8_t)q;
+      cr[c] = (uint8_t)(k + z);
       const float4* ur = reinterpret_cast<const float4*>(ud + i * SS);
 #pragma unroll
       for (int q4 = (i + 1) / 4; q4 < SS / 4; ++q4) {
@@ -378,11 +438,18 @@ gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int 
   }
   CUtensorMap th, tl;
   const int64_t mr = error_rows(m);     // whole boxes: a clipped box store is slow
+  CUtensorMap tw;
+  const int strip_tma = ((n & 3) == 0) ? 1 : 0;   // row pitch a multiple of 16 bytes
+  if (strip_tma &&
+      !encode_tiled_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Wp, n, mr, n * 4, SS, RT))
+    return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's strip");
+  if (!strip_tma) memset(&tw, 0, sizeof(tw));
   if (!encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ehi, SB, mr, SB * 4, SS, RT) ||
       !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, SB * 4, SS, RT))
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const unsigned grid = (unsigned)ceil_div(m, RT);
-  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, Wp, m, n, j0, bw,
+  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, tw, strip_tma, Wp, m,
+              n, j0, bw,
               reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
               scale, zero, loss_row, info);
   return GPTQ_OK;

@@ -38,7 +38,7 @@ namespace {
 constexpr int TM = 128, TN = 128, TK = 16;
 
 __global__ void __launch_bounds__(256)
-trailing_simt_kernel(float* __restrict__ Wp, int64_t m, int64_t n, int64_t c0,
+trailing_simt_kernel(float* __restrict__ Wp, int64_t m, int64_t n, int64_t c0, int64_t c1,
                      const float* __restrict__ Ehi, const float* __restrict__ Elo,
                      int64_t k0, int kw, const float* __restrict__ U) {
   __shared__ __align__(16) float as[TK][TM];
@@ -55,7 +55,7 @@ trailing_simt_kernel(float* __restrict__ Wp, int64_t m, int64_t n, int64_t c0,
     }
     for (int e = tid; e < TK * TN; e += 256) {
       const int kk = e / TN, c = e % TN;
-      bs[kk][c] = (kb + kk < kw && cb + c < n) ? U[(k0 + kb + kk) * n + cb + c] : 0.f;
+      bs[kk][c] = (kb + kk < kw && cb + c < c1) ? U[(k0 + kb + kk) * n + cb + c] : 0.f;
     }
     __syncthreads();
 #pragma unroll
@@ -82,7 +82,7 @@ trailing_simt_kernel(float* __restrict__ Wp, int64_t m, int64_t n, int64_t c0,
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t c = cb + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
-      if (c < n) Wp[r * n + c] -= acc[i][j];
+      if (c < c1) Wp[r * n + c] -= acc[i][j];
     }
   }
 }
@@ -132,7 +132,7 @@ struct TrailMaps {
 
 __global__ void __launch_bounds__(128, 1)
 trailing_tc_kernel(const __grid_constant__ TrailMaps maps, int64_t m, int64_t n, int64_t c0,
-                   int64_t k0, int kw, int32_t* info) {
+                   int64_t c1, int64_t k0, int kw, int32_t* info) {
   extern __shared__ unsigned char smraw[];
   const uint32_t raw = smem_addr(smraw);
   unsigned char* ring = smraw + ((1024 - (raw & 1023)) & 1023);
@@ -238,7 +238,7 @@ trailing_tc_kernel(const __grid_constant__ TrailMaps maps, int64_t m, int64_t n,
   if (write && tid == 0) {
 #pragma unroll 1
     for (int b = 0; b < QN / 32; ++b)
-      if ((int64_t)cb + 32 * b < n) tma_reduce_add_2d(&maps.c, cb + 32 * b, r0, ring + b * C_BOX);
+      if ((int64_t)cb + 32 * b < c1) tma_reduce_add_2d(&maps.c, cb + 32 * b, r0, ring + b * C_BOX);
     bulk_commit();
     bulk_wait_all();
   }
@@ -267,11 +267,12 @@ gptq_status launch_split_tf32_t(const float* x, int64_t n, float* hiT, float* lo
   return GPTQ_OK;
 }
 
-gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, const float* Ehi,
-                            const float* Elo, int64_t k0, int kw, const float* U,
-                            const float* Uhi, const float* Ulo, int32_t* info,
+gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, int64_t c1,
+                            const float* Ehi, const float* Elo, int64_t k0, int kw,
+                            const float* U, const float* Uhi, const float* Ulo, int32_t* info,
                             cudaStream_t s) {
-  if (c0 >= n || kw <= 0 || m <= 0) return GPTQ_OK;
+  if (c1 > n) c1 = n;
+  if (c0 >= c1 || kw <= 0 || m <= 0) return GPTQ_OK;
   if (Uhi != nullptr && trailing_uses_tensor_cores(n, kw)) {
     TrailMaps maps;
     const int64_t mr = error_rows(m);
@@ -286,13 +287,13 @@ gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, const f
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QSMEM));
       g_attr = true;
     }
-    const dim3 grid((unsigned)ceil_div(n - c0, QN), (unsigned)ceil_div(m, QM));
-    GPTQ_LAUNCH(KK_TRAIL, s, trailing_tc_kernel, grid, 128, QSMEM, maps, m, n, c0, k0, kw,
+    const dim3 grid((unsigned)ceil_div(c1 - c0, QN), (unsigned)ceil_div(m, QM));
+    GPTQ_LAUNCH(KK_TRAIL, s, trailing_tc_kernel, grid, 128, QSMEM, maps, m, n, c0, c1, k0, kw,
                 info);
     return GPTQ_OK;
   }
-  const dim3 grid((unsigned)ceil_div(n - c0, TN), (unsigned)ceil_div(m, TM));
-  GPTQ_LAUNCH(KK_TRAIL, s, trailing_simt_kernel, grid, 256, 0, Wp, m, n, c0, Ehi, Elo, k0,
+  const dim3 grid((unsigned)ceil_div(c1 - c0, TN), (unsigned)ceil_div(m, TM));
+  GPTQ_LAUNCH(KK_TRAIL, s, trailing_simt_kernel, grid, 256, 0, Wp, m, n, c0, c1, Ehi, Elo, k0,
               kw, U);
   return GPTQ_OK;
 }
