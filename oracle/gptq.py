@@ -20,7 +20,8 @@ Sources (page title, then the place on the page)
      Algorithm" (gist.science summary), §2.1 (layer-output L2 error as a CVP
      on the lattice B = X·diag(s), Satz 1), §2.2 (Satz 4: GPTQ run back to
      front is Babai's nearest-plane algorithm), §2.3 (Satz 5 bound; act-order
-     is the descending Hessian diagonal).
+     is the descending Hessian diagonal; the min-pivot order takes the
+     smallest diagonal entry at every LDL step, to shrink the trace of D).
 
 Readings taken where the pages are silent or disagree
 -----------------------------------------------------
@@ -43,13 +44,19 @@ Readings taken where the pages are silent or disagree
   the damping is taken before that fix.
 * act-order sorts the Hessian diagonal (dead entries read as 1) in descending
   order; equal entries keep ascending column index.
+* min-pivot order: the D of Satz 5 comes from the LDL factorisation that
+  eliminates the last processed column first (1/U_jj² are its pivots), so the
+  column eliminated at step t is processed at position n−1−t.  Each step takes
+  the smallest diagonal entry of the current Schur complement of the damped,
+  dead-fixed H_d; equal entries go to the larger column index, so that a
+  diagonal H gives act-order and H = I the natural order.
 """
 from __future__ import annotations
 
 import numpy as np
 from scipy.linalg import solve_triangular
 
-ORDERS = ("natural", "act", "reverse", "custom")
+ORDERS = ("natural", "act", "reverse", "custom", "minpivot")
 
 
 # --------------------------------------------------------------------------
@@ -81,13 +88,43 @@ def damp_and_fix(H, damp: float):
     return H, dead, mean_diag
 
 
-def order_permutation(H, dead, order: str, perm=None) -> np.ndarray:
+def min_pivot_order(Hd) -> np.ndarray:
+    """Processing order of the min-pivot rule ([P2] §2.3, "Rolle der Reihenfolge").
+
+    Symmetric elimination of H_d, one column at a time: take the remaining
+    column with the smallest Schur-complement diagonal (ties: the larger
+    column index), then S ← S − s_j·s_jᵀ/S_jj.  The column eliminated at step t
+    is processed at position n−1−t.  Raises LinAlgError on a pivot ≤ 0.
+    """
+    S = np.array(Hd, dtype=np.float64, copy=True)
+    n = S.shape[0]
+    alive = np.ones(n, dtype=bool)
+    elim = np.empty(n, dtype=np.int64)
+    for t in range(n):
+        d = np.where(alive, np.diag(S), np.inf)
+        dmin = d.min()
+        if not dmin > 0.0:
+            raise np.linalg.LinAlgError(f"min-pivot order: pivot {dmin} at step {t}")
+        j = int(np.flatnonzero(d == dmin)[-1])
+        elim[t] = j
+        alive[j] = False
+        col = S[:, j].copy()
+        S -= np.outer(col, col) / col[j]
+    return elim[::-1].copy()
+
+
+def order_permutation(H, dead, order: str, perm=None, Hd=None) -> np.ndarray:
     """Processing order: perm[p] = original column processed at position p.
 
     natural: 0..n−1.  reverse: n−1..0 ([P2] §2.2, Satz 4).  act: descending
     Hessian diagonal ([P1] Schritt 2 "act-order"; [P2] §2.3).  custom: given.
+    minpivot: the min-pivot rule on the damped H_d ([P2] §2.3).
     """
     n = H.shape[0]
+    if order == "minpivot":
+        if Hd is None:
+            raise ValueError("the min-pivot order needs the damped Hessian")
+        return min_pivot_order(Hd)
     if order == "natural":
         return np.arange(n, dtype=np.int64)
     if order == "reverse":
@@ -122,7 +159,7 @@ def prepare(H, damp: float = 0.01, order: str = "natural", perm=None) -> dict:
     """Damp, fix dead columns, order, and factor: the whole prepare step."""
     H = np.asarray(H, dtype=np.float64)
     Hd, dead, mean_diag = damp_and_fix(H, damp)
-    perm = order_permutation(H, dead, order, perm)
+    perm = order_permutation(H, dead, order, perm, Hd=Hd)
     Hp = Hd[np.ix_(perm, perm)]
     U = inverse_cholesky_upper(Hp)
     return {"U": U, "perm": perm, "dead": dead, "Hd": Hd, "Hp": Hp,

@@ -408,3 +408,88 @@ def test_pins_catch_planted_mistakes(kind):
             caught = True
             break
     assert caught, kind
+
+
+# ---------------------------------------------------------------- min-pivot order
+
+def _schur_diagonal(H, eliminated):
+    """diag(H_RR − H_RE·H_EE⁻¹·H_ER) over the remaining columns R, by a solve."""
+    n = H.shape[0]
+    E = np.array(eliminated, dtype=np.int64)
+    R = np.array([i for i in range(n) if i not in set(eliminated)], dtype=np.int64)
+    if len(E) == 0:
+        return R, np.diag(H)[R].copy()
+    X = np.linalg.solve(H[np.ix_(E, E)], H[np.ix_(E, R)])
+    return R, np.diag(H[np.ix_(R, R)] - H[np.ix_(R, E)] @ X).copy()
+
+
+def test_min_pivot_golden(golden):
+    for (n,), flat, want in golden("min_pivot_order.txt"):
+        n = int(n)
+        H = np.array([float(v) for v in flat]).reshape(n, n)
+        want = [int(v) for v in want]
+        assert og.min_pivot_order(H).tolist() == want
+        assert og.prepare(H, 0.0, "minpivot")["perm"].tolist() == want
+
+
+def test_min_pivot_diagonal_is_act_order():
+    """On a diagonal H (ties and a dead column included) min-pivot = act-order."""
+    rng = np.random.default_rng(41)
+    for trial in range(20):
+        n = 40
+        d = rng.choice([0.5, 1.0, 2.0, 3.5, 7.0], size=n)
+        d[rng.integers(n)] = 0.0                      # a dead column
+        H = np.diag(d)
+        a = og.prepare(H, 0.01, "act")["perm"]
+        b = og.prepare(H, 0.01, "minpivot")["perm"]
+        assert np.array_equal(a, b)
+
+
+def test_min_pivot_takes_the_schur_minimum():
+    """Every step eliminates the smallest Schur-complement diagonal.
+
+    The Schur complements are recomputed from scratch with a linear solve
+    (not the oracle's rank-1 updates), and the LDL pivots 1/U_jj² of the
+    resulting order are those minima.
+    """
+    rng = np.random.default_rng(42)
+    for trial in range(6):
+        n = 14
+        H = _spd(n, rng)
+        p = og.prepare(H, 0.01, "minpivot")
+        Hd = p["Hd"]
+        elim = p["perm"][::-1]
+        pivots = []
+        for t in range(n):
+            R, sd = _schur_diagonal(Hd, list(elim[:t]))
+            k = int(np.flatnonzero(R == elim[t])[0])
+            assert sd[k] <= sd.min() * (1 + 1e-12)
+            pivots.append(sd[k])
+        assert np.allclose(1.0 / np.diag(p["U"]) ** 2, np.array(pivots)[::-1], rtol=1e-9)
+
+
+def test_min_pivot_catches_planted_mistakes(golden):
+    """A largest-pivot rule or a rule on the undamped, un-updated diagonal fails."""
+    rows = golden("min_pivot_order.txt")
+    (n,), flat, want = rows[1]
+    H = np.array([float(v) for v in flat]).reshape(int(n), int(n))
+    want = [int(v) for v in want]
+
+    def largest(Hd):
+        S = np.array(Hd, dtype=np.float64, copy=True)
+        alive = np.ones(S.shape[0], bool)
+        elim = []
+        for _ in range(S.shape[0]):
+            d = np.where(alive, np.diag(S), -np.inf)
+            j = int(np.flatnonzero(d == d.max())[-1])
+            elim.append(j)
+            alive[j] = False
+            c = S[:, j].copy()
+            S -= np.outer(c, c) / c[j]
+        return elim[::-1]
+
+    def static_diagonal(Hd):                     # no Schur updates
+        return list(np.argsort(np.diag(Hd), kind="stable")[::-1])
+
+    assert largest(H) != want
+    assert static_diagonal(H) != want
