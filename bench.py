@@ -66,14 +66,15 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def workload_name(cid: int, bits: int) -> str:
+def workload_name(cid: int, bits: int, order: str | None = None) -> str:
     c = CONFIGS[cid]
+    tail = "" if order is None else f", {order} order"
     if c["kind"] == "decoder":
         h, kv, it = c["hidden"], c["kv"], c["inter"]
         rows = 2 * h + 2 * kv + 2 * it
         return (f"{c['name']}: q/k/v/o/gate/up {rows}x{h} on one H + down {h}x{it}, "
-                f"T={c['T']} cone tokens, {bits}-bit g128 b128 damp0.01, per layer")
-    return f"{c['name']}: W {c['m']}x{c['n']}, T={c['T']}, {bits}-bit g128 b128 damp0.01"
+                f"T={c['T']} cone tokens, {bits}-bit g128 b128 damp0.01, per layer{tail}")
+    return f"{c['name']}: W {c['m']}x{c['n']}, T={c['T']}, {bits}-bit g128 b128 damp0.01{tail}"
 
 
 # ---------------------------------------------------------------- clocks
@@ -292,7 +293,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(device)
     cfg = CONFIGS[args.config]
     bits = args.bits or cfg["bits"][0]
-    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits)
+    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits, order=args.order)
     layer = Layer(probs, device)
     params = sum(p.params for p in probs)
     main = torch.cuda.Stream(device=device)     # non-default: graphs capture here
@@ -419,7 +420,7 @@ def run_ours(args, rank, world, local):
         roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2),
                 "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
                 "peak_source": note,
-                "traffic": traffic_for(dom, workload_name(args.config, bits)),
+                "traffic": traffic_for(dom, workload_name(args.config, bits, args.order)),
                 "launches_per_step": launches_per_step,
                 "share": round(tot[dom] / max(1e-9, sum(tot.values())), 4)}
 
@@ -449,7 +450,7 @@ def run_ours(args, rank, world, local):
         "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": workload_name(args.config, bits), "params_per_step_per_gpu": params,
+        "config": {"workload": workload_name(args.config, bits, args.order), "params_per_step_per_gpu": params,
                    "global_batch": len(probs) * world, "seq_len": probs[0].T,
                    "parallelism": f"independent layers x{world}",
                    "l2": "flushed between timed steps (256 MB write)",
@@ -509,7 +510,7 @@ def run_reference(args, rank, world):
         return None
     cfg = CONFIGS[args.config]
     bits = args.bits or cfg["bits"][0]
-    probs = problems_for(args.config, layer=0, bits=bits)
+    probs = problems_for(args.config, layer=0, bits=bits, order=args.order)
     for _ in range(args.warmup):
         oracle_pass(probs)
     t0 = time.perf_counter()
@@ -525,7 +526,7 @@ def run_reference(args, rank, world):
         "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": workload_name(args.config, bits)},
+        "config": {"workload": workload_name(args.config, bits, args.order)},
         "cpu_baseline": {"value": round(value, 1), "unit": "params/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"{args.steps} timed passes of one layer on the host cores"},
@@ -544,6 +545,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--order", default=None,
+                    choices=["natural", "act", "reverse", "minpivot"],
+                    help="processing order for every problem (default: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -59,7 +59,14 @@ typedef enum {
                               Babai page, §2.3, defines it by the diagonal)   */
   GPTQ_ORDER_REVERSE = 2,  /* columns n−1..0: back to front, the order in which
                               GPTQ is Babai's algorithm (Babai page, §2.2)    */
-  GPTQ_ORDER_CUSTOM = 3    /* caller's permutation, read from `perm`          */
+  GPTQ_ORDER_CUSTOM = 3,   /* caller's permutation, read from `perm`          */
+  GPTQ_ORDER_MINPIVOT = 4  /* min-pivot: the LDL of Satz 5 takes the smallest
+                              Schur-complement diagonal of H_d at every step
+                              (Babai page, §2.3); that LDL eliminates the last
+                              processed column first, so the column eliminated
+                              at step t is processed at position n−1−t; equal
+                              entries go to the larger column index;
+                              n ≤ 16384, else UNSUPPORTED                     */
 } gptq_order;
 
 typedef enum {
@@ -107,11 +114,13 @@ size_t gptq_prepare_workspace_bytes(int64_t n);
  *   dead   uint8[n], device, output: 1 where H_jj == 0.
  *   info   int32[2], device, output: {status, index}; NOT_PD sets index to
  *          the failing pivot (processing position) + 1; NONFINITE to the
- *          flattened index + 1 of a NaN/Inf entry of H.
+ *          flattened index + 1 of a NaN/Inf entry of H.  With MINPIVOT a pivot
+ *          ≤ 0 met while choosing the order is reported the same way.
  *   ws     device workspace of at least gptq_prepare_workspace_bytes(n),
  *          256-byte aligned.
  * Source: CHMC page, Schritt 2 (damping, act-order, "H⁻¹ über die
- * Cholesky-Zerlegung"); Babai page, §2.3 (ordering by the Hessian diagonal).
+ * Cholesky-Zerlegung"); Babai page, §2.3 (ordering by the Hessian diagonal,
+ * the min-pivot order).
  * Errors: INVALID_ARG (null pointer, n < 1, damp < 0 or not finite, bad
  * order, workspace too small; a CUSTOM perm that is not a permutation is
  * reported through info), CUDA; NOT_PD / NONFINITE through info.

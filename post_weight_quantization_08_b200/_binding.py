@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libgptq_b200.so")
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_NOT_PD",
           3: "GPTQ_ERR_NONFINITE", 4: "GPTQ_ERR_UNSUPPORTED",
           5: "GPTQ_ERR_TIMEOUT", 6: "GPTQ_ERR_CUDA"}
-ORDERS = {"natural": 0, "act": 1, "reverse": 2, "custom": 3}
+ORDERS = {"natural": 0, "act": 1, "reverse": 2, "custom": 3, "minpivot": 4}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 # name: (restype, argtypes)

@@ -21,6 +21,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "minpivot.cuh"
 
 namespace gptq {
 namespace {
@@ -905,7 +906,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare: n=%lld", (long long)n);
   if (!(damp >= 0.0) || !std::isfinite(damp))
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare: damp must be finite and >= 0");
-  if (order < GPTQ_ORDER_NATURAL || order > GPTQ_ORDER_CUSTOM)
+  if (order < GPTQ_ORDER_NATURAL || order > GPTQ_ORDER_MINPIVOT)
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare: order=%d", order);
   if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0)
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare: workspace not 256-byte aligned");
@@ -933,8 +934,17 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   if (order == GPTQ_ORDER_CUSTOM)
     GPTQ_CUDA(cudaMemsetAsync(w.seen, 0, sizeof(int32_t) * n, s));
   GPTQ_LAUNCH(KK_PREP_STATS, s, prep_stats_kernel, 1, 1024, 0, H, n, dead, w.mean, info);
-  GPTQ_LAUNCH(KK_PREP_ORDER, s, prep_order_kernel, (int)ceil_div(n, 256), 256, 0,
-              H, n, order, perm, w.seen, info);
+  if (order == GPTQ_ORDER_MINPIVOT) {
+    // the order comes from a pivoted factorisation of its own, on the
+    // workspace's two float64 arrays (both rewritten by the gather below)
+    if (min_pivot_scratch_doubles(n) > (size_t)(np * np))
+      return fail(GPTQ_ERR_INVALID_ARG, "gptq_prepare: min-pivot scratch does not fit");
+    gptq_status st = launch_min_pivot_order(H, n, w.mean, damp, w.M, np, w.A, perm, info, s);
+    if (st != GPTQ_OK) return st;
+  } else {
+    GPTQ_LAUNCH(KK_PREP_ORDER, s, prep_order_kernel, (int)ceil_div(n, 256), 256, 0,
+                H, n, order, perm, w.seen, info);
+  }
   GPTQ_LAUNCH(KK_PREP_GATHER, s, prep_gather_kernel, (unsigned)ceil_div(np * np, 256),
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);

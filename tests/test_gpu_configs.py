@@ -79,3 +79,10 @@ def test_stress_layer_sampled(order):
     S = 2.0 * (np.abs(Xs).T @ np.abs(Xs))
     T = Xs.shape[0]
     assert np.all(np.abs(H[:256, :256] - Hr) <= 2.0 * T * 2.0 ** -24 * S + 1e-30)
+
+
+def test_smollm_down_min_pivot():
+    """The SmolLM down projection (576×1536) under the min-pivot order, every row."""
+    p = problems_for(1, order="minpivot")[1]
+    st, _ = _check_problem(p, full_rows=True)
+    assert st["code_diff"] <= 1e-3 * st["codes"]

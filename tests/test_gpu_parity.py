@@ -3,7 +3,8 @@
 Sizes span several tiles and a ragged tail (n = 576 is 4½ groups of 128;
 m = 300 is not a multiple of the 64-row CTA) and stay small enough for the
 oracle to finish in seconds.  Edge cases: n = 1 / 8 / 64, m = 1 / 7, every bit
-width, groups of 32/64/128, all four orders, dead columns, and the error paths.
+width, groups of 32/64/128, every order (min-pivot included), dead columns,
+and the error paths.
 """
 import numpy as np
 import pytest
@@ -55,10 +56,64 @@ def test_group_block(group, block):
     _full_check(X, W, 4, group, block)
 
 
-@pytest.mark.parametrize("order", ["natural", "act", "reverse"])
+@pytest.mark.parametrize("order", ["natural", "act", "reverse", "minpivot"])
 def test_orders(order):
     X, W = _layer(768, 448, 96, 11)
     _full_check(X, W, 4, 64, 128, order)
+
+
+def _assert_min_pivot_sequence(Hd, perm, rtol=1e-10):
+    """Along the elimination order (perm reversed) every step takes a smallest
+    Schur-complement diagonal (float64, recomputed here), ties to the larger
+    column."""
+    S = np.array(Hd, dtype=np.float64, copy=True)
+    n = len(perm)
+    alive = np.ones(n, dtype=bool)
+    assert sorted(perm.tolist()) == list(range(n))
+    for t, j in enumerate(perm[::-1]):
+        d = np.where(alive, np.diag(S), np.inf)
+        assert alive[j] and d[j] <= d.min() + rtol * abs(d.min()), (t, j)
+        alive[j] = False
+        c = S[:, j].copy()
+        S -= np.outer(c, c) / c[j]
+
+
+@pytest.mark.parametrize("T,n,m", [(512, 40, 30), (768, 130, 50), (1024, 300, 64), (2048, 576, 96)])
+def test_min_pivot_order(T, n, m):
+    """The GPU's min-pivot order is a valid min-pivot sequence, equals the
+    oracle's, and the rest of the path follows it to parity."""
+    X, W = _layer(T, n, m, 21 + n)
+    out = P.run_gpu(X, W, 4, 64, 128, 0.01, "minpivot", None, DEV)
+    Hd, _, _ = og.damp_and_fix(out["H"].astype(np.float64), 0.01)
+    _assert_min_pivot_sequence(Hd, out["perm"])
+    _, st = P.check_prepare(out["H"], out, 0.01, "minpivot")
+    st.update(P.check_quantize(W, out, None, 4, 64, 128))
+    st.update(P.check_layer_loss(X, W, out, 4, 64, 128, 0.01, "minpivot"))
+
+
+def test_min_pivot_identity_and_diagonal():
+    """H = I gives the natural order; a diagonal H (ties included) gives act-order."""
+    import post_weight_quantization_08_b200 as g
+    n = 150
+    p = g.prepare(torch.eye(n, device=DEV), 0.01, "minpivot")
+    assert np.array_equal(p["perm"].cpu().numpy(), np.arange(n))
+    d = torch.tensor(np.random.default_rng(5).choice([0.5, 1.0, 2.0, 4.0], size=n),
+                     dtype=torch.float32)
+    H = torch.diag(d).to(DEV)
+    a = g.prepare(H, 0.01, "act")["perm"].cpu().numpy()
+    b = g.prepare(H, 0.01, "minpivot")["perm"].cpu().numpy()
+    assert np.array_equal(a, b)
+
+
+def test_min_pivot_not_positive_definite():
+    """A negative pivot is met at the first elimination step: processed last."""
+    import post_weight_quantization_08_b200 as g
+    n = 90
+    H = torch.eye(n, device=DEV)
+    H[5, 5] = -1.0
+    out = g.prepare(H, 0.0, "minpivot", check=False)
+    st, idx = g.gptq_check(out["info"])
+    assert st == 2 and idx == n
 
 
 def test_custom_order():
