@@ -55,6 +55,27 @@ __device__ __forceinline__ void report(int32_t* info, int32_t st, int64_t index)
     if (e__ != cudaSuccess) return gptq::cuda_fail(e__, #kernel);              \
   } while (0)
 
+// The same with programmatic dependent launch: the kernel may start (and run
+// its prologue) while the previous kernel of the stream finishes; it must
+// execute pdl_wait() (sm100.cuh) before touching anything that kernel writes.
+#define GPTQ_LAUNCH_PDL(kind, strm, kernel, grid, block, smem, ...)          \
+  do {                                                                         \
+    gptq::launch_begin((kind), (strm));                                        \
+    cudaLaunchConfig_t cfg__ = {};                                             \
+    cfg__.gridDim = dim3(grid);                                                \
+    cfg__.blockDim = dim3(block);                                              \
+    cfg__.dynamicSmemBytes = (smem);                                           \
+    cfg__.stream = (strm);                                                     \
+    cudaLaunchAttribute at__[1];                                               \
+    at__[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;           \
+    at__[0].val.programmaticStreamSerializationAllowed = 1;                    \
+    cfg__.attrs = at__;                                                        \
+    cfg__.numAttrs = 1;                                                        \
+    cudaError_t e__ = cudaLaunchKernelEx(&cfg__, kernel, __VA_ARGS__);         \
+    gptq::launch_end((kind), (strm));                                          \
+    if (e__ != cudaSuccess) return gptq::cuda_fail(e__, #kernel);              \
+  } while (0)
+
 #define GPTQ_CUDA(call)                                                        \
   do {                                                                         \
     cudaError_t e__ = (call);                                                  \

@@ -184,6 +184,8 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  pdl_wait();                           // the strip was written by the previous kernel
+  pdl_trigger();
   if (t == 0) {
     // the package and, when the rows allow a tensor map, the strip: four
     // boxes at (j0 + 32q, r0); columns past n read as zero, and Wp holds whole
@@ -448,7 +450,7 @@ gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int 
       !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, SB * 4, SS, RT))
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const unsigned grid = (unsigned)ceil_div(m, RT);
-  GPTQ_LAUNCH(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, tw, strip_tma, Wp, m,
+  GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, tw, strip_tma, Wp, m,
               n, j0, bw,
               reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
               scale, zero, loss_row, info);

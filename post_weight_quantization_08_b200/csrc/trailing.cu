@@ -164,6 +164,8 @@ trailing_tc_kernel(const __grid_constant__ TrailMaps maps, int64_t m, int64_t n,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();                           // the errors come from the previous kernel
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     for (int c = 0; c < nk; ++c) {
@@ -288,8 +290,8 @@ gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, int64_t
       g_attr = true;
     }
     const dim3 grid((unsigned)ceil_div(c1 - c0, QN), (unsigned)ceil_div(m, QM));
-    GPTQ_LAUNCH(KK_TRAIL, s, trailing_tc_kernel, grid, 128, QSMEM, maps, m, n, c0, c1, k0, kw,
-                info);
+    GPTQ_LAUNCH_PDL(KK_TRAIL, s, trailing_tc_kernel, grid, 128, QSMEM, maps, m, n, c0, c1, k0,
+                    kw, info);
     return GPTQ_OK;
   }
   const dim3 grid((unsigned)ceil_div(c1 - c0, TN), (unsigned)ceil_div(m, TM));
