@@ -442,7 +442,8 @@ def run_ours(args, rank, world, local):
         kernels[k] = {"ms_per_step": round(per_step_ms, 4),
                       "launches_per_step": kprof[k][1] / args.steps,
                       "bound": bound, "achieved": round(ach, 2), "unit": unit,
-                      "peak": round(peak, 1), "frac": round(ach / peak, 4)}
+                      "peak": round(peak, 1), "frac": round(ach / peak, 4),
+                      "traffic": traffic_for(k, workload_name(args.config, bits, args.order))}
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "params/s", "n_gpus": world,
