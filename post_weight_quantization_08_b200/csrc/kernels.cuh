@@ -29,10 +29,24 @@ gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
 // TF32 split Ehi + Elo (each error_rows(m)×128, Ehi = TF32(e), Elo = e − Ehi
 // exactly) and
 // adds Σe² to loss_row (may be NULL).
+//
+// With pre.kw > 0 the sweep first applies the previous block's contribution to
+// its own columns: D = (pre.Ehi + pre.Elo)[:, 0:pre.kw]·U[pre.k0 : pre.k0+pre.kw,
+// j0 : j0+bw] on the tensor cores (pre.Uhi/Ulo: the transposed TF32 split of U,
+// n % 4 == 0), so that no separate trailing update is needed for those columns.
+struct SweepPrologue {
+  const float* Ehi = nullptr;   // previous block's errors (error_rows(m) × 128)
+  const float* Elo = nullptr;
+  const float* Uhi = nullptr;   // transposed TF32 split of U
+  const float* Ulo = nullptr;
+  int64_t k0 = 0;               // first column of the previous block
+  int kw = 0;                   // its width (a multiple of 32), 0 for none
+};
 gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
-                         float* Elo, float* loss_row, int32_t* info, cudaStream_t s);
+                         float* Elo, const SweepPrologue& pre, float* loss_row, int32_t* info,
+                         cudaStream_t s);
 
 // Whether the trailing update runs on the tensor cores for this shape.
 bool trailing_uses_tensor_cores(int64_t n, int block);

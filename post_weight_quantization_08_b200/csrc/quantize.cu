@@ -70,8 +70,9 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162flo
 // life of the process.
 struct SideStream {
   cudaStream_t s2 = nullptr;
-  cudaEvent_t swept = nullptr;   // recorded on the caller's stream after a sweep
-  cudaEvent_t far = nullptr;     // recorded on the side stream after a far update
+  cudaEvent_t swept = nullptr;    // recorded on the caller's stream after a sweep
+  cudaEvent_t far[2] = {};        // recorded on the side stream after the far update
+                                  // of an even / odd block
 };
 
 gptq_status side_stream_for(cudaStream_t s, SideStream** out) {
@@ -84,7 +85,8 @@ gptq_status side_stream_for(cudaStream_t s, SideStream** out) {
   if (e.s2 == nullptr) {
     GPTQ_CUDA(cudaStreamCreateWithFlags(&e.s2, cudaStreamNonBlocking));
     GPTQ_CUDA(cudaEventCreateWithFlags(&e.swept, cudaEventDisableTiming));
-    GPTQ_CUDA(cudaEventCreateWithFlags(&e.far, cudaEventDisableTiming));
+    GPTQ_CUDA(cudaEventCreateWithFlags(&e.far[0], cudaEventDisableTiming));
+    GPTQ_CUDA(cudaEventCreateWithFlags(&e.far[1], cudaEventDisableTiming));
   }
   *out = &e;
   return GPTQ_OK;
@@ -230,44 +232,64 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
     st = launch_split_tf32_t(U, n, w.Uhi, w.Ulo, s);
     if (st != GPTQ_OK) return st;
   }
-  // Block b: sweep, then the update of block b+1's columns on the caller's
-  // stream (the next sweep waits for it), and the update of the columns after
-  // that on the side stream, overlapping sweep b+1.  Every column still
-  // receives the blocks' contributions in block order: the update of block
-  // b+1's columns by block b waits for the far update of block b−1, and the
-  // two error buffers alternate so that a far update's input is not
-  // overwritten by the next sweep.
+  // Block b's errors reach the later columns in two parts:
+  //  * block b+1's columns: on the tensor-core path, sweep b+1 applies them
+  //    itself in its prologue (in TMEM, before its first column); otherwise a
+  //    trailing update on the caller's stream;
+  //  * the columns from block b+2 on: a trailing update on the side stream,
+  //    overlapping sweep b+1.
+  // Every column still receives the blocks' contributions in block order:
+  // whatever touches block b's columns first waits for the far update of
+  // block b−2 (which also reached them), and the two error buffers alternate,
+  // so a far update's input is not overwritten before it is read.
   SideStream* side = nullptr;
   st = side_stream_for(s, &side);
   if (st != GPTQ_OK) return st;
-  bool far_pending = false;
+  const bool fused = w.Uhi != nullptr && trailing_uses_tensor_cores(n, block);
+  bool pending[2] = {false, false};
   for (int64_t j0 = 0, b = 0; j0 < n; j0 += block, ++b) {
     const int bw = (int)((n - j0 < block) ? (n - j0) : block);
     float* ehi = w.Ehi[b & 1];
     float* elo = w.Elo[b & 1];
+    if (pending[b & 1]) {                      // the far update of block b−2
+      GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[b & 1], 0));
+      pending[b & 1] = false;
+    }
+    SweepPrologue pre;
+    if (fused && b > 0) {
+      pre.Ehi = w.Ehi[(b - 1) & 1];
+      pre.Elo = w.Elo[(b - 1) & 1];
+      pre.Uhi = w.Uhi;
+      pre.Ulo = w.Ulo;
+      pre.k0 = j0 - block;
+      pre.kw = block;
+    }
     const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
     st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes, scale,
-                      zero, ehi, elo, loss_row, info, s);
+                      zero, ehi, elo, pre, loss_row, info, s);
     if (st != GPTQ_OK) return st;
     const int64_t c0 = j0 + bw, c1 = c0 + block;
     if (c0 >= n) break;
+    if (!fused) {
+      if (b > 0 && pending[(b - 1) & 1]) {     // the far update of block b−1
+        GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[(b - 1) & 1], 0));
+        pending[(b - 1) & 1] = false;
+      }
+      st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info, s);
+      if (st != GPTQ_OK) return st;
+    }
     if (c1 < n) {
       GPTQ_CUDA(cudaEventRecord(side->swept, s));
       GPTQ_CUDA(cudaStreamWaitEvent(side->s2, side->swept, 0));
-    }
-    if (far_pending) GPTQ_CUDA(cudaStreamWaitEvent(s, side->far, 0));
-    st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info, s);
-    if (st != GPTQ_OK) return st;
-    far_pending = false;
-    if (c1 < n) {
       st = launch_trailing(w.Wp, m, n, c1, n, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info,
                            side->s2);
       if (st != GPTQ_OK) return st;
-      GPTQ_CUDA(cudaEventRecord(side->far, side->s2));
-      far_pending = true;
+      GPTQ_CUDA(cudaEventRecord(side->far[b & 1], side->s2));
+      pending[b & 1] = true;
     }
   }
-  if (far_pending) GPTQ_CUDA(cudaStreamWaitEvent(s, side->far, 0));
+  for (int p = 0; p < 2; ++p)
+    if (pending[p]) GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[p], 0));
 
   const unsigned gpk = (unsigned)ceil_div(m * ceil_div(n, 32), 256);
   switch (bits) {

@@ -62,10 +62,16 @@ constexpr uint32_t SM_ALO = SM_AHI + RT * 128;
 constexpr uint32_t SM_VALS = SM_ALO + RT * 128;
 constexpr uint32_t VBOX = RT * 128;                // 128 rows × 32 floats, swizzled
 constexpr uint32_t SM_CODES = SM_VALS + 4 * VBOX;
-constexpr uint32_t SM_BARS = (SM_CODES + RT * LDB + 15) / 16 * 16;
-constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 32;
+// the prologue's U chunk: TF32 hi part in its own box, lo part in the code
+// rows' space (1024-aligned, unused until the column steps)
+constexpr uint32_t SM_BPHI = (SM_CODES + RT * LDB + 1023) / 1024 * 1024;
+constexpr uint32_t SM_BPLO = SM_CODES;
+constexpr uint32_t SM_BARS = SM_BPHI + 32 * RT * 4;
+constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 64;
 static_assert(SM_AHI >= PK_BYTES && SM_AHI % 1024 == 0, "A operand placement");
 static_assert(SM_VALS % 1024 == 0, "the strip's boxes use the 128-byte swizzle");
+static_assert(SM_CODES % 1024 == 0 && RT * LDB >= 32 * RT * 4, "U chunk lo part placement");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
 // The block's strip of Wp in shared memory: four boxes of 32 columns × 128
 // rows with the TMA 128-byte swizzle, the 16-byte chunk j of row r at
@@ -149,6 +155,9 @@ __device__ __forceinline__ float div_fma(float x, float s, float rs) {
 __global__ void __launch_bounds__(RT, 1)
 sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
              const __grid_constant__ CUtensorMap tmW, int strip_tma,
+             const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmPlo,
+             const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo,
+             int64_t k0p, int kwp,
              const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
              const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
              uint8_t* __restrict__ codes, float* __restrict__ scale,
@@ -164,7 +173,11 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   uint8_t* cs = sm + SM_CODES;
   uint64_t* pkg_bar = reinterpret_cast<uint64_t*>(sm + SM_BARS);
   uint64_t* mma_bar = pkg_bar + 1;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+  uint64_t* pro_bar = mma_bar + 1;      // prologue chunk loads
+  uint64_t* pro_mma = pro_bar + 1;      // prologue products but the last
+  uint64_t* pro_done = pro_mma + 1;     // the last prologue product
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(pro_done + 1);
+  const bool pro = kwp > 0;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t r0 = (int64_t)blockIdx.x * RT;
@@ -173,6 +186,9 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   if (t == 0) {
     mbar_init(pkg_bar, 1);
     mbar_init(mma_bar, 1);
+    mbar_init(pro_bar, 1);
+    mbar_init(pro_mma, 1);
+    mbar_init(pro_done, 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -196,6 +212,50 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         tma_load_2d(vals + q * VBOX, &tmW, (int)j0 + 32 * q, (int)r0, pkg_bar);
+    }
+    if (pro) {
+      // Prologue: D = E_prev·U[prev block, this block] in TMEM, the previous
+      // block's contribution to this block's columns (the part of the
+      // lazy-batch update the next sweep needs first), 3xTF32 like the
+      // trailing update, in K-chunks of 32 through the A buffers and the U
+      // chunk boxes.  Chunks but the last complete on pro_mma, the last on
+      // pro_done, which every thread waits for before reading D.
+      const int nk = kwp / SS;
+      const uint32_t idesc = idesc_f32acc(2, 2, 0, 0, RT, SB);
+      const uint32_t ah = smem_addr(ahi), al = smem_addr(alo);
+      const uint32_t bh = smem_addr(sm + SM_BPHI), bl = smem_addr(sm + SM_BPLO);
+      for (int c = 0; c < nk; ++c) {
+        mbar_arrive_expect_tx(pro_bar, 4 * VBOX);
+        tma_load_2d(ahi, &tmPhi, SS * c, (int)r0, pro_bar);
+        tma_load_2d(alo, &tmPlo, SS * c, (int)r0, pro_bar);
+        tma_load_2d(sm + SM_BPHI, &tmUhi, (int)k0p + SS * c, (int)j0, pro_bar);
+        tma_load_2d(sm + SM_BPLO, &tmUlo, (int)k0p + SS * c, (int)j0, pro_bar);
+        if (!mbar_wait_bounded(pro_bar, c & 1)) {
+          report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+          mbar_wait_bounded(pro_bar, c & 1);          // let our own copies land first
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < SS / 8; ++ks) {
+          const uint64_t dah = sdesc_sw128(ah + ks * 32, SW128_KMAJOR_LBO, 1024);
+          const uint64_t dal = sdesc_sw128(al + ks * 32, SW128_KMAJOR_LBO, 1024);
+          const uint64_t dbh = sdesc_sw128(bh + ks * 32, SW128_KMAJOR_LBO, 1024);
+          const uint64_t dbl = sdesc_sw128(bl + ks * 32, SW128_KMAJOR_LBO, 1024);
+          umma_tf32_ss(tmem, dah, dbh, idesc, (c > 0 || ks > 0) ? 1u : 0u);
+          umma_tf32_ss(tmem, dah, dbl, idesc, 1u);
+          umma_tf32_ss(tmem, dal, dbh, idesc, 1u);
+        }
+        if (c + 1 < nk) {
+          umma_commit(pro_mma);
+          if (!mbar_wait_bounded(pro_mma, c & 1)) {     // the buffers are read again next
+            report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+            break;
+          }
+        } else {
+          umma_commit(pro_done);
+        }
+      }
     }
   }
 
@@ -244,13 +304,24 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
     const int c0 = sb * SS;
     float v[SS], e[SS];
     if (sb == 0) {
+      float d[32];
+      if (pro) {
+        const bool ok = mbar_wait_bounded(pro_done, 0);
+        if (__syncthreads_or(!ok)) {
+          report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+          abort = true;
+          break;
+        }
+        tc_fence_after();
+        tmem_ld_32x32b_x32(trow, d);
+      }
 #pragma unroll
       for (int j = 0; j < SS / 4; ++j) {
         const float4 f = strip_chunk(vals, 0, t, j);
-        v[4 * j] = f.x;
-        v[4 * j + 1] = f.y;
-        v[4 * j + 2] = f.z;
-        v[4 * j + 3] = f.w;
+        v[4 * j] = f.x - (pro ? d[4 * j] : 0.f);
+        v[4 * j + 1] = f.y - (pro ? d[4 * j + 1] : 0.f);
+        v[4 * j + 2] = f.z - (pro ? d[4 * j + 2] : 0.f);
+        v[4 * j + 3] = f.w - (pro ? d[4 * j + 3] : 0.f);
       }
     } else {
       const bool ok = mbar_wait_bounded(mma_bar, (sb - 1) & 1);
@@ -284,7 +355,8 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
       const int gend = min(c0 + group, bw);
       for (int cs0 = c0 + SS; cs0 < gend; cs0 += SS) {
         float d[32];
-        if (sb > 0) tmem_ld_32x32b_x32(trow + cs0, d);
+        const bool upd = sb > 0 || pro;            // D holds updates for these columns
+        if (upd) tmem_ld_32x32b_x32(trow + cs0, d);
 #pragma unroll
         for (int j = 0; j < SS / 4; ++j) {
           const float4 f = strip_chunk(vals, cs0 / SS, t, j);
@@ -292,7 +364,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
             const int k = 4 * j + k4;
-            const float x = (cs0 + k < gend) ? fv[k4] - (sb > 0 ? d[k] : 0.f) : 0.f;
+            const float x = (cs0 + k < gend) ? fv[k4] - (upd ? d[k] : 0.f) : 0.f;
             xmin = fminf(xmin, x);
             xmax = fmaxf(xmax, x);
           }
@@ -368,7 +440,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
           const uint64_t dal = sdesc_sw128(al + ks * 32, SW128_KMAJOR_LBO, 1024);
           const uint64_t dbh = sdesc_sw128(bhi + ks * 32, SW128_KMAJOR_LBO, 1024);
           const uint64_t dbl = sdesc_sw128(blo + ks * 32, SW128_KMAJOR_LBO, 1024);
-          umma_tf32_ss(dcol, dah, dbh, idesc, (sb > 0 || ks > 0) ? 1u : 0u);
+          umma_tf32_ss(dcol, dah, dbh, idesc, (pro || sb > 0 || ks > 0) ? 1u : 0u);
           umma_tf32_ss(dcol, dah, dbl, idesc, 1u);
           umma_tf32_ss(dcol, dal, dbh, idesc, 1u);
         }
@@ -409,6 +481,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   if (t == 0) bulk_wait_all();          // the error boxes are in global memory
   if (abort && t == 0 && issued > 0)            // no MMA may still write TMEM
     mbar_wait_bounded(mma_bar, (issued - 1) & 1, 1u << 16);
+  if (abort && t == 0 && pro) mbar_wait_bounded(pro_done, 0, 1u << 16);
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, SB);
 }
@@ -432,7 +505,8 @@ gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
 gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
-                         float* Elo, float* loss_row, int32_t* info, cudaStream_t s) {
+                         float* Elo, const SweepPrologue& pre, float* loss_row, int32_t* info,
+                         cudaStream_t s) {
   if (!g_attr_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)SMEM_BYTES));
@@ -446,11 +520,28 @@ gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int 
       !encode_tiled_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Wp, n, mr, n * 4, SS, RT))
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's strip");
   if (!strip_tma) memset(&tw, 0, sizeof(tw));
+  CUtensorMap tph, tpl, tuh, tul;
+  const int kwp = (pre.kw > 0 && pre.Ehi && pre.Elo && pre.Uhi && pre.Ulo) ? pre.kw : 0;
+  if (kwp > 0) {
+    if (kwp % SS != 0 || pre.kw > SB)
+      return fail(GPTQ_ERR_INVALID_ARG, "sweep prologue: width %d", pre.kw);
+    if (!encode_tiled_2d(&tph, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Ehi, SB, mr, SB * 4, SS, RT) ||
+        !encode_tiled_2d(&tpl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Elo, SB, mr, SB * 4, SS, RT) ||
+        !encode_tiled_2d(&tuh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Uhi, n, n, n * 4, SS, RT) ||
+        !encode_tiled_2d(&tul, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Ulo, n, n, n * 4, SS, RT))
+      return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's prologue");
+  } else {
+    memset(&tph, 0, sizeof(tph));
+    memset(&tpl, 0, sizeof(tpl));
+    memset(&tuh, 0, sizeof(tuh));
+    memset(&tul, 0, sizeof(tul));
+  }
   if (!encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ehi, SB, mr, SB * 4, SS, RT) ||
       !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, SB * 4, SS, RT))
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const unsigned grid = (unsigned)ceil_div(m, RT);
-  GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, tw, strip_tma, Wp, m,
+  GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, tw, strip_tma, tph,
+                  tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m,
               n, j0, bw,
               reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
               scale, zero, loss_row, info);
