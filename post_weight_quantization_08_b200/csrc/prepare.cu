@@ -194,10 +194,35 @@ __constant__ unsigned char kTri8I[36] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3, 4, 4, 4, 
 __constant__ unsigned char kTri8J[36] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3, 0, 1, 2, 3, 4, 0, 1, 2,
                                          3, 4, 5, 0, 1, 2, 3, 4, 5, 6, 0, 1, 2, 3, 4, 5, 6, 7};
 
-// Named barriers of the diagonal tile (0 is __syncthreads): 1 joins warps
-// 1–7; 2 hands X and the next panel block from warp 0 to warps 1–7; 3 hands
-// finished trailing updates from warps 1–7 back to warp 0.
+constexpr uint32_t kSpinLimit = 1u << 22;   // ≈ a few seconds with the back-off below
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Tiles the otherwise idle warp 4 of the diagonal tile fetches ahead: a tile
+// is final once *flag ≥ target; up to two 64×64 float64 tiles (leading
+// dimension ld) into shared memory.
+struct TilePrefetch {
+  const int* flag[2];
+  int target[2];
+  const double* src[2];
+  double (*dst[2])[LDM];
+  int64_t ld;
+  int count;
+};
+
+// Named barriers of the diagonal tile (0 is __syncthreads): 1 joins the six
+// working warps (1–3, 5–7); 2 hands X and the next panel block from warp 0 to
+// them; 3 hands their finished trailing updates back to warp 0.  Warp 4 shares
+// warp 0's scheduler and stays out of them (it prefetches).
 constexpr int kBarRest = 1, kBarX = 2, kBarDone = 3;
+constexpr int kRest = 192, kHand = 224;     // 6 working warps; + warp 0
 
 __device__ __forceinline__ void bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -299,25 +324,32 @@ __device__ __forceinline__ int chol8_pairs(double (&l)[36], double (&x)[8], int 
 // (a: lower triangle of A on entry, overwritten; b: zero on entry, D on
 // exit; xs: 3 × 64 doubles), blocked by 8 columns and software-pipelined:
 //   warp 0, step kb: Cholesky of the diagonal block kb (registers), X_kb =
-//     its inverse; then, once warps 1–7 have applied step kb−1 to block row
+//     its inverse; then, once the working warps have applied step kb−1 to block row
 //     kb+1, the panel block L_{kb+1,kb} = A_{kb+1,kb}·X_kbᵀ and the diagonal
 //     block A_{kb+1,kb+1} −= L_{kb+1,kb}·L_{kb+1,kb}ᵀ, so that step kb+1 can
 //     start at once;
-//   warps 1–7, step kb: the other panel blocks L_{I,kb} (I ≥ kb+2), the
+//   warps 1–3 and 5–7, step kb: the other panel blocks L_{I,kb} (I ≥ kb+2), the
 //     other trailing blocks A_{IJ} −= L_{I,kb}·L_{J,kb}ᵀ, and block row kb of
 //     D: D_{kb,J} = X_kb·D_{kb,J} (J < kb), D_{kb,kb} = X_kb, then
 //     D_{IJ} −= L_{I,kb}·D_{kb,J} for I > kb, J ≤ kb (the elimination applied
 //     to an identity matrix).
-// Each block row of D goes out to dout (leading dimension ld) as soon as it is
-// final.  All products are 8×8 blocks on the float64 tensor cores.  A bad pivot is
+// Warp 4 shares warp 0's scheduler and float64 pipe, so it takes none of this
+// work; it fetches the tiles in pf meanwhile (see TilePrefetch).  Each block
+// row of D goes out to dout (leading dimension ld) as soon as it is final.  All products are 8×8 blocks on the float64 tensor cores.  A bad pivot is
 // reported through info (the factorisation runs to the end on zeros, so that
 // every barrier is met) and makes the function return false.  Called by a
 // whole CTA of 256 threads.
 __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
                                double* __restrict__ dout, int64_t ld, int64_t n, int64_t base,
-                               int32_t* info, int* bad_s) {
+                               int32_t* info, int* bad_s, const TilePrefetch& pf,
+                               volatile int* s_stop, int* s_got) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q = lane & 3;
+  if (tid == 0) {
+    *s_stop = 0;
+    *s_got = 0;
+  }
+  __syncthreads();
   if (warp == 0) {
     double l[36];
 #pragma unroll
@@ -338,7 +370,7 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
       __syncwarp();
       // warps 1–7 have applied step kb−1 (and so have all passed barrier X
       // of step kb−1: no arrival below can fall into an older generation)
-      if (kb > 0) bar_sync(kBarDone, 256);
+      if (kb > 0) bar_sync(kBarDone, kHand);
       if (kb < 7) {
         const int r1 = c0 + 8;
         block8_nt<false, false>(&a[r1][c0], &a[r1][c0], LDM, X, 8, lane);
@@ -350,26 +382,56 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
 #pragma unroll
           for (int j = 0; j <= i; ++j) l[i * (i + 1) / 2 + j] = a[r1 + i][r1 + j];
       }
-      bar_arrive(kBarX, 256);                          // X_kb and L_{kb+1,kb} ready
+      bar_arrive(kBarX, kHand);                        // X_kb and L_{kb+1,kb} ready
     }
+    if (lane == 0) *s_stop = 1;                        // the prefetcher may give up now
     if (lane == 0 && bad < 64) {
       *bad_s = 1;
       report(info, GPTQ_ERR_NOT_PD, n - 1 - (base + bad));
     }
+  } else if (warp == 4) {
+    // The prefetcher: each tile of pf as soon as its flag says it is final
+    // (lane 0 polls with acquire loads; the copies are cp.async through L2),
+    // until both are in or warp 0 is done.  The master skips what it got.
+    int got = 0;
+    const int all = (1 << pf.count) - 1;
+    for (uint32_t it = 0; it < kSpinLimit && got != all; ++it) {
+      int ready = 0;
+      if (lane == 0) {
+        for (int t2 = 0; t2 < pf.count; ++t2)
+          if (!((got >> t2) & 1) && ld_acquire(pf.flag[t2]) >= pf.target[t2]) ready |= 1 << t2;
+      }
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      __syncwarp();
+      for (int t2 = 0; t2 < pf.count; ++t2) {
+        if (!((ready >> t2) & 1)) continue;
+        for (int r = 0; r < NB; ++r) {
+          const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&pf.dst[t2][r][2 * lane]));
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
+                       "l"(pf.src[t2] + (int64_t)r * pf.ld + 2 * lane)
+                       : "memory");
+        }
+        got |= 1 << t2;
+      }
+      if (got == all || *s_stop) break;
+      __nanosleep(128);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (lane == 0) *s_got = got;
   } else {
-    // Warp 4 shares a scheduler (and its float64 pipe) with warp 0, so it
-    // takes no work: v numbers the six working warps.
-    const int v = (warp < 4) ? warp - 1 : ((warp > 4) ? warp - 2 : -1);
+    // v numbers the six working warps (warp 4 prefetches)
+    const int v = (warp < 4) ? warp - 1 : warp - 2;
     for (int kb = 0; kb < 8; ++kb) {
       const int c0 = 8 * kb;
       const double* X = xs + 64 * (kb % 3);
-      bar_sync(kBarX, 256);
+      bar_sync(kBarX, kHand);
       // panel blocks I ≥ kb + 2
       if (v >= 0 && kb + 2 + v < 8) {
         const int r = 8 * (kb + 2 + v);
         block8_nt<false, false>(&a[r][c0], &a[r][c0], LDM, X, 8, lane);
       }
-      bar_sync(kBarRest, 224);
+      bar_sync(kBarRest, kRest);
       // trailing blocks kb+1 ≤ J ≤ I ≤ 7 except (kb+1, kb+1); operands first
       const int rem = 7 - kb;
       const int nblk = rem * (rem + 1) / 2;
@@ -398,7 +460,7 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
           *reinterpret_cast<double2*>(&a[8 * bi + g][8 * bj + 2 * q]) = make_double2(acc[0], acc[1]);
         }
       }
-      if (kb < 7) bar_arrive(kBarDone, 256);           // warp 0 waits for steps 0..6
+      if (kb < 7) bar_arrive(kBarDone, kHand);         // warp 0 waits for steps 0..6
       // block row kb of D
       if (v >= 0) {
         for (int J = v; J < kb; J += 6) block8_xb(&b[c0][8 * J], X, &b[c0][8 * J], lane);
@@ -406,7 +468,7 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
       if (v == 5) {
         for (int e = lane; e < 64; e += 32) b[c0 + (e >> 3)][c0 + (e & 7)] = X[e];
       }
-      bar_sync(kBarRest, 224);
+      bar_sync(kBarRest, kRest);
       // block row kb of D is final: out to global memory now, so that little
       // is left in flight when the tile is published
       if (v >= 0) {
@@ -646,16 +708,7 @@ __device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
 // loads; every wait is bounded and a time-out (or a bad pivot) raises a
 // shared abort flag.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kSpinLimit = 1u << 22;   // ≈ a few seconds with the back-off below
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 struct CholSync {
   int* ctrl;        // [0] next task, [1] arrivals, [2] abort
@@ -747,7 +800,8 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int64_t n, int64_t np, int N,
                        int ntasks, int* sync_base, int32_t* info) {
   extern __shared__ double sm[];
-  __shared__ int s_role, s_task, s_ok, s_bad;
+  __shared__ int s_role, s_task, s_ok, s_bad, s_got;
+  __shared__ volatile int s_stop;
   const CholSync S = sync_view(sync_base, N);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) s_role = atomicAdd(&S.ctrl[1], 1);
@@ -776,7 +830,22 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       const bool more = k + 1 < N;
       double* Lp = A + (base + NB) * np + base;          // tile (k+1, k)
       const double* An = A + (base + NB) * np + base + NB;   // tile (k+1, k+1)
-      if (!diag_tile_smem(a, b, xs, M + base * np + base, np, n, base, info, &s_bad)) {
+      // warp 4 fetches the next step's two input tiles during the diagonal
+      // tile, as soon as the workers have finished them
+      TilePrefetch pf = {};
+      if (more) {
+        pf.count = 2;
+        pf.flag[0] = &S.upd[(k + 1) * N + k];
+        pf.flag[1] = &S.upd[(k + 1) * N + k + 1];
+        pf.target[0] = pf.target[1] = k;
+        pf.src[0] = Lp;
+        pf.src[1] = An;
+        pf.dst[0] = x;
+        pf.dst[1] = an;
+        pf.ld = np;
+      }
+      if (!diag_tile_smem(a, b, xs, M + base * np + base, np, n, base, info, &s_bad, pf,
+                          &s_stop, &s_got)) {
         if (tid == 0) atomicExch(&S.ctrl[2], 1);
         return;
       }
@@ -785,10 +854,13 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
         st_release(&S.diag_done[k], 1);
       }
       if (!more) break;
+      const int got = s_got;                        // read after the tile's last barrier
       // L_{k+1,k} = A_{k+1,k}·D_kᵀ
-      if (!cta_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok)) return;
-      copy_tile_async(x, Lp, np, tid);
-      copy_wait_all();
+      if (!(got & 1)) {
+        if (!cta_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok)) return;
+        copy_tile_async(x, Lp, np, tid);
+        copy_wait_all();
+      }
       __syncthreads();
       double acc[4][2][2] = {};
       panel_mm(x, b, acc, warp, lane);
@@ -796,9 +868,11 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       panel_store(x, Lp, np, acc, warp, lane);
       zero_tile(b, tid);
       // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
-      if (!cta_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok)) return;
-      copy_tile_async(an, An, np, tid);
-      copy_wait_all();
+      if (!(got & 2)) {
+        if (!cta_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok)) return;
+        copy_tile_async(an, An, np, tid);
+        copy_wait_all();
+      }
       __syncthreads();
       lower_syrk(an, x, warp, lane);
       __syncthreads();
