@@ -1023,10 +1023,12 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);
   const int ntasks = total_tasks(N);
-  // Workers: about as many as the dataflow keeps busy (a step offers ≈ N²/2
-  // tile tasks, each ≈ a third of the chain's step), never more than one CTA
-  // per SM besides the chain's, so that work on other streams finds SMs.
-  int workers = N * N / 6 + 2;
+  // Workers: enough that the two tiles the chain needs next are never queued
+  // behind other ready tasks (a step offers ≈ N²/2 tile tasks, each ≈ a third
+  // of the chain's step; N²/6 workers left the chain waiting ≈ 6.8 K cycles a
+  // step for its panel input, N²/3 ≈ 0.5 K), never more than one CTA per SM
+  // besides the chain's, so that work on other streams finds SMs.
+  int workers = N * N / 3 + 2;
   if (workers > g_num_sms - 1) workers = g_num_sms - 1;
   if (workers > ntasks) workers = ntasks;
   const int grid = 1 + workers;
