@@ -217,11 +217,21 @@ struct TilePrefetch {
   int count;
 };
 
+// The panel of the step before, still in shared memory (src), goes to global
+// memory (dst, leading dimension ld) at the start of the diagonal tile, and
+// *flag is released once it is there; dst = nullptr: none.
+struct PanelOut {
+  const double (*src)[LDM];
+  double* dst;
+  int* flag;
+};
+
 // Named barriers of the diagonal tile (0 is __syncthreads): 1 joins the six
 // working warps (1–3, 5–7); 2 hands X and the next panel block from warp 0 to
-// them; 3 hands their finished trailing updates back to warp 0.  Warp 4 shares
-// warp 0's scheduler and stays out of them (it prefetches).
-constexpr int kBarRest = 1, kBarX = 2, kBarDone = 3;
+// them; 3 hands their finished trailing updates back to warp 0; 4 tells warp 4
+// that they have stored the panel of the step before.  Warp 4 shares warp 0's
+// scheduler and stays out of 1–3 (it prefetches).
+constexpr int kBarRest = 1, kBarX = 2, kBarDone = 3, kBarPanel = 4;
 constexpr int kRest = 192, kHand = 224;     // 6 working warps; + warp 0
 
 __device__ __forceinline__ void bar_sync(int id, int count) {
@@ -334,15 +344,19 @@ __device__ __forceinline__ int chol8_pairs(double (&l)[36], double (&x)[8], int 
 //     D_{IJ} −= L_{I,kb}·D_{kb,J} for I > kb, J ≤ kb (the elimination applied
 //     to an identity matrix).
 // Warp 4 shares warp 0's scheduler and float64 pipe, so it takes none of this
-// work; it fetches the tiles in pf meanwhile (see TilePrefetch).  Each block
-// row of D goes out to dout (leading dimension ld) as soon as it is final.  All products are 8×8 blocks on the float64 tensor cores.  A bad pivot is
+// work: it publishes the panel of the step before once the working warps have
+// stored it (po, while warp 0 factors the first block), clears the blocks
+// below the diagonal of bz (the D buffer of the step before, zero above the
+// diagonal already), and fetches the tiles in pf.  Each block row of D goes
+// out to dout (leading dimension ld) as soon as it is final.  All products
+// are 8×8 blocks on the float64 tensor cores.  A bad pivot is
 // reported through info (the factorisation runs to the end on zeros, so that
 // every barrier is met) and makes the function return false.  Called by a
 // whole CTA of 256 threads.
-__device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
-                               double* __restrict__ dout, int64_t ld, int64_t n, int64_t base,
-                               int32_t* info, int* bad_s, const TilePrefetch& pf,
-                               volatile int* s_stop, int* s_got) {
+__device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double (*bz)[LDM],
+                               double* xs, double* __restrict__ dout, int64_t ld, int64_t n,
+                               int64_t base, int32_t* info, int* bad_s, const TilePrefetch& pf,
+                               const PanelOut& po, volatile int* s_stop, int* s_got) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q = lane & 3;
   if (tid == 0) {
@@ -393,6 +407,20 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
     // The prefetcher: each tile of pf as soon as its flag says it is final
     // (lane 0 polls with acquire loads; the copies are cp.async through L2),
     // until both are in or warp 0 is done.  The master skips what it got.
+    if (po.dst) {
+      bar_sync(kBarPanel, kHand);       // the working warps have stored it
+      if (lane == 0) {
+        __threadfence();
+        st_release(po.flag, 1);
+      }
+      __syncwarp();
+    }
+    if (bz) {
+#pragma unroll 4
+      for (int r = 8; r < NB; ++r)
+        if (lane < 4 * (r >> 3))
+          *reinterpret_cast<double2*>(&bz[r][2 * lane]) = make_double2(0.0, 0.0);
+    }
     int got = 0;
     const int all = (1 << pf.count) - 1;
     for (uint32_t it = 0; it < kSpinLimit && got != all; ++it) {
@@ -422,6 +450,14 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double* xs,
   } else {
     // v numbers the six working warps (warp 4 prefetches)
     const int v = (warp < 4) ? warp - 1 : warp - 2;
+    if (po.dst) {
+      for (int e = 32 * v + lane; e < NB * NB / 2; e += 192) {
+        const int r = e >> 5, c = (e & 31) * 2;
+        *reinterpret_cast<double2*>(po.dst + (int64_t)r * ld + c) =
+            *reinterpret_cast<const double2*>(&po.src[r][c]);
+      }
+      bar_arrive(kBarPanel, kHand);
+    }
     for (int kb = 0; kb < 8; ++kb) {
       const int c0 = 8 * kb;
       const double* X = xs + 64 * (kb % 3);
@@ -515,17 +551,6 @@ __device__ __forceinline__ void zero_tile(double (*dst)[LDM], int tid) {
     *reinterpret_cast<double2*>(&dst[e >> 5][(e & 31) * 2]) = make_double2(0.0, 0.0);
   }
 }
-__device__ __forceinline__ void store_tile(double* dst, int64_t ld, const double (*src)[LDM],
-                                           int tid) {
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int e = tid + 256 * s;
-    const int r = e >> 5, c = (e & 31) * 2;
-    *reinterpret_cast<double2*>(dst + (int64_t)r * ld + c) =
-        *reinterpret_cast<const double2*>(&src[r][c]);
-  }
-}
-
 // Asynchronous 64×64 tile copy global → shared memory (16-byte cp.async
 // through L2 only; tiles are rewritten by other CTAs of the same launch).
 __device__ __forceinline__ void copy_tile_async(double (*dst)[LDM], const double* src, int64_t ld,
@@ -546,30 +571,50 @@ __device__ __forceinline__ void copy_wait_all() { asm volatile("cp.async.wait_al
 // column J of L needs only q < 8·(J+1).  Warp w owns row blocks 4·(w/4) .. +4
 // and block columns J = w mod 4 and 7 − J, which gives every warp the same
 // number of products (and every scheduler the same load).  acc[i][c] is
-// block (4·(w/4) + i, c ? 7 − J : J).
-__device__ __forceinline__ void panel_mm(const double (*x)[LDM], const double (*d)[LDM],
-                                         double acc[4][2][2], int warp, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const int rb = 32 * (warp >> 2), J = warp & 3, J1 = 7 - J;
-  const int qlo = 8 * (J + 1), qhi = 8 * (J1 + 1);
-  for (int q = 0; q < qhi; q += 4) {
+// block (4·(w/4) + i, c ? 7 − J : J).  The k-loops have compile-time bounds
+// (one instance per J) and are unrolled, so that the fragment loads run ahead
+// of the products and the float64 pipe stays busy.
+template <int J>
+__device__ __forceinline__ void panel_mm_j(const double (*x)[LDM], const double (*d)[LDM],
+                                           double acc[4][2][2], int rb, int g, int t) {
+  constexpr int J1 = 7 - J, qlo = 8 * (J + 1), qhi = 8 * (J1 + 1);
+#pragma unroll
+  for (int q = 0; q < qlo; q += 4) {
+    double a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    const double b0 = d[8 * J + g][q + t], b1 = d[8 * J1 + g][q + t];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      dmma_884(acc[i][0], a[i], b0);
+      dmma_884(acc[i][1], a[i], b1);
+    }
+  }
+#pragma unroll
+  for (int q = qlo; q < qhi; q += 4) {
     double a[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
     const double b1 = d[8 * J1 + g][q + t];
 #pragma unroll
     for (int i = 0; i < 4; ++i) dmma_884(acc[i][1], a[i], b1);
-    if (q < qlo) {
-      const double b0 = d[8 * J + g][q + t];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dmma_884(acc[i][0], a[i], b0);
-    }
+  }
+}
+__device__ __forceinline__ void panel_mm(const double (*x)[LDM], const double (*d)[LDM],
+                                         double acc[4][2][2], int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3, rb = 32 * (warp >> 2);
+  switch (warp & 3) {
+    case 0: panel_mm_j<0>(x, d, acc, rb, g, t); break;
+    case 1: panel_mm_j<1>(x, d, acc, rb, g, t); break;
+    case 2: panel_mm_j<2>(x, d, acc, rb, g, t); break;
+    default: panel_mm_j<3>(x, d, acc, rb, g, t); break;
   }
 }
 
-// Writes the panel accumulators to a shared-memory tile and to global memory.
-__device__ __forceinline__ void panel_store(double (*xs_)[LDM], double* out, int64_t ld,
-                                            const double acc[4][2][2], int warp, int lane) {
+// Writes the panel accumulators to a shared-memory tile (it goes to global
+// memory from there later, off the chain).
+__device__ __forceinline__ void panel_to_smem(double (*xs_)[LDM], const double acc[4][2][2],
+                                              int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int rb = 32 * (warp >> 2), J = warp & 3;
 #pragma unroll
@@ -577,40 +622,65 @@ __device__ __forceinline__ void panel_store(double (*xs_)[LDM], double* out, int
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int r = rb + 8 * i + g, col = 8 * (c ? 7 - J : J) + 2 * t;
-      const double2 v = make_double2(acc[i][c][0], acc[i][c][1]);
-      *reinterpret_cast<double2*>(&xs_[r][col]) = v;
-      *reinterpret_cast<double2*>(out + (int64_t)r * ld + col) = v;
+      *reinterpret_cast<double2*>(&xs_[r][col]) = make_double2(acc[i][c][0], acc[i][c][1]);
     }
 }
 
-// T −= L·Lᵀ on the 36 lower 8×8 blocks of a 64×64 shared-memory tile (the
-// blocks above the diagonal are never read).  Warp w takes blocks w + 8·s, so
-// the two warps of each scheduler share nine blocks.
+// T −= L·Lᵀ on the lower triangle of a 64×64 shared-memory tile, in groups of
+// 2×2 blocks of 8×8 that share their fragment loads: warps 0–5 take the six
+// 16×16 groups below the diagonal (four products from four loads per k-step),
+// warps 6 and 7 two diagonal groups each (three products from two loads per
+// group; blocks above the diagonal are neither computed nor read).
 __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[LDM], int warp,
                                            int lane) {
   const int g = lane >> 2, t = lane & 3;
-  double acc[5][2] = {};
-  int bi[5], bj[5];
-#pragma unroll
-  for (int s = 0; s < 5; ++s) {
-    const int e = warp + 8 * s;
-    bi[s] = (e < 36) ? kTri8I[e] : 0;
-    bj[s] = (e < 36) ? kTri8J[e] : 0;
-  }
-#pragma unroll 2
-  for (int q = 0; q < NB; q += 4) {
-#pragma unroll
-    for (int s = 0; s < 5; ++s) {
-      if (warp + 8 * s < 36)
-        dmma_884(acc[s], l[8 * bi[s] + g][q + t], l[8 * bj[s] + g][q + t]);
+  if (warp < 6) {
+    // groups (I, J), I > J: warp 0 → (1,0), 1 → (2,0), 2 → (2,1), 3 → (3,0), ...
+    const int I = (warp < 1) ? 1 : ((warp < 3) ? 2 : 3);
+    const int J = warp - I * (I - 1) / 2;
+    const int ra = 16 * I + g, rb = 16 * J + g;
+    double acc[2][2][2] = {};
+#pragma unroll 4
+    for (int q = 0; q < NB; q += 4) {
+      const double a0 = l[ra][q + t], a1 = l[ra + 8][q + t];
+      const double b0 = l[rb][q + t], b1 = l[rb + 8][q + t];
+      dmma_884(acc[0][0], a0, b0);
+      dmma_884(acc[0][1], a0, b1);
+      dmma_884(acc[1][0], a1, b0);
+      dmma_884(acc[1][1], a1, b1);
     }
-  }
 #pragma unroll
-  for (int s = 0; s < 5; ++s) {
-    if (warp + 8 * s < 36) {
-      double2* p = reinterpret_cast<double2*>(&tt[8 * bi[s] + g][8 * bj[s] + 2 * t]);
-      const double2 o = *p;
-      *p = make_double2(o.x - acc[s][0], o.y - acc[s][1]);
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        double2* p = reinterpret_cast<double2*>(&tt[ra + 8 * i][16 * J + 8 * j + 2 * t]);
+        const double2 o = *p;
+        *p = make_double2(o.x - acc[i][j][0], o.y - acc[i][j][1]);
+      }
+  } else {
+    // diagonal groups 2·(warp − 6) and the next: blocks (0,0), (1,0), (1,1) of each
+    const int r0 = 32 * (warp - 6) + g;
+    double acc[2][3][2] = {};
+#pragma unroll 4
+    for (int q = 0; q < NB; q += 4) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const double u0 = l[r0 + 16 * h][q + t], u1 = l[r0 + 16 * h + 8][q + t];
+        dmma_884(acc[h][0], u0, u0);
+        dmma_884(acc[h][1], u1, u0);
+        dmma_884(acc[h][2], u1, u1);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = r0 + 16 * h, c = 32 * (warp - 6) + 16 * h + 2 * t;
+      double2* p0 = reinterpret_cast<double2*>(&tt[r][c]);
+      double2* p1 = reinterpret_cast<double2*>(&tt[r + 8][c]);
+      double2* p2 = reinterpret_cast<double2*>(&tt[r + 8][c + 8]);
+      const double2 o0 = *p0, o1 = *p1, o2 = *p2;
+      *p0 = make_double2(o0.x - acc[h][0][0], o0.y - acc[h][0][1]);
+      *p1 = make_double2(o1.x - acc[h][1][0], o1.y - acc[h][1][1]);
+      *p2 = make_double2(o2.x - acc[h][2][0], o2.y - acc[h][2][1]);
     }
   }
 }
@@ -693,17 +763,22 @@ __device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
 // warm): DIAG(k) — D_k = L_kk⁻¹ —, then PANEL(k,k+1) — L_{k+1,k} =
 // A_{k+1,k}·D_kᵀ — and the last update of tile (k+1,k+1), once those two
 // tiles have received their first k updates from the workers.
-// The other CTAs take the remaining tasks of step k (64-column block k) in
-// a fixed global order (those the next steps wait for first):
-//   PANEL(k,i) i > k+1, TRAIL(k,i,k+1) i > k+1, MROW(k,c) c < k,
-//   MTRAIL(k,k+1,c), TRAIL(k,i,j) k+1 < j ≤ i, MTRAIL(k,i,c) i > k+1
+// The other CTAs take the remaining tasks in a fixed global order of slots.
+// Slot s holds the factor tasks of step s (64-column block s), those the
+// next steps wait for first,
+//   PANEL(s,i) i > s+1, TRAIL(s,i,s+1) i > s+1, TRAIL(s,i,j) s+1 < j ≤ i,
+// and then the inverse tasks of step s − kMLag,
+//   MROW(k,c) c < k, MTRAIL(k,k+1,c), MTRAIL(k,i,c) i > k+1   (k = s − kMLag),
 // with PANEL:  L_ik = A_ik·D_kᵀ          (needs D_k and tile (i,k) updated k times)
 //      MROW:   M_kc = D_k·M_kc           (needs D_k and M_kc updated k−c times)
 //      TRAIL:  A_ij −= L_ik·L_jkᵀ         (needs L_ik, L_jk, tile (i,j) updated k times)
 //      MTRAIL: M_ic −= L_ik·M_kc          (needs L_ik, final M_kc, M_ic updated k−c times)
-// Every dependency of a task is an earlier task or a step of the chain, the
-// chain at step k waits only for tasks of step k−1, and tasks are taken in
-// order only by running CTAs, so the launch needs no co-residency guarantee.
+// The chain never reads M, so its tasks trail the factor by kMLag steps and
+// leave the workers to the tiles the chain waits for when a step has many
+// tasks.  Every dependency of a task is an earlier task or a step of the
+// chain, the chain at step k waits only for factor tasks of step k−1, and
+// tasks are taken in order only by running CTAs, so the launch needs no
+// co-residency guarantee.
 // Flags are set with release stores after a fence and polled with acquire
 // loads; every wait is bounded and a time-out (or a bad pivot) raises a
 // shared abort flag.
@@ -759,39 +834,54 @@ __device__ __forceinline__ void cta_signal(int* flag, int value) {
   }
 }
 
-__host__ __device__ inline int step_tasks(int N, int k) {
+constexpr int kMLag = 2;
+
+// Factor and inverse tasks of step k (r = N − k − 1 blocks below it).
+__host__ __device__ inline int factor_tasks(int N, int k) {
   const int r = N - k - 1;
-  if (r <= 0) return k;                              // MROW only
-  return 2 * (r - 1) + k + (k + 1) + (r - 1) * r / 2 + (r - 1) * (k + 1);
+  return r <= 0 ? 0 : 2 * (r - 1) + (r - 1) * r / 2;
+}
+__host__ __device__ inline int inverse_tasks(int N, int k) {
+  const int r = N - k - 1;
+  return r <= 0 ? k : k + (k + 1) + (r - 1) * (k + 1);
+}
+__host__ __device__ inline int slot_tasks(int N, int s) {
+  return (s < N ? factor_tasks(N, s) : 0) +
+         (s >= kMLag && s - kMLag < N ? inverse_tasks(N, s - kMLag) : 0);
 }
 
 int total_tasks(int N) {
   int t = 0;
-  for (int k = 0; k < N; ++k) t += step_tasks(N, k);
+  for (int s = 0; s < N + kMLag; ++s) t += slot_tasks(N, s);
   return t;
 }
 
 enum TaskKind { T_PANEL = 0, T_MROW, T_TRAIL, T_MTRAIL };
 
 __device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) {
-  k = 0;
-  while (task >= step_tasks(N, k)) { task -= step_tasks(N, k); ++k; }
+  int s = 0;
+  while (task >= slot_tasks(N, s)) { task -= slot_tasks(N, s); ++s; }
+  if (s < N) {
+    const int nf = factor_tasks(N, s);
+    if (task < nf) {
+      k = s;
+      const int r = N - k - 1;
+      if (task < r - 1) { kind = T_PANEL; i = k + 2 + task; j = k; return; }
+      task -= r - 1;
+      if (task < r - 1) { kind = T_TRAIL; i = k + 2 + task; j = k + 1; return; }
+      task -= r - 1;
+      int ii = 0;
+      while (task >= ii + 1) { task -= ii + 1; ++ii; }
+      kind = T_TRAIL; i = k + 2 + ii; j = k + 2 + task; return;
+    }
+    task -= nf;
+  }
+  k = s - kMLag;
   const int r = N - k - 1;
-  if (r <= 0) { kind = T_MROW; i = k; j = task; return; }
-  if (task < r - 1) { kind = T_PANEL; i = k + 2 + task; j = k; return; }
-  task -= r - 1;
-  if (task < r - 1) { kind = T_TRAIL; i = k + 2 + task; j = k + 1; return; }
-  task -= r - 1;
-  if (task < k) { kind = T_MROW; i = k; j = task; return; }
+  if (r <= 0 || task < k) { kind = T_MROW; i = k; j = task; return; }
   task -= k;
   if (task < k + 1) { kind = T_MTRAIL; i = k + 1; j = task; return; }
   task -= k + 1;
-  if (task < (r - 1) * r / 2) {
-    int ii = 0;
-    while (task >= ii + 1) { task -= ii + 1; ++ii; }
-    kind = T_TRAIL; i = k + 2 + ii; j = k + 2 + task; return;
-  }
-  task -= (r - 1) * r / 2;
   kind = T_MTRAIL; i = k + 2 + task / (k + 1); j = task % (k + 1);
 }
 
@@ -811,25 +901,38 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   if (s_role == 0) {
     // ---- the critical chain: DIAG(k), then PANEL(k, k+1) and the last
     // update of tile (k+1, k+1), which stays in shared memory for DIAG(k+1).
-    // Two buffers alternate as the diagonal tile.  D_k leaves block row by
-    // block row during DIAG(k), and L_{k+1,k} is published only after the
-    // update that follows it, so neither signal waits long for its stores.
+    // Two buffers alternate as the diagonal tile and two as D (warp 4 clears
+    // the one of the step before during the diagonal tile).  D_k leaves block
+    // row by block row during DIAG(k); L_{k+1,k} stays in shared memory and
+    // leaves (and is published) during the first block of DIAG(k+1), so that
+    // no store stands in the way of the chain's shared-memory loads.
     double (*t0)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
     double (*t1)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
-    double (*b)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * NB * LDM);
+    double (*b0)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * NB * LDM);
     double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 3 * NB * LDM);
-    double* xs = sm + 4 * NB * LDM;
+    double (*b1)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 4 * NB * LDM);
+    double* xs = sm + 5 * NB * LDM;
     load_lower(t0, A, np, tid);
-    zero_tile(b, tid);
+    zero_tile(b0, tid);
+    zero_tile(b1, tid);
     if (tid == 0) s_bad = 0;
     __syncthreads();
     for (int k = 0; k < N; ++k) {
       const int64_t base = (int64_t)k * NB;
       double (*a)[LDM] = (k & 1) ? t1 : t0;
       double (*an)[LDM] = (k & 1) ? t0 : t1;
+      double (*b)[LDM] = (k & 1) ? b1 : b0;
+      double (*bz)[LDM] = (k > 0) ? ((k & 1) ? b0 : b1) : nullptr;
       const bool more = k + 1 < N;
       double* Lp = A + (base + NB) * np + base;          // tile (k+1, k)
       const double* An = A + (base + NB) * np + base + NB;   // tile (k+1, k+1)
+      // L_{k,k−1}, computed in the step before, still in x
+      PanelOut po = {};
+      if (k > 0) {
+        po.src = x;
+        po.dst = A + base * np + base - NB;
+        po.flag = &S.pdone[(k - 1) * N + k];
+      }
       // warp 4 fetches the next step's two input tiles during the diagonal
       // tile, as soon as the workers have finished them
       TilePrefetch pf = {};
@@ -844,7 +947,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
         pf.dst[1] = an;
         pf.ld = np;
       }
-      if (!diag_tile_smem(a, b, xs, M + base * np + base, np, n, base, info, &s_bad, pf,
+      if (!diag_tile_smem(a, b, bz, xs, M + base * np + base, np, n, base, info, &s_bad, pf, po,
                           &s_stop, &s_got)) {
         if (tid == 0) atomicExch(&S.ctrl[2], 1);
         return;
@@ -865,8 +968,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       double acc[4][2][2] = {};
       panel_mm(x, b, acc, warp, lane);
       __syncthreads();
-      panel_store(x, Lp, np, acc, warp, lane);
-      zero_tile(b, tid);
+      panel_to_smem(x, acc, warp, lane);
       // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
       if (!(got & 2)) {
         if (!cta_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok)) return;
@@ -876,10 +978,6 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       __syncthreads();
       lower_syrk(an, x, warp, lane);
       __syncthreads();
-      if (tid == 0) {                 // L_{k+1,k} is out (its stores drained meanwhile)
-        __threadfence();
-        st_release(&S.pdone[k * N + k + 1], 1);
-      }
     }
     return;
   }
@@ -993,7 +1091,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  const size_t tile_smem = (4 * NB * LDM + 192) * sizeof(double);
+  const size_t tile_smem = (5 * NB * LDM + 192) * sizeof(double);
   if (!g_smem_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(chol_persistent_kernel,
               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
