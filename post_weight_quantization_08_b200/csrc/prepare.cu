@@ -229,9 +229,11 @@ struct PanelOut {
 // Named barriers of the diagonal tile (0 is __syncthreads): 1 joins the six
 // working warps (1–3, 5–7); 2 hands X and the next panel block from warp 0 to
 // them; 3 hands their finished trailing updates back to warp 0; 4 tells warp 4
-// that they have stored the panel of the step before.  Warp 4 shares warp 0's
-// scheduler and stays out of 1–3 (it prefetches).
-constexpr int kBarRest = 1, kBarX = 2, kBarDone = 3, kBarPanel = 4;
+// that they have stored the panel of the step before; 5 joins warps 0–3 and
+// 5–7 in the panel phase after the diagonal tile (warp 4 publishes the tile
+// meanwhile); 6 tells them there that warp 4's prefetched tiles have landed.
+// Warp 4 shares warp 0's scheduler and stays out of 1–3 and 5.
+constexpr int kBarRest = 1, kBarX = 2, kBarDone = 3, kBarPanel = 4, kBarChain = 5, kBarFetch = 6;
 constexpr int kRest = 192, kHand = 224;     // 6 working warps; + warp 0
 
 __device__ __forceinline__ void bar_sync(int id, int count) {
@@ -353,7 +355,7 @@ __device__ __forceinline__ int chol8_pairs(double (&l)[36], double (&x)[8], int 
 // reported through info (the factorisation runs to the end on zeros, so that
 // every barrier is met) and makes the function return false.  Called by a
 // whole CTA of 256 threads.
-__device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double (*bz)[LDM],
+__device__ __forceinline__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double (*bz)[LDM],
                                double* xs, double* __restrict__ dout, int64_t ld, int64_t n,
                                int64_t base, int32_t* info, int* bad_s, const TilePrefetch& pf,
                                const PanelOut& po, volatile int* s_stop, int* s_got) {
@@ -406,7 +408,8 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double (*bz)[
   } else if (warp == 4) {
     // The prefetcher: each tile of pf as soon as its flag says it is final
     // (lane 0 polls with acquire loads; the copies are cp.async through L2),
-    // until both are in or warp 0 is done.  The master skips what it got.
+    // until both are issued or warp 0 is done.  s_got says which were issued:
+    // the master copies the others itself.
     if (po.dst) {
       bar_sync(kBarPanel, kHand);       // the working warps have stored it
       if (lane == 0) {
@@ -444,8 +447,9 @@ __device__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM], double (*bz)[
       if (got == all || *s_stop) break;
       __nanosleep(128);
     }
+    // the copies land while the panel phase starts: warp 4 waits for them
+    // there and announces them on barrier kBarFetch
     asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) *s_got = got;
   } else {
     // v numbers the six working warps (warp 4 prefetches)
@@ -551,13 +555,13 @@ __device__ __forceinline__ void zero_tile(double (*dst)[LDM], int tid) {
     *reinterpret_cast<double2*>(&dst[e >> 5][(e & 31) * 2]) = make_double2(0.0, 0.0);
   }
 }
-// Asynchronous 64×64 tile copy global → shared memory (16-byte cp.async
-// through L2 only; tiles are rewritten by other CTAs of the same launch).
-__device__ __forceinline__ void copy_tile_async(double (*dst)[LDM], const double* src, int64_t ld,
-                                                int tid) {
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int e = tid + 256 * s;
+// Asynchronous 64×64 tile copies global → shared memory are 16-byte cp.async
+// through L2 only (tiles are rewritten by other CTAs of the same launch).
+__device__ __forceinline__ void copy_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// One tile, copied by the 224 threads of warps 0–3 and 5–7 (gt numbers them).
+__device__ __forceinline__ void copy_tile_async_group(double (*dst)[LDM], const double* src,
+                                                      int64_t ld, int gt) {
+  for (int e = gt; e < NB * NB / 2; e += kHand) {
     const int r = e >> 5, c = (e & 31) * 2;
     const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&dst[r][c]));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + (int64_t)r * ld + c)
@@ -565,7 +569,6 @@ __device__ __forceinline__ void copy_tile_async(double (*dst)[LDM], const double
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
-__device__ __forceinline__ void copy_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // L = A·Dᵀ for 64×64 shared-memory tiles with D lower triangular, so block
 // column J of L needs only q < 8·(J+1).  Warp w owns row blocks 4·(w/4) .. +4
@@ -574,70 +577,87 @@ __device__ __forceinline__ void copy_wait_all() { asm volatile("cp.async.wait_al
 // block (4·(w/4) + i, c ? 7 − J : J).  The k-loops have compile-time bounds
 // (one instance per J) and are unrolled, so that the fragment loads run ahead
 // of the products and the float64 pipe stays busy.
-template <int J>
+template <int J, int NH>
 __device__ __forceinline__ void panel_mm_j(const double (*x)[LDM], const double (*d)[LDM],
-                                           double acc[4][2][2], int rb, int g, int t) {
+                                           double acc[2][4][2][2], int rb, int g, int t) {
   constexpr int J1 = 7 - J, qlo = 8 * (J + 1), qhi = 8 * (J1 + 1);
 #pragma unroll
   for (int q = 0; q < qlo; q += 4) {
-    double a[4];
+    double a[NH][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[h][i] = x[rb + 32 * h + 8 * i + g][q + t];
     const double b0 = d[8 * J + g][q + t], b1 = d[8 * J1 + g][q + t];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      dmma_884(acc[i][0], a[i], b0);
-      dmma_884(acc[i][1], a[i], b1);
-    }
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dmma_884(acc[h][i][0], a[h][i], b0);
+        dmma_884(acc[h][i][1], a[h][i], b1);
+      }
   }
 #pragma unroll
   for (int q = qlo; q < qhi; q += 4) {
-    double a[4];
+    double a[NH][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[h][i] = x[rb + 32 * h + 8 * i + g][q + t];
     const double b1 = d[8 * J1 + g][q + t];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dmma_884(acc[i][1], a[i], b1);
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dmma_884(acc[h][i][1], a[h][i], b1);
   }
 }
+// The panel over warps 0–3 and 5–7: warp w ≠ 0 owns row blocks 4·(w/4) .. +4
+// and block columns J = w mod 4 and 7 − J; warp 0 owns both row halves of
+// J = 0 (what warps 0 and 4 would own), so that every scheduler keeps the
+// same share.  acc[h] is row half h (warp 0) or the warp's only half (h = 0).
 __device__ __forceinline__ void panel_mm(const double (*x)[LDM], const double (*d)[LDM],
-                                         double acc[4][2][2], int warp, int lane) {
+                                         double acc[2][4][2][2], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3, rb = 32 * (warp >> 2);
   switch (warp & 3) {
-    case 0: panel_mm_j<0>(x, d, acc, rb, g, t); break;
-    case 1: panel_mm_j<1>(x, d, acc, rb, g, t); break;
-    case 2: panel_mm_j<2>(x, d, acc, rb, g, t); break;
-    default: panel_mm_j<3>(x, d, acc, rb, g, t); break;
+    case 0: panel_mm_j<0, 2>(x, d, acc, 0, g, t); break;      // warp 0: both halves
+    case 1: panel_mm_j<1, 1>(x, d, acc, rb, g, t); break;
+    case 2: panel_mm_j<2, 1>(x, d, acc, rb, g, t); break;
+    default: panel_mm_j<3, 1>(x, d, acc, rb, g, t); break;
   }
 }
 
 // Writes the panel accumulators to a shared-memory tile (it goes to global
 // memory from there later, off the chain).
-__device__ __forceinline__ void panel_to_smem(double (*xs_)[LDM], const double acc[4][2][2],
+__device__ __forceinline__ void panel_to_smem(double (*xs_)[LDM], const double acc[2][4][2][2],
                                               int warp, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const int rb = 32 * (warp >> 2), J = warp & 3;
+  const int g = lane >> 2, t = lane & 3, J = warp & 3;
+  const int nh = (warp == 0) ? 2 : 1;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int h = 0; h < 2; ++h) {
+    if (h >= nh) break;
+    const int rb = (warp == 0) ? 32 * h : 32 * (warp >> 2);
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int r = rb + 8 * i + g, col = 8 * (c ? 7 - J : J) + 2 * t;
-      *reinterpret_cast<double2*>(&xs_[r][col]) = make_double2(acc[i][c][0], acc[i][c][1]);
-    }
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int r = rb + 8 * i + g, col = 8 * (c ? 7 - J : J) + 2 * t;
+        *reinterpret_cast<double2*>(&xs_[r][col]) = make_double2(acc[h][i][c][0], acc[h][i][c][1]);
+      }
+  }
 }
 
 // T −= L·Lᵀ on the lower triangle of a 64×64 shared-memory tile, in groups of
-// 2×2 blocks of 8×8 that share their fragment loads: warps 0–5 take the six
-// 16×16 groups below the diagonal (four products from four loads per k-step),
-// warps 6 and 7 two diagonal groups each (three products from two loads per
+// 2×2 blocks of 8×8 that share their fragment loads.  Group G < 6 is one of
+// the six 16×16 groups below the diagonal, (I, J) = (1,0), (2,0), (2,1),
+// (3,0), (3,1), (3,2) (four products from four loads per k-step); groups 6
+// and 7 are two diagonal groups each (three products from two loads per
 // group; blocks above the diagonal are neither computed nor read).
-__device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[LDM], int warp,
-                                           int lane) {
+__device__ __forceinline__ void lower_syrk_group(double (*tt)[LDM], const double (*l)[LDM],
+                                                 int G, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  if (warp < 6) {
-    // groups (I, J), I > J: warp 0 → (1,0), 1 → (2,0), 2 → (2,1), 3 → (3,0), ...
-    const int I = (warp < 1) ? 1 : ((warp < 3) ? 2 : 3);
-    const int J = warp - I * (I - 1) / 2;
+  if (G < 6) {
+    const int I = (G < 1) ? 1 : ((G < 3) ? 2 : 3);
+    const int J = G - I * (I - 1) / 2;
     const int ra = 16 * I + g, rb = 16 * J + g;
     double acc[2][2][2] = {};
 #pragma unroll 4
@@ -658,8 +678,8 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
         *p = make_double2(o.x - acc[i][j][0], o.y - acc[i][j][1]);
       }
   } else {
-    // diagonal groups 2·(warp − 6) and the next: blocks (0,0), (1,0), (1,1) of each
-    const int r0 = 32 * (warp - 6) + g;
+    // diagonal groups 2·(G − 6) and the next: blocks (0,0), (1,0), (1,1) of each
+    const int r0 = 32 * (G - 6) + g;
     double acc[2][3][2] = {};
 #pragma unroll 4
     for (int q = 0; q < NB; q += 4) {
@@ -673,7 +693,7 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int r = r0 + 16 * h, c = 32 * (warp - 6) + 16 * h + 2 * t;
+      const int r = r0 + 16 * h, c = 32 * (G - 6) + 16 * h + 2 * t;
       double2* p0 = reinterpret_cast<double2*>(&tt[r][c]);
       double2* p1 = reinterpret_cast<double2*>(&tt[r + 8][c]);
       double2* p2 = reinterpret_cast<double2*>(&tt[r + 8][c + 8]);
@@ -683,6 +703,12 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
       *p2 = make_double2(o2.x - acc[h][2][0], o2.y - acc[h][2][1]);
     }
   }
+}
+// Over warps 0–3 and 5–7: warp w takes group w, and warp 0 also group 4.
+__device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[LDM], int warp,
+                                           int lane) {
+  lower_syrk_group(tt, l, warp, lane);
+  if (warp == 0) lower_syrk_group(tt, l, 4, lane);
 }
 
 // 64×64 float64 tile products.  Warp w owns rows 16·(w/2) .. +16 and columns
@@ -826,6 +852,28 @@ __device__ bool cta_wait(const int* flag, int target, int* abortp, int32_t* info
   return ok;
 }
 
+// The same wait for warps 0–3 and 5–7 (thread 0 polls), joined by barrier
+// kBarChain.
+__device__ bool group_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok) {
+  if (threadIdx.x == 0) {
+    bool ok = false;
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+      if (ld_acquire(flag) >= target) { ok = true; break; }
+      if (*reinterpret_cast<volatile int*>(abortp)) break;
+      if (it > 32) __nanosleep(64);
+    }
+    if (!ok && !*reinterpret_cast<volatile int*>(abortp)) {
+      report(info, GPTQ_ERR_TIMEOUT, target);
+      atomicExch(abortp, 1);
+    }
+    *s_ok = ok ? 1 : 0;
+  }
+  bar_sync(kBarChain, kHand);
+  const bool ok = *s_ok != 0;
+  bar_sync(kBarChain, kHand);
+  return ok;
+}
+
 __device__ __forceinline__ void cta_signal(int* flag, int value) {
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -890,7 +938,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int64_t n, int64_t np, int N,
                        int ntasks, int* sync_base, int32_t* info) {
   extern __shared__ double sm[];
-  __shared__ int s_role, s_task, s_ok, s_bad, s_got;
+  __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail;
   __shared__ volatile int s_stop;
   const CholSync S = sync_view(sync_base, N);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -915,7 +963,10 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     load_lower(t0, A, np, tid);
     zero_tile(b0, tid);
     zero_tile(b1, tid);
-    if (tid == 0) s_bad = 0;
+    if (tid == 0) {
+      s_bad = 0;
+      s_fail = 0;
+    }
     __syncthreads();
     for (int k = 0; k < N; ++k) {
       const int64_t base = (int64_t)k * NB;
@@ -952,32 +1003,61 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
         if (tid == 0) atomicExch(&S.ctrl[2], 1);
         return;
       }
-      if (tid == 0) {                 // D_k is out (the diagonal tile ended with a barrier)
-        __threadfence();
-        st_release(&S.diag_done[k], 1);
+      if (!more) {
+        if (tid == 0) {               // D_k is out (the diagonal tile ended with a barrier)
+          __threadfence();
+          st_release(&S.diag_done[k], 1);
+        }
+        break;
       }
-      if (!more) break;
       const int got = s_got;                        // read after the tile's last barrier
-      // L_{k+1,k} = A_{k+1,k}·D_kᵀ
-      if (!(got & 1)) {
-        if (!cta_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok)) return;
-        copy_tile_async(x, Lp, np, tid);
-        copy_wait_all();
+      if (warp == 4) {
+        if (got) {                    // the prefetched tiles have landed
+          asm volatile("cp.async.wait_all;" ::: "memory");
+          __syncwarp();
+          bar_arrive(kBarFetch, kHand + 32);
+        }
+        // D_k is out (the diagonal tile ended with a barrier); the fence waits
+        // for its last stores while the other warps compute the panel
+        if (lane == 0) {
+          __threadfence();
+          st_release(&S.diag_done[k], 1);
+        }
+      } else {
+        const int gt = (warp < 4) ? tid : tid - 32;   // 0..223 over warps 0–3, 5–7
+        bool ok = true;
+        if (got) bar_sync(kBarFetch, kHand + 32);
+        // L_{k+1,k} = A_{k+1,k}·D_kᵀ
+        if (!(got & 1)) {
+          ok = group_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok);
+          if (ok) {
+            copy_tile_async_group(x, Lp, np, gt);
+            copy_wait_all();
+          }
+        }
+        if (ok) {
+          bar_sync(kBarChain, kHand);
+          double acc[2][4][2][2] = {};
+          panel_mm(x, b, acc, warp, lane);
+          bar_sync(kBarChain, kHand);
+          panel_to_smem(x, acc, warp, lane);
+          // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
+          if (!(got & 2)) {
+            ok = group_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok);
+            if (ok) {
+              copy_tile_async_group(an, An, np, gt);
+              copy_wait_all();
+            }
+          }
+          if (ok) {
+            bar_sync(kBarChain, kHand);
+            lower_syrk(an, x, warp, lane);
+          }
+        }
+        if (!ok && tid == 0) s_fail = 1;
       }
       __syncthreads();
-      double acc[4][2][2] = {};
-      panel_mm(x, b, acc, warp, lane);
-      __syncthreads();
-      panel_to_smem(x, acc, warp, lane);
-      // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
-      if (!(got & 2)) {
-        if (!cta_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok)) return;
-        copy_tile_async(an, An, np, tid);
-        copy_wait_all();
-      }
-      __syncthreads();
-      lower_syrk(an, x, warp, lane);
-      __syncthreads();
+      if (s_fail) return;
     }
     return;
   }
