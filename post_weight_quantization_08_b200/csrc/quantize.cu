@@ -236,16 +236,21 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
   //  * block b+1's columns: on the tensor-core path, sweep b+1 applies them
   //    itself in its prologue (in TMEM, before its first column); otherwise a
   //    trailing update on the caller's stream;
-  //  * the columns from block b+2 on: a trailing update on the side stream,
+  //  * the columns from block b+2 on: on the tensor-core path, CTAs of sweep
+  //    b+1's own launch (those columns are not sweep b+1's, and the errors
+  //    come from the launch before), so that the sweeps follow each other on
+  //    one stream; otherwise a trailing update on the side stream,
   //    overlapping sweep b+1.
   // Every column still receives the blocks' contributions in block order:
   // whatever touches block b's columns first waits for the far update of
   // block b−2 (which also reached them), and the two error buffers alternate,
   // so a far update's input is not overwritten before it is read.
-  SideStream* side = nullptr;
-  st = side_stream_for(s, &side);
-  if (st != GPTQ_OK) return st;
   const bool fused = w.Uhi != nullptr && trailing_uses_tensor_cores(n, block);
+  SideStream* side = nullptr;
+  if (!fused) {
+    st = side_stream_for(s, &side);
+    if (st != GPTQ_OK) return st;
+  }
   bool pending[2] = {false, false};
   for (int64_t j0 = 0, b = 0; j0 < n; j0 += block, ++b) {
     const int bw = (int)((n - j0 < block) ? (n - j0) : block);
@@ -256,28 +261,29 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
       pending[b & 1] = false;
     }
     SweepPrologue pre;
+    SweepFar far;
     if (fused && b > 0) {
-      pre.Ehi = w.Ehi[(b - 1) & 1];
-      pre.Elo = w.Elo[(b - 1) & 1];
-      pre.Uhi = w.Uhi;
-      pre.Ulo = w.Ulo;
-      pre.k0 = j0 - block;
-      pre.kw = block;
+      pre.Ehi = far.Ehi = w.Ehi[(b - 1) & 1];
+      pre.Elo = far.Elo = w.Elo[(b - 1) & 1];
+      pre.Uhi = far.Uhi = w.Uhi;
+      pre.Ulo = far.Ulo = w.Ulo;
+      pre.k0 = far.k0 = j0 - block;
+      pre.kw = far.kw = block;
+      far.c0 = j0 + bw;                        // block b+1 on: the far columns of block b−1
+      far.c1 = n;
     }
     const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
     st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes, scale,
-                      zero, ehi, elo, pre, loss_row, info, s);
+                      zero, ehi, elo, pre, far, loss_row, info, s);
     if (st != GPTQ_OK) return st;
     const int64_t c0 = j0 + bw, c1 = c0 + block;
-    if (c0 >= n) break;
-    if (!fused) {
-      if (b > 0 && pending[(b - 1) & 1]) {     // the far update of block b−1
-        GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[(b - 1) & 1], 0));
-        pending[(b - 1) & 1] = false;
-      }
-      st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info, s);
-      if (st != GPTQ_OK) return st;
+    if (c0 >= n || fused) continue;
+    if (b > 0 && pending[(b - 1) & 1]) {       // the far update of block b−1
+      GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[(b - 1) & 1], 0));
+      pending[(b - 1) & 1] = false;
     }
+    st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info, s);
+    if (st != GPTQ_OK) return st;
     if (c1 < n) {
       GPTQ_CUDA(cudaEventRecord(side->swept, s));
       GPTQ_CUDA(cudaStreamWaitEvent(side->s2, side->swept, 0));

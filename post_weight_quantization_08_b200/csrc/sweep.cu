@@ -32,6 +32,7 @@
 
 #include "kernels.cuh"
 #include "sm100.cuh"
+#include "trailing_tc.cuh"
 
 namespace gptq {
 namespace {
@@ -67,7 +68,7 @@ constexpr uint32_t SM_CODES = SM_VALS + 4 * VBOX;
 constexpr uint32_t SM_BPHI = (SM_CODES + RT * LDB + 1023) / 1024 * 1024;
 constexpr uint32_t SM_BPLO = SM_CODES;
 constexpr uint32_t SM_BARS = SM_BPHI + 32 * RT * 4;
-constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 64;
+constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 128;
 static_assert(SM_AHI >= PK_BYTES && SM_AHI % 1024 == 0, "A operand placement");
 static_assert(SM_VALS % 1024 == 0, "the strip's boxes use the 128-byte swizzle");
 static_assert(SM_CODES % 1024 == 0 && RT * LDB >= 32 * RT * 4, "U chunk lo part placement");
@@ -152,17 +153,16 @@ __device__ __forceinline__ float div_fma(float x, float s, float rs) {
   return fmaf(r, rs, q0);
 }
 
-__global__ void __launch_bounds__(RT, 1)
-sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
-             const __grid_constant__ CUtensorMap tmW, int strip_tma,
-             const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmPlo,
-             const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo,
-             int64_t k0p, int kwp,
-             const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
-             const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
-             uint8_t* __restrict__ codes, float* __restrict__ scale,
-             uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info) {
-  extern __shared__ unsigned char smraw[];
+// One CTA (bx: the 128-row tile) of the sweep; smraw: SMEM_BYTES of dynamic
+// shared memory.
+__device__ __forceinline__ void sweep_body(
+    const CUtensorMap& tmEhi, const CUtensorMap& tmElo, const CUtensorMap& tmW, int strip_tma,
+    const CUtensorMap& tmPhi, const CUtensorMap& tmPlo, const CUtensorMap& tmUhi,
+    const CUtensorMap& tmUlo, int64_t k0p, int kwp, const float* __restrict__ Wp, int64_t m,
+    int64_t n, int64_t j0, int bw, const unsigned char* __restrict__ pkg, int bits, int group,
+    int64_t ngroups, uint8_t* __restrict__ codes, float* __restrict__ scale,
+    uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info, int bx,
+    unsigned char* smraw) {
   const uint32_t raw = smem_addr(smraw);
   unsigned char* sm = smraw + ((1024 - (raw & 1023)) & 1023);
   const float* Ud = reinterpret_cast<const float*>(sm + SM_PKG + PK_UD);
@@ -173,22 +173,26 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   uint8_t* cs = sm + SM_CODES;
   uint64_t* pkg_bar = reinterpret_cast<uint64_t*>(sm + SM_BARS);
   uint64_t* mma_bar = pkg_bar + 1;
-  uint64_t* pro_bar = mma_bar + 1;      // prologue chunk loads
-  uint64_t* pro_mma = pro_bar + 1;      // prologue products but the last
-  uint64_t* pro_done = pro_mma + 1;     // the last prologue product
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(pro_done + 1);
+  uint64_t* pro_bar = mma_bar + 1;      // prologue chunk loads, one per buffer set
+  uint64_t* pro_mma = pro_bar + 2;      // prologue products but the last, one per set
+  uint64_t* pro_done = pro_mma + 2;     // the last prologue product
+  uint64_t* strip_bar = pro_done + 1;   // the strip's four boxes
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(strip_bar + 1);
   const bool pro = kwp > 0;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int64_t r0 = (int64_t)blockIdx.x * RT;
+  const int64_t r0 = (int64_t)bx * RT;
   const int64_t row = r0 + t;
 
   if (t == 0) {
     mbar_init(pkg_bar, 1);
     mbar_init(mma_bar, 1);
-    mbar_init(pro_bar, 1);
-    mbar_init(pro_mma, 1);
+    mbar_init(&pro_bar[0], 1);
+    mbar_init(&pro_bar[1], 1);
+    mbar_init(&pro_mma[0], 1);
+    mbar_init(&pro_mma[1], 1);
     mbar_init(pro_done, 1);
+    mbar_init(strip_bar, 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -203,39 +207,55 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   pdl_wait();                           // the strip was written by the previous kernel
   pdl_trigger();
   if (t == 0) {
-    // the package and, when the rows allow a tensor map, the strip: four
-    // boxes at (j0 + 32q, r0); columns past n read as zero, and Wp holds whole
-    // 128-row boxes
-    mbar_arrive_expect_tx(pkg_bar, PK_BYTES + (strip_tma ? 4 * VBOX : 0));
-    bulk_g2s(sm + SM_PKG, pkg, PK_BYTES, pkg_bar);
+    // the strip, when the rows allow a tensor map: four boxes at (j0 + 32q,
+    // r0); columns past n read as zero, and Wp holds whole 128-row boxes
     if (strip_tma) {
+      mbar_arrive_expect_tx(strip_bar, 4 * VBOX);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        tma_load_2d(vals + q * VBOX, &tmW, (int)j0 + 32 * q, (int)r0, pkg_bar);
+        tma_load_2d(vals + q * VBOX, &tmW, (int)j0 + 32 * q, (int)r0, strip_bar);
     }
-    if (pro) {
+    if (!pro) {
+      mbar_arrive_expect_tx(pkg_bar, PK_BYTES);
+      bulk_g2s(sm + SM_PKG, pkg, PK_BYTES, pkg_bar);
+    } else {
       // Prologue: D = E_prev·U[prev block, this block] in TMEM, the previous
       // block's contribution to this block's columns (the part of the
       // lazy-batch update the next sweep needs first), 3xTF32 like the
-      // trailing update, in K-chunks of 32 through the A buffers and the U
-      // chunk boxes.  Chunks but the last complete on pro_mma, the last on
-      // pro_done, which every thread waits for before reading D.
+      // trailing update, in K-chunks of 32.  The chunks alternate between two
+      // buffer sets, the A/B buffers and the package's region, so that the
+      // next chunk's copies run under this chunk's products; the package
+      // follows the last product (all threads wait for pro_done before they
+      // read D, and for the package before the first column step).
       const int nk = kwp / SS;
       const uint32_t idesc = idesc_f32acc(2, 2, 0, 0, RT, SB);
-      const uint32_t ah = smem_addr(ahi), al = smem_addr(alo);
-      const uint32_t bh = smem_addr(sm + SM_BPHI), bl = smem_addr(sm + SM_BPLO);
-      for (int c = 0; c < nk; ++c) {
-        mbar_arrive_expect_tx(pro_bar, 4 * VBOX);
-        tma_load_2d(ahi, &tmPhi, SS * c, (int)r0, pro_bar);
-        tma_load_2d(alo, &tmPlo, SS * c, (int)r0, pro_bar);
-        tma_load_2d(sm + SM_BPHI, &tmUhi, (int)k0p + SS * c, (int)j0, pro_bar);
-        tma_load_2d(sm + SM_BPLO, &tmUlo, (int)k0p + SS * c, (int)j0, pro_bar);
-        if (!mbar_wait_bounded(pro_bar, c & 1)) {
-          report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
-          mbar_wait_bounded(pro_bar, c & 1);          // let our own copies land first
+      auto opnd = [&](int st, int w) -> unsigned char* {      // w: A hi, A lo, B hi, B lo
+        if (st) return sm + SM_PKG + w * VBOX;
+        return w == 0 ? ahi : (w == 1 ? alo : (w == 2 ? sm + SM_BPHI : sm + SM_BPLO));
+      };
+      auto load = [&](int c) {
+        const int st = c & 1;
+        mbar_arrive_expect_tx(&pro_bar[st], 4 * VBOX);
+        tma_load_2d(opnd(st, 0), &tmPhi, SS * c, (int)r0, &pro_bar[st]);
+        tma_load_2d(opnd(st, 1), &tmPlo, SS * c, (int)r0, &pro_bar[st]);
+        tma_load_2d(opnd(st, 2), &tmUhi, (int)k0p + SS * c, (int)j0, &pro_bar[st]);
+        tma_load_2d(opnd(st, 3), &tmUlo, (int)k0p + SS * c, (int)j0, &pro_bar[st]);
+      };
+      load(0);
+      if (nk > 1) load(1);
+      int landed = 0;                   // chunks whose copies are known to have landed
+      const int loaded = nk;            // every chunk is loaded unless a wait fails
+      bool fail = false;
+      for (int c = 0; c < nk && !fail; ++c) {
+        const int st = c & 1;
+        if (!mbar_wait_bounded(&pro_bar[st], (c >> 1) & 1)) {
+          fail = true;
           break;
         }
+        landed = c + 1;
         tc_fence_after();
+        const uint32_t ah = smem_addr(opnd(st, 0)), al = smem_addr(opnd(st, 1));
+        const uint32_t bh = smem_addr(opnd(st, 2)), bl = smem_addr(opnd(st, 3));
 #pragma unroll
         for (int ks = 0; ks < SS / 8; ++ks) {
           const uint64_t dah = sdesc_sw128(ah + ks * 32, SW128_KMAJOR_LBO, 1024);
@@ -246,15 +266,25 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
           umma_tf32_ss(tmem, dah, dbl, idesc, 1u);
           umma_tf32_ss(tmem, dal, dbh, idesc, 1u);
         }
-        if (c + 1 < nk) {
-          umma_commit(pro_mma);
-          if (!mbar_wait_bounded(pro_mma, c & 1)) {     // the buffers are read again next
-            report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+        umma_commit(c + 1 < nk ? &pro_mma[st] : pro_done);
+        // the set of chunk c − 1 is free once its products are: chunk c + 1
+        if (c >= 1 && c + 1 < nk) {
+          if (!mbar_wait_bounded(&pro_mma[(c - 1) & 1], ((c - 1) >> 1) & 1)) {
+            fail = true;
             break;
           }
-        } else {
-          umma_commit(pro_done);
+          load(c + 1);
         }
+      }
+      if (fail) {
+        report(info, GPTQ_ERR_TIMEOUT, bx);
+        // let our own copies land before the CTA gives up (at most two sets
+        // are in flight: chunks landed and landed + 1)
+        for (int c = landed; c < loaded && c < landed + 2; ++c)
+          mbar_wait_bounded(&pro_bar[c & 1], (c >> 1) & 1);
+      } else if (mbar_wait_bounded(pro_done, 0)) {
+        mbar_arrive_expect_tx(pkg_bar, PK_BYTES);  // the package's region is free again
+        bulk_g2s(sm + SM_PKG, pkg, PK_BYTES, pkg_bar);
       }
     }
   }
@@ -289,10 +319,17 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
     __syncthreads();
   }
 
-  bool abort = !mbar_wait_bounded(pkg_bar, 0);
+  // the strip (and, without a prologue, the package); with a prologue the
+  // package is waited for after the group statistics, before the first step
+  bool ok0 = !strip_tma || mbar_wait_bounded(strip_bar, 0);
+  if (!pro) ok0 = mbar_wait_bounded(pkg_bar, 0) && ok0;
+  bool abort = __syncthreads_or(!ok0) != 0;
   if (abort) {
-    report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
-    if (t == 0) mbar_wait_bounded(pkg_bar, 0);   // let our own copy land first
+    report(info, GPTQ_ERR_TIMEOUT, bx);
+    if (t == 0) {                       // let our own copies land first
+      if (strip_tma) mbar_wait_bounded(strip_bar, 0);
+      if (!pro) mbar_wait_bounded(pkg_bar, 0);
+    }
   }
 
   const float maxq = (float)((1 << bits) - 1);
@@ -308,7 +345,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
       if (pro) {
         const bool ok = mbar_wait_bounded(pro_done, 0);
         if (__syncthreads_or(!ok)) {
-          report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+          report(info, GPTQ_ERR_TIMEOUT, bx);
           abort = true;
           break;
         }
@@ -327,7 +364,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
       const bool ok = mbar_wait_bounded(mma_bar, (sb - 1) & 1);
       if (t == 0) bulk_wait_read_all();   // the previous errors have left the A buffers
       if (__syncthreads_or(!ok)) {
-        report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
+        report(info, GPTQ_ERR_TIMEOUT, bx);
         abort = true;
         break;
       }
@@ -380,6 +417,15 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
         const int64_t g = (j0 + c0) / group;
         scale[row * ngroups + g] = s;
         zero[row * ngroups + g] = (uint8_t)z;
+      }
+    }
+    if (sb == 0 && pro) {               // the package, loaded after the prologue
+      const bool okp = mbar_wait_bounded(pkg_bar, 0);
+      if (__syncthreads_or(!okp)) {
+        report(info, GPTQ_ERR_TIMEOUT, bx);
+        if (t == 0) mbar_wait_bounded(pkg_bar, 0);   // let our own copy land first
+        abort = true;
+        break;
       }
     }
     // ---- the 32 dependent column steps
@@ -486,6 +532,34 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   if (warp == 0) tmem_dealloc(tmem, SB);
 }
 
+// The sweep of one block (CTAs 0 .. nsweep−1) and, in the same launch, the
+// far-column update of the block before (the CTAs after them, fx tiles of
+// 256 columns per 128-row tile): the two touch different columns, and both
+// take their inputs from earlier launches, so that consecutive sweeps follow
+// each other with nothing between them but the programmatic launch edge.
+__global__ void __launch_bounds__(RT, 1)
+sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
+             const __grid_constant__ CUtensorMap tmW, int strip_tma,
+             const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmPlo,
+             const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo,
+             int64_t k0p, int kwp,
+             const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
+             const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
+             uint8_t* __restrict__ codes, float* __restrict__ scale,
+             uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info,
+             int nsweep, const __grid_constant__ TrailMaps far, int64_t fc0, int64_t fc1,
+             int64_t fk0, int fkw, int fx) {
+  extern __shared__ unsigned char smraw[];
+  const int b = (int)blockIdx.x;
+  if (b < nsweep) {
+    sweep_body(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp, Wp, m, n, j0,
+               bw, pkg, bits, group, ngroups, codes, scale, zero, loss_row, info, b, smraw);
+  } else {
+    const int f = b - nsweep;
+    trailing_tc_body(far, m, n, fc0, fc1, fk0, fkw, info, f % fx, f / fx, smraw);
+  }
+}
+
 bool g_attr_set = false;
 
 }  // namespace
@@ -502,15 +576,29 @@ gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
   return GPTQ_OK;
 }
 
-gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
+gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
-                         float* Elo, const SweepPrologue& pre, float* loss_row, int32_t* info,
-                         cudaStream_t s) {
+                         float* Elo, const SweepPrologue& pre, const SweepFar& far,
+                         float* loss_row, int32_t* info, cudaStream_t s) {
+  constexpr size_t kSmem = SMEM_BYTES > QSMEM ? SMEM_BYTES : QSMEM;
   if (!g_attr_set) {
     GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)SMEM_BYTES));
+                                   (int)kSmem));
     g_attr_set = true;
+  }
+  // the far-column update riding along: fx 256-column tiles per 128-row tile
+  TrailMaps fm;
+  memset(&fm, 0, sizeof(fm));
+  const int64_t fc1 = far.c1 < n ? far.c1 : n;
+  int fx = 0, nfar = 0;
+  if (far.kw > 0 && far.c0 < fc1 && far.Ehi && far.Elo && far.Uhi && far.Ulo) {
+    if (far.kw % QK != 0 || far.kw > SB || (n % 4) != 0)
+      return fail(GPTQ_ERR_INVALID_ARG, "sweep far update: width %d", far.kw);
+    if (!make_trail_maps(&fm, Wp, m, n, far.Ehi, far.Elo, far.Uhi, far.Ulo))
+      return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's far update");
+    fx = (int)ceil_div(fc1 - far.c0, QN);
+    nfar = fx * (int)ceil_div(m, QM);
   }
   CUtensorMap th, tl;
   const int64_t mr = error_rows(m);     // whole boxes: a clipped box store is slow
@@ -539,12 +627,13 @@ gptq_status launch_sweep(const float* Wp, int64_t m, int64_t n, int64_t j0, int 
   if (!encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ehi, SB, mr, SB * 4, SS, RT) ||
       !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, SB * 4, SS, RT))
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
-  const unsigned grid = (unsigned)ceil_div(m, RT);
-  GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel, grid, RT, SMEM_BYTES, th, tl, tw, strip_tma, tph,
-                  tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m,
-              n, j0, bw,
-              reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
-              scale, zero, loss_row, info);
+  const int nsweep = (int)ceil_div(m, RT);
+  const unsigned grid = (unsigned)(nsweep + nfar);
+  GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel, grid, RT, kSmem, th, tl, tw, strip_tma, tph, tpl,
+                  tuh, tul, (int64_t)pre.k0, kwp, (const float*)Wp, m, n, j0, bw,
+                  reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
+                  scale, zero, loss_row, info, nsweep, fm, far.c0, fc1, far.k0, far.kw,
+                  fx > 0 ? fx : 1);
   return GPTQ_OK;
 }
 

@@ -29,6 +29,7 @@
 
 #include "kernels.cuh"
 #include "sm100.cuh"
+#include "trailing_tc.cuh"
 
 namespace gptq {
 namespace {
@@ -117,135 +118,11 @@ split_tf32_t_kernel(const float* __restrict__ x, int64_t n, float* __restrict__ 
 
 // ---------------------------------------------------------------- tcgen05 path
 
-constexpr int QM = 128, QN = 256, QK = 32, QSTAGES = 2;
-constexpr uint32_t A_BOX = QK * QM * 4;          // 32 K × 128 rows, 16 KB
-constexpr uint32_t B_OPER = QK * QN * 4;         // 32 K × 256 columns, 32 KB
-constexpr uint32_t STAGE = 2 * A_BOX + 2 * B_OPER;          // 96 KB
-constexpr uint32_t C_BOX = 32 * QM * 4;                     // 32 columns × 128 rows
-constexpr uint32_t QIDESC = idesc_f32acc(2, 2, 0, 0, QM, QN) | (1u << 13);  // tf32 K-major, −A
-constexpr size_t QSMEM = 1024 + QSTAGES * STAGE + 256;
-static_assert(QSTAGES * STAGE >= (QN / 32) * C_BOX, "epilogue boxes reuse the ring");
-
-struct TrailMaps {
-  CUtensorMap ahi, alo, bhi, blo, c;
-};
-
 __global__ void __launch_bounds__(128, 1)
 trailing_tc_kernel(const __grid_constant__ TrailMaps maps, int64_t m, int64_t n, int64_t c0,
                    int64_t c1, int64_t k0, int kw, int32_t* info) {
   extern __shared__ unsigned char smraw[];
-  const uint32_t raw = smem_addr(smraw);
-  unsigned char* ring = smraw + ((1024 - (raw & 1023)) & 1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + QSTAGES * STAGE);
-  uint64_t* empty = full + QSTAGES;
-  uint64_t* done = empty + QSTAGES;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r0 = blockIdx.y * QM;
-  const int cb = (int)(c0 + (int64_t)blockIdx.x * QN);
-  const int nk = kw / QK;
-
-  if (tid == 0) {
-    for (int s = 0; s < QSTAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tslot, QN);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-  pdl_wait();                           // the errors come from the previous kernel
-  pdl_trigger();
-
-  if (warp == 0 && lane == 0) {
-    for (int c = 0; c < nk; ++c) {
-      const int s = c % QSTAGES;
-      if (c >= QSTAGES && !mbar_wait_bounded(&empty[s], ((c / QSTAGES) - 1) & 1)) {
-        report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
-        *abort_flag = 1;
-        break;
-      }
-      unsigned char* st = ring + s * STAGE;
-      const int kq = c * QK;
-      mbar_arrive_expect_tx(&full[s], STAGE);
-      tma_load_2d(st, &maps.ahi, kq, r0, &full[s]);
-      tma_load_2d(st + A_BOX, &maps.alo, kq, r0, &full[s]);
-      tma_load_2d(st + 2 * A_BOX, &maps.bhi, (int)k0 + kq, cb, &full[s]);
-      tma_load_2d(st + 2 * A_BOX + B_OPER, &maps.blo, (int)k0 + kq, cb, &full[s]);
-    }
-  } else if (warp == 1 && lane == 0) {
-    for (int c = 0; c < nk; ++c) {
-      const int s = c % QSTAGES;
-      if (!mbar_wait_bounded(&full[s], (c / QSTAGES) & 1)) {
-        report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
-        *abort_flag = 1;
-        break;
-      }
-      if (*abort_flag) break;
-      tc_fence_after();
-      const uint32_t st = smem_addr(ring + s * STAGE);
-      const uint32_t ahi = st, alo = st + A_BOX;
-      const uint32_t bhi = st + 2 * A_BOX, blo = bhi + B_OPER;
-#pragma unroll
-      for (int ks = 0; ks < QK / 8; ++ks) {
-        // both K-major: 8 TF32 = 32 bytes further inside each 128-byte row;
-        // 8-row groups 1024 bytes apart.
-        const uint64_t dah = sdesc_sw128(ahi + ks * 32, SW128_KMAJOR_LBO, 1024);
-        const uint64_t dal = sdesc_sw128(alo + ks * 32, SW128_KMAJOR_LBO, 1024);
-        const uint64_t dbh = sdesc_sw128(bhi + ks * 32, SW128_KMAJOR_LBO, 1024);
-        const uint64_t dbl = sdesc_sw128(blo + ks * 32, SW128_KMAJOR_LBO, 1024);
-        umma_tf32_ss(tmem, dah, dbh, QIDESC, (c > 0 || ks > 0) ? 1u : 0u);
-        umma_tf32_ss(tmem, dah, dbl, QIDESC, 1u);
-        umma_tf32_ss(tmem, dal, dbh, QIDESC, 1u);
-      }
-      umma_commit(&empty[s]);
-    }
-    umma_commit(done);
-  }
-  __syncwarp();
-
-  const bool ok = mbar_wait_bounded(done, 0);
-  if (!ok) report(info, GPTQ_ERR_TIMEOUT, blockIdx.x);
-  tc_fence_after();
-  const bool write = ok && !*abort_flag;
-  if (write) {
-    // −Err·U rows into 128-byte-swizzled boxes (row r at r·128 B, 16-byte
-    // chunk q stored at chunk q ^ (r mod 8)), which the TMA reduce reads.
-    const int r = warp * 32 + lane;
-#pragma unroll 1
-    for (int b = 0; b < QN / 32; ++b) {
-      float v[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + b * 32, v);
-      unsigned char* box = ring + b * C_BOX + r * 128;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float4 w = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        *reinterpret_cast<float4*>(box + ((q ^ (r & 7)) * 16)) = w;
-      }
-    }
-    fence_proxy_async_smem();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (write && tid == 0) {
-#pragma unroll 1
-    for (int b = 0; b < QN / 32; ++b)
-      if ((int64_t)cb + 32 * b < c1) tma_reduce_add_2d(&maps.c, cb + 32 * b, r0, ring + b * C_BOX);
-    bulk_commit();
-    bulk_wait_all();
-  }
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, QN);
+  trailing_tc_body(maps, m, n, c0, c1, k0, kw, info, (int)blockIdx.x, (int)blockIdx.y, smraw);
 }
 
 bool encode_f32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
@@ -257,6 +134,16 @@ bool encode_f32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t oute
 bool g_attr = false;
 
 }  // namespace
+
+bool make_trail_maps(TrailMaps* maps, float* Wp, int64_t m, int64_t n, const float* Ehi,
+                     const float* Elo, const float* UhiT, const float* UloT) {
+  const int64_t mr = error_rows(m);
+  return encode_f32(&maps->ahi, Ehi, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
+         encode_f32(&maps->alo, Elo, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
+         encode_f32(&maps->bhi, UhiT, n, n, n * 4, QK, QN) &&
+         encode_f32(&maps->blo, UloT, n, n, n * 4, QK, QN) &&
+         encode_f32(&maps->c, Wp, n, mr, n * 4, 32, QM);
+}
 
 bool trailing_uses_tensor_cores(int64_t n, int block) {
   return (n % 4 == 0) && (block % QK == 0) && n <= (1 << 30);
@@ -277,13 +164,8 @@ gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, int64_t
   if (c0 >= c1 || kw <= 0 || m <= 0) return GPTQ_OK;
   if (Uhi != nullptr && trailing_uses_tensor_cores(n, kw)) {
     TrailMaps maps;
-    const int64_t mr = error_rows(m);
-    bool ok = encode_f32(&maps.ahi, Ehi, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
-              encode_f32(&maps.alo, Elo, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
-              encode_f32(&maps.bhi, Uhi, n, n, n * 4, QK, QN) &&
-              encode_f32(&maps.blo, Ulo, n, n, n * 4, QK, QN) &&
-              encode_f32(&maps.c, Wp, n, mr, n * 4, 32, QM);
-    if (!ok) return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the trailing update");
+    if (!make_trail_maps(&maps, Wp, m, n, Ehi, Elo, Uhi, Ulo))
+      return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the trailing update");
     if (!g_attr) {
       GPTQ_CUDA(cudaFuncSetAttribute(trailing_tc_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QSMEM));
