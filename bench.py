@@ -159,9 +159,13 @@ def kernel_work(probs, block: int):
     cholesky  flops of the executed float64 tile products (Σ_k tiles·2·64³)
               plus the diagonal tiles' Cholesky and inverse (2·64³/3 each)
     sweep     bytes: strip read + Err write (4+4 B) + codes (1 B) per element,
-              U panel 4·bw², scale+zero 5 B per (row, group)
-    trailing  bytes: W read+write 8 B per trailing element, Err 4·m·bw,
-              U panel 4·bw·N2
+              U panel 4·bw², scale+zero 5 B per (row, group); on the
+              tensor-core path (n % 4 == 0) also the trailing update's bytes
+              (W read+write 8 B per trailing element, Err 4·m·bw, U panel
+              4·bw·N2): its near columns run in the sweep's prologue and its
+              far columns in CTAs of the sweep's own launch
+    trailing  bytes: the transposed TF32 split of U (12 B per element) on
+              the tensor-core path, else the SIMT trailing update's bytes
     pack      bytes: codes 1 B + packed bits/8 B per element, scale/zero
     ingest    bytes: W in (2 or 4 B) + float32 out per element
     """
@@ -175,12 +179,15 @@ def kernel_work(probs, block: int):
             w["cholesky"] += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
             w["cholesky"] += 2 * 64 ** 3 / 3         # Cholesky + inverse of a tile
         ng = -(-n // p.group)
+        fused = n % 4 == 0 and n > block
+        if fused:
+            w["trailing"] += 12 * n * n
         for j0 in range(0, n, block):
             bw = min(block, n - j0)
             n2 = n - j0 - bw
             w["sweep"] += 9 * m * bw + 4 * bw * bw + 5 * m * (-(-bw // p.group))
             if n2 > 0:
-                w["trailing"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
+                w["sweep" if fused else "trailing"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
         w["pack"] += m * n + m * n * p.bits / 8 + 5 * m * ng
         w["ingest"] += m * n * (p.W.element_size() + 4)
     units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s",

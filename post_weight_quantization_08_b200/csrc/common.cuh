@@ -19,8 +19,8 @@ enum KernelKind : int {
   KK_CHOL,            // blocked Cholesky + triangular inverse (one dataflow launch)
   KK_PREP_OUT,        // U = reversed L⁻¹, rounded to float32
   KK_INGEST,          // W → float32 working copy in processing order
-  KK_SWEEP,           // one block of the column sweep
-  KK_TRAIL,           // lazy-batch trailing update W −= Err·U
+  KK_SWEEP,           // one block of the column sweep (+ the far update of the block before)
+  KK_TRAIL,           // TF32 split of U, or the SIMT lazy-batch trailing update
   KK_PACK,            // codes → packed words, g_idx, dequantized copy
   KK_COUNT
 };

@@ -70,11 +70,11 @@ gptq_status launch_split_tf32_t(const float* x, int64_t n, float* hiT, float* lo
                                 cudaStream_t s);
 
 // Wp[:, c0:c1] −= (Ehi+Elo)[:, 0:kw]·U[k0:k0+kw, c0:c1]   (lazy-batch update;
-// c1 is clipped to n).  With UhiT/UloT (the transposed TF32 split of U) the
-// product runs on the tensor cores.
+// c1 is clipped to n) in float32 SIMT tiles: the path for n % 4 ≠ 0, where
+// the tensor-core update (which rides in the sweep launches, SweepFar) cannot
+// take its operands by tensor map.
 gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, int64_t c1,
                             const float* Ehi, const float* Elo, int64_t k0, int kw,
-                            const float* U, const float* Uhi, const float* Ulo, int32_t* info,
-                            cudaStream_t s);
+                            const float* U, cudaStream_t s);
 
 }  // namespace gptq

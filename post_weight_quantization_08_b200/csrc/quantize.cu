@@ -282,13 +282,12 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
       GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[(b - 1) & 1], 0));
       pending[(b - 1) & 1] = false;
     }
-    st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info, s);
+    st = launch_trailing(w.Wp, m, n, c0, c1, ehi, elo, j0, bw, U, s);
     if (st != GPTQ_OK) return st;
     if (c1 < n) {
       GPTQ_CUDA(cudaEventRecord(side->swept, s));
       GPTQ_CUDA(cudaStreamWaitEvent(side->s2, side->swept, 0));
-      st = launch_trailing(w.Wp, m, n, c1, n, ehi, elo, j0, bw, U, w.Uhi, w.Ulo, info,
-                           side->s2);
+      st = launch_trailing(w.Wp, m, n, c1, n, ehi, elo, j0, bw, U, side->s2);
       if (st != GPTQ_OK) return st;
       GPTQ_CUDA(cudaEventRecord(side->far[b & 1], side->s2));
       pending[b & 1] = true;

@@ -5,27 +5,10 @@
 // Applied once per block instead of once per column this is one product with
 // K = block width; the result is the same up to float32 rounding order.
 //
-// Tensor-core path (n a multiple of 4): tcgen05.mma kind::tf32 with a
-// three-term split.  Every float32 operand is written as hi + lo with
-// hi = TF32(x) (round to nearest) and lo = x − hi (exact), and
-//   Err·U ≈ Err_hi·U_hi + Err_hi·U_lo + Err_lo·U_hi
-// (the dropped lo·lo term and the TF32 truncation of lo are ≈ 2⁻²¹ relative,
-// float32-grade; a single TF32 product would be 2⁻¹¹ and move pre-rounding
-// values by far more than the 1e-4 code units the parity criterion allows).
-// The sweep writes Err_hi/Err_lo; the split of U is written once per call,
-// transposed (UT[c][k] = U[k][c]), so that both tf32 operands are K-major:
-// MN-major tf32 operands would need the 32-byte-atom variant of the 128-byte
-// swizzle, K-major ones take the plain 128-byte swizzle.
-//
-// One CTA per 128-row × 256-column tile of W:
-//   warp 0 lane 0  TMA: Err_hi/lo boxes 128 rows × 32 K and Uᵀ_hi/lo boxes
-//                  256 columns × 32 K (both K-major), 128-byte swizzle,
-//                  2-stage ring over K in chunks of 32;
-//   warp 1 lane 0  3 × tcgen05.mma (M=128, N=256, K=8) per 8 K, A negated so
-//                  the 256 TMEM columns hold −Err·U;
-//   4 warps        drain TMEM into swizzled shared boxes, then one TMA
-//                  reduce-add per 32-column box adds them into W.
-// Fallback: float32 SIMT tiles.
+// The tensor-core update (n a multiple of 4) is trailing_tc.cuh's CTA body,
+// run by the CTAs that ride in each sweep's launch; this file holds the
+// transposed TF32 split of U it reads, its tensor maps, and the float32 SIMT
+// tiles that take over when n % 4 ≠ 0.
 
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -118,20 +101,11 @@ split_tf32_t_kernel(const float* __restrict__ x, int64_t n, float* __restrict__ 
 
 // ---------------------------------------------------------------- tcgen05 path
 
-__global__ void __launch_bounds__(128, 1)
-trailing_tc_kernel(const __grid_constant__ TrailMaps maps, int64_t m, int64_t n, int64_t c0,
-                   int64_t c1, int64_t k0, int kw, int32_t* info) {
-  extern __shared__ unsigned char smraw[];
-  trailing_tc_body(maps, m, n, c0, c1, k0, kw, info, (int)blockIdx.x, (int)blockIdx.y, smraw);
-}
-
 bool encode_f32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   return encode_tiled_2d(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, inner, outer, row_bytes,
                          box_inner, box_outer);
 }
-
-bool g_attr = false;
 
 }  // namespace
 
@@ -158,24 +132,9 @@ gptq_status launch_split_tf32_t(const float* x, int64_t n, float* hiT, float* lo
 
 gptq_status launch_trailing(float* Wp, int64_t m, int64_t n, int64_t c0, int64_t c1,
                             const float* Ehi, const float* Elo, int64_t k0, int kw,
-                            const float* U, const float* Uhi, const float* Ulo, int32_t* info,
-                            cudaStream_t s) {
+                            const float* U, cudaStream_t s) {
   if (c1 > n) c1 = n;
   if (c0 >= c1 || kw <= 0 || m <= 0) return GPTQ_OK;
-  if (Uhi != nullptr && trailing_uses_tensor_cores(n, kw)) {
-    TrailMaps maps;
-    if (!make_trail_maps(&maps, Wp, m, n, Ehi, Elo, Uhi, Ulo))
-      return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the trailing update");
-    if (!g_attr) {
-      GPTQ_CUDA(cudaFuncSetAttribute(trailing_tc_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QSMEM));
-      g_attr = true;
-    }
-    const dim3 grid((unsigned)ceil_div(c1 - c0, QN), (unsigned)ceil_div(m, QM));
-    GPTQ_LAUNCH_PDL(KK_TRAIL, s, trailing_tc_kernel, grid, 128, QSMEM, maps, m, n, c0, c1, k0,
-                    kw, info);
-    return GPTQ_OK;
-  }
   const dim3 grid((unsigned)ceil_div(c1 - c0, TN), (unsigned)ceil_div(m, TM));
   GPTQ_LAUNCH(KK_TRAIL, s, trailing_simt_kernel, grid, 256, 0, Wp, m, n, c0, c1, Ehi, Elo, k0,
               kw, U);

@@ -1,6 +1,28 @@
-// The tensor-core trailing update's CTA body, shared by its own launch and by
-// the sweep launch that carries the far-column update of the block before
-// (see trailing.cu for the method).
+// K4 on the tensor cores: the lazy-batch trailing update
+// W[:, c0:c1] −= Err·U[k0:k0+kw, c0:c1] as a CTA body, run by the CTAs that
+// ride in each sweep's launch (the far columns of the block before).
+//
+// Tensor-core path (n a multiple of 4): tcgen05.mma kind::tf32 with a
+// three-term split.  Every float32 operand is written as hi + lo with
+// hi = TF32(x) (round to nearest) and lo = x − hi (exact), and
+//   Err·U ≈ Err_hi·U_hi + Err_hi·U_lo + Err_lo·U_hi
+// (the dropped lo·lo term and the TF32 truncation of lo are ≈ 2⁻²¹ relative,
+// float32-grade; a single TF32 product would be 2⁻¹¹ and move pre-rounding
+// values by far more than the 1e-4 code units the parity criterion allows).
+// The sweep writes Err_hi/Err_lo; the split of U is written once per call,
+// transposed (UT[c][k] = U[k][c]), so that both tf32 operands are K-major:
+// MN-major tf32 operands would need the 32-byte-atom variant of the 128-byte
+// swizzle, K-major ones take the plain 128-byte swizzle.
+//
+// One CTA per 128-row × 256-column tile of W:
+//   warp 0 lane 0  TMA: Err_hi/lo boxes 128 rows × 32 K and Uᵀ_hi/lo boxes
+//                  256 columns × 32 K (both K-major), 128-byte swizzle,
+//                  2-stage ring over K in chunks of 32;
+//   warp 1 lane 0  3 × tcgen05.mma (M=128, N=256, K=8) per 8 K, A negated so
+//                  the 256 TMEM columns hold −Err·U;
+//   4 warps        drain TMEM into swizzled shared boxes, then one TMA
+//                  reduce-add per 32-column box adds them into W.
+// Fallback (n % 4 ≠ 0): float32 SIMT tiles, trailing.cu.
 #pragma once
 
 #include "kernels.cuh"
