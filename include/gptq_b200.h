@@ -198,6 +198,81 @@ gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
                           int32_t* info, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* ---- CHMC frontend (next to the hot path) -------------------------------
+ * "Warum Geometrie Gewichte nicht komprimiert", section "Methodik. Was ist
+ * CHMC": every weight matrix W (o × i) is split into a low-rank part W_lr
+ * along the activation cone (Schritt 1) and a residual R = W − W_lr quantized
+ * by GPTQ with scales along the output channels (Schritt 2); the rank comes
+ * from the bit budget (Schritt 3).
+ */
+
+/* Output-channel group size of gptq_quantize_rowgroups (the page's gs). */
+#define GPTQ_ROWGROUP_SIZE 128
+/* Largest rank gptq_chmc_lowrank accepts. */
+#define GPTQ_CHMC_MAX_RANK 32
+
+/*
+ * Schritt 3, the rank rule (host arithmetic, no device work):
+ *   r = floor((bpw_target·o·i − bits·o·i − 16·ceil(o/gs)·i) / (16·(o + i))),
+ * clamped to [0, min(o, i)].  Returns 0 for invalid arguments.
+ */
+int gptq_chmc_rank(int64_t o, int64_t i, int bits, int gs, double bpw_target);
+
+/* Bytes of device workspace gptq_chmc_lowrank needs (256-byte aligned);
+ * 0 if r is outside [0, GPTQ_CHMC_MAX_RANK]. */
+size_t gptq_chmc_workspace_bytes(int64_t o, int64_t i, int r);
+
+/*
+ * Schritt 1: the low-rank part and the residual.
+ *   W        o × i, device, float32 or bfloat16 (w_dtype), row-major (rows are
+ *            output channels).  Not modified.
+ *   H        i × i float32, device: 2·XᵀX over `tokens` calibration rows (the
+ *            Hessian of gptq_hessian_accumulate).  Only its diagonal is read:
+ *            c_j = H_jj/(2·tokens) + lam·mean_j(H_jj/(2·tokens)), the page's
+ *            damped activation energies (lam = 0.05 on the page).
+ *   Omega    i × r float32, device, row-major: the randomized SVD's test
+ *            matrix (standard normal entries, drawn by the caller).
+ *   r        rank, 0..GPTQ_CHMC_MAX_RANK and at most min(o, i); r = 0 copies W
+ *            to R (H and Omega may then be NULL).
+ *   niter    power iterations (the page uses 5), 0..64.
+ *   Q        o × r float32 or NULL, output: an orthonormal basis of the range
+ *            found by the randomized subspace iteration on W·diag(√c).
+ *   P        r × i float32 or NULL, output: Qᵀ·W, so that W_lr = Q·P
+ *            (= (U·S)·Vᵀ·diag(1/√c) of the page: B = Qᵀ·W̃ has exactly r rows,
+ *            so its SVD only rotates the factors).
+ *   R        o × i float32, output: W − Q·P, computed in float64.
+ *   info     int32[2], device, output (INVALID_ARG with the column index if an
+ *            activation energy is not positive).
+ * Computes in float64 throughout; deterministic.  Errors: INVALID_ARG,
+ * UNSUPPORTED (rank, niter), CUDA.
+ */
+gptq_status gptq_chmc_lowrank(const void* W, int w_dtype, int64_t o, int64_t i,
+                              const float* H, int64_t tokens, double lam,
+                              const float* Omega, int r, int niter, float* Q, float* P,
+                              float* R, int32_t* info, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/*
+ * Schritt 2: GPTQ with scales along the output channels ("eine gemeinsame
+ * Skala pro Gruppe von Ausgabekanälen", ceil(o/gs)·i scales).  As
+ * gptq_quantize, except:
+ *   gs       rows per scale group; must be GPTQ_ROWGROUP_SIZE.
+ *   scale    ceil(m/gs) × n float32, output: scale[g][c] for rows
+ *            [g·gs, (g+1)·gs) and ORIGINAL column c; zero: same shape, uint8.
+ *            Each column's parameters come from the column's current
+ *            (error-updated) values over the group's rows, when the column is
+ *            processed (min-max, 0 inside the range, all-zero → [−1, 1]).
+ *   block    lazy-batch width: a multiple of 32, at most 128.
+ *   (no g_idx: every column has its own scale per row group.)
+ * Workspace: gptq_quantize_workspace_bytes(m, n, block).
+ */
+gptq_status gptq_quantize_rowgroups(const void* W, int w_dtype, int64_t m, int64_t n,
+                                    const float* U, const int32_t* perm,
+                                    const uint8_t* dead, int bits, int gs, int block,
+                                    uint32_t* qweight, float* scale, uint8_t* zero,
+                                    float* loss_row, float* Qdq, int32_t* info, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /*
  * Synchronize `stream`, read info[0..1] and return info[0] (a gptq_status).
  * If `index` is not NULL it receives info[1].  `info` is a device pointer.

@@ -10,17 +10,22 @@ from __future__ import annotations
 import torch
 
 from ._binding import (DTYPES, ORDERS, GptqError, exported_symbols,
-                       gptq_check, gptq_hessian_accumulate, gptq_launch_count,
-                       gptq_prepare, gptq_prepare_workspace_bytes,
+                       gptq_check, gptq_chmc_lowrank, gptq_chmc_rank,
+                       gptq_chmc_workspace_bytes, gptq_hessian_accumulate,
+                       gptq_launch_count, gptq_prepare, gptq_prepare_workspace_bytes,
                        gptq_profile_start, gptq_profile_stop, gptq_quantize,
-                       gptq_quantize_workspace_bytes, kernel_names, lib)
+                       gptq_quantize_rowgroups, gptq_quantize_workspace_bytes,
+                       kernel_names, lib)
 
 __all__ = [
     "GptqError", "ORDERS", "DTYPES", "lib", "exported_symbols", "kernel_names",
     "gptq_hessian_accumulate", "gptq_prepare", "gptq_quantize", "gptq_check",
     "gptq_prepare_workspace_bytes", "gptq_quantize_workspace_bytes",
     "gptq_launch_count", "gptq_profile_start", "gptq_profile_stop",
+    "gptq_quantize_rowgroups", "gptq_chmc_rank", "gptq_chmc_workspace_bytes",
+    "gptq_chmc_lowrank",
     "hessian", "prepare", "quantize", "workspace",
+    "chmc_lowrank", "quantize_rowgroups", "chmc_layer",
 ]
 
 
@@ -93,3 +98,68 @@ def quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
     if check:
         _raise_info(out["info"], stream, "gptq_quantize")
     return out
+
+
+# ---- CHMC frontend ("Warum Geometrie Gewichte nicht komprimiert", Methodik)
+
+def chmc_lowrank(W: torch.Tensor, H: torch.Tensor, tokens: int, Omega: torch.Tensor | None,
+                 r: int, lam: float = 0.05, niter: int = 5, ws: torch.Tensor | None = None,
+                 stream=None, check: bool = True) -> dict:
+    """Schritt 1: returns {"Q", "P", "R"} with W_lr = Q·P and R = W − W_lr."""
+    o, i = W.shape
+    dev = W.device
+    out = {
+        "Q": torch.empty(o, r, dtype=torch.float32, device=dev) if r > 0 else None,
+        "P": torch.empty(r, i, dtype=torch.float32, device=dev) if r > 0 else None,
+        "R": torch.empty(o, i, dtype=torch.float32, device=dev),
+        "info": torch.zeros(2, dtype=torch.int32, device=dev),
+    }
+    if ws is None:
+        ws = workspace(gptq_chmc_workspace_bytes(o, i, r), dev)
+    gptq_chmc_lowrank(W, H, tokens, lam, Omega, r, niter, out["Q"], out["P"], out["R"],
+                      out["info"], ws, stream)
+    if check:
+        _raise_info(out["info"], stream, "gptq_chmc_lowrank")
+    return out
+
+
+def quantize_rowgroups(W: torch.Tensor, prep: dict, bits: int = 4, gs: int = 128,
+                       block: int = 128, want_loss: bool = True, want_qdq: bool = False,
+                       ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+    """Schritt 2: GPTQ with scales along the output channels; scale and zero
+    are ⌈m/gs⌉ × n in the original column order."""
+    m, n = W.shape
+    dev = W.device
+    ngr = -(-m // gs)
+    nwords = -(-n * bits // 32)
+    out = {
+        "qweight": torch.empty(m, nwords, dtype=torch.int32, device=dev),
+        "scale": torch.empty(ngr, n, dtype=torch.float32, device=dev),
+        "zero": torch.empty(ngr, n, dtype=torch.uint8, device=dev),
+        "loss_row": torch.empty(m, dtype=torch.float32, device=dev) if want_loss else None,
+        "Qdq": torch.empty(m, n, dtype=torch.float32, device=dev) if want_qdq else None,
+        "info": torch.zeros(2, dtype=torch.int32, device=dev),
+    }
+    if ws is None:
+        ws = workspace(gptq_quantize_workspace_bytes(m, n, block), dev)
+    gptq_quantize_rowgroups(W, prep["U"], prep["perm"], prep["dead"], bits, gs, block,
+                            out["qweight"], out["scale"], out["zero"], out["loss_row"],
+                            out["Qdq"], out["info"], ws, stream)
+    if check:
+        _raise_info(out["info"], stream, "gptq_quantize_rowgroups")
+    return out
+
+
+def chmc_layer(W: torch.Tensor, H: torch.Tensor, tokens: int, Omega: torch.Tensor | None,
+               r: int | None = None, bits: int = 4, gs: int = 128, bpw_target: float = 4.2875,
+               lam: float = 0.05, damp: float = 0.05, order: str = "act", niter: int = 5,
+               block: int = 128, stream=None) -> dict:
+    """Schritte 1–3 on one layer: the low-rank part, then GPTQ of the residual
+    with output-channel scales.  ``r`` defaults to the rank rule."""
+    o, i = W.shape
+    if r is None:
+        r = gptq_chmc_rank(o, i, bits, gs, bpw_target)
+    lr = chmc_lowrank(W, H, tokens, Omega, r, lam, niter, stream=stream)
+    prep = prepare(H, damp, order, stream=stream)
+    q = quantize_rowgroups(lr["R"], prep, bits, gs, block, want_qdq=True, stream=stream)
+    return {"rank": r, **lr, **{"prep_" + k: v for k, v in prep.items()}, **q}

@@ -39,6 +39,17 @@ _SIGS = {
                                 C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                 C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                 C.c_size_t, C.c_void_p]),
+    "gptq_quantize_rowgroups": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64,
+                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
+                                          C.c_int, C.c_int, C.c_void_p, C.c_void_p,
+                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                          C.c_void_p, C.c_size_t, C.c_void_p]),
+    "gptq_chmc_rank": (C.c_int, [C.c_int64, C.c_int64, C.c_int, C.c_int, C.c_double]),
+    "gptq_chmc_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int]),
+    "gptq_chmc_lowrank": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
+                                    C.c_int64, C.c_double, C.c_void_p, C.c_int, C.c_int,
+                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                    C.c_void_p, C.c_size_t, C.c_void_p]),
     "gptq_check": (C.c_int, [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]),
     "gptq_last_error": (C.c_char_p, []),
     "gptq_status_string": (C.c_char_p, [C.c_int]),
@@ -177,6 +188,68 @@ def gptq_quantize(W, U, perm, dead, bits, group, block, qweight, scale, zero,
                                _ptr(qweight), _ptr(scale), _ptr(zero), _ptr(g_idx),
                                _ptr(loss_row), _ptr(Qdq), _ptr(info), _ptr(ws),
                                ws.numel(), _stream(stream, dev)))
+
+
+def gptq_quantize_rowgroups(W, U, perm, dead, bits, gs, block, qweight, scale, zero,
+                            loss_row, Qdq, info, ws, stream=None):
+    """Quantize W with scales along the output channels (see include/gptq_b200.h)."""
+    if W.dtype not in DTYPES:
+        raise TypeError("W must be float32 or bfloat16")
+    _need(W, "W", W.dtype)
+    m, n = W.shape
+    dev = W.device
+    ngr = -(-m // gs)
+    nwords = -(-n * bits // 32)
+    _need(U, "U", torch.float32, (n, n), dev)
+    _need(perm, "perm", torch.int32, (n,), dev)
+    _need(dead, "dead", torch.uint8, (n,), dev)
+    _need(qweight, "qweight", torch.int32, (m, nwords), dev)
+    _need(scale, "scale", torch.float32, (ngr, n), dev)
+    _need(zero, "zero", torch.uint8, (ngr, n), dev)
+    if loss_row is not None:
+        _need(loss_row, "loss_row", torch.float32, (m,), dev)
+    if Qdq is not None:
+        _need(Qdq, "Qdq", torch.float32, (m, n), dev)
+    _need(info, "info", torch.int32, (2,), dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _raise(lib().gptq_quantize_rowgroups(_ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm),
+                                         _ptr(dead), int(bits), int(gs), int(block),
+                                         _ptr(qweight), _ptr(scale), _ptr(zero),
+                                         _ptr(loss_row), _ptr(Qdq), _ptr(info), _ptr(ws),
+                                         ws.numel(), _stream(stream, dev)))
+
+
+def gptq_chmc_rank(o: int, i: int, bits: int = 4, gs: int = 128,
+                   bpw_target: float = 4.2875) -> int:
+    """The rank rule of the bit budget (see include/gptq_b200.h)."""
+    return int(lib().gptq_chmc_rank(int(o), int(i), int(bits), int(gs), float(bpw_target)))
+
+
+def gptq_chmc_workspace_bytes(o: int, i: int, r: int) -> int:
+    return int(lib().gptq_chmc_workspace_bytes(int(o), int(i), int(r)))
+
+
+def gptq_chmc_lowrank(W, H, tokens, lam, Omega, r, niter, Q, P, R, info, ws, stream=None):
+    """Low-rank part and residual of W (see include/gptq_b200.h)."""
+    if W.dtype not in DTYPES:
+        raise TypeError("W must be float32 or bfloat16")
+    _need(W, "W", W.dtype)
+    o, i = W.shape
+    dev = W.device
+    if r > 0:
+        _need(H, "H", torch.float32, (i, i), dev)
+        _need(Omega, "Omega", torch.float32, (i, r), dev)
+    if Q is not None:
+        _need(Q, "Q", torch.float32, (o, r), dev)
+    if P is not None:
+        _need(P, "P", torch.float32, (r, i), dev)
+    _need(R, "R", torch.float32, (o, i), dev)
+    _need(info, "info", torch.int32, (2,), dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _raise(lib().gptq_chmc_lowrank(_ptr(W), DTYPES[W.dtype], o, i, _ptr(H), int(tokens),
+                                   float(lam), _ptr(Omega), int(r), int(niter), _ptr(Q),
+                                   _ptr(P), _ptr(R), _ptr(info), _ptr(ws), ws.numel(),
+                                   _stream(stream, dev)))
 
 
 def gptq_check(info, stream=None) -> tuple[int, int]:

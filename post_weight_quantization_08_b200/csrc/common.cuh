@@ -22,6 +22,7 @@ enum KernelKind : int {
   KK_SWEEP,           // one block of the column sweep (+ the far update of the block before)
   KK_TRAIL,           // TF32 split of U, or the SIMT lazy-batch trailing update
   KK_PACK,            // codes → packed words, g_idx, dequantized copy
+  KK_CHMC,            // CHMC frontend: activation energies, randomized subspace iteration, residual
   KK_COUNT
 };
 

@@ -42,6 +42,11 @@ struct SweepPrologue {
   int64_t k0 = 0;               // first column of the previous block
   int kw = 0;                   // its width (a multiple of 32), 0 for none
 };
+// rowgroup_perm != NULL: scales along the output channels instead (groups of
+// the CTA's 128 rows, one scale and zero per row group and column, from the
+// column's current values), stored as scale[g·n + rowgroup_perm[j]] for
+// processing position j; `group` and `ngroups` are then unused.
+//
 // With far.kw > 0 and far.c0 < far.c1 the same launch also applies the
 // block before's far-column update, Wp[:, c0:c1] −= (far.Ehi + far.Elo)[:, 0:kw]·
 // U[far.k0 : far.k0+kw, c0:c1] (tensor cores, far.Uhi/Ulo as above): columns
@@ -59,7 +64,8 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
                          float* Elo, const SweepPrologue& pre, const SweepFar& far,
-                         float* loss_row, int32_t* info, cudaStream_t s);
+                         float* loss_row, int32_t* info, const int32_t* rowgroup_perm,
+                         cudaStream_t s);
 
 // Whether the trailing update runs on the tensor cores for this shape.
 bool trailing_uses_tensor_cores(int64_t n, int block);

@@ -101,7 +101,7 @@ pinv_kernel(const int32_t* __restrict__ perm, int64_t n, int group,
   const int32_t c = perm[p];
   if (c < 0 || c >= n) { report(info, GPTQ_ERR_INVALID_ARG, p); return; }
   pinv[c] = (int32_t)p;
-  g_idx[c] = (int32_t)(p / group);
+  if (g_idx) g_idx[c] = (int32_t)(p / group);
 }
 
 // Wp[r][p] = W[r][perm[p]] as float32; dead columns read as 0.
@@ -127,7 +127,7 @@ ingest_kernel(const T* __restrict__ W, int64_t m, int64_t n,
 template <int BITS>
 __global__ void __launch_bounds__(256)
 pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
-            const int32_t* __restrict__ pinv, int group, int64_t ngroups,
+            const int32_t* __restrict__ pinv, int group, int64_t ngroups, int rowgs,
             const float* __restrict__ scale, const uint8_t* __restrict__ zero,
             uint32_t* __restrict__ qweight, int64_t nwords,
             float* __restrict__ Qdq, int32_t* info) {
@@ -149,8 +149,10 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
       } else {
         q = codes[r * n + p];
         if (Qdq != nullptr) {
-          const int64_t g = p / group;
-          Qdq[r * n + c] = scale[r * ngroups + g] * ((float)q - (float)zero[r * ngroups + g]);
+          // input-channel groups: [row][group of processing position p];
+          // output-channel groups (rowgs rows): [row group][original column c]
+          const int64_t sx = rowgs > 0 ? (r / rowgs) * n + c : r * ngroups + p / group;
+          Qdq[r * n + c] = scale[sx] * ((float)q - (float)zero[sx]);
         }
       }
       const int off = k * BITS, wi = off >> 5, sh = off & 31;
@@ -175,15 +177,19 @@ extern "C" size_t gptq_quantize_workspace_bytes(int64_t m, int64_t n, int block)
   return quant_ws_layout(m, n, block, nullptr, nullptr);
 }
 
-extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
-                                     int64_t n, const float* U,
-                                     const int32_t* perm, const uint8_t* dead,
-                                     int bits, int group, int block,
-                                     uint32_t* qweight, float* scale,
-                                     uint8_t* zero, int32_t* g_idx,
-                                     float* loss_row, float* Qdq, int32_t* info,
-                                     void* ws, size_t ws_bytes, void* stream) {
-  if (!W || !U || !perm || !dead || !qweight || !scale || !zero || !g_idx || !info || !ws)
+namespace gptq {
+namespace {
+
+// The quantize path of gptq_quantize (rowgs = 0: scale groups of `group`
+// columns) and gptq_quantize_rowgroups (rowgs = 128: scale groups of the
+// rows, per column).
+gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, const float* U,
+                          const int32_t* perm, const uint8_t* dead, int bits, int group,
+                          int block, int rowgs, uint32_t* qweight, float* scale, uint8_t* zero,
+                          int32_t* g_idx, float* loss_row, float* Qdq, int32_t* info, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (!W || !U || !perm || !dead || !qweight || !scale || !zero || (!g_idx && rowgs == 0) ||
+      !info || !ws)
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: null pointer");
   if (m < 1 || n < 1 || m > ((int64_t)1 << 31) || n > ((int64_t)1 << 20))
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: m=%lld n=%lld", (long long)m,
@@ -206,7 +212,7 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   QuantWs w;
   quant_ws_layout(m, n, block, &w, static_cast<char*>(ws));
-  const int64_t ngroups = ceil_div(n, group);
+  const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
   const int64_t nwords = ceil_div(n * bits, 32);
 
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
@@ -274,7 +280,7 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
     }
     const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
     st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes, scale,
-                      zero, ehi, elo, pre, far, loss_row, info, s);
+                      zero, ehi, elo, pre, far, loss_row, info, rowgs > 0 ? perm : nullptr, s);
     if (st != GPTQ_OK) return st;
     const int64_t c0 = j0 + bw, c1 = c0 + block;
     if (c0 >= n || fused) continue;
@@ -300,20 +306,50 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
   switch (bits) {
     case 2:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
       break;
     case 3:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
       break;
     case 4:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
       break;
     default:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
       break;
   }
   return GPTQ_OK;
+}
+
+}  // namespace
+}  // namespace gptq
+
+extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
+                                     int64_t n, const float* U,
+                                     const int32_t* perm, const uint8_t* dead,
+                                     int bits, int group, int block,
+                                     uint32_t* qweight, float* scale,
+                                     uint8_t* zero, int32_t* g_idx,
+                                     float* loss_row, float* Qdq, int32_t* info,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  return quantize_impl(W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, qweight, scale,
+                       zero, g_idx, loss_row, Qdq, info, ws, ws_bytes, stream);
+}
+
+extern "C" gptq_status gptq_quantize_rowgroups(const void* W, int w_dtype, int64_t m,
+                                               int64_t n, const float* U,
+                                               const int32_t* perm, const uint8_t* dead,
+                                               int bits, int gs, int block,
+                                               uint32_t* qweight, float* scale,
+                                               uint8_t* zero, float* loss_row, float* Qdq,
+                                               int32_t* info, void* ws, size_t ws_bytes,
+                                               void* stream) {
+  if (gs != GPTQ_ROWGROUP_SIZE)
+    return fail(GPTQ_ERR_UNSUPPORTED, "gptq_quantize_rowgroups: gs=%d (only %d)", gs,
+                GPTQ_ROWGROUP_SIZE);
+  return quantize_impl(W, w_dtype, m, n, U, perm, dead, bits, block, block, gs, qweight, scale,
+                       zero, nullptr, loss_row, Qdq, info, ws, ws_bytes, stream);
 }

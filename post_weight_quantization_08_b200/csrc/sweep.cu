@@ -68,7 +68,9 @@ constexpr uint32_t SM_CODES = SM_VALS + 4 * VBOX;
 constexpr uint32_t SM_BPHI = (SM_CODES + RT * LDB + 1023) / 1024 * 1024;
 constexpr uint32_t SM_BPLO = SM_CODES;
 constexpr uint32_t SM_BARS = SM_BPHI + 32 * RT * 4;
-constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 128;
+constexpr uint32_t SM_RGRED = SM_BARS + 128;        // 2 × 8 floats: row-group min/max
+static_assert(GPTQ_ROWGROUP_SIZE == RT, "an output-channel group is one CTA's rows");
+constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 192;
 static_assert(SM_AHI >= PK_BYTES && SM_AHI % 1024 == 0, "A operand placement");
 static_assert(SM_VALS % 1024 == 0, "the strip's boxes use the 128-byte swizzle");
 static_assert(SM_CODES % 1024 == 0 && RT * LDB >= 32 * RT * 4, "U chunk lo part placement");
@@ -154,15 +156,19 @@ __device__ __forceinline__ float div_fma(float x, float s, float rs) {
 }
 
 // One CTA (bx: the 128-row tile) of the sweep; smraw: SMEM_BYTES of dynamic
-// shared memory.
+// shared memory.  ROWG: scales along the output channels (CHMC page, Schritt
+// 2 and 3: ⌈o/gs⌉·i scales, gs = 128 rows, the CTA's own rows): each column's
+// scale and zero come from the column's current values over the CTA's rows,
+// and are stored at [bx][perm[j0 + c]] (row group × original column).
+template <bool ROWG>
 __device__ __forceinline__ void sweep_body(
     const CUtensorMap& tmEhi, const CUtensorMap& tmElo, const CUtensorMap& tmW, int strip_tma,
     const CUtensorMap& tmPhi, const CUtensorMap& tmPlo, const CUtensorMap& tmUhi,
     const CUtensorMap& tmUlo, int64_t k0p, int kwp, const float* __restrict__ Wp, int64_t m,
     int64_t n, int64_t j0, int bw, const unsigned char* __restrict__ pkg, int bits, int group,
     int64_t ngroups, uint8_t* __restrict__ codes, float* __restrict__ scale,
-    uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info, int bx,
-    unsigned char* smraw) {
+    uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info,
+    const int32_t* __restrict__ perm, int bx, unsigned char* smraw) {
   const uint32_t raw = smem_addr(smraw);
   unsigned char* sm = smraw + ((1024 - (raw & 1023)) & 1023);
   const float* Ud = reinterpret_cast<const float*>(sm + SM_PKG + PK_UD);
@@ -380,7 +386,7 @@ __device__ __forceinline__ void sweep_body(
         v[4 * j + 3] = f.w - d[4 * j + 3];
       }
     }
-    if (c0 % group == 0) {
+    if (!ROWG && c0 % group == 0) {
       // the group's current values: this sub-block, then later ones in the group
       float xmin = 0.f, xmax = 0.f;
 #pragma unroll
@@ -433,6 +439,39 @@ __device__ __forceinline__ void sweep_body(
 #pragma unroll
     for (int i = 0; i < SS; ++i) {
       const int c = c0 + i;
+      if constexpr (ROWG) {
+        // the column's min and max over the CTA's rows (0 inside the range):
+        // warp shuffles, then the four warps through shared memory (two
+        // buffers by column parity, so one barrier per column suffices)
+        float mn = fminf(v[i], 0.f), mx = fmaxf(v[i], 0.f);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        }
+        float* red = reinterpret_cast<float*>(sm + SM_RGRED) + (i & 1) * 8;
+        if (lane == 0) {
+          red[warp] = mn;
+          red[4 + warp] = mx;
+        }
+        __syncthreads();
+        float xmin = fminf(fminf(red[0], red[1]), fminf(red[2], red[3]));
+        float xmax = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
+        if (xmin == 0.f && xmax == 0.f) {
+          xmin = -1.f;
+          xmax = 1.f;
+        }
+        s = __fdiv_rn(xmax - xmin, maxq);
+        rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
+        z = rintf(div_rn(-xmin, s));
+        klo = -z;
+        khi = maxq - z;
+        if (t == 0 && c < bw) {
+          const int64_t oc = perm[j0 + c];
+          scale[(int64_t)bx * n + oc] = s;
+          zero[(int64_t)bx * n + oc] = (uint8_t)z;
+        }
+      }
       // q − z = clamp(rint(v/s), −z, maxq − z) exactly (small integers), so
       // the clamp works on k = q − z and the error takes one FMA
       const float k = fminf(fmaxf(rintf(div_fma(v[i], s, rs)), klo), khi);
@@ -537,6 +576,7 @@ __device__ __forceinline__ void sweep_body(
 // 256 columns per 128-row tile): the two touch different columns, and both
 // take their inputs from earlier launches, so that consecutive sweeps follow
 // each other with nothing between them but the programmatic launch edge.
+template <bool ROWG>
 __global__ void __launch_bounds__(RT, 1)
 sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
              const __grid_constant__ CUtensorMap tmW, int strip_tma,
@@ -547,20 +587,22 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
              const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
              uint8_t* __restrict__ codes, float* __restrict__ scale,
              uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info,
-             int nsweep, const __grid_constant__ TrailMaps far, int64_t fc0, int64_t fc1,
-             int64_t fk0, int fkw, int fx) {
+             const int32_t* __restrict__ perm, int nsweep,
+             const __grid_constant__ TrailMaps far, int64_t fc0, int64_t fc1, int64_t fk0,
+             int fkw, int fx) {
   extern __shared__ unsigned char smraw[];
   const int b = (int)blockIdx.x;
   if (b < nsweep) {
-    sweep_body(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp, Wp, m, n, j0,
-               bw, pkg, bits, group, ngroups, codes, scale, zero, loss_row, info, b, smraw);
+    sweep_body<ROWG>(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp, Wp, m,
+                     n, j0, bw, pkg, bits, group, ngroups, codes, scale, zero, loss_row, info,
+                     perm, b, smraw);
   } else {
     const int f = b - nsweep;
     trailing_tc_body(far, m, n, fc0, fc1, fk0, fkw, info, f % fx, f / fx, smraw);
   }
 }
 
-bool g_attr_set = false;
+bool g_attr_set[2] = {false, false};
 
 }  // namespace
 
@@ -580,12 +622,18 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
                          float* Elo, const SweepPrologue& pre, const SweepFar& far,
-                         float* loss_row, int32_t* info, cudaStream_t s) {
+                         float* loss_row, int32_t* info, const int32_t* rowgroup_perm,
+                         cudaStream_t s) {
   constexpr size_t kSmem = SMEM_BYTES > QSMEM ? SMEM_BYTES : QSMEM;
-  if (!g_attr_set) {
-    GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kSmem));
-    g_attr_set = true;
+  const bool rowg = rowgroup_perm != nullptr;
+  if (!g_attr_set[rowg]) {
+    if (rowg)
+      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
+    else
+      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
+    g_attr_set[rowg] = true;
   }
   // the far-column update riding along: fx 256-column tiles per 128-row tile
   TrailMaps fm;
@@ -629,11 +677,18 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const int nsweep = (int)ceil_div(m, RT);
   const unsigned grid = (unsigned)(nsweep + nfar);
-  GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel, grid, RT, kSmem, th, tl, tw, strip_tma, tph, tpl,
-                  tuh, tul, (int64_t)pre.k0, kwp, (const float*)Wp, m, n, j0, bw,
-                  reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
-                  scale, zero, loss_row, info, nsweep, fm, far.c0, fc1, far.k0, far.kw,
-                  fx > 0 ? fx : 1);
+  if (rowg)
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel<true>, grid, RT, kSmem, th, tl, tw, strip_tma, tph,
+                    tpl, tuh, tul, (int64_t)pre.k0, kwp, (const float*)Wp, m, n, j0, bw,
+                    reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
+                    scale, zero, loss_row, info, rowgroup_perm, nsweep, fm, far.c0, fc1, far.k0,
+                    far.kw, fx > 0 ? fx : 1);
+  else
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel<false>, grid, RT, kSmem, th, tl, tw, strip_tma, tph,
+                    tpl, tuh, tul, (int64_t)pre.k0, kwp, (const float*)Wp, m, n, j0, bw,
+                    reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
+                    scale, zero, loss_row, info, (const int32_t*)nullptr, nsweep, fm, far.c0,
+                    fc1, far.k0, far.kw, fx > 0 ? fx : 1);
   return GPTQ_OK;
 }
 

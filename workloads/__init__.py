@@ -4,8 +4,9 @@ This package draws inputs only: it holds none of GPTQ's arithmetic, so both
 the CUDA path and the float64 oracle can be fed from it without sharing code.
 """
 from .configs import CONFIGS, Problem, problems_for
-from .synth import (cone_activations, gaussian_weights, student_t_activations,
-                    swiglu_input)
+from .synth import (cone_activations, gaussian_weights, normal_matrix, spectral_weights,
+                    student_t_activations, swiglu_input)
 
 __all__ = ["CONFIGS", "Problem", "problems_for", "cone_activations",
-           "gaussian_weights", "student_t_activations", "swiglu_input"]
+           "gaussian_weights", "normal_matrix", "spectral_weights",
+           "student_t_activations", "swiglu_input"]

@@ -81,3 +81,26 @@ def swiglu_input(X: torch.Tensor, W_gate: torch.Tensor,
     G = Xf @ W_gate.to(torch.bfloat16).to(torch.float32).T
     Up = Xf @ W_up.to(torch.bfloat16).to(torch.float32).T
     return (torch.nn.functional.silu(G) * Up).to(torch.bfloat16)
+
+
+def normal_matrix(rows: int, cols: int, seed: int) -> torch.Tensor:
+    """rows × cols float32 standard normal entries (e.g. a randomized SVD's
+    test matrix, drawn by the caller)."""
+    g = _gen(seed)
+    return torch.randn(rows, cols, generator=g, dtype=torch.float32)
+
+
+def spectral_weights(rows: int, cols: int, seed: int, decay: float = 0.8,
+                     std: float = 0.02) -> torch.Tensor:
+    """rows × cols float32 weights with singular values k^−decay (random
+    orthonormal bases), scaled to an entry std of about ``std``."""
+    g = _gen(seed)
+    k = min(rows, cols)
+    a = torch.randn(rows, k, generator=g, dtype=torch.float64)
+    b = torch.randn(cols, k, generator=g, dtype=torch.float64)
+    qa, _ = torch.linalg.qr(a)
+    qb, _ = torch.linalg.qr(b)
+    sig = torch.arange(1, k + 1, dtype=torch.float64).pow(-decay)
+    w = (qa * sig) @ qb.T
+    w = w * (std / w.std())
+    return w.to(torch.float32)
