@@ -30,7 +30,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from workloads import CONFIGS, problems_for  # noqa: E402
+from workloads import CONFIGS, normal_matrix, problems_for  # noqa: E402
 
 METRIC = "GPTQ weights quantized/sec (params/s incl. Hessian) & % of roofline, 1 B200"
 L2_BYTES = 126 * 1024 * 1024
@@ -474,6 +474,261 @@ def run_ours(args, rank, world, local):
     return out, probs, params
 
 
+# ---------------------------------------------------------------- the CHMC frontend
+
+CHMC_METRIC = ("CHMC weights compressed/sec (params/s incl. Hessian, low-rank part and "
+               "residual GPTQ) & % of roofline, 1 B200")
+CHMC_NITER, CHMC_LAM, CHMC_DAMP, CHMC_BPW, CHMC_GS = 5, 0.05, 0.05, 4.2875, 128
+
+
+class ChmcLayer:
+    """Device buffers of one layer under the CHMC frontend ("Warum Geometrie
+    Gewichte nicht komprimiert", Methodik): per weight matrix its rank from the
+    bit budget, its test matrix Ω, its factors and residual, and the residual's
+    codes with output-channel scales; per Hessian its inverse-Cholesky factor."""
+
+    def __init__(self, probs, device):
+        import post_weight_quantization_08_b200 as g
+        self.g = g
+        self.items = []
+        for pi, p in enumerate(probs):
+            n = p.n
+            it = {"p": p, "X": p.X.to(device).contiguous(),
+                  "H": torch.zeros(n, n, dtype=torch.float32, device=device),
+                  "perm": torch.empty(n, dtype=torch.int32, device=device),
+                  "U": torch.empty(n, n, dtype=torch.float32, device=device),
+                  "dead": torch.empty(n, dtype=torch.uint8, device=device),
+                  "info_h": torch.zeros(2, dtype=torch.int32, device=device),
+                  "info_p": torch.zeros(2, dtype=torch.int32, device=device),
+                  "ws_p": g.workspace(g.gptq_prepare_workspace_bytes(n), device),
+                  "stream": torch.cuda.Stream(device=device), "parts": []}
+            row0 = 0
+            for k, (name, rows) in enumerate(p.parts):
+                W = p.W[row0:row0 + rows].to(device).contiguous()
+                row0 += rows
+                r = g.gptq_chmc_rank(rows, n, p.bits, CHMC_GS, CHMC_BPW)
+                nw = -(-n * p.bits // 32)
+                it["parts"].append({
+                    "name": name, "W": W, "r": r,
+                    "Om": normal_matrix(n, max(r, 1), 9000 + 100 * pi + k)[:, :r].contiguous().to(device),
+                    "Q": torch.empty(rows, max(r, 1), dtype=torch.float32, device=device)[:, :r],
+                    "P": torch.empty(max(r, 1), n, dtype=torch.float32, device=device)[:r],
+                    "R": torch.empty(rows, n, dtype=torch.float32, device=device),
+                    "info_l": torch.zeros(2, dtype=torch.int32, device=device),
+                    "ws_l": g.workspace(g.gptq_chmc_workspace_bytes(rows, n, r), device),
+                    "qweight": torch.empty(rows, nw, dtype=torch.int32, device=device),
+                    "scale": torch.empty(-(-rows // CHMC_GS), n, dtype=torch.float32, device=device),
+                    "zero": torch.empty(-(-rows // CHMC_GS), n, dtype=torch.uint8, device=device),
+                    "loss": torch.empty(rows, dtype=torch.float32, device=device),
+                    "info_q": torch.zeros(2, dtype=torch.int32, device=device),
+                    "ws_q": g.workspace(g.gptq_quantize_workspace_bytes(rows, n, p.block), device),
+                })
+            self.items.append(it)
+
+    def run_problem(self, it):
+        g, p, s = self.g, it["p"], it["stream"]
+        with torch.cuda.stream(s):
+            it["H"].zero_()
+        g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
+        g.gptq_prepare(it["H"], CHMC_DAMP, "act", it["perm"], it["U"], it["dead"],
+                       it["info_p"], it["ws_p"], s)
+        for q in it["parts"]:
+            g.gptq_chmc_lowrank(q["W"], it["H"], p.T, CHMC_LAM, q["Om"], q["r"], CHMC_NITER,
+                                q["Q"] if q["r"] > 0 else None, q["P"] if q["r"] > 0 else None,
+                                q["R"], q["info_l"], q["ws_l"], s)
+            g.gptq_quantize_rowgroups(q["R"], it["U"], it["perm"], it["dead"], p.bits, CHMC_GS,
+                                      p.block, q["qweight"], q["scale"], q["zero"], q["loss"],
+                                      None, q["info_q"], q["ws_q"], s)
+
+    def step(self, main):
+        fork = torch.cuda.Event()
+        fork.record(main)
+        joins = []
+        for it in self.items:
+            it["stream"].wait_event(fork)
+            self.run_problem(it)
+            e = torch.cuda.Event()
+            e.record(it["stream"])
+            joins.append(e)
+        for e in joins:
+            main.wait_event(e)
+
+    def step_serial(self, main):
+        for it in self.items:
+            s = it["stream"]
+            it["stream"] = main
+            try:
+                self.run_problem(it)
+            finally:
+                it["stream"] = s
+
+    def check(self):
+        for it in self.items:
+            for key in ("info_h", "info_p"):
+                st, idx = self.g.gptq_check(it[key], it["stream"])
+                if st != 0:
+                    raise RuntimeError(f"device reported status {st} at {idx}")
+            for q in it["parts"]:
+                for key in ("info_l", "info_q"):
+                    st, idx = self.g.gptq_check(q[key], it["stream"])
+                    if st != 0:
+                        raise RuntimeError(f"{q['name']}: device reported status {st} at {idx}")
+
+
+def chmc_work(layer):
+    """Algorithmic work per kernel kind for one CHMC step.
+
+    hessian, cholesky as for GPTQ; chmc bytes: W read 2·niter + 3 times (the
+    sketch, niter power iterations of two products each, Qᵀ·W, the residual)
+    plus the float32 residual written; sweep/ingest/pack as for GPTQ on the
+    float32 residual (scale and zero per row group and column)."""
+    w = {k: 0.0 for k in ("hessian", "cholesky", "chmc", "sweep", "pack", "ingest")}
+    for it in layer.items:
+        p = it["p"]
+        n, T = p.n, p.T
+        w["hessian"] += T * n * (n + 1)
+        N = -(-n // 64)
+        for k in range(N):
+            r = N - k - 1
+            w["cholesky"] += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
+            w["cholesky"] += 2 * 64 ** 3 / 3
+        for q in it["parts"]:
+            m = q["W"].shape[0]
+            sw = q["W"].element_size()
+            w["chmc"] += (2 * CHMC_NITER + 3) * m * n * sw + 4 * m * n
+            fused = n % 4 == 0 and n > p.block
+            for j0 in range(0, n, p.block):
+                bw = min(p.block, n - j0)
+                n2 = n - j0 - bw
+                w["sweep"] += 9 * m * bw + 4 * bw * bw + 5 * (-(-m // CHMC_GS)) * bw
+                if n2 > 0 and fused:
+                    w["sweep"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
+            w["pack"] += m * n + m * n * p.bits / 8 + 5 * (-(-m // CHMC_GS)) * n
+            w["ingest"] += m * n * 8
+    units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s", "chmc": "GB/s", "sweep": "GB/s",
+             "pack": "GB/s", "ingest": "GB/s"}
+    return {k: (units[k], v) for k, v in w.items()}
+
+
+def run_chmc(args, rank, world, local):
+    """The CHMC frontend over the layer: device-timed graph replay and the
+    per-kernel event profile, as for the GPTQ path (no host-copy leg)."""
+    import post_weight_quantization_08_b200 as g
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = CONFIGS[args.config]
+    bits = args.bits or cfg["bits"][0]
+    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits, order="act")
+    layer = ChmcLayer(probs, device)
+    params = sum(p.params for p in probs)
+    main = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(main)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(args.warmup):
+        layer.step(main)
+    torch.cuda.synchronize(device)
+    layer.check()
+    graph = torch.cuda.CUDAGraph()
+    c0 = g.gptq_launch_count()
+    with torch.cuda.graph(graph, stream=main):
+        layer.step(main)
+    launches_per_step = g.gptq_launch_count() - c0
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(device)
+    layer.check()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        graph.replay()
+        b.record(main)
+        evs.append((a, b))
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    layer.check()
+    dev_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
+    total_params = sum_over_ranks(params * args.steps, world, device)
+    g.gptq_profile_start(1 << 16)
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        layer.step_serial(main)
+    torch.cuda.synchronize(device)
+    kprof = g.gptq_profile_stop()
+    work = chmc_work(layer)
+    peaks, src = _peaks()
+    kernels = {}
+    for k, (unit, amount) in work.items():
+        if k not in kprof or kprof[k][1] <= 0 or amount <= 0:
+            continue
+        per_step_ms = kprof[k][0] / args.steps
+        if unit == "TFLOP/s":
+            ach = amount / (per_step_ms / 1e3) / 1e12
+            bound, peak = (("tensor", peaks["bf16_tflops"]) if k == "hessian" else
+                           ("alu", fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))))
+        else:
+            ach = amount / (per_step_ms / 1e3) / 1e9
+            bound, peak = "hbm", peaks["hbm_gbs"]
+        kernels[k] = {"ms_per_step": round(per_step_ms, 4),
+                      "launches_per_step": kprof[k][1] / args.steps, "bound": bound,
+                      "achieved": round(ach, 2), "unit": unit, "peak": round(peak, 1),
+                      "frac": round(ach / peak, 4)}
+    ranks = {q["name"]: q["r"] for it in layer.items for q in it["parts"]}
+    return {
+        "metric": CHMC_METRIC, "value": round(total_params / (dev_ms / 1e3), 1),
+        "unit": "params/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->f32 Hessian, f64 prepare and low-rank part, f32 sweep",
+        "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
+        "config": {"workload": f"{cfg['name']} CHMC: per-matrix rank from the {CHMC_BPW}-bit "
+                               f"budget, niter {CHMC_NITER}, lambda {CHMC_LAM}, damp {CHMC_DAMP}, "
+                               f"act-order, residual {bits}-bit with {CHMC_GS}-row output-channel "
+                               f"groups, block {probs[0].block}",
+                   "params_per_step_per_gpu": params, "ranks": ranks,
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "launch": "CUDA graph replay per step"},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "kernels": kernels,
+        "kernels_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in kprof.items()
+                                if v[0] > 0},
+        "clocks": clk,
+    }, probs
+
+
+def chmc_cpu_baseline(probs):
+    """The CHMC oracle over the whole layer (every matrix, each Hessian from X
+    inside the timed region), params/s."""
+    from oracle import chmc as oc
+    from oracle import gptq as og
+    t0 = time.perf_counter()
+    total = 0
+    for pi, p in enumerate(probs):
+        X = p.X.to(torch.float64).numpy()
+        H = og.hessian(X)
+        row0 = 0
+        for k, (name, rows) in enumerate(p.parts):
+            W = p.W[row0:row0 + rows].to(torch.float64).numpy()
+            row0 += rows
+            r = oc.chmc_rank(rows, p.n, p.bits, CHMC_GS, CHMC_BPW)
+            Om = normal_matrix(p.n, max(r, 1), 9000 + 100 * pi + k)[:, :r].to(torch.float64).numpy()
+            oc.chmc_layer(W, H, p.T, Om, rank=r, bits=p.bits, gs=CHMC_GS, damp=CHMC_DAMP,
+                          niter=CHMC_NITER, block=p.block)
+            total += rows * p.n
+    dt = time.perf_counter() - t0
+    return {"value": round(total / dt, 1), "unit": "params/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": "one full pass over the layer's seven matrices, "
+                                        "both Hessians from X included"}
+
+
 # ---------------------------------------------------------------- CPU oracle arm
 
 def oracle_pass(probs):
@@ -553,6 +808,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--frontend", default="gptq", choices=["gptq", "chmc"],
+                    help="chmc: the CHMC frontend over the layer (a separate metric)")
     ap.add_argument("--order", default=None,
                     choices=["natural", "act", "reverse", "minpivot"],
                     help="processing order for every problem (default: the workload's)")
@@ -573,10 +830,15 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
-        out, probs, _ = run_ours(args, rank, world, local)
-        if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
+        if args.frontend == "chmc":
+            out, probs = run_chmc(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = chmc_cpu_baseline(probs)
+        else:
+            out, probs, _ = run_ours(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(probs)
+        if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
         if world > 1:
