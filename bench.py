@@ -522,23 +522,42 @@ class ChmcLayer:
                     "loss": torch.empty(rows, dtype=torch.float32, device=device),
                     "info_q": torch.zeros(2, dtype=torch.int32, device=device),
                     "ws_q": g.workspace(g.gptq_quantize_workspace_bytes(rows, n, p.block), device),
+                    "stream": torch.cuda.Stream(device=device),
                 })
             self.items.append(it)
 
-    def run_problem(self, it):
+    def run_problem(self, it, serial=False):
+        """The matrices sharing one H run on streams of their own: each low-rank
+        part beside the factorisation (both read only H), each residual's
+        quantization once the factor is there (``serial``: all on one stream)."""
         g, p, s = self.g, it["p"], it["stream"]
         with torch.cuda.stream(s):
             it["H"].zero_()
         g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
-        g.gptq_prepare(it["H"], CHMC_DAMP, "act", it["perm"], it["U"], it["dead"],
-                       it["info_p"], it["ws_p"], s)
+        h_ready = torch.cuda.Event()
+        h_ready.record(s)
         for q in it["parts"]:
+            qs = s if serial else q["stream"]
+            if not serial:
+                qs.wait_event(h_ready)
             g.gptq_chmc_lowrank(q["W"], it["H"], p.T, CHMC_LAM, q["Om"], q["r"], CHMC_NITER,
                                 q["Q"] if q["r"] > 0 else None, q["P"] if q["r"] > 0 else None,
-                                q["R"], q["info_l"], q["ws_l"], s)
+                                q["R"], q["info_l"], q["ws_l"], qs)
+        g.gptq_prepare(it["H"], CHMC_DAMP, "act", it["perm"], it["U"], it["dead"],
+                       it["info_p"], it["ws_p"], s)
+        prep_done = torch.cuda.Event()
+        prep_done.record(s)
+        for q in it["parts"]:
+            qs = s if serial else q["stream"]
+            if not serial:
+                qs.wait_event(prep_done)
             g.gptq_quantize_rowgroups(q["R"], it["U"], it["perm"], it["dead"], p.bits, CHMC_GS,
                                       p.block, q["qweight"], q["scale"], q["zero"], q["loss"],
-                                      None, q["info_q"], q["ws_q"], s)
+                                      None, q["info_q"], q["ws_q"], qs)
+            if not serial:
+                e = torch.cuda.Event()
+                e.record(qs)
+                s.wait_event(e)
 
     def step(self, main):
         fork = torch.cuda.Event()
@@ -558,7 +577,7 @@ class ChmcLayer:
             s = it["stream"]
             it["stream"] = main
             try:
-                self.run_problem(it)
+                self.run_problem(it, serial=True)
             finally:
                 it["stream"] = s
 

@@ -78,7 +78,7 @@ __global__ void chmc_to_f64_kernel(const float* __restrict__ x, int64_t count,
 
 // Y[row][k] = Σ_j W[row][j]·(sq ? sq[j] : 1)·X[j][k]: one warp per row, lanes
 // along the row (coalesced), then a fixed shuffle tree per k.
-template <typename T>
+template <typename T, int RMAX>
 __global__ void __launch_bounds__(256)
 chmc_rowprod_kernel(const T* __restrict__ W, int64_t o, int64_t i,
                     const double* __restrict__ sq, const double* __restrict__ X, int r,
@@ -86,19 +86,29 @@ chmc_rowprod_kernel(const T* __restrict__ W, int64_t o, int64_t i,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
   if (row >= o) return;
-  double acc[CHMC_MAX_RANK];
+  double acc[RMAX];
 #pragma unroll
-  for (int k = 0; k < CHMC_MAX_RANK; ++k) acc[k] = 0.0;
-  for (int64_t j = lane; j < i; j += 32) {
-    double w = to_f64(W[row * i + j]);
-    if (sq) w *= sq[j];
-    const double* x = X + j * r;
+  for (int k = 0; k < RMAX; ++k) acc[k] = 0.0;
+  for (int64_t j0 = lane; j0 < i; j0 += 128) {
+    double w[4];
 #pragma unroll
-    for (int k = 0; k < CHMC_MAX_RANK; ++k)
-      if (k < r) acc[k] = fma(w, x[k], acc[k]);
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = j0 + 32 * u;
+      w[u] = (j < i) ? to_f64(W[row * i + j]) * (sq ? sq[j] : 1.0) : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = j0 + 32 * u;
+      if (j < i) {
+        const double* x = X + j * r;
+#pragma unroll
+        for (int k = 0; k < RMAX; ++k)
+          if (k < r) acc[k] = fma(w[u], x[k], acc[k]);
+      }
+    }
   }
 #pragma unroll
-  for (int k = 0; k < CHMC_MAX_RANK; ++k) {
+  for (int k = 0; k < RMAX; ++k) {
     if (k < r) {
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], off);
@@ -106,38 +116,76 @@ chmc_rowprod_kernel(const T* __restrict__ W, int64_t o, int64_t i,
   }
   if (lane == 0) {
 #pragma unroll
-    for (int k = 0; k < CHMC_MAX_RANK; ++k)
+    for (int k = 0; k < RMAX; ++k)
       if (k < r) Y[row * r + k] = acc[k];
   }
 }
 
-// Zp[chunk][j][k] = Σ_{row in chunk} W[row][j]·Qo[row][k]: one thread per
-// column of W, one CTA per (128 columns, 128-row chunk).
-template <typename T>
-__global__ void __launch_bounds__(128)
+// Zp[chunk][j][k] = Σ_{row in chunk} W[row][j]·Qo[row][k]: one CTA per (64
+// columns, 128-row chunk); thread (column, slice) sums 32 rows with eight
+// loads in flight, and the four slices are added in a fixed order.
+constexpr int CP_COLS = 64, CP_SLICES = 4;
+template <typename T, int RMAX>
+__global__ void __launch_bounds__(256)
 chmc_colprod_kernel(const T* __restrict__ W, int64_t o, int64_t i,
                     const double* __restrict__ Qo, int r, double* __restrict__ Zp) {
-  __shared__ double qs[CHUNK * CHMC_MAX_RANK];
-  const int64_t j = (int64_t)blockIdx.x * 128 + threadIdx.x;
+  __shared__ double qs[CHUNK * CHMC_MAX_RANK];   // Q rows, then the slices' sums
+  static_assert(2 * CP_COLS * CHMC_MAX_RANK <= CHUNK * CHMC_MAX_RANK, "reduction space");
+  const int tid = threadIdx.x, jc = tid % CP_COLS, sl = tid / CP_COLS;
+  const int64_t j = (int64_t)blockIdx.x * CP_COLS + jc;
   const int64_t r0 = (int64_t)blockIdx.y * CHUNK;
   const int rows = (int)((o - r0 < CHUNK) ? (o - r0) : CHUNK);
-  for (int e = threadIdx.x; e < rows * r; e += 128) qs[e] = Qo[r0 * r + e];
+  for (int e = tid; e < rows * r; e += 256) qs[e] = Qo[r0 * r + e];
   __syncthreads();
-  if (j >= i) return;
-  double acc[CHMC_MAX_RANK];
+  double acc[RMAX];
 #pragma unroll
-  for (int k = 0; k < CHMC_MAX_RANK; ++k) acc[k] = 0.0;
-  for (int rr = 0; rr < rows; ++rr) {
-    const double w = to_f64(W[(r0 + rr) * i + j]);
-    const double* q = qs + rr * r;
+  for (int k = 0; k < RMAX; ++k) acc[k] = 0.0;
+  const int rs = sl * (CHUNK / CP_SLICES);
+  const int re = (rs + CHUNK / CP_SLICES < rows) ? rs + CHUNK / CP_SLICES : rows;
+  if (j < i) {
+    for (int rr0 = rs; rr0 < re; rr0 += 8) {
+      double w[8];
 #pragma unroll
-    for (int k = 0; k < CHMC_MAX_RANK; ++k)
-      if (k < r) acc[k] = fma(w, q[k], acc[k]);
+      for (int u = 0; u < 8; ++u)
+        w[u] = (rr0 + u < re) ? to_f64(W[(r0 + rr0 + u) * i + j]) : 0.0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (rr0 + u < re) {
+          const double* q = qs + (rr0 + u) * r;
+#pragma unroll
+          for (int k = 0; k < RMAX; ++k)
+            if (k < r) acc[k] = fma(w[u], q[k], acc[k]);
+        }
+      }
+    }
   }
-  double* out = Zp + ((int64_t)blockIdx.y * i + j) * r;
+  // ((slice 0 + slice 2) + (slice 1 + slice 3)) through the Q staging space
+  double* red = qs;                                  // [2][CP_COLS][r]
+  __syncthreads();
+  if (sl >= 2) {
 #pragma unroll
-  for (int k = 0; k < CHMC_MAX_RANK; ++k)
-    if (k < r) out[k] = acc[k];
+    for (int k = 0; k < RMAX; ++k)
+      if (k < r) red[((sl - 2) * CP_COLS + jc) * r + k] = acc[k];
+  }
+  __syncthreads();
+  if (sl < 2) {
+#pragma unroll
+    for (int k = 0; k < RMAX; ++k)
+      if (k < r) acc[k] += red[(sl * CP_COLS + jc) * r + k];
+  }
+  __syncthreads();
+  if (sl == 1) {
+#pragma unroll
+    for (int k = 0; k < RMAX; ++k)
+      if (k < r) red[jc * r + k] = acc[k];
+  }
+  __syncthreads();
+  if (sl == 0 && j < i) {
+    double* out = Zp + ((int64_t)blockIdx.y * i + j) * r;
+#pragma unroll
+    for (int k = 0; k < RMAX; ++k)
+      if (k < r) out[k] = acc[k] + red[jc * r + k];
+  }
 }
 
 // Z[j][k] = (sq ? sq[j] : 1)·Σ_chunk Zp[chunk][j][k], chunks in order.
@@ -238,6 +286,106 @@ __global__ void chmc_apply_kernel(const double* __restrict__ Y, int64_t rows, in
   }
 }
 
+// CholeskyQR2 of a rows × r matrix that fits in shared memory, in one CTA:
+// Y is staged once; each pass forms the Gram matrix (a warp per (a, b) pair,
+// lanes over the rows, a fixed shuffle tree), factors it with warp 0 as
+// chmc_chol_kernel does (dropping non-positive pivots), and multiplies in
+// place by R⁻¹.  Q receives the result.
+constexpr int ORTH_SMALL_MAX = 12288;          // rows·r doubles staged (96 KB)
+constexpr int ORTH_T = 256;
+__global__ void __launch_bounds__(ORTH_T)
+chmc_orth_small_kernel(const double* __restrict__ Yin, int rows, int r, double* __restrict__ Q) {
+  extern __shared__ double osm[];
+  double* Y = osm;                                  // rows × r
+  __shared__ double G[CHMC_MAX_RANK][CHMC_MAX_RANK + 1];
+  __shared__ double L[CHMC_MAX_RANK][CHMC_MAX_RANK + 1];
+  __shared__ double Ri[CHMC_MAX_RANK * CHMC_MAX_RANK];
+  const int t = threadIdx.x, lane = t & 31;
+#pragma unroll 8
+  for (int e = t; e < rows * r; e += ORTH_T) Y[e] = Yin[e];
+  const int npair = r * (r + 1) / 2;
+  const int warp = t >> 5;
+  auto pair_ab = [&](int pidx, int& a, int& b) {
+    int rem = pidx;
+    a = 0;
+    while (rem >= r - a) { rem -= r - a; ++a; }
+    b = a + rem;
+  };
+  for (int pass = 0; pass < 2; ++pass) {
+    __syncthreads();
+    // Gram entries: warp w takes pairs w, w + 8, ...; its lanes stride the
+    // rows four at a time, then a fixed shuffle tree adds the lanes
+    for (int pidx = warp; pidx < npair; pidx += ORTH_T / 32) {
+      int a, b;
+      pair_ab(pidx, a, b);
+      double acc0 = 0.0, acc1 = 0.0;
+      int rr = lane;
+      for (; rr + 96 < rows; rr += 128) {
+        const double y0 = Y[rr * r + a], z0 = Y[rr * r + b];
+        const double y1 = Y[(rr + 32) * r + a], z1 = Y[(rr + 32) * r + b];
+        const double y2 = Y[(rr + 64) * r + a], z2 = Y[(rr + 64) * r + b];
+        const double y3 = Y[(rr + 96) * r + a], z3 = Y[(rr + 96) * r + b];
+        acc0 = fma(y0, z0, acc0);
+        acc1 = fma(y1, z1, acc1);
+        acc0 = fma(y2, z2, acc0);
+        acc1 = fma(y3, z3, acc1);
+      }
+      for (; rr < rows; rr += 32) acc0 = fma(Y[rr * r + a], Y[rr * r + b], acc0);
+      double acc = acc0 + acc1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) {
+        G[a][b] = acc;
+        G[b][a] = acc;
+      }
+    }
+    __syncthreads();
+    if (t < 32) {
+      for (int b = 0; b < r; ++b)
+        if (lane < r) L[lane][b] = 0.0;
+      double tr = 0.0;
+      for (int k = 0; k < r; ++k) tr += G[k][k];
+      const double floor_piv = 1e-28 * (tr > 0.0 ? tr : 1.0);
+      __syncwarp();
+      for (int k = 0; k < r; ++k) {
+        const double piv = G[k][k];
+        const bool keep = piv > floor_piv;
+        const double d = keep ? sqrt(piv) : 0.0;
+        __syncwarp();
+        if (lane >= k && lane < r) L[lane][k] = keep ? G[lane][k] / d : 0.0;
+        __syncwarp();
+        if (lane > k && lane < r)
+          for (int l = k + 1; l <= lane; ++l) G[lane][l] -= L[lane][k] * L[l][k];
+        __syncwarp();
+      }
+      if (lane < r) {
+        double x[CHMC_MAX_RANK];
+#pragma unroll
+        for (int i = 0; i < CHMC_MAX_RANK; ++i) x[i] = 0.0;
+        for (int i = lane; i < r; ++i) {
+          double sacc = (i == lane) ? 1.0 : 0.0;
+          for (int m2 = lane; m2 < i; ++m2) sacc -= L[i][m2] * x[m2];
+          x[i] = (L[i][i] != 0.0) ? sacc / L[i][i] : 0.0;
+        }
+        for (int i = 0; i < r; ++i) Ri[lane * r + i] = (i >= lane) ? x[i] : 0.0;
+      }
+    }
+    __syncthreads();
+    // Y ← Y·R⁻¹ in place, a row per thread: column k needs columns l ≤ k, so
+    // the columns are formed from the last to the first
+    for (int row = t; row < rows; row += ORTH_T) {
+      double* y = Y + row * r;
+      for (int k = r - 1; k >= 0; --k) {
+        double acc = 0.0;
+        for (int l = 0; l <= k; ++l) acc = fma(y[l], Ri[l * r + k], acc);
+        y[k] = acc;
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = t; e < rows * r; e += ORTH_T) Q[e] = Y[e];
+}
+
 // Outputs: Qf = Q (o × r), Pf = Pᵀ stored r × i, Res = W − Q·P (o × i); all float32.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -297,6 +445,11 @@ size_t chmc_layout(int64_t o, int64_t i, int r, char* base, double** sq, double*
 // thread reads its whole row before writing it), then Q = Y·R₂⁻¹.
 gptq_status orth_rows(double* Y, int64_t rows, int r, double* Q, double* Gp, double* Rinv,
                       cudaStream_t s) {
+  if (rows * r <= ORTH_SMALL_MAX) {               // one CTA, Y in shared memory
+    const size_t smem = sizeof(double) * (size_t)rows * r;
+    GPTQ_LAUNCH(KK_CHMC, s, chmc_orth_small_kernel, 1, ORTH_T, smem, Y, (int)rows, r, Q);
+    return GPTQ_OK;
+  }
   const unsigned nch = (unsigned)ceil_div(rows, CHUNK);
   const unsigned ga = (unsigned)ceil_div(rows, 256);
   for (int pass = 0; pass < 2; ++pass) {
@@ -308,6 +461,40 @@ gptq_status orth_rows(double* Y, int64_t rows, int r, double* Q, double* Gp, dou
   return GPTQ_OK;
 }
 
+// The thin products at the smallest compiled rank bound that holds r.
+template <typename T, int RM>
+gptq_status rowprod_at(unsigned grid, const T* W, int64_t o, int64_t i, const double* sq,
+                       const double* X, int r, double* Y, cudaStream_t s) {
+  const auto kfn = &chmc_rowprod_kernel<T, RM>;
+  GPTQ_LAUNCH(KK_CHMC, s, kfn, grid, 256, 0, W, o, i, sq, X, r, Y);
+  return GPTQ_OK;
+}
+template <typename T>
+gptq_status launch_rowprod(unsigned grid, const T* W, int64_t o, int64_t i, const double* sq,
+                           const double* X, int r, double* Y, cudaStream_t s) {
+  if (r <= 4) return rowprod_at<T, 4>(grid, W, o, i, sq, X, r, Y, s);
+  if (r <= 8) return rowprod_at<T, 8>(grid, W, o, i, sq, X, r, Y, s);
+  if (r <= 16) return rowprod_at<T, 16>(grid, W, o, i, sq, X, r, Y, s);
+  return rowprod_at<T, 32>(grid, W, o, i, sq, X, r, Y, s);
+}
+template <typename T, int RM>
+gptq_status colprod_at(dim3 grid, const T* W, int64_t o, int64_t i, const double* Q, int r,
+                       double* Zp, cudaStream_t s) {
+  const auto kfn = &chmc_colprod_kernel<T, RM>;
+  GPTQ_LAUNCH(KK_CHMC, s, kfn, grid, 256, 0, W, o, i, Q, r, Zp);
+  return GPTQ_OK;
+}
+template <typename T>
+gptq_status launch_colprod(dim3 grid, const T* W, int64_t o, int64_t i, const double* Q, int r,
+                           double* Zp, cudaStream_t s) {
+  if (r <= 4) return colprod_at<T, 4>(grid, W, o, i, Q, r, Zp, s);
+  if (r <= 8) return colprod_at<T, 8>(grid, W, o, i, Q, r, Zp, s);
+  if (r <= 16) return colprod_at<T, 16>(grid, W, o, i, Q, r, Zp, s);
+  return colprod_at<T, 32>(grid, W, o, i, Q, r, Zp, s);
+}
+
+bool g_orth_attr = false;
+
 template <typename T>
 gptq_status lowrank_impl(const T* W, int64_t o, int64_t i, const float* H, int64_t tokens,
                          double lam, const float* Omega, int r, int niter, float* Qf,
@@ -315,6 +502,12 @@ gptq_status lowrank_impl(const T* W, int64_t o, int64_t i, const float* H, int64
   double *sq, *om, *Y, *Q, *Z, *Qi, *Zp, *Gp, *Rinv, *P;
   chmc_layout(o, i, r, ws, &sq, &om, &Y, &Q, &Z, &Qi, &Zp, &Gp, &Rinv, &P);
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
+  if (!g_orth_attr) {
+    GPTQ_CUDA(cudaFuncSetAttribute(chmc_orth_small_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)(sizeof(double) * ORTH_SMALL_MAX)));
+    g_orth_attr = true;
+  }
   if (r == 0) {
     GPTQ_LAUNCH(KK_CHMC, s, chmc_copy_kernel<T>, (unsigned)ceil_div(o * i, 256), 256, 0, W,
                 o * i, Res);
@@ -324,26 +517,30 @@ gptq_status lowrank_impl(const T* W, int64_t o, int64_t i, const float* H, int64
   GPTQ_LAUNCH(KK_CHMC, s, chmc_to_f64_kernel, (unsigned)ceil_div(i * r, 256), 256, 0, Omega,
               i * r, om);
   const unsigned grow = (unsigned)ceil_div(o, 8);
-  const dim3 gcol((unsigned)ceil_div(i, 128), (unsigned)ceil_div(o, CHUNK));
+  const dim3 gcol((unsigned)ceil_div(i, CP_COLS), (unsigned)ceil_div(o, CHUNK));
   const int nco = (int)ceil_div(o, CHUNK);
   const unsigned gred = (unsigned)ceil_div(i * r, 256);
   // Y = W̃·Ω, Q = orth(Y)
-  GPTQ_LAUNCH(KK_CHMC, s, chmc_rowprod_kernel<T>, grow, 256, 0, W, o, i, sq, om, r, Y);
-  gptq_status st = orth_rows(Y, o, r, Q, Gp, Rinv, s);
+  gptq_status st = launch_rowprod(grow, W, o, i, sq, om, r, Y, s);
+  if (st != GPTQ_OK) return st;
+  st = orth_rows(Y, o, r, Q, Gp, Rinv, s);
   if (st != GPTQ_OK) return st;
   for (int it = 0; it < niter; ++it) {
     // Qi = orth(W̃ᵀ·Q) with W̃ᵀ·Q = diag(√c)·Wᵀ·Q
-    GPTQ_LAUNCH(KK_CHMC, s, chmc_colprod_kernel<T>, gcol, 128, 0, W, o, i, Q, r, Zp);
+    st = launch_colprod(gcol, W, o, i, Q, r, Zp, s);
+    if (st != GPTQ_OK) return st;
     GPTQ_LAUNCH(KK_CHMC, s, chmc_colreduce_kernel, gred, 256, 0, Zp, nco, i, r, sq, Z);
     st = orth_rows(Z, i, r, Qi, Gp, Rinv, s);
     if (st != GPTQ_OK) return st;
     // Q = orth(W̃·Qi)
-    GPTQ_LAUNCH(KK_CHMC, s, chmc_rowprod_kernel<T>, grow, 256, 0, W, o, i, sq, Qi, r, Y);
+    st = launch_rowprod(grow, W, o, i, sq, Qi, r, Y, s);
+    if (st != GPTQ_OK) return st;
     st = orth_rows(Y, o, r, Q, Gp, Rinv, s);
     if (st != GPTQ_OK) return st;
   }
   // P = Qᵀ·W (stored i × r), then the residual W − Q·P and the factors
-  GPTQ_LAUNCH(KK_CHMC, s, chmc_colprod_kernel<T>, gcol, 128, 0, W, o, i, Q, r, Zp);
+  st = launch_colprod(gcol, W, o, i, Q, r, Zp, s);
+  if (st != GPTQ_OK) return st;
   GPTQ_LAUNCH(KK_CHMC, s, chmc_colreduce_kernel, gred, 256, 0, Zp, nco, i, r,
               (const double*)nullptr, P);
   const dim3 gres((unsigned)ceil_div(i, 256), (unsigned)o);

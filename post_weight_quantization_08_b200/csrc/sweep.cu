@@ -155,6 +155,13 @@ __device__ __forceinline__ float div_fma(float x, float s, float rs) {
   return fmaf(r, rs, q0);
 }
 
+// Signed-integer image of a float that orders like the float (finite values).
+__device__ __forceinline__ int ord_key(float f) {
+  const int b = __float_as_int(f);
+  return b ^ ((b >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ int ord_key_inv(int k) { return k ^ ((k >> 31) & 0x7fffffff); }
+
 // One CTA (bx: the 128-row tile) of the sweep; smraw: SMEM_BYTES of dynamic
 // shared memory.  ROWG: scales along the output channels (CHMC page, Schritt
 // 2 and 3: ⌈o/gs⌉·i scales, gs = 128 rows, the CTA's own rows): each column's
@@ -443,12 +450,14 @@ __device__ __forceinline__ void sweep_body(
         // the column's min and max over the CTA's rows (0 inside the range):
         // warp shuffles, then the four warps through shared memory (two
         // buffers by column parity, so one barrier per column suffices)
-        float mn = fminf(v[i], 0.f), mx = fmaxf(v[i], 0.f);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        }
+        // warp min and max in one instruction each, on an integer image of
+        // the floats that orders like them (negative values get their
+        // magnitude bits flipped; the map is its own inverse)
+        const int kn = ord_key(fminf(v[i], 0.f)), kx = ord_key(fmaxf(v[i], 0.f));
+        int wn, wx;
+        asm volatile("redux.sync.min.s32 %0, %1, 0xffffffff;" : "=r"(wn) : "r"(kn));
+        asm volatile("redux.sync.max.s32 %0, %1, 0xffffffff;" : "=r"(wx) : "r"(kx));
+        const float mn = __int_as_float(ord_key_inv(wn)), mx = __int_as_float(ord_key_inv(wx));
         float* red = reinterpret_cast<float*>(sm + SM_RGRED) + (i & 1) * 8;
         if (lane == 0) {
           red[warp] = mn;
