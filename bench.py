@@ -248,28 +248,69 @@ class Layer:
                 "g_idx": torch.empty(n, dtype=torch.int32, device=device),
                 "loss": torch.empty(m, dtype=torch.float32, device=device),
                 "stream": torch.cuda.Stream(device=device),
+                "cstream": torch.cuda.Stream(device=device),
             }
             self.items.append(it)
 
-    def run_problem(self, it):
+    OUTS = ("qweight", "scale", "zero", "g_idx", "loss")
+
+    def run_problem(self, it, w_ready=None, host=None):
+        """One problem on its stream; ``w_ready``: the event after which W is
+        in place; ``host``: pinned buffers that receive the results."""
         g, p, s = self.g, it["p"], it["stream"]
         with torch.cuda.stream(s):
             it["H"].zero_()
         g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
         g.gptq_prepare(it["H"], p.damp, p.order, it["perm"], it["U"], it["dead"],
                        it["info_p"], it["ws_p"], s)
+        if w_ready is not None:
+            s.wait_event(w_ready)
         g.gptq_quantize(it["W"], it["U"], it["perm"], it["dead"], p.bits, p.group, p.block,
                         it["qweight"], it["scale"], it["zero"], it["g_idx"], it["loss"],
                         None, it["info_q"], it["ws_q"], s)
+        if host is not None:
+            with torch.cuda.stream(s):
+                for k in self.OUTS:
+                    host[k].copy_(it[k], non_blocking=True)
 
-    def step(self, main):
-        """Fork the layer's problems onto their own streams, join on `main`."""
+    def step(self, main, hosts=None):
+        """Fork the layer's problems onto their own streams, join on `main`.
+
+        ``hosts``: per problem pinned input/output buffers (the end-to-end
+        step).  Then every problem's X is copied in first, largest n first
+        (the problem on the critical path starts earliest), each problem starts
+        as soon as its own X is in, and the W copies follow on copy streams of
+        their own while the factorisations run; each quantize waits only for
+        its W."""
         fork = torch.cuda.Event()
         fork.record(main)
         joins = []
-        for it in self.items:
+        order = list(range(len(self.items)))
+        w_ready = [None] * len(self.items)
+        if hosts is not None:
+            order.sort(key=lambda k: -self.items[k]["p"].n)
+            prev = None
+            for k in order:                      # X, in priority order
+                it, s = self.items[k], self.items[k]["stream"]
+                s.wait_event(fork)
+                if prev is not None:
+                    s.wait_event(prev)
+                with torch.cuda.stream(s):
+                    it["X"].copy_(hosts[k]["X"], non_blocking=True)
+                prev = torch.cuda.Event()
+                prev.record(s)
+            for k in order:                      # then W, on the copy streams
+                it, cs = self.items[k], self.items[k]["cstream"]
+                cs.wait_event(prev)
+                with torch.cuda.stream(cs):
+                    it["W"].copy_(hosts[k]["W"], non_blocking=True)
+                prev = torch.cuda.Event()
+                prev.record(cs)
+                w_ready[k] = prev
+        for k in order:
+            it = self.items[k]
             it["stream"].wait_event(fork)
-            self.run_problem(it)
+            self.run_problem(it, w_ready[k], hosts[k] if hosts is not None else None)
             e = torch.cuda.Event()
             e.record(it["stream"])
             joins.append(e)
@@ -370,21 +411,28 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(device)
     kprof = g.gptq_profile_stop()
 
-    # ---- end to end: pinned host inputs in, packed results out, every step
-    host_in = [(it, it["X"].cpu().pin_memory(), it["W"].cpu().pin_memory()) for it in layer.items]
-    host_out = [{k: torch.empty(it[k].shape, dtype=it[k].dtype).pin_memory()
-                 for k in ("qweight", "scale", "zero", "g_idx", "loss")} for it in layer.items]
-    h2d = sum(x.numel() * x.element_size() + w.numel() * w.element_size() for _, x, w in host_in)
-    d2h = sum(t.numel() * t.element_size() for o in host_out for t in o.values())
+    # ---- end to end: pinned host inputs in, packed results out, every step.
+    # The copies are part of the captured step, on the problems' own streams:
+    # the activations of the problem on the critical path go first, each
+    # problem starts as soon as its own activations are in, and the weights
+    # arrive while the factorisations run.
+    hosts = [{"X": it["X"].cpu().pin_memory(), "W": it["W"].cpu().pin_memory(),
+              **{k: torch.empty(it[k].shape, dtype=it[k].dtype).pin_memory()
+                 for k in Layer.OUTS}} for it in layer.items]
+    h2d = sum(h["X"].numel() * h["X"].element_size() + h["W"].numel() * h["W"].element_size()
+              for h in hosts)
+    d2h = sum(h[k].numel() * h[k].element_size() for h in hosts for k in Layer.OUTS)
+    e2e_graph = None
+    if not args.no_graph:
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e2e_graph, stream=main):
+            layer.step(main, hosts)
 
     def e2e_step():
-        for (it, x, w) in host_in:
-            it["X"].copy_(x, non_blocking=True)
-            it["W"].copy_(w, non_blocking=True)
-        run_step()
-        for it, o in zip(layer.items, host_out):
-            for k, t in o.items():
-                t.copy_(it[k], non_blocking=True)
+        if e2e_graph is not None:
+            e2e_graph.replay()
+        else:
+            layer.step(main, hosts)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
