@@ -1,0 +1,315 @@
+"""Pins of the SSQR oracle against what the page and the mathematics fix.
+
+Page: "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+Algorithm", §3 (SSQR: outliers kept in full precision, a binary search on the
+scales for a target outlier density) and §2.3 (Satz 5: the error bound that
+clipping breaks).  Each pin compares the oracle with something other than its
+own formula: explicit scalar loops, the hot path's pinned GPTQ oracle in a
+case where the two must agree, the Satz 5 bound, or a count whose threshold is
+known in closed form.  The last test plants plausible mistakes in the oracle
+and checks that the pins catch each of them.
+"""
+import numpy as np
+import pytest
+
+from oracle import gptq as G
+from oracle import ssqr as S
+
+
+def _spd(n, rng):
+    A = rng.standard_normal((n + 3, n))
+    return A.T @ A + 0.05 * np.eye(n)
+
+
+def _heavy(m, n, rng, scale=0.02):
+    """Weights with a heavy tail (Student-t, 3 degrees of freedom)."""
+    return rng.standard_t(3, size=(m, n)) * scale
+
+
+# ---------------------------------------------------------------- pin helpers
+
+def _rtn_with_outliers_by_loops(W, bits, group, alpha):
+    """U = I (no error feedback): round-to-nearest on the adjusted grid, the
+    out-of-grid weights kept, by scalar float32 loops."""
+    m, n = W.shape
+    maxq = 2 ** bits - 1
+    codes = np.zeros((m, n), np.int64)
+    mask = np.zeros((m, n), bool)
+    for r in range(m):
+        for g0 in range(0, n, group):
+            vals = [np.float32(W[r, c]) for c in range(g0, min(g0 + group, n))]
+            lo = min(min(vals), np.float32(0))
+            hi = max(max(vals), np.float32(0))
+            if lo == 0 and hi == 0:
+                lo, hi = np.float32(-1), np.float32(1)
+            s0 = np.float32((hi - lo) / np.float32(maxq))
+            z = np.float32(np.rint(np.float32(-lo) / s0))
+            s = np.float32(s0 * np.float32(alpha))
+            for c in range(g0, min(g0 + group, n)):
+                q = np.rint(np.float32(W[r, c]) / s) + z
+                mask[r, c] = q < 0 or q > maxq
+                codes[r, c] = int(min(max(q, 0), maxq))
+    return codes, mask
+
+
+def _satz5_holds(res, U, group):
+    """Per row: Σ e_j² ≤ ¼·Σ s_j²/U_jj² (inliers within half a step, outliers
+    with no error), and outliers carry e = 0."""
+    n = U.shape[0]
+    s = res["scale"][:, np.arange(n) // group].astype(np.float64)
+    bound = 0.25 * np.sum(s ** 2 / np.diag(U)[None, :] ** 2, axis=1)
+    loss = np.sum(res["err"] ** 2, axis=1)
+    return bool(np.all(loss <= bound * (1 + 1e-12)) and np.all(res["err"][res["mask"]] == 0))
+
+
+def _loss_identity_holds(Wp, res, Hp, group):
+    """(w − q̂)ᵀ H_p (w − q̂) = Σ_j e_j² per row, q̂ the outlier value where kept."""
+    n = Wp.shape[1]
+    g = np.arange(n) // group
+    Q = np.where(res["mask"], res["value"],
+                 G.dequantize(res["codes"], res["scale"][:, g], res["zero"][:, g]))
+    D = Wp - Q
+    lhs = np.einsum("ij,jk,ik->i", D, Hp, D)
+    return bool(np.allclose(lhs, np.sum(res["err"] ** 2, axis=1), rtol=1e-9, atol=1e-300))
+
+
+# ---------------------------------------------------------------- the sweep
+
+def test_alpha_one_with_one_column_groups_is_gptq():
+    """group = 1, α = 1: every value lies on its own row's grid range, so no
+    weight is an outlier and SSQR is the hot path's GPTQ bit for bit."""
+    rng = np.random.default_rng(1)
+    n = 40
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(13, n, rng)[:, p["perm"]]
+    a = S.ssqr_blocked(Wp, p["U"], 3, 1, 8, 1.0)
+    b = G.gptq_blocked(Wp, p["U"], 3, 1, 8)
+    assert S.count(a) == 0
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.array_equal(a["scale"], b["scale"])
+    assert np.array_equal(a["err"], b["err"])
+
+
+@pytest.mark.parametrize("alpha", [1.0, 0.75, 0.3])
+@pytest.mark.parametrize("bits,group", [(2, 8), (3, 16), (4, 32)])
+def test_identity_factor_is_rtn_with_outliers_kept(alpha, bits, group):
+    rng = np.random.default_rng(2)
+    W = _heavy(9, 64, rng)
+    res = S.ssqr_blocked(W, np.eye(64), bits, group, 32, alpha)
+    codes, mask = _rtn_with_outliers_by_loops(W, bits, group, alpha)
+    assert np.array_equal(res["mask"], mask)
+    assert np.array_equal(res["codes"], codes)
+    assert np.array_equal(res["value"][mask], W[mask])
+    if alpha < 1:
+        assert mask.any()
+
+
+@pytest.mark.parametrize("alpha", [1.0, 0.6, 0.35])
+def test_satz5_bound_holds_for_every_alpha(alpha):
+    """§2.3 Satz 5 bounds the unclipped error by ¼·Σ s_j²·D_jj; SSQR keeps it
+    for every α because overflowing weights are kept, not clipped."""
+    rng = np.random.default_rng(3)
+    n = 64
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(25, n, rng)[:, p["perm"]]
+    res = S.ssqr_blocked(Wp, p["U"], 2, 16, 32, alpha)
+    assert _satz5_holds(res, p["U"], 16)
+    assert _loss_identity_holds(Wp, res, p["Hp"], 16)
+
+
+def test_clipping_breaks_the_half_step_that_ssqr_keeps():
+    """The page's motivation.  Satz 5's bound adds up one term per column,
+    |w_j − q̂_j| ≤ s_j/2 (a nearest-plane step).  A clipped weight breaks its
+    term; SSQR at α = 1 keeps every term, since overflowing weights are
+    stored instead."""
+    rng = np.random.default_rng(4)
+    n = 64
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(40, n, rng)[:, p["perm"]]
+    d = np.diag(p["U"])[None, :]
+    clipped = G.gptq_blocked(Wp, p["U"], 2, 64, 64)
+    s = clipped["scale"][:, np.arange(n) // 64].astype(np.float64)
+    assert np.any(np.abs(clipped["err"]) * d > s / 2.0 * (1 + 1e-12))
+    ss = S.ssqr_blocked(Wp, p["U"], 2, 64, 64, 1.0)
+    s = ss["scale"][:, np.arange(n) // 64].astype(np.float64)
+    assert S.count(ss) > 0 and _satz5_holds(ss, p["U"], 64)
+    assert np.all(np.abs(ss["err"]) * d <= s / 2.0 * (1 + 1e-12))
+
+
+@pytest.mark.parametrize("n,group,block", [(96, 32, 32), (100, 32, 64), (64, 16, 64)])
+def test_blocked_equals_sequential(n, group, block):
+    rng = np.random.default_rng(5)
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(17, n, rng)[:, p["perm"]]
+    a = S.ssqr_sequential(Wp, p["U"], 3, group, 0.55)
+    b = S.ssqr_blocked(Wp, p["U"], 3, group, block, 0.55)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["mask"], b["mask"])
+    assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- the search
+
+def _threshold_run(x, c):
+    """A count that falls monotonically in α: outliers are |x| > α·c."""
+    return lambda a: {"mask": np.abs(x) > float(a) * c}
+
+
+@pytest.mark.parametrize("n_max", [0, 3, 17, 60])
+def test_bisection_finds_a_known_threshold(n_max):
+    """count(α) = #{|x_i| > α·c}: the smallest admissible α is v/c with v the
+    (n_max+1)-th largest |x_i|; the search ends within its bracket's last
+    width above it, and its last rejected α is below it."""
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal(200)
+    c = 4.0
+    v = np.sort(np.abs(x))[::-1][n_max]
+    a_star = v / c
+    iters = 20
+    alpha, res, trace = S.bisect_alpha(_threshold_run(x, c), n_max, iters, 1.0 / 16, 1.0)
+    assert S.count(res) <= n_max
+    assert alpha >= a_star
+    assert alpha - a_star <= (1.0 - 1.0 / 16) / 2 ** iters + 1e-7
+    rejected = [a for a, k in trace if k > n_max]
+    assert rejected and max(rejected) < a_star
+
+
+def test_bisection_stops_at_the_upper_end_when_it_is_over_budget():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(50)
+    alpha, res, trace = S.bisect_alpha(_threshold_run(x, 0.1), 0, 16, 0.25, 1.0)
+    assert alpha == np.float32(1.0) and len(trace) == 1 and S.count(res) > 0
+
+
+def test_bisection_with_an_unlimited_budget_reaches_the_lower_end():
+    x = np.ones(10)
+    alpha, _, trace = S.bisect_alpha(_threshold_run(x, 1.0), 10, 12, 0.25, 1.0)
+    assert alpha == np.float32(0.25 + 0.75 / 2 ** 12)
+    assert len(trace) == 13 and all(k <= 10 for _, k in trace)
+
+
+def test_max_outliers_is_the_floor():
+    assert S.max_outliers(0.01, 576, 576) == 3317
+    assert S.max_outliers(0.0, 10, 10) == 0
+    assert S.max_outliers(1.0, 7, 3) == 21
+
+
+# ---------------------------------------------------------------- the layer
+
+def test_layer_outputs_are_consistent():
+    rng = np.random.default_rng(8)
+    n, m, T = 96, 40, 256
+    X = rng.standard_normal((T, n)) * np.linspace(2.0, 0.3, n)
+    H = G.hessian(X)
+    W = _heavy(m, n, rng)
+    out = S.ssqr_layer(W, H, bits=3, group=32, block=64, target=0.02, iters=12)
+    assert out["count"] <= S.max_outliers(0.02, m, n)
+    assert out["alpha"] < 1.0
+    # the outlier list is the mask, row-major, with the kept values
+    r, c = np.nonzero(out["mask"])
+    assert np.array_equal(r, out["outlier_rows"]) and np.array_equal(c, out["outlier_cols"])
+    assert np.array_equal(out["Q"][r, c], out["outlier_vals"])
+    # inliers dequantize with their group's adjusted scale
+    g = out["g_idx"]
+    inl = ~out["mask"]
+    deq = out["scale"][:, g] * (out["codes"] - out["zero"][:, g].astype(np.float64))
+    assert np.allclose(out["Q"][inl], deq[inl], rtol=0, atol=1e-15)
+    assert 0 <= out["codes"].min() and out["codes"].max() <= 7
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_ssqr_beats_gptq_on_heavy_tailed_layers(seed):
+    """Observed on seeded layers, not a theorem: at 3 bits with 1 % outliers
+    kept, the layer loss falls below GPTQ's with clipping (the page reports
+    SSQR ahead of GPTQ in the 2–4-bit range)."""
+    rng = np.random.default_rng(10 + seed)
+    n, m, T = 128, 64, 512
+    X = rng.standard_normal((T, n)) * np.linspace(2.0, 0.3, n) + 0.3 * rng.standard_normal((T, 1))
+    H = G.hessian(X)
+    W = _heavy(m, n, rng)
+    g = G.gptq_layer(W, H, 3, 64, 64, 0.01, "act")
+    s = S.ssqr_layer(W, H, bits=3, group=64, block=64, target=0.01, iters=14)
+    assert s["loss"] < g["loss"]
+
+
+def test_follow_accepts_its_own_decisions_and_flags_a_planted_one():
+    rng = np.random.default_rng(9)
+    n = 64
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(30, n, rng)[:, p["perm"]]
+    ref = S.ssqr_blocked(Wp, p["U"], 3, 32, 64, 0.5)
+    args = (Wp, p["U"], 3, 32, 64, 0.5)
+    ok = S.follow_ssqr(*args, ref["codes"], ref["mask"], ref["value"], ref["scale"], ref["zero"])
+    assert ok["n_diff"] == 0 and ok["n_bad"] == 0 and ok["max_scale_rel"] == 0.0
+    assert ok["max_val_rel"] == 0.0 and np.allclose(ok["err"], ref["err"], atol=1e-15)
+    # an outlier flag dropped far from any rounding boundary
+    frac = np.abs(ref["pre"] - np.floor(ref["pre"]) - 0.5)
+    cand = np.argwhere(ref["mask"] & (frac > 0.1))
+    r, j = cand[0]
+    mask = ref["mask"].copy()
+    mask[r, j] = False
+    bad = S.follow_ssqr(*args, ref["codes"], mask, ref["value"], ref["scale"], ref["zero"])
+    assert bad["n_bad"] >= 1
+
+
+# ---------------------------------------------------------------- mutations
+
+def _mutant_adjusted(kind):
+    orig = S.adjusted_params
+
+    def f(cur, bits, alpha):
+        s, z, s0 = orig(cur, bits, alpha)
+        if kind == "zero_from_adjusted_scale":
+            v = np.asarray(cur, np.float32)
+            xmin = np.minimum(v.min(axis=1), np.float32(0))
+            z = np.rint(-xmin / s).astype(np.float32)
+        elif kind == "scale_not_adjusted":
+            s = s0
+        return s, z, s0
+    return f
+
+
+def _mutant_column(kind):
+    def col(W, j, s, z, bits, U, out):
+        out["pre"][:, j] = W[:, j] / s.astype(np.float64)
+        q, o = S.quantize_column_outliers(W[:, j], s, z, bits)
+        qhat = G.dequantize(q, s, z)
+        if kind == "outlier_error_kept":
+            pass                                  # clipped error still propagates
+        elif kind == "outlier_wrong_side":
+            o = q >= 2 ** bits - 1                # the flag tested on the clipped code
+            qhat = np.where(o, W[:, j], qhat)
+        else:
+            qhat = np.where(o, W[:, j], qhat)
+        e = (W[:, j] - qhat) / U[j, j]
+        if kind == "error_sign":
+            e = -e
+        out["codes"][:, j] = q.astype(np.int64)
+        out["mask"][:, j] = o
+        out["value"][:, j] = np.where(o, W[:, j], 0.0)
+        out["err"][:, j] = e
+        return e
+    return col
+
+
+@pytest.mark.parametrize("kind", ["zero_from_adjusted_scale", "scale_not_adjusted",
+                                  "outlier_error_kept", "outlier_wrong_side", "error_sign"])
+def test_pins_catch_planted_mistakes(kind, monkeypatch):
+    if kind in ("zero_from_adjusted_scale", "scale_not_adjusted"):
+        monkeypatch.setattr(S, "adjusted_params", _mutant_adjusted(kind))
+    else:
+        monkeypatch.setattr(S, "_column", _mutant_column(kind))
+    rng = np.random.default_rng(11)
+    failures = 0
+    # pin 1: U = I against the scalar loops
+    W = _heavy(9, 64, rng)
+    res = S.ssqr_blocked(W, np.eye(64), 3, 16, 32, 0.5)
+    codes, mask = _rtn_with_outliers_by_loops(W, 3, 16, 0.5)
+    failures += not (np.array_equal(res["mask"], mask) and np.array_equal(res["codes"], codes))
+    # pins 2 and 3: the Satz 5 bound and the loss identity on a real factor
+    n = 64
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(25, n, rng)[:, p["perm"]]
+    res = S.ssqr_blocked(Wp, p["U"], 2, 16, 32, 0.6)
+    failures += not _satz5_holds(res, p["U"], 16)
+    failures += not _loss_identity_holds(Wp, res, p["Hp"], 16)
+    assert failures >= 1, kind
