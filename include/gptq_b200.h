@@ -49,7 +49,8 @@ typedef enum {
   GPTQ_ERR_NONFINITE = 3,    /* NaN or Inf in H or W                         */
   GPTQ_ERR_UNSUPPORTED = 4,  /* bits/group/block combination not implemented */
   GPTQ_ERR_TIMEOUT = 5,      /* a bounded device wait ran out                */
-  GPTQ_ERR_CUDA = 6          /* a CUDA runtime call failed                   */
+  GPTQ_ERR_CUDA = 6,         /* a CUDA runtime call failed                   */
+  GPTQ_ERR_CAPACITY = 7      /* more results than the caller's buffer holds  */
 } gptq_status;
 
 typedef enum {
@@ -272,6 +273,66 @@ gptq_status gptq_quantize_rowgroups(const void* W, int w_dtype, int64_t m, int64
                                     uint32_t* qweight, float* scale, uint8_t* zero,
                                     float* loss_row, float* Qdq, int32_t* info, void* ws,
                                     size_t ws_bytes, void* stream);
+
+/* ---- SSQR (next to the hot path) ----------------------------------------
+ * "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+ * Algorithm" (gist.science summary), §3: scale-adjusted SpQR keeps the
+ * weights that overflow the grid (the outliers) in full precision as a sparse
+ * part and quantizes the rest (the inliers) with GPTQ; a binary search on the
+ * scales meets a target outlier density.  §2.3: clipping those weights would
+ * break Satz 5's error bound.
+ */
+
+/* Bytes of device workspace gptq_ssqr_quantize needs (256-byte aligned). */
+size_t gptq_ssqr_workspace_bytes(int64_t m, int64_t n, int block);
+
+/*
+ * As gptq_quantize (W, U, perm, dead, group, block, qweight, scale, zero,
+ * g_idx, loss_row, Qdq, info have the same meaning), except:
+ *   bits       2, 3 or 4.
+ *   Scales     the min-max step s0 of each group (taken where gptq_quantize
+ *              takes it) becomes s = alpha·s0 (float32); the zero point stays
+ *              rint(−xmin/s0).  `scale` holds s.
+ *   Outliers   a weight whose unclipped code rint(w/s) + z falls outside
+ *              [0, 2^bits − 1] keeps its current (error-updated) value: its
+ *              error is 0 and nothing propagates from it.  Its code in
+ *              qweight is the clipped one; dequantization uses the value.
+ *   Search     (all on the device, no host synchronisation):
+ *              n_max = floor(target·m·n).  Pass 0 runs at alpha_hi; more than
+ *              n_max outliers there ends the search with alpha = alpha_hi.
+ *              Otherwise each of up to `iters` passes runs at
+ *              mid = float32((lo + hi)/2) of the bracket [alpha_lo, alpha_hi]
+ *              and makes mid the new hi when it has at most n_max outliers,
+ *              else the new lo; a mid equal to lo or hi ends the search.  A
+ *              last pass at hi writes the outputs.  Cost: iters + 2 sweeps of
+ *              the layer.
+ *   target     outlier density, 0..1.  iters 0..64.
+ *   alpha_lo, alpha_hi   the bracket, 0 < alpha_lo ≤ alpha_hi ≤ 16.
+ *   row_ptr    int64[m + 1], output: CSR row pointers of the outliers
+ *              (row_ptr[m] = their number).
+ *   col_idx, val  int32 / float32 [nnz_cap], output: ORIGINAL column and
+ *              kept value of each outlier, row-major, columns ascending.
+ *              Entries beyond nnz_cap are dropped and info reports
+ *              GPTQ_ERR_CAPACITY (row_ptr stays complete).  May be NULL when
+ *              nnz_cap == 0.
+ *   alpha      float32[1], output: the chosen factor.
+ *   trace_alpha, trace_count   float32 / int64 [iters + 1] or NULL: the α of
+ *              each search pass and its outlier count (−1 for a pass run
+ *              after the search had ended).
+ *   ws         device workspace of at least gptq_ssqr_workspace_bytes().
+ * Errors: INVALID_ARG (null pointer, target, iters, bracket, nnz_cap < 0,
+ * workspace), UNSUPPORTED (bits, group, block), CUDA; NONFINITE and CAPACITY
+ * through info.
+ */
+gptq_status gptq_ssqr_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
+                               const float* U, const int32_t* perm, const uint8_t* dead,
+                               int bits, int group, int block, double target, int iters,
+                               float alpha_lo, float alpha_hi, uint32_t* qweight,
+                               float* scale, uint8_t* zero, int32_t* g_idx,
+                               int64_t* row_ptr, int32_t* col_idx, float* val,
+                               int64_t nnz_cap, float* alpha, float* trace_alpha,
+                               int64_t* trace_count, float* loss_row, float* Qdq,
+                               int32_t* info, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Synchronize `stream`, read info[0..1] and return info[0] (a gptq_status).

@@ -455,6 +455,10 @@ def follow(Wp, U, bits: int, group: int, block: int, codes_p, scale, zero,
                 z_diff += int(zd.sum())
                 near_z = np.abs(zpre - np.floor(zpre) - 0.5) <= tol
                 z_bad += int((zd & ~near_z).sum())
+                # a zero point flipped at a near-tie shifts the group's codes by
+                # one: decide this group's codes with the other side's zero, so
+                # that the one allowed flip does not count once per column
+                z_o = np.where(zd & near_z, z_g, z_o).astype(np.float32)
             x = W[:, j] / s_o.astype(np.float64)
             q_o = quantize_column(W[:, j], s_o, z_o, bits).astype(np.int64)
             q_g = codes_p[:, j]

@@ -184,7 +184,7 @@ def ssqr_layer(W, H, bits: int = 3, group: int = 128, block: int = 128, damp: fl
 
 
 def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p, vals_p,
-                scale, zero, tol: float = 1e-4) -> dict:
+                scale, zero, tol: float = 1e-4, scale_rtol: float = 1e-5) -> dict:
     """Walk the SSQR sweep with another implementation's decisions.
 
     At each column the oracle forms its own current values (float64, from the
@@ -195,6 +195,16 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
     side's decision: an outlier contributes no error.  ``vals_p`` holds the
     other side's stored outlier values; their largest deviation from the
     oracle's current value is reported relative to |w| + s₀·(2^b − 1).
+
+    Scales: ``scale_rtol`` relative, or, where the group's own float32
+    working precision is coarser, the forward-error bound of the float32
+    propagation that built its current values: |Δs| ≤ 2·γ_K·M/(2^b − 1)·α
+    with M the largest |w| + Σ|e_k·U_kj| over the group at its start, K the
+    columns processed before it and γ_K = 2⁻²¹ + K·2⁻²⁴ (a three-term TF32
+    product and K float32 additions).  ``scale_bad`` counts groups beyond both;
+    ``scale_wide_over`` counts groups of at least 32 columns beyond
+    ``scale_rtol`` alone.  Kept values likewise: ``val_bad`` counts those off
+    by more than both 1e-5·(|w| + s₀·(2^b − 1)) and γ_j·M_j (j their column).
 
     Arrays in processing order: codes_p, mask_p, vals_p (m × n); scale and
     zero (m × ngroups).
@@ -207,9 +217,11 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
     scale = np.asarray(scale, dtype=np.float32)
     zero = np.asarray(zero, dtype=np.float32)
     maxq = 2 ** bits - 1
-    n_diff = n_bad = z_bad = 0
+    n_diff = n_bad = z_bad = scale_bad = scale_wide_over = val_bad = 0
     max_scale_rel = max_val_rel = 0.0
+    worst = None
     err = np.zeros((m, n))
+    mag = np.abs(W)                   # |w| + Σ|e_k·U_kj| of the updates so far
     s_o = z_o = s0 = None
     for b0 in range(0, n, block):
         b1 = min(b0 + block, n)
@@ -221,9 +233,25 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
                 c32 = np.asarray(cur, np.float32)
                 zpre = -np.minimum(c32.min(axis=1), 0).astype(np.float64) / s0.astype(np.float64)
                 rel = np.abs(scale[:, g].astype(np.float64) - s_o) / np.abs(s_o)
+                width = cur.shape[1]
+                M = mag[:, j:j + width].max(axis=1)
+                gam = 2.0 ** -21 + j * 2.0 ** -24
+                bound = 2.0 * gam * M / maxq * float(alpha) / np.abs(s_o)
+                scale_bad += int(np.sum(rel > np.maximum(scale_rtol, bound)))
+                if width >= 32:
+                    scale_wide_over += int(np.sum(rel > scale_rtol))
+                if float(rel.max()) > max_scale_rel:
+                    r = int(np.argmax(rel))
+                    rng = float(s0[r]) * maxq
+                    worst = {"row": r, "group": g, "cols": cur.shape[1],
+                             "mag_over_range": float(mag[r, j:j + cur.shape[1]].max()) / rng}
                 max_scale_rel = max(max_scale_rel, float(rel.max()))
                 zd = zero[:, g] != z_o
-                z_bad += int((zd & ~(np.abs(zpre - np.floor(zpre) - 0.5) <= tol)).sum())
+                near_z = np.abs(zpre - np.floor(zpre) - 0.5) <= tol
+                z_bad += int((zd & ~near_z).sum())
+                # a zero point flipped at a near-tie shifts the group's codes by
+                # one: decide this group's codes with the other side's zero
+                z_o = np.where(zd & near_z, zero[:, g], z_o).astype(np.float32)
             s_g, z_g = scale[:, g], zero[:, g]
             x = W[:, j] / s_o.astype(np.float64)
             q_o, o_o = quantize_column_outliers(W[:, j], s_o, z_o, bits)
@@ -238,12 +266,19 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
                 v = np.asarray(vals_p[:, j], np.float64)[o_g]
                 ref = W[o_g, j]
                 den = np.abs(ref) + s0[o_g].astype(np.float64) * maxq
-                max_val_rel = max(max_val_rel, float(np.max(np.abs(v - ref) / den)))
+                dv = np.abs(v - ref)
+                max_val_rel = max(max_val_rel, float(np.max(dv / den)))
+                gam = 2.0 ** -21 + j * 2.0 ** -24
+                val_bad += int(np.sum(dv > np.maximum(1e-5 * den, gam * mag[o_g, j])))
             qhat = np.where(o_g, W[:, j], G.dequantize(q_g, s_g, z_g))
             e = (W[:, j] - qhat) / U[j, j]
             W[:, j + 1:b1] -= np.outer(e, U[j, j + 1:b1])
+            mag[:, j + 1:b1] += np.outer(np.abs(e), np.abs(U[j, j + 1:b1]))
             err[:, j] = e
         if b1 < n:
             W[:, b1:] -= err[:, b0:b1] @ U[b0:b1, b1:]
+            mag[:, b1:] += np.abs(err[:, b0:b1]) @ np.abs(U[b0:b1, b1:])
     return {"n_diff": n_diff, "n_bad": n_bad, "z_bad": z_bad, "max_scale_rel": max_scale_rel,
-            "max_val_rel": max_val_rel, "err": err, "count": int(mask_p.sum())}
+            "scale_bad": scale_bad, "scale_wide_over": scale_wide_over, "worst_scale": worst,
+            "val_bad": val_bad, "max_val_rel": max_val_rel, "err": err,
+            "count": int(mask_p.sum())}

@@ -15,7 +15,7 @@ from ._binding import (DTYPES, ORDERS, GptqError, exported_symbols,
                        gptq_launch_count, gptq_prepare, gptq_prepare_workspace_bytes,
                        gptq_profile_start, gptq_profile_stop, gptq_quantize,
                        gptq_quantize_rowgroups, gptq_quantize_workspace_bytes,
-                       kernel_names, lib)
+                       gptq_ssqr_quantize, gptq_ssqr_workspace_bytes, kernel_names, lib)
 
 __all__ = [
     "GptqError", "ORDERS", "DTYPES", "lib", "exported_symbols", "kernel_names",
@@ -23,9 +23,9 @@ __all__ = [
     "gptq_prepare_workspace_bytes", "gptq_quantize_workspace_bytes",
     "gptq_launch_count", "gptq_profile_start", "gptq_profile_stop",
     "gptq_quantize_rowgroups", "gptq_chmc_rank", "gptq_chmc_workspace_bytes",
-    "gptq_chmc_lowrank",
+    "gptq_chmc_lowrank", "gptq_ssqr_quantize", "gptq_ssqr_workspace_bytes",
     "hessian", "prepare", "quantize", "workspace",
-    "chmc_lowrank", "quantize_rowgroups", "chmc_layer",
+    "chmc_lowrank", "quantize_rowgroups", "chmc_layer", "ssqr_quantize",
 ]
 
 
@@ -163,3 +163,51 @@ def chmc_layer(W: torch.Tensor, H: torch.Tensor, tokens: int, Omega: torch.Tenso
     prep = prepare(H, damp, order, stream=stream)
     q = quantize_rowgroups(lr["R"], prep, bits, gs, block, want_qdq=True, stream=stream)
     return {"rank": r, **lr, **{"prep_" + k: v for k, v in prep.items()}, **q}
+
+
+# ---- SSQR ("The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+# Algorithm", §3)
+
+def ssqr_quantize(W: torch.Tensor, prep: dict, bits: int = 3, group: int = 128,
+                  block: int = 128, target: float = 0.01, iters: int = 16,
+                  alpha_lo: float = 1.0 / 16, alpha_hi: float = 1.0, nnz_cap: int | None = None,
+                  want_loss: bool = True, want_qdq: bool = False, want_trace: bool = False,
+                  ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+    """GPTQ with the overflowing weights kept: packed inlier codes, scales,
+    zeros, g_idx and the outliers in CSR (row_ptr, col_idx, val, original
+    columns).  ``nnz_cap`` (default floor(target·m·n), at least 1) sizes the
+    CSR arrays; with ``check`` the arrays are trimmed to the outlier count."""
+    m, n = W.shape
+    dev = W.device
+    ng = -(-n // group)
+    nwords = -(-n * bits // 32)
+    if nnz_cap is None:
+        nnz_cap = max(int(target * m * n), 1)
+    out = {
+        "qweight": torch.empty(m, nwords, dtype=torch.int32, device=dev),
+        "scale": torch.empty(m, ng, dtype=torch.float32, device=dev),
+        "zero": torch.empty(m, ng, dtype=torch.uint8, device=dev),
+        "g_idx": torch.empty(n, dtype=torch.int32, device=dev),
+        "row_ptr": torch.empty(m + 1, dtype=torch.int64, device=dev),
+        "col_idx": torch.empty(nnz_cap, dtype=torch.int32, device=dev),
+        "val": torch.empty(nnz_cap, dtype=torch.float32, device=dev),
+        "alpha": torch.empty(1, dtype=torch.float32, device=dev),
+        "trace_alpha": torch.empty(iters + 1, dtype=torch.float32, device=dev) if want_trace else None,
+        "trace_count": torch.empty(iters + 1, dtype=torch.int64, device=dev) if want_trace else None,
+        "loss_row": torch.empty(m, dtype=torch.float32, device=dev) if want_loss else None,
+        "Qdq": torch.empty(m, n, dtype=torch.float32, device=dev) if want_qdq else None,
+        "info": torch.zeros(2, dtype=torch.int32, device=dev),
+    }
+    if ws is None:
+        ws = workspace(gptq_ssqr_workspace_bytes(m, n, block), dev)
+    gptq_ssqr_quantize(W, prep["U"], prep["perm"], prep["dead"], bits, group, block, target,
+                       iters, alpha_lo, alpha_hi, out["qweight"], out["scale"], out["zero"],
+                       out["g_idx"], out["row_ptr"], out["col_idx"], out["val"], out["alpha"],
+                       out["trace_alpha"], out["trace_count"], out["loss_row"], out["Qdq"],
+                       out["info"], ws, stream)
+    if check:
+        _raise_info(out["info"], stream, "gptq_ssqr_quantize")
+        nnz = int(out["row_ptr"][-1])
+        out["col_idx"] = out["col_idx"][:nnz]
+        out["val"] = out["val"][:nnz]
+    return out

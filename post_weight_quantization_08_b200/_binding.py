@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libgptq_b200.so")
 
 STATUS = {0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_NOT_PD",
           3: "GPTQ_ERR_NONFINITE", 4: "GPTQ_ERR_UNSUPPORTED",
-          5: "GPTQ_ERR_TIMEOUT", 6: "GPTQ_ERR_CUDA"}
+          5: "GPTQ_ERR_TIMEOUT", 6: "GPTQ_ERR_CUDA", 7: "GPTQ_ERR_CAPACITY"}
 ORDERS = {"natural": 0, "act": 1, "reverse": 2, "custom": 3, "minpivot": 4}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
@@ -50,6 +50,15 @@ _SIGS = {
                                     C.c_int64, C.c_double, C.c_void_p, C.c_int, C.c_int,
                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                     C.c_void_p, C.c_size_t, C.c_void_p]),
+    "gptq_ssqr_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int]),
+    "gptq_ssqr_quantize": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
+                                     C.c_double, C.c_int, C.c_float, C.c_float,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
+                                     C.c_void_p]),
     "gptq_check": (C.c_int, [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]),
     "gptq_last_error": (C.c_char_p, []),
     "gptq_status_string": (C.c_char_p, [C.c_int]),
@@ -217,6 +226,53 @@ def gptq_quantize_rowgroups(W, U, perm, dead, bits, gs, block, qweight, scale, z
                                          _ptr(qweight), _ptr(scale), _ptr(zero),
                                          _ptr(loss_row), _ptr(Qdq), _ptr(info), _ptr(ws),
                                          ws.numel(), _stream(stream, dev)))
+
+
+def gptq_ssqr_workspace_bytes(m: int, n: int, block: int) -> int:
+    return int(lib().gptq_ssqr_workspace_bytes(m, n, block))
+
+
+def gptq_ssqr_quantize(W, U, perm, dead, bits, group, block, target, iters, alpha_lo,
+                       alpha_hi, qweight, scale, zero, g_idx, row_ptr, col_idx, val, alpha,
+                       trace_alpha, trace_count, loss_row, Qdq, info, ws, stream=None):
+    """SSQR: GPTQ with kept outliers and a binary search on the scale factor
+    (see include/gptq_b200.h)."""
+    if W.dtype not in DTYPES:
+        raise TypeError("W must be float32 or bfloat16")
+    _need(W, "W", W.dtype)
+    m, n = W.shape
+    dev = W.device
+    ng = -(-n // group)
+    nwords = -(-n * bits // 32)
+    _need(U, "U", torch.float32, (n, n), dev)
+    _need(perm, "perm", torch.int32, (n,), dev)
+    _need(dead, "dead", torch.uint8, (n,), dev)
+    _need(qweight, "qweight", torch.int32, (m, nwords), dev)
+    _need(scale, "scale", torch.float32, (m, ng), dev)
+    _need(zero, "zero", torch.uint8, (m, ng), dev)
+    _need(g_idx, "g_idx", torch.int32, (n,), dev)
+    _need(row_ptr, "row_ptr", torch.int64, (m + 1,), dev)
+    cap = 0 if col_idx is None else col_idx.numel()
+    if cap:
+        _need(col_idx, "col_idx", torch.int32, (cap,), dev)
+        _need(val, "val", torch.float32, (cap,), dev)
+    _need(alpha, "alpha", torch.float32, (1,), dev)
+    if trace_alpha is not None:
+        _need(trace_alpha, "trace_alpha", torch.float32, (iters + 1,), dev)
+        _need(trace_count, "trace_count", torch.int64, (iters + 1,), dev)
+    if loss_row is not None:
+        _need(loss_row, "loss_row", torch.float32, (m,), dev)
+    if Qdq is not None:
+        _need(Qdq, "Qdq", torch.float32, (m, n), dev)
+    _need(info, "info", torch.int32, (2,), dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _raise(lib().gptq_ssqr_quantize(
+        _ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm), _ptr(dead), int(bits),
+        int(group), int(block), float(target), int(iters), float(alpha_lo), float(alpha_hi),
+        _ptr(qweight), _ptr(scale), _ptr(zero), _ptr(g_idx), _ptr(row_ptr),
+        _ptr(col_idx) if cap else None, _ptr(val) if cap else None, cap, _ptr(alpha),
+        _ptr(trace_alpha), _ptr(trace_count), _ptr(loss_row), _ptr(Qdq), _ptr(info),
+        _ptr(ws), ws.numel(), _stream(stream, dev)))
 
 
 def gptq_chmc_rank(o: int, i: int, bits: int = 4, gs: int = 128,

@@ -23,6 +23,7 @@ enum KernelKind : int {
   KK_TRAIL,           // TF32 split of U, or the SIMT lazy-batch trailing update
   KK_PACK,            // codes → packed words, g_idx, dequantized copy
   KK_CHMC,            // CHMC frontend: activation energies, randomized subspace iteration, residual
+  KK_SSQR,            // SSQR: the binary search's state, the outlier list
   KK_COUNT
 };
 

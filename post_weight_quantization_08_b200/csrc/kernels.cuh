@@ -60,12 +60,66 @@ struct SweepFar {
   int64_t k0 = 0;               // first column of the block whose errors they are
   int kw = 0;                   // its width, 0 for none
 };
+//
+// outl != NULL (SSQR): every group's step is multiplied by *outl->alpha (a
+// device float, read when the launch starts; the zero point stays that of the
+// min-max step).  A weight whose unclipped code falls outside [0, 2^bits − 1]
+// is an outlier: its error is 0, its code byte carries OUTLIER_FLAG on top of
+// the clipped code, its current value is written to Wp at its own position,
+// and it is counted in outl->row_cnt[row] and *outl->total.  bits ≤ 7.
+constexpr uint8_t OUTLIER_FLAG = 0x80;
+struct OutlierArgs {
+  const float* alpha = nullptr;
+  int32_t* row_cnt = nullptr;          // m counts, accumulated over the blocks
+  unsigned long long* total = nullptr; // all outliers of the pass
+};
 gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
                          float* Elo, const SweepPrologue& pre, const SweepFar& far,
                          float* loss_row, int32_t* info, const int32_t* rowgroup_perm,
-                         cudaStream_t s);
+                         const OutlierArgs* outl, cudaStream_t s);
+
+// ---- the stages of gptq_quantize, shared with the SSQR entry point
+
+struct QuantWs {
+  float* Wp;        // error_rows(m) × n working copy, processing order
+  uint8_t* codes;   // m × n codes, processing order
+  float* Ehi[2];    // error_rows(m) × 128 scaled errors of a block, TF32 part
+  float* Elo[2];    // remainder e − Ehi; two sets, alternating by block
+  int32_t* pinv;    // n: processing position of each original column
+  float* panels;    // pre-transposed U panels, one per block
+  float* Uhi;       // n × n TF32 part of Uᵀ (tensor-core trailing update only)
+  float* Ulo;       // n × n remainder, transposed likewise
+};
+// Bytes of the layout (256-byte aligned parts); fills *w when both are given.
+size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base);
+
+// Host checks shared by the quantize entry points (no device work).
+gptq_status quant_check_args(int w_dtype, int64_t m, int64_t n, int bits, int group,
+                             int block, const void* ws, size_t ws_bytes, size_t need);
+
+// Once per call: info and pinv reset, pinv/g_idx, the panels and the TF32
+// split of U.
+gptq_status quant_setup(const QuantWs& w, int64_t m, int64_t n, const float* U,
+                        const int32_t* perm, int group, int block, int32_t* g_idx,
+                        int32_t* info, cudaStream_t s);
+
+// One pass of the column sweep over the whole layer: W → Wp (processing
+// order, dead columns zeroed), then the block loop of sweeps and trailing
+// updates.  rowgs > 0: output-channel groups (rowgroup mode).
+gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, int64_t n,
+                       const float* U, const int32_t* perm, const uint8_t* dead, int bits,
+                       int group, int block, int rowgs, float* scale, uint8_t* zero,
+                       float* loss_row, const OutlierArgs* outl, int32_t* info,
+                       cudaStream_t s);
+
+// Codes → packed words in original column order, and the optional
+// dequantized copy.  outl_vals != NULL: code bytes carry OUTLIER_FLAG, and the
+// dequantized value of a flagged weight is outl_vals at its processing position.
+gptq_status quant_pack(const QuantWs& w, int64_t m, int64_t n, int bits, int group, int rowgs,
+                       const float* scale, const uint8_t* zero, uint32_t* qweight,
+                       float* Qdq, const float* outl_vals, int32_t* info, cudaStream_t s);
 
 // Whether the trailing update runs on the tensor cores for this shape.
 bool trailing_uses_tensor_cores(int64_t n, int block);

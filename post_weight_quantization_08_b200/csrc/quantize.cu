@@ -14,18 +14,6 @@
 #include "kernels.cuh"
 
 namespace gptq {
-namespace {
-
-struct QuantWs {
-  float* Wp;        // error_rows(m) × n working copy, processing order
-  uint8_t* codes;   // m × n codes, processing order
-  float* Ehi[2];    // error_rows(m) × 128 scaled errors of a block, TF32 part
-  float* Elo[2];    // remainder e − Ehi; two sets, alternating by block
-  int32_t* pinv;    // n: processing position of each original column
-  float* panels;    // pre-transposed U panels, one per block
-  float* Uhi;       // n × n TF32 part of Uᵀ (tensor-core trailing update only)
-  float* Ulo;       // n × n remainder, transposed likewise
-};
 
 size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) {
   size_t off = 0;
@@ -60,6 +48,8 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   }
   return off;
 }
+
+namespace {
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -130,7 +120,7 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
             const int32_t* __restrict__ pinv, int group, int64_t ngroups, int rowgs,
             const float* __restrict__ scale, const uint8_t* __restrict__ zero,
             uint32_t* __restrict__ qweight, int64_t nwords,
-            float* __restrict__ Qdq, int32_t* info) {
+            float* __restrict__ Qdq, const float* __restrict__ outv, int32_t* info) {
   const int64_t chunks = (n + 31) / 32;
   const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (e >= m * chunks) return;
@@ -148,11 +138,16 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
         report(info, GPTQ_ERR_INVALID_ARG, c);
       } else {
         q = codes[r * n + p];
+        bool kept = false;                 // an SSQR outlier: its value, not its code
+        if (outv != nullptr) {
+          kept = (q & OUTLIER_FLAG) != 0;
+          q &= ~(uint32_t)OUTLIER_FLAG;
+        }
         if (Qdq != nullptr) {
           // input-channel groups: [row][group of processing position p];
           // output-channel groups (rowgs rows): [row group][original column c]
           const int64_t sx = rowgs > 0 ? (r / rowgs) * n + c : r * ngroups + p / group;
-          Qdq[r * n + c] = scale[sx] * ((float)q - (float)zero[sx]);
+          Qdq[r * n + c] = kept ? outv[r * n + p] : scale[sx] * ((float)q - (float)zero[sx]);
         }
       }
       const int off = k * BITS, wi = off >> 5, sh = off & 31;
@@ -168,29 +163,9 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
 }
 
 }  // namespace
-}  // namespace gptq
 
-using namespace gptq;
-
-extern "C" size_t gptq_quantize_workspace_bytes(int64_t m, int64_t n, int block) {
-  if (m < 1 || n < 1 || block < 1) return 0;
-  return quant_ws_layout(m, n, block, nullptr, nullptr);
-}
-
-namespace gptq {
-namespace {
-
-// The quantize path of gptq_quantize (rowgs = 0: scale groups of `group`
-// columns) and gptq_quantize_rowgroups (rowgs = 128: scale groups of the
-// rows, per column).
-gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, const float* U,
-                          const int32_t* perm, const uint8_t* dead, int bits, int group,
-                          int block, int rowgs, uint32_t* qweight, float* scale, uint8_t* zero,
-                          int32_t* g_idx, float* loss_row, float* Qdq, int32_t* info, void* ws,
-                          size_t ws_bytes, void* stream) {
-  if (!W || !U || !perm || !dead || !qweight || !scale || !zero || (!g_idx && rowgs == 0) ||
-      !info || !ws)
-    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: null pointer");
+gptq_status quant_check_args(int w_dtype, int64_t m, int64_t n, int bits, int group,
+                             int block, const void* ws, size_t ws_bytes, size_t need) {
   if (m < 1 || n < 1 || m > ((int64_t)1 << 31) || n > ((int64_t)1 << 20))
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: m=%lld n=%lld", (long long)m,
                 (long long)n);
@@ -204,22 +179,36 @@ gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, cons
                 "multiple of group, block <= 128)", group, block);
   if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0)
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: workspace not 256-byte aligned");
-  const size_t need = quant_ws_layout(m, n, block, nullptr, nullptr);
   if (ws_bytes < need)
-    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: workspace %zu < %zu bytes",
-                ws_bytes, need);
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: workspace %zu < %zu bytes", ws_bytes,
+                need);
+  return GPTQ_OK;
+}
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  QuantWs w;
-  quant_ws_layout(m, n, block, &w, static_cast<char*>(ws));
-  const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
-  const int64_t nwords = ceil_div(n * bits, 32);
-
+gptq_status quant_setup(const QuantWs& w, int64_t m, int64_t n, const float* U,
+                        const int32_t* perm, int group, int block, int32_t* g_idx,
+                        int32_t* info, cudaStream_t s) {
+  (void)m;
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
   GPTQ_CUDA(cudaMemsetAsync(w.pinv, 0xFF, sizeof(int32_t) * n, s));
-  if (loss_row) GPTQ_CUDA(cudaMemsetAsync(loss_row, 0, sizeof(float) * m, s));
   GPTQ_LAUNCH(KK_INGEST, s, pinv_kernel, (unsigned)ceil_div(n, 256), 256, 0, perm, n,
               group, w.pinv, g_idx, info);
+  gptq_status st = launch_panels(U, n, block, w.panels, s);
+  if (st != GPTQ_OK) return st;
+  if (w.Uhi != nullptr && n > block) {
+    st = launch_split_tf32_t(U, n, w.Uhi, w.Ulo, s);
+    if (st != GPTQ_OK) return st;
+  }
+  return GPTQ_OK;
+}
+
+gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, int64_t n,
+                       const float* U, const int32_t* perm, const uint8_t* dead, int bits,
+                       int group, int block, int rowgs, float* scale, uint8_t* zero,
+                       float* loss_row, const OutlierArgs* outl, int32_t* info,
+                       cudaStream_t s) {
+  const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
+  if (loss_row) GPTQ_CUDA(cudaMemsetAsync(loss_row, 0, sizeof(float) * m, s));
   const unsigned gin = (unsigned)ceil_div(m * n, 256);
   if (w_dtype == GPTQ_DTYPE_BF16)
     GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<__nv_bfloat16>, gin, 256, 0,
@@ -232,12 +221,6 @@ gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, cons
   // every sweep and trailing update reads defined values
   if (error_rows(m) > m)
     GPTQ_CUDA(cudaMemsetAsync(w.Wp + m * n, 0, sizeof(float) * (size_t)(error_rows(m) - m) * n, s));
-  gptq_status st = launch_panels(U, n, block, w.panels, s);
-  if (st != GPTQ_OK) return st;
-  if (w.Uhi != nullptr && n > block) {
-    st = launch_split_tf32_t(U, n, w.Uhi, w.Ulo, s);
-    if (st != GPTQ_OK) return st;
-  }
   // Block b's errors reach the later columns in two parts:
   //  * block b+1's columns: on the tensor-core path, sweep b+1 applies them
   //    itself in its prologue (in TMEM, before its first column); otherwise a
@@ -254,7 +237,7 @@ gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, cons
   const bool fused = w.Uhi != nullptr && trailing_uses_tensor_cores(n, block);
   SideStream* side = nullptr;
   if (!fused) {
-    st = side_stream_for(s, &side);
+    gptq_status st = side_stream_for(s, &side);
     if (st != GPTQ_OK) return st;
   }
   bool pending[2] = {false, false};
@@ -279,8 +262,9 @@ gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, cons
       far.c1 = n;
     }
     const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
-    st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes, scale,
-                      zero, ehi, elo, pre, far, loss_row, info, rowgs > 0 ? perm : nullptr, s);
+    gptq_status st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes,
+                                  scale, zero, ehi, elo, pre, far, loss_row, info,
+                                  rowgs > 0 ? perm : nullptr, outl, s);
     if (st != GPTQ_OK) return st;
     const int64_t c0 = j0 + bw, c1 = c0 + block;
     if (c0 >= n || fused) continue;
@@ -301,27 +285,71 @@ gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, cons
   }
   for (int p = 0; p < 2; ++p)
     if (pending[p]) GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[p], 0));
+  return GPTQ_OK;
+}
 
+gptq_status quant_pack(const QuantWs& w, int64_t m, int64_t n, int bits, int group, int rowgs,
+                       const float* scale, const uint8_t* zero, uint32_t* qweight,
+                       float* Qdq, const float* outl_vals, int32_t* info, cudaStream_t s) {
+  const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
+  const int64_t nwords = ceil_div(n * bits, 32);
   const unsigned gpk = (unsigned)ceil_div(m * ceil_div(n, 32), 256);
   switch (bits) {
     case 2:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
       break;
     case 3:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
       break;
     case 4:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
       break;
     default:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
       break;
   }
   return GPTQ_OK;
+}
+
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" size_t gptq_quantize_workspace_bytes(int64_t m, int64_t n, int block) {
+  if (m < 1 || n < 1 || block < 1) return 0;
+  return quant_ws_layout(m, n, block, nullptr, nullptr);
+}
+
+namespace gptq {
+namespace {
+
+// The quantize path of gptq_quantize (rowgs = 0: scale groups of `group`
+// columns) and gptq_quantize_rowgroups (rowgs = 128: scale groups of the
+// rows, per column).
+gptq_status quantize_impl(const void* W, int w_dtype, int64_t m, int64_t n, const float* U,
+                          const int32_t* perm, const uint8_t* dead, int bits, int group,
+                          int block, int rowgs, uint32_t* qweight, float* scale, uint8_t* zero,
+                          int32_t* g_idx, float* loss_row, float* Qdq, int32_t* info, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (!W || !U || !perm || !dead || !qweight || !scale || !zero || (!g_idx && rowgs == 0) ||
+      !info || !ws)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize: null pointer");
+  const size_t need = (m >= 1 && n >= 1 && block >= 1) ? quant_ws_layout(m, n, block, nullptr, nullptr) : 0;
+  gptq_status st = quant_check_args(w_dtype, m, n, bits, group, block, ws, ws_bytes, need);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  QuantWs w;
+  quant_ws_layout(m, n, block, &w, static_cast<char*>(ws));
+  st = quant_setup(w, m, n, U, perm, group, block, g_idx, info, s);
+  if (st != GPTQ_OK) return st;
+  st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, rowgs, scale, zero,
+                  loss_row, nullptr, info, s);
+  if (st != GPTQ_OK) return st;
+  return quant_pack(w, m, n, bits, group, rowgs, scale, zero, qweight, Qdq, nullptr, info, s);
 }
 
 }  // namespace

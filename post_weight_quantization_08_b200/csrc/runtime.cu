@@ -21,7 +21,7 @@ std::atomic<uint64_t> g_launches{0};
 const char* const kKindNames[KK_COUNT] = {
     "hessian",  "prep_stats", "prep_order", "prep_gather", "cholesky",
     "prep_out", "ingest",     "sweep",      "trailing",    "pack",
-    "chmc"};
+    "chmc",     "ssqr"};
 
 struct Profiler {
   std::mutex mu;
@@ -123,6 +123,7 @@ const char* gptq_status_string(int status) {
     case GPTQ_ERR_UNSUPPORTED: return "GPTQ_ERR_UNSUPPORTED";
     case GPTQ_ERR_TIMEOUT: return "GPTQ_ERR_TIMEOUT";
     case GPTQ_ERR_CUDA: return "GPTQ_ERR_CUDA";
+    case GPTQ_ERR_CAPACITY: return "GPTQ_ERR_CAPACITY";
     default: return "GPTQ_ERR_UNKNOWN";
   }
 }
@@ -140,7 +141,7 @@ gptq_status gptq_check(const int32_t* info, int32_t* index, void* stream) {
   int32_t h[2] = {0, 0};
   GPTQ_CUDA(cudaMemcpy(h, info, sizeof(h), cudaMemcpyDeviceToHost));
   if (index) *index = h[1];
-  if (h[0] < 0 || h[0] > GPTQ_ERR_CUDA)
+  if (h[0] < 0 || h[0] > GPTQ_ERR_CAPACITY)
     return fail(GPTQ_ERR_CUDA, "gptq_check: corrupt info word %d", h[0]);
   return static_cast<gptq_status>(h[0]);
 }

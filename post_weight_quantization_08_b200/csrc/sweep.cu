@@ -167,15 +167,20 @@ __device__ __forceinline__ int ord_key_inv(int k) { return k ^ ((k >> 31) & 0x7f
 // 2 and 3: ⌈o/gs⌉·i scales, gs = 128 rows, the CTA's own rows): each column's
 // scale and zero come from the column's current values over the CTA's rows,
 // and are stored at [bx][perm[j0 + c]] (row group × original column).
-template <bool ROWG>
+// OUTL (SSQR, "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+// Algorithm", §3): the group's step is α·s₀ with the zero point of s₀; a
+// weight whose unclipped code leaves the grid is an outlier: it keeps its
+// current value (written to Wp at its own position, the strip being loaded
+// already), contributes no error, and its code byte carries OUTLIER_FLAG.
+template <bool ROWG, bool OUTL>
 __device__ __forceinline__ void sweep_body(
     const CUtensorMap& tmEhi, const CUtensorMap& tmElo, const CUtensorMap& tmW, int strip_tma,
     const CUtensorMap& tmPhi, const CUtensorMap& tmPlo, const CUtensorMap& tmUhi,
-    const CUtensorMap& tmUlo, int64_t k0p, int kwp, const float* __restrict__ Wp, int64_t m,
+    const CUtensorMap& tmUlo, int64_t k0p, int kwp, float* Wp, int64_t m,
     int64_t n, int64_t j0, int bw, const unsigned char* __restrict__ pkg, int bits, int group,
     int64_t ngroups, uint8_t* __restrict__ codes, float* __restrict__ scale,
     uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info,
-    const int32_t* __restrict__ perm, int bx, unsigned char* smraw) {
+    const int32_t* __restrict__ perm, const OutlierArgs& oa, int bx, unsigned char* smraw) {
   const uint32_t raw = smem_addr(smraw);
   unsigned char* sm = smraw + ((1024 - (raw & 1023)) & 1023);
   const float* Ud = reinterpret_cast<const float*>(sm + SM_PKG + PK_UD);
@@ -219,6 +224,8 @@ __device__ __forceinline__ void sweep_body(
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
   pdl_wait();                           // the strip was written by the previous kernel
   pdl_trigger();
+  float alpha = 1.f;
+  if constexpr (OUTL) alpha = *oa.alpha;
   if (t == 0) {
     // the strip, when the rows allow a tensor map: four boxes at (j0 + 32q,
     // r0); columns past n read as zero, and Wp holds whole 128-row boxes
@@ -348,6 +355,7 @@ __device__ __forceinline__ void sweep_body(
   const float maxq = (float)((1 << bits) - 1);
   float s = 1.f, z = 0.f, loss = 0.f, rs = 1.f, klo = 0.f, khi = maxq;
   uint8_t* cr = cs + t * LDB;
+  int ocnt = 0;                         // this row's outliers in the block
   const int nsb = (bw + SS - 1) / SS;
   int issued = 0;                       // MMA groups committed to mma_bar
   for (int sb = 0; sb < nsb && !abort; ++sb) {
@@ -422,8 +430,9 @@ __device__ __forceinline__ void sweep_body(
       }
       if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
       s = __fdiv_rn(xmax - xmin, maxq);
-      rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
       z = rintf(div_rn(-xmin, s));
+      if constexpr (OUTL) s = __fmul_rn(s, alpha);
+      rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
       klo = -z;
       khi = maxq - z;
       if (row < m) {
@@ -483,11 +492,20 @@ __device__ __forceinline__ void sweep_body(
       }
       // q − z = clamp(rint(v/s), −z, maxq − z) exactly (small integers), so
       // the clamp works on k = q − z and the error takes one FMA
-      const float k = fminf(fmaxf(rintf(div_fma(v[i], s, rs)), klo), khi);
-      const float ei = fmaf(-s, k, v[i]) * rdiag[c];
+      const float raw = rintf(div_fma(v[i], s, rs));
+      const float k = fminf(fmaxf(raw, klo), khi);
+      float ei = fmaf(-s, k, v[i]) * rdiag[c];
+      if constexpr (OUTL) {
+        const bool o = raw != k;        // the unclipped code leaves the grid
+        ei = o ? 0.f : ei;
+        ocnt += o ? 1 : 0;
+        if (o && row < m && c < bw) Wp[row * n + j0 + c] = v[i];
+        cr[c] = (uint8_t)(k + z) | (o ? OUTLIER_FLAG : (uint8_t)0);
+      } else {
+        cr[c] = (uint8_t)(k + z);
+      }
       e[i] = ei;
       loss = fmaf(ei, ei, loss);
-      cr[c] = (uint8_t)(k + z);
       const float4* ur = reinterpret_cast<const float4*>(ud + i * SS);
 #pragma unroll
       for (int q4 = (i + 1) / 4; q4 < SS / 4; ++q4) {
@@ -548,6 +566,11 @@ __device__ __forceinline__ void sweep_body(
     if (sb + 1 < nsb) ++issued;
   }
   if (!abort && row < m && loss_row != nullptr) loss_row[row] += loss;
+  if constexpr (OUTL) {
+    if (!abort && row < m) oa.row_cnt[row] += ocnt;
+    const int wc = __reduce_add_sync(0xffffffffu, ocnt);
+    if (lane == 0 && wc != 0 && !abort) atomicAdd(oa.total, (unsigned long long)wc);
+  }
   tc_fence_before();
   __syncthreads();
 
@@ -585,33 +608,33 @@ __device__ __forceinline__ void sweep_body(
 // 256 columns per 128-row tile): the two touch different columns, and both
 // take their inputs from earlier launches, so that consecutive sweeps follow
 // each other with nothing between them but the programmatic launch edge.
-template <bool ROWG>
+template <bool ROWG, bool OUTL>
 __global__ void __launch_bounds__(RT, 1)
 sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
              const __grid_constant__ CUtensorMap tmW, int strip_tma,
              const __grid_constant__ CUtensorMap tmPhi, const __grid_constant__ CUtensorMap tmPlo,
              const __grid_constant__ CUtensorMap tmUhi, const __grid_constant__ CUtensorMap tmUlo,
              int64_t k0p, int kwp,
-             const float* __restrict__ Wp, int64_t m, int64_t n, int64_t j0, int bw,
+             float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
              const unsigned char* __restrict__ pkg, int bits, int group, int64_t ngroups,
              uint8_t* __restrict__ codes, float* __restrict__ scale,
              uint8_t* __restrict__ zero, float* __restrict__ loss_row, int32_t* info,
-             const int32_t* __restrict__ perm, int nsweep,
+             const int32_t* __restrict__ perm, const OutlierArgs oa, int nsweep,
              const __grid_constant__ TrailMaps far, int64_t fc0, int64_t fc1, int64_t fk0,
              int fkw, int fx) {
   extern __shared__ unsigned char smraw[];
   const int b = (int)blockIdx.x;
   if (b < nsweep) {
-    sweep_body<ROWG>(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp, Wp, m,
-                     n, j0, bw, pkg, bits, group, ngroups, codes, scale, zero, loss_row, info,
-                     perm, b, smraw);
+    sweep_body<ROWG, OUTL>(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp,
+                           Wp, m, n, j0, bw, pkg, bits, group, ngroups, codes, scale, zero,
+                           loss_row, info, perm, oa, b, smraw);
   } else {
     const int f = b - nsweep;
     trailing_tc_body(far, m, n, fc0, fc1, fk0, fkw, info, f % fx, f / fx, smraw);
   }
 }
 
-bool g_attr_set[2] = {false, false};
+bool g_attr_set[3] = {false, false, false};   // plain, row groups, outliers
 
 }  // namespace
 
@@ -632,18 +655,27 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
                          float* Elo, const SweepPrologue& pre, const SweepFar& far,
                          float* loss_row, int32_t* info, const int32_t* rowgroup_perm,
-                         cudaStream_t s) {
+                         const OutlierArgs* outl, cudaStream_t s) {
   constexpr size_t kSmem = SMEM_BYTES > QSMEM ? SMEM_BYTES : QSMEM;
   const bool rowg = rowgroup_perm != nullptr;
-  if (!g_attr_set[rowg]) {
-    if (rowg)
-      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<true>,
+  if (rowg && outl != nullptr)
+    return fail(GPTQ_ERR_UNSUPPORTED, "sweep: outliers with output-channel groups");
+  if (outl != nullptr && (!outl->alpha || !outl->row_cnt || !outl->total || bits > 7))
+    return fail(GPTQ_ERR_INVALID_ARG, "sweep: outlier arguments");
+  const int variant = rowg ? 1 : (outl != nullptr ? 2 : 0);
+  if (!g_attr_set[variant]) {
+    if (variant == 1)
+      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<true, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
+    else if (variant == 2)
+      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<false, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
     else
-      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<false>,
+      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<false, false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-    g_attr_set[rowg] = true;
+    g_attr_set[variant] = true;
   }
+  const OutlierArgs oa = outl != nullptr ? *outl : OutlierArgs();
   // the far-column update riding along: fx 256-column tiles per 128-row tile
   TrailMaps fm;
   memset(&fm, 0, sizeof(fm));
@@ -686,18 +718,23 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const int nsweep = (int)ceil_div(m, RT);
   const unsigned grid = (unsigned)(nsweep + nfar);
-  if (rowg)
-    GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel<true>, grid, RT, kSmem, th, tl, tw, strip_tma, tph,
-                    tpl, tuh, tul, (int64_t)pre.k0, kwp, (const float*)Wp, m, n, j0, bw,
-                    reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
-                    scale, zero, loss_row, info, rowgroup_perm, nsweep, fm, far.c0, fc1, far.k0,
-                    far.kw, fx > 0 ? fx : 1);
+  const unsigned char* pk = reinterpret_cast<const unsigned char*>(panel);
+  const int fxx = fx > 0 ? fx : 1;
+  if (variant == 1)
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<true, false>), grid, RT, kSmem, th, tl, tw,
+                    strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
+                    bits, group, ngroups, codes, scale, zero, loss_row, info, rowgroup_perm, oa,
+                    nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
+  else if (variant == 2)
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, true>), grid, RT, kSmem, th, tl, tw,
+                    strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
+                    bits, group, ngroups, codes, scale, zero, loss_row, info,
+                    (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
   else
-    GPTQ_LAUNCH_PDL(KK_SWEEP, s, sweep_kernel<false>, grid, RT, kSmem, th, tl, tw, strip_tma, tph,
-                    tpl, tuh, tul, (int64_t)pre.k0, kwp, (const float*)Wp, m, n, j0, bw,
-                    reinterpret_cast<const unsigned char*>(panel), bits, group, ngroups, codes,
-                    scale, zero, loss_row, info, (const int32_t*)nullptr, nsweep, fm, far.c0,
-                    fc1, far.k0, far.kw, fx > 0 ? fx : 1);
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, false>), grid, RT, kSmem, th, tl, tw,
+                    strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
+                    bits, group, ngroups, codes, scale, zero, loss_row, info,
+                    (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
   return GPTQ_OK;
 }
 

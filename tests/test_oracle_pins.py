@@ -493,3 +493,24 @@ def test_min_pivot_catches_planted_mistakes(golden):
 
     assert largest(H) != want
     assert static_diagonal(H) != want
+
+
+def test_follow_accepts_a_zero_point_flipped_at_a_tie():
+    """A zero point decided at a near-tie may go either way; the other side's
+    codes then sit one step over for the whole group.  Follow mode must count
+    the one allowed zero flip and no code difference (the codes are the same
+    grid, shifted)."""
+    W = np.array([[-1.0, 5.0, 0.3, 2.0, -0.7, 4.1, 1.1, 3.3]])
+    s, z = og.group_params(W[:, :4], 4)                  # −xmin/s = 2.5 up to rounding
+    zpre = 1.0 / float(s[0])
+    assert abs(zpre - 2.5) < 1e-6
+    z2 = np.float32(z[0] + (1 if z[0] == 2 else -1))
+    s2, zb = og.group_params(W[:, 4:], 4)
+    q = np.concatenate([
+        np.clip(np.rint(np.float32(W[0, :4]) / s[0]) + z2, 0, 15),
+        np.clip(np.rint(np.float32(W[0, 4:]) / s2[0]) + zb[0], 0, 15)])[None, :]
+    scale = np.stack([s, s2], axis=1)
+    zero = np.array([[z2, zb[0]]], np.float32)
+    f = og.follow(W, np.eye(8), 4, 4, 8, q.astype(np.int64), scale, zero)
+    assert f["zero_diff"] == 1 and f["zero_diff_disallowed"] == 0
+    assert f["code_diff_disallowed"] == 0

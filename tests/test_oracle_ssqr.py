@@ -313,3 +313,16 @@ def test_pins_catch_planted_mistakes(kind, monkeypatch):
     failures += not _satz5_holds(res, p["U"], 16)
     failures += not _loss_identity_holds(Wp, res, p["Hp"], 16)
     assert failures >= 1, kind
+
+
+def test_follow_accepts_a_zero_point_flipped_at_a_tie():
+    """As the GPTQ checker: a zero flipped at a near-tie shifts the group's
+    codes by one step; that is one allowed flip, not a code difference per
+    column."""
+    W = np.array([[-1.0, 5.0, 0.3, 2.0]])
+    s, z, s0 = S.adjusted_params(W, 4, 1.0)
+    z2 = np.float32(z[0] + (1 if z[0] == 2 else -1))
+    q = np.clip(np.rint(np.float32(W[0]) / s[0]) + z2, 0, 15)[None, :].astype(np.int64)
+    f = S.follow_ssqr(W, np.eye(4), 4, 4, 4, 1.0, q, np.zeros((1, 4), bool),
+                      np.zeros((1, 4)), s[:, None], np.array([[z2]], np.float32))
+    assert f["z_bad"] == 0 and f["n_bad"] == 0 and f["n_diff"] == 0

@@ -104,3 +104,16 @@ def spectral_weights(rows: int, cols: int, seed: int, decay: float = 0.8,
     w = (qa * sig) @ qb.T
     w = w * (std / w.std())
     return w.to(torch.float32)
+
+
+def student_t_weights(rows: int, cols: int, seed: int, df: int = 3,
+                      std: float = 0.02) -> torch.Tensor:
+    """rows × cols float32 weights std·t with t ~ Student-t(df) (z over
+    sqrt(χ²_df/df)): a heavy-tailed layer, the case outlier-keeping schemes
+    are made for."""
+    g = _gen(seed)
+    z = torch.randn(rows, cols, generator=g, dtype=torch.float32)
+    chi2 = torch.zeros(rows, cols, dtype=torch.float32)
+    for _ in range(df):
+        chi2 += torch.randn(rows, cols, generator=g, dtype=torch.float32).square()
+    return z / torch.sqrt(chi2 / df) * std
