@@ -796,6 +796,267 @@ def chmc_cpu_baseline(probs):
                                         "both Hessians from X included"}
 
 
+# ---------------------------------------------------------------- SSQR
+
+SSQR_METRIC = ("SSQR weights compressed/sec (params/s incl. Hessian, the binary search's "
+               "sweeps and the CSR outliers) & % of roofline, 1 B200")
+SSQR_BITS, SSQR_TARGET, SSQR_ITERS, SSQR_LO, SSQR_HI = 3, 0.01, 12, 1.0 / 16, 1.0
+
+
+class SsqrLayer:
+    """Device buffers of one layer under SSQR ("The Geometry of LLM
+    Quantization: GPTQ as Babai's Nearest Plane Algorithm", §3): per Hessian
+    its factor, per weight matrix its codes, scales, CSR outliers and the
+    search's trace (each matrix meets the outlier target on its own)."""
+
+    def __init__(self, probs, device):
+        import post_weight_quantization_08_b200 as g
+        self.g = g
+        self.items = []
+        for p in probs:
+            n = p.n
+            it = {"p": p, "X": p.X.to(device).contiguous(),
+                  "H": torch.zeros(n, n, dtype=torch.float32, device=device),
+                  "perm": torch.empty(n, dtype=torch.int32, device=device),
+                  "U": torch.empty(n, n, dtype=torch.float32, device=device),
+                  "dead": torch.empty(n, dtype=torch.uint8, device=device),
+                  "info_h": torch.zeros(2, dtype=torch.int32, device=device),
+                  "info_p": torch.zeros(2, dtype=torch.int32, device=device),
+                  "ws_p": g.workspace(g.gptq_prepare_workspace_bytes(n), device),
+                  "stream": torch.cuda.Stream(device=device), "parts": []}
+            row0 = 0
+            for name, rows in p.parts:
+                W = p.W[row0:row0 + rows].to(device).contiguous()
+                row0 += rows
+                ng = -(-n // p.group)
+                cap = max(int(SSQR_TARGET * rows * n), 1)
+                it["parts"].append({
+                    "name": name, "W": W,
+                    "qweight": torch.empty(rows, -(-n * SSQR_BITS // 32), dtype=torch.int32,
+                                           device=device),
+                    "scale": torch.empty(rows, ng, dtype=torch.float32, device=device),
+                    "zero": torch.empty(rows, ng, dtype=torch.uint8, device=device),
+                    "g_idx": torch.empty(n, dtype=torch.int32, device=device),
+                    "row_ptr": torch.empty(rows + 1, dtype=torch.int64, device=device),
+                    "col_idx": torch.empty(cap, dtype=torch.int32, device=device),
+                    "val": torch.empty(cap, dtype=torch.float32, device=device),
+                    "alpha": torch.empty(1, dtype=torch.float32, device=device),
+                    "loss": torch.empty(rows, dtype=torch.float32, device=device),
+                    "info_q": torch.zeros(2, dtype=torch.int32, device=device),
+                    "ws_q": g.workspace(g.gptq_ssqr_workspace_bytes(rows, n, p.block), device),
+                    "stream": torch.cuda.Stream(device=device),
+                })
+            self.items.append(it)
+
+    def run_problem(self, it, serial=False):
+        """Hessian and factor on the problem's stream, then each matrix's
+        search on a stream of its own (``serial``: all on one stream)."""
+        g, p, s = self.g, it["p"], it["stream"]
+        with torch.cuda.stream(s):
+            it["H"].zero_()
+        g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
+        g.gptq_prepare(it["H"], p.damp, "act", it["perm"], it["U"], it["dead"],
+                       it["info_p"], it["ws_p"], s)
+        prep_done = torch.cuda.Event()
+        prep_done.record(s)
+        for q in it["parts"]:
+            qs = s if serial else q["stream"]
+            if not serial:
+                qs.wait_event(prep_done)
+            g.gptq_ssqr_quantize(q["W"], it["U"], it["perm"], it["dead"], SSQR_BITS, p.group,
+                                 p.block, SSQR_TARGET, SSQR_ITERS, SSQR_LO, SSQR_HI,
+                                 q["qweight"], q["scale"], q["zero"], q["g_idx"], q["row_ptr"],
+                                 q["col_idx"], q["val"], q["alpha"], None, None, q["loss"],
+                                 None, q["info_q"], q["ws_q"], qs)
+            if not serial:
+                e = torch.cuda.Event()
+                e.record(qs)
+                s.wait_event(e)
+
+    step = ChmcLayer.step
+    step_serial = ChmcLayer.step_serial
+
+    def check(self):
+        for it in self.items:
+            for key in ("info_h", "info_p"):
+                st, idx = self.g.gptq_check(it[key], it["stream"])
+                if st != 0:
+                    raise RuntimeError(f"device reported status {st} at {idx}")
+            for q in it["parts"]:
+                st, idx = self.g.gptq_check(q["info_q"], it["stream"])
+                if st != 0:
+                    raise RuntimeError(f"{q['name']}: device reported status {st} at {idx}")
+
+
+def ssqr_work(layer):
+    """Algorithmic work per kernel kind for one SSQR step: the hot path's
+    per-kind figures (kernel_work) with the sweep and ingest counted once per
+    pass (iters + 2 passes per matrix), the TF32 split of U and the packing
+    once per matrix, and the ssqr kind's CSR fill (codes read, 1 B per
+    weight)."""
+    w = {k: 0.0 for k in ("hessian", "cholesky", "sweep", "trailing", "pack", "ingest", "ssqr")}
+    passes = SSQR_ITERS + 2
+    for it in layer.items:
+        p = it["p"]
+        n, T, block = p.n, p.T, p.block
+        w["hessian"] += T * n * (n + 1)
+        N = -(-n // 64)
+        for k in range(N):
+            r = N - k - 1
+            w["cholesky"] += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
+            w["cholesky"] += 2 * 64 ** 3 / 3
+        fused = n % 4 == 0 and n > block
+        for q in it["parts"]:
+            m = q["W"].shape[0]
+            if fused:
+                w["trailing"] += 12 * n * n
+            for j0 in range(0, n, block):
+                bw = min(block, n - j0)
+                n2 = n - j0 - bw
+                w["sweep"] += passes * (9 * m * bw + 4 * bw * bw + 5 * m * (-(-bw // p.group)))
+                if n2 > 0:
+                    w["sweep" if fused else "trailing"] += passes * (8 * m * n2 + 4 * m * bw
+                                                                     + 4 * bw * n2)
+            w["pack"] += m * n + m * n * SSQR_BITS / 8 + 5 * m * (-(-n // p.group))
+            w["ingest"] += passes * m * n * (q["W"].element_size() + 4)
+            w["ssqr"] += m * n
+    units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s", "sweep": "GB/s", "trailing": "GB/s",
+             "pack": "GB/s", "ingest": "GB/s", "ssqr": "GB/s"}
+    return {k: (units[k], v) for k, v in w.items()}
+
+
+def ssqr_cpu_baseline(probs, budget_s: float = 20.0):
+    """The SSQR oracle on the layer's matrices in order (Hessian from X, the
+    whole binary search), until the time budget is spent; params/s over the
+    matrices completed."""
+    from oracle import gptq as og
+    from oracle import ssqr as osq
+    t0 = time.perf_counter()
+    total, done = 0, []
+    for p in probs:
+        H = og.hessian(p.X.to(torch.float64).numpy())
+        prep = og.prepare(H, p.damp, "act")
+        row0 = 0
+        for name, rows in p.parts:
+            W = p.W[row0:row0 + rows].to(torch.float64).numpy()
+            row0 += rows
+            osq.ssqr_layer(W, H, bits=SSQR_BITS, group=p.group, block=p.block, damp=p.damp,
+                           target=SSQR_TARGET, iters=SSQR_ITERS, alpha_lo=SSQR_LO,
+                           alpha_hi=SSQR_HI, prep=prep)
+            total += rows * p.n
+            done.append(name)
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(total / dt, 1), "unit": "params/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"the layer's matrices in order until {budget_s:.0f} s: {', '.join(done)} "
+                      f"({dt:.1f} s, Hessians and factors included)"}
+
+
+def run_ssqr(args, rank, world, local):
+    """SSQR over the layer: device-timed graph replay and the per-kernel
+    event profile, as for the CHMC frontend."""
+    import post_weight_quantization_08_b200 as g
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = CONFIGS[args.config]
+    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=SSQR_BITS, order="act")
+    layer = SsqrLayer(probs, device)
+    params = sum(p.params for p in probs)
+    out = _time_frontend(args, layer, device, world, local, ssqr_work(layer))
+    alphas = {q["name"]: float(q["alpha"].cpu()[0]) for it in layer.items for q in it["parts"]}
+    nnz = {q["name"]: int(q["row_ptr"][-1]) for it in layer.items for q in it["parts"]}
+    dev_ms, launches, kernels, kms, clk = out
+    total_params = sum_over_ranks(params * args.steps, world, device)
+    return {
+        "metric": SSQR_METRIC, "value": round(total_params / (dev_ms / 1e3), 1),
+        "unit": "params/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep",
+        "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
+        "config": {"workload": f"{cfg['name']} SSQR: {SSQR_BITS}-bit, group {probs[0].group}, "
+                               f"act-order, target outlier density {SSQR_TARGET} per matrix, "
+                               f"{SSQR_ITERS} bisection steps on alpha in [{SSQR_LO}, {SSQR_HI}], "
+                               f"block {probs[0].block}",
+                   "params_per_step_per_gpu": params, "alpha": alphas, "outliers": nnz,
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "launch": "CUDA graph replay per step"},
+        "gpu_launches": int(launches * args.steps),
+        "kernels": kernels, "kernels_ms_per_step": kms, "clocks": clk,
+    }, probs
+
+
+def _time_frontend(args, layer, device, world, local, work):
+    """Warm up, capture one step in a CUDA graph, time K replays with the L2
+    flushed between them (max over ranks), then time every kernel kind with
+    the library's event profiler on a serialised step."""
+    import post_weight_quantization_08_b200 as g
+    main = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(main)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(args.warmup):
+        layer.step(main)
+    torch.cuda.synchronize(device)
+    layer.check()
+    graph = torch.cuda.CUDAGraph()
+    c0 = g.gptq_launch_count()
+    with torch.cuda.graph(graph, stream=main):
+        layer.step(main)
+    launches_per_step = g.gptq_launch_count() - c0
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(device)
+    layer.check()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        graph.replay()
+        b.record(main)
+        evs.append((a, b))
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    layer.check()
+    dev_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
+    g.gptq_profile_start(1 << 17)
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        layer.step_serial(main)
+    torch.cuda.synchronize(device)
+    kprof = g.gptq_profile_stop()
+    peaks, src = _peaks()
+    kernels = {}
+    for k, (unit, amount) in work.items():
+        if k not in kprof or kprof[k][1] <= 0 or amount <= 0:
+            continue
+        per_step_ms = kprof[k][0] / args.steps
+        if unit == "TFLOP/s":
+            ach = amount / (per_step_ms / 1e3) / 1e12
+            bound, peak = (("tensor", peaks["bf16_tflops"]) if k == "hessian" else
+                           ("alu", fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))))
+        else:
+            ach = amount / (per_step_ms / 1e3) / 1e9
+            bound, peak = "hbm", peaks["hbm_gbs"]
+        kernels[k] = {"ms_per_step": round(per_step_ms, 4),
+                      "launches_per_step": kprof[k][1] / args.steps, "bound": bound,
+                      "achieved": round(ach, 2), "unit": unit, "peak": round(peak, 1),
+                      "frac": round(ach / peak, 4)}
+    kms = {k: round(v[0] / args.steps, 4) for k, v in kprof.items() if v[0] > 0}
+    return dev_ms, launches_per_step, kernels, kms, clk
+
+
 # ---------------------------------------------------------------- CPU oracle arm
 
 def oracle_pass(probs):
@@ -875,8 +1136,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--frontend", default="gptq", choices=["gptq", "chmc"],
-                    help="chmc: the CHMC frontend over the layer (a separate metric)")
+    ap.add_argument("--frontend", default="gptq", choices=["gptq", "chmc", "ssqr"],
+                    help="chmc: the CHMC frontend over the layer; ssqr: SSQR over the "
+                         "layer (separate metrics)")
     ap.add_argument("--order", default=None,
                     choices=["natural", "act", "reverse", "minpivot"],
                     help="processing order for every problem (default: the workload's)")
@@ -901,6 +1163,10 @@ def main(argv=None):
             out, probs = run_chmc(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = chmc_cpu_baseline(probs)
+        elif args.frontend == "ssqr":
+            out, probs = run_ssqr(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = ssqr_cpu_baseline(probs)
         else:
             out, probs, _ = run_ours(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
