@@ -334,6 +334,72 @@ gptq_status gptq_ssqr_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
                                int64_t* trace_count, float* loss_row, float* Qdq,
                                int32_t* info, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- HPTQ (next to the hot path) ----------------------------------------
+ * "The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+ * Algorithm", §3: Huffman-encoded PTQ quantizes inliers and outliers on one
+ * unbounded integer grid (no clipping, so Satz 5's bound of §2.3 holds) and
+ * Huffman-codes the integers to meet a compression budget; §4 names 3.125
+ * bits per weight.
+ */
+
+/* Symbol window of the code: symbol = q + GPTQ_HPTQ_SYMBOL_OFFSET, in
+ * [0, GPTQ_HPTQ_SYMBOLS).  Codes outside it are reported as UNSUPPORTED. */
+#define GPTQ_HPTQ_SYMBOLS 4096
+#define GPTQ_HPTQ_SYMBOL_OFFSET 2048
+
+/* Bytes of device workspace gptq_hptq_quantize needs (256-byte aligned). */
+size_t gptq_hptq_workspace_bytes(int64_t m, int64_t n, int block);
+
+/*
+ * As gptq_quantize (W, U, perm, dead, group, block, scale, g_idx, loss_row,
+ * Qdq, info have the same meaning), except:
+ *   bits       nominal bits of the min-max step s0 = range/(2^bits − 1),
+ *              2, 3, 4 or 8.
+ *   Grid       the lattice s·Z of each group, s = alpha·s0 (float32): a
+ *              weight's integer is q = rint(w/s), any integer (no clamp and
+ *              no zero point, which an unbounded grid does not need); its
+ *              error is w − s·q (|·| ≤ s/2).  Dequantized: s·q.
+ *   Code       one Huffman code per call over the integers q; its cost (the
+ *              payload bits Σ count(q)·len(q)) drives the search.  A single
+ *              used symbol gets length 1.  Code words are canonical: in order
+ *              of (length, symbol) each is the previous plus one, shifted
+ *              left when the length grows.
+ *   Search     as gptq_ssqr_quantize's, with "admissible" meaning coded bits
+ *              ≤ floor(budget·m·n): alpha_hi (the coarsest grid) first, then up
+ *              to `iters` bisection steps; a last pass at the chosen alpha is
+ *              encoded.  Cost: iters + 2 sweeps of the layer.
+ *   budget     payload bits per weight, (0, 64].  iters 0..64.
+ *   alpha_lo, alpha_hi   0 < alpha_lo ≤ alpha_hi ≤ 256.
+ *   codes      m×n int16 or NULL, output: q in ORIGINAL column order.
+ *   code_len   uint8[GPTQ_HPTQ_SYMBOLS], output: length per symbol (0: unused).
+ *   code_word  uint64[GPTQ_HPTQ_SYMBOLS] or NULL, output: canonical code
+ *              words, right-aligned.
+ *   row_off    int64[m + 1], output: bit offset of each row in the stream
+ *              (row_off[m] = the coded bits).
+ *   stream_words  uint32[stream_cap], output: rows one after another in
+ *              original column order, each code most significant bit first,
+ *              words filled from their most significant bit.  Bits past
+ *              stream_cap·32 are dropped and info reports CAPACITY.  May be
+ *              NULL when stream_cap == 0.
+ *   alpha      float32[1], output: the chosen factor.
+ *   trace_alpha, trace_bits   float32 / int64 [iters + 1] or NULL: the alpha and
+ *              coded bits of each search pass (−1 after the search ended).
+ *   ws         device workspace of at least gptq_hptq_workspace_bytes().
+ * Errors: INVALID_ARG (null pointer, budget, iters, bracket, stream_cap < 0,
+ * workspace), UNSUPPORTED (bits, group, block), CUDA; NONFINITE, CAPACITY and
+ * UNSUPPORTED (a code outside the symbol window, a code longer than 64 bits)
+ * through info.
+ */
+gptq_status gptq_hptq_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
+                               const float* U, const int32_t* perm, const uint8_t* dead,
+                               int bits, int group, int block, double budget, int iters,
+                               float alpha_lo, float alpha_hi, int16_t* codes, float* scale,
+                               int32_t* g_idx, uint8_t* code_len,
+                               uint64_t* code_word, int64_t* row_off, uint32_t* stream_words,
+                               int64_t stream_cap, float* alpha, float* trace_alpha,
+                               int64_t* trace_bits, float* loss_row, float* Qdq,
+                               int32_t* info, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * Synchronize `stream`, read info[0..1] and return info[0] (a gptq_status).
  * If `index` is not NULL it receives info[1].  `info` is a device pointer.

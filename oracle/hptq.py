@@ -16,14 +16,17 @@ Source (page title, then the place on the page)
 
 Readings taken where the page is silent
 ---------------------------------------
-* The grid is the hot path's group quantizer without the clamp: the group's
-  min-max step s₀ (from ``bits`` nominal bits, taken at the group's first
-  column from its current values) becomes s = fl32(α·s₀), the zero point stays
-  z = rint(−xmin/s₀), and q = rint(w/s) + z is any integer.  Every weight's
-  error is w − s·(q − z) (no clipping, so |error| ≤ s/2).
-* One Huffman code per weight matrix over its integers q.  The budget counts
+* The grid is the lattice s·ℤ of each group: the group's min-max step s₀
+  (the hot path's, from ``bits`` nominal bits, taken at the group's first
+  column from its current values) becomes s = fl32(α·s₀), and a weight's
+  integer is k = rint(w/s), any integer, decided in float32.  Its error is
+  w − s·k (no clipping, so |error| ≤ s/2).  With no clamp a zero point has no
+  role (rint(w/s) + z − z = rint(w/s) for an integer z), so the integers are
+  the lattice coordinates themselves, centred on 0, and one code serves every
+  group: "one unbounded integer grid".
+* One Huffman code per weight matrix over its integers k.  The budget counts
   the coded payload: Σ_q count(q)·len(q) ≤ B_max = floor(budget·m·n) bits.
-  Scales, zeros and the code table are stored beside it and not counted.
+  The scales and the code table are stored beside it and not counted.
 * A matrix whose codes take one value only codes it with 1 bit.
 * Huffman lengths are not unique where counts tie; the optimal total cost is.
   Both sides' decisions use the cost; a code table is checked as valid (Kraft
@@ -51,9 +54,14 @@ def max_bits(budget: float, m: int, n: int) -> int:
     return int(np.floor(float(budget) * float(m) * float(n)))
 
 
+def lattice_column(cur, scale):
+    """k = rint(w/s) in float32: the weight's coordinate on s·ℤ."""
+    return np.rint(np.asarray(cur, dtype=np.float32) / scale).astype(np.float32)
+
+
 def hptq_blocked(Wp, U, bits: int, group: int, block: int, alpha) -> dict:
     """The unclipped sweep, lazy-batch form, columns in processing order;
-    codes are unbounded integers."""
+    codes are the unbounded lattice coordinates k."""
     if block % group != 0:
         raise ValueError("block must be a multiple of group")
     W = np.array(Wp, dtype=np.float64, copy=True)
@@ -61,21 +69,20 @@ def hptq_blocked(Wp, U, bits: int, group: int, block: int, alpha) -> dict:
     m, n = W.shape
     ng = -(-n // group)
     out = {"codes": np.zeros((m, n), np.int64), "scale": np.zeros((m, ng), np.float32),
-           "zero": np.zeros((m, ng), np.float32), "err": np.zeros((m, n)),
-           "pre": np.zeros((m, n))}
-    s = z = None
+           "err": np.zeros((m, n)), "pre": np.zeros((m, n))}
+    s = None
     a32 = np.float32(alpha)
     for b0 in range(0, n, block):
         b1 = min(b0 + block, n)
         for j in range(b0, b1):
             g = j // group
             if j % group == 0:
-                s0, z = G.group_params(W[:, j:min(j + group, n)], bits)
+                s0, _ = G.group_params(W[:, j:min(j + group, n)], bits)
                 s = (s0 * a32).astype(np.float32)
-                out["scale"][:, g], out["zero"][:, g] = s, z
+                out["scale"][:, g] = s
             out["pre"][:, j] = W[:, j] / s.astype(np.float64)
-            q = G.quantize_column(W[:, j], s, z, bits, clip=False)
-            e = (W[:, j] - G.dequantize(q, s, z)) / U[j, j]
+            q = lattice_column(W[:, j], s)
+            e = (W[:, j] - s.astype(np.float64) * q.astype(np.float64)) / U[j, j]
             W[:, j + 1:b1] -= np.outer(e, U[j, j + 1:b1])
             out["codes"][:, j] = q.astype(np.int64)
             out["err"][:, j] = e
@@ -225,24 +232,23 @@ def hptq_layer(W, H, bits: int = 4, group: int = 128, block: int = 128, damp: fl
     inv = G.inverse_permutation(perm)
     codes = res["codes"][:, inv]
     g_idx = (inv // group).astype(np.int64)
-    Q = G.dequantize(codes, res["scale"][:, g_idx], res["zero"][:, g_idx])
+    Q = res["scale"][:, g_idx].astype(np.float64) * codes
     hist = histogram(codes)
     lengths = huffman_lengths(hist)
     return {"alpha": alpha, "trace": trace, "codes": codes, "scale": res["scale"],
-            "zero": res["zero"], "g_idx": g_idx, "Q": Q, "hist": hist, "lengths": lengths,
+            "g_idx": g_idx, "Q": Q, "hist": hist, "lengths": lengths,
             "bits": cost(hist, lengths), "perm": perm, "dead": prep["dead"], "U": prep["U"],
             "res_p": res, "loss": G.layer_loss(W, Q, H)}
 
 
-def follow_hptq(Wp, U, bits: int, group: int, block: int, alpha, codes_p, scale, zero,
+def follow_hptq(Wp, U, bits: int, group: int, block: int, alpha, codes_p, scale,
                 tol: float = 1e-4, scale_rtol: float = 1e-5) -> dict:
     """Walk the unclipped sweep with another implementation's codes.
 
     As the SSQR checker: the oracle forms its own current values from the
-    other side's earlier decisions, its own scale and zero at group starts and
+    other side's earlier decisions, its own scale at group starts and
     its own code; a differing code is allowed only within ``tol`` code units
-    of a rounding boundary; a zero point flipped at a near-tie moves the
-    group's codes with it; scales are held to ``scale_rtol`` or, in a group
+    of a rounding boundary; scales are held to ``scale_rtol`` or, in a group
     narrower than 32 columns, to the float32 forward-error bound of the
     propagation (2·γ_K·M/(2^b − 1)·α, γ_K = 2⁻²¹ + K·2⁻²⁴, M the largest
     |w| + Σ|e_k·U_kj| of the group).  Arrays in processing order.
@@ -252,13 +258,12 @@ def follow_hptq(Wp, U, bits: int, group: int, block: int, alpha, codes_p, scale,
     m, n = W.shape
     codes_p = np.asarray(codes_p, dtype=np.int64)
     scale = np.asarray(scale, dtype=np.float32)
-    zero = np.asarray(zero, dtype=np.float32)
     maxq = 2 ** bits - 1
-    n_diff = n_bad = z_bad = scale_bad = scale_wide_over = 0
+    n_diff = n_bad = scale_bad = scale_wide_over = 0
     max_scale_rel = 0.0
     err = np.zeros((m, n))
     mag = np.abs(W)
-    s_o = z_o = None
+    s_o = None
     a32 = np.float32(alpha)
     for b0 in range(0, n, block):
         b1 = min(b0 + block, n)
@@ -266,10 +271,8 @@ def follow_hptq(Wp, U, bits: int, group: int, block: int, alpha, codes_p, scale,
             g = j // group
             if j % group == 0:
                 cur = W[:, j:min(j + group, n)]
-                s0, z_o = G.group_params(cur, bits)
+                s0, _ = G.group_params(cur, bits)
                 s_o = (s0 * a32).astype(np.float32)
-                c32 = np.asarray(cur, np.float32)
-                zpre = -np.minimum(c32.min(axis=1), 0).astype(np.float64) / s0.astype(np.float64)
                 rel = np.abs(scale[:, g].astype(np.float64) - s_o) / np.abs(s_o)
                 width = cur.shape[1]
                 M = mag[:, j:j + width].max(axis=1)
@@ -278,25 +281,21 @@ def follow_hptq(Wp, U, bits: int, group: int, block: int, alpha, codes_p, scale,
                 if width >= 32:
                     scale_wide_over += int(np.sum(rel > scale_rtol))
                 max_scale_rel = max(max_scale_rel, float(rel.max()))
-                zd = zero[:, g] != z_o
-                near_z = np.abs(zpre - np.floor(zpre) - 0.5) <= tol
-                z_bad += int((zd & ~near_z).sum())
-                z_o = np.where(zd & near_z, zero[:, g], z_o).astype(np.float32)
-            s_g, z_g = scale[:, g], zero[:, g]
+            s_g = scale[:, g]
             x = W[:, j] / s_o.astype(np.float64)
-            q_o = G.quantize_column(W[:, j], s_o, z_o, bits, clip=False).astype(np.int64)
+            q_o = lattice_column(W[:, j], s_o).astype(np.int64)
             q_g = codes_p[:, j]
             d = q_o != q_g
             if d.any():
                 near = np.abs(x - np.floor(x) - 0.5) <= tol
                 n_diff += int(d.sum())
                 n_bad += int((d & ~near).sum())
-            e = (W[:, j] - G.dequantize(q_g, s_g, z_g)) / U[j, j]
+            e = (W[:, j] - s_g.astype(np.float64) * q_g) / U[j, j]
             W[:, j + 1:b1] -= np.outer(e, U[j, j + 1:b1])
             mag[:, j + 1:b1] += np.outer(np.abs(e), np.abs(U[j, j + 1:b1]))
             err[:, j] = e
         if b1 < n:
             W[:, b1:] -= err[:, b0:b1] @ U[b0:b1, b1:]
             mag[:, b1:] += np.abs(err[:, b0:b1]) @ np.abs(U[b0:b1, b1:])
-    return {"n_diff": n_diff, "n_bad": n_bad, "z_bad": z_bad, "max_scale_rel": max_scale_rel,
+    return {"n_diff": n_diff, "n_bad": n_bad, "max_scale_rel": max_scale_rel,
             "scale_bad": scale_bad, "scale_wide_over": scale_wide_over, "err": err}

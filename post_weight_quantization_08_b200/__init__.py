@@ -15,7 +15,9 @@ from ._binding import (DTYPES, ORDERS, GptqError, exported_symbols,
                        gptq_launch_count, gptq_prepare, gptq_prepare_workspace_bytes,
                        gptq_profile_start, gptq_profile_stop, gptq_quantize,
                        gptq_quantize_rowgroups, gptq_quantize_workspace_bytes,
-                       gptq_ssqr_quantize, gptq_ssqr_workspace_bytes, kernel_names, lib)
+                       gptq_ssqr_quantize, gptq_ssqr_workspace_bytes, gptq_hptq_quantize,
+                       gptq_hptq_workspace_bytes, HPTQ_SYMBOLS, HPTQ_SYMBOL_OFFSET,
+                       kernel_names, lib)
 
 __all__ = [
     "GptqError", "ORDERS", "DTYPES", "lib", "exported_symbols", "kernel_names",
@@ -24,8 +26,9 @@ __all__ = [
     "gptq_launch_count", "gptq_profile_start", "gptq_profile_stop",
     "gptq_quantize_rowgroups", "gptq_chmc_rank", "gptq_chmc_workspace_bytes",
     "gptq_chmc_lowrank", "gptq_ssqr_quantize", "gptq_ssqr_workspace_bytes",
+    "gptq_hptq_quantize", "gptq_hptq_workspace_bytes", "HPTQ_SYMBOLS", "HPTQ_SYMBOL_OFFSET",
     "hessian", "prepare", "quantize", "workspace",
-    "chmc_lowrank", "quantize_rowgroups", "chmc_layer", "ssqr_quantize",
+    "chmc_lowrank", "quantize_rowgroups", "chmc_layer", "ssqr_quantize", "hptq_quantize",
 ]
 
 
@@ -210,4 +213,53 @@ def ssqr_quantize(W: torch.Tensor, prep: dict, bits: int = 3, group: int = 128,
         nnz = int(out["row_ptr"][-1])
         out["col_idx"] = out["col_idx"][:nnz]
         out["val"] = out["val"][:nnz]
+    return out
+
+
+# ---- HPTQ ("The Geometry of LLM Quantization: GPTQ as Babai's Nearest Plane
+# Algorithm", §3)
+
+def hptq_quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
+                  block: int = 128, budget: float = 3.125, iters: int = 16,
+                  alpha_lo: float = 1.0 / 16, alpha_hi: float = 16.0,
+                  stream_cap: int | None = None, want_loss: bool = True,
+                  want_qdq: bool = False, want_codes: bool = True, want_trace: bool = False,
+                  ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+    """GPTQ on the unbounded lattice s·ℤ, Huffman-coded: the integers
+    (original column order), scales, g_idx, the code table (length and canonical word
+    per symbol), the row bit offsets and the bit stream.  ``stream_cap``
+    (default: the budget's bits, in 32-bit words, plus one word per row)
+    sizes the stream; with ``check`` it is trimmed to the coded length."""
+    m, n = W.shape
+    dev = W.device
+    ng = -(-n // group)
+    if stream_cap is None:
+        stream_cap = int(budget * m * n) // 32 + m + 1
+    out = {
+        "codes": torch.empty(m, n, dtype=torch.int16, device=dev) if want_codes else None,
+        "scale": torch.empty(m, ng, dtype=torch.float32, device=dev),
+        "g_idx": torch.empty(n, dtype=torch.int32, device=dev),
+        "code_len": torch.empty(HPTQ_SYMBOLS, dtype=torch.uint8, device=dev),
+        "code_word": torch.empty(HPTQ_SYMBOLS, dtype=torch.int64, device=dev),
+        "row_off": torch.empty(m + 1, dtype=torch.int64, device=dev),
+        "stream": torch.empty(max(stream_cap, 1), dtype=torch.int32, device=dev),
+        "alpha": torch.empty(1, dtype=torch.float32, device=dev),
+        "trace_alpha": torch.empty(iters + 1, dtype=torch.float32, device=dev) if want_trace else None,
+        "trace_bits": torch.empty(iters + 1, dtype=torch.int64, device=dev) if want_trace else None,
+        "loss_row": torch.empty(m, dtype=torch.float32, device=dev) if want_loss else None,
+        "Qdq": torch.empty(m, n, dtype=torch.float32, device=dev) if want_qdq else None,
+        "info": torch.zeros(2, dtype=torch.int32, device=dev),
+    }
+    if ws is None:
+        ws = workspace(gptq_hptq_workspace_bytes(m, n, block), dev)
+    gptq_hptq_quantize(W, prep["U"], prep["perm"], prep["dead"], bits, group, block, budget,
+                       iters, alpha_lo, alpha_hi, out["codes"], out["scale"],
+                       out["g_idx"], out["code_len"], out["code_word"], out["row_off"],
+                       out["stream"] if stream_cap > 0 else None, out["alpha"],
+                       out["trace_alpha"], out["trace_bits"], out["loss_row"], out["Qdq"],
+                       out["info"], ws, stream)
+    if check:
+        _raise_info(out["info"], stream, "gptq_hptq_quantize")
+        nbits = int(out["row_off"][-1])
+        out["stream"] = out["stream"][:-(-nbits // 32)]
     return out

@@ -59,6 +59,15 @@ _SIGS = {
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
                                      C.c_void_p]),
+    "gptq_hptq_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int]),
+    "gptq_hptq_quantize": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
+                                     C.c_double, C.c_int, C.c_float, C.c_float,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_size_t, C.c_void_p]),
     "gptq_check": (C.c_int, [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]),
     "gptq_last_error": (C.c_char_p, []),
     "gptq_status_string": (C.c_char_p, [C.c_int]),
@@ -273,6 +282,59 @@ def gptq_ssqr_quantize(W, U, perm, dead, bits, group, block, target, iters, alph
         _ptr(col_idx) if cap else None, _ptr(val) if cap else None, cap, _ptr(alpha),
         _ptr(trace_alpha), _ptr(trace_count), _ptr(loss_row), _ptr(Qdq), _ptr(info),
         _ptr(ws), ws.numel(), _stream(stream, dev)))
+
+
+HPTQ_SYMBOLS = 4096
+HPTQ_SYMBOL_OFFSET = 2048
+
+
+def gptq_hptq_workspace_bytes(m: int, n: int, block: int) -> int:
+    return int(lib().gptq_hptq_workspace_bytes(m, n, block))
+
+
+def gptq_hptq_quantize(W, U, perm, dead, bits, group, block, budget, iters, alpha_lo,
+                       alpha_hi, codes, scale, g_idx, code_len, code_word, row_off,
+                       stream_words, alpha, trace_alpha, trace_bits, loss_row, Qdq, info, ws,
+                       stream=None):
+    """HPTQ: unclipped GPTQ codes, Huffman-coded to a bit budget (see
+    include/gptq_b200.h)."""
+    if W.dtype not in DTYPES:
+        raise TypeError("W must be float32 or bfloat16")
+    _need(W, "W", W.dtype)
+    m, n = W.shape
+    dev = W.device
+    ng = -(-n // group)
+    _need(U, "U", torch.float32, (n, n), dev)
+    _need(perm, "perm", torch.int32, (n,), dev)
+    _need(dead, "dead", torch.uint8, (n,), dev)
+    if codes is not None:
+        _need(codes, "codes", torch.int16, (m, n), dev)
+    _need(scale, "scale", torch.float32, (m, ng), dev)
+    _need(g_idx, "g_idx", torch.int32, (n,), dev)
+    _need(code_len, "code_len", torch.uint8, (HPTQ_SYMBOLS,), dev)
+    if code_word is not None:
+        _need(code_word, "code_word", torch.int64, (HPTQ_SYMBOLS,), dev)
+    _need(row_off, "row_off", torch.int64, (m + 1,), dev)
+    cap = 0 if stream_words is None else stream_words.numel()
+    if cap:
+        _need(stream_words, "stream_words", torch.int32, (cap,), dev)
+    _need(alpha, "alpha", torch.float32, (1,), dev)
+    if trace_alpha is not None:
+        _need(trace_alpha, "trace_alpha", torch.float32, (iters + 1,), dev)
+        _need(trace_bits, "trace_bits", torch.int64, (iters + 1,), dev)
+    if loss_row is not None:
+        _need(loss_row, "loss_row", torch.float32, (m,), dev)
+    if Qdq is not None:
+        _need(Qdq, "Qdq", torch.float32, (m, n), dev)
+    _need(info, "info", torch.int32, (2,), dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _raise(lib().gptq_hptq_quantize(
+        _ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm), _ptr(dead), int(bits),
+        int(group), int(block), float(budget), int(iters), float(alpha_lo), float(alpha_hi),
+        _ptr(codes), _ptr(scale), _ptr(g_idx), _ptr(code_len), _ptr(code_word),
+        _ptr(row_off), _ptr(stream_words) if cap else None, cap, _ptr(alpha),
+        _ptr(trace_alpha), _ptr(trace_bits), _ptr(loss_row), _ptr(Qdq), _ptr(info), _ptr(ws),
+        ws.numel(), _stream(stream, dev)))
 
 
 def gptq_chmc_rank(o: int, i: int, bits: int = 4, gs: int = 128,

@@ -24,6 +24,7 @@ enum KernelKind : int {
   KK_PACK,            // codes → packed words, g_idx, dequantized copy
   KK_CHMC,            // CHMC frontend: activation energies, randomized subspace iteration, residual
   KK_SSQR,            // SSQR: the binary search's state, the outlier list
+  KK_HPTQ,            // HPTQ: histogram, Huffman code and search step, encoder
   KK_COUNT
 };
 

@@ -67,11 +67,18 @@ struct SweepFar {
 // is an outlier: its error is 0, its code byte carries OUTLIER_FLAG on top of
 // the clipped code, its current value is written to Wp at its own position,
 // and it is counted in outl->row_cnt[row] and *outl->total.  bits ≤ 7.
+//
+// outl->unclipped (HPTQ): the same α-scaled step, no clamp and no outliers;
+// every weight's lattice coordinate k = rint(v/s) is written as int16
+// (saturated) to outl->codes16 (m × n, processing order) instead of `codes`,
+// and its error is v − s·k.
 constexpr uint8_t OUTLIER_FLAG = 0x80;
 struct OutlierArgs {
   const float* alpha = nullptr;
   int32_t* row_cnt = nullptr;          // m counts, accumulated over the blocks
   unsigned long long* total = nullptr; // all outliers of the pass
+  bool unclipped = false;
+  int16_t* codes16 = nullptr;
 };
 gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,

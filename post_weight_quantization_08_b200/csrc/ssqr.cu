@@ -17,113 +17,28 @@
 #include <cmath>
 
 #include "kernels.cuh"
+#include "search.cuh"
 
 namespace gptq {
 namespace {
 
-struct SsqrState {
-  float lo, hi;            // the bracket: hi admissible (or α_hi), lo not
-  float a;                 // the α of the next pass
-  int32_t done;            // the search has ended: later passes run at hi
-  unsigned long long count;// outliers of the running pass
-};
-
-size_t ssqr_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, SsqrState** st,
+size_t ssqr_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, SearchState** st,
                       int32_t** row_cnt, char* base) {
   const size_t q = quant_ws_layout(m, n, block, w, base);
   const size_t o_st = q;
-  const size_t o_cnt = align_up(o_st + sizeof(SsqrState), 256);
+  const size_t o_cnt = align_up(o_st + sizeof(SearchState), 256);
   const size_t end = align_up(o_cnt + sizeof(int32_t) * (size_t)m, 256);
   if (base) {
-    *st = reinterpret_cast<SsqrState*>(base + o_st);
+    *st = reinterpret_cast<SearchState*>(base + o_st);
     *row_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
   }
   return end;
 }
 
-__global__ void ssqr_init_kernel(SsqrState* st, float lo, float hi) {
-  st->lo = lo;
-  st->hi = hi;
-  st->a = hi;
-  st->done = 0;
-  st->count = 0ull;
-}
-
-// After pass k (run at st->a with st->count outliers).  Pass 0 evaluates α_hi:
-// over the budget ends the search there.  Later passes evaluate the bracket's
-// midpoint and keep it as hi when admissible, else as lo.  The next midpoint
-// is (lo + hi)/2 rounded once to float32; one equal to an end of the bracket
-// ends the search.
-__global__ void ssqr_step_kernel(SsqrState* st, int k, long long n_max, float* trace_alpha,
+// Between passes: the outlier count against the budget (search.cuh).
+__global__ void ssqr_step_kernel(SearchState* st, int k, long long n_max, float* trace_alpha,
                                  int64_t* trace_count) {
-  const unsigned long long c = st->count;
-  const float a = st->a;
-  const bool was_done = st->done != 0;
-  if (trace_alpha != nullptr) trace_alpha[k] = a;
-  if (trace_count != nullptr) trace_count[k] = was_done ? -1 : (int64_t)c;
-  if (!was_done) {
-    bool done = false;
-    if (k == 0) {
-      done = c > (unsigned long long)n_max;
-    } else if (c <= (unsigned long long)n_max) {
-      st->hi = a;
-    } else {
-      st->lo = a;
-    }
-    if (!done) {
-      const float mid = __double2float_rn(((double)st->lo + (double)st->hi) * 0.5);
-      if (mid <= st->lo || mid >= st->hi) done = true;
-      else st->a = mid;
-    }
-    if (done) {
-      st->done = 1;
-      st->a = st->hi;
-    }
-  }
-  st->count = 0ull;
-}
-
-// row_ptr[0] = 0, row_ptr[r+1] = Σ_{i≤r} cnt[i] (one CTA: a contiguous run of
-// rows per thread, a block-wide scan of the runs' sums).  Reports CAPACITY
-// when the total exceeds the caller's capacity, and writes the chosen α.
-__global__ void __launch_bounds__(1024)
-ssqr_scan_kernel(const int32_t* __restrict__ cnt, int64_t m, int64_t* __restrict__ row_ptr,
-                 int64_t cap, const SsqrState* st, float* alpha_out, int32_t* info) {
-  __shared__ long long wsum[32];
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int64_t per = (m + 1023) / 1024;
-  const int64_t r0 = min(m, (int64_t)t * per), r1 = min(m, r0 + per);
-  long long mine = 0;
-  for (int64_t r = r0; r < r1; ++r) mine += cnt[r];
-  long long x = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) wsum[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    long long w = wsum[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    wsum[lane] = w;
-  }
-  __syncthreads();
-  long long base = x - mine + (warp > 0 ? wsum[warp - 1] : 0ll);
-  if (t == 0) row_ptr[0] = 0;
-  for (int64_t r = r0; r < r1; ++r) {
-    base += cnt[r];
-    row_ptr[r + 1] = base;
-  }
-  if (t == 0) {
-    const long long total = wsum[31];
-    if (total > cap) report(info, GPTQ_ERR_CAPACITY, total < 0x7ffffffe ? total : 0x7ffffffe);
-    if (alpha_out != nullptr) *alpha_out = st->hi;
-  }
+  search_step(st, k, n_max, trace_alpha, trace_count);
 }
 
 // One warp per row: the row's flagged codes in original column order (32
@@ -199,14 +114,14 @@ extern "C" gptq_status gptq_ssqr_quantize(
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   QuantWs w;
-  SsqrState* state = nullptr;
+  SearchState* state = nullptr;
   int32_t* row_cnt = nullptr;
   ssqr_ws_layout(m, n, block, &w, &state, &row_cnt, static_cast<char*>(ws));
   const long long n_max = (long long)std::floor(target * (double)m * (double)n);
 
   st = quant_setup(w, m, n, U, perm, group, block, g_idx, info, s);
   if (st != GPTQ_OK) return st;
-  GPTQ_LAUNCH(KK_SSQR, s, ssqr_init_kernel, 1, 1, 0, state, alpha_lo, alpha_hi);
+  GPTQ_LAUNCH(KK_SSQR, s, search_init_kernel, 1, 1, 0, state, alpha_lo, alpha_hi);
   OutlierArgs search;
   search.alpha = &state->a;
   search.row_cnt = row_cnt;
@@ -226,7 +141,7 @@ extern "C" gptq_status gptq_ssqr_quantize(
   st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, scale, zero,
                   loss_row, &fin, info, s);
   if (st != GPTQ_OK) return st;
-  GPTQ_LAUNCH(KK_SSQR, s, ssqr_scan_kernel, 1, 1024, 0, row_cnt, m, row_ptr, nnz_cap, state,
+  GPTQ_LAUNCH(KK_SSQR, s, row_scan_kernel, 1, 1024, 0, row_cnt, m, row_ptr, nnz_cap, state,
               alpha, info);
   GPTQ_LAUNCH(KK_SSQR, s, ssqr_fill_kernel, (unsigned)ceil_div(m, 8), 256, 0, w.codes, w.pinv,
               w.Wp, m, n, row_ptr, nnz_cap, col_idx, val);

@@ -172,7 +172,11 @@ __device__ __forceinline__ int ord_key_inv(int k) { return k ^ ((k >> 31) & 0x7f
 // weight whose unclipped code leaves the grid is an outlier: it keeps its
 // current value (written to Wp at its own position, the strip being loaded
 // already), contributes no error, and its code byte carries OUTLIER_FLAG.
-template <bool ROWG, bool OUTL>
+// QM selects the quantizer: 0 the hot path's clamp, 1 SSQR's outliers, 2
+// HPTQ's unbounded lattice s·ℤ (same α-scaled step, k = rint(v/s) with no
+// clamp; each int16 coordinate goes to the thread's own row of the strip box
+// it was loaded from, which nothing reads again, and leaves with the block).
+template <bool ROWG, int QM>
 __device__ __forceinline__ void sweep_body(
     const CUtensorMap& tmEhi, const CUtensorMap& tmElo, const CUtensorMap& tmW, int strip_tma,
     const CUtensorMap& tmPhi, const CUtensorMap& tmPlo, const CUtensorMap& tmUhi,
@@ -225,7 +229,7 @@ __device__ __forceinline__ void sweep_body(
   pdl_wait();                           // the strip was written by the previous kernel
   pdl_trigger();
   float alpha = 1.f;
-  if constexpr (OUTL) alpha = *oa.alpha;
+  if constexpr (QM != 0) alpha = *oa.alpha;
   if (t == 0) {
     // the strip, when the rows allow a tensor map: four boxes at (j0 + 32q,
     // r0); columns past n read as zero, and Wp holds whole 128-row boxes
@@ -431,7 +435,7 @@ __device__ __forceinline__ void sweep_body(
       if (xmin == 0.f && xmax == 0.f) { xmin = -1.f; xmax = 1.f; }
       s = __fdiv_rn(xmax - xmin, maxq);
       z = rintf(div_rn(-xmin, s));
-      if constexpr (OUTL) s = __fmul_rn(s, alpha);
+      if constexpr (QM != 0) s = __fmul_rn(s, alpha);
       rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
       klo = -z;
       khi = maxq - z;
@@ -493,9 +497,13 @@ __device__ __forceinline__ void sweep_body(
       // q − z = clamp(rint(v/s), −z, maxq − z) exactly (small integers), so
       // the clamp works on k = q − z and the error takes one FMA
       const float raw = rintf(div_fma(v[i], s, rs));
-      const float k = fminf(fmaxf(raw, klo), khi);
+      const float k = QM == 2 ? raw : fminf(fmaxf(raw, klo), khi);
       float ei = fmaf(-s, k, v[i]) * rdiag[c];
-      if constexpr (OUTL) {
+      if constexpr (QM == 2) {
+        const int qi = __float2int_rn(k);          // the lattice coordinate; saturating
+        const int q16 = max(-32768, min(32767, qi));
+        *reinterpret_cast<int16_t*>(vals + sb * VBOX + t * 128 + i * 2) = (int16_t)q16;
+      } else if constexpr (QM == 1) {
         const bool o = raw != k;        // the unclipped code leaves the grid
         ei = o ? 0.f : ei;
         ocnt += o ? 1 : 0;
@@ -566,7 +574,7 @@ __device__ __forceinline__ void sweep_body(
     if (sb + 1 < nsb) ++issued;
   }
   if (!abort && row < m && loss_row != nullptr) loss_row[row] += loss;
-  if constexpr (OUTL) {
+  if constexpr (QM == 1) {
     if (!abort && row < m) oa.row_cnt[row] += ocnt;
     const int wc = __reduce_add_sync(0xffffffffu, ocnt);
     if (lane == 0 && wc != 0 && !abort) atomicAdd(oa.total, (unsigned long long)wc);
@@ -576,7 +584,25 @@ __device__ __forceinline__ void sweep_body(
 
   // codes out, one warp per row, coalesced (four codes per lane and store
   // when rows and the block width allow it; j0 is a multiple of 32)
-  if (!abort) {
+  if (QM == 2 && !abort) {
+    // int16 codes from the strip boxes: column c of row rr at box c/32,
+    // byte rr·128 + (c mod 32)·2
+    const bool wide = ((n & 3) == 0);
+    for (int rr = warp; rr < RT; rr += RT / 32) {
+      const int64_t r = r0 + rr;
+      if (r >= m) break;
+      const int c = 4 * lane;
+      if (c >= bw) continue;
+      const unsigned char* src = vals + (c >> 5) * VBOX + rr * 128 + (c & 31) * 2;
+      int16_t* dst = oa.codes16 + r * n + j0 + c;
+      if (wide && c + 3 < bw) {
+        *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+      } else {
+        for (int k = 0; k < 4 && c + k < bw; ++k)
+          dst[k] = reinterpret_cast<const int16_t*>(src)[k];
+      }
+    }
+  } else if (!abort) {
     const bool wide = ((n & 3) == 0) && ((bw & 3) == 0);
     for (int rr = warp; rr < RT; rr += RT / 32) {
       const int64_t r = r0 + rr;
@@ -608,7 +634,7 @@ __device__ __forceinline__ void sweep_body(
 // 256 columns per 128-row tile): the two touch different columns, and both
 // take their inputs from earlier launches, so that consecutive sweeps follow
 // each other with nothing between them but the programmatic launch edge.
-template <bool ROWG, bool OUTL>
+template <bool ROWG, int QM>
 __global__ void __launch_bounds__(RT, 1)
 sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ CUtensorMap tmElo,
              const __grid_constant__ CUtensorMap tmW, int strip_tma,
@@ -625,7 +651,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   extern __shared__ unsigned char smraw[];
   const int b = (int)blockIdx.x;
   if (b < nsweep) {
-    sweep_body<ROWG, OUTL>(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp,
+    sweep_body<ROWG, QM>(tmEhi, tmElo, tmW, strip_tma, tmPhi, tmPlo, tmUhi, tmUlo, k0p, kwp,
                            Wp, m, n, j0, bw, pkg, bits, group, ngroups, codes, scale, zero,
                            loss_row, info, perm, oa, b, smraw);
   } else {
@@ -634,7 +660,7 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   }
 }
 
-bool g_attr_set[3] = {false, false, false};   // plain, row groups, outliers
+bool g_attr_set[4] = {false, false, false, false};   // plain, row groups, outliers, unclipped
 
 }  // namespace
 
@@ -660,19 +686,18 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
   const bool rowg = rowgroup_perm != nullptr;
   if (rowg && outl != nullptr)
     return fail(GPTQ_ERR_UNSUPPORTED, "sweep: outliers with output-channel groups");
-  if (outl != nullptr && (!outl->alpha || !outl->row_cnt || !outl->total || bits > 7))
+  if (outl != nullptr && !outl->unclipped &&
+      (!outl->alpha || !outl->row_cnt || !outl->total || bits > 7))
     return fail(GPTQ_ERR_INVALID_ARG, "sweep: outlier arguments");
-  const int variant = rowg ? 1 : (outl != nullptr ? 2 : 0);
+  if (outl != nullptr && outl->unclipped && (!outl->alpha || !outl->codes16))
+    return fail(GPTQ_ERR_INVALID_ARG, "sweep: unclipped-grid arguments");
+  const int variant = rowg ? 1 : (outl == nullptr ? 0 : (outl->unclipped ? 3 : 2));
   if (!g_attr_set[variant]) {
-    if (variant == 1)
-      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<true, false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-    else if (variant == 2)
-      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<false, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-    else
-      GPTQ_CUDA(cudaFuncSetAttribute(sweep_kernel<false, false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
+    const void* fn = variant == 1 ? (const void*)sweep_kernel<true, 0>
+                     : variant == 2 ? (const void*)sweep_kernel<false, 1>
+                     : variant == 3 ? (const void*)sweep_kernel<false, 2>
+                                    : (const void*)sweep_kernel<false, 0>;
+    GPTQ_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
     g_attr_set[variant] = true;
   }
   const OutlierArgs oa = outl != nullptr ? *outl : OutlierArgs();
@@ -721,17 +746,22 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
   const unsigned char* pk = reinterpret_cast<const unsigned char*>(panel);
   const int fxx = fx > 0 ? fx : 1;
   if (variant == 1)
-    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<true, false>), grid, RT, kSmem, th, tl, tw,
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<true, 0>), grid, RT, kSmem, th, tl, tw,
                     strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
                     bits, group, ngroups, codes, scale, zero, loss_row, info, rowgroup_perm, oa,
                     nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
   else if (variant == 2)
-    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, true>), grid, RT, kSmem, th, tl, tw,
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, 1>), grid, RT, kSmem, th, tl, tw,
+                    strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
+                    bits, group, ngroups, codes, scale, zero, loss_row, info,
+                    (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
+  else if (variant == 3)
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, 2>), grid, RT, kSmem, th, tl, tw,
                     strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
                     bits, group, ngroups, codes, scale, zero, loss_row, info,
                     (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
   else
-    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, false>), grid, RT, kSmem, th, tl, tw,
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, 0>), grid, RT, kSmem, th, tl, tw,
                     strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
                     bits, group, ngroups, codes, scale, zero, loss_row, info,
                     (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);

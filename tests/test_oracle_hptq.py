@@ -91,6 +91,8 @@ def test_canonical_code_is_prefix_free_and_round_trips():
 # ---------------------------------------------------------------- the sweep
 
 def _rtn_unclipped_by_loops(W, bits, group, alpha):
+    """U = I: each weight's coordinate rint(w/s) on its group's lattice s·ℤ,
+    s = α·(min-max step), by scalar float32 loops."""
     m, n = W.shape
     maxq = 2 ** bits - 1
     codes = np.zeros((m, n), np.int64)
@@ -102,10 +104,9 @@ def _rtn_unclipped_by_loops(W, bits, group, alpha):
             if lo == 0 and hi == 0:
                 lo, hi = np.float32(-1), np.float32(1)
             s0 = np.float32((hi - lo) / np.float32(maxq))
-            z = np.float32(np.rint(np.float32(-lo) / s0))
             s = np.float32(s0 * np.float32(alpha))
             for c in range(g0, min(g0 + group, n)):
-                codes[r, c] = int(np.rint(np.float32(W[r, c]) / s) + z)
+                codes[r, c] = int(np.rint(np.float32(W[r, c]) / s))
     return codes
 
 
@@ -118,13 +119,16 @@ def test_identity_factor_is_unclipped_rtn(alpha):
 
 
 def test_alpha_one_with_one_column_groups_is_gptq():
+    """group = 1, α = 1: no weight leaves its own row's range, so GPTQ never
+    clips and its q − z is the lattice coordinate k, error for error."""
     rng = np.random.default_rng(2)
     n = 40
     p = G.prepare(_spd(n, rng), 0.01, "act")
     Wp = _heavy(13, n, rng)[:, p["perm"]]
     a = Hq.hptq_blocked(Wp, p["U"], 3, 1, 8, 1.0)
     b = G.gptq_blocked(Wp, p["U"], 3, 1, 8)
-    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["err"], b["err"])
+    assert np.array_equal(a["codes"], b["codes"] - b["zero"].astype(np.int64))
+    assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-15)
 
 
 def _half_step_holds(res, U, group):
@@ -143,7 +147,7 @@ def test_satz5_half_step_for_every_alpha(alpha):
     assert _half_step_holds(res, p["U"], 16)
     n_ = Wp.shape[1]
     g = np.arange(n_) // 16
-    D = Wp - G.dequantize(res["codes"], res["scale"][:, g], res["zero"][:, g])
+    D = Wp - res["scale"][:, g].astype(np.float64) * res["codes"]
     lhs = np.einsum("ij,jk,ik->i", D, p["Hp"], D)
     assert np.allclose(lhs, np.sum(res["err"] ** 2, axis=1), rtol=1e-9)
 
@@ -198,13 +202,13 @@ def test_follow_accepts_its_own_codes_and_flags_a_planted_one():
     p = G.prepare(_spd(n, rng), 0.01, "act")
     Wp = _heavy(30, n, rng)[:, p["perm"]]
     ref = Hq.hptq_blocked(Wp, p["U"], 3, 32, 64, 1.5)
-    ok = Hq.follow_hptq(Wp, p["U"], 3, 32, 64, 1.5, ref["codes"], ref["scale"], ref["zero"])
+    ok = Hq.follow_hptq(Wp, p["U"], 3, 32, 64, 1.5, ref["codes"], ref["scale"])
     assert ok["n_diff"] == 0 and ok["n_bad"] == 0 and ok["max_scale_rel"] == 0.0
     frac = np.abs(ref["pre"] - np.floor(ref["pre"]) - 0.5)
     r, j = np.unravel_index(np.argmax(frac), frac.shape)
     bad = ref["codes"].copy()
     bad[r, j] += 1
-    assert Hq.follow_hptq(Wp, p["U"], 3, 32, 64, 1.5, bad, ref["scale"], ref["zero"])["n_bad"] >= 1
+    assert Hq.follow_hptq(Wp, p["U"], 3, 32, 64, 1.5, bad, ref["scale"])["n_bad"] >= 1
 
 
 # ---------------------------------------------------------------- mutations
@@ -224,7 +228,7 @@ def _wrong_merge(hist):
     return depth
 
 
-@pytest.mark.parametrize("kind", ["wrong_merge", "clipped", "zero_from_adjusted_step",
+@pytest.mark.parametrize("kind", ["wrong_merge", "clipped", "zero_point_kept",
                                   "length_off_by_one"])
 def test_pins_catch_planted_mistakes(kind, monkeypatch):
     failures = 0
@@ -244,18 +248,13 @@ def test_pins_catch_planted_mistakes(kind, monkeypatch):
             L = Hq.huffman_lengths(h)
             failures += Hq.cost(h, L) != _optimal_cost_by_search(counts)
     else:
-        orig_q = G.quantize_column
-        orig_p = G.group_params
-        if kind == "clipped":
-            monkeypatch.setattr(G, "quantize_column",
-                                lambda cur, s, z, bits, clip=True: orig_q(cur, s, z, bits, True))
-        else:
-            def gp(cur, bits):
-                s0, z = orig_p(cur, bits)
-                v = np.asarray(cur, np.float32)
-                xmin = np.minimum(v.min(axis=1), np.float32(0))
-                return s0, np.rint(-xmin / (s0 * np.float32(0.4))).astype(np.float32)
-            monkeypatch.setattr(G, "group_params", gp)
+        orig_k = Hq.lattice_column
+        if kind == "clipped":               # the coordinate clamped to the nominal range
+            monkeypatch.setattr(Hq, "lattice_column",
+                                lambda cur, s: np.clip(orig_k(cur, s), -4, 3).astype(np.float32))
+        else:                               # a zero point of 1 added to every code
+            monkeypatch.setattr(Hq, "lattice_column",
+                                lambda cur, s: (orig_k(cur, s) + 1).astype(np.float32))
         W = _heavy(9, 64, rng)
         res = Hq.hptq_blocked(W, np.eye(64), 3, 16, 32, 0.4)
         failures += not np.array_equal(res["codes"], _rtn_unclipped_by_loops(W, 3, 16, 0.4))
