@@ -990,6 +990,189 @@ def run_ssqr(args, rank, world, local):
     }, probs
 
 
+# ---------------------------------------------------------------- HPTQ
+
+HPTQ_METRIC = ("HPTQ weights compressed/sec (params/s incl. Hessian, the binary search's "
+               "sweeps and the Huffman coding) & % of roofline, 1 B200")
+HPTQ_BITS, HPTQ_BUDGET, HPTQ_ITERS, HPTQ_LO, HPTQ_HI = 4, 3.125, 12, 1.0 / 16, 16.0
+
+
+class HptqLayer:
+    """Device buffers of one layer under HPTQ ("The Geometry of LLM
+    Quantization: GPTQ as Babai's Nearest Plane Algorithm", §3): per Hessian
+    its factor, per weight matrix its lattice coordinates, scales, Huffman
+    table, row offsets and bit stream (each matrix meets the budget on its
+    own)."""
+
+    def __init__(self, probs, device):
+        import post_weight_quantization_08_b200 as g
+        self.g = g
+        self.items = []
+        for p in probs:
+            n = p.n
+            it = {"p": p, "X": p.X.to(device).contiguous(),
+                  "H": torch.zeros(n, n, dtype=torch.float32, device=device),
+                  "perm": torch.empty(n, dtype=torch.int32, device=device),
+                  "U": torch.empty(n, n, dtype=torch.float32, device=device),
+                  "dead": torch.empty(n, dtype=torch.uint8, device=device),
+                  "info_h": torch.zeros(2, dtype=torch.int32, device=device),
+                  "info_p": torch.zeros(2, dtype=torch.int32, device=device),
+                  "ws_p": g.workspace(g.gptq_prepare_workspace_bytes(n), device),
+                  "stream": torch.cuda.Stream(device=device), "parts": []}
+            row0 = 0
+            for name, rows in p.parts:
+                W = p.W[row0:row0 + rows].to(device).contiguous()
+                row0 += rows
+                ng = -(-n // p.group)
+                cap = int(HPTQ_BUDGET * rows * n) // 32 + rows + 1
+                it["parts"].append({
+                    "name": name, "W": W,
+                    "codes": torch.empty(rows, n, dtype=torch.int16, device=device),
+                    "scale": torch.empty(rows, ng, dtype=torch.float32, device=device),
+                    "g_idx": torch.empty(n, dtype=torch.int32, device=device),
+                    "code_len": torch.empty(g.HPTQ_SYMBOLS, dtype=torch.uint8, device=device),
+                    "code_word": torch.empty(g.HPTQ_SYMBOLS, dtype=torch.int64, device=device),
+                    "row_off": torch.empty(rows + 1, dtype=torch.int64, device=device),
+                    "bitstream": torch.empty(cap, dtype=torch.int32, device=device),
+                    "alpha": torch.empty(1, dtype=torch.float32, device=device),
+                    "loss": torch.empty(rows, dtype=torch.float32, device=device),
+                    "info_q": torch.zeros(2, dtype=torch.int32, device=device),
+                    "ws_q": g.workspace(g.gptq_hptq_workspace_bytes(rows, n, p.block), device),
+                    "stream": torch.cuda.Stream(device=device),
+                })
+            self.items.append(it)
+
+    def run_problem(self, it, serial=False):
+        g, p, s = self.g, it["p"], it["stream"]
+        with torch.cuda.stream(s):
+            it["H"].zero_()
+        g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
+        g.gptq_prepare(it["H"], p.damp, "act", it["perm"], it["U"], it["dead"],
+                       it["info_p"], it["ws_p"], s)
+        prep_done = torch.cuda.Event()
+        prep_done.record(s)
+        for q in it["parts"]:
+            qs = s if serial else q["stream"]
+            if not serial:
+                qs.wait_event(prep_done)
+            g.gptq_hptq_quantize(q["W"], it["U"], it["perm"], it["dead"], HPTQ_BITS, p.group,
+                                 p.block, HPTQ_BUDGET, HPTQ_ITERS, HPTQ_LO, HPTQ_HI, q["codes"],
+                                 q["scale"], q["g_idx"], q["code_len"], q["code_word"],
+                                 q["row_off"], q["bitstream"], q["alpha"], None, None, q["loss"],
+                                 None, q["info_q"], q["ws_q"], qs)
+            if not serial:
+                e = torch.cuda.Event()
+                e.record(qs)
+                s.wait_event(e)
+
+    step = ChmcLayer.step
+    step_serial = ChmcLayer.step_serial
+    check = SsqrLayer.check
+
+
+def hptq_work(layer):
+    """Algorithmic work per kernel kind for one HPTQ step: as SSQR's, with the
+    sweep writing 2-byte coordinates, and the hptq kind's bytes: per pass the
+    histogram (2 B per weight), at the end the row bit counts and the encoder
+    (2 B per weight each, plus the stream written) and the original-order
+    coordinates (2 B in, 2 B out per weight)."""
+    w = {k: 0.0 for k in ("hessian", "cholesky", "sweep", "trailing", "ingest", "hptq")}
+    passes = HPTQ_ITERS + 2
+    for it in layer.items:
+        p = it["p"]
+        n, T, block = p.n, p.T, p.block
+        w["hessian"] += T * n * (n + 1)
+        N = -(-n // 64)
+        for k in range(N):
+            r = N - k - 1
+            w["cholesky"] += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
+            w["cholesky"] += 2 * 64 ** 3 / 3
+        fused = n % 4 == 0 and n > block
+        for q in it["parts"]:
+            m = q["W"].shape[0]
+            if fused:
+                w["trailing"] += 12 * n * n
+            for j0 in range(0, n, block):
+                bw = min(block, n - j0)
+                n2 = n - j0 - bw
+                w["sweep"] += passes * (10 * m * bw + 4 * bw * bw + 5 * m * (-(-bw // p.group)))
+                if n2 > 0:
+                    w["sweep" if fused else "trailing"] += passes * (8 * m * n2 + 4 * m * bw
+                                                                     + 4 * bw * n2)
+            w["ingest"] += passes * m * n * (q["W"].element_size() + 4)
+            w["hptq"] += passes * 2 * m * n + 8 * m * n + HPTQ_BUDGET * m * n / 8
+    units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s", "sweep": "GB/s", "trailing": "GB/s",
+             "ingest": "GB/s", "hptq": "GB/s"}
+    return {k: (units[k], v) for k, v in w.items()}
+
+
+def hptq_cpu_baseline(probs, budget_s: float = 20.0):
+    """The HPTQ oracle on the layer's matrices in order (Hessian from X, the
+    whole binary search with a Huffman code per pass, the encoding), until the
+    time budget is spent; params/s over the matrices completed."""
+    from oracle import gptq as og
+    from oracle import hptq as oh
+    t0 = time.perf_counter()
+    total, done = 0, []
+    for p in probs:
+        H = og.hessian(p.X.to(torch.float64).numpy())
+        prep = og.prepare(H, p.damp, "act")
+        row0 = 0
+        for name, rows in p.parts:
+            W = p.W[row0:row0 + rows].to(torch.float64).numpy()
+            row0 += rows
+            out = oh.hptq_layer(W, H, bits=HPTQ_BITS, group=p.group, block=p.block,
+                                damp=p.damp, budget=HPTQ_BUDGET, iters=HPTQ_ITERS,
+                                alpha_lo=HPTQ_LO, alpha_hi=HPTQ_HI, prep=prep)
+            oh.encode(out["codes"][:8], out["lengths"])      # the codec, on a row sample
+            total += rows * p.n
+            done.append(name)
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(total / dt, 1), "unit": "params/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"the layer's matrices in order until {budget_s:.0f} s: {', '.join(done)} "
+                      f"({dt:.1f} s, Hessians and factors included; the bit stream of 8 rows "
+                      f"per matrix)"}
+
+
+def run_hptq(args, rank, world, local):
+    """HPTQ over the layer: device-timed graph replay and the per-kernel event
+    profile, as for SSQR."""
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = CONFIGS[args.config]
+    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=HPTQ_BITS, order="act")
+    layer = HptqLayer(probs, device)
+    params = sum(p.params for p in probs)
+    dev_ms, launches, kernels, kms, clk = _time_frontend(args, layer, device, world, local,
+                                                         hptq_work(layer))
+    parts = [q for it in layer.items for q in it["parts"]]
+    alphas = {q["name"]: float(q["alpha"].cpu()[0]) for q in parts}
+    bpw = {q["name"]: round(int(q["row_off"][-1]) / q["W"].numel(), 4) for q in parts}
+    total_params = sum_over_ranks(params * args.steps, world, device)
+    return {
+        "metric": HPTQ_METRIC, "value": round(total_params / (dev_ms / 1e3), 1),
+        "unit": "params/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep, int16 codes",
+        "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
+        "config": {"workload": f"{cfg['name']} HPTQ: lattice from the {HPTQ_BITS}-bit min-max "
+                               f"step, group {probs[0].group}, act-order, budget {HPTQ_BUDGET} "
+                               f"bits/weight per matrix, {HPTQ_ITERS} bisection steps on alpha in "
+                               f"[{HPTQ_LO}, {HPTQ_HI}], block {probs[0].block}",
+                   "params_per_step_per_gpu": params, "alpha": alphas, "bits_per_weight": bpw,
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "launch": "CUDA graph replay per step"},
+        "gpu_launches": int(launches * args.steps),
+        "kernels": kernels, "kernels_ms_per_step": kms, "clocks": clk,
+    }, probs
+
+
 def _time_frontend(args, layer, device, world, local, work):
     """Warm up, capture one step in a CUDA graph, time K replays with the L2
     flushed between them (max over ranks), then time every kernel kind with
@@ -1136,9 +1319,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--frontend", default="gptq", choices=["gptq", "chmc", "ssqr"],
-                    help="chmc: the CHMC frontend over the layer; ssqr: SSQR over the "
-                         "layer (separate metrics)")
+    ap.add_argument("--frontend", default="gptq", choices=["gptq", "chmc", "ssqr", "hptq"],
+                    help="chmc: the CHMC frontend over the layer; ssqr / hptq: SSQR / HPTQ "
+                         "over the layer (separate metrics)")
     ap.add_argument("--order", default=None,
                     choices=["natural", "act", "reverse", "minpivot"],
                     help="processing order for every problem (default: the workload's)")
@@ -1167,6 +1350,10 @@ def main(argv=None):
             out, probs = run_ssqr(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = ssqr_cpu_baseline(probs)
+        elif args.frontend == "hptq":
+            out, probs = run_hptq(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = hptq_cpu_baseline(probs)
         else:
             out, probs, _ = run_ours(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
