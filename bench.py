@@ -847,6 +847,13 @@ class SsqrLayer:
                     "stream": torch.cuda.Stream(device=device),
                 })
             self.items.append(it)
+        # the matrices with the most blocks per pass set the step's critical
+        # path: their searches look ahead (three passes side by side), the
+        # others take one pass a step and leave the SMs to them
+        most = max(-(-it["p"].n // it["p"].block) for it in self.items)
+        for it in self.items:
+            for q in it["parts"]:
+                q["lookahead"] = -(-it["p"].n // it["p"].block) == most
 
     def run_problem(self, it, serial=False):
         """Hessian and factor on the problem's stream, then each matrix's
@@ -867,7 +874,7 @@ class SsqrLayer:
                                  p.block, SSQR_TARGET, SSQR_ITERS, SSQR_LO, SSQR_HI,
                                  q["qweight"], q["scale"], q["zero"], q["g_idx"], q["row_ptr"],
                                  q["col_idx"], q["val"], q["alpha"], None, None, q["loss"],
-                                 None, q["info_q"], q["ws_q"], qs)
+                                 None, q["info_q"], q["ws_q"], qs, q["lookahead"])
             if not serial:
                 e = torch.cuda.Event()
                 e.record(qs)
@@ -1041,6 +1048,13 @@ class HptqLayer:
                     "stream": torch.cuda.Stream(device=device),
                 })
             self.items.append(it)
+        # the matrices with the most blocks per pass set the step's critical
+        # path: their searches look ahead (three passes side by side), the
+        # others take one pass a step and leave the SMs to them
+        most = max(-(-it["p"].n // it["p"].block) for it in self.items)
+        for it in self.items:
+            for q in it["parts"]:
+                q["lookahead"] = -(-it["p"].n // it["p"].block) == most
 
     def run_problem(self, it, serial=False):
         g, p, s = self.g, it["p"], it["stream"]
@@ -1059,7 +1073,7 @@ class HptqLayer:
                                  p.block, HPTQ_BUDGET, HPTQ_ITERS, HPTQ_LO, HPTQ_HI, q["codes"],
                                  q["scale"], q["g_idx"], q["code_len"], q["code_word"],
                                  q["row_off"], q["bitstream"], q["alpha"], None, None, q["loss"],
-                                 None, q["info_q"], q["ws_q"], qs)
+                                 None, q["info_q"], q["ws_q"], qs, q["lookahead"])
             if not serial:
                 e = torch.cuda.Event()
                 e.record(qs)

@@ -305,7 +305,13 @@ size_t gptq_ssqr_workspace_bytes(int64_t m, int64_t n, int block);
  *              and makes mid the new hi when it has at most n_max outliers,
  *              else the new lo; a mid equal to lo or hi ends the search.  A
  *              last pass at hi writes the outputs.  Cost: iters + 2 sweeps of
- *              the layer.
+ *              the layer, one after another.
+ *   lookahead  0: one pass per bisection step.  1: each round runs the
+ *              midpoint and both quarter points of the step after it side by
+ *              side (on `stream` and two streams forked from it, joined before
+ *              the call returns) and takes both steps: the same steps and
+ *              result, about half the passes in sequence and 1.5 times the
+ *              work; worth it when the GPU has SMs to spare beside the call.
  *   target     outlier density, 0..1.  iters 0..64.
  *   alpha_lo, alpha_hi   the bracket, 0 < alpha_lo ≤ alpha_hi ≤ 16.
  *   row_ptr    int64[m + 1], output: CSR row pointers of the outliers
@@ -327,7 +333,7 @@ size_t gptq_ssqr_workspace_bytes(int64_t m, int64_t n, int block);
 gptq_status gptq_ssqr_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
                                const float* U, const int32_t* perm, const uint8_t* dead,
                                int bits, int group, int block, double target, int iters,
-                               float alpha_lo, float alpha_hi, uint32_t* qweight,
+                               float alpha_lo, float alpha_hi, int lookahead, uint32_t* qweight,
                                float* scale, uint8_t* zero, int32_t* g_idx,
                                int64_t* row_ptr, int32_t* col_idx, float* val,
                                int64_t nnz_cap, float* alpha, float* trace_alpha,
@@ -368,6 +374,7 @@ size_t gptq_hptq_workspace_bytes(int64_t m, int64_t n, int block);
  *              ≤ floor(budget·m·n): alpha_hi (the coarsest grid) first, then up
  *              to `iters` bisection steps; a last pass at the chosen alpha is
  *              encoded.  Cost: iters + 2 sweeps of the layer.
+ *   lookahead  as gptq_ssqr_quantize's.
  *   budget     payload bits per weight, (0, 64].  iters 0..64.
  *   alpha_lo, alpha_hi   0 < alpha_lo ≤ alpha_hi ≤ 256.
  *   codes      m×n int16 or NULL, output: q in ORIGINAL column order.
@@ -393,7 +400,8 @@ size_t gptq_hptq_workspace_bytes(int64_t m, int64_t n, int block);
 gptq_status gptq_hptq_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
                                const float* U, const int32_t* perm, const uint8_t* dead,
                                int bits, int group, int block, double budget, int iters,
-                               float alpha_lo, float alpha_hi, int16_t* codes, float* scale,
+                               float alpha_lo, float alpha_hi, int lookahead, int16_t* codes,
+                               float* scale,
                                int32_t* g_idx, uint8_t* code_len,
                                uint64_t* code_word, int64_t* row_off, uint32_t* stream_words,
                                int64_t stream_cap, float* alpha, float* trace_alpha,

@@ -175,7 +175,8 @@ def ssqr_quantize(W: torch.Tensor, prep: dict, bits: int = 3, group: int = 128,
                   block: int = 128, target: float = 0.01, iters: int = 16,
                   alpha_lo: float = 1.0 / 16, alpha_hi: float = 1.0, nnz_cap: int | None = None,
                   want_loss: bool = True, want_qdq: bool = False, want_trace: bool = False,
-                  ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+                  ws: torch.Tensor | None = None, stream=None, check: bool = True,
+                  lookahead: bool = True) -> dict:
     """GPTQ with the overflowing weights kept: packed inlier codes, scales,
     zeros, g_idx and the outliers in CSR (row_ptr, col_idx, val, original
     columns).  ``nnz_cap`` (default floor(target·m·n), at least 1) sizes the
@@ -207,7 +208,7 @@ def ssqr_quantize(W: torch.Tensor, prep: dict, bits: int = 3, group: int = 128,
                        iters, alpha_lo, alpha_hi, out["qweight"], out["scale"], out["zero"],
                        out["g_idx"], out["row_ptr"], out["col_idx"], out["val"], out["alpha"],
                        out["trace_alpha"], out["trace_count"], out["loss_row"], out["Qdq"],
-                       out["info"], ws, stream)
+                       out["info"], ws, stream, lookahead)
     if check:
         _raise_info(out["info"], stream, "gptq_ssqr_quantize")
         nnz = int(out["row_ptr"][-1])
@@ -224,7 +225,8 @@ def hptq_quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
                   alpha_lo: float = 1.0 / 16, alpha_hi: float = 16.0,
                   stream_cap: int | None = None, want_loss: bool = True,
                   want_qdq: bool = False, want_codes: bool = True, want_trace: bool = False,
-                  ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+                  ws: torch.Tensor | None = None, stream=None, check: bool = True,
+                  lookahead: bool = True) -> dict:
     """GPTQ on the unbounded lattice s·ℤ, Huffman-coded: the integers
     (original column order), scales, g_idx, the code table (length and canonical word
     per symbol), the row bit offsets and the bit stream.  ``stream_cap``
@@ -257,7 +259,7 @@ def hptq_quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
                        out["g_idx"], out["code_len"], out["code_word"], out["row_off"],
                        out["stream"] if stream_cap > 0 else None, out["alpha"],
                        out["trace_alpha"], out["trace_bits"], out["loss_row"], out["Qdq"],
-                       out["info"], ws, stream)
+                       out["info"], ws, stream, lookahead)
     if check:
         _raise_info(out["info"], stream, "gptq_hptq_quantize")
         nbits = int(out["row_off"][-1])

@@ -53,7 +53,7 @@ _SIGS = {
     "gptq_ssqr_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int]),
     "gptq_ssqr_quantize": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
-                                     C.c_double, C.c_int, C.c_float, C.c_float,
+                                     C.c_double, C.c_int, C.c_float, C.c_float, C.c_int,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
@@ -62,7 +62,7 @@ _SIGS = {
     "gptq_hptq_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64, C.c_int]),
     "gptq_hptq_quantize": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
-                                     C.c_double, C.c_int, C.c_float, C.c_float,
+                                     C.c_double, C.c_int, C.c_float, C.c_float, C.c_int,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
@@ -243,7 +243,8 @@ def gptq_ssqr_workspace_bytes(m: int, n: int, block: int) -> int:
 
 def gptq_ssqr_quantize(W, U, perm, dead, bits, group, block, target, iters, alpha_lo,
                        alpha_hi, qweight, scale, zero, g_idx, row_ptr, col_idx, val, alpha,
-                       trace_alpha, trace_count, loss_row, Qdq, info, ws, stream=None):
+                       trace_alpha, trace_count, loss_row, Qdq, info, ws, stream=None,
+                       lookahead=1):
     """SSQR: GPTQ with kept outliers and a binary search on the scale factor
     (see include/gptq_b200.h)."""
     if W.dtype not in DTYPES:
@@ -278,7 +279,7 @@ def gptq_ssqr_quantize(W, U, perm, dead, bits, group, block, target, iters, alph
     _raise(lib().gptq_ssqr_quantize(
         _ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm), _ptr(dead), int(bits),
         int(group), int(block), float(target), int(iters), float(alpha_lo), float(alpha_hi),
-        _ptr(qweight), _ptr(scale), _ptr(zero), _ptr(g_idx), _ptr(row_ptr),
+        int(bool(lookahead)), _ptr(qweight), _ptr(scale), _ptr(zero), _ptr(g_idx), _ptr(row_ptr),
         _ptr(col_idx) if cap else None, _ptr(val) if cap else None, cap, _ptr(alpha),
         _ptr(trace_alpha), _ptr(trace_count), _ptr(loss_row), _ptr(Qdq), _ptr(info),
         _ptr(ws), ws.numel(), _stream(stream, dev)))
@@ -295,7 +296,7 @@ def gptq_hptq_workspace_bytes(m: int, n: int, block: int) -> int:
 def gptq_hptq_quantize(W, U, perm, dead, bits, group, block, budget, iters, alpha_lo,
                        alpha_hi, codes, scale, g_idx, code_len, code_word, row_off,
                        stream_words, alpha, trace_alpha, trace_bits, loss_row, Qdq, info, ws,
-                       stream=None):
+                       stream=None, lookahead=1):
     """HPTQ: unclipped GPTQ codes, Huffman-coded to a bit budget (see
     include/gptq_b200.h)."""
     if W.dtype not in DTYPES:
@@ -331,7 +332,7 @@ def gptq_hptq_quantize(W, U, perm, dead, bits, group, block, budget, iters, alph
     _raise(lib().gptq_hptq_quantize(
         _ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm), _ptr(dead), int(bits),
         int(group), int(block), float(budget), int(iters), float(alpha_lo), float(alpha_hi),
-        _ptr(codes), _ptr(scale), _ptr(g_idx), _ptr(code_len), _ptr(code_word),
+        int(bool(lookahead)), _ptr(codes), _ptr(scale), _ptr(g_idx), _ptr(code_len), _ptr(code_word),
         _ptr(row_off), _ptr(stream_words) if cap else None, cap, _ptr(alpha),
         _ptr(trace_alpha), _ptr(trace_bits), _ptr(loss_row), _ptr(Qdq), _ptr(info), _ptr(ws),
         ws.numel(), _stream(stream, dev)))

@@ -14,7 +14,9 @@
 // Every pass of the device-side search (search.cuh) is: the sweep's
 // unclipped variant at α (int16 coordinates), a histogram of the codes over a
 // window of GPTQ_HPTQ_SYMBOLS symbols, and a one-CTA Huffman construction
-// whose optimal cost (coded bits) drives the bisection step.  A last pass at
+// whose optimal cost (coded bits) drives the bisection; after the pass at
+// α_hi, a round runs the midpoint and both quarter points of the next level
+// side by side and takes two steps.  A last pass at
 // the chosen α is encoded: canonical codes, per-row bit counts, their scan,
 // and one warp per row writing its codes most significant bit first.
 #include <algorithm>
@@ -30,36 +32,52 @@ constexpr int NSYM = GPTQ_HPTQ_SYMBOLS;
 constexpr int SYM0 = GPTQ_HPTQ_SYMBOL_OFFSET;
 constexpr int MAXLEN = 64;
 
+// The workspace: three working sets (slot 0 the call's, with the U-derived
+// parts; slots 1 and 2 for the quarter-point passes of a round), and per slot
+// the lattice coordinates, histogram, scales and zero points of its pass
+// (slot 0's scales are the caller's; the zero points of the min-max steps are
+// written by the sweep and unused by the unbounded grid).
 struct HptqWs {
+  QuantWs w[3];
   SearchState* st;
-  int16_t* codes16;             // m × n lattice coordinates, processing order
-  uint8_t* zero;                // m × ngroups zero points of the min-max steps (unused
-                                // by the unbounded grid, written by the sweep)
-  unsigned long long* hist;     // NSYM counts of the running pass
+  int16_t* codes16[3];          // m × n lattice coordinates, processing order
+  unsigned long long* hist[3];  // NSYM counts of the slot's pass
+  float* scale[3];
+  uint8_t* zero[3];
   unsigned char* lens;          // NSYM code lengths (0: unused symbol)
   unsigned long long* canon;    // NSYM canonical code words (right-aligned)
   int32_t* rowbits;             // m coded bits per row
 };
 
-size_t hptq_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, HptqWs* h, char* base) {
-  size_t off = quant_ws_layout(m, n, block, w, base);
+size_t hptq_ws_layout(int64_t m, int64_t n, int block, HptqWs* h, char* base) {
+  size_t off = quant_ws_layout(m, n, block, h ? &h->w[0] : nullptr, base);
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off = align_up(off + bytes, 256);
     return o;
   };
+  const size_t ngmax = (size_t)ceil_div(n, 32);        // group ≥ 32
   const size_t o_st = take(sizeof(SearchState));
-  const size_t o_c = take(sizeof(int16_t) * (size_t)m * (size_t)n);
-  const size_t o_h = take(sizeof(unsigned long long) * NSYM);
+  size_t o_c[3], o_h[3], o_s[3], o_z[3], o_slot[3];
+  for (int k = 0; k < 3; ++k) {
+    o_c[k] = take(sizeof(int16_t) * (size_t)m * (size_t)n);
+    o_h[k] = take(sizeof(unsigned long long) * NSYM);
+    o_s[k] = take(sizeof(float) * (size_t)m * ngmax);
+    o_z[k] = take((size_t)m * ngmax);
+    o_slot[k] = k ? take(quant_slot_layout(m, n, nullptr, nullptr, nullptr)) : 0;
+  }
   const size_t o_l = take(NSYM);
   const size_t o_k = take(sizeof(unsigned long long) * NSYM);
   const size_t o_r = take(sizeof(int32_t) * (size_t)m);
-  const size_t o_z = take((size_t)m * (size_t)ceil_div(n, 32));
   if (base && h) {
-    h->zero = reinterpret_cast<uint8_t*>(base + o_z);
     h->st = reinterpret_cast<SearchState*>(base + o_st);
-    h->codes16 = reinterpret_cast<int16_t*>(base + o_c);
-    h->hist = reinterpret_cast<unsigned long long*>(base + o_h);
+    for (int k = 0; k < 3; ++k) {
+      h->codes16[k] = reinterpret_cast<int16_t*>(base + o_c[k]);
+      h->hist[k] = reinterpret_cast<unsigned long long*>(base + o_h[k]);
+      h->scale[k] = reinterpret_cast<float*>(base + o_s[k]);
+      h->zero[k] = reinterpret_cast<uint8_t*>(base + o_z[k]);
+      if (k) quant_slot_layout(m, n, &h->w[0], &h->w[k], base + o_slot[k]);
+    }
     h->lens = reinterpret_cast<unsigned char*>(base + o_l);
     h->canon = reinterpret_cast<unsigned long long*>(base + o_k);
     h->rowbits = reinterpret_cast<int32_t*>(base + o_r);
@@ -99,8 +117,8 @@ hptq_hist_kernel(const int16_t* __restrict__ codes, int64_t total,
 }
 
 // One CTA: the optimal prefix code of the pass's histogram, its cost, and
-// (k ≥ 0) the bisection step on that cost; with `final`, the code lengths
-// and canonical code words for the encoder.
+// (k ≥ 0) the bisection step on that cost, else the cost into *cost_out; with
+// `final`, the code lengths and canonical code words for the encoder.
 //  1. the used symbols, compacted in symbol order (a block scan);
 //  2. sorted by (count, symbol) by rank counting;
 //  3. Huffman's construction with two queues (sorted leaves, internal nodes
@@ -115,6 +133,7 @@ constexpr size_t HUF_SMEM = (size_t)NSYM * 8 * 3 + (size_t)NSYM * 2 * 2 + (size_
 static_assert(HUF_SMEM <= 227 * 1024, "shared memory per CTA");
 __global__ void __launch_bounds__(1024)
 hptq_huffman_kernel(const unsigned long long* __restrict__ hist, SearchState* st, int k,
+                    unsigned long long* cost_out,
                     long long limit, float* trace_alpha, int64_t* trace_count, int final_pass,
                     unsigned char* __restrict__ lens_out, unsigned long long* __restrict__ canon_out,
                     int32_t* info) {
@@ -236,8 +255,12 @@ hptq_huffman_kernel(const unsigned long long* __restrict__ hist, SearchState* st
     unsigned long long c = 0ull;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) c += red[w];
     if (bad_len) report(info, GPTQ_ERR_UNSUPPORTED, 0);
-    st->count = c;
-    if (k >= 0) search_step(st, k, limit, trace_alpha, trace_count);
+    if (k >= 0) {
+      st->count = c;
+      search_step(st, k, limit, trace_alpha, trace_count);
+    } else if (cost_out != nullptr) {
+      *cost_out = c;
+    }
   }
   if (!final_pass) return;
 
@@ -365,32 +388,33 @@ hptq_out_kernel(const int16_t* __restrict__ codes16, const int32_t* __restrict__
 
 bool g_huf_attr = false;
 
-// One pass at *alpha: sweep (unclipped), histogram, Huffman (+ the step).
-gptq_status hptq_pass(const QuantWs& w, const HptqWs& h, const void* W, int w_dtype, int64_t m,
+// One pass of slot `slot` at *alpha: sweep (unclipped), histogram, Huffman;
+// k ≥ 0: the bisection step on its cost; k < 0: the cost into *cost_out.
+gptq_status hptq_pass(const HptqWs& h, int slot, const void* W, int w_dtype, int64_t m,
                       int64_t n, const float* U, const int32_t* perm, const uint8_t* dead,
-                      int bits, int group, int block, float* scale,
-                      float* loss_row, const float* alpha, int k, long long limit,
+                      int bits, int group, int block, float* scale, float* loss_row,
+                      const float* alpha, int k, unsigned long long* cost_out, long long limit,
                       float* trace_alpha, int64_t* trace_count, int final_pass, int32_t* info,
                       cudaStream_t s) {
   OutlierArgs oa;
   oa.alpha = alpha;
   oa.unclipped = true;
-  oa.codes16 = h.codes16;
-  GPTQ_CUDA(cudaMemsetAsync(h.hist, 0, sizeof(unsigned long long) * NSYM, s));
-  gptq_status st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, scale,
-                              h.zero, loss_row, &oa, info, s);
+  oa.codes16 = h.codes16[slot];
+  GPTQ_CUDA(cudaMemsetAsync(h.hist[slot], 0, sizeof(unsigned long long) * NSYM, s));
+  gptq_status st = quant_pass(h.w[slot], W, w_dtype, m, n, U, perm, dead, bits, group, block, 0,
+                              scale, h.zero[slot], loss_row, &oa, info, s);
   if (st != GPTQ_OK) return st;
   const int64_t total = m * n;
   const unsigned gh = (unsigned)std::min<int64_t>(ceil_div(total, 512 * 8), 148 * 4);
-  GPTQ_LAUNCH(KK_HPTQ, s, hptq_hist_kernel, gh > 0 ? gh : 1, 512, 0, h.codes16, total, h.hist,
-              info);
+  GPTQ_LAUNCH(KK_HPTQ, s, hptq_hist_kernel, gh > 0 ? gh : 1, 512, 0, h.codes16[slot], total,
+              h.hist[slot], info);
   if (!g_huf_attr) {
     GPTQ_CUDA(cudaFuncSetAttribute(hptq_huffman_kernel,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HUF_SMEM));
     g_huf_attr = true;
   }
-  GPTQ_LAUNCH(KK_HPTQ, s, hptq_huffman_kernel, 1, 1024, HUF_SMEM, h.hist, h.st, k, limit,
-              trace_alpha, trace_count, final_pass, h.lens, h.canon, info);
+  GPTQ_LAUNCH(KK_HPTQ, s, hptq_huffman_kernel, 1, 1024, HUF_SMEM, h.hist[slot], h.st, k,
+              cost_out, limit, trace_alpha, trace_count, final_pass, h.lens, h.canon, info);
   return GPTQ_OK;
 }
 
@@ -401,13 +425,13 @@ using namespace gptq;
 
 extern "C" size_t gptq_hptq_workspace_bytes(int64_t m, int64_t n, int block) {
   if (m < 1 || n < 1 || block < 1) return 0;
-  return hptq_ws_layout(m, n, block, nullptr, nullptr, nullptr);
+  return hptq_ws_layout(m, n, block, nullptr, nullptr);
 }
 
 extern "C" gptq_status gptq_hptq_quantize(
     const void* W, int w_dtype, int64_t m, int64_t n, const float* U, const int32_t* perm,
     const uint8_t* dead, int bits, int group, int block, double budget, int iters,
-    float alpha_lo, float alpha_hi, int16_t* codes, float* scale,
+    float alpha_lo, float alpha_hi, int lookahead, int16_t* codes, float* scale,
     int32_t* g_idx, uint8_t* code_len, uint64_t* code_word, int64_t* row_off,
     uint32_t* stream_words, int64_t stream_cap, float* alpha, float* trace_alpha,
     int64_t* trace_bits, float* loss_row, float* Qdq, int32_t* info, void* ws,
@@ -426,44 +450,60 @@ extern "C" gptq_status gptq_hptq_quantize(
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_hptq_quantize: stream_cap=%lld",
                 (long long)stream_cap);
   const size_t need = (m >= 1 && n >= 1 && block >= 1)
-                          ? hptq_ws_layout(m, n, block, nullptr, nullptr, nullptr)
+                          ? hptq_ws_layout(m, n, block, nullptr, nullptr)
                           : 0;
   gptq_status st = quant_check_args(w_dtype, m, n, bits, group, block, ws, ws_bytes, need);
   if (st != GPTQ_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  QuantWs w;
   HptqWs h;
-  hptq_ws_layout(m, n, block, &w, &h, static_cast<char*>(ws));
+  hptq_ws_layout(m, n, block, &h, static_cast<char*>(ws));
+  const QuantWs& w = h.w[0];
   const long long b_max = (long long)std::floor(budget * (double)m * (double)n);
 
   st = quant_setup(w, m, n, U, perm, group, block, g_idx, info, s);
   if (st != GPTQ_OK) return st;
   GPTQ_LAUNCH(KK_HPTQ, s, search_init_kernel, 1, 1, 0, h.st, alpha_lo, alpha_hi);
-  for (int k = 0; k <= iters; ++k) {
-    st = hptq_pass(w, h, W, w_dtype, m, n, U, perm, dead, bits, group, block, scale,
-                   loss_row, &h.st->a, k, b_max, trace_alpha, trace_bits, 0, info, s);
+  // pass 0 at α_hi, then one pass a bisection step, or (lookahead) two levels
+  // a round (slot 0 the midpoint, slots 1 and 2 the quarter points side by side)
+  st = hptq_pass(h, 0, W, w_dtype, m, n, U, perm, dead, bits, group, block, scale, nullptr,
+                 &h.st->a, 0, nullptr, b_max, trace_alpha, trace_bits, 0, info, s);
+  if (st != GPTQ_OK) return st;
+  for (int k = 1; k <= iters && !lookahead; ++k) {
+    st = hptq_pass(h, 0, W, w_dtype, m, n, U, perm, dead, bits, group, block, scale, nullptr,
+                   &h.st->a, k, nullptr, b_max, trace_alpha, trace_bits, 0, info, s);
+    if (st != GPTQ_OK) return st;
+  }
+  for (int k0 = 1; k0 <= iters && lookahead; k0 += 2) {
+    st = search_round(h.st, k0, iters, b_max, trace_alpha, trace_bits, KK_HPTQ, s,
+                      [&](int slot, cudaStream_t ss) -> gptq_status {
+                        return hptq_pass(h, slot, W, w_dtype, m, n, U, perm, dead, bits, group,
+                                         block, slot ? h.scale[slot] : scale, nullptr,
+                                         &h.st->cand[slot], -1, &h.st->ccount[slot], b_max,
+                                         nullptr, nullptr, 0, info, ss);
+                      });
     if (st != GPTQ_OK) return st;
   }
   // the outputs: one more pass at the chosen α (the bracket's hi), encoded
-  st = hptq_pass(w, h, W, w_dtype, m, n, U, perm, dead, bits, group, block, scale,
-                 loss_row, &h.st->hi, -1, b_max, nullptr, nullptr, 1, info, s);
+  st = hptq_pass(h, 0, W, w_dtype, m, n, U, perm, dead, bits, group, block, scale, loss_row,
+                 &h.st->hi, -1, nullptr, b_max, nullptr, nullptr, 1, info, s);
   if (st != GPTQ_OK) return st;
   const unsigned g8 = (unsigned)ceil_div(m, 8);
-  GPTQ_LAUNCH(KK_HPTQ, s, hptq_rowbits_kernel, g8, 256, 0, h.codes16, m, n, h.lens, h.rowbits);
+  GPTQ_LAUNCH(KK_HPTQ, s, hptq_rowbits_kernel, g8, 256, 0, h.codes16[0], m, n, h.lens,
+              h.rowbits);
   GPTQ_LAUNCH(KK_HPTQ, s, row_scan_kernel, 1, 1024, 0, h.rowbits, m, row_off, stream_cap * 32,
               h.st, alpha, info);
   if (stream_cap > 0) {
     GPTQ_CUDA(cudaMemsetAsync(stream_words, 0, sizeof(uint32_t) * (size_t)stream_cap, s));
-    GPTQ_LAUNCH(KK_HPTQ, s, hptq_encode_kernel, g8, 256, 0, h.codes16, w.pinv, m, n, h.lens,
-                h.canon, row_off, stream_words, stream_cap);
+    GPTQ_LAUNCH(KK_HPTQ, s, hptq_encode_kernel, g8, 256, 0, h.codes16[0], w.pinv, m, n,
+                h.lens, h.canon, row_off, stream_words, stream_cap);
   }
   GPTQ_CUDA(cudaMemcpyAsync(code_len, h.lens, NSYM, cudaMemcpyDeviceToDevice, s));
   if (code_word != nullptr)
     GPTQ_CUDA(cudaMemcpyAsync(code_word, h.canon, sizeof(uint64_t) * NSYM,
                               cudaMemcpyDeviceToDevice, s));
   if (codes != nullptr || Qdq != nullptr)
-    GPTQ_LAUNCH(KK_HPTQ, s, hptq_out_kernel, (unsigned)ceil_div(m * n, 256), 256, 0, h.codes16,
-                w.pinv, m, n, group, ceil_div(n, group), scale, codes, Qdq);
+    GPTQ_LAUNCH(KK_HPTQ, s, hptq_out_kernel, (unsigned)ceil_div(m * n, 256), 256, 0,
+                h.codes16[0], w.pinv, m, n, group, ceil_div(n, group), scale, codes, Qdq);
   return GPTQ_OK;
 }

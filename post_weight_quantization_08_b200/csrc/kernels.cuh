@@ -102,6 +102,11 @@ struct QuantWs {
 // Bytes of the layout (256-byte aligned parts); fills *w when both are given.
 size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base);
 
+// A second working set for a pass that runs beside another: its own Wp,
+// codes and error buffers at `base`, the U-derived parts (pinv, panels, the
+// TF32 split) shared with `shared`.  Returns its bytes; fills *w when given.
+size_t quant_slot_layout(int64_t m, int64_t n, const QuantWs* shared, QuantWs* w, char* base);
+
 // Host checks shared by the quantize entry points (no device work).
 gptq_status quant_check_args(int w_dtype, int64_t m, int64_t n, int bits, int group,
                              int block, const void* ws, size_t ws_bytes, size_t need);

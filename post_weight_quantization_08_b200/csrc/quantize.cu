@@ -49,6 +49,30 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   return off;
 }
 
+size_t quant_slot_layout(int64_t m, int64_t n, const QuantWs* shared, QuantWs* w, char* base) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t mrows = (size_t)error_rows(m);
+  const size_t o_wp = take(sizeof(float) * mrows * (size_t)n);
+  const size_t o_codes = take((size_t)m * (size_t)n);
+  size_t o_e[4];
+  for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
+  if (w && base && shared) {
+    *w = *shared;
+    w->Wp = reinterpret_cast<float*>(base + o_wp);
+    w->codes = reinterpret_cast<uint8_t*>(base + o_codes);
+    for (int k = 0; k < 2; ++k) {
+      w->Ehi[k] = reinterpret_cast<float*>(base + o_e[2 * k]);
+      w->Elo[k] = reinterpret_cast<float*>(base + o_e[2 * k + 1]);
+    }
+  }
+  return off;
+}
+
 namespace {
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

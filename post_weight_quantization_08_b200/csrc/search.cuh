@@ -5,6 +5,10 @@
 // both use for their per-row outputs.
 #pragma once
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "common.cuh"
 
 namespace gptq {
@@ -15,6 +19,11 @@ struct SearchState {
   float a;                  // the α of the next pass
   int32_t done;             // the search has ended: later passes run at hi
   unsigned long long count; // the running pass's measure (outliers, coded bits)
+  // two bisection levels per round: the midpoint and both quarter points of
+  // the level after it, evaluated side by side
+  float cand[3];            // mid, lower quarter, upper quarter
+  int32_t steps;            // bisection steps taken (pass 0 excluded)
+  unsigned long long ccount[3];
 };
 
 __global__ void search_init_kernel(SearchState* st, float lo, float hi) {
@@ -23,6 +32,7 @@ __global__ void search_init_kernel(SearchState* st, float lo, float hi) {
   st->a = hi;
   st->done = 0;
   st->count = 0ull;
+  st->steps = 0;
 }
 
 // After pass k (run at st->a, whose measure is st->count): pass 0 evaluates
@@ -58,6 +68,116 @@ __device__ __forceinline__ void search_step(SearchState* st, int k, long long li
     }
   }
   st->count = 0ull;
+}
+
+__device__ __forceinline__ float bisect_mid(float lo, float hi) {
+  return __double2float_rn(((double)lo + (double)hi) * 0.5);
+}
+
+// Before a round: the candidates are the next midpoint (st->a, set by the
+// step before) and the midpoints of its two halves, each rounded as a
+// bisection step would round it.  After the search has ended all three are hi.
+__global__ void search_plan_kernel(SearchState* st) {
+  if (st->done) {
+    st->cand[0] = st->cand[1] = st->cand[2] = st->hi;
+  } else {
+    const float mid = st->a;
+    st->cand[0] = mid;
+    st->cand[1] = bisect_mid(st->lo, mid);
+    st->cand[2] = bisect_mid(mid, st->hi);
+  }
+  st->ccount[0] = st->ccount[1] = st->ccount[2] = 0ull;
+}
+
+// After a round (its first trace entry k0): the midpoint's measure decides
+// the first level exactly as a bisection step; the second level's midpoint is
+// then the quarter on the side kept, whose measure decides it.  A midpoint
+// equal to an end of the bracket, or `iters` steps, ends the search; trace
+// entries of steps not taken read (hi, −1).
+__global__ void search_decide_kernel(SearchState* st, int k0, int iters, long long limit,
+                                     float* trace_alpha, int64_t* trace_count) {
+  bool lower = false;                 // the first level kept the lower half
+  for (int lev = 0; lev < 2; ++lev) {
+    const int k = k0 + lev;
+    if (k > iters) break;
+    if (st->done) {
+      if (trace_alpha != nullptr) trace_alpha[k] = st->hi;
+      if (trace_count != nullptr) trace_count[k] = -1;
+      continue;
+    }
+    const float a = st->a;
+    const int slot = lev == 0 ? 0 : (lower ? 1 : 2);
+    const unsigned long long c = st->ccount[slot];
+    if (trace_alpha != nullptr) trace_alpha[k] = a;
+    if (trace_count != nullptr) trace_count[k] = (int64_t)c;
+    if (c <= (unsigned long long)limit) {
+      st->hi = a;
+      lower = true;
+    } else {
+      st->lo = a;
+      lower = false;
+    }
+    st->steps += 1;
+    const float mid = bisect_mid(st->lo, st->hi);
+    if (mid <= st->lo || mid >= st->hi || st->steps >= iters) {
+      st->done = 1;
+      st->a = st->hi;
+    } else {
+      st->a = mid;
+    }
+  }
+}
+
+// Two streams forked from a caller's stream for the round's side passes, and
+// the events that fork and join them; one set per (device, caller stream),
+// created on first use and kept for the life of the process.
+struct ForkStreams {
+  cudaStream_t side[2] = {nullptr, nullptr};
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join[2] = {nullptr, nullptr};
+};
+
+inline gptq_status fork_streams_for(cudaStream_t s, ForkStreams** out) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, ForkStreams> reg;
+  int dev = 0;
+  GPTQ_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(mu);
+  ForkStreams& f = reg[{dev, s}];
+  if (f.side[0] == nullptr) {
+    for (int i = 0; i < 2; ++i) {
+      GPTQ_CUDA(cudaStreamCreateWithFlags(&f.side[i], cudaStreamNonBlocking));
+      GPTQ_CUDA(cudaEventCreateWithFlags(&f.join[i], cudaEventDisableTiming));
+    }
+    GPTQ_CUDA(cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming));
+  }
+  *out = &f;
+  return GPTQ_OK;
+}
+
+// One round: plan the three candidates, run `pass(slot, stream)` for the
+// midpoint on the caller's stream and for the two quarter points on forked
+// streams, join, and decide two levels (trace entries k0 and k0 + 1).
+template <typename Pass>
+gptq_status search_round(SearchState* st, int k0, int iters, long long limit, float* trace_alpha,
+                         int64_t* trace_count, int kind, cudaStream_t s, Pass&& pass) {
+  ForkStreams* f = nullptr;
+  gptq_status r = fork_streams_for(s, &f);
+  if (r != GPTQ_OK) return r;
+  GPTQ_LAUNCH(kind, s, search_plan_kernel, 1, 1, 0, st);
+  GPTQ_CUDA(cudaEventRecord(f->fork, s));
+  for (int i = 0; i < 2; ++i) GPTQ_CUDA(cudaStreamWaitEvent(f->side[i], f->fork, 0));
+  r = pass(0, s);
+  if (r != GPTQ_OK) return r;
+  for (int i = 0; i < 2; ++i) {
+    r = pass(i + 1, f->side[i]);
+    if (r != GPTQ_OK) return r;
+    GPTQ_CUDA(cudaEventRecord(f->join[i], f->side[i]));
+    GPTQ_CUDA(cudaStreamWaitEvent(s, f->join[i], 0));
+  }
+  GPTQ_LAUNCH(kind, s, search_decide_kernel, 1, 1, 0, st, k0, iters, limit, trace_alpha,
+              trace_count);
+  return GPTQ_OK;
 }
 
 // ptr[0] = 0, ptr[r+1] = Σ_{i≤r} cnt[i] (one CTA of 1024 threads: a

@@ -8,10 +8,13 @@
 // bound, which keeping it does not.
 //
 // The search runs on the device: one sweep of the whole layer per candidate
-// scale factor α (the sweep kernel's outlier variant reads α from the state
-// below and counts its outliers there), and a one-thread step kernel between
-// the passes updates the bracket.  No host round trip, so the whole call can
-// be captured in a CUDA graph.  A last pass at the chosen α produces the
+// scale factor α (the sweep kernel's outlier variant reads α from the search
+// state and counts its outliers there).  After the pass at α_hi, each round
+// runs the bracket's midpoint and both quarter points of the next level side
+// by side on three streams, and a one-thread kernel takes the two bisection
+// steps they decide (search.cuh): the same steps as one pass at a time, in
+// half the passes on the critical path.  No host round trip, so the whole
+// call can be captured in a CUDA graph.  A last pass at the chosen α produces the
 // outputs; the outlier list is then compacted into CSR (one warp per row,
 // original column order) and the codes are packed.
 #include <cmath>
@@ -22,17 +25,46 @@
 namespace gptq {
 namespace {
 
-size_t ssqr_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, SearchState** st,
-                      int32_t** row_cnt, char* base) {
-  const size_t q = quant_ws_layout(m, n, block, w, base);
-  const size_t o_st = q;
-  const size_t o_cnt = align_up(o_st + sizeof(SearchState), 256);
-  const size_t end = align_up(o_cnt + sizeof(int32_t) * (size_t)m, 256);
-  if (base) {
-    *st = reinterpret_cast<SearchState*>(base + o_st);
-    *row_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
+// The workspace: the call's working set (slot 0, which also holds the
+// U-derived parts), two more for the quarter-point passes of a round, the
+// search state, and per slot the row counts and the scale and zero of its
+// pass (slot 0 uses the caller's).
+struct SsqrWs {
+  QuantWs w[3];
+  SearchState* st;
+  int32_t* row_cnt[3];
+  float* scale[3];
+  uint8_t* zero[3];
+};
+
+size_t ssqr_ws_layout(int64_t m, int64_t n, int block, SsqrWs* o, char* base) {
+  size_t off = quant_ws_layout(m, n, block, o ? &o->w[0] : nullptr, base);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t ngmax = (size_t)ceil_div(n, 32);        // group ≥ 32
+  const size_t o_st = take(sizeof(SearchState));
+  size_t o_cnt[3], o_sc[3], o_z[3], o_slot[3];
+  for (int k = 0; k < 3; ++k) o_cnt[k] = take(sizeof(int32_t) * (size_t)m);
+  for (int k = 1; k < 3; ++k) {
+    o_sc[k] = take(sizeof(float) * (size_t)m * ngmax);
+    o_z[k] = take((size_t)m * ngmax);
+    o_slot[k] = take(quant_slot_layout(m, n, nullptr, nullptr, nullptr));
   }
-  return end;
+  if (base && o) {
+    o->st = reinterpret_cast<SearchState*>(base + o_st);
+    for (int k = 0; k < 3; ++k) o->row_cnt[k] = reinterpret_cast<int32_t*>(base + o_cnt[k]);
+    o->scale[0] = nullptr;
+    o->zero[0] = nullptr;
+    for (int k = 1; k < 3; ++k) {
+      o->scale[k] = reinterpret_cast<float*>(base + o_sc[k]);
+      o->zero[k] = reinterpret_cast<uint8_t*>(base + o_z[k]);
+      quant_slot_layout(m, n, &o->w[0], &o->w[k], base + o_slot[k]);
+    }
+  }
+  return off;
 }
 
 // Between passes: the outlier count against the budget (search.cuh).
@@ -82,13 +114,13 @@ using namespace gptq;
 
 extern "C" size_t gptq_ssqr_workspace_bytes(int64_t m, int64_t n, int block) {
   if (m < 1 || n < 1 || block < 1) return 0;
-  return ssqr_ws_layout(m, n, block, nullptr, nullptr, nullptr, nullptr);
+  return ssqr_ws_layout(m, n, block, nullptr, nullptr);
 }
 
 extern "C" gptq_status gptq_ssqr_quantize(
     const void* W, int w_dtype, int64_t m, int64_t n, const float* U, const int32_t* perm,
     const uint8_t* dead, int bits, int group, int block, double target, int iters,
-    float alpha_lo, float alpha_hi, uint32_t* qweight, float* scale, uint8_t* zero,
+    float alpha_lo, float alpha_hi, int lookahead, uint32_t* qweight, float* scale, uint8_t* zero,
     int32_t* g_idx, int64_t* row_ptr, int32_t* col_idx, float* val, int64_t nnz_cap,
     float* alpha, float* trace_alpha, int64_t* trace_count, float* loss_row, float* Qdq,
     int32_t* info, void* ws, size_t ws_bytes, void* stream) {
@@ -107,41 +139,65 @@ extern "C" gptq_status gptq_ssqr_quantize(
   if (nnz_cap < 0)
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_ssqr_quantize: nnz_cap=%lld", (long long)nnz_cap);
   const size_t need = (m >= 1 && n >= 1 && block >= 1)
-                          ? ssqr_ws_layout(m, n, block, nullptr, nullptr, nullptr, nullptr)
+                          ? ssqr_ws_layout(m, n, block, nullptr, nullptr)
                           : 0;
   gptq_status st = quant_check_args(w_dtype, m, n, bits, group, block, ws, ws_bytes, need);
   if (st != GPTQ_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  QuantWs w;
-  SearchState* state = nullptr;
-  int32_t* row_cnt = nullptr;
-  ssqr_ws_layout(m, n, block, &w, &state, &row_cnt, static_cast<char*>(ws));
+  SsqrWs o;
+  ssqr_ws_layout(m, n, block, &o, static_cast<char*>(ws));
+  const QuantWs& w = o.w[0];
+  SearchState* state = o.st;
   const long long n_max = (long long)std::floor(target * (double)m * (double)n);
 
   st = quant_setup(w, m, n, U, perm, group, block, g_idx, info, s);
   if (st != GPTQ_OK) return st;
   GPTQ_LAUNCH(KK_SSQR, s, search_init_kernel, 1, 1, 0, state, alpha_lo, alpha_hi);
-  OutlierArgs search;
-  search.alpha = &state->a;
-  search.row_cnt = row_cnt;
-  search.total = &state->count;
-  for (int k = 0; k <= iters; ++k) {
-    GPTQ_CUDA(cudaMemsetAsync(row_cnt, 0, sizeof(int32_t) * (size_t)m, s));
+  // pass 0 at α_hi
+  OutlierArgs first;
+  first.alpha = &state->a;
+  first.row_cnt = o.row_cnt[0];
+  first.total = &state->count;
+  GPTQ_CUDA(cudaMemsetAsync(o.row_cnt[0], 0, sizeof(int32_t) * (size_t)m, s));
+  st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, scale, zero,
+                  nullptr, &first, info, s);
+  if (st != GPTQ_OK) return st;
+  GPTQ_LAUNCH(KK_SSQR, s, ssqr_step_kernel, 1, 1, 0, state, 0, n_max, trace_alpha,
+              trace_count);
+  // the bisection: one pass a step, or (lookahead) two levels a round, slot 0
+  // the midpoint and slots 1 and 2 the quarter points side by side
+  for (int k = 1; k <= iters && !lookahead; ++k) {
+    GPTQ_CUDA(cudaMemsetAsync(o.row_cnt[0], 0, sizeof(int32_t) * (size_t)m, s));
     st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, scale, zero,
-                    loss_row, &search, info, s);
+                    nullptr, &first, info, s);
     if (st != GPTQ_OK) return st;
     GPTQ_LAUNCH(KK_SSQR, s, ssqr_step_kernel, 1, 1, 0, state, k, n_max, trace_alpha,
                 trace_count);
   }
+  for (int k0 = 1; k0 <= iters && lookahead; k0 += 2) {
+    st = search_round(state, k0, iters, n_max, trace_alpha, trace_count, KK_SSQR, s,
+                      [&](int slot, cudaStream_t ss) -> gptq_status {
+                        OutlierArgs a;
+                        a.alpha = &state->cand[slot];
+                        a.row_cnt = o.row_cnt[slot];
+                        a.total = &state->ccount[slot];
+                        GPTQ_CUDA(cudaMemsetAsync(o.row_cnt[slot], 0,
+                                                  sizeof(int32_t) * (size_t)m, ss));
+                        return quant_pass(o.w[slot], W, w_dtype, m, n, U, perm, dead, bits,
+                                          group, block, 0, slot ? o.scale[slot] : scale,
+                                          slot ? o.zero[slot] : zero, nullptr, &a, info, ss);
+                      });
+    if (st != GPTQ_OK) return st;
+  }
   // the outputs: one more pass at the chosen α (the bracket's hi)
-  OutlierArgs fin = search;
+  OutlierArgs fin = first;
   fin.alpha = &state->hi;
-  GPTQ_CUDA(cudaMemsetAsync(row_cnt, 0, sizeof(int32_t) * (size_t)m, s));
+  GPTQ_CUDA(cudaMemsetAsync(o.row_cnt[0], 0, sizeof(int32_t) * (size_t)m, s));
   st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, scale, zero,
                   loss_row, &fin, info, s);
   if (st != GPTQ_OK) return st;
-  GPTQ_LAUNCH(KK_SSQR, s, row_scan_kernel, 1, 1024, 0, row_cnt, m, row_ptr, nnz_cap, state,
+  GPTQ_LAUNCH(KK_SSQR, s, row_scan_kernel, 1, 1024, 0, o.row_cnt[0], m, row_ptr, nnz_cap, state,
               alpha, info);
   GPTQ_LAUNCH(KK_SSQR, s, ssqr_fill_kernel, (unsigned)ceil_div(m, 8), 256, 0, w.codes, w.pinv,
               w.Wp, m, n, row_ptr, nnz_cap, col_idx, val);

@@ -121,17 +121,17 @@ def test_fixed_alpha_matches_oracle(m, n, bits, group, block, alpha, order):
         assert codes.min() < -half or codes.max() >= half   # the grid is unbounded
 
 
-@pytest.mark.parametrize("m,n,bits,group,budget,wdtype", [
-    (576, 576, 4, 128, 3.125, torch.bfloat16),    # a SmolLM-135M projection at the page's budget
-    (192, 576, 3, 64, 2.5, torch.float32),
-    (300, 260, 4, 32, 3.125, torch.float32),      # a trailing group of 4 columns
+@pytest.mark.parametrize("m,n,bits,group,budget,wdtype,iters,lookahead", [
+    (576, 576, 4, 128, 3.125, torch.bfloat16, 10, True),  # SmolLM-135M, the page's budget
+    (576, 576, 4, 128, 3.125, torch.bfloat16, 10, False), # one pass a step: the same trace
+    (192, 576, 3, 64, 2.5, torch.float32, 9, True),       # an odd step count
+    (300, 260, 4, 32, 3.125, torch.float32, 10, True),    # a trailing group of 4 columns
 ])
-def test_binary_search_matches_oracle(m, n, bits, group, budget, wdtype):
+def test_binary_search_matches_oracle(m, n, bits, group, budget, wdtype, iters, lookahead):
     g = _g()
-    iters = 10
     W, prep, U32, gp, Wz = _setup(m, n, "act", 222, wdtype=wdtype)
     q = g.hptq_quantize(W.to(DEV), gp, bits, group, 128, budget=budget, iters=iters,
-                        want_qdq=True, want_trace=True)
+                        want_qdq=True, want_trace=True, lookahead=lookahead)
     torch.cuda.synchronize()
     ta = q["trace_alpha"].cpu().numpy()
     tb = q["trace_bits"].cpu().numpy()

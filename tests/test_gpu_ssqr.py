@@ -125,17 +125,17 @@ def _oracle_search(Wp, U, bits, group, block, n_max, iters, lo, hi):
                             n_max, iters, lo, hi)
 
 
-@pytest.mark.parametrize("m,n,bits,group,target,wdtype", [
-    (576, 576, 3, 128, 0.01, torch.bfloat16),     # a SmolLM-135M attention projection
-    (192, 576, 2, 64, 0.005, torch.float32),
-    (300, 260, 4, 32, 0.02, torch.float32),       # a trailing group of 4 columns
+@pytest.mark.parametrize("m,n,bits,group,target,wdtype,iters,lookahead", [
+    (576, 576, 3, 128, 0.01, torch.bfloat16, 10, True),   # a SmolLM-135M attention projection
+    (576, 576, 3, 128, 0.01, torch.bfloat16, 10, False),  # one pass a step: the same trace
+    (192, 576, 2, 64, 0.005, torch.float32, 9, True),     # an odd step count
+    (300, 260, 4, 32, 0.02, torch.float32, 10, True),     # a trailing group of 4 columns
 ])
-def test_binary_search_matches_oracle(m, n, bits, group, target, wdtype):
+def test_binary_search_matches_oracle(m, n, bits, group, target, wdtype, iters, lookahead):
     g = _g()
-    iters = 10
     W, H, prep, U32, gp, Wz = _setup(m, n, "act", 202, wdtype=wdtype)
     q = g.ssqr_quantize(W.to(DEV), gp, bits, group, 128, target=target, iters=iters,
-                        want_qdq=True, want_trace=True)
+                        want_qdq=True, want_trace=True, lookahead=lookahead)
     torch.cuda.synchronize()
     ta = q["trace_alpha"].cpu().numpy()
     tc = q["trace_count"].cpu().numpy()

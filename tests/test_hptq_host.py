@@ -18,13 +18,13 @@ def _lib():
 
 def _call(L, p, **kw):
     a = dict(W=p, dtype=0, m=64, n=64, U=p, perm=p, dead=p, bits=4, group=32, block=64,
-             budget=3.125, iters=8, lo=1.0 / 16, hi=16.0, codes=None, scale=p,
+             budget=3.125, iters=8, lo=1.0 / 16, hi=16.0, la=1, codes=None, scale=p,
              g_idx=p, code_len=p, code_word=None, row_off=p, stream=p, cap=64, alpha=p,
              ta=None, tb=None, loss=None, qdq=None, info=p, ws=p, ws_bytes=1 << 30)
     a.update(kw)
     return L.gptq_hptq_quantize(a["W"], a["dtype"], a["m"], a["n"], a["U"], a["perm"],
                                 a["dead"], a["bits"], a["group"], a["block"], a["budget"],
-                                a["iters"], a["lo"], a["hi"], a["codes"], a["scale"],
+                                a["iters"], a["lo"], a["hi"], a["la"], a["codes"], a["scale"],
                                 a["g_idx"], a["code_len"], a["code_word"], a["row_off"],
                                 a["stream"], a["cap"], a["alpha"], a["ta"], a["tb"], a["loss"],
                                 a["qdq"], a["info"], a["ws"], a["ws_bytes"], None)

@@ -18,13 +18,13 @@ def _lib():
 
 def _call(L, p, **kw):
     a = dict(W=p, dtype=0, m=64, n=64, U=p, perm=p, dead=p, bits=3, group=32, block=64,
-             target=0.01, iters=8, lo=1.0 / 16, hi=1.0, qweight=p, scale=p, zero=p, g_idx=p,
+             target=0.01, iters=8, lo=1.0 / 16, hi=1.0, la=1, qweight=p, scale=p, zero=p, g_idx=p,
              row_ptr=p, col_idx=p, val=p, cap=16, alpha=p, ta=None, tc=None, loss=None,
              qdq=None, info=p, ws=p, ws_bytes=1 << 30)
     a.update(kw)
     return L.gptq_ssqr_quantize(a["W"], a["dtype"], a["m"], a["n"], a["U"], a["perm"],
                                 a["dead"], a["bits"], a["group"], a["block"], a["target"],
-                                a["iters"], a["lo"], a["hi"], a["qweight"], a["scale"],
+                                a["iters"], a["lo"], a["hi"], a["la"], a["qweight"], a["scale"],
                                 a["zero"], a["g_idx"], a["row_ptr"], a["col_idx"], a["val"],
                                 a["cap"], a["alpha"], a["ta"], a["tc"], a["loss"], a["qdq"],
                                 a["info"], a["ws"], a["ws_bytes"], None)
