@@ -209,3 +209,48 @@ def test_argument_errors():
         g.hptq_quantize(W, prep, 4, 32, 64, budget=0.0)
     with pytest.raises(g.GptqError):
         g.hptq_quantize(W, prep, 4, 32, 64, alpha_lo=2.0, alpha_hi=1.0)
+
+
+@pytest.mark.parametrize("m,n,alpha", [(130, 200, 0.6), (1, 96, 2.0)])
+def test_dead_columns_zero_rows_and_one_row(m, n, alpha):
+    """Dead columns and an all-zero row code as the lattice point 0; a single
+    row, on a coarse grid, may leave one symbol (coded in 1 bit)."""
+    g = _g()
+    X = cone_activations(2048, n, 515).to(torch.bfloat16)
+    X[:, [0, 7, n - 1]] = 0
+    W = student_t_weights(m, n, 516)
+    if m > 1:
+        W[3] = 0
+    H = og.hessian(X.to(torch.float64).numpy())
+    prep = og.prepare(H, 0.01, "act")
+    U32 = prep["U"].astype(np.float32)
+    gp = {"U": torch.from_numpy(U32).to(DEV),
+          "perm": torch.from_numpy(prep["perm"].astype(np.int32)).to(DEV),
+          "dead": torch.from_numpy(prep["dead"].astype(np.uint8)).to(DEV)}
+    Wz = W.to(torch.float64).numpy().copy()
+    Wz[:, prep["dead"]] = 0.0
+    q = g.hptq_quantize(W.to(DEV), gp, 4, 32, 64, budget=64.0, iters=0, alpha_lo=alpha,
+                        alpha_hi=alpha, stream_cap=2 * m * n + 64, want_qdq=True)
+    torch.cuda.synchronize()
+    _, codes = _check_outputs(q, W, Wz, prep, U32, 4, 32, 64, np.float32(alpha))
+    assert np.all(codes[:, prep["dead"]] == 0)
+    if m > 1:
+        assert np.all(codes[3] == 0)
+
+
+def test_a_single_symbol_codes_in_one_bit():
+    """An all-zero matrix: every coordinate is 0, one symbol, 1 bit a weight."""
+    g = _g()
+    m, n = 40, 64
+    X = cone_activations(256, n, 525).to(torch.bfloat16)
+    prep = og.prepare(og.hessian(X.to(torch.float64).numpy()), 0.01, "act")
+    gp = {"U": torch.from_numpy(prep["U"].astype(np.float32)).to(DEV),
+          "perm": torch.from_numpy(prep["perm"].astype(np.int32)).to(DEV),
+          "dead": torch.from_numpy(prep["dead"].astype(np.uint8)).to(DEV)}
+    q = g.hptq_quantize(torch.zeros(m, n, device=DEV), gp, 4, 32, 64, budget=1.0, iters=4)
+    torch.cuda.synchronize()
+    lens = q["code_len"].cpu().numpy()
+    assert lens[2048] == 1 and lens.sum() == 1
+    assert int(q["row_off"][-1]) == m * n
+    assert np.all(q["codes"].cpu().numpy() == 0)
+    assert np.all(q["stream"].cpu().numpy() == 0)

@@ -231,3 +231,32 @@ def test_argument_errors():
         g.ssqr_quantize(W, prep, 3, 32, 64, target=1.5)
     with pytest.raises(g.GptqError):
         g.ssqr_quantize(W, prep, 3, 32, 64, alpha_lo=0.5, alpha_hi=0.25)
+
+
+@pytest.mark.parametrize("m,n,alpha", [(130, 200, 0.6), (1, 96, 0.5)])
+def test_dead_columns_zero_rows_and_one_row(m, n, alpha):
+    """Dead columns (inputs that never fire: W zeroed there, never an outlier),
+    an all-zero weight row (its groups take [−1, 1]), and a single row."""
+    g = _g()
+    X = cone_activations(2048, n, 505).to(torch.bfloat16)
+    X[:, [0, 7, n - 1]] = 0
+    W = student_t_weights(m, n, 506)
+    if m > 1:
+        W[3] = 0
+    H = og.hessian(X.to(torch.float64).numpy())
+    prep = og.prepare(H, 0.01, "act")
+    assert prep["dead"].sum() == 3
+    U32 = prep["U"].astype(np.float32)
+    gp = {"U": torch.from_numpy(U32).to(DEV),
+          "perm": torch.from_numpy(prep["perm"].astype(np.int32)).to(DEV),
+          "dead": torch.from_numpy(prep["dead"].astype(np.uint8)).to(DEV)}
+    Wz = W.to(torch.float64).numpy().copy()
+    Wz[:, prep["dead"]] = 0.0
+    q = g.ssqr_quantize(W.to(DEV), gp, 3, 32, 64, target=1.0, iters=0, alpha_lo=alpha,
+                        alpha_hi=alpha, nnz_cap=m * n, want_qdq=True)
+    torch.cuda.synchronize()
+    f, mask = _check_outputs(q, W, Wz, prep, U32, 3, 32, 64, np.float32(alpha))
+    assert not mask[:, prep["dead"]].any()
+    if m > 1:
+        assert not mask[3].any()
+        assert np.all(q["Qdq"].cpu().numpy()[3] == 0)
