@@ -764,6 +764,8 @@ def run_chmc(args, rank, world, local):
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step"},
         "gpu_launches": int(launches_per_step * args.steps),
+        "roofline": _frontend_roofline(kernels, {k: round(v[0] / args.steps, 4)
+                                                 for k, v in kprof.items() if v[0] > 0}),
         "kernels": kernels,
         "kernels_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in kprof.items()
                                 if v[0] > 0},
@@ -993,6 +995,7 @@ def run_ssqr(args, rank, world, local):
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step"},
         "gpu_launches": int(launches * args.steps),
+        "roofline": _frontend_roofline(kernels, kms),
         "kernels": kernels, "kernels_ms_per_step": kms, "clocks": clk,
     }, probs
 
@@ -1183,8 +1186,27 @@ def run_hptq(args, rank, world, local):
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step"},
         "gpu_launches": int(launches * args.steps),
+        "roofline": _frontend_roofline(kernels, kms),
         "kernels": kernels, "kernels_ms_per_step": kms, "clocks": clk,
     }, probs
+
+
+def _frontend_roofline(kernels, kms):
+    """The roofline object of a frontend line: its dominant kernel kind (the
+    most device time in the serialised event profile) with the same figures
+    as its entry in ``kernels``; no ncu DRAM capture is kept for these
+    workloads, so traffic is null."""
+    if not kernels:
+        return None
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+    e = kernels[dom]
+    _, src = _peaks()
+    note = ("fp64 148 SMs x 64 FMA x 2 x max clock" if e["bound"] == "alu"
+            else (f"bf16 {src}" if e["bound"] == "tensor" else f"copy bandwidth, {src}"))
+    return {"kernel": dom, "bound": e["bound"], "achieved": e["achieved"], "peak": e["peak"],
+            "unit": e["unit"], "frac": e["frac"], "peak_source": note, "traffic": None,
+            "launches_per_step": e["launches_per_step"],
+            "share": round(e["ms_per_step"] / max(1e-9, sum(kms.values())), 4)}
 
 
 def _time_frontend(args, layer, device, world, local, work):
