@@ -283,7 +283,9 @@ gptq_status gptq_quantize_rowgroups(const void* W, int w_dtype, int64_t m, int64
  * break Satz 5's error bound.
  */
 
-/* Bytes of device workspace gptq_ssqr_quantize needs (256-byte aligned). */
+/* Bytes of device workspace gptq_ssqr_quantize needs (256-byte aligned): three
+ * working sets of gptq_quantize's (the second and third serve lookahead),
+ * the search state and per-set row counts, scales and zero points. */
 size_t gptq_ssqr_workspace_bytes(int64_t m, int64_t n, int block);
 
 /*
@@ -353,7 +355,9 @@ gptq_status gptq_ssqr_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
 #define GPTQ_HPTQ_SYMBOLS 4096
 #define GPTQ_HPTQ_SYMBOL_OFFSET 2048
 
-/* Bytes of device workspace gptq_hptq_quantize needs (256-byte aligned). */
+/* Bytes of device workspace gptq_hptq_quantize needs (256-byte aligned): as
+ * gptq_ssqr_workspace_bytes, plus per set m×n int16 coordinates and a
+ * histogram, and the code table. */
 size_t gptq_hptq_workspace_bytes(int64_t m, int64_t n, int block);
 
 /*
