@@ -230,6 +230,10 @@ __device__ __forceinline__ void sweep_body(
   pdl_trigger();
   float alpha = 1.f;
   if constexpr (QM != 0) alpha = *oa.alpha;
+  // row groups: column j0 + t's original index, so that thread c stores column
+  // c's scale and zero without a load in the column chain
+  int32_t perm_t = 0;
+  if constexpr (ROWG) perm_t = (t < bw) ? perm[j0 + t] : 0;
   if (t == 0) {
     // the strip, when the rows allow a tensor map: four boxes at (j0 + 32q,
     // r0); columns past n read as zero, and Wp holds whole 128-row boxes
@@ -357,6 +361,7 @@ __device__ __forceinline__ void sweep_body(
   }
 
   const float maxq = (float)((1 << bits) - 1);
+  const float rmaxq = __frcp_rn(maxq);
   float s = 1.f, z = 0.f, loss = 0.f, rs = 1.f, klo = 0.f, khi = maxq;
   uint8_t* cr = cs + t * LDB;
   int ocnt = 0;                         // this row's outliers in the block
@@ -483,15 +488,17 @@ __device__ __forceinline__ void sweep_body(
           xmin = -1.f;
           xmax = 1.f;
         }
-        s = __fdiv_rn(xmax - xmin, maxq);
+        // range/maxq correctly rounded: Markstein's correction from RN(1/maxq)
+        // for a normal range, the division itself for a tiny one
+        const float range = xmax - xmin;
+        s = range >= 1e-30f ? div_fma(range, maxq, rmaxq) : __fdiv_rn(range, maxq);
         rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
         z = rintf(div_rn(-xmin, s));
         klo = -z;
         khi = maxq - z;
-        if (t == 0 && c < bw) {
-          const int64_t oc = perm[j0 + c];
-          scale[(int64_t)bx * n + oc] = s;
-          zero[(int64_t)bx * n + oc] = (uint8_t)z;
+        if (t == c && c < bw) {
+          scale[(int64_t)bx * n + perm_t] = s;
+          zero[(int64_t)bx * n + perm_t] = (uint8_t)z;
         }
       }
       // q − z = clamp(rint(v/s), −z, maxq − z) exactly (small integers), so
