@@ -199,6 +199,28 @@ gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m, int64_t n,
                           int32_t* info, void* ws, size_t ws_bytes,
                           void* stream);
 
+/*
+ * Static groups: as gptq_quantize, except that every group's scale and zero
+ * are fixed before the sweep from the ORIGINAL weights (dead columns read 0)
+ * of `group` consecutive ORIGINAL columns [g·group, (g+1)·group), with the
+ * same min-max quantizer; the sweep then quantizes processing column j with
+ * the parameters of group perm[j] / group and recomputes nothing from the
+ * current values.  The pages define only the groups met in processing order
+ * (CHMC page, Schritt 2 and 3); this is the common variant that lets act-order
+ * change the order of the columns but not which columns share a scale.
+ *   group    any width ≥ 1 (groups need not align with blocks).
+ *   block    a multiple of 32, at most 128.
+ *   scale, zero   m × ceil(n/group), group g = original columns as above.
+ *   g_idx    int32[n], output: c / group.
+ * Workspace: gptq_quantize_workspace_bytes(m, n, block).
+ */
+gptq_status gptq_quantize_static(const void* W, int w_dtype, int64_t m, int64_t n,
+                                 const float* U, const int32_t* perm, const uint8_t* dead,
+                                 int bits, int group, int block, uint32_t* qweight,
+                                 float* scale, uint8_t* zero, int32_t* g_idx,
+                                 float* loss_row, float* Qdq, int32_t* info, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* ---- CHMC frontend (next to the hot path) -------------------------------
  * "Warum Geometrie Gewichte nicht komprimiert", section "Methodik. Was ist
  * CHMC": every weight matrix W (o × i) is split into a low-rank part W_lr

@@ -77,12 +77,15 @@ def prepare(H: torch.Tensor, damp: float = 0.01, order: str = "natural",
 
 def quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
              block: int = 128, want_loss: bool = True, want_qdq: bool = False,
-             ws: torch.Tensor | None = None, stream=None, check: bool = True) -> dict:
+             ws: torch.Tensor | None = None, stream=None, check: bool = True,
+             static_groups: bool = False) -> dict:
     """Returns qweight (int32 bit patterns of the uint32 words), scale, zero,
-    g_idx and optionally loss_row / Qdq."""
+    g_idx and optionally loss_row / Qdq.  ``static_groups``: every group's
+    parameters fixed from the original weights of consecutive original
+    columns (gptq_quantize_static)."""
     m, n = W.shape
     dev = W.device
-    ng = -(-n // group)
+    ng = -(-n // max(group, 1))             # the library rejects group < 1 itself
     nwords = -(-n * bits // 32)
     out = {
         "qweight": torch.empty(m, nwords, dtype=torch.int32, device=dev),
@@ -97,7 +100,7 @@ def quantize(W: torch.Tensor, prep: dict, bits: int = 4, group: int = 128,
         ws = workspace(gptq_quantize_workspace_bytes(m, n, block), dev)
     gptq_quantize(W, prep["U"], prep["perm"], prep["dead"], bits, group, block,
                   out["qweight"], out["scale"], out["zero"], out["g_idx"],
-                  out["loss_row"], out["Qdq"], out["info"], ws, stream)
+                  out["loss_row"], out["Qdq"], out["info"], ws, stream, static_groups)
     if check:
         _raise_info(out["info"], stream, "gptq_quantize")
     return out

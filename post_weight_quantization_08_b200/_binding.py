@@ -39,6 +39,11 @@ _SIGS = {
                                 C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                 C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                 C.c_size_t, C.c_void_p]),
+    "gptq_quantize_static": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_void_p,
+                                       C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
+                                       C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.c_size_t, C.c_void_p]),
     "gptq_quantize_rowgroups": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_int64,
                                           C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                                           C.c_int, C.c_int, C.c_void_p, C.c_void_p,
@@ -179,14 +184,15 @@ def gptq_prepare(H, damp, order, perm, U, dead, info, ws, stream=None):
 
 
 def gptq_quantize(W, U, perm, dead, bits, group, block, qweight, scale, zero,
-                  g_idx, loss_row, Qdq, info, ws, stream=None):
-    """Quantize W with U (see include/gptq_b200.h)."""
+                  g_idx, loss_row, Qdq, info, ws, stream=None, static_groups=False):
+    """Quantize W with U (see include/gptq_b200.h); ``static_groups`` calls
+    gptq_quantize_static (parameters fixed from the original weights)."""
     if W.dtype not in DTYPES:
         raise TypeError("W must be float32 or bfloat16")
     _need(W, "W", W.dtype)
     m, n = W.shape
     dev = W.device
-    ng = -(-n // group)
+    ng = -(-n // max(group, 1))           # the library rejects group < 1 itself
     nwords = -(-n * bits // 32)
     _need(U, "U", torch.float32, (n, n), dev)
     _need(perm, "perm", torch.int32, (n,), dev)
@@ -201,7 +207,8 @@ def gptq_quantize(W, U, perm, dead, bits, group, block, qweight, scale, zero,
         _need(Qdq, "Qdq", torch.float32, (m, n), dev)
     _need(info, "info", torch.int32, (2,), dev)
     _need(ws, "ws", torch.uint8, None, dev)
-    _raise(lib().gptq_quantize(_ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm),
+    fn = lib().gptq_quantize_static if static_groups else lib().gptq_quantize
+    _raise(fn(_ptr(W), DTYPES[W.dtype], m, n, _ptr(U), _ptr(perm),
                                _ptr(dead), int(bits), int(group), int(block),
                                _ptr(qweight), _ptr(scale), _ptr(zero), _ptr(g_idx),
                                _ptr(loss_row), _ptr(Qdq), _ptr(info), _ptr(ws),
@@ -252,7 +259,7 @@ def gptq_ssqr_quantize(W, U, perm, dead, bits, group, block, target, iters, alph
     _need(W, "W", W.dtype)
     m, n = W.shape
     dev = W.device
-    ng = -(-n // group)
+    ng = -(-n // max(group, 1))           # the library rejects group < 1 itself
     nwords = -(-n * bits // 32)
     _need(U, "U", torch.float32, (n, n), dev)
     _need(perm, "perm", torch.int32, (n,), dev)
@@ -304,7 +311,7 @@ def gptq_hptq_quantize(W, U, perm, dead, bits, group, block, budget, iters, alph
     _need(W, "W", W.dtype)
     m, n = W.shape
     dev = W.device
-    ng = -(-n // group)
+    ng = -(-n // max(group, 1))           # the library rejects group < 1 itself
     _need(U, "U", torch.float32, (n, n), dev)
     _need(perm, "perm", torch.int32, (n,), dev)
     _need(dead, "dead", torch.uint8, (n,), dev)

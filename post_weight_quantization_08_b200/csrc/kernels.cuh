@@ -73,12 +73,22 @@ struct SweepFar {
 // (saturated) to outl->codes16 (m × n, processing order) instead of `codes`,
 // and its error is v − s·k.
 constexpr uint8_t OUTLIER_FLAG = 0x80;
+//
+// outl->static_groups: the hot path's clamped quantizer with every group's
+// scale and zero fixed beforehand (st_scale / st_zero, m × st_ng, group g =
+// perm[j] / group of processing column j); nothing is taken from the current
+// values and the sweep writes no scale or zero.
 struct OutlierArgs {
   const float* alpha = nullptr;
   int32_t* row_cnt = nullptr;          // m counts, accumulated over the blocks
   unsigned long long* total = nullptr; // all outliers of the pass
   bool unclipped = false;
   int16_t* codes16 = nullptr;
+  bool static_groups = false;
+  const float* st_scale = nullptr;
+  const uint8_t* st_zero = nullptr;
+  const int32_t* perm = nullptr;
+  int64_t st_ng = 0;
 };
 gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
@@ -115,7 +125,7 @@ gptq_status quant_check_args(int w_dtype, int64_t m, int64_t n, int bits, int gr
 // split of U.
 gptq_status quant_setup(const QuantWs& w, int64_t m, int64_t n, const float* U,
                         const int32_t* perm, int group, int block, int32_t* g_idx,
-                        int32_t* info, cudaStream_t s);
+                        int32_t* info, cudaStream_t s, bool static_groups = false);
 
 // One pass of the column sweep over the whole layer: W → Wp (processing
 // order, dead columns zeroed), then the block loop of sweeps and trailing
@@ -131,7 +141,8 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
 // dequantized value of a flagged weight is outl_vals at its processing position.
 gptq_status quant_pack(const QuantWs& w, int64_t m, int64_t n, int bits, int group, int rowgs,
                        const float* scale, const uint8_t* zero, uint32_t* qweight,
-                       float* Qdq, const float* outl_vals, int32_t* info, cudaStream_t s);
+                       float* Qdq, const float* outl_vals, int32_t* info, cudaStream_t s,
+                       bool static_groups = false);
 
 // Whether the trailing update runs on the tensor cores for this shape.
 bool trailing_uses_tensor_cores(int64_t n, int block);

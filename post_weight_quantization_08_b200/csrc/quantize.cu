@@ -106,16 +106,54 @@ gptq_status side_stream_for(cudaStream_t s, SideStream** out) {
   return GPTQ_OK;
 }
 
-// pinv[perm[p]] = p and g_idx[perm[p]] = p / group.
+// pinv[perm[p]] = p and g_idx[perm[p]] = p / group (static groups: c / group).
 __global__ void __launch_bounds__(256)
 pinv_kernel(const int32_t* __restrict__ perm, int64_t n, int group,
-            int32_t* __restrict__ pinv, int32_t* __restrict__ g_idx, int32_t* info) {
+            int32_t* __restrict__ pinv, int32_t* __restrict__ g_idx, int static_groups,
+            int32_t* info) {
   const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (p >= n) return;
   const int32_t c = perm[p];
   if (c < 0 || c >= n) { report(info, GPTQ_ERR_INVALID_ARG, p); return; }
   pinv[c] = (int32_t)p;
-  if (g_idx) g_idx[c] = (int32_t)(p / group);
+  if (g_idx) g_idx[c] = (int32_t)((static_groups ? c : p) / group);
+}
+
+// Static groups: a warp per (row, group) takes the min-max parameters of the
+// group's original columns [g·group, (g+1)·group) of W (dead columns read 0),
+// with the hot path's quantizer: 0 inside the range, an all-zero group → [−1,
+// 1], s = (xmax − xmin)/maxq and z = rint(−xmin/s) correctly rounded in
+// float32.
+template <typename T>
+__global__ void __launch_bounds__(256)
+static_params_kernel(const T* __restrict__ W, int64_t m, int64_t n,
+                     const uint8_t* __restrict__ dead, int group, int64_t ngroups, int bits,
+                     float* __restrict__ scale, uint8_t* __restrict__ zero) {
+  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= m * ngroups) return;
+  const int64_t r = wid / ngroups, g = wid % ngroups;
+  const int64_t c0 = g * group, c1 = min(n, c0 + group);
+  float xmin = 0.f, xmax = 0.f;
+  for (int64_t c = c0 + lane; c < c1; c += 32) {
+    const float v = dead[c] ? 0.f : to_f32(W[r * n + c]);
+    xmin = fminf(xmin, v);
+    xmax = fmaxf(xmax, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    xmin = fminf(xmin, __shfl_xor_sync(0xffffffffu, xmin, o));
+    xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, o));
+  }
+  if (lane != 0) return;
+  if (xmin == 0.f && xmax == 0.f) {
+    xmin = -1.f;
+    xmax = 1.f;
+  }
+  const float maxq = (float)((1 << bits) - 1);
+  const float s = __fdiv_rn(xmax - xmin, maxq);
+  scale[r * ngroups + g] = s;
+  zero[r * ngroups + g] = (uint8_t)rintf(__fdiv_rn(-xmin, s));
 }
 
 // Wp[r][p] = W[r][perm[p]] as float32; dead columns read as 0.
@@ -144,7 +182,8 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
             const int32_t* __restrict__ pinv, int group, int64_t ngroups, int rowgs,
             const float* __restrict__ scale, const uint8_t* __restrict__ zero,
             uint32_t* __restrict__ qweight, int64_t nwords,
-            float* __restrict__ Qdq, const float* __restrict__ outv, int32_t* info) {
+            float* __restrict__ Qdq, const float* __restrict__ outv, int static_groups,
+            int32_t* info) {
   const int64_t chunks = (n + 31) / 32;
   const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (e >= m * chunks) return;
@@ -170,7 +209,8 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
         if (Qdq != nullptr) {
           // input-channel groups: [row][group of processing position p];
           // output-channel groups (rowgs rows): [row group][original column c]
-          const int64_t sx = rowgs > 0 ? (r / rowgs) * n + c : r * ngroups + p / group;
+          const int64_t sx = rowgs > 0 ? (r / rowgs) * n + c
+                                       : r * ngroups + (static_groups ? c : p) / group;
           Qdq[r * n + c] = kept ? outv[r * n + p] : scale[sx] * ((float)q - (float)zero[sx]);
         }
       }
@@ -211,12 +251,12 @@ gptq_status quant_check_args(int w_dtype, int64_t m, int64_t n, int bits, int gr
 
 gptq_status quant_setup(const QuantWs& w, int64_t m, int64_t n, const float* U,
                         const int32_t* perm, int group, int block, int32_t* g_idx,
-                        int32_t* info, cudaStream_t s) {
+                        int32_t* info, cudaStream_t s, bool static_groups) {
   (void)m;
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
   GPTQ_CUDA(cudaMemsetAsync(w.pinv, 0xFF, sizeof(int32_t) * n, s));
   GPTQ_LAUNCH(KK_INGEST, s, pinv_kernel, (unsigned)ceil_div(n, 256), 256, 0, perm, n,
-              group, w.pinv, g_idx, info);
+              group, w.pinv, g_idx, static_groups ? 1 : 0, info);
   gptq_status st = launch_panels(U, n, block, w.panels, s);
   if (st != GPTQ_OK) return st;
   if (w.Uhi != nullptr && n > block) {
@@ -314,26 +354,28 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
 
 gptq_status quant_pack(const QuantWs& w, int64_t m, int64_t n, int bits, int group, int rowgs,
                        const float* scale, const uint8_t* zero, uint32_t* qweight,
-                       float* Qdq, const float* outl_vals, int32_t* info, cudaStream_t s) {
+                       float* Qdq, const float* outl_vals, int32_t* info, cudaStream_t s,
+                       bool static_groups) {
+  const int sg = static_groups ? 1 : 0;
   const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
   const int64_t nwords = ceil_div(n * bits, 32);
   const unsigned gpk = (unsigned)ceil_div(m * ceil_div(n, 32), 256);
   switch (bits) {
     case 2:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
       break;
     case 3:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
       break;
     case 4:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
       break;
     default:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
       break;
   }
   return GPTQ_OK;
@@ -389,6 +431,50 @@ extern "C" gptq_status gptq_quantize(const void* W, int w_dtype, int64_t m,
                                      void* ws, size_t ws_bytes, void* stream) {
   return quantize_impl(W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, qweight, scale,
                        zero, g_idx, loss_row, Qdq, info, ws, ws_bytes, stream);
+}
+
+extern "C" gptq_status gptq_quantize_static(const void* W, int w_dtype, int64_t m, int64_t n,
+                                            const float* U, const int32_t* perm,
+                                            const uint8_t* dead, int bits, int group, int block,
+                                            uint32_t* qweight, float* scale, uint8_t* zero,
+                                            int32_t* g_idx, float* loss_row, float* Qdq,
+                                            int32_t* info, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  if (!W || !U || !perm || !dead || !qweight || !scale || !zero || !g_idx || !info || !ws)
+    return fail(GPTQ_ERR_INVALID_ARG, "gptq_quantize_static: null pointer");
+  if (group < 1 || block < 32 || block > 128 || block % 32 != 0)
+    return fail(GPTQ_ERR_UNSUPPORTED,
+                "gptq_quantize_static: group=%d block=%d (group >= 1, block a multiple of 32, "
+                "at most 128)", group, block);
+  const size_t need =
+      (m >= 1 && n >= 1) ? quant_ws_layout(m, n, block, nullptr, nullptr) : 0;
+  // the hot path's checks with the block standing in for the group (any
+  // static group width goes with any block)
+  gptq_status st = quant_check_args(w_dtype, m, n, bits, block, block, ws, ws_bytes, need);
+  if (st != GPTQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  QuantWs w;
+  quant_ws_layout(m, n, block, &w, static_cast<char*>(ws));
+  const int64_t ng = ceil_div(n, group);
+  st = quant_setup(w, m, n, U, perm, group, block, g_idx, info, s, true);
+  if (st != GPTQ_OK) return st;
+  const unsigned gsp = (unsigned)ceil_div(m * ng, 8);
+  if (w_dtype == GPTQ_DTYPE_BF16)
+    GPTQ_LAUNCH(KK_INGEST, s, static_params_kernel<__nv_bfloat16>, gsp, 256, 0,
+                static_cast<const __nv_bfloat16*>(W), m, n, dead, group, ng, bits, scale, zero);
+  else
+    GPTQ_LAUNCH(KK_INGEST, s, static_params_kernel<float>, gsp, 256, 0,
+                static_cast<const float*>(W), m, n, dead, group, ng, bits, scale, zero);
+  OutlierArgs sa;
+  sa.static_groups = true;
+  sa.st_scale = scale;
+  sa.st_zero = zero;
+  sa.perm = perm;
+  sa.st_ng = ng;
+  st = quant_pass(w, W, w_dtype, m, n, U, perm, dead, bits, group, block, 0, scale, zero,
+                  loss_row, &sa, info, s);
+  if (st != GPTQ_OK) return st;
+  return quant_pack(w, m, n, bits, group, 0, scale, zero, qweight, Qdq, nullptr, info, s, true);
 }
 
 extern "C" gptq_status gptq_quantize_rowgroups(const void* W, int w_dtype, int64_t m,

@@ -69,8 +69,9 @@ constexpr uint32_t SM_BPHI = (SM_CODES + RT * LDB + 1023) / 1024 * 1024;
 constexpr uint32_t SM_BPLO = SM_CODES;
 constexpr uint32_t SM_BARS = SM_BPHI + 32 * RT * 4;
 constexpr uint32_t SM_RGRED = SM_BARS + 128;        // 2 × 8 floats: row-group min/max
+constexpr uint32_t SM_SGRP = SM_BARS + 192;         // 128 ints: static group of each column
 static_assert(GPTQ_ROWGROUP_SIZE == RT, "an output-channel group is one CTA's rows");
-constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 192;
+constexpr size_t SMEM_BYTES = 1024 + SM_BARS + 192 + SB * 4;
 static_assert(SM_AHI >= PK_BYTES && SM_AHI % 1024 == 0, "A operand placement");
 static_assert(SM_VALS % 1024 == 0, "the strip's boxes use the 128-byte swizzle");
 static_assert(SM_CODES % 1024 == 0 && RT * LDB >= 32 * RT * 4, "U chunk lo part placement");
@@ -175,7 +176,9 @@ __device__ __forceinline__ int ord_key_inv(int k) { return k ^ ((k >> 31) & 0x7f
 // QM selects the quantizer: 0 the hot path's clamp, 1 SSQR's outliers, 2
 // HPTQ's unbounded lattice s·ℤ (same α-scaled step, k = rint(v/s) with no
 // clamp; each int16 coordinate goes to the thread's own row of the strip box
-// it was loaded from, which nothing reads again, and leaves with the block).
+// it was loaded from, which nothing reads again, and leaves with the block),
+// 3 static groups (the clamp, with the scale and zero of each column's
+// original group fixed beforehand and read per column).
 template <bool ROWG, int QM>
 __device__ __forceinline__ void sweep_body(
     const CUtensorMap& tmEhi, const CUtensorMap& tmElo, const CUtensorMap& tmW, int strip_tma,
@@ -234,6 +237,8 @@ __device__ __forceinline__ void sweep_body(
   // c's scale and zero without a load in the column chain
   int32_t perm_t = 0;
   if constexpr (ROWG) perm_t = (t < bw) ? perm[j0 + t] : 0;
+  int* sgrp = reinterpret_cast<int*>(sm + SM_SGRP);
+  if constexpr (QM == 3) sgrp[t] = (t < bw) ? oa.perm[j0 + t] / group : 0;   // read after a barrier
   if (t == 0) {
     // the strip, when the rows allow a tensor map: four boxes at (j0 + 32q,
     // r0); columns past n read as zero, and Wp holds whole 128-row boxes
@@ -410,7 +415,7 @@ __device__ __forceinline__ void sweep_body(
         v[4 * j + 3] = f.w - d[4 * j + 3];
       }
     }
-    if (!ROWG && c0 % group == 0) {
+    if (!ROWG && QM != 3 && c0 % group == 0) {
       // the group's current values: this sub-block, then later ones in the group
       float xmin = 0.f, xmax = 0.f;
 #pragma unroll
@@ -500,6 +505,14 @@ __device__ __forceinline__ void sweep_body(
           scale[(int64_t)bx * n + perm_t] = s;
           zero[(int64_t)bx * n + perm_t] = (uint8_t)z;
         }
+      }
+      if constexpr (QM == 3) {
+        const int64_t gx = row * oa.st_ng + sgrp[c];
+        s = row < m ? oa.st_scale[gx] : 1.f;
+        z = row < m ? (float)oa.st_zero[gx] : 0.f;
+        rs = fminf(__frcp_rn(s), 3.4028234663852886e38f);
+        klo = -z;
+        khi = maxq - z;
       }
       // q − z = clamp(rint(v/s), −z, maxq − z) exactly (small integers), so
       // the clamp works on k = q − z and the error takes one FMA
@@ -667,7 +680,8 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   }
 }
 
-bool g_attr_set[4] = {false, false, false, false};   // plain, row groups, outliers, unclipped
+bool g_attr_set[5] = {false, false, false, false, false};  // plain, row groups, outliers,
+                                                          // unclipped, static groups
 
 }  // namespace
 
@@ -693,16 +707,22 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
   const bool rowg = rowgroup_perm != nullptr;
   if (rowg && outl != nullptr)
     return fail(GPTQ_ERR_UNSUPPORTED, "sweep: outliers with output-channel groups");
-  if (outl != nullptr && !outl->unclipped &&
+  if (outl != nullptr && outl->static_groups &&
+      (!outl->st_scale || !outl->st_zero || !outl->perm || outl->st_ng < 1))
+    return fail(GPTQ_ERR_INVALID_ARG, "sweep: static-group arguments");
+  if (outl != nullptr && !outl->unclipped && !outl->static_groups &&
       (!outl->alpha || !outl->row_cnt || !outl->total || bits > 7))
     return fail(GPTQ_ERR_INVALID_ARG, "sweep: outlier arguments");
   if (outl != nullptr && outl->unclipped && (!outl->alpha || !outl->codes16))
     return fail(GPTQ_ERR_INVALID_ARG, "sweep: unclipped-grid arguments");
-  const int variant = rowg ? 1 : (outl == nullptr ? 0 : (outl->unclipped ? 3 : 2));
+  const int variant = rowg ? 1
+                      : (outl == nullptr ? 0
+                                         : (outl->static_groups ? 4 : (outl->unclipped ? 3 : 2)));
   if (!g_attr_set[variant]) {
     const void* fn = variant == 1 ? (const void*)sweep_kernel<true, 0>
                      : variant == 2 ? (const void*)sweep_kernel<false, 1>
                      : variant == 3 ? (const void*)sweep_kernel<false, 2>
+                     : variant == 4 ? (const void*)sweep_kernel<false, 3>
                                     : (const void*)sweep_kernel<false, 0>;
     GPTQ_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
     g_attr_set[variant] = true;
@@ -759,6 +779,11 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                     nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
   else if (variant == 2)
     GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, 1>), grid, RT, kSmem, th, tl, tw,
+                    strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
+                    bits, group, ngroups, codes, scale, zero, loss_row, info,
+                    (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
+  else if (variant == 4)
+    GPTQ_LAUNCH_PDL(KK_SWEEP, s, (sweep_kernel<false, 3>), grid, RT, kSmem, th, tl, tw,
                     strip_tma, tph, tpl, tuh, tul, (int64_t)pre.k0, kwp, Wp, m, n, j0, bw, pk,
                     bits, group, ngroups, codes, scale, zero, loss_row, info,
                     (const int32_t*)nullptr, oa, nsweep, fm, far.c0, fc1, far.k0, far.kw, fxx);
