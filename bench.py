@@ -66,9 +66,11 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def workload_name(cid: int, bits: int, order: str | None = None) -> str:
+def workload_name(cid: int, bits: int, order: str | None = None,
+                  static_groups: bool = False) -> str:
     c = CONFIGS[cid]
-    tail = "" if order is None else f", {order} order"
+    tail = ("" if order is None else f", {order} order") + (", static groups" if static_groups
+                                                            else "")
     if c["kind"] == "decoder":
         h, kv, it = c["hidden"], c["kv"], c["inter"]
         rows = 2 * h + 2 * kv + 2 * it
@@ -217,13 +219,16 @@ def traffic_for(kernel: str, workload: str):
 # ---------------------------------------------------------------- the GPU arm
 
 class Layer:
-    """Device buffers of one layer's problems, allocated once."""
+    """Device buffers of one layer's problems, allocated once; with
+    ``static_groups`` the quantize call fixes every group's parameters from
+    the original weights (gptq_quantize_static)."""
 
-    def __init__(self, probs, device):
+    def __init__(self, probs, device, static_groups=False):
         import post_weight_quantization_08_b200 as g
         self.g = g
         self.probs = probs
         self.dev = device
+        self.static_groups = bool(static_groups)
         self.items = []
         for p in probs:
             m, n = p.m, p.n
@@ -267,7 +272,7 @@ class Layer:
             s.wait_event(w_ready)
         g.gptq_quantize(it["W"], it["U"], it["perm"], it["dead"], p.bits, p.group, p.block,
                         it["qweight"], it["scale"], it["zero"], it["g_idx"], it["loss"],
-                        None, it["info_q"], it["ws_q"], s)
+                        None, it["info_q"], it["ws_q"], s, self.static_groups)
         if host is not None:
             with torch.cuda.stream(s):
                 for k in self.OUTS:
@@ -342,7 +347,7 @@ def run_ours(args, rank, world, local):
     cfg = CONFIGS[args.config]
     bits = args.bits or cfg["bits"][0]
     probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits, order=args.order)
-    layer = Layer(probs, device)
+    layer = Layer(probs, device, args.static_groups)
     params = sum(p.params for p in probs)
     main = torch.cuda.Stream(device=device)     # non-default: graphs capture here
     torch.cuda.set_stream(main)
@@ -475,7 +480,7 @@ def run_ours(args, rank, world, local):
         roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2),
                 "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
                 "peak_source": note,
-                "traffic": traffic_for(dom, workload_name(args.config, bits, args.order)),
+                "traffic": traffic_for(dom, workload_name(args.config, bits, args.order, args.static_groups)),
                 "launches_per_step": launches_per_step,
                 "share": round(tot[dom] / max(1e-9, sum(tot.values())), 4)}
 
@@ -498,7 +503,7 @@ def run_ours(args, rank, world, local):
                       "launches_per_step": kprof[k][1] / args.steps,
                       "bound": bound, "achieved": round(ach, 2), "unit": unit,
                       "peak": round(peak, 1), "frac": round(ach / peak, 4),
-                      "traffic": traffic_for(k, workload_name(args.config, bits, args.order))}
+                      "traffic": traffic_for(k, workload_name(args.config, bits, args.order, args.static_groups))}
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "params/s", "n_gpus": world,
@@ -506,7 +511,7 @@ def run_ours(args, rank, world, local):
         "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": workload_name(args.config, bits, args.order), "params_per_step_per_gpu": params,
+        "config": {"workload": workload_name(args.config, bits, args.order, args.static_groups), "params_per_step_per_gpu": params,
                    "global_batch": len(probs) * world, "seq_len": probs[0].T,
                    "parallelism": f"independent layers x{world}",
                    "l2": "flushed between timed steps (256 MB write)",
@@ -1278,15 +1283,18 @@ def _time_frontend(args, layer, device, world, local, work):
 
 # ---------------------------------------------------------------- CPU oracle arm
 
-def oracle_pass(probs):
+def oracle_pass(probs, static_groups=False):
     """One pass of the float64 oracle over the problems (test infrastructure)."""
-    import numpy as np
     from oracle import gptq as og
+    from oracle import static as ost
     for p in probs:
         X = p.X.to(torch.float64).numpy()
         W = p.W.to(torch.float64).numpy()
         H = og.hessian(X)
-        og.gptq_layer(W, H, p.bits, p.group, p.block, p.damp, p.order)
+        if static_groups:
+            ost.gptq_layer_static(W, H, p.bits, p.group, p.block, p.damp, p.order)
+        else:
+            og.gptq_layer(W, H, p.bits, p.group, p.block, p.damp, p.order)
     return sum(p.params for p in probs)
 
 
@@ -1301,11 +1309,11 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_baseline(probs, budget_s: float = 12.0):
+def cpu_baseline(probs, budget_s: float = 12.0, static_groups=False):
     done, t0 = 0, time.perf_counter()
     passes = 0
     while True:
-        done += oracle_pass(probs)
+        done += oracle_pass(probs, static_groups)
         passes += 1
         el = time.perf_counter() - t0
         if el >= budget_s or passes >= 50:
@@ -1322,11 +1330,11 @@ def run_reference(args, rank, world):
     bits = args.bits or cfg["bits"][0]
     probs = problems_for(args.config, layer=0, bits=bits, order=args.order)
     for _ in range(args.warmup):
-        oracle_pass(probs)
+        oracle_pass(probs, args.static_groups)
     t0 = time.perf_counter()
     params = 0
     for _ in range(args.steps):
-        params += oracle_pass(probs)
+        params += oracle_pass(probs, args.static_groups)
     el = time.perf_counter() - t0
     value = params / el
     cores = blas_threads()
@@ -1336,7 +1344,7 @@ def run_reference(args, rank, world):
         "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": workload_name(args.config, bits, args.order)},
+        "config": {"workload": workload_name(args.config, bits, args.order, args.static_groups)},
         "cpu_baseline": {"value": round(value, 1), "unit": "params/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"{args.steps} timed passes of one layer on the host cores"},
@@ -1358,6 +1366,9 @@ def main(argv=None):
     ap.add_argument("--frontend", default="gptq", choices=["gptq", "chmc", "ssqr", "hptq"],
                     help="chmc: the CHMC frontend over the layer; ssqr / hptq: SSQR / HPTQ "
                          "over the layer (separate metrics)")
+    ap.add_argument("--static-groups", action="store_true",
+                    help="group parameters fixed from the original weights (a variant of "
+                         "the same metric)")
     ap.add_argument("--order", default=None,
                     choices=["natural", "act", "reverse", "minpivot"],
                     help="processing order for every problem (default: the workload's)")
@@ -1393,7 +1404,7 @@ def main(argv=None):
         else:
             out, probs, _ = run_ours(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
-                out["cpu_baseline"] = cpu_baseline(probs)
+                out["cpu_baseline"] = cpu_baseline(probs, static_groups=args.static_groups)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
