@@ -326,3 +326,45 @@ def test_follow_accepts_a_zero_point_flipped_at_a_tie():
     f = S.follow_ssqr(W, np.eye(4), 4, 4, 4, 1.0, q, np.zeros((1, 4), bool),
                       np.zeros((1, 4)), s[:, None], np.array([[z2]], np.float32))
     assert f["z_bad"] == 0 and f["n_bad"] == 0 and f["n_diff"] == 0
+
+
+def test_follow_bounds_flag_a_planted_scale_and_value_error():
+    """The checker's scale and kept-value bounds are not vacuous: a 1e-3
+    relative scale error in a group of 32 columns, and a kept value off by
+    1e-3 of its range, are reported; the oracle's own output is not."""
+    rng = np.random.default_rng(12)
+    n = 64
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(30, n, rng)[:, p["perm"]]
+    ref = S.ssqr_blocked(Wp, p["U"], 3, 32, 64, 0.5)
+    args = (Wp, p["U"], 3, 32, 64, 0.5, ref["codes"], ref["mask"])
+    ok = S.follow_ssqr(*args, ref["value"], ref["scale"], ref["zero"])
+    assert ok["scale_bad"] == 0 and ok["scale_wide_over"] == 0 and ok["val_bad"] == 0
+    sc = ref["scale"].copy()
+    sc[4, 1] *= np.float32(1.001)
+    bad = S.follow_ssqr(*args, ref["value"], sc, ref["zero"])
+    assert bad["scale_bad"] >= 1 and bad["scale_wide_over"] >= 1
+    r, j = np.argwhere(ref["mask"])[0]
+    vals = ref["value"].copy()
+    vals[r, j] += 1e-3 * (abs(vals[r, j]) + float(ref["scale"][r, j // 32]) / 0.5 * 7)
+    assert S.follow_ssqr(*args, vals, ref["scale"], ref["zero"])["val_bad"] >= 1
+
+
+def test_follow_accepts_a_narrow_tail_group_within_its_float32_bound():
+    """A 4-column trailing group whose scale is off by less than the float32
+    forward-error bound of its propagation (but more than 1e-5) is accepted and
+    counted as narrow, not wide.  After K = 256 columns the bound is at least
+    γ_K = 2⁻²¹ + K·2⁻²⁴ ≈ 1.57e-5 relative (the range spans at most twice the
+    largest accumulated magnitude), so 1.2e-5 lies inside it."""
+    rng = np.random.default_rng(13)
+    n = 260                                  # groups of 32: a tail of 4 columns
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(20, n, rng)[:, p["perm"]]
+    ref = S.ssqr_blocked(Wp, p["U"], 3, 32, 64, 1.0)
+    sc = ref["scale"].copy()
+    sc[:, 8] = (sc[:, 8].astype(np.float64) * (1 + 1.2e-5)).astype(np.float32)
+    f = S.follow_ssqr(Wp, p["U"], 3, 32, 64, 1.0, ref["codes"], ref["mask"], ref["value"], sc,
+                      ref["zero"])
+    assert f["max_scale_rel"] > 1e-5
+    assert f["scale_wide_over"] == 0
+    assert f["scale_bad"] == 0
