@@ -4,6 +4,18 @@ The C ABI (include/gptq_b200.h) is exposed under the same names by
 :mod:`._binding`.  The helpers below only allocate the output tensors with
 torch (device memory is the caller's) and call those functions; every step of
 the path runs in the library's CUDA kernels.
+
+  hessian, prepare, quantize       the path (quantize(static_groups=True):
+                                   group parameters fixed from the original
+                                   weights; prepare(order="minpivot"))
+  chmc_lowrank, quantize_rowgroups,
+  chmc_layer                       the CHMC frontend ("Warum Geometrie Gewichte
+                                   nicht komprimiert", Methodik)
+  ssqr_quantize                    GPTQ with full-precision outliers and a
+                                   binary search on the scales ("The Geometry
+                                   of LLM Quantization", §3)
+  hptq_quantize                    GPTQ on one unbounded integer grid,
+                                   Huffman-coded to a bit budget (same, §3)
 """
 from __future__ import annotations
 
