@@ -35,14 +35,23 @@ __global__ void search_init_kernel(SearchState* st, float lo, float hi) {
   st->steps = 0;
 }
 
+// (lo + hi)/2 rounded once to float32 (exact in double for float operands).
+__host__ __device__ __forceinline__ float bisect_mid(float lo, float hi) {
+#ifdef __CUDA_ARCH__
+  return __double2float_rn(((double)lo + (double)hi) * 0.5);
+#else
+  return (float)(((double)lo + (double)hi) * 0.5);   // round to nearest even
+#endif
+}
+
 // After pass k (run at st->a, whose measure is st->count): pass 0 evaluates
 // α_hi, and a measure over `limit` there ends the search.  Later passes
 // evaluate the bracket's midpoint and keep it as hi when admissible (measure
 // ≤ limit), else as lo.  The next midpoint is (lo + hi)/2 rounded once to
 // float32; one equal to an end of the bracket ends the search.  The trace
 // records (α, measure) per pass, −1 for a pass run after the end.
-__device__ __forceinline__ void search_step(SearchState* st, int k, long long limit,
-                                            float* trace_alpha, int64_t* trace_count) {
+__host__ __device__ __forceinline__ void search_step(SearchState* st, int k, long long limit,
+                                                     float* trace_alpha, int64_t* trace_count) {
   const unsigned long long c = st->count;
   const float a = st->a;
   const bool was_done = st->done != 0;
@@ -58,7 +67,7 @@ __device__ __forceinline__ void search_step(SearchState* st, int k, long long li
       st->lo = a;
     }
     if (!done) {
-      const float mid = __double2float_rn(((double)st->lo + (double)st->hi) * 0.5);
+      const float mid = bisect_mid(st->lo, st->hi);
       if (mid <= st->lo || mid >= st->hi) done = true;
       else st->a = mid;
     }
@@ -70,14 +79,10 @@ __device__ __forceinline__ void search_step(SearchState* st, int k, long long li
   st->count = 0ull;
 }
 
-__device__ __forceinline__ float bisect_mid(float lo, float hi) {
-  return __double2float_rn(((double)lo + (double)hi) * 0.5);
-}
-
 // Before a round: the candidates are the next midpoint (st->a, set by the
 // step before) and the midpoints of its two halves, each rounded as a
 // bisection step would round it.  After the search has ended all three are hi.
-__global__ void search_plan_kernel(SearchState* st) {
+__host__ __device__ __forceinline__ void search_plan(SearchState* st) {
   if (st->done) {
     st->cand[0] = st->cand[1] = st->cand[2] = st->hi;
   } else {
@@ -89,13 +94,16 @@ __global__ void search_plan_kernel(SearchState* st) {
   st->ccount[0] = st->ccount[1] = st->ccount[2] = 0ull;
 }
 
+__global__ void search_plan_kernel(SearchState* st) { search_plan(st); }
+
 // After a round (its first trace entry k0): the midpoint's measure decides
 // the first level exactly as a bisection step; the second level's midpoint is
 // then the quarter on the side kept, whose measure decides it.  A midpoint
 // equal to an end of the bracket, or `iters` steps, ends the search; trace
 // entries of steps not taken read (hi, −1).
-__global__ void search_decide_kernel(SearchState* st, int k0, int iters, long long limit,
-                                     float* trace_alpha, int64_t* trace_count) {
+__host__ __device__ __forceinline__ void search_decide(SearchState* st, int k0, int iters,
+                                                       long long limit, float* trace_alpha,
+                                                       int64_t* trace_count) {
   bool lower = false;                 // the first level kept the lower half
   for (int lev = 0; lev < 2; ++lev) {
     const int k = k0 + lev;
@@ -126,6 +134,11 @@ __global__ void search_decide_kernel(SearchState* st, int k0, int iters, long lo
       st->a = mid;
     }
   }
+}
+
+__global__ void search_decide_kernel(SearchState* st, int k0, int iters, long long limit,
+                                     float* trace_alpha, int64_t* trace_count) {
+  search_decide(st, k0, iters, limit, trace_alpha, trace_count);
 }
 
 // Two streams forked from a caller's stream for the round's side passes, and
