@@ -1,6 +1,6 @@
 """GPU-vs-oracle parity checks shared by the GPU tests.
 
-Tolerances (written here, derived in the design doc):
+Tolerances (written here, each derived from the arithmetic it checks):
   * H: |ΔH_ij| ≤ 2·T·2⁻²⁴·S_ij with S = 2·|X|ᵀ|X| — the float32 summation
     bound γ_T of a length-T dot product (bf16 products are exact in float32).
   * U: the library computes in float64 and rounds once to float32, so

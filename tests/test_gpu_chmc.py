@@ -5,7 +5,7 @@ Every input handed to the GPU here is computed on the host (the oracle's
 Hessian and inverse-Cholesky factor, rounded to float32 where the library takes
 float32), so the oracle never sees a value that came from the CUDA path.
 
-Tolerances (derived in DESIGN.md):
+Tolerances (from the arithmetic of each side):
   * low-rank stage: both sides run the same float64 iteration from the same Ω;
     R differs by its float32 rounding (2⁻²³·|R|) plus 1e-9·max|W|.
   * residual quantization: the hot path's criterion (codes within 1e-4 code

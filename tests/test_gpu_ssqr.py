@@ -5,7 +5,7 @@ Algorithm", §3 (SSQR) and §2.3 (Satz 5).  The GPU receives the oracle's own
 preparation (U rounded to float32, perm, dead), so no value the oracle sees
 comes from the CUDA path.
 
-Tolerances (the hot path's criterion, derived in the design doc):
+Tolerances (the hot path's criterion, with the float32 bound stated below):
   * a (code, outlier flag) pair may differ only where the oracle's
     pre-rounding value lies within 1e-4 code units of a rounding boundary, at
     most 0.1 % of the weights; zeros equal except at such a near-tie; layer
