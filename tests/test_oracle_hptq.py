@@ -263,3 +263,11 @@ def test_pins_catch_planted_mistakes(kind, monkeypatch):
         Wp = _heavy(25, n, rng)[:, p["perm"]]
         failures += not _half_step_holds(Hq.hptq_blocked(Wp, p["U"], 2, 16, 32, 0.5), p["U"], 16)
     assert failures >= 1, kind
+
+
+def test_canonical_codes_golden(golden):
+    """The canonical-code rule against the DEFLATE format's worked example."""
+    for lens, codes in golden("canonical_code_deflate.txt"):
+        lengths = {i: int(l) for i, l in enumerate(lens)}
+        cb = Hq.canonical_codes(lengths)
+        assert [format(cb[i][0], f"0{cb[i][1]}b") for i in range(len(lens))] == codes
