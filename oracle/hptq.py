@@ -59,6 +59,29 @@ def lattice_column(cur, scale):
     return np.rint(np.asarray(cur, dtype=np.float32) / scale).astype(np.float32)
 
 
+def hptq_sequential(Wp, U, bits: int, group: int, alpha) -> dict:
+    """The definition: one column at a time, each error pushed onto every
+    later column with the full row of U (columns in processing order)."""
+    W = np.array(Wp, dtype=np.float64, copy=True)
+    U = np.asarray(U, dtype=np.float64)
+    m, n = W.shape
+    ng = -(-n // group)
+    out = {"codes": np.zeros((m, n), np.int64), "scale": np.zeros((m, ng), np.float32),
+           "err": np.zeros((m, n))}
+    s = None
+    for j in range(n):
+        if j % group == 0:
+            s0, _ = G.group_params(W[:, j:j + group], bits)
+            s = (s0 * np.float32(alpha)).astype(np.float32)
+            out["scale"][:, j // group] = s
+        q = lattice_column(W[:, j], s)
+        e = (W[:, j] - s.astype(np.float64) * q.astype(np.float64)) / U[j, j]
+        W[:, j + 1:] -= np.outer(e, U[j, j + 1:])
+        out["codes"][:, j] = q.astype(np.int64)
+        out["err"][:, j] = e
+    return out
+
+
 def hptq_blocked(Wp, U, bits: int, group: int, block: int, alpha) -> dict:
     """The unclipped sweep, lazy-batch form, columns in processing order;
     codes are the unbounded lattice coordinates k."""

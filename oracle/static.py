@@ -43,6 +43,25 @@ def static_params(Wz, bits: int, group: int):
     return scale, zero
 
 
+def gptq_static_sequential(Wp, U, bits: int, col_group, scale, zero) -> dict:
+    """The definition: one column at a time with the full row of U, the
+    parameters of each column's original group."""
+    W = np.array(Wp, dtype=np.float64, copy=True)
+    U = np.asarray(U, dtype=np.float64)
+    m, n = W.shape
+    col_group = np.asarray(col_group, dtype=np.int64)
+    out = {"codes": np.zeros((m, n), np.int64), "err": np.zeros((m, n))}
+    for j in range(n):
+        s = np.asarray(scale[:, col_group[j]], np.float32)
+        z = np.asarray(zero[:, col_group[j]], np.float32)
+        q = G.quantize_column(W[:, j], s, z, bits)
+        e = (W[:, j] - G.dequantize(q, s, z)) / U[j, j]
+        W[:, j + 1:] -= np.outer(e, U[j, j + 1:])
+        out["codes"][:, j] = q.astype(np.int64)
+        out["err"][:, j] = e
+    return out
+
+
 def gptq_static_blocked(Wp, U, bits: int, col_group, scale, zero, block: int = 128) -> dict:
     """The lazy-batch sweep with fixed parameters; ``col_group[j]`` is the
     group of processing column j.  Any block width."""

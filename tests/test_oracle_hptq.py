@@ -271,3 +271,15 @@ def test_canonical_codes_golden(golden):
         lengths = {i: int(l) for i, l in enumerate(lens)}
         cb = Hq.canonical_codes(lengths)
         assert [format(cb[i][0], f"0{cb[i][1]}b") for i in range(len(lens))] == codes
+
+
+@pytest.mark.parametrize("n,group,block,alpha", [(96, 32, 32, 1.0), (100, 32, 64, 0.6),
+                                                 (64, 16, 64, 2.5)])
+def test_blocked_equals_sequential(n, group, block, alpha):
+    rng = np.random.default_rng(40)
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(17, n, rng)[:, p["perm"]]
+    a = Hq.hptq_sequential(Wp, p["U"], 3, group, alpha)
+    b = Hq.hptq_blocked(Wp, p["U"], 3, group, block, alpha)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scale"], b["scale"])
+    assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-12)

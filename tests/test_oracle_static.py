@@ -138,3 +138,18 @@ def test_pins_catch_planted_mistakes(kind, monkeypatch):
         q_g = r["codes"][0][G.inverse_permutation(p["perm"])]
         failures += not np.array_equal(L.babai(F, F @ w, s, z, 3), q_g)
     assert failures >= 1, kind
+
+
+@pytest.mark.parametrize("n,group,block", [(96, 32, 32), (100, 40, 64), (130, 17, 96)])
+def test_blocked_equals_sequential_in_act_order(n, group, block):
+    """Any block width with any group width: the lazy batch changes only the
+    order of the float64 additions."""
+    rng = np.random.default_rng(41)
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    W = rng.standard_normal((15, n)) * 0.02
+    scale, zero = S.static_params(W, 3, group)
+    cg = p["perm"] // group
+    a = S.gptq_static_sequential(W[:, p["perm"]], p["U"], 3, cg, scale, zero)
+    b = S.gptq_static_blocked(W[:, p["perm"]], p["U"], 3, cg, scale, zero, block)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-12)
