@@ -283,3 +283,20 @@ def test_blocked_equals_sequential(n, group, block, alpha):
     b = Hq.hptq_blocked(Wp, p["U"], 3, group, block, alpha)
     assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scale"], b["scale"])
     assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-12)
+
+
+def test_hptq_is_ssqr_without_outliers():
+    """One unbounded grid and the outlier-keeping grid coincide where nothing
+    overflows: with one-column groups at α = 1 no weight leaves its range, and
+    SSQR's code minus its zero point is HPTQ's lattice coordinate, error for
+    error (the two oracles are written separately)."""
+    from oracle import ssqr as Sq
+    rng = np.random.default_rng(42)
+    n = 48
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    Wp = _heavy(11, n, rng)[:, p["perm"]]
+    a = Sq.ssqr_blocked(Wp, p["U"], 3, 1, 16, 1.0)
+    b = Hq.hptq_blocked(Wp, p["U"], 3, 1, 16, 1.0)
+    assert Sq.count(a) == 0
+    assert np.array_equal(a["codes"] - a["zero"].astype(np.int64), b["codes"])
+    assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-15)
