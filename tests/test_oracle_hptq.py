@@ -300,3 +300,25 @@ def test_hptq_is_ssqr_without_outliers():
     assert Sq.count(a) == 0
     assert np.array_equal(a["codes"] - a["zero"].astype(np.int64), b["codes"])
     assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("alpha", [0.5, 1.0, 2.0])
+def test_back_to_front_is_babai_without_clipping(alpha):
+    """Satz 4 for the unbounded grid: with one group (its step taken at the
+    first column, before any update, so from the original weights), HPTQ
+    back to front is Babai's nearest plane on F·diag(s) with no clamp and no
+    zero point (the separately written lattice oracle), identical integers."""
+    from oracle import lattice as L
+    rng = np.random.default_rng(50)
+    for trial in range(40):
+        n = int(rng.integers(2, 9))
+        H = _spd(n, rng)
+        w = rng.standard_normal(n) * 0.02
+        p = G.prepare(H, 0.01, "reverse")
+        r = Hq.hptq_blocked(w[None, p["perm"]], p["U"], 3, n, n, alpha)
+        s = np.full(n, float(r["scale"][0, 0]))
+        Hd, _, _ = G.damp_and_fix(H, 0.01)
+        F = np.linalg.cholesky(Hd).T
+        q_b = L.babai(F, F @ w, s, np.zeros(n), 3, clip=False)
+        q_g = r["codes"][0][G.inverse_permutation(p["perm"])]
+        assert np.array_equal(q_b, q_g), (trial, q_b, q_g)
