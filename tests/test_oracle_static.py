@@ -153,3 +153,21 @@ def test_blocked_equals_sequential_in_act_order(n, group, block):
     b = S.gptq_static_blocked(W[:, p["perm"]], p["U"], 3, cg, scale, zero, block)
     assert np.array_equal(a["codes"], b["codes"])
     assert np.allclose(a["err"], b["err"], rtol=0, atol=1e-12)
+
+
+def test_requantizing_the_result_is_a_no_op():
+    """Composition (the Babai page §2.2 reading of GPTQ as a lattice
+    projection): the dequantized weights lie on the fixed grid, so a second
+    static-group sweep over them, with the same parameters and order, returns
+    the same codes and no error at all."""
+    rng = np.random.default_rng(6)
+    n = 120
+    p = G.prepare(_spd(n, rng), 0.01, "act")
+    W = rng.standard_normal((14, n)) * 0.02
+    scale, zero = S.static_params(W, 3, 40)
+    cg = p["perm"] // 40
+    r1 = S.gptq_static_blocked(W[:, p["perm"]], p["U"], 3, cg, scale, zero, 64)
+    Qp = G.dequantize(r1["codes"], scale[:, cg], zero[:, cg])
+    r2 = S.gptq_static_blocked(Qp, p["U"], 3, cg, scale, zero, 64)
+    assert np.array_equal(r2["codes"], r1["codes"])
+    assert np.abs(r2["err"]).max() == 0.0
