@@ -237,6 +237,9 @@ def follow_rowgroups(Wp, U, bits: int, gs: int, block: int, codes_p, scale, zero
                 near_z = np.abs(zpre - np.floor(zpre) - 0.5) <= tol
                 z_diff += int(zd.sum())
                 z_bad += int((zd & ~near_z).sum())
+                # a zero point flipped at a near-tie shifts the row group's codes
+                # in this column by one: decide them with the other side's zero
+                z_o = np.where(zd & near_z, z_g, z_o).astype(np.float32)
             so, zo = _rows(s_o, m, gs), _rows(z_o, m, gs)
             x = W[:, j] / so.astype(np.float64)
             q_o = G.quantize_column(W[:, j], so, zo, bits).astype(np.int64)

@@ -211,3 +211,23 @@ def test_chmc_layer_reconstructs_from_its_parts():
     assert out["scale"].shape == (3, i) and out["codes"].shape == (o, i)
     assert 0 <= out["codes"].min() and out["codes"].max() <= 15
     assert out["bpw"] == pytest.approx(C.bpw_chmc(o, i, r, 4, 16))
+
+
+def test_follow_rowgroups_accepts_a_zero_point_flipped_at_a_tie():
+    """A row group whose −xmin/s sits on a half-integer may take either zero
+    point; the other side's codes of that column then sit one step over for
+    every row of the group.  That is one allowed zero flip, no code
+    difference."""
+    W = np.array([[-1.0, 0.2], [5.0, -0.3], [0.3, 0.1], [2.0, 0.4]])
+    s, z = C.rowgroup_params(W[:, 0], 4, 4)
+    assert abs(1.0 / float(s[0]) - 2.5) < 1e-6          # −xmin/s = 2.5 up to rounding
+    z2 = np.float32(z[0] + (1 if z[0] == 2 else -1))
+    q0 = np.clip(np.rint(np.float32(W[:, 0]) / s[0]) + z2, 0, 15)
+    s1, z1 = C.rowgroup_params(W[:, 1], 4, 4)
+    q1 = np.clip(np.rint(np.float32(W[:, 1]) / s1[0]) + z1[0], 0, 15)
+    codes = np.stack([q0, q1], axis=1).astype(np.int64)
+    scale = np.array([[s[0], s1[0]]], np.float32)
+    zero = np.array([[z2, z1[0]]], np.float32)
+    f = C.follow_rowgroups(W, np.eye(2), 4, 4, 2, codes, scale, zero)
+    assert f["z_diff"] == 1 and f["z_bad"] == 0
+    assert f["n_bad"] == 0
