@@ -761,10 +761,8 @@ def run_chmc(args, rank, world, local):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16->f32 Hessian, f64 prepare and low-rank part, f32 sweep",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": f"{cfg['name']} CHMC: per-matrix rank from the {CHMC_BPW}-bit "
-                               f"budget, niter {CHMC_NITER}, lambda {CHMC_LAM}, damp {CHMC_DAMP}, "
-                               f"act-order, residual {bits}-bit with {CHMC_GS}-row output-channel "
-                               f"groups, block {probs[0].block}",
+        "config": {"workload": frontend_workload("chmc", cfg, bits, probs[0].group,
+                                                 probs[0].block),
                    "params_per_step_per_gpu": params, "ranks": ranks,
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step"},
@@ -992,10 +990,8 @@ def run_ssqr(args, rank, world, local):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": f"{cfg['name']} SSQR: {SSQR_BITS}-bit, group {probs[0].group}, "
-                               f"act-order, target outlier density {SSQR_TARGET} per matrix, "
-                               f"{SSQR_ITERS} bisection steps on alpha in [{SSQR_LO}, {SSQR_HI}], "
-                               f"block {probs[0].block}",
+        "config": {"workload": frontend_workload("ssqr", cfg, SSQR_BITS, probs[0].group,
+                                                 probs[0].block),
                    "params_per_step_per_gpu": params, "alpha": alphas, "outliers": nnz,
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step"},
@@ -1183,10 +1179,8 @@ def run_hptq(args, rank, world, local):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep, int16 codes",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": f"{cfg['name']} HPTQ: lattice from the {HPTQ_BITS}-bit min-max "
-                               f"step, group {probs[0].group}, act-order, budget {HPTQ_BUDGET} "
-                               f"bits/weight per matrix, {HPTQ_ITERS} bisection steps on alpha in "
-                               f"[{HPTQ_LO}, {HPTQ_HI}], block {probs[0].block}",
+        "config": {"workload": frontend_workload("hptq", cfg, HPTQ_BITS, probs[0].group,
+                                                 probs[0].block),
                    "params_per_step_per_gpu": params, "alpha": alphas, "bits_per_weight": bpw,
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step"},
@@ -1323,9 +1317,62 @@ def cpu_baseline(probs, budget_s: float = 12.0, static_groups=False):
             "sample": f"{passes} full passes of the layer's problems ({el:.1f} s, float64 numpy)"}
 
 
+def frontend_workload(frontend: str, cfg, bits: int, group: int, block: int) -> str:
+    """The workload string of a frontend line (the GPU and the oracle arm)."""
+    if frontend == "chmc":
+        return (f"{cfg['name']} CHMC: per-matrix rank from the {CHMC_BPW}-bit budget, niter "
+                f"{CHMC_NITER}, lambda {CHMC_LAM}, damp {CHMC_DAMP}, act-order, residual "
+                f"{bits}-bit with {CHMC_GS}-row output-channel groups, block {block}")
+    if frontend == "ssqr":
+        return (f"{cfg['name']} SSQR: {SSQR_BITS}-bit, group {group}, act-order, target outlier "
+                f"density {SSQR_TARGET} per matrix, {SSQR_ITERS} bisection steps on alpha in "
+                f"[{SSQR_LO}, {SSQR_HI}], block {block}")
+    return (f"{cfg['name']} HPTQ: lattice from the {HPTQ_BITS}-bit min-max step, group {group}, "
+            f"act-order, budget {HPTQ_BUDGET} bits/weight per matrix, {HPTQ_ITERS} bisection "
+            f"steps on alpha in [{HPTQ_LO}, {HPTQ_HI}], block {block}")
+
+
+def run_reference_frontend(args, world):
+    """The oracle arm of a frontend line: each step one bounded sample of the
+    frontend's float64 oracle over the layer's matrices (the same function as
+    the line's cpu_baseline), its metric, unit and workload."""
+    cfg = CONFIGS[args.config]
+    fb = {"chmc": (CHMC_METRIC, args.bits or cfg["bits"][0], chmc_cpu_baseline),
+          "ssqr": (SSQR_METRIC, SSQR_BITS, ssqr_cpu_baseline),
+          "hptq": (HPTQ_METRIC, HPTQ_BITS, hptq_cpu_baseline)}[args.frontend]
+    metric, bits, fn = fb
+    probs = problems_for(args.config, layer=0, bits=bits, order="act")
+    kw = {} if args.frontend == "chmc" else {"budget_s": 0.0}
+    for _ in range(args.warmup):
+        fn(probs, **kw)                            # one matrix each (budget 0)
+    t0 = time.perf_counter()
+    vals, sample = [], ""
+    for _ in range(args.steps):
+        r = fn(probs)
+        vals.append(r["value"])
+        sample = r["sample"]
+    el = time.perf_counter() - t0
+    value = sum(vals) / len(vals)
+    return {
+        "impl": "reference", "metric": metric, "value": round(value, 1), "unit": "params/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
+        "config": {"workload": frontend_workload(args.frontend, cfg, bits, probs[0].group,
+                                                 probs[0].block)},
+        "cpu_baseline": {"value": round(value, 1), "unit": "params/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": f"per step: {sample}"},
+        "e2e": {"value": round(value, 1), "unit": "params/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    if args.frontend != "gptq":
+        return run_reference_frontend(args, world)
     cfg = CONFIGS[args.config]
     bits = args.bits or cfg["bits"][0]
     probs = problems_for(args.config, layer=0, bits=bits, order=args.order)
