@@ -146,7 +146,8 @@ gptq_status gptq_prepare(const float* H, int64_t n, double damp, int order,
  *   GPTQ_ERR_INVALID_ARG with a message (use gptq_prepare instead).
  *   The first call on each device looks up the array's device address
  *   (with that device current); make that first call before any stream
- *   capture.
+ *   capture.  The address is kept for the life of the process, so a device
+ *   reset (cudaDeviceReset) between calls is not supported.
  *   All calls on one device share the array and it keeps the last call's
  *   contents; the call initialises every part it reads.  Calls whose work
  *   overlaps on the GPU (different streams, or different host threads, on

@@ -73,6 +73,12 @@ def hessian(X) -> np.ndarray:
     return 2.0 * (X.T @ X)
 
 
+def hessian_block(A, B) -> np.ndarray:
+    """One block of H = 2·XᵀX: rows from the columns A = X[:, I], columns
+    from B = X[:, J] (float64), for checking a large H tile by tile."""
+    return 2.0 * (np.asarray(A, dtype=np.float64).T @ np.asarray(B, dtype=np.float64))
+
+
 def damp_and_fix(H, damp: float):
     """Relative damping and the dead-column fix.
 

@@ -77,6 +77,33 @@ def rtn(W, bits: int, group: int):
     return codes, scale, zero, Q
 
 
+def rtn_dequant(W, bits: int, group: int) -> np.ndarray:
+    """The dequantized weights of :func:`rtn`, all rows and groups at once.
+
+    The same float32 steps as ``rtn`` (range [min(0, min v), max(0, max v)],
+    an all-zero group on [−1, 1], scale (hi − lo)/(2^bits − 1), zero point and
+    codes rounded half to even, codes clamped to [0, 2^bits − 1]) on whole
+    arrays, for layers too large for the element loop; pinned equal to it.
+    """
+    W32 = np.asarray(W, dtype=np.float32)
+    m, n = W32.shape
+    maxq = np.float32(2 ** bits - 1)
+    Q = np.zeros((m, n))
+    for c0 in range(0, n, group):
+        v = W32[:, c0:c0 + group]
+        lo = np.minimum(v.min(axis=1), np.float32(0))
+        hi = np.maximum(v.max(axis=1), np.float32(0))
+        empty = (lo == 0) & (hi == 0)
+        lo = np.where(empty, np.float32(-1), lo)
+        hi = np.where(empty, np.float32(1), hi)
+        s = ((hi - lo) / maxq).astype(np.float32)
+        z = np.rint((-lo) / s).astype(np.float32)
+        q = np.clip(np.rint(v / s[:, None]) + z[:, None], 0, maxq)
+        Q[:, c0:c0 + group] = s[:, None].astype(np.float64) * (
+            q.astype(np.float64) - z[:, None].astype(np.float64))
+    return Q
+
+
 def babai(B, y, scale, zero, bits: int, clip: bool = True):
     """Babai's nearest-plane algorithm, basis vectors processed last to first.
 

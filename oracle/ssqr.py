@@ -217,7 +217,7 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
     scale = np.asarray(scale, dtype=np.float32)
     zero = np.asarray(zero, dtype=np.float32)
     maxq = 2 ** bits - 1
-    n_diff = n_bad = z_bad = scale_bad = scale_wide_over = val_bad = 0
+    n_diff = n_bad = z_diff = z_bad = scale_bad = scale_wide_over = val_bad = 0
     max_scale_rel = max_val_rel = 0.0
     worst = None
     err = np.zeros((m, n))
@@ -248,6 +248,7 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
                 max_scale_rel = max(max_scale_rel, float(rel.max()))
                 zd = zero[:, g] != z_o
                 near_z = np.abs(zpre - np.floor(zpre) - 0.5) <= tol
+                z_diff += int(zd.sum())
                 z_bad += int((zd & ~near_z).sum())
                 # a zero point flipped at a near-tie shifts the group's codes by
                 # one: decide this group's codes with the other side's zero
@@ -278,7 +279,8 @@ def follow_ssqr(Wp, U, bits: int, group: int, block: int, alpha, codes_p, mask_p
         if b1 < n:
             W[:, b1:] -= err[:, b0:b1] @ U[b0:b1, b1:]
             mag[:, b1:] += np.abs(err[:, b0:b1]) @ np.abs(U[b0:b1, b1:])
-    return {"n_diff": n_diff, "n_bad": n_bad, "z_bad": z_bad, "max_scale_rel": max_scale_rel,
+    return {"n_diff": n_diff, "n_bad": n_bad, "z_diff": z_diff, "z_bad": z_bad,
+            "max_scale_rel": max_scale_rel,
             "scale_bad": scale_bad, "scale_wide_over": scale_wide_over, "worst_scale": worst,
             "val_bad": val_bad, "max_val_rel": max_val_rel, "err": err,
             "count": int(mask_p.sum())}

@@ -493,7 +493,6 @@ gptq_status launch_colprod(dim3 grid, const T* W, int64_t o, int64_t i, const do
   return colprod_at<T, 32>(grid, W, o, i, Q, r, Zp, s);
 }
 
-bool g_orth_attr = false;
 
 template <typename T>
 gptq_status lowrank_impl(const T* W, int64_t o, int64_t i, const float* H, int64_t tokens,
@@ -502,11 +501,11 @@ gptq_status lowrank_impl(const T* W, int64_t o, int64_t i, const float* H, int64
   double *sq, *om, *Y, *Q, *Z, *Qi, *Zp, *Gp, *Rinv, *P;
   chmc_layout(o, i, r, ws, &sq, &om, &Y, &Q, &Z, &Qi, &Zp, &Gp, &Rinv, &P);
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
-  if (!g_orth_attr) {
-    GPTQ_CUDA(cudaFuncSetAttribute(chmc_orth_small_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)(sizeof(double) * ORTH_SMALL_MAX)));
-    g_orth_attr = true;
+  {
+    const gptq_status st = ensure_smem_limit((const void*)chmc_orth_small_kernel,
+                                             (int)(sizeof(double) * ORTH_SMALL_MAX),
+                                             "chmc_orth_small_kernel");
+    if (st != GPTQ_OK) return st;
   }
   if (r == 0) {
     GPTQ_LAUNCH(KK_CHMC, s, chmc_copy_kernel<T>, (unsigned)ceil_div(o * i, 256), 256, 0, W,

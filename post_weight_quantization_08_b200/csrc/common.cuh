@@ -38,6 +38,15 @@ void launch_end(int kind, cudaStream_t s);
 gptq_status fail(gptq_status st, const char* fmt, ...);
 gptq_status cuda_fail(cudaError_t e, const char* what);
 
+// Per-device set-up.  A kernel's dynamic shared-memory limit is an attribute
+// held by the device's context, and the SM count is a property of the device,
+// so both are kept per device ordinal, under a lock (one process may drive
+// several GPUs, from several host threads).  Each is set or read once per
+// device, with that device current; a device reset between calls is not
+// supported (the cached set-up would not be redone).
+gptq_status ensure_smem_limit(const void* kernel, int bytes, const char* name);
+gptq_status device_sm_count(int* sms);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

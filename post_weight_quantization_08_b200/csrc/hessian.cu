@@ -250,7 +250,6 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant
   if (warp == 0) tmem_dealloc(tmem, TC_TILE);
 }
 
-bool g_tc_attr = false;
 
 }  // namespace
 }  // namespace gptq
@@ -273,10 +272,10 @@ extern "C" gptq_status gptq_hessian_accumulate(const void* X, int64_t T, int64_t
     if (!encode_tiled_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, n, T, n * 2, 64, TC_KT) ||
         !encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, H, n, n, n * 4, 32, TC_TILE))
       return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the Hessian");
-    if (!g_tc_attr) {
-      GPTQ_CUDA(cudaFuncSetAttribute(hessian_tc_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM));
-      g_tc_attr = true;
+    {
+      const gptq_status st = ensure_smem_limit((const void*)hessian_tc_kernel, (int)TC_SMEM,
+                                               "hessian_tc_kernel");
+      if (st != GPTQ_OK) return st;
     }
     const int nt = (int)ceil_div(n, TC_TILE);
     GPTQ_LAUNCH(KK_HESSIAN, s, hessian_tc_kernel, nt * (nt + 1) / 2, 128, TC_SMEM, tm, th, T, n,

@@ -386,7 +386,6 @@ hptq_out_kernel(const int16_t* __restrict__ codes16, const int32_t* __restrict__
   if (Qdq != nullptr) Qdq[e] = scale[r * ngroups + p / group] * (float)q;
 }
 
-bool g_huf_attr = false;
 
 // One pass of slot `slot` at *alpha: sweep (unclipped), histogram, Huffman;
 // k ≥ 0: the bisection step on its cost; k < 0: the cost into *cost_out.
@@ -408,10 +407,10 @@ gptq_status hptq_pass(const HptqWs& h, int slot, const void* W, int w_dtype, int
   const unsigned gh = (unsigned)std::min<int64_t>(ceil_div(total, 512 * 8), 148 * 4);
   GPTQ_LAUNCH(KK_HPTQ, s, hptq_hist_kernel, gh > 0 ? gh : 1, 512, 0, h.codes16[slot], total,
               h.hist[slot], info);
-  if (!g_huf_attr) {
-    GPTQ_CUDA(cudaFuncSetAttribute(hptq_huffman_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HUF_SMEM));
-    g_huf_attr = true;
+  {
+    const gptq_status st = ensure_smem_limit((const void*)hptq_huffman_kernel, (int)HUF_SMEM,
+                                             "hptq_huffman_kernel");
+    if (st != GPTQ_OK) return st;
   }
   GPTQ_LAUNCH(KK_HPTQ, s, hptq_huffman_kernel, 1, 1024, HUF_SMEM, h.hist[slot], h.st, k,
               cost_out, limit, trace_alpha, trace_count, final_pass, h.lens, h.canon, info);

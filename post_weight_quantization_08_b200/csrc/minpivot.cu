@@ -272,9 +272,11 @@ gptq_status launch_min_pivot_order(const float* H, int64_t n, const double* mean
     if (dbytes + sizeof(double) * (size_t)n * (w + 1) <= budget) { pw = w; lp_smem = 1; break; }
   }
   const size_t panel_smem = dbytes + (lp_smem ? sizeof(double) * (size_t)n * (pw + 1) : 0);
-  if (panel_smem > 48 * 1024)
-    GPTQ_CUDA(cudaFuncSetAttribute(mp_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)panel_smem));
+  if (panel_smem > 48 * 1024) {
+    const gptq_status st = ensure_smem_limit((const void*)mp_panel_kernel, (int)panel_smem,
+                                             "mp_panel_kernel");
+    if (st != GPTQ_OK) return st;
+  }
   for (int64_t t0 = 0; t0 < n; t0 += pw) {
     GPTQ_LAUNCH(KK_PREP_ORDER, s, mp_panel_kernel, 1, MP_THREADS, panel_smem, S, n, ld, d, Lp,
                 elim, t0, pw, lp_smem, info);

@@ -1135,8 +1135,6 @@ prep_out_kernel(const double* __restrict__ M, int64_t n, int64_t np,
   U[e] = (j >= i) ? (float)M[(n - 1 - i) * np + (n - 1 - j)] : 0.0f;
 }
 
-bool g_smem_set = false;
-int g_num_sms = 148;
 
 }  // namespace
 }  // namespace gptq
@@ -1172,13 +1170,12 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
   const size_t tile_smem = (5 * NB * LDM + 192) * sizeof(double);
-  if (!g_smem_set) {
-    GPTQ_CUDA(cudaFuncSetAttribute(chol_persistent_kernel,
-              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tile_smem));
-    int dev = 0;
-    GPTQ_CUDA(cudaGetDevice(&dev));
-    GPTQ_CUDA(cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev));
-    g_smem_set = true;
+  int num_sms = 0;
+  {
+    gptq_status st = ensure_smem_limit((const void*)chol_persistent_kernel, (int)tile_smem,
+                                       "chol_persistent_kernel");
+    if (st == GPTQ_OK) st = device_sm_count(&num_sms);
+    if (st != GPTQ_OK) return st;
   }
 
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
@@ -1207,7 +1204,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   // step for its panel input, N²/3 ≈ 0.5 K), never more than one CTA per SM
   // besides the chain's, so that work on other streams finds SMs.
   int workers = N * N / 3 + 2;
-  if (workers > g_num_sms - 1) workers = g_num_sms - 1;
+  if (workers > num_sms - 1) workers = num_sms - 1;
   if (workers > ntasks) workers = ntasks;
   const int grid = 1 + workers;
   GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, n, np,

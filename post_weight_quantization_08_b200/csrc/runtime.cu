@@ -79,6 +79,60 @@ void launch_end(int kind, cudaStream_t s) {
   p.pending = false;
 }
 
+namespace {
+
+constexpr int kMaxDev = 128;
+
+struct DeviceSetup {
+  std::mutex mu;
+  // (device, kernel) pairs whose limit is set, with the limit
+  std::vector<std::pair<std::pair<int, const void*>, int>> smem;
+  int sms[kMaxDev] = {};
+};
+
+DeviceSetup& setup() {
+  static DeviceSetup d;
+  return d;
+}
+
+}  // namespace
+
+gptq_status ensure_smem_limit(const void* kernel, int bytes, const char* name) {
+  int dev = 0;
+  GPTQ_CUDA(cudaGetDevice(&dev));
+  DeviceSetup& d = setup();
+  std::lock_guard<std::mutex> lk(d.mu);
+  for (auto& e : d.smem)
+    if (e.first.first == dev && e.first.second == kernel) {
+      if (e.second >= bytes) return GPTQ_OK;
+      cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           bytes);
+      if (r != cudaSuccess) return cuda_fail(r, name);
+      e.second = bytes;
+      return GPTQ_OK;
+    }
+  cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bytes);
+  if (r != cudaSuccess) return cuda_fail(r, name);
+  d.smem.push_back({{dev, kernel}, bytes});
+  return GPTQ_OK;
+}
+
+gptq_status device_sm_count(int* sms) {
+  int dev = 0;
+  GPTQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDev) return fail(GPTQ_ERR_INVALID_ARG, "device ordinal %d", dev);
+  DeviceSetup& d = setup();
+  std::lock_guard<std::mutex> lk(d.mu);
+  if (d.sms[dev] == 0) {
+    int v = 0;
+    GPTQ_CUDA(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev));
+    d.sms[dev] = v;
+  }
+  *sms = d.sms[dev];
+  return GPTQ_OK;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;

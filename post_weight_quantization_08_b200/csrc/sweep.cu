@@ -680,9 +680,6 @@ sweep_kernel(const __grid_constant__ CUtensorMap tmEhi, const __grid_constant__ 
   }
 }
 
-bool g_attr_set[5] = {false, false, false, false, false};  // plain, row groups, outliers,
-                                                          // unclipped, static groups
-
 }  // namespace
 
 size_t panel_workspace_bytes(int64_t n, int block) {
@@ -718,14 +715,14 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
   const int variant = rowg ? 1
                       : (outl == nullptr ? 0
                                          : (outl->static_groups ? 4 : (outl->unclipped ? 3 : 2)));
-  if (!g_attr_set[variant]) {
+  {
     const void* fn = variant == 1 ? (const void*)sweep_kernel<true, 0>
                      : variant == 2 ? (const void*)sweep_kernel<false, 1>
                      : variant == 3 ? (const void*)sweep_kernel<false, 2>
                      : variant == 4 ? (const void*)sweep_kernel<false, 3>
                                     : (const void*)sweep_kernel<false, 0>;
-    GPTQ_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
-    g_attr_set[variant] = true;
+    const gptq_status st = ensure_smem_limit(fn, (int)kSmem, "sweep_kernel");
+    if (st != GPTQ_OK) return st;
   }
   const OutlierArgs oa = outl != nullptr ? *outl : OutlierArgs();
   // the far-column update riding along: fx 256-column tiles per 128-row tile

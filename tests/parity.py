@@ -9,8 +9,12 @@ Tolerances (written here, each derived from the arithmetic it checks):
   * quantize (oracle in follow mode on the GPU's own H/U): a code may differ
     only where the oracle's pre-rounding value lies within 1e-4 code units of
     a rounding boundary, and such codes are at most 0.1 % of all codes;
-    scales agree to 1e-5 relative; zeros are equal unless at such a near-tie;
+    scales agree to 1e-5 relative; zeros are equal unless at such a near-tie,
+    and such zero flips are at most 0.1 % of the (row, group) pairs (the same
+    cap as codes: a flipped zero is a rounding decision of the same kind);
     the layer loss agrees to 1e-3 relative.
+  * round-to-nearest dominance: the GPU result's layer loss tr((W−Q)H(W−Q)ᵀ)
+    does not exceed that of round-to-nearest with the same groups.
   * end to end (oracle from X alone, float64 throughout): layer loss to 1e-3
     relative.
 """
@@ -23,6 +27,7 @@ from oracle import gptq as og
 
 CODE_TOL = 1e-4
 CODE_FRAC = 1e-3
+ZERO_FRAC = 1e-3
 SCALE_RTOL = 1e-5
 LOSS_RTOL = 1e-3
 
@@ -109,6 +114,7 @@ def check_quantize(W, out, ref_prep_U, bits, group, block, rows=None):
     assert f["code_diff"] <= CODE_FRAC * f["codes"], f
     assert f["max_scale_rel"] <= SCALE_RTOL, f
     assert f["zero_diff_disallowed"] == 0, f
+    assert f["zero_diff"] <= ZERO_FRAC * out["scale"][sel].size, f
     lg = out["loss_row"][sel].astype(np.float64)
     lo = f["loss_rows"]
     assert abs(lg.sum() - lo.sum()) <= LOSS_RTOL * lo.sum(), (lg.sum(), lo.sum())
@@ -135,10 +141,28 @@ def check_layer_loss(X, W, out, bits, group, block, damp, order, perm=None):
     Wf = W.to(torch.float64).numpy()
     H = og.hessian(Xf)
     ref = og.gptq_layer(Wf, H, bits, group, block, damp, order, perm)
-    g = out["g_idx"]
-    Q = out["scale"][:, g].astype(np.float64) * (out["codes"] - out["zero"][:, g].astype(np.float64))
-    lg = og.layer_loss(Wf, Q, H)
+    lg = og.layer_loss(Wf, dequantized(out), H)
     rel = abs(lg - ref["loss"]) / ref["loss"]
     assert rel <= LOSS_RTOL, (lg, ref["loss"], rel)
     return {"loss_gpu": lg, "loss_oracle": ref["loss"], "loss_rel": rel,
             "code_agree": float(np.mean(ref["codes"] == out["codes"]))}
+
+
+def dequantized(out):
+    """Q = s·(q − z) in float64 from the GPU's codes, scales, zeros and g_idx."""
+    g = out["g_idx"]
+    return out["scale"][:, g].astype(np.float64) * (
+        out["codes"] - out["zero"][:, g].astype(np.float64))
+
+
+def check_rtn_dominance(W, out, H, bits, group):
+    """The GPU result's layer loss does not exceed round-to-nearest's (min-max
+    groups of the original W along the input channels), both measured with
+    the same float64 H."""
+    from oracle import lattice as ol
+    Wf = W.to(torch.float64).numpy() if isinstance(W, torch.Tensor) else np.asarray(W, np.float64)
+    H = np.asarray(H, dtype=np.float64)
+    lg = og.layer_loss(Wf, dequantized(out), H)
+    lr = og.layer_loss(Wf, ol.rtn_dequant(Wf, bits, group), H)
+    assert lg <= lr, (lg, lr)
+    return {"loss_gpu_undamped": lg, "loss_rtn": lr, "loss_over_rtn": lg / lr}

@@ -110,6 +110,7 @@ def test_quantize_rowgroups_matches_oracle(m, n, bits, block, order):
                             codes[:, perm], scale[:, perm], zero[:, perm])
     assert f["n_bad"] == 0 and f["z_bad"] == 0, f
     assert f["n_diff"] <= P.CODE_FRAC * m * n, f
+    assert f["z_diff"] <= P.ZERO_FRAC * zero.size, f
     assert f["max_scale_rel"] <= P.SCALE_RTOL, f
     loss_or = float(np.sum(f["err"] ** 2))
     loss_gpu = float(q["loss_row"].cpu().to(torch.float64).sum())

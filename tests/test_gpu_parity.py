@@ -34,6 +34,8 @@ def _full_check(X, W, bits, group, block, order="natural", damp=0.01, perm=None)
     stats.update(s2)
     stats.update(P.check_quantize(W, out, None, bits, group, block))
     stats.update(P.check_layer_loss(X, W, out, bits, group, block, damp, order, perm))
+    Xf = X.to(torch.bfloat16).to(torch.float64).numpy()
+    stats.update(P.check_rtn_dominance(W, out, og.hessian(Xf), bits, group))
     return out, stats
 
 

@@ -83,6 +83,7 @@ def _check_outputs(q, W, Wz, prep, U32, bits, group, block, alpha):
                         codes[:, perm], mask[:, perm], vals[:, perm], scale, zero)
     assert f["n_bad"] == 0 and f["z_bad"] == 0, f
     assert f["n_diff"] <= P.CODE_FRAC * m * n, f
+    assert f["z_diff"] <= P.ZERO_FRAC * zero.size, f
     assert f["scale_bad"] == 0 and f["scale_wide_over"] == 0 and f["val_bad"] == 0, f
     if n % group == 0 or n % group >= 32:
         assert f["max_scale_rel"] <= P.SCALE_RTOL, f

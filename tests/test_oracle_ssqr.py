@@ -326,6 +326,7 @@ def test_follow_accepts_a_zero_point_flipped_at_a_tie():
     f = S.follow_ssqr(W, np.eye(4), 4, 4, 4, 1.0, q, np.zeros((1, 4), bool),
                       np.zeros((1, 4)), s[:, None], np.array([[z2]], np.float32))
     assert f["z_bad"] == 0 and f["n_bad"] == 0 and f["n_diff"] == 0
+    assert f["z_diff"] == 1                # counted toward the cap on zero flips
 
 
 def test_follow_bounds_flag_a_planted_scale_and_value_error():
