@@ -131,6 +131,18 @@ gptq_status gptq_prepare(const float* H, int64_t n, double damp, int order,
                          void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Polls each bounded wait of gptq_prepare's dataflow factorisation makes
+ * (one launch whose CTAs wait on each other's tiles through flags in the
+ * workspace) before it gives up, reports GPTQ_ERR_TIMEOUT through info,
+ * raises the launch's abort flag so that every CTA returns, and leaves U
+ * undefined.  0 restores the default, 2^22 polls with a back-off of 64 ns
+ * after the first 32 (a few seconds).  Process-wide, read at each
+ * gptq_prepare call.  A small limit makes the time-out path run on purpose
+ * (tests of failure detection); normal use never needs to set it.
+ */
+void gptq_set_wait_limit(uint32_t polls);
+
+/*
  * gptq_prepare without a workspace argument: the same operation, arguments
  * and results as gptq_prepare, for callers that cannot hand this library a
  * block of device memory — for example code that runs while another

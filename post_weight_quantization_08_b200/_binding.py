@@ -73,6 +73,7 @@ _SIGS = {
                                      C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
+    "gptq_set_wait_limit": (None, [C.c_uint32]),
     "gptq_check": (C.c_int, [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]),
     "gptq_last_error": (C.c_char_p, []),
     "gptq_status_string": (C.c_char_p, [C.c_int]),

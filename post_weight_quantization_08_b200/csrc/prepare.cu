@@ -18,6 +18,7 @@
 //             block row k of L⁻¹
 //   trail(k): A_ij −= L_ik·L_jkᵀ (k < j ≤ i);  M_ic −= L_ik·M_kc (i > k, c ≤ k)
 // A is padded with an identity block to a multiple of 64.
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -194,7 +195,9 @@ __constant__ unsigned char kTri8I[36] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3, 4, 4, 4, 
 __constant__ unsigned char kTri8J[36] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3, 0, 1, 2, 3, 4, 0, 1, 2,
                                          3, 4, 5, 0, 1, 2, 3, 4, 5, 6, 0, 1, 2, 3, 4, 5, 6, 7};
 
-constexpr uint32_t kSpinLimit = 1u << 22;   // ≈ a few seconds with the back-off below
+// Polls a bounded wait makes before it reports GPTQ_ERR_TIMEOUT (≈ a few
+// seconds with the back-off below); gptq_set_wait_limit() may lower it.
+constexpr uint32_t kSpinLimit = 1u << 22;
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
@@ -215,6 +218,7 @@ struct TilePrefetch {
   double (*dst[2])[LDM];
   int64_t ld;
   int count;
+  uint32_t spin;     // polls before the prefetcher leaves the tiles to the panel phase
 };
 
 // The panel of the step before, still in shared memory (src), goes to global
@@ -426,7 +430,7 @@ __device__ __forceinline__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM
     }
     int got = 0;
     const int all = (1 << pf.count) - 1;
-    for (uint32_t it = 0; it < kSpinLimit && got != all; ++it) {
+    for (uint32_t it = 0; it < pf.spin && got != all; ++it) {
       int ready = 0;
       if (lane == 0) {
         for (int t2 = 0; t2 < pf.count; ++t2)
@@ -832,10 +836,11 @@ __device__ CholSync sync_view(int* base, int N) {
 }
 
 // Whole-CTA bounded wait for *flag ≥ target; false on abort or time-out.
-__device__ bool cta_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok) {
+__device__ bool cta_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok,
+                         uint32_t limit) {
   if (threadIdx.x == 0) {
     bool ok = false;
-    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
       if (ld_acquire(flag) >= target) { ok = true; break; }
       if (*reinterpret_cast<volatile int*>(abortp)) break;
       if (it > 32) __nanosleep(64);
@@ -854,10 +859,11 @@ __device__ bool cta_wait(const int* flag, int target, int* abortp, int32_t* info
 
 // The same wait for warps 0–3 and 5–7 (thread 0 polls), joined by barrier
 // kBarChain.
-__device__ bool group_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok) {
+__device__ bool group_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok,
+                           uint32_t limit) {
   if (threadIdx.x == 0) {
     bool ok = false;
-    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
       if (ld_acquire(flag) >= target) { ok = true; break; }
       if (*reinterpret_cast<volatile int*>(abortp)) break;
       if (it > 32) __nanosleep(64);
@@ -936,7 +942,7 @@ __device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) 
 __global__ void __launch_bounds__(256, 1)
 chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int64_t n, int64_t np, int N,
-                       int ntasks, int* sync_base, int32_t* info) {
+                       int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
   __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail;
   __shared__ volatile int s_stop;
@@ -987,6 +993,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       // warp 4 fetches the next step's two input tiles during the diagonal
       // tile, as soon as the workers have finished them
       TilePrefetch pf = {};
+      pf.spin = spin;
       if (more) {
         pf.count = 2;
         pf.flag[0] = &S.upd[(k + 1) * N + k];
@@ -1029,7 +1036,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
         if (got) bar_sync(kBarFetch, kHand + 32);
         // L_{k+1,k} = A_{k+1,k}·D_kᵀ
         if (!(got & 1)) {
-          ok = group_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok);
+          ok = group_wait(&S.upd[(k + 1) * N + k], k, &S.ctrl[2], info, &s_ok, spin);
           if (ok) {
             copy_tile_async_group(x, Lp, np, gt);
             copy_wait_all();
@@ -1043,7 +1050,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
           panel_to_smem(x, acc, warp, lane);
           // A_{k+1,k+1} −= L_{k+1,k}·L_{k+1,k}ᵀ, in shared memory
           if (!(got & 2)) {
-            ok = group_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok);
+            ok = group_wait(&S.upd[(k + 1) * N + k + 1], k, &S.ctrl[2], info, &s_ok, spin);
             if (ok) {
               copy_tile_async_group(an, An, np, gt);
               copy_wait_all();
@@ -1074,8 +1081,8 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     decode_task(task, N, kind, k, i, j);
     double acc[2][4][2] = {};
     if (kind == T_PANEL) {
-      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) return;
-      if (!cta_wait(&S.upd[i * N + k], k, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok, spin)) return;
+      if (!cta_wait(&S.upd[i * N + k], k, &S.ctrl[2], info, &s_ok, spin)) return;
       double* out = A + (int64_t)i * NB * np + (int64_t)k * NB;
       load_tile(x, out, np, false, tid);
       load_tile(y, M + (int64_t)k * NB * np + (int64_t)k * NB, np, true, tid);
@@ -1085,8 +1092,8 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       cta_signal(&S.pdone[k * N + i], 1);
     } else if (kind == T_MROW) {
       const int c = j;
-      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) return;
-      if (!cta_wait(&S.mupd[k * N + c], k - c, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok, spin)) return;
+      if (!cta_wait(&S.mupd[k * N + c], k - c, &S.ctrl[2], info, &s_ok, spin)) return;
       double* out = M + (int64_t)k * NB * np + (int64_t)c * NB;
       load_tile(x, M + (int64_t)k * NB * np + (int64_t)k * NB, np, false, tid);
       load_tile(y, out, np, false, tid);
@@ -1095,9 +1102,9 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       tile_store<false>(out, np, acc, warp, lane);
       cta_signal(&S.mdone[k * N + c], 1);
     } else if (kind == T_TRAIL) {
-      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok)) return;
-      if (j != i && !cta_wait(&S.pdone[k * N + j], 1, &S.ctrl[2], info, &s_ok)) return;
-      if (!cta_wait(&S.upd[i * N + j], k, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok, spin)) return;
+      if (j != i && !cta_wait(&S.pdone[k * N + j], 1, &S.ctrl[2], info, &s_ok, spin)) return;
+      if (!cta_wait(&S.upd[i * N + j], k, &S.ctrl[2], info, &s_ok, spin)) return;
       double* out = A + (int64_t)i * NB * np + (int64_t)j * NB;
       load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
       load_tile(y, A + (int64_t)j * NB * np + (int64_t)k * NB, np, true, tid);
@@ -1107,13 +1114,13 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       cta_signal(&S.upd[i * N + j], k + 1);
     } else {   // T_MTRAIL
       const int c = j;
-      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok, spin)) return;
       if (c < k) {
-        if (!cta_wait(&S.mdone[k * N + c], 1, &S.ctrl[2], info, &s_ok)) return;
-      } else if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok)) {
+        if (!cta_wait(&S.mdone[k * N + c], 1, &S.ctrl[2], info, &s_ok, spin)) return;
+      } else if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok, spin)) {
         return;
       }
-      if (!cta_wait(&S.mupd[i * N + c], k - c, &S.ctrl[2], info, &s_ok)) return;
+      if (!cta_wait(&S.mupd[i * N + c], k - c, &S.ctrl[2], info, &s_ok, spin)) return;
       double* out = M + (int64_t)i * NB * np + (int64_t)c * NB;
       load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
       load_tile(y, M + (int64_t)k * NB * np + (int64_t)c * NB, np, false, tid);
@@ -1124,6 +1131,9 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     }
   }
 }
+
+// Host side: the poll limit of the factorisation's waits (0: kSpinLimit).
+std::atomic<uint32_t> g_wait_limit{0};
 
 // U[i][j] = L⁻¹[n−1−i][n−1−j] for j ≥ i, 0 below the diagonal.
 __global__ void __launch_bounds__(256)
@@ -1140,6 +1150,10 @@ prep_out_kernel(const double* __restrict__ M, int64_t n, int64_t np,
 }  // namespace gptq
 
 using namespace gptq;
+
+extern "C" void gptq_set_wait_limit(uint32_t polls) {
+  g_wait_limit.store(polls, std::memory_order_relaxed);
+}
 
 extern "C" size_t gptq_prepare_workspace_bytes(int64_t n) {
   if (n < 1) return 0;
@@ -1207,8 +1221,9 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   if (workers > num_sms - 1) workers = num_sms - 1;
   if (workers > ntasks) workers = ntasks;
   const int grid = 1 + workers;
+  const uint32_t lim = g_wait_limit.load(std::memory_order_relaxed);
   GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, n, np,
-              N, ntasks, w.sync, info);
+              N, ntasks, w.sync, info, lim != 0 ? lim : kSpinLimit);
   GPTQ_LAUNCH(KK_PREP_OUT, s, prep_out_kernel, (unsigned)ceil_div(n * n, 256), 256, 0,
               w.M, n, np, U);
   return GPTQ_OK;

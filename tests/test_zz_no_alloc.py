@@ -3,7 +3,10 @@ memory to the library (it uses a fixed scratch array inside the library).
 
 Called through the C ABI and compared with gptq_prepare on the same inputs,
 twice in a row with different problems, so that leftovers of the first call
-in the shared scratch would show up in the second.  Collected last (file
+in the shared scratch would show up in the second.  The second pair runs at the
+size limit itself, where the scratch is used to its last byte, with the
+min-pivot order first (it reuses the scratch's two float64 arrays for a
+factorisation of its own before the regular one overwrites them).  Collected last (file
 name) so that a run stopping at the first failure has run everything else.
 """
 import ctypes as C
@@ -52,7 +55,8 @@ def _hessian(T, n, seed):
     return g.hessian(X)
 
 
-@pytest.mark.parametrize("first,second", [((576, "act", 1), (320, "natural", 2))])
+@pytest.mark.parametrize("first,second", [((576, "act", 1), (320, "natural", 2)),
+                                          ((1024, "minpivot", 3), (1024, "reverse", 4))])
 def test_noalloc_matches_prepare_twice(first, second):
     for n, order, seed in (first, second):
         H = _hessian(1024, n, seed)
