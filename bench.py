@@ -150,8 +150,40 @@ def _peaks():
 
 
 def fp64_peak_tflops(sm_mhz: float) -> float:
-    """B200 float64: 148 SMs × 64 FP64 FMA lanes × 2 flops × clock."""
+    """B200 float64 from the data sheet's unit counts: 148 SMs × 64 FP64 FMA
+    lanes × 2 flops × clock (context beside the probed figure)."""
     return 148 * 64 * 2 * sm_mhz * 1e6 / 1e12
+
+
+PROBE_ITERS = {"fp64": (0, 32768), "tf32": (1, 65536), "bf16": (2, 65536)}
+
+
+def probe_peaks(device) -> dict:
+    """Measured pipe rates (TFLOP/s) from the library's peak probes: float64
+    tensor-core products, tcgen05 TF32 and tcgen05 bf16 (a check of the
+    probe against the cuBLAS bf16 figure).  Each probe runs ~20 ms; best of 3
+    launches after one warm-up, CUDA events on the launching stream."""
+    from post_weight_quantization_08_b200 import _binding as b
+    info = torch.zeros(2, dtype=torch.int32, device=device)
+    sink = torch.zeros(1, dtype=torch.float64, device=device)
+    s = torch.cuda.current_stream(device)
+    out = {}
+    for name, (kind, iters) in PROBE_ITERS.items():
+        best = None
+        for rep in range(4):
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            flops = b.gptq_peak_probe(kind, iters, info, sink, s)
+            e.record(s)
+            e.synchronize()
+            if rep > 0:
+                t = flops / (a.elapsed_time(e) / 1e3) / 1e12
+                best = t if best is None else max(best, t)
+        st, _ = b.gptq_check(info, s)
+        if st != 0:
+            raise RuntimeError(f"peak probe {name}: device status {st}")
+        out[name] = round(best, 1)
+    return out
 
 
 def kernel_work(probs, block: int):

@@ -131,6 +131,26 @@ gptq_status gptq_prepare(const float* H, int64_t n, double damp, int order,
                          void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Peak probe (a measurement aid; the pages have no counterpart): one launch
+ * that keeps a single arithmetic pipe busy, for the roofline denominators of
+ * the kernels that use it.  The caller times the launch with CUDA events on
+ * `stream` and divides *flops by the time.
+ *   kind 0  float64 tensor-core products (mma.sync m8n8k4), 4 CTAs of 8 warps
+ *           per SM, each warp 8 independent accumulators, `iters` rounds;
+ *   kind 1  tcgen05.mma kind::tf32 128×256×8 from shared memory into tensor
+ *           memory, one CTA per SM, 4·iters products each;
+ *   kind 2  the same with kind::f16 on bf16 operands (K = 16).
+ *   flops  host, output: the floating-point operations of the launch
+ *          (2 per multiply-add).
+ *   info   int32[2] on the device: a bounded wait that runs out sets TIMEOUT.
+ *   sink   ≥ 8 bytes of device memory (never written in practice; it keeps
+ *          the products from being optimised away).
+ * Errors: INVALID_ARG (kind outside 0..2, iters < 1, a null pointer), CUDA.
+ */
+gptq_status gptq_peak_probe(int kind, int64_t iters, double* flops, int32_t* info, void* sink,
+                            void* stream);
+
+/*
  * Polls each bounded wait of gptq_prepare's dataflow factorisation makes
  * (one launch whose CTAs wait on each other's tiles through flags in the
  * workspace) before it gives up, reports GPTQ_ERR_TIMEOUT through info,

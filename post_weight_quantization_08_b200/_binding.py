@@ -74,6 +74,8 @@ _SIGS = {
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
     "gptq_set_wait_limit": (None, [C.c_uint32]),
+    "gptq_peak_probe": (C.c_int, [C.c_int, C.c_int64, C.POINTER(C.c_double), C.c_void_p,
+                                  C.c_void_p, C.c_void_p]),
     "gptq_check": (C.c_int, [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]),
     "gptq_last_error": (C.c_char_p, []),
     "gptq_status_string": (C.c_char_p, [C.c_int]),
@@ -387,6 +389,17 @@ def gptq_check(info, stream=None) -> tuple[int, int]:
     if st == 6:
         _raise(st)
     return int(st), int(idx.value)
+
+
+def gptq_peak_probe(kind: int, iters: int, info, sink, stream=None) -> float:
+    """Launch one peak probe (0 float64, 1 TF32, 2 bf16) on ``stream``; returns
+    the launch's floating-point operations (time it with CUDA events)."""
+    _need(info, "info", torch.int32, (2,))
+    _need(sink, "sink", torch.float64)
+    flops = C.c_double(0.0)
+    _raise(lib().gptq_peak_probe(int(kind), int(iters), C.byref(flops), _ptr(info), _ptr(sink),
+                                 _stream(stream, info.device)))
+    return float(flops.value)
 
 
 def gptq_launch_count() -> int:

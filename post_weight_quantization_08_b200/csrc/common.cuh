@@ -25,6 +25,7 @@ enum KernelKind : int {
   KK_CHMC,            // CHMC frontend: activation energies, randomized subspace iteration, residual
   KK_SSQR,            // SSQR: the binary search's state, the outlier list
   KK_HPTQ,            // HPTQ: histogram, Huffman code and search step, encoder
+  KK_PROBE,           // peak probes (float64, TF32, bf16 tensor pipes)
   KK_COUNT
 };
 

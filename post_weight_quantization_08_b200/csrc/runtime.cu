@@ -21,7 +21,7 @@ std::atomic<uint64_t> g_launches{0};
 const char* const kKindNames[KK_COUNT] = {
     "hessian",  "prep_stats", "prep_order", "prep_gather", "cholesky",
     "prep_out", "ingest",     "sweep",      "trailing",    "pack",
-    "chmc",     "ssqr",       "hptq"};
+    "chmc",     "ssqr",       "hptq",        "probe"};
 
 struct Profiler {
   std::mutex mu;
