@@ -67,16 +67,26 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
 
 
 def workload_name(cid: int, bits: int, order: str | None = None,
-                  static_groups: bool = False) -> str:
+                  static_groups: bool = False, layers: int = 1) -> str:
     c = CONFIGS[cid]
     tail = ("" if order is None else f", {order} order") + (", static groups" if static_groups
                                                             else "")
     if c["kind"] == "decoder":
         h, kv, it = c["hidden"], c["kv"], c["inter"]
         rows = 2 * h + 2 * kv + 2 * it
+        scope = "per layer" if layers == 1 else f"{layers} layers per step"
         return (f"{c['name']}: q/k/v/o/gate/up {rows}x{h} on one H + down {h}x{it}, "
-                f"T={c['T']} cone tokens, {bits}-bit g128 b128 damp0.01, per layer{tail}")
+                f"T={c['T']} cone tokens, {bits}-bit g128 b128 damp0.01, {scope}{tail}")
     return f"{c['name']}: W {c['m']}x{c['n']}, T={c['T']}, {bits}-bit g128 b128 damp0.01{tail}"
+
+
+def stack_layers(args) -> int:
+    """Layers quantized per step: every layer of a decoder stack (--layers
+    limits it), one for the single and stress layers."""
+    c = CONFIGS[args.config]
+    if c["kind"] != "decoder":
+        return 1
+    return max(1, min(int(args.layers or c["layers"]), c["layers"]))
 
 
 # ---------------------------------------------------------------- clocks
@@ -186,20 +196,33 @@ def probe_peaks(device) -> dict:
     return out
 
 
+def chol_tile_flops(n: int) -> float:
+    """Floating-point operations the factorisation executes: its 64×64 tile
+    products (padded to whole tiles) and the diagonal tiles' Cholesky and
+    inverse (2·64³/3 each)."""
+    N = -(-n // 64)
+    f = 0.0
+    for k in range(N):
+        r = N - k - 1
+        f += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
+        f += 2 * 64 ** 3 / 3
+    return f
+
+
 def kernel_work(probs, block: int):
     """Algorithmic work per kernel kind for one step: {kind: (unit, amount)}.
 
-    hessian   flops T·n·(n+1)               (upper triangle incl. diagonal)
-    cholesky  flops of the executed float64 tile products (Σ_k tiles·2·64³)
-              plus the diagonal tiles' Cholesky and inverse (2·64³/3 each)
-    sweep     bytes: strip read + Err write (4+4 B) + codes (1 B) per element,
-              U panel 4·bw², scale+zero 5 B per (row, group); on the
-              tensor-core path (n % 4 == 0) also the trailing update's bytes
-              (W read+write 8 B per trailing element, Err 4·m·bw, U panel
-              4·bw·N2): its near columns run in the sweep's prologue and its
-              far columns in CTAs of the sweep's own launch
-    trailing  bytes: the transposed TF32 split of U (12 B per element) on
-              the tensor-core path, else the SIMT trailing update's bytes
+    hessian   flops T·n(n+1) (the upper triangle with the diagonal)
+    cholesky  flops 2n³/3 (Cholesky of the reversed matrix and its triangular
+              inverse; the executed, tile-padded figure is reported beside it)
+    sweep     bytes per block: strip read + Err write (4 + 4 B) + codes (1 B)
+              per element, the U panel 4·bw², scale + zero 5 B per (row,
+              group); on the tensor-core path (n % 4 == 0) also the trailing
+              update's bytes (W read + write 8 B per trailing element, Err
+              4·m·bw, the U panel 4·bw·N2), since its near columns run in the
+              sweep's prologue and its far columns in CTAs of the sweep's launch
+    trailing  bytes: the transposed TF32 split of U (12 B per element) on the
+              tensor-core path, else the SIMT trailing update's bytes
     pack      bytes: codes 1 B + packed bits/8 B per element, scale/zero
     ingest    bytes: W in (2 or 4 B) + float32 out per element
     """
@@ -207,11 +230,7 @@ def kernel_work(probs, block: int):
     for p in probs:
         m, n, T = p.m, p.n, p.T
         w["hessian"] += T * n * (n + 1)
-        N = -(-n // 64)
-        for k in range(N):
-            r = N - k - 1
-            w["cholesky"] += (r * (r + 1) // 2 + r * (k + 1) + r + k) * 2 * 64 ** 3
-            w["cholesky"] += 2 * 64 ** 3 / 3         # Cholesky + inverse of a tile
+        w["cholesky"] += 2.0 * n ** 3 / 3.0
         ng = -(-n // p.group)
         fused = n % 4 == 0 and n > block
         if fused:
@@ -227,6 +246,56 @@ def kernel_work(probs, block: int):
     units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s",
              "sweep": "GB/s", "trailing": "GB/s", "pack": "GB/s", "ingest": "GB/s"}
     return {k: (units[k], v) for k, v in w.items()}
+
+
+def trailing_flops(probs, block: int) -> float:
+    """Flops of the lazy-batch trailing update, 2·m·bw·N2 per block (the
+    sweep launches carry it on the tensor-core path)."""
+    f = 0.0
+    for p in probs:
+        for j0 in range(0, p.n, block):
+            bw = min(block, p.n - j0)
+            f += 2.0 * p.m * bw * (p.n - j0 - bw)
+    return f
+
+
+def kernel_figures(work, kprof, steps, peaks, src, probed):
+    """Per kernel kind: device time per step (the library's event profiler),
+    achieved = algorithmic work ÷ time, and the fraction of its peak: HBM copy
+    bandwidth and bf16 from MEASURED_PEAKS.json, float64 from the library's
+    probe (the data-sheet unit count otherwise).  Returns (kernels, roofline
+    of the kind with the largest time)."""
+    fp64 = probed.get("fp64") if isinstance(probed, dict) else None
+    fp64_src = "fp64 DMMA probe, measured" if fp64 else "fp64 148 SMs x 64 FMA x 2 x max clock"
+    fp64 = fp64 or fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+    kernels = {}
+    for k, (unit, amount) in work.items():
+        if k not in kprof or kprof[k][1] <= 0 or amount <= 0:
+            continue
+        ms = kprof[k][0] / steps
+        if unit == "TFLOP/s":
+            ach = amount / (ms / 1e3) / 1e12
+            if k == "hessian":
+                bound, peak, note = "tensor", peaks["bf16_tflops"], f"bf16 burst, {src}"
+            else:
+                bound, peak, note = "tensor", fp64, fp64_src
+        else:
+            ach = amount / (ms / 1e3) / 1e9
+            bound, peak, note = "hbm", peaks["hbm_gbs"], f"copy bandwidth, {src}"
+        kernels[k] = {"ms_per_step": round(ms, 4), "launches_per_step": kprof[k][1] / steps,
+                      "bound": bound, "achieved": round(ach, 2), "unit": unit,
+                      "peak": round(peak, 1), "frac": round(ach / peak, 4),
+                      "peak_source": note}
+    roof = None
+    if kernels:
+        tot = sum(v["ms_per_step"] for v in kernels.values())
+        dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+        d = kernels[dom]
+        roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"],
+                "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+                "peak_source": d["peak_source"], "launches_per_step": d["launches_per_step"],
+                "share": round(d["ms_per_step"] / max(1e-9, tot), 4)}
+    return kernels, roof
 
 
 def traffic_for(kernel: str, workload: str):
@@ -250,12 +319,24 @@ def traffic_for(kernel: str, workload: str):
 
 # ---------------------------------------------------------------- the GPU arm
 
-class Layer:
-    """Device buffers of one layer's problems, allocated once; with
-    ``static_groups`` the quantize call fixes every group's parameters from
-    the original weights (gptq_quantize_static)."""
+def est_cost(p) -> float:
+    """Relative device time of one problem, for spreading problems over lanes:
+    the float64 factorisation (2n³/3 at ≈ 30 TFLOP/s) plus the 3×TF32 trailing
+    update (3·m·n² at ≈ 1 PFLOP/s)."""
+    return (2.0 / 3.0) * p.n ** 3 / 30e12 + 3.0 * p.m * p.n * p.n / 1e15
 
-    def __init__(self, probs, device, static_groups=False):
+
+class Job:
+    """Device buffers of a list of problems (every layer of a stack), allocated
+    once.  The problems run on ``lanes`` streams: each lane takes its share one
+    after the other, the lanes side by side; problems go, most expensive first,
+    to the lane with the least work so far.  With ``static_groups`` the
+    quantize call fixes every group's parameters from the original weights
+    (gptq_quantize_static)."""
+
+    OUTS = ("qweight", "scale", "zero", "g_idx", "loss")
+
+    def __init__(self, probs, device, lanes, static_groups=False):
         import post_weight_quantization_08_b200 as g
         self.g = g
         self.probs = probs
@@ -266,7 +347,7 @@ class Layer:
             m, n = p.m, p.n
             ng = -(-n // p.group)
             nw = -(-n * p.bits // 32)
-            it = {
+            self.items.append({
                 "p": p,
                 "X": p.X.to(device).contiguous(),
                 "W": p.W.to(device).contiguous(),
@@ -284,17 +365,22 @@ class Layer:
                 "zero": torch.empty(m, ng, dtype=torch.uint8, device=device),
                 "g_idx": torch.empty(n, dtype=torch.int32, device=device),
                 "loss": torch.empty(m, dtype=torch.float32, device=device),
-                "stream": torch.cuda.Stream(device=device),
-                "cstream": torch.cuda.Stream(device=device),
-            }
-            self.items.append(it)
+            })
+        nl = max(1, min(int(lanes), len(probs)))
+        self.lanes = [{"s": torch.cuda.Stream(device=device),
+                       "cs": torch.cuda.Stream(device=device), "plan": [], "load": 0.0}
+                      for _ in range(nl)]
+        for k in sorted(range(len(probs)), key=lambda k: -est_cost(probs[k])):
+            lane = min(self.lanes, key=lambda ln: ln["load"])
+            lane["plan"].append(k)
+            lane["load"] += est_cost(probs[k])
 
-    OUTS = ("qweight", "scale", "zero", "g_idx", "loss")
-
-    def run_problem(self, it, w_ready=None, host=None):
-        """One problem on its stream; ``w_ready``: the event after which W is
-        in place; ``host``: pinned buffers that receive the results."""
-        g, p, s = self.g, it["p"], it["stream"]
+    def run_problem(self, it, s, x_ready=None, w_ready=None, host=None):
+        """One problem on stream ``s``; ``x_ready`` / ``w_ready``: events after
+        which X / W are in place; ``host``: pinned buffers for the results."""
+        g, p = self.g, it["p"]
+        if x_ready is not None:
+            s.wait_event(x_ready)
         with torch.cuda.stream(s):
             it["H"].zero_()
         g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
@@ -311,63 +397,52 @@ class Layer:
                     host[k].copy_(it[k], non_blocking=True)
 
     def step(self, main, hosts=None):
-        """Fork the layer's problems onto their own streams, join on `main`.
+        """Fork the lanes off ``main`` and join them back.
 
         ``hosts``: per problem pinned input/output buffers (the end-to-end
-        step).  Then every problem's X is copied in first, largest n first
-        (the problem on the critical path starts earliest), each problem starts
-        as soon as its own X is in, and the W copies follow on copy streams of
-        their own while the factorisations run; each quantize waits only for
-        its W."""
+        step).  Each lane's copy stream then brings in, in the lane's order,
+        every problem's X and then its W, ahead of the compute; a problem
+        starts once its X is in and quantizes once its W is in, and its
+        results go back to the host on the lane's stream."""
         fork = torch.cuda.Event()
         fork.record(main)
         joins = []
-        order = list(range(len(self.items)))
-        w_ready = [None] * len(self.items)
-        if hosts is not None:
-            order.sort(key=lambda k: -self.items[k]["p"].n)
-            prev = None
-            for k in order:                      # X, in priority order
-                it, s = self.items[k], self.items[k]["stream"]
-                s.wait_event(fork)
-                if prev is not None:
-                    s.wait_event(prev)
-                with torch.cuda.stream(s):
-                    it["X"].copy_(hosts[k]["X"], non_blocking=True)
-                prev = torch.cuda.Event()
-                prev.record(s)
-            for k in order:                      # then W, on the copy streams
-                it, cs = self.items[k], self.items[k]["cstream"]
-                cs.wait_event(prev)
-                with torch.cuda.stream(cs):
-                    it["W"].copy_(hosts[k]["W"], non_blocking=True)
-                prev = torch.cuda.Event()
-                prev.record(cs)
-                w_ready[k] = prev
-        for k in order:
-            it = self.items[k]
-            it["stream"].wait_event(fork)
-            self.run_problem(it, w_ready[k], hosts[k] if hosts is not None else None)
+        for lane in self.lanes:
+            s, cs = lane["s"], lane["cs"]
+            s.wait_event(fork)
+            ready = []
+            if hosts is not None:
+                cs.wait_event(fork)
+                for k in lane["plan"]:
+                    it = self.items[k]
+                    evs = []
+                    with torch.cuda.stream(cs):
+                        for key in ("X", "W"):
+                            it[key].copy_(hosts[k][key], non_blocking=True)
+                            e = torch.cuda.Event()
+                            e.record(cs)
+                            evs.append(e)
+                    ready.append(evs)
+            for r, k in enumerate(lane["plan"]):
+                xr, wr = ready[r] if hosts is not None else (None, None)
+                self.run_problem(self.items[k], s, xr, wr,
+                                 hosts[k] if hosts is not None else None)
             e = torch.cuda.Event()
-            e.record(it["stream"])
+            e.record(s)
             joins.append(e)
         for e in joins:
             main.wait_event(e)
 
     def step_serial(self, main):
-        """Every problem on `main`, one after the other (for kernel timing)."""
+        """Every problem on ``main``, one after the other (for kernel timing)."""
         for it in self.items:
-            s = it["stream"]
-            it["stream"] = main
-            try:
-                self.run_problem(it)
-            finally:
-                it["stream"] = s
+            self.run_problem(it, main)
 
     def check(self):
+        s = self.lanes[0]["s"]
         for it in self.items:
             for key in ("info_h", "info_p", "info_q"):
-                st, idx = self.g.gptq_check(it[key], it["stream"])
+                st, idx = self.g.gptq_check(it[key], s)
                 if st != 0:
                     raise RuntimeError(f"device reported status {st} at {idx}")
 
@@ -378,8 +453,11 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(device)
     cfg = CONFIGS[args.config]
     bits = args.bits or cfg["bits"][0]
-    probs = problems_for(args.config, layer=layer_for_rank(rank), bits=bits, order=args.order)
-    layer = Layer(probs, device, args.static_groups)
+    nl = stack_layers(args)
+    probs = [p for l in range(nl)
+             for p in problems_for(args.config, layer=layer_for_rank(rank) * nl + l, bits=bits,
+                                   order=args.order)]
+    layer = Job(probs, device, args.lanes, args.static_groups)
     params = sum(p.params for p in probs)
     main = torch.cuda.Stream(device=device)     # non-default: graphs capture here
     torch.cuda.set_stream(main)
@@ -390,7 +468,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(device)
     layer.check()
 
-    # ---- one step captured as a CUDA graph (both problems, forked streams)
+    # ---- one step captured as a CUDA graph (every problem, forked lanes)
     graph = None
     launches_per_step = 0
     if not args.no_graph:
@@ -441,24 +519,25 @@ def run_ours(args, rank, world, local):
     # launch bracketed by CUDA events on its own stream
     # (problems one after the other on one stream, so that no kernel's
     # interval includes time spent waiting for the other problem's kernels)
-    g.gptq_profile_start(1 << 16)
-    for _ in range(args.steps):
+    prof_steps = max(1, min(args.steps, args.profile_steps))
+    g.gptq_profile_start(1 << 17)
+    for _ in range(prof_steps):
         flush.fill_(1.0)
         layer.step_serial(main)
     torch.cuda.synchronize(device)
     kprof = g.gptq_profile_stop()
 
     # ---- end to end: pinned host inputs in, packed results out, every step.
-    # The copies are part of the captured step, on the problems' own streams:
-    # the activations of the problem on the critical path go first, each
-    # problem starts as soon as its own activations are in, and the weights
-    # arrive while the factorisations run.
+    # The copies are part of the captured step: each lane's copy stream brings
+    # in its problems' activations and weights ahead of the lane's compute, a
+    # problem starts once its activations are in and quantizes once its
+    # weights are, and its results go back on the lane's stream.
     hosts = [{"X": it["X"].cpu().pin_memory(), "W": it["W"].cpu().pin_memory(),
               **{k: torch.empty(it[k].shape, dtype=it[k].dtype).pin_memory()
-                 for k in Layer.OUTS}} for it in layer.items]
+                 for k in Job.OUTS}} for it in layer.items]
     h2d = sum(h["X"].numel() * h["X"].element_size() + h["W"].numel() * h["W"].element_size()
               for h in hosts)
-    d2h = sum(h[k].numel() * h[k].element_size() for h in hosts for k in Layer.OUTS)
+    d2h = sum(h[k].numel() * h[k].element_size() for h in hosts for k in Job.OUTS)
     e2e_graph = None
     if not args.no_graph:
         e2e_graph = torch.cuda.CUDAGraph()
@@ -488,64 +567,31 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e2e_ms, world, device)
     layer.check()
 
-    # ---- roofline of the dominant kernel
-    work = kernel_work(probs, probs[0].block)
-    tot = {k: v[0] for k, v in kprof.items()}
-    dom = max(tot, key=lambda k: tot[k])
+    # ---- per-kernel figures and the roofline of the dominant kernel
     peaks, src = _peaks()
-    sm_mhz = (clk or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
-    roof = None
-    if dom in work and kprof[dom][1] > 0:
-        unit, amount = work[dom]
-        per_step_ms = tot[dom] / args.steps
-        if unit == "TFLOP/s":
-            achieved = amount / (per_step_ms / 1e3) / 1e12
-            if dom == "hessian":
-                bound, peak, note = "tensor", peaks["bf16_tflops"], f"bf16 {src}"
-            else:
-                bound, peak = "alu", fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
-                note = "fp64 148 SMs x 64 FMA x 2 x max clock"
-        else:
-            achieved = amount / (per_step_ms / 1e3) / 1e9
-            bound, peak, note = "hbm", peaks["hbm_gbs"], f"copy bandwidth, {src}"
-        launches_per_step = kprof[dom][1] / args.steps
-        roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2),
-                "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
-                "peak_source": note,
-                "traffic": traffic_for(dom, workload_name(args.config, bits, args.order, args.static_groups)),
-                "launches_per_step": launches_per_step,
-                "share": round(tot[dom] / max(1e-9, sum(tot.values())), 4)}
+    try:
+        probed = probe_peaks(device)
+    except Exception as e:                     # the probes are a measurement aid
+        probed = {"error": str(e)[:200]}
+    work = kernel_work(probs, probs[0].block)
+    kernels, roof = kernel_figures(work, kprof, prof_steps, peaks, src, probed)
+    wl = workload_name(args.config, bits, args.order, args.static_groups, nl)
+    for k, v in kernels.items():
+        v["traffic"] = traffic_for(k, wl)
+    if roof is not None:
+        roof["traffic"] = kernels[roof["kernel"]]["traffic"]
 
-    # ---- the same figures for every kernel kind with a work model
-    kernels = {}
-    for k, (unit, amount) in work.items():
-        if k not in kprof or kprof[k][1] <= 0 or amount <= 0:
-            continue
-        per_step_ms = kprof[k][0] / args.steps
-        if unit == "TFLOP/s":
-            ach = amount / (per_step_ms / 1e3) / 1e12
-            if k == "hessian":
-                bound, peak = "tensor", peaks["bf16_tflops"]
-            else:
-                bound, peak = "alu", fp64_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
-        else:
-            ach = amount / (per_step_ms / 1e3) / 1e9
-            bound, peak = "hbm", peaks["hbm_gbs"]
-        kernels[k] = {"ms_per_step": round(per_step_ms, 4),
-                      "launches_per_step": kprof[k][1] / args.steps,
-                      "bound": bound, "achieved": round(ach, 2), "unit": unit,
-                      "peak": round(peak, 1), "frac": round(ach / peak, 4),
-                      "traffic": traffic_for(k, workload_name(args.config, bits, args.order, args.static_groups))}
-
+    tot = {k: v[0] for k, v in kprof.items()}
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "params/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dev_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16->f32 Hessian, f64 prepare, f32 sweep",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": workload_name(args.config, bits, args.order, args.static_groups), "params_per_step_per_gpu": params,
+        "config": {"workload": wl, "params_per_step_per_gpu": params,
                    "global_batch": len(probs) * world, "seq_len": probs[0].T,
                    "parallelism": f"independent layers x{world}",
+                   "lanes": len(layer.lanes),
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step" if graph is not None else "eager launches"},
         "e2e": {"value": round(total_params / (e2e_ms / 1e3), 1), "unit": "params/s",
@@ -553,7 +599,8 @@ def run_ours(args, rank, world, local):
         "gpu_launches": int(launches),
         "roofline": roof,
         "kernels": kernels,
-        "kernels_ms_per_step": {k: round(v / args.steps, 4) for k, v in tot.items() if v > 0},
+        "kernels_ms_per_step": {k: round(v / prof_steps, 4) for k, v in tot.items() if v > 0},
+        "peaks_probed_tflops": probed,
         "clocks": clk,
     }
     return out, probs, params
@@ -1336,17 +1383,21 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(probs, budget_s: float = 12.0, static_groups=False):
-    done, t0 = 0, time.perf_counter()
-    passes = 0
+    """The float64 oracle on the host cores over whole problems of the step
+    (each with its Hessian, factorisation and sweep), one after the other in
+    the step's order, until ``budget_s`` has passed (at least one problem)."""
+    done, t0, count = 0, time.perf_counter(), 0
     while True:
-        done += oracle_pass(probs, static_groups)
-        passes += 1
+        done += oracle_pass([probs[count % len(probs)]], static_groups)
+        count += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or passes >= 50:
+        if el >= budget_s or count >= 50:
             break
+    names = sorted({f"{probs[k % len(probs)].m}x{probs[k % len(probs)].n}" for k in range(count)})
     return {"value": round(done / el, 1), "unit": "params/s", "cores": blas_threads(),
             "kind": "oracle",
-            "sample": f"{passes} full passes of the layer's problems ({el:.1f} s, float64 numpy)"}
+            "sample": (f"{count} whole problems of the step ({', '.join(names)}; "
+                       f"{el:.1f} s, float64 numpy)")}
 
 
 def frontend_workload(frontend: str, cfg, bits: int, group: int, block: int) -> str:
@@ -1401,32 +1452,39 @@ def run_reference_frontend(args, world):
 
 
 def run_reference(args, rank, world):
+    """The oracle arm: each step one bounded sample of the same workload, the
+    float64 oracle over one whole problem of the step (Hessian, factorisation,
+    sweep), taking the step's problems in turn."""
     if rank != 0:
         return None
     if args.frontend != "gptq":
         return run_reference_frontend(args, world)
     cfg = CONFIGS[args.config]
     bits = args.bits or cfg["bits"][0]
+    nl = stack_layers(args)
     probs = problems_for(args.config, layer=0, bits=bits, order=args.order)
-    for _ in range(args.warmup):
-        oracle_pass(probs, args.static_groups)
+    for k in range(args.warmup):
+        oracle_pass([probs[k % len(probs)]], args.static_groups)
     t0 = time.perf_counter()
     params = 0
-    for _ in range(args.steps):
-        params += oracle_pass(probs, args.static_groups)
+    for k in range(args.steps):
+        params += oracle_pass([probs[k % len(probs)]], args.static_groups)
     el = time.perf_counter() - t0
     value = params / el
     cores = blas_threads()
+    shapes = ", ".join(f"{p.m}x{p.n}" for p in probs)
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "params/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
-        "config": {"workload": workload_name(args.config, bits, args.order, args.static_groups)},
+        "config": {"workload": workload_name(args.config, bits, args.order, args.static_groups,
+                                             nl)},
         "cpu_baseline": {"value": round(value, 1), "unit": "params/s", "cores": cores,
                          "kind": "oracle",
-                         "sample": f"{args.steps} timed passes of one layer on the host cores"},
+                         "sample": (f"per step one whole problem of a layer ({shapes}, in "
+                                    f"turn), {args.steps} timed steps on the host cores")},
         "e2e": {"value": round(value, 1), "unit": "params/s",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -1437,7 +1495,16 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=None,
+                    help="workload (0 single 576x576, 1 SmolLM-135M layer, 2 Qwen2.5-0.5B "
+                         "x24, 3 TinyLlama-1.1B x22, 4 stress 8192^2; default 3, and 1 "
+                         "for the frontends)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decoder layers per step (default: every layer of the stack)")
+    ap.add_argument("--lanes", type=int, default=4,
+                    help="streams the problems of a step are spread over")
+    ap.add_argument("--profile-steps", type=int, default=2,
+                    help="steps of the serialised per-kernel timing pass")
     ap.add_argument("--bits", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1454,6 +1521,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.config is None:
+        args.config = 3 if args.frontend == "gptq" else 1
     rank, world, local = dist_env()
 
     if args.impl == "reference":

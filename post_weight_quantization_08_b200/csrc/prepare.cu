@@ -715,9 +715,15 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
   if (warp == 0) lower_syrk_group(tt, l, 4, lane);
 }
 
-// 64×64 float64 tile products.  Warp w owns rows 16·(w/2) .. +16 and columns
-// 32·(w%2) .. +32 of C: 2 × 4 accumulator blocks of 8×8.
-
+// 64×64 float64 tile products C = X·B of the worker tasks.  Warp w owns rows
+// 16·(w/2) .. +16 and columns 32·(w%2) .. +32 of C: 2 × 4 accumulator blocks
+// of 8×8.  X is held row-major (row r of C, column q of the sum).  B comes in
+// one of two layouts, both copied from global memory as they are:
+//   NT: y holds Bᵀ (row n of C, column q): C = X·Yᵀ;
+//   NN: y holds B (row q, column n):       C = X·Y.
+// With the row pitch LDM ≡ 4 (mod 16) doubles, every fragment load of either
+// layout touches each bank pair exactly twice (two wavefronts, no conflict).
+template <bool NT>
 __device__ __forceinline__ void tile_mm(const double (*x)[LDM], const double (*y)[LDM],
                                         double acc[2][4][2], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
@@ -728,7 +734,7 @@ __device__ __forceinline__ void tile_mm(const double (*x)[LDM], const double (*y
 #pragma unroll
     for (int i = 0; i < 2; ++i) a[i] = x[rb + 8 * i + g][q + t];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = y[q + t][cb + 8 * j + g];
+    for (int j = 0; j < 4; ++j) b[j] = NT ? y[cb + 8 * j + g][q + t] : y[q + t][cb + 8 * j + g];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -736,10 +742,24 @@ __device__ __forceinline__ void tile_mm(const double (*x)[LDM], const double (*y
   }
 }
 
-// out ±= C (sign = +1 stores C, −1 subtracts it), leading dimension ld.
+// The part of a 64×64 output tile (leading dimension ld) that a thread's
+// accumulators cover, read ahead of the products (for C −= X·B).
+__device__ __forceinline__ void tile_load_c(const double* out, int64_t ld, double2 (&c)[2][4],
+                                            int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      c[i][j] = __ldcg(reinterpret_cast<const double2*>(out + (int64_t)(rb + 8 * i + g) * ld +
+                                                        cb + 8 * j + 2 * t));
+}
+
+// out = C, or out = c − C with c the values read by tile_load_c.
 template <bool SUBTRACT>
 __device__ __forceinline__ void tile_store(double* out, int64_t ld, const double acc[2][4][2],
-                                           int warp, int lane) {
+                                           const double2 (&c)[2][4], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
 #pragma unroll
@@ -747,42 +767,28 @@ __device__ __forceinline__ void tile_store(double* out, int64_t ld, const double
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       double2* p = reinterpret_cast<double2*>(out + (int64_t)(rb + 8 * i + g) * ld + cb + 8 * j + 2 * t);
-      double2 v;
-      if (SUBTRACT) {
-        v = __ldcg(p);
-        v.x -= acc[i][j][0];
-        v.y -= acc[i][j][1];
-      } else {
-        v = make_double2(acc[i][j][0], acc[i][j][1]);
-      }
-      *p = v;
+      *p = SUBTRACT ? make_double2(c[i][j].x - acc[i][j][0], c[i][j].y - acc[i][j][1])
+                    : make_double2(acc[i][j][0], acc[i][j][1]);
     }
 }
 
-// 64×64 float64 tile from global (leading dimension ld) into shared memory,
-// optionally transposed; 16-byte loads (L2 only: tiles are rewritten by other
-// CTAs of the same launch), all issued before the stores.
-__device__ __forceinline__ void load_tile(double (*dst)[LDM], const double* src,
-                                          int64_t ld, bool transpose, int tid) {
-  double2 buf[8];
+// One 64×64 float64 tile (leading dimension ld) into shared memory as it is,
+// by the CTA's 256 threads: 16-byte cp.async through L2 only (tiles are
+// rewritten by other CTAs of the same launch).  The caller commits the group.
+__device__ __forceinline__ void copy_tile_async(double (*dst)[LDM], const double* src, int64_t ld,
+                                                int tid) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const int e = tid + 256 * k;            // 2048 pairs
-    const int r = e >> 5, c2 = (e & 31) * 2;
-    buf[k] = __ldcg(reinterpret_cast<const double2*>(src + (int64_t)r * ld + c2));
+    const int e = tid + 256 * k;            // 2048 chunks of 16 bytes
+    const int r = e >> 5, c = (e & 31) * 2;
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&dst[r][c]));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + (int64_t)r * ld + c)
+                 : "memory");
   }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int e = tid + 256 * k;
-    const int r = e >> 5, c2 = (e & 31) * 2;
-    if (transpose) {
-      dst[c2][r] = buf[k].x;
-      dst[c2 + 1][r] = buf[k].y;
-    } else {
-      dst[r][c2] = buf[k].x;
-      dst[r][c2 + 1] = buf[k].y;
-    }
-  }
+}
+__device__ __forceinline__ void copy_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void copy_wait_but_one() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -939,12 +945,92 @@ __device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) 
   kind = T_MTRAIL; i = k + 2 + task / (k + 1); j = task % (k + 1);
 }
 
+// A worker task as operands, output and dependencies:
+//   PANEL  (k,i):   L_ik = A_ik·D_kᵀ     x = A_ik, y = D_k (NT)
+//   MROW   (k,c):   M_kc = D_k·M_kc      x = D_k,  y = M_kc (NN)
+//   TRAIL  (k,i,j): A_ij −= L_ik·L_jkᵀ   x = L_ik, y = L_jk (NT)
+//   MTRAIL (k,i,c): M_ic −= L_ik·M_kc    x = L_ik, y = M_kc (NN)
+// (D_k = L_kk⁻¹ is stored in tile (k,k) of M.)  The task may start once
+// every dep[d] flag is ≥ its target; it then sets *flag = value.
+struct WorkTask {
+  const double* x;
+  const double* y;
+  double* out;
+  bool nt, subtract;
+  int* flag;
+  int value;
+  int ndep;
+  const int* dep[3];
+  int target[3];
+};
+
+__device__ WorkTask work_task(int task, int N, int64_t np, double* A, double* M,
+                              const CholSync& S) {
+  int kind, k, i, j;
+  decode_task(task, N, kind, k, i, j);
+  auto tile = [np](double* base, int r, int c) { return base + (int64_t)r * NB * np + (int64_t)c * NB; };
+  WorkTask t = {};
+  if (kind == T_PANEL) {
+    t.x = tile(A, i, k); t.y = tile(M, k, k); t.out = tile(A, i, k);
+    t.nt = true; t.subtract = false;
+    t.flag = &S.pdone[k * N + i]; t.value = 1;
+    t.dep[0] = &S.diag_done[k]; t.target[0] = 1;
+    t.dep[1] = &S.upd[i * N + k]; t.target[1] = k;
+    t.ndep = 2;
+  } else if (kind == T_MROW) {
+    const int c = j;
+    t.x = tile(M, k, k); t.y = tile(M, k, c); t.out = tile(M, k, c);
+    t.nt = false; t.subtract = false;
+    t.flag = &S.mdone[k * N + c]; t.value = 1;
+    t.dep[0] = &S.diag_done[k]; t.target[0] = 1;
+    t.dep[1] = &S.mupd[k * N + c]; t.target[1] = k - c;
+    t.ndep = 2;
+  } else if (kind == T_TRAIL) {
+    t.x = tile(A, i, k); t.y = tile(A, j, k); t.out = tile(A, i, j);
+    t.nt = true; t.subtract = true;
+    t.flag = &S.upd[i * N + j]; t.value = k + 1;
+    t.dep[0] = &S.pdone[k * N + i]; t.target[0] = 1;
+    t.dep[1] = &S.pdone[k * N + j]; t.target[1] = 1;
+    t.dep[2] = &S.upd[i * N + j]; t.target[2] = k;
+    t.ndep = 3;
+  } else {   // T_MTRAIL
+    const int c = j;
+    t.x = tile(A, i, k); t.y = tile(M, k, c); t.out = tile(M, i, c);
+    t.nt = false; t.subtract = true;
+    t.flag = &S.mupd[i * N + c]; t.value = k - c + 1;
+    t.dep[0] = &S.pdone[k * N + i]; t.target[0] = 1;
+    t.dep[1] = (c < k) ? &S.mdone[k * N + c] : &S.diag_done[k]; t.target[1] = 1;
+    t.dep[2] = &S.mupd[i * N + c]; t.target[2] = k - c;
+    t.ndep = 3;
+  }
+  return t;
+}
+
+// One look at a task's dependencies (thread 0 of a CTA): all final?
+__device__ bool task_ready(const WorkTask& t) {
+  bool ok = true;
+#pragma unroll
+  for (int d = 0; d < 3; ++d)
+    if (d < t.ndep && ok) ok = ld_acquire(t.dep[d]) >= t.target[d];
+  return ok;
+}
+
+// Whole-CTA bounded wait for every dependency of a task; false on abort or
+// time-out.
+__device__ bool wait_task(const WorkTask& t, int* abortp, int32_t* info, int* s_ok,
+                          uint32_t spin) {
+#pragma unroll
+  for (int d = 0; d < 3; ++d)
+    if (d < t.ndep && !cta_wait(t.dep[d], t.target[d], abortp, info, s_ok, spin)) return false;
+  return true;
+}
+
 __global__ void __launch_bounds__(256, 1)
 chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int64_t n, int64_t np, int N,
                        int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
-  __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail;
+  __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail, s_next, s_ready;
   __shared__ volatile int s_stop;
   const CholSync S = sync_view(sync_base, N);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1069,66 +1155,69 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     return;
   }
 
-  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm);
-  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + NB * LDM);
+  // ---- the workers, two tasks in flight: while the products of the current
+  // task run, the next task (claimed in order, its dependencies polled once
+  // and found final) has its operand tiles copied into the other buffer set.
+  // A next task that is not ready yet is waited for, and copied, only after
+  // the current one is stored and signalled (it may depend on it).
+  // buffer set b: x at tile 2b, y at tile 2b + 1 of the dynamic shared memory
+  auto xb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + 2 * b * NB * LDM); };
+  auto yb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + (2 * b + 1) * NB * LDM); };
+  if (tid == 0) s_task = atomicAdd(&S.ctrl[0], 1);
+  __syncthreads();
+  int cur = s_task;
+  __syncthreads();
+  if (cur >= ntasks || *reinterpret_cast<volatile int*>(&S.ctrl[2])) return;
+  WorkTask tc = work_task(cur, N, np, A, M, S);
+  if (!wait_task(tc, &S.ctrl[2], info, &s_ok, spin)) return;
+  copy_tile_async(xb(0), tc.x, np, tid);
+  copy_tile_async(yb(0), tc.y, np, tid);
+  copy_commit();
+  int sb = 0;
   for (;;) {
-    if (tid == 0) s_task = atomicAdd(&S.ctrl[0], 1);
-    __syncthreads();
-    const int task = s_task;
-    __syncthreads();
-    if (task >= ntasks || *reinterpret_cast<volatile int*>(&S.ctrl[2])) return;
-    int kind, k, i, j;
-    decode_task(task, N, kind, k, i, j);
-    double acc[2][4][2] = {};
-    if (kind == T_PANEL) {
-      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok, spin)) return;
-      if (!cta_wait(&S.upd[i * N + k], k, &S.ctrl[2], info, &s_ok, spin)) return;
-      double* out = A + (int64_t)i * NB * np + (int64_t)k * NB;
-      load_tile(x, out, np, false, tid);
-      load_tile(y, M + (int64_t)k * NB * np + (int64_t)k * NB, np, true, tid);
-      __syncthreads();
-      tile_mm(x, y, acc, warp, lane);
-      tile_store<false>(out, np, acc, warp, lane);
-      cta_signal(&S.pdone[k * N + i], 1);
-    } else if (kind == T_MROW) {
-      const int c = j;
-      if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok, spin)) return;
-      if (!cta_wait(&S.mupd[k * N + c], k - c, &S.ctrl[2], info, &s_ok, spin)) return;
-      double* out = M + (int64_t)k * NB * np + (int64_t)c * NB;
-      load_tile(x, M + (int64_t)k * NB * np + (int64_t)k * NB, np, false, tid);
-      load_tile(y, out, np, false, tid);
-      __syncthreads();
-      tile_mm(x, y, acc, warp, lane);
-      tile_store<false>(out, np, acc, warp, lane);
-      cta_signal(&S.mdone[k * N + c], 1);
-    } else if (kind == T_TRAIL) {
-      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok, spin)) return;
-      if (j != i && !cta_wait(&S.pdone[k * N + j], 1, &S.ctrl[2], info, &s_ok, spin)) return;
-      if (!cta_wait(&S.upd[i * N + j], k, &S.ctrl[2], info, &s_ok, spin)) return;
-      double* out = A + (int64_t)i * NB * np + (int64_t)j * NB;
-      load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
-      load_tile(y, A + (int64_t)j * NB * np + (int64_t)k * NB, np, true, tid);
-      __syncthreads();
-      tile_mm(x, y, acc, warp, lane);
-      tile_store<true>(out, np, acc, warp, lane);
-      cta_signal(&S.upd[i * N + j], k + 1);
-    } else {   // T_MTRAIL
-      const int c = j;
-      if (!cta_wait(&S.pdone[k * N + i], 1, &S.ctrl[2], info, &s_ok, spin)) return;
-      if (c < k) {
-        if (!cta_wait(&S.mdone[k * N + c], 1, &S.ctrl[2], info, &s_ok, spin)) return;
-      } else if (!cta_wait(&S.diag_done[k], 1, &S.ctrl[2], info, &s_ok, spin)) {
-        return;
-      }
-      if (!cta_wait(&S.mupd[i * N + c], k - c, &S.ctrl[2], info, &s_ok, spin)) return;
-      double* out = M + (int64_t)i * NB * np + (int64_t)c * NB;
-      load_tile(x, A + (int64_t)i * NB * np + (int64_t)k * NB, np, false, tid);
-      load_tile(y, M + (int64_t)k * NB * np + (int64_t)c * NB, np, false, tid);
-      __syncthreads();
-      tile_mm(x, y, acc, warp, lane);
-      tile_store<true>(out, np, acc, warp, lane);
-      cta_signal(&S.mupd[i * N + c], k - c + 1);
+    if (tid == 0) {
+      int nx = atomicAdd(&S.ctrl[0], 1);
+      int ready = 0;
+      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) nx = ntasks;
+      if (nx < ntasks) ready = task_ready(work_task(nx, N, np, A, M, S)) ? 1 : 0;
+      s_next = nx;
+      s_ready = ready;
     }
+    __syncthreads();
+    const int nx = s_next;
+    const bool pre = s_ready != 0;
+    WorkTask tn = {};
+    if (nx < ntasks) tn = work_task(nx, N, np, A, M, S);
+    if (pre) {
+      copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
+      copy_tile_async(yb(sb ^ 1), tn.y, np, tid);
+      copy_commit();
+      copy_wait_but_one();
+    } else {
+      copy_wait_all();
+    }
+    __syncthreads();
+    double2 cv[2][4];
+    if (tc.subtract) tile_load_c(tc.out, np, cv, warp, lane);
+    double acc[2][4][2] = {};
+    if (tc.nt)
+      tile_mm<true>(xb(sb), yb(sb), acc, warp, lane);
+    else
+      tile_mm<false>(xb(sb), yb(sb), acc, warp, lane);
+    if (tc.subtract)
+      tile_store<true>(tc.out, np, acc, cv, warp, lane);
+    else
+      tile_store<false>(tc.out, np, acc, cv, warp, lane);
+    cta_signal(tc.flag, tc.value);
+    if (nx >= ntasks) return;
+    if (!pre) {
+      if (!wait_task(tn, &S.ctrl[2], info, &s_ok, spin)) return;
+      copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
+      copy_tile_async(yb(sb ^ 1), tn.y, np, tid);
+      copy_commit();
+    }
+    tc = tn;
+    sb ^= 1;
   }
 }
 

@@ -5,6 +5,7 @@
 // "Warum Geometrie Gewichte nicht komprimiert", Methodik, Schritt 2 (the
 // column loop) and Table 1 (GPTQ stores integer indices plus group scales);
 // Schritt 3 (GPTQ's groups run along the input channels).
+#include <algorithm>
 #include <cuda_bf16.h>
 
 #include <map>
@@ -175,7 +176,14 @@ ingest_kernel(const T* __restrict__ W, int64_t m, int64_t n,
   Wp[e] = v;
 }
 
-// One thread packs 32 consecutive original columns of one row into BITS words.
+// Packing.  A CTA takes `rpb` consecutive rows: their codes (processing
+// order, contiguous in the code array) come into shared memory with coalesced
+// 16-byte loads.  Then a warp takes 32 original columns of one row at a time,
+// lane l column c = 32·chunk + l: its processing position pinv[c] (a coalesced
+// load), its code from shared memory, its dequantized value (a coalesced
+// store).  The chunk's BITS words are formed with one warp OR-reduction each:
+// lane l's code sits at bit offset BITS·l of the chunk, in word BITS·l/32 and,
+// when it straddles a word boundary, the low bits of the next one.
 template <int BITS>
 __global__ void __launch_bounds__(256)
 pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
@@ -183,24 +191,36 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
             const float* __restrict__ scale, const uint8_t* __restrict__ zero,
             uint32_t* __restrict__ qweight, int64_t nwords,
             float* __restrict__ Qdq, const float* __restrict__ outv, int static_groups,
-            int32_t* info) {
+            int rpb, int staged, int32_t* info) {
+  extern __shared__ __align__(16) uint8_t sc[];
+  const int64_t r0 = (int64_t)blockIdx.x * rpb;
+  const int rows = (int)(m - r0 < rpb ? m - r0 : (int64_t)rpb);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint8_t* src = codes + r0 * n;
+  const int64_t bytes = (int64_t)rows * n;
+  if (!staged) {
+    // a row too long for shared memory: codes gathered from global memory
+  } else if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+    const int64_t v16 = bytes >> 4;
+    for (int64_t e = tid; e < v16; e += 256)
+      reinterpret_cast<uint4*>(sc)[e] = __ldg(reinterpret_cast<const uint4*>(src) + e);
+    for (int64_t e = (v16 << 4) + tid; e < bytes; e += 256) sc[e] = src[e];
+  } else {
+    for (int64_t e = tid; e < bytes; e += 256) sc[e] = src[e];
+  }
+  __syncthreads();
   const int64_t chunks = (n + 31) / 32;
-  const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (e >= m * chunks) return;
-  const int64_t r = e / chunks, ch = e % chunks;
-  uint32_t w[BITS];
-#pragma unroll
-  for (int i = 0; i < BITS; ++i) w[i] = 0u;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const int64_t c = ch * 32 + k;
+  for (int64_t task = warp; task < rows * chunks; task += 8) {
+    const int rl = (int)(task / chunks);
+    const int64_t ch = task % chunks, r = r0 + rl;
+    const int64_t c = ch * 32 + lane;
+    uint32_t q = 0;
     if (c < n) {
       const int32_t p = pinv[c];
-      uint32_t q = 0;
       if (p < 0 || p >= n) {
         report(info, GPTQ_ERR_INVALID_ARG, c);
       } else {
-        q = codes[r * n + p];
+        q = staged ? sc[(int64_t)rl * n + p] : src[(int64_t)rl * n + p];
         bool kept = false;                 // an SSQR outlier: its value, not its code
         if (outv != nullptr) {
           kept = (q & OUTLIER_FLAG) != 0;
@@ -214,17 +234,28 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
           Qdq[r * n + c] = kept ? outv[r * n + p] : scale[sx] * ((float)q - (float)zero[sx]);
         }
       }
-      const int off = k * BITS, wi = off >> 5, sh = off & 31;
-      w[wi] |= q << sh;
-      if (sh + BITS > 32) w[wi + 1] |= q >> (32 - sh);
     }
-  }
+    const int off = BITS * lane, w0 = off >> 5, sh = off & 31;
+    const uint32_t lo = q << sh;
+    const uint32_t hi = (sh + BITS > 32) ? (q >> (32 - sh)) : 0u;
+    uint32_t mine = 0;
 #pragma unroll
-  for (int i = 0; i < BITS; ++i) {
-    const int64_t word = ch * BITS + i;
-    if (word < nwords) qweight[r * nwords + word] = w[i];
+    for (int j = 0; j < BITS; ++j) {
+      const uint32_t part = (w0 == j ? lo : 0u) | (w0 == j - 1 ? hi : 0u);
+      const uint32_t word = __reduce_or_sync(0xffffffffu, part);
+      if (lane == j) mine = word;
+    }
+    const int64_t wi = ch * BITS + lane;
+    if (lane < BITS && wi < nwords) qweight[r * nwords + wi] = mine;
   }
 }
+
+// Rows per packing CTA: up to 16 KB of codes in shared memory (one row, read
+// from global memory, when a row is longer than 48 KB).
+inline int pack_rows_per_block(int64_t n) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(16, 16384 / n));
+}
+constexpr int64_t kPackStageMax = 48 * 1024;
 
 }  // namespace
 
@@ -359,23 +390,26 @@ gptq_status quant_pack(const QuantWs& w, int64_t m, int64_t n, int bits, int gro
   const int sg = static_groups ? 1 : 0;
   const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
   const int64_t nwords = ceil_div(n * bits, 32);
-  const unsigned gpk = (unsigned)ceil_div(m * ceil_div(n, 32), 256);
+  const int rpb = pack_rows_per_block(n);
+  const unsigned gpk = (unsigned)ceil_div(m, rpb);
+  const int staged = (int64_t)rpb * n <= kPackStageMax ? 1 : 0;
+  const size_t psm = staged ? align_up((size_t)rpb * (size_t)n, 16) : 0;
   switch (bits) {
     case 2:
-      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
       break;
     case 3:
-      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
       break;
     case 4:
-      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
       break;
     default:
-      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, 0, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, info);
+      GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
       break;
   }
   return GPTQ_OK;
