@@ -22,6 +22,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "chol_tasks.cuh"
 #include "minpivot.cuh"
 
 namespace gptq {
@@ -894,57 +895,6 @@ __device__ __forceinline__ void cta_signal(int* flag, int value) {
   }
 }
 
-constexpr int kMLag = 2;
-
-// Factor and inverse tasks of step k (r = N − k − 1 blocks below it).
-__host__ __device__ inline int factor_tasks(int N, int k) {
-  const int r = N - k - 1;
-  return r <= 0 ? 0 : 2 * (r - 1) + (r - 1) * r / 2;
-}
-__host__ __device__ inline int inverse_tasks(int N, int k) {
-  const int r = N - k - 1;
-  return r <= 0 ? k : k + (k + 1) + (r - 1) * (k + 1);
-}
-__host__ __device__ inline int slot_tasks(int N, int s) {
-  return (s < N ? factor_tasks(N, s) : 0) +
-         (s >= kMLag && s - kMLag < N ? inverse_tasks(N, s - kMLag) : 0);
-}
-
-int total_tasks(int N) {
-  int t = 0;
-  for (int s = 0; s < N + kMLag; ++s) t += slot_tasks(N, s);
-  return t;
-}
-
-enum TaskKind { T_PANEL = 0, T_MROW, T_TRAIL, T_MTRAIL };
-
-__device__ void decode_task(int task, int N, int& kind, int& k, int& i, int& j) {
-  int s = 0;
-  while (task >= slot_tasks(N, s)) { task -= slot_tasks(N, s); ++s; }
-  if (s < N) {
-    const int nf = factor_tasks(N, s);
-    if (task < nf) {
-      k = s;
-      const int r = N - k - 1;
-      if (task < r - 1) { kind = T_PANEL; i = k + 2 + task; j = k; return; }
-      task -= r - 1;
-      if (task < r - 1) { kind = T_TRAIL; i = k + 2 + task; j = k + 1; return; }
-      task -= r - 1;
-      int ii = 0;
-      while (task >= ii + 1) { task -= ii + 1; ++ii; }
-      kind = T_TRAIL; i = k + 2 + ii; j = k + 2 + task; return;
-    }
-    task -= nf;
-  }
-  k = s - kMLag;
-  const int r = N - k - 1;
-  if (r <= 0 || task < k) { kind = T_MROW; i = k; j = task; return; }
-  task -= k;
-  if (task < k + 1) { kind = T_MTRAIL; i = k + 1; j = task; return; }
-  task -= k + 1;
-  kind = T_MTRAIL; i = k + 2 + task / (k + 1); j = task % (k + 1);
-}
-
 // A worker task as operands, output and dependencies:
 //   PANEL  (k,i):   L_ik = A_ik·D_kᵀ     x = A_ik, y = D_k (NT)
 //   MROW   (k,c):   M_kc = D_k·M_kc      x = D_k,  y = M_kc (NN)
@@ -964,10 +914,10 @@ struct WorkTask {
   int target[3];
 };
 
-__device__ WorkTask work_task(int task, int N, int64_t np, double* A, double* M,
-                              const CholSync& S) {
+__device__ WorkTask work_task(int task, int N, const int* prefix, int64_t np, double* A,
+                              double* M, const CholSync& S) {
   int kind, k, i, j;
-  decode_task(task, N, kind, k, i, j);
+  decode_task(task, N, prefix, kind, k, i, j);
   auto tile = [np](double* base, int r, int c) { return base + (int64_t)r * NB * np + (int64_t)c * NB; };
   WorkTask t = {};
   if (kind == T_PANEL) {
@@ -1031,10 +981,16 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
   __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail, s_next, s_ready;
+  __shared__ WorkTask s_wt;
+  // the task numbering's slot prefix, after the tiles
+  int* prefix = reinterpret_cast<int*>(sm + 5 * NB * LDM + 192);
   __shared__ volatile int s_stop;
   const CholSync S = sync_view(sync_base, N);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) s_role = atomicAdd(&S.ctrl[1], 1);
+  if (tid == 0) {
+    s_role = atomicAdd(&S.ctrl[1], 1);
+    build_slot_prefix(N, prefix);
+  }
   __syncthreads();
   if (*reinterpret_cast<volatile int32_t*>(info) != 0) return;
 
@@ -1163,23 +1119,30 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   // buffer set b: x at tile 2b, y at tile 2b + 1 of the dynamic shared memory
   auto xb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + 2 * b * NB * LDM); };
   auto yb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + (2 * b + 1) * NB * LDM); };
-  if (tid == 0) s_task = atomicAdd(&S.ctrl[0], 1);
+  if (tid == 0) {
+    s_task = atomicAdd(&S.ctrl[0], 1);
+    if (s_task < ntasks) s_wt = work_task(s_task, N, prefix, np, A, M, S);
+  }
   __syncthreads();
-  int cur = s_task;
-  __syncthreads();
+  const int cur = s_task;
   if (cur >= ntasks || *reinterpret_cast<volatile int*>(&S.ctrl[2])) return;
-  WorkTask tc = work_task(cur, N, np, A, M, S);
+  WorkTask tc = s_wt;
   if (!wait_task(tc, &S.ctrl[2], info, &s_ok, spin)) return;
   copy_tile_async(xb(0), tc.x, np, tid);
   copy_tile_async(yb(0), tc.y, np, tid);
   copy_commit();
   int sb = 0;
   for (;;) {
+    // thread 0 claims the next task, decodes it for the CTA and looks once
+    // at its dependencies
     if (tid == 0) {
       int nx = atomicAdd(&S.ctrl[0], 1);
       int ready = 0;
       if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) nx = ntasks;
-      if (nx < ntasks) ready = task_ready(work_task(nx, N, np, A, M, S)) ? 1 : 0;
+      if (nx < ntasks) {
+        s_wt = work_task(nx, N, prefix, np, A, M, S);
+        ready = task_ready(s_wt) ? 1 : 0;
+      }
       s_next = nx;
       s_ready = ready;
     }
@@ -1187,7 +1150,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     const int nx = s_next;
     const bool pre = s_ready != 0;
     WorkTask tn = {};
-    if (nx < ntasks) tn = work_task(nx, N, np, A, M, S);
+    if (nx < ntasks) tn = s_wt;
     if (pre) {
       copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
       copy_tile_async(yb(sb ^ 1), tn.y, np, tid);
@@ -1272,7 +1235,13 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  const size_t tile_smem = (5 * NB * LDM + 192) * sizeof(double);
+  // five tiles and the chain's 8×8 pivot blocks, then the task numbering's
+  // slot prefix (N + kMLag + 1 ints)
+  const size_t tile_smem = (5 * NB * LDM + 192) * sizeof(double) +
+                           sizeof(int) * (size_t)(task_slots(N) + 1);
+  if (total_tasks(N) >= ((int64_t)1 << 31) || tile_smem > 227 * 1024)
+    return fail(GPTQ_ERR_UNSUPPORTED, "gptq_prepare: n=%lld is too large for the factorisation",
+                (long long)n);
   int num_sms = 0;
   {
     gptq_status st = ensure_smem_limit((const void*)chol_persistent_kernel, (int)tile_smem,
@@ -1300,7 +1269,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   GPTQ_LAUNCH(KK_PREP_GATHER, s, prep_gather_kernel, (unsigned)ceil_div(np * np, 256),
               256, 0, H, n, np, perm, w.seen, order == GPTQ_ORDER_CUSTOM ? 1 : 0,
               w.mean, damp, w.A, w.M, info);
-  const int ntasks = total_tasks(N);
+  const int ntasks = (int)total_tasks(N);
   // Workers: enough that the two tiles the chain needs next are never queued
   // behind other ready tasks (a step offers ≈ N²/2 tile tasks, each ≈ a third
   // of the chain's step; N²/6 workers left the chain waiting ≈ 6.8 K cycles a
