@@ -956,12 +956,22 @@ __device__ WorkTask work_task(int task, int N, const int* prefix, int64_t np, do
   return t;
 }
 
-// One look at a task's dependencies (thread 0 of a CTA): all final?
+// One look at a task's dependencies (thread 0 of a CTA): all final?  The
+// flags are read at once (relaxed), and a fence after the last read gives the
+// acquire that the CTA's later loads of the tiles need.
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ bool task_ready(const WorkTask& t) {
+  int v[3];
+#pragma unroll
+  for (int d = 0; d < 3; ++d) v[d] = d < t.ndep ? ld_relaxed(t.dep[d]) : 0;
   bool ok = true;
 #pragma unroll
-  for (int d = 0; d < 3; ++d)
-    if (d < t.ndep && ok) ok = ld_acquire(t.dep[d]) >= t.target[d];
+  for (int d = 0; d < 3; ++d) ok = ok && (d >= t.ndep || v[d] >= t.target[d]);
+  if (ok) asm volatile("fence.acq_rel.gpu;" ::: "memory");
   return ok;
 }
 
@@ -981,7 +991,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
   __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail, s_next, s_ready;
-  __shared__ WorkTask s_wt;
+  __shared__ WorkTask s_wt, s_wt2;
   // the task numbering's slot prefix, after the tiles
   int* prefix = reinterpret_cast<int*>(sm + 5 * NB * LDM + 192);
   __shared__ volatile int s_stop;
@@ -1111,46 +1121,46 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     return;
   }
 
-  // ---- the workers, two tasks in flight: while the products of the current
-  // task run, the next task (claimed in order, its dependencies polled once
-  // and found final) has its operand tiles copied into the other buffer set.
-  // A next task that is not ready yet is waited for, and copied, only after
+  // ---- the workers.  Three tasks per CTA are claimed at a time (in numbering
+  // order): the current one (its tiles in buffer set sb), the next one and
+  // the one after.  Thread 0 claims the one after at the start of an
+  // iteration and decodes it after the current task's products, so that the
+  // atomic's round trip runs under them; it looks at the next task's
+  // dependencies (all flags at once) before the products, and a next task
+  // found final has its tiles copied into the other buffer set under them.
+  // A next task that is not final yet is waited for, and copied, only after
   // the current one is stored and signalled (it may depend on it).
   // buffer set b: x at tile 2b, y at tile 2b + 1 of the dynamic shared memory
   auto xb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + 2 * b * NB * LDM); };
   auto yb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + (2 * b + 1) * NB * LDM); };
   if (tid == 0) {
-    s_task = atomicAdd(&S.ctrl[0], 1);
-    if (s_task < ntasks) s_wt = work_task(s_task, N, prefix, np, A, M, S);
+    int c0 = atomicAdd(&S.ctrl[0], 1);
+    int c1 = atomicAdd(&S.ctrl[0], 1);
+    if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c0 = c1 = ntasks;
+    s_task = c0;
+    s_next = c1;
+    if (c0 < ntasks) s_wt = work_task(c0, N, prefix, np, A, M, S);
+    if (c1 < ntasks) s_wt2 = work_task(c1, N, prefix, np, A, M, S);
   }
   __syncthreads();
-  const int cur = s_task;
-  if (cur >= ntasks || *reinterpret_cast<volatile int*>(&S.ctrl[2])) return;
+  if (s_task >= ntasks) return;
   WorkTask tc = s_wt;
+  int nx = s_next;
+  WorkTask tn = {};
+  if (nx < ntasks) tn = s_wt2;
   if (!wait_task(tc, &S.ctrl[2], info, &s_ok, spin)) return;
   copy_tile_async(xb(0), tc.x, np, tid);
   copy_tile_async(yb(0), tc.y, np, tid);
   copy_commit();
   int sb = 0;
   for (;;) {
-    // thread 0 claims the next task, decodes it for the CTA and looks once
-    // at its dependencies
+    int claim = 0;
     if (tid == 0) {
-      int nx = atomicAdd(&S.ctrl[0], 1);
-      int ready = 0;
-      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) nx = ntasks;
-      if (nx < ntasks) {
-        s_wt = work_task(nx, N, prefix, np, A, M, S);
-        ready = task_ready(s_wt) ? 1 : 0;
-      }
-      s_next = nx;
-      s_ready = ready;
+      claim = atomicAdd(&S.ctrl[0], 1);     // the task after the next; used below
+      s_ready = (nx < ntasks && task_ready(tn)) ? 1 : 0;
     }
     __syncthreads();
-    const int nx = s_next;
     const bool pre = s_ready != 0;
-    WorkTask tn = {};
-    if (nx < ntasks) tn = s_wt;
     if (pre) {
       copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
       copy_tile_async(yb(sb ^ 1), tn.y, np, tid);
@@ -1167,12 +1177,17 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       tile_mm<true>(xb(sb), yb(sb), acc, warp, lane);
     else
       tile_mm<false>(xb(sb), yb(sb), acc, warp, lane);
+    if (tid == 0) {
+      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) claim = ntasks;
+      s_next = claim;
+      if (claim < ntasks) s_wt = work_task(claim, N, prefix, np, A, M, S);
+    }
     if (tc.subtract)
       tile_store<true>(tc.out, np, acc, cv, warp, lane);
     else
       tile_store<false>(tc.out, np, acc, cv, warp, lane);
-    cta_signal(tc.flag, tc.value);
-    if (nx >= ntasks) return;
+    cta_signal(tc.flag, tc.value);          // begins with a barrier: s_next, s_wt visible
+    if (nx >= ntasks) return;               // (then every later claim is past the end too)
     if (!pre) {
       if (!wait_task(tn, &S.ctrl[2], info, &s_ok, spin)) return;
       copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
@@ -1180,6 +1195,8 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       copy_commit();
     }
     tc = tn;
+    nx = s_next;
+    if (nx < ntasks) tn = s_wt;
     sb ^= 1;
   }
 }
