@@ -1,16 +1,22 @@
 """Throughput of the GPTQ hot path: weights quantized per second.
 
-One step = one pass of the whole path over one decoder layer's problems:
-  for every Hessian of the layer: zero H, gptq_hessian_accumulate (K1),
-  gptq_prepare (K2), gptq_quantize (ingest, K3/K4 per block, K5).
-Default workload: one SmolLM-135M-shaped decoder layer (q/k/v/o/gate/up
-4608×576 on one H, down 576×1536 on another), 2048 cone-structured
-calibration tokens, 4-bit, group 128, block 128, damp 0.01.
+One step = one pass of the whole path over every problem of the workload:
+  for every Hessian: zero H, gptq_hessian_accumulate (K1), gptq_prepare (K2),
+  gptq_quantize (ingest, K3/K4 per block, K5).
+A problem is one Hessian with every row that shares it: in a decoder layer the
+q/k/v/o/gate/up projections read the layer input (one stack on one H) and
+down_proj reads SiLU(gate)·up (its own H).  The decoder workloads quantize
+every layer of the stack per step.  Default workload: the TinyLlama-1.1B-shaped
+stack, 22 layers × (15872×2048 on one H + 2048×5632), 2048 cone-structured
+calibration tokens, 4-bit, group 128, block 128, damp 0.01.  The problems run
+on --lanes streams (each lane its share one after the other); the step is
+captured once as a CUDA graph and replayed.
 
-    python bench.py --gpus N --steps K --warmup W [--config C] [--impl reference]
+    python bench.py --gpus N --steps K --warmup W [--config C] [--bits B]
+                    [--layers L] [--lanes S] [--impl reference]
 
 Multi-GPU: one process per GPU (torchrun); every rank quantizes its own,
-independent layer (no collective on the data path: weak scaling); timing is
+independent stack (no collective on the data path: weak scaling); timing is
 the max over ranks of the device time.
 """
 from __future__ import annotations
@@ -165,7 +171,8 @@ def fp64_peak_tflops(sm_mhz: float) -> float:
     return 148 * 64 * 2 * sm_mhz * 1e6 / 1e12
 
 
-PROBE_ITERS = {"fp64": (0, 32768), "tf32": (1, 65536), "bf16": (2, 65536)}
+PROBE_ITERS = {"fp64": (0, 32768), "tf32": (1, 65536), "bf16": (2, 65536),
+               "fp64_8warps_per_sm": (3, 32768)}
 
 
 def probe_peaks(device) -> dict:
@@ -298,21 +305,31 @@ def kernel_figures(work, kprof, steps, peaks, src, probed):
     return kernels, roof
 
 
+def source_sha(files) -> str:
+    """First 16 hex digits of the SHA-256 of the named csrc files, in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "post_weight_quantization_08_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_for(kernel: str, workload: str):
-    """dram bytes per launch from the committed ncu summary, if still current."""
+    """DRAM bytes per launch of a kernel kind on a workload, from the committed
+    ncu summary (profiles/traffic.json), if its sources are unchanged since
+    the capture; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
             d = json.load(f)
-        e = d.get(kernel)
-        if not e or e.get("workload") != workload:
-            return None
-        import hashlib
-        src = os.path.join(ROOT, "post_weight_quantization_08_b200", "csrc", e["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return e["bytes_per_launch"] if h == e.get("source_sha") else None
+        for e in d.get("entries", []):
+            if e.get("kernel") == kernel and e.get("workload") == workload:
+                if source_sha(e["sources"]) == e.get("source_sha"):
+                    return e["bytes_per_launch"]
+        return None
     except Exception:
         return None
 

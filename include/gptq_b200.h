@@ -139,13 +139,14 @@ gptq_status gptq_prepare(const float* H, int64_t n, double damp, int order,
  *           per SM, each warp 8 independent accumulators, `iters` rounds;
  *   kind 1  tcgen05.mma kind::tf32 128×256×8 from shared memory into tensor
  *           memory, one CTA per SM, 4·iters products each;
- *   kind 2  the same with kind::f16 on bf16 operands (K = 16).
+ *   kind 2  the same with kind::f16 on bf16 operands (K = 16);
+ *   kind 3  kind 0 with one CTA of 8 warps per SM.
  *   flops  host, output: the floating-point operations of the launch
  *          (2 per multiply-add).
  *   info   int32[2] on the device: a bounded wait that runs out sets TIMEOUT.
  *   sink   ≥ 8 bytes of device memory (never written in practice; it keeps
  *          the products from being optimised away).
- * Errors: INVALID_ARG (kind outside 0..2, iters < 1, a null pointer), CUDA.
+ * Errors: INVALID_ARG (kind outside 0..3, iters < 1, a null pointer), CUDA.
  */
 gptq_status gptq_peak_probe(int kind, int64_t iters, double* flops, int32_t* info, void* sink,
                             void* stream);

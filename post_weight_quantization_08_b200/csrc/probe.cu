@@ -8,6 +8,8 @@
 //           shared memory (zeros), accumulator in tensor memory, one issuing
 //           thread per CTA, one CTA per SM
 //   kind 2  the same with kind::f16 (bf16 operands, K = 16)
+//   kind 3  kind 0 with one CTA of 8 warps per SM (two warps per scheduler,
+//           the occupancy of the float64 factorisation's CTAs)
 //
 // The operands' values do not matter for the rate; nothing is read from or
 // written to global memory except one sink word that is never written in
@@ -102,7 +104,7 @@ using namespace gptq;
 
 extern "C" gptq_status gptq_peak_probe(int kind, int64_t iters, double* flops, int32_t* info,
                                        void* sink, void* stream) {
-  if (kind < 0 || kind > 2 || iters < 1 || !flops || !info || !sink)
+  if (kind < 0 || kind > 3 || iters < 1 || !flops || !info || !sink)
     return fail(GPTQ_ERR_INVALID_ARG, "gptq_peak_probe: kind=%d iters=%lld", kind,
                 (long long)iters);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -112,8 +114,8 @@ extern "C" gptq_status gptq_peak_probe(int kind, int64_t iters, double* flops, i
     if (st != GPTQ_OK) return st;
   }
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
-  if (kind == 0) {
-    const int grid = 4 * sms;
+  if (kind == 0 || kind == 3) {
+    const int grid = (kind == 0 ? 4 : 1) * sms;
     GPTQ_LAUNCH(KK_PROBE, s, probe_dmma_kernel, grid, 256, 0, iters,
                 static_cast<double*>(sink), -1.2345e300);
     *flops = (double)grid * 8 * 8 * (double)iters * 2.0 * 8 * 8 * 4;

@@ -181,9 +181,9 @@ ingest_kernel(const T* __restrict__ W, int64_t m, int64_t n,
 // 16-byte loads.  Then a warp takes 32 original columns of one row at a time,
 // lane l column c = 32·chunk + l: its processing position pinv[c] (a coalesced
 // load), its code from shared memory, its dequantized value (a coalesced
-// store).  The chunk's BITS words are formed with one warp OR-reduction each:
-// lane l's code sits at bit offset BITS·l of the chunk, in word BITS·l/32 and,
-// when it straddles a word boundary, the low bits of the next one.
+// store).  The chunk's BITS words are formed in registers: for widths that
+// divide 32 an OR over each word's group of lanes (shuffles), for 3 bits a
+// transpose through ballots (bit planes of the codes, then the words).
 template <int BITS>
 __global__ void __launch_bounds__(256)
 pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
@@ -209,11 +209,11 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
     for (int64_t e = tid; e < bytes; e += 256) sc[e] = src[e];
   }
   __syncthreads();
-  const int64_t chunks = (n + 31) / 32;
-  for (int64_t task = warp; task < rows * chunks; task += 8) {
-    const int rl = (int)(task / chunks);
-    const int64_t ch = task % chunks, r = r0 + rl;
-    const int64_t c = ch * 32 + lane;
+  const int chunks = (int)((n + 31) / 32);
+  for (int rl = 0; rl < rows; ++rl)
+  for (int ch = warp; ch < chunks; ch += 8) {
+    const int64_t r = r0 + rl;
+    const int64_t c = (int64_t)ch * 32 + lane;
     uint32_t q = 0;
     if (c < n) {
       const int32_t p = pinv[c];
@@ -229,23 +229,39 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
         if (Qdq != nullptr) {
           // input-channel groups: [row][group of processing position p];
           // output-channel groups (rowgs rows): [row group][original column c]
-          const int64_t sx = rowgs > 0 ? (r / rowgs) * n + c
-                                       : r * ngroups + (static_groups ? c : p) / group;
+          // (32-bit quotients: rows < 2^31, columns < 2^20)
+          const int64_t sx = rowgs > 0 ? (int64_t)((int)r / rowgs) * n + c
+                                       : r * ngroups + (static_groups ? (int)c : p) / group;
           Qdq[r * n + c] = kept ? outv[r * n + p] : scale[sx] * ((float)q - (float)zero[sx]);
         }
       }
     }
-    const int off = BITS * lane, w0 = off >> 5, sh = off & 31;
-    const uint32_t lo = q << sh;
-    const uint32_t hi = (sh + BITS > 32) ? (q >> (32 - sh)) : 0u;
-    uint32_t mine = 0;
+    uint32_t mine = 0;                     // lane j < BITS: word j of the chunk
+    if constexpr (32 % BITS == 0) {
+      // G = 32/BITS codes per word: OR within groups of G lanes, then lane j
+      // takes word j from the first lane of group j
+      constexpr int G = 32 / BITS;
+      uint32_t v = q << (BITS * (lane % G));
 #pragma unroll
-    for (int j = 0; j < BITS; ++j) {
-      const uint32_t part = (w0 == j ? lo : 0u) | (w0 == j - 1 ? hi : 0u);
-      const uint32_t word = __reduce_or_sync(0xffffffffu, part);
-      if (lane == j) mine = word;
+      for (int o = 1; o < G; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+      mine = __shfl_sync(0xffffffffu, v, (lane % BITS) * G);
+    } else {
+      // codes straddle words: one ballot per code bit (plane b: bit b of every
+      // lane's code), then one ballot per word, lane t supplying bit t
+      uint32_t plane[BITS];
+#pragma unroll
+      for (int b = 0; b < BITS; ++b) plane[b] = __ballot_sync(0xffffffffu, (q >> b) & 1u);
+#pragma unroll
+      for (int j = 0; j < BITS; ++j) {
+        const int idx = 32 * j + lane, code = idx / BITS, b = idx % BITS;
+        uint32_t pb = plane[0];
+#pragma unroll
+        for (int bb = 1; bb < BITS; ++bb) pb = (b == bb) ? plane[bb] : pb;
+        const uint32_t word = __ballot_sync(0xffffffffu, (pb >> code) & 1u);
+        if (lane == j) mine = word;
+      }
     }
-    const int64_t wi = ch * BITS + lane;
+    const int64_t wi = (int64_t)ch * BITS + lane;
     if (lane < BITS && wi < nwords) qweight[r * nwords + wi] = mine;
   }
 }
