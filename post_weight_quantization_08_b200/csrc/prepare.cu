@@ -716,55 +716,56 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
   if (warp == 0) lower_syrk_group(tt, l, 4, lane);
 }
 
-// 64×64 float64 tile products C = X·B of the worker tasks.  Warp w owns rows
-// 16·(w/2) .. +16 and columns 32·(w%2) .. +32 of C: 2 × 4 accumulator blocks
-// of 8×8.  X is held row-major (row r of C, column q of the sum).  B comes in
-// one of two layouts, both copied from global memory as they are:
+// 64×64 float64 tile products C = X·B of a worker half (4 warps).  Warp w
+// owns rows 32·(w/2) .. +32 and columns 32·(w%2) .. +32 of C: 4 × 4
+// accumulator blocks of 8×8.  X is held row-major (row r of C, column q of
+// the sum).  B comes in one of two layouts, both copied from global memory
+// as they are:
 //   NT: y holds Bᵀ (row n of C, column q): C = X·Yᵀ;
 //   NN: y holds B (row q, column n):       C = X·Y.
 // With the row pitch LDM ≡ 4 (mod 16) doubles, every fragment load of either
 // layout touches each bank pair exactly twice (two wavefronts, no conflict).
 template <bool NT>
-__device__ __forceinline__ void tile_mm(const double (*x)[LDM], const double (*y)[LDM],
-                                        double acc[2][4][2], int warp, int lane) {
+__device__ __forceinline__ void half_mm(const double (*x)[LDM], const double (*y)[LDM],
+                                        double acc[4][4][2], int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
-#pragma unroll 4
+  const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
+#pragma unroll 2
   for (int q = 0; q < NB; q += 4) {
-    double a[2], b[4];
+    double a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
 #pragma unroll
     for (int j = 0; j < 4; ++j) b[j] = NT ? y[cb + 8 * j + g][q + t] : y[q + t][cb + 8 * j + g];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) dmma_884(acc[i][j], a[i], b[j]);
   }
 }
 
-// The part of a 64×64 output tile (leading dimension ld) that a thread's
+// The part of a 64×64 output tile (leading dimension ld) that a lane's
 // accumulators cover, read ahead of the products (for C −= X·B).
-__device__ __forceinline__ void tile_load_c(const double* out, int64_t ld, double2 (&c)[2][4],
-                                            int warp, int lane) {
+__device__ __forceinline__ void half_load_c(const double* out, int64_t ld, double2 (&c)[4][4],
+                                            int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+  const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       c[i][j] = __ldcg(reinterpret_cast<const double2*>(out + (int64_t)(rb + 8 * i + g) * ld +
                                                         cb + 8 * j + 2 * t));
 }
 
-// out = C, or out = c − C with c the values read by tile_load_c.
+// out = C, or out = c − C with c the values read by half_load_c.
 template <bool SUBTRACT>
-__device__ __forceinline__ void tile_store(double* out, int64_t ld, const double acc[2][4][2],
-                                           const double2 (&c)[2][4], int warp, int lane) {
+__device__ __forceinline__ void half_store(double* out, int64_t ld, const double acc[4][4][2],
+                                           const double2 (&c)[4][4], int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int rb = 16 * (warp >> 1), cb = 32 * (warp & 1);
+  const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       double2* p = reinterpret_cast<double2*>(out + (int64_t)(rb + 8 * i + g) * ld + cb + 8 * j + 2 * t);
@@ -774,22 +775,18 @@ __device__ __forceinline__ void tile_store(double* out, int64_t ld, const double
 }
 
 // One 64×64 float64 tile (leading dimension ld) into shared memory as it is,
-// by the CTA's 256 threads: 16-byte cp.async through L2 only (tiles are
+// by a half's 128 threads: 16-byte cp.async through L2 only (tiles are
 // rewritten by other CTAs of the same launch).  The caller commits the group.
-__device__ __forceinline__ void copy_tile_async(double (*dst)[LDM], const double* src, int64_t ld,
-                                                int tid) {
+__device__ __forceinline__ void half_copy(double (*dst)[LDM], const double* src, int64_t ld,
+                                          int ht) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int e = tid + 256 * k;            // 2048 chunks of 16 bytes
+  for (int k = 0; k < 16; ++k) {
+    const int e = ht + 128 * k;             // 2048 chunks of 16 bytes
     const int r = e >> 5, c = (e & 31) * 2;
     const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&dst[r][c]));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + (int64_t)r * ld + c)
                  : "memory");
   }
-}
-__device__ __forceinline__ void copy_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void copy_wait_but_one() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -842,28 +839,6 @@ __device__ CholSync sync_view(int* base, int N) {
   return s;
 }
 
-// Whole-CTA bounded wait for *flag ≥ target; false on abort or time-out.
-__device__ bool cta_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok,
-                         uint32_t limit) {
-  if (threadIdx.x == 0) {
-    bool ok = false;
-    for (uint32_t it = 0; it < limit; ++it) {
-      if (ld_acquire(flag) >= target) { ok = true; break; }
-      if (*reinterpret_cast<volatile int*>(abortp)) break;
-      if (it > 32) __nanosleep(64);
-    }
-    if (!ok && !*reinterpret_cast<volatile int*>(abortp)) {
-      report(info, GPTQ_ERR_TIMEOUT, target);
-      atomicExch(abortp, 1);
-    }
-    *s_ok = ok ? 1 : 0;
-  }
-  __syncthreads();
-  const bool ok = *s_ok != 0;
-  __syncthreads();
-  return ok;
-}
-
 // The same wait for warps 0–3 and 5–7 (thread 0 polls), joined by barrier
 // kBarChain.
 __device__ bool group_wait(const int* flag, int target, int* abortp, int32_t* info, int* s_ok,
@@ -887,13 +862,6 @@ __device__ bool group_wait(const int* flag, int target, int* abortp, int32_t* in
   return ok;
 }
 
-__device__ __forceinline__ void cta_signal(int* flag, int value) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    st_release(flag, value);
-  }
-}
 
 // A worker task as operands, output and dependencies:
 //   PANEL  (k,i):   L_ik = A_ik·D_kᵀ     x = A_ik, y = D_k (NT)
@@ -956,33 +924,50 @@ __device__ WorkTask work_task(int task, int N, const int* prefix, int64_t np, do
   return t;
 }
 
-// One look at a task's dependencies (thread 0 of a CTA): all final?  The
-// flags are read at once (relaxed), and a fence after the last read gives the
-// acquire that the CTA's later loads of the tiles need.
 __device__ __forceinline__ int ld_relaxed(const int* p) {
   int v;
   asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ bool task_ready(const WorkTask& t) {
+
+// One look at every dependency of t (relaxed loads, all in flight at once).
+__device__ __forceinline__ bool deps_final(const WorkTask& t) {
   int v[3];
 #pragma unroll
   for (int d = 0; d < 3; ++d) v[d] = d < t.ndep ? ld_relaxed(t.dep[d]) : 0;
   bool ok = true;
 #pragma unroll
   for (int d = 0; d < 3; ++d) ok = ok && (d >= t.ndep || v[d] >= t.target[d]);
-  if (ok) asm volatile("fence.acq_rel.gpu;" ::: "memory");
   return ok;
 }
 
-// Whole-CTA bounded wait for every dependency of a task; false on abort or
-// time-out.
-__device__ bool wait_task(const WorkTask& t, int* abortp, int32_t* info, int* s_ok,
-                          uint32_t spin) {
-#pragma unroll
-  for (int d = 0; d < 3; ++d)
-    if (d < t.ndep && !cta_wait(t.dep[d], t.target[d], abortp, info, s_ok, spin)) return false;
-  return true;
+// A worker half's bounded wait for every dependency of t (thread 0 of the
+// half polls; a fence after the final look gives the acquire the half's
+// tile loads need); false on abort or time-out (reported).
+__device__ bool half_wait(const WorkTask& t, int* abortp, int32_t* info, int* s_ok, uint32_t spin,
+                          int ht, int hbar) {
+  if (ht == 0) {
+    bool ok = false;
+    for (uint32_t it = 0; it < spin; ++it) {
+      if (deps_final(t)) {
+        ok = true;
+        break;
+      }
+      if (*reinterpret_cast<volatile int*>(abortp)) break;
+      if (it > 32) __nanosleep(64);
+    }
+    if (ok) {
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    } else if (!*reinterpret_cast<volatile int*>(abortp)) {
+      report(info, GPTQ_ERR_TIMEOUT, t.target[0]);
+      atomicExch(abortp, 1);
+    }
+    *s_ok = ok ? 1 : 0;
+  }
+  bar_sync(hbar, 128);
+  const bool ok = *s_ok != 0;
+  bar_sync(hbar, 128);
+  return ok;
 }
 
 __global__ void __launch_bounds__(256, 1)
@@ -990,8 +975,9 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int64_t n, int64_t np, int N,
                        int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
-  __shared__ int s_role, s_task, s_ok, s_bad, s_got, s_fail, s_next, s_ready;
-  __shared__ WorkTask s_wt, s_wt2;
+  __shared__ int s_role, s_ok, s_bad, s_got, s_fail;
+  __shared__ int s_htask[2], s_hok[2];
+  __shared__ WorkTask s_hwt[2];
   // the task numbering's slot prefix, after the tiles
   int* prefix = reinterpret_cast<int*>(sm + 5 * NB * LDM + 192);
   __shared__ volatile int s_stop;
@@ -1121,83 +1107,52 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     return;
   }
 
-  // ---- the workers.  Three tasks per CTA are claimed at a time (in numbering
-  // order): the current one (its tiles in buffer set sb), the next one and
-  // the one after.  Thread 0 claims the one after at the start of an
-  // iteration and decodes it after the current task's products, so that the
-  // atomic's round trip runs under them; it looks at the next task's
-  // dependencies (all flags at once) before the products, and a next task
-  // found final has its tiles copied into the other buffer set under them.
-  // A next task that is not final yet is waited for, and copied, only after
-  // the current one is stored and signalled (it may depend on it).
-  // buffer set b: x at tile 2b, y at tile 2b + 1 of the dynamic shared memory
-  auto xb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + 2 * b * NB * LDM); };
-  auto yb = [&](int b) { return reinterpret_cast<double (*)[LDM]>(sm + (2 * b + 1) * NB * LDM); };
-  if (tid == 0) {
-    int c0 = atomicAdd(&S.ctrl[0], 1);
-    int c1 = atomicAdd(&S.ctrl[0], 1);
-    if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c0 = c1 = ntasks;
-    s_task = c0;
-    s_next = c1;
-    if (c0 < ntasks) s_wt = work_task(c0, N, prefix, np, A, M, S);
-    if (c1 < ntasks) s_wt2 = work_task(c1, N, prefix, np, A, M, S);
-  }
-  __syncthreads();
-  if (s_task >= ntasks) return;
-  WorkTask tc = s_wt;
-  int nx = s_next;
-  WorkTask tn = {};
-  if (nx < ntasks) tn = s_wt2;
-  if (!wait_task(tc, &S.ctrl[2], info, &s_ok, spin)) return;
-  copy_tile_async(xb(0), tc.x, np, tid);
-  copy_tile_async(yb(0), tc.y, np, tid);
-  copy_commit();
-  int sb = 0;
+  // ---- the workers: two independent halves of 4 warps (h = warp / 4), each
+  // claiming and computing its own tasks in numbering order, as two workers
+  // would.  One half's waits (its claim, its dependency poll, its tile
+  // copies and the release of its result) then run under the other half's
+  // float64 products.  Half h synchronises on named barrier 1 + h (128
+  // threads) and uses tiles 2h (x) and 2h + 1 (y).
+  const int h = warp >> 2, hw = warp & 3, ht = tid & 127, hbar = 1 + h;
+  double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * h * NB * LDM);
+  double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + (2 * h + 1) * NB * LDM);
+  int next = 0;
+  if (ht == 0) next = atomicAdd(&S.ctrl[0], 1);
   for (;;) {
-    int claim = 0;
-    if (tid == 0) {
-      claim = atomicAdd(&S.ctrl[0], 1);     // the task after the next; used below
-      s_ready = (nx < ntasks && task_ready(tn)) ? 1 : 0;
+    if (ht == 0) {
+      int c = next;
+      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
+      s_htask[h] = c;
+      if (c < ntasks) {
+        s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
+        next = atomicAdd(&S.ctrl[0], 1);       // the one after: its round trip runs meanwhile
+      }
     }
-    __syncthreads();
-    const bool pre = s_ready != 0;
-    if (pre) {
-      copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
-      copy_tile_async(yb(sb ^ 1), tn.y, np, tid);
-      copy_commit();
-      copy_wait_but_one();
-    } else {
-      copy_wait_all();
-    }
-    __syncthreads();
-    double2 cv[2][4];
-    if (tc.subtract) tile_load_c(tc.out, np, cv, warp, lane);
-    double acc[2][4][2] = {};
-    if (tc.nt)
-      tile_mm<true>(xb(sb), yb(sb), acc, warp, lane);
+    bar_sync(hbar, 128);
+    if (s_htask[h] >= ntasks) return;
+    const WorkTask t = s_hwt[h];
+    if (!half_wait(t, &S.ctrl[2], info, &s_hok[h], spin, ht, hbar)) return;
+    half_copy(x, t.x, np, ht);
+    half_copy(y, t.y, np, ht);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    double2 cv[4][4];
+    if (t.subtract) half_load_c(t.out, np, cv, hw, lane);
+    copy_wait_all();
+    bar_sync(hbar, 128);
+    double acc[4][4][2] = {};
+    if (t.nt)
+      half_mm<true>(x, y, acc, hw, lane);
     else
-      tile_mm<false>(xb(sb), yb(sb), acc, warp, lane);
-    if (tid == 0) {
-      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) claim = ntasks;
-      s_next = claim;
-      if (claim < ntasks) s_wt = work_task(claim, N, prefix, np, A, M, S);
-    }
-    if (tc.subtract)
-      tile_store<true>(tc.out, np, acc, cv, warp, lane);
+      half_mm<false>(x, y, acc, hw, lane);
+    if (t.subtract)
+      half_store<true>(t.out, np, acc, cv, hw, lane);
     else
-      tile_store<false>(tc.out, np, acc, cv, warp, lane);
-    cta_signal(tc.flag, tc.value);          // begins with a barrier: s_next, s_wt visible
-    if (nx >= ntasks) return;               // (then every later claim is past the end too)
-    if (!pre) {
-      if (!wait_task(tn, &S.ctrl[2], info, &s_ok, spin)) return;
-      copy_tile_async(xb(sb ^ 1), tn.x, np, tid);
-      copy_tile_async(yb(sb ^ 1), tn.y, np, tid);
-      copy_commit();
+      half_store<false>(t.out, np, acc, cv, hw, lane);
+    bar_sync(hbar, 128);                          // the half's stores are issued
+    if (ht == 0) {
+      __threadfence();
+      st_release(t.flag, t.value);
     }
-    tc = tn;
-    nx = s_next;
-    if (nx < ntasks) tn = s_wt;
-    sb ^= 1;
   }
 }
 
