@@ -157,23 +157,56 @@ static_params_kernel(const T* __restrict__ W, int64_t m, int64_t n,
   zero[r * ngroups + g] = (uint8_t)rintf(__fdiv_rn(-xmin, s));
 }
 
-// Wp[r][p] = W[r][perm[p]] as float32; dead columns read as 0.
+// Wp[r][p] = W[r][perm[p]] as float32; dead columns read as 0.  A CTA takes
+// `rpb` consecutive rows: they come into shared memory as they are (coalesced
+// 16-byte loads; rows of W are contiguous), and each thread then writes
+// consecutive processing positions of a row (coalesced stores), gathering
+// through perm from shared memory.  Rows longer than the staging area are
+// gathered from global memory instead (staged = 0).
 template <typename T>
 __global__ void __launch_bounds__(256)
 ingest_kernel(const T* __restrict__ W, int64_t m, int64_t n,
               const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
-              float* __restrict__ Wp, int32_t* info) {
-  const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (e >= m * n) return;
-  const int64_t r = e / n, p = e % n;
-  const int32_t c = perm[p];
-  float v = 0.f;
-  if (c >= 0 && c < n) {
-    v = to_f32(W[r * n + c]);
-    if (!isfinite(v)) { report(info, GPTQ_ERR_NONFINITE, r * n + c); v = 0.f; }
-    if (dead[c]) v = 0.f;
+              float* __restrict__ Wp, int rpb, int staged, int32_t* info) {
+  extern __shared__ __align__(16) unsigned char ig[];
+  T* sw = reinterpret_cast<T*>(ig);
+  const int64_t r0 = (int64_t)blockIdx.x * rpb;
+  const int rows = (int)(m - r0 < rpb ? m - r0 : (int64_t)rpb);
+  const int tid = threadIdx.x;
+  const T* src = W + r0 * n;
+  const int64_t elems = (int64_t)rows * n;
+  if (staged) {
+    const int64_t bytes = elems * (int64_t)sizeof(T);
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+      const int64_t v16 = bytes >> 4;
+      for (int64_t e = tid; e < v16; e += 256)
+        reinterpret_cast<uint4*>(ig)[e] = __ldg(reinterpret_cast<const uint4*>(src) + e);
+      for (int64_t e = (v16 << 4) / (int64_t)sizeof(T) + tid; e < elems; e += 256) sw[e] = src[e];
+    } else {
+      for (int64_t e = tid; e < elems; e += 256) sw[e] = src[e];
+    }
+    __syncthreads();
   }
-  Wp[e] = v;
+  const T* rowsrc = staged ? sw : src;
+  for (int rl = 0; rl < rows; ++rl) {
+    const int64_t r = r0 + rl;
+    for (int p = tid; p < n; p += 256) {
+      const int32_t c = perm[p];
+      float v = 0.f;
+      if (c >= 0 && c < n) {
+        v = to_f32(rowsrc[(int64_t)rl * n + c]);
+        if (!isfinite(v)) { report(info, GPTQ_ERR_NONFINITE, r * n + c); v = 0.f; }
+        if (dead[c]) v = 0.f;
+      }
+      Wp[r * n + p] = v;
+    }
+  }
+}
+
+// Rows per ingest CTA: up to 32 KB of W in shared memory (one row, read from
+// global memory, when a row is longer than 48 KB).
+inline int ingest_rows_per_block(int64_t n, size_t elem) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(16, 32768 / (n * (int64_t)elem)));
 }
 
 // Packing.  A CTA takes `rpb` consecutive rows: their codes (processing
@@ -320,13 +353,19 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
                        cudaStream_t s) {
   const int64_t ngroups = rowgs > 0 ? ceil_div(m, rowgs) : ceil_div(n, group);
   if (loss_row) GPTQ_CUDA(cudaMemsetAsync(loss_row, 0, sizeof(float) * m, s));
-  const unsigned gin = (unsigned)ceil_div(m * n, 256);
-  if (w_dtype == GPTQ_DTYPE_BF16)
-    GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<__nv_bfloat16>, gin, 256, 0,
-                static_cast<const __nv_bfloat16*>(W), m, n, perm, dead, w.Wp, info);
-  else
-    GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<float>, gin, 256, 0,
-                static_cast<const float*>(W), m, n, perm, dead, w.Wp, info);
+  {
+    const size_t es = w_dtype == GPTQ_DTYPE_BF16 ? 2 : 4;
+    const int rpb = ingest_rows_per_block(n, es);
+    const int staged = (int64_t)rpb * n * (int64_t)es <= 48 * 1024 ? 1 : 0;
+    const size_t ism = staged ? align_up((size_t)rpb * (size_t)n * es, 16) : 0;
+    const unsigned gin = (unsigned)ceil_div(m, rpb);
+    if (w_dtype == GPTQ_DTYPE_BF16)
+      GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<__nv_bfloat16>, gin, 256, ism,
+                  static_cast<const __nv_bfloat16*>(W), m, n, perm, dead, w.Wp, rpb, staged, info);
+    else
+      GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<float>, gin, 256, ism,
+                  static_cast<const float*>(W), m, n, perm, dead, w.Wp, rpb, staged, info);
+  }
 
   // padding rows of the working copy: zero, so that the last row box of
   // every sweep and trailing update reads defined values
