@@ -1116,18 +1116,16 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   const int h = warp >> 2, hw = warp & 3, ht = tid & 127, hbar = 1 + h;
   double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * h * NB * LDM);
   double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + (2 * h + 1) * NB * LDM);
+  // thread 0 of the half claims the next task before the current one's
+  // products and decodes it after them (the atomic's round trip and the
+  // decoding run while the other threads compute and store)
   int next = 0;
-  if (ht == 0) next = atomicAdd(&S.ctrl[0], 1);
+  if (ht == 0) {
+    const int c = atomicAdd(&S.ctrl[0], 1);
+    s_htask[h] = c;
+    if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
+  }
   for (;;) {
-    if (ht == 0) {
-      int c = next;
-      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
-      s_htask[h] = c;
-      if (c < ntasks) {
-        s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
-        next = atomicAdd(&S.ctrl[0], 1);       // the one after: its round trip runs meanwhile
-      }
-    }
     bar_sync(hbar, 128);
     if (s_htask[h] >= ntasks) return;
     const WorkTask t = s_hwt[h];
@@ -1139,20 +1137,24 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     if (t.subtract) half_load_c(t.out, np, cv, hw, lane);
     copy_wait_all();
     bar_sync(hbar, 128);
+    if (ht == 0) next = atomicAdd(&S.ctrl[0], 1);
     double acc[4][4][2] = {};
     if (t.nt)
       half_mm<true>(x, y, acc, hw, lane);
     else
       half_mm<false>(x, y, acc, hw, lane);
+    if (ht == 0) {
+      int c = next;
+      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
+      s_htask[h] = c;                         // read after the barrier below
+      if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
+    }
     if (t.subtract)
       half_store<true>(t.out, np, acc, cv, hw, lane);
     else
       half_store<false>(t.out, np, acc, cv, hw, lane);
     bar_sync(hbar, 128);                          // the half's stores are issued
-    if (ht == 0) {
-      __threadfence();
-      st_release(t.flag, t.value);
-    }
+    if (ht == 0) st_release(t.flag, t.value);    // orders them (through the barrier) before the flag
   }
 }
 
