@@ -242,17 +242,45 @@ def kernel_work(probs, block: int):
         fused = n % 4 == 0 and n > block
         if fused:
             w["trailing"] += 12 * n * n
+        for c0, c1, kw in far_updates(n, block, fused):
+            w["sweep" if fused else "trailing"] += 8 * m * (c1 - c0) + 4 * m * kw + 4 * kw * (c1 - c0)
         for j0 in range(0, n, block):
             bw = min(block, n - j0)
-            n2 = n - j0 - bw
             w["sweep"] += 9 * m * bw + 4 * bw * bw + 5 * m * (-(-bw // p.group))
-            if n2 > 0:
-                w["sweep" if fused else "trailing"] += 8 * m * n2 + 4 * m * bw + 4 * bw * n2
         w["pack"] += m * n + m * n * p.bits / 8 + 5 * m * ng
         w["ingest"] += m * n * (p.W.element_size() + 4)
     units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s",
              "sweep": "GB/s", "trailing": "GB/s", "pack": "GB/s", "ingest": "GB/s"}
     return {k: (units[k], v) for k, v in w.items()}
+
+
+SUPER_BLOCKS = 4
+
+
+def far_updates(n: int, block: int, fused: bool):
+    """The trailing-update applications of one quantize call, as (first
+    column, end column, K): block b's errors reach block b+1 in its sweep's
+    prologue and the rest as listed.  On the tensor-core path with 128-column
+    blocks, super-blocks of SUPER_BLOCKS blocks: inside one, block b−1's errors
+    reach the rest of the super-block and the block after it; the first block
+    of the next super-block's launch applies the whole previous super-block to
+    every column past that block."""
+    S = SUPER_BLOCKS if (fused and block == 128) else 1
+    out = []
+    nb = -(-n // block)
+    for b in range(1, nb):
+        j0 = b * block
+        c0 = j0 + min(block, n - j0)
+        if b % S != 0:
+            c1, kw = min(n, (b // S + 1) * S * block + block), block
+        else:
+            c1, kw = n, S * block
+        if c0 < c1:
+            out.append((c0, c1, kw))
+    if not fused:
+        # off the tensor-core path block b's errors go to the rest in one update
+        out = [(b * block + block, n, block) for b in range(nb - 1) if b * block + block < n]
+    return out
 
 
 def trailing_flops(probs, block: int) -> float:
@@ -417,31 +445,34 @@ class Job:
         """Fork the lanes off ``main`` and join them back.
 
         ``hosts``: per problem pinned input/output buffers (the end-to-end
-        step).  Each lane's copy stream then brings in, in the lane's order,
-        every problem's X and then its W, ahead of the compute; a problem
-        starts once its X is in and quantizes once its W is in, and its
-        results go back to the host on the lane's stream."""
+        step).  The host→device copies then run on one copy stream, in the
+        order the lanes need them: round r brings in the activations of every
+        lane's r-th problem, then their weights.  A problem starts once its
+        activations are in and quantizes once its weights are; its results go
+        back to the host on its lane's stream."""
         fork = torch.cuda.Event()
         fork.record(main)
-        joins = []
-        for lane in self.lanes:
-            s, cs = lane["s"], lane["cs"]
-            s.wait_event(fork)
-            ready = []
-            if hosts is not None:
-                cs.wait_event(fork)
-                for k in lane["plan"]:
-                    it = self.items[k]
-                    evs = []
-                    with torch.cuda.stream(cs):
-                        for key in ("X", "W"):
-                            it[key].copy_(hosts[k][key], non_blocking=True)
+        ready = {}
+        if hosts is not None:
+            cs = self.lanes[0]["cs"]
+            cs.wait_event(fork)
+            rounds = max(len(lane["plan"]) for lane in self.lanes)
+            with torch.cuda.stream(cs):
+                for r in range(rounds):
+                    batch = [lane["plan"][r] for lane in self.lanes if r < len(lane["plan"])]
+                    for key in ("X", "W"):
+                        for k in batch:
+                            self.items[k][key].copy_(hosts[k][key], non_blocking=True)
                             e = torch.cuda.Event()
                             e.record(cs)
-                            evs.append(e)
-                    ready.append(evs)
-            for r, k in enumerate(lane["plan"]):
-                xr, wr = ready[r] if hosts is not None else (None, None)
+                            ready.setdefault(k, {})[key] = e
+        joins = []
+        for lane in self.lanes:
+            s = lane["s"]
+            s.wait_event(fork)
+            for k in lane["plan"]:
+                xr = ready[k]["X"] if hosts is not None else None
+                wr = ready[k]["W"] if hosts is not None else None
                 self.run_problem(self.items[k], s, xr, wr,
                                  hosts[k] if hosts is not None else None)
             e = torch.cuda.Event()
@@ -476,6 +507,8 @@ def run_ours(args, rank, world, local):
                                    order=args.order)]
     layer = Job(probs, device, args.lanes, args.static_groups)
     params = sum(p.params for p in probs)
+    if args.factor_workers:
+        g.lib().gptq_set_factor_workers(int(args.factor_workers))
     main = torch.cuda.Stream(device=device)     # non-default: graphs capture here
     torch.cuda.set_stream(main)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
@@ -545,10 +578,10 @@ def run_ours(args, rank, world, local):
     kprof = g.gptq_profile_stop()
 
     # ---- end to end: pinned host inputs in, packed results out, every step.
-    # The copies are part of the captured step: each lane's copy stream brings
-    # in its problems' activations and weights ahead of the lane's compute, a
+    # The copies are part of the captured step: one copy stream brings in the
+    # problems' activations and weights in the order the lanes need them, a
     # problem starts once its activations are in and quantizes once its
-    # weights are, and its results go back on the lane's stream.
+    # weights are, and its results go back on its lane's stream.
     hosts = [{"X": it["X"].cpu().pin_memory(), "W": it["W"].cpu().pin_memory(),
               **{k: torch.empty(it[k].shape, dtype=it[k].dtype).pin_memory()
                  for k in Job.OUTS}} for it in layer.items]
@@ -609,6 +642,7 @@ def run_ours(args, rank, world, local):
                    "global_batch": len(probs) * world, "seq_len": probs[0].T,
                    "parallelism": f"independent layers x{world}",
                    "lanes": len(layer.lanes),
+                   "factor_workers": args.factor_workers or "every SM but one",
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step" if graph is not None else "eager launches"},
         "e2e": {"value": round(total_params / (e2e_ms / 1e3), 1), "unit": "params/s",
@@ -1520,6 +1554,8 @@ def main(argv=None):
                     help="decoder layers per step (default: every layer of the stack)")
     ap.add_argument("--lanes", type=int, default=4,
                     help="streams the problems of a step are spread over")
+    ap.add_argument("--factor-workers", type=int, default=0,
+                    help="most worker CTAs a factorisation may use (0: every SM but one)")
     ap.add_argument("--profile-steps", type=int, default=2,
                     help="steps of the serialised per-kernel timing pass")
     ap.add_argument("--bits", type=int, default=None)

@@ -164,6 +164,17 @@ gptq_status gptq_peak_probe(int kind, int64_t iters, double* flops, int32_t* inf
 void gptq_set_wait_limit(uint32_t polls);
 
 /*
+ * The most worker CTAs (one per SM, beside the one CTA that runs the
+ * factorisation's critical chain) a gptq_prepare launch may use; 0 restores
+ * the default, every SM but one.  Process-wide, read at each gptq_prepare
+ * call.  A caller running several factorisations and sweeps side by side on
+ * different streams may leave SMs to the other streams' kernels this way
+ * (the factorisation's CTAs stay resident until its last task).  The result
+ * does not depend on it.
+ */
+void gptq_set_factor_workers(int max_ctas);
+
+/*
  * gptq_prepare without a workspace argument: the same operation, arguments
  * and results as gptq_prepare, for callers that cannot hand this library a
  * block of device memory — for example code that runs while another

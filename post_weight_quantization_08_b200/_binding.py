@@ -74,6 +74,7 @@ _SIGS = {
                                      C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_size_t, C.c_void_p]),
     "gptq_set_wait_limit": (None, [C.c_uint32]),
+    "gptq_set_factor_workers": (None, [C.c_int]),
     "gptq_peak_probe": (C.c_int, [C.c_int, C.c_int64, C.POINTER(C.c_double), C.c_void_p,
                                   C.c_void_p, C.c_void_p]),
     "gptq_check": (C.c_int, [C.c_void_p, C.POINTER(C.c_int32), C.c_void_p]),

@@ -64,7 +64,7 @@ size_t hptq_ws_layout(int64_t m, int64_t n, int block, HptqWs* h, char* base) {
     o_h[k] = take(sizeof(unsigned long long) * NSYM);
     o_s[k] = take(sizeof(float) * (size_t)m * ngmax);
     o_z[k] = take((size_t)m * ngmax);
-    o_slot[k] = k ? take(quant_slot_layout(m, n, nullptr, nullptr, nullptr)) : 0;
+    o_slot[k] = k ? take(quant_slot_layout(m, n, block, nullptr, nullptr, nullptr)) : 0;
   }
   const size_t o_l = take(NSYM);
   const size_t o_k = take(sizeof(unsigned long long) * NSYM);
@@ -76,7 +76,7 @@ size_t hptq_ws_layout(int64_t m, int64_t n, int block, HptqWs* h, char* base) {
       h->hist[k] = reinterpret_cast<unsigned long long*>(base + o_h[k]);
       h->scale[k] = reinterpret_cast<float*>(base + o_s[k]);
       h->zero[k] = reinterpret_cast<uint8_t*>(base + o_z[k]);
-      if (k) quant_slot_layout(m, n, &h->w[0], &h->w[k], base + o_slot[k]);
+      if (k) quant_slot_layout(m, n, block, &h->w[0], &h->w[k], base + o_slot[k]);
     }
     h->lens = reinterpret_cast<unsigned char*>(base + o_l);
     h->canon = reinterpret_cast<unsigned long long*>(base + o_k);

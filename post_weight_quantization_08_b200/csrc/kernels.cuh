@@ -35,8 +35,9 @@ gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
 // j0 : j0+bw] on the tensor cores (pre.Uhi/Ulo: the transposed TF32 split of U,
 // n % 4 == 0), so that no separate trailing update is needed for those columns.
 struct SweepPrologue {
-  const float* Ehi = nullptr;   // previous block's errors (error_rows(m) × 128)
+  const float* Ehi = nullptr;   // previous block's errors (error_rows(m) rows, pitch epitch)
   const float* Elo = nullptr;
+  int64_t epitch = SWEEP_BLOCK_MAX;  // floats between rows of the error buffers
   const float* Uhi = nullptr;   // transposed TF32 split of U
   const float* Ulo = nullptr;
   int64_t k0 = 0;               // first column of the previous block
@@ -52,13 +53,14 @@ struct SweepPrologue {
 // U[far.k0 : far.k0+kw, c0:c1] (tensor cores, far.Uhi/Ulo as above): columns
 // the sweep does not touch, from inputs of earlier launches.
 struct SweepFar {
-  const float* Ehi = nullptr;
+  const float* Ehi = nullptr;   // errors: kw columns from here on each row, pitch epitch
   const float* Elo = nullptr;
+  int64_t epitch = SWEEP_BLOCK_MAX;
   const float* Uhi = nullptr;
   const float* Ulo = nullptr;
   int64_t c0 = 0, c1 = 0;       // columns (c1 is clipped to n)
-  int64_t k0 = 0;               // first column of the block whose errors they are
-  int kw = 0;                   // its width, 0 for none
+  int64_t k0 = 0;               // first column of the blocks whose errors they are
+  int kw = 0;                   // their width (one block, or a super-block), 0 for none
 };
 //
 // outl != NULL (SSQR): every group's step is multiplied by *outl->alpha (a
@@ -93,17 +95,61 @@ struct OutlierArgs {
 gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
-                         float* Elo, const SweepPrologue& pre, const SweepFar& far,
+                         float* Elo, int64_t epitch, const SweepPrologue& pre, const SweepFar& far,
                          float* loss_row, int32_t* info, const int32_t* rowgroup_perm,
                          const OutlierArgs* outl, cudaStream_t s);
 
 // ---- the stages of gptq_quantize, shared with the SSQR entry point
 
+// The two-level lazy batch: on the tensor-core path with 128-column blocks,
+// the errors of kSuperBlocks consecutive blocks (a super-block) sit side by
+// side, and the columns past the super-block (and the block after it)
+// receive them in one K = kSuperBlocks·128 product instead of one product a
+// block.
+constexpr int kSuperBlocks = 4;
+// Floats per row of the error buffers: a super-block, or one block elsewhere.
+int error_width(int64_t n, int block);
+
+// The far part of the trailing update carried by sweep b's launch (b ≥ 1) on
+// the tensor-core path with super-blocks of S blocks (S = 1: none).  Block
+// b−1's errors reach block b in sweep b's prologue; the far CTAs then apply
+//  * inside a super-block (b mod S ≠ 0): block b−1's errors (K = block,
+//    errors from column k0) to the rest of the super-block and the block
+//    after it;
+//  * at the first block of a super-block: the whole previous super-block's
+//    errors (K = S·block) to every column past block b.
+// Columns [c0, c1); empty when c0 ≥ c1.
+struct FarRange {
+  int64_t c0, c1, k0;
+  int kw;
+  bool whole;       // the previous super-block's errors
+};
+inline FarRange far_range(int64_t n, int block, int S, int64_t b) {
+  const int64_t j0 = b * block;
+  const int64_t bw = (n - j0 < block) ? (n - j0) : block;
+  FarRange r;
+  r.c0 = j0 + bw;
+  if (b % S != 0) {
+    const int64_t end = (b / S + 1) * S * (int64_t)block + block;
+    r.c1 = end < n ? end : n;
+    r.k0 = j0 - block;
+    r.kw = block;
+    r.whole = false;
+  } else {
+    r.c1 = n;
+    r.k0 = j0 - (int64_t)S * block;
+    r.kw = S * block;
+    r.whole = true;
+  }
+  return r;
+}
+
 struct QuantWs {
   float* Wp;        // error_rows(m) × n working copy, processing order
   uint8_t* codes;   // m × n codes, processing order
-  float* Ehi[2];    // error_rows(m) × 128 scaled errors of a block, TF32 part
-  float* Elo[2];    // remainder e − Ehi; two sets, alternating by block
+  float* Ehi[2];    // error_rows(m) × ew scaled errors of a super-block, TF32 part
+  float* Elo[2];    // remainder e − Ehi; two sets, alternating by super-block
+  int ew;           // floats per row of the error buffers (error_width)
   int32_t* pinv;    // n: processing position of each original column
   float* panels;    // pre-transposed U panels, one per block
   float* Uhi;       // n × n TF32 part of Uᵀ (tensor-core trailing update only)
@@ -115,7 +161,8 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base);
 // A second working set for a pass that runs beside another: its own Wp,
 // codes and error buffers at `base`, the U-derived parts (pinv, panels, the
 // TF32 split) shared with `shared`.  Returns its bytes; fills *w when given.
-size_t quant_slot_layout(int64_t m, int64_t n, const QuantWs* shared, QuantWs* w, char* base);
+size_t quant_slot_layout(int64_t m, int64_t n, int block, const QuantWs* shared, QuantWs* w,
+                         char* base);
 
 // Host checks shared by the quantize entry points (no device work).
 gptq_status quant_check_args(int w_dtype, int64_t m, int64_t n, int bits, int group,

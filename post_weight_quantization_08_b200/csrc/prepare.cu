@@ -1158,8 +1158,10 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   }
 }
 
-// Host side: the poll limit of the factorisation's waits (0: kSpinLimit).
+// Host side: the poll limit of the factorisation's waits (0: kSpinLimit), and
+// the most worker CTAs one factorisation launch may use (0: every SM but one).
 std::atomic<uint32_t> g_wait_limit{0};
+std::atomic<int> g_max_workers{0};
 
 // U[i][j] = L⁻¹[n−1−i][n−1−j] for j ≥ i, 0 below the diagonal.
 __global__ void __launch_bounds__(256)
@@ -1179,6 +1181,10 @@ using namespace gptq;
 
 extern "C" void gptq_set_wait_limit(uint32_t polls) {
   g_wait_limit.store(polls, std::memory_order_relaxed);
+}
+
+extern "C" void gptq_set_factor_workers(int max_ctas) {
+  g_max_workers.store(max_ctas > 0 ? max_ctas : 0, std::memory_order_relaxed);
 }
 
 extern "C" size_t gptq_prepare_workspace_bytes(int64_t n) {
@@ -1251,6 +1257,8 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   // besides the chain's, so that work on other streams finds SMs.
   int workers = N * N / 3 + 2;
   if (workers > num_sms - 1) workers = num_sms - 1;
+  const int cap = g_max_workers.load(std::memory_order_relaxed);
+  if (cap > 0 && workers > cap) workers = cap;
   if (workers > ntasks) workers = ntasks;
   const int grid = 1 + workers;
   const uint32_t lim = g_wait_limit.load(std::memory_order_relaxed);

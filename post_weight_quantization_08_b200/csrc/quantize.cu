@@ -16,6 +16,12 @@
 
 namespace gptq {
 
+int error_width(int64_t n, int block) {
+  return (trailing_uses_tensor_cores(n, block) && block == SWEEP_BLOCK_MAX)
+             ? kSuperBlocks * SWEEP_BLOCK_MAX
+             : SWEEP_BLOCK_MAX;
+}
+
 size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) {
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -28,8 +34,9 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   const size_t mrows = (size_t)error_rows(m);
   size_t o_wp = take(sizeof(float) * mrows * (size_t)n);
   size_t o_codes = take((size_t)m * (size_t)n);
+  const int ew = error_width(n, block);
   size_t o_e[4];
-  for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
+  for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * (size_t)ew);
   size_t o_pinv = take(sizeof(int32_t) * (size_t)n);
   size_t o_pan = take(panel_workspace_bytes(n, block));
   const bool tc = trailing_uses_tensor_cores(n, block);
@@ -42,6 +49,7 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
       w->Ehi[k] = reinterpret_cast<float*>(base + o_e[2 * k]);
       w->Elo[k] = reinterpret_cast<float*>(base + o_e[2 * k + 1]);
     }
+    w->ew = ew;
     w->pinv = reinterpret_cast<int32_t*>(base + o_pinv);
     w->panels = reinterpret_cast<float*>(base + o_pan);
     w->Uhi = tc ? reinterpret_cast<float*>(base + o_uhi) : nullptr;
@@ -50,7 +58,8 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   return off;
 }
 
-size_t quant_slot_layout(int64_t m, int64_t n, const QuantWs* shared, QuantWs* w, char* base) {
+size_t quant_slot_layout(int64_t m, int64_t n, int block, const QuantWs* shared, QuantWs* w,
+                         char* base) {
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -60,8 +69,9 @@ size_t quant_slot_layout(int64_t m, int64_t n, const QuantWs* shared, QuantWs* w
   const size_t mrows = (size_t)error_rows(m);
   const size_t o_wp = take(sizeof(float) * mrows * (size_t)n);
   const size_t o_codes = take((size_t)m * (size_t)n);
+  const int ew = error_width(n, block);
   size_t o_e[4];
-  for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * SWEEP_BLOCK_MAX);
+  for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * (size_t)ew);
   if (w && base && shared) {
     *w = *shared;
     w->Wp = reinterpret_cast<float*>(base + o_wp);
@@ -209,16 +219,58 @@ inline int ingest_rows_per_block(int64_t n, size_t elem) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(16, 32768 / (n * (int64_t)elem)));
 }
 
+// What the packer needs to fetch one code (and write its dequantized value).
+struct PackRow {
+  const uint8_t* codes;       // the CTA's rows of codes (shared or global memory)
+  int64_t n;
+  const int32_t* pinv;
+  const float* outv;
+  float* Qdq;
+  const float* scale;
+  const uint8_t* zero;
+  int group;
+  int64_t ngroups;
+  int rowgs;
+  int static_groups;
+  int32_t* info;
+};
+
+// Code of original column c of local row rl (row r), and its dequantized
+// value into Qdq when asked for.
+__device__ __forceinline__ uint32_t pack_code(const PackRow& a, int rl, int64_t r, int64_t c) {
+  const int64_t n = a.n;
+  if (c >= n) return 0u;
+  const int32_t p = a.pinv[c];
+  if (p < 0 || p >= n) {
+    report(a.info, GPTQ_ERR_INVALID_ARG, c);
+    return 0u;
+  }
+  uint32_t q = a.codes[(int64_t)rl * n + p];
+  bool kept = false;                 // an SSQR outlier: its value, not its code
+  if (a.outv != nullptr) {
+    kept = (q & OUTLIER_FLAG) != 0;
+    q &= ~(uint32_t)OUTLIER_FLAG;
+  }
+  if (a.Qdq != nullptr) {
+    // input-channel groups: [row][group of processing position p];
+    // output-channel groups (rowgs rows): [row group][original column c]
+    // (32-bit quotients: rows < 2^31, columns < 2^20)
+    const int64_t sx = a.rowgs > 0 ? (int64_t)((int)r / a.rowgs) * n + c
+                                   : r * a.ngroups + (a.static_groups ? (int)c : p) / a.group;
+    a.Qdq[r * n + c] = kept ? a.outv[r * n + p] : a.scale[sx] * ((float)q - (float)a.zero[sx]);
+  }
+  return q;
+}
+
 // Packing.  A CTA takes `rpb` consecutive rows: their codes (processing
 // order, contiguous in the code array) come into shared memory with coalesced
-// 16-byte loads.  Then a warp takes 32 original columns of one row at a time,
-// lane l column c = 32·chunk + l: its processing position pinv[c] (a coalesced
-// load), its code from shared memory, its dequantized value (a coalesced
-// store).  The chunk's BITS words are formed in registers: for widths that
-// divide 32 an OR over each word's group of lanes (shuffles), for 3 bits a
-// transpose through ballots (bit planes of the codes, then the words).
+// 16-byte loads.  Then a warp walks a row's original columns in chunks: each
+// column's processing position pinv[c] (a coalesced load), its code from
+// shared memory, its dequantized value (a coalesced store).  The chunk's
+// words are formed in registers: for widths that divide 32 by shuffles over
+// groups of lanes, for 3 bits by a transpose through ballots.
 template <int BITS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
             const int32_t* __restrict__ pinv, int group, int64_t ngroups, int rowgs,
             const float* __restrict__ scale, const uint8_t* __restrict__ zero,
@@ -242,48 +294,41 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
     for (int64_t e = tid; e < bytes; e += 256) sc[e] = src[e];
   }
   __syncthreads();
-  const int chunks = (int)((n + 31) / 32);
-  for (int rl = 0; rl < rows; ++rl)
-  for (int ch = warp; ch < chunks; ch += 8) {
-    const int64_t r = r0 + rl;
-    const int64_t c = (int64_t)ch * 32 + lane;
-    uint32_t q = 0;
-    if (c < n) {
-      const int32_t p = pinv[c];
-      if (p < 0 || p >= n) {
-        report(info, GPTQ_ERR_INVALID_ARG, c);
-      } else {
-        q = staged ? sc[(int64_t)rl * n + p] : src[(int64_t)rl * n + p];
-        bool kept = false;                 // an SSQR outlier: its value, not its code
-        if (outv != nullptr) {
-          kept = (q & OUTLIER_FLAG) != 0;
-          q &= ~(uint32_t)OUTLIER_FLAG;
-        }
-        if (Qdq != nullptr) {
-          // input-channel groups: [row][group of processing position p];
-          // output-channel groups (rowgs rows): [row group][original column c]
-          // (32-bit quotients: rows < 2^31, columns < 2^20)
-          const int64_t sx = rowgs > 0 ? (int64_t)((int)r / rowgs) * n + c
-                                       : r * ngroups + (static_groups ? (int)c : p) / group;
-          Qdq[r * n + c] = kept ? outv[r * n + p] : scale[sx] * ((float)q - (float)zero[sx]);
-        }
-      }
-    }
-    uint32_t mine = 0;                     // lane j < BITS: word j of the chunk
-    if constexpr (32 % BITS == 0) {
-      // G = 32/BITS codes per word: OR within groups of G lanes, then lane j
-      // takes word j from the first lane of group j
-      constexpr int G = 32 / BITS;
-      uint32_t v = q << (BITS * (lane % G));
+  const PackRow pr = {staged ? sc : src, n, pinv, outv, Qdq, scale, zero, group, ngroups, rowgs,
+                      static_groups, info};
+  if constexpr (32 % BITS == 0) {
+    // widths that divide 32: a warp takes 128 columns at a time, lane l the
+    // four columns 4l .. 4l+3 (a 4·BITS-bit piece at bit 4l·BITS of the
+    // chunk); G = 8/BITS lanes fill a word, OR-ed together by shuffles, and
+    // the first lane of each group stores it (4·BITS consecutive words)
+    constexpr int G = 8 / BITS;
+    const int chunks = (int)((n + 127) / 128);
+    for (int rl = 0; rl < rows; ++rl)
+    for (int ch = warp; ch < chunks; ch += 8) {
+      const int64_t r = r0 + rl;
+      const int64_t c0 = (int64_t)ch * 128 + 4 * lane;
+      uint32_t v = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v |= pack_code(pr, rl, r, c0 + i) << (BITS * i);
+      v <<= 4 * BITS * (lane % G);
 #pragma unroll
       for (int o = 1; o < G; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
-      mine = __shfl_sync(0xffffffffu, v, (lane % BITS) * G);
-    } else {
-      // codes straddle words: one ballot per code bit (plane b: bit b of every
-      // lane's code), then one ballot per word, lane t supplying bit t
+      const int64_t wi = (int64_t)ch * 4 * BITS + lane / G;
+      if (lane % G == 0 && wi < nwords) qweight[r * nwords + wi] = v;
+    }
+  } else {
+    // codes straddle words: a warp takes 32 columns at a time, lane l column
+    // 32·chunk + l; one ballot per code bit (plane b: bit b of every lane's
+    // code), then one ballot per word, lane t supplying bit t
+    const int chunks = (int)((n + 31) / 32);
+    for (int rl = 0; rl < rows; ++rl)
+    for (int ch = warp; ch < chunks; ch += 8) {
+      const int64_t r = r0 + rl;
+      const uint32_t q = pack_code(pr, rl, r, (int64_t)ch * 32 + lane);
       uint32_t plane[BITS];
 #pragma unroll
       for (int b = 0; b < BITS; ++b) plane[b] = __ballot_sync(0xffffffffu, (q >> b) & 1u);
+      uint32_t mine = 0;                   // lane j < BITS: word j of the chunk
 #pragma unroll
       for (int j = 0; j < BITS; ++j) {
         const int idx = 32 * j + lane, code = idx / BITS, b = idx % BITS;
@@ -293,9 +338,9 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
         const uint32_t word = __ballot_sync(0xffffffffu, (pb >> code) & 1u);
         if (lane == j) mine = word;
       }
+      const int64_t wi = (int64_t)ch * BITS + lane;
+      if (lane < BITS && wi < nwords) qweight[r * nwords + wi] = mine;
     }
-    const int64_t wi = (int64_t)ch * BITS + lane;
-    if (lane < BITS && wi < nwords) qweight[r * nwords + wi] = mine;
   }
 }
 
@@ -371,7 +416,7 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
   // every sweep and trailing update reads defined values
   if (error_rows(m) > m)
     GPTQ_CUDA(cudaMemsetAsync(w.Wp + m * n, 0, sizeof(float) * (size_t)(error_rows(m) - m) * n, s));
-  // Block b's errors reach the later columns in two parts:
+  // Block b's errors reach the later columns in parts:
   //  * block b+1's columns: on the tensor-core path, sweep b+1 applies them
   //    itself in its prologue (in TMEM, before its first column); otherwise a
   //    trailing update on the caller's stream;
@@ -379,11 +424,15 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
   //    b+1's own launch (those columns are not sweep b+1's, and the errors
   //    come from the launch before), so that the sweeps follow each other on
   //    one stream; otherwise a trailing update on the side stream,
-  //    overlapping sweep b+1.
-  // Every column still receives the blocks' contributions in block order:
-  // whatever touches block b's columns first waits for the far update of
-  // block b−2 (which also reached them), and the two error buffers alternate,
-  // so a far update's input is not overwritten before it is read.
+  //    overlapping sweep b+1.  On the tensor-core path with super-blocks of
+  //    S blocks, those CTAs cover only the rest of b's super-block and the
+  //    block after it; the columns past that receive the whole super-block's
+  //    errors at once, from the CTAs of the next super-block's first sweep.
+  // Every column still receives the contributions in block order: the
+  // launches follow each other on one stream (or whatever touches block b's
+  // columns first waits for the far update of block b−2), and the error
+  // buffers alternate by super-block, so a far update's input is not
+  // overwritten before it is read.
   const bool fused = w.Uhi != nullptr && trailing_uses_tensor_cores(n, block);
   SideStream* side = nullptr;
   if (!fused) {
@@ -391,10 +440,17 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
     if (st != GPTQ_OK) return st;
   }
   bool pending[2] = {false, false};
+  // errors: block b's slot of its super-block's buffer (S blocks a buffer,
+  // the two buffers alternate by super-block; S = 1 off the tensor-core path)
+  const int S = w.ew / SWEEP_BLOCK_MAX;
+  auto eslot = [&](int64_t bb, int hi) -> float* {
+    float* const* e = hi ? w.Ehi : w.Elo;
+    return e[(bb / S) & 1] + (bb % S) * SWEEP_BLOCK_MAX;
+  };
   for (int64_t j0 = 0, b = 0; j0 < n; j0 += block, ++b) {
     const int bw = (int)((n - j0 < block) ? (n - j0) : block);
-    float* ehi = w.Ehi[b & 1];
-    float* elo = w.Elo[b & 1];
+    float* ehi = eslot(b, 1);
+    float* elo = eslot(b, 0);
     if (pending[b & 1]) {                      // the far update of block b−2
       GPTQ_CUDA(cudaStreamWaitEvent(s, side->far[b & 1], 0));
       pending[b & 1] = false;
@@ -402,18 +458,27 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
     SweepPrologue pre;
     SweepFar far;
     if (fused && b > 0) {
-      pre.Ehi = far.Ehi = w.Ehi[(b - 1) & 1];
-      pre.Elo = far.Elo = w.Elo[(b - 1) & 1];
+      // block b−1's errors on this block's columns: the sweep's prologue
+      pre.Ehi = eslot(b - 1, 1);
+      pre.Elo = eslot(b - 1, 0);
+      pre.epitch = far.epitch = w.ew;
       pre.Uhi = far.Uhi = w.Uhi;
       pre.Ulo = far.Ulo = w.Ulo;
-      pre.k0 = far.k0 = j0 - block;
-      pre.kw = far.kw = block;
-      far.c0 = j0 + bw;                        // block b+1 on: the far columns of block b−1
-      far.c1 = n;
+      pre.k0 = j0 - block;
+      pre.kw = block;
+      // the far columns: block b−1's errors inside a super-block, the whole
+      // previous super-block's at the first block of the next (far_range)
+      const FarRange fr = far_range(n, block, S, b);
+      far.c0 = fr.c0;
+      far.c1 = fr.c1;
+      far.k0 = fr.k0;
+      far.kw = fr.kw;
+      far.Ehi = fr.whole ? w.Ehi[(b / S - 1) & 1] : pre.Ehi;
+      far.Elo = fr.whole ? w.Elo[(b / S - 1) & 1] : pre.Elo;
     }
     const float* panel = w.panels + (size_t)(j0 / block) * (PANEL_BYTES / sizeof(float));
     gptq_status st = launch_sweep(w.Wp, m, n, j0, bw, panel, bits, group, ngroups, w.codes,
-                                  scale, zero, ehi, elo, pre, far, loss_row, info,
+                                  scale, zero, ehi, elo, w.ew, pre, far, loss_row, info,
                                   rowgs > 0 ? perm : nullptr, outl, s);
     if (st != GPTQ_OK) return st;
     const int64_t c0 = j0 + bw, c1 = c0 + block;

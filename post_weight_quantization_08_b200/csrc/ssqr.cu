@@ -51,7 +51,7 @@ size_t ssqr_ws_layout(int64_t m, int64_t n, int block, SsqrWs* o, char* base) {
   for (int k = 1; k < 3; ++k) {
     o_sc[k] = take(sizeof(float) * (size_t)m * ngmax);
     o_z[k] = take((size_t)m * ngmax);
-    o_slot[k] = take(quant_slot_layout(m, n, nullptr, nullptr, nullptr));
+    o_slot[k] = take(quant_slot_layout(m, n, block, nullptr, nullptr, nullptr));
   }
   if (base && o) {
     o->st = reinterpret_cast<SearchState*>(base + o_st);
@@ -61,7 +61,7 @@ size_t ssqr_ws_layout(int64_t m, int64_t n, int block, SsqrWs* o, char* base) {
     for (int k = 1; k < 3; ++k) {
       o->scale[k] = reinterpret_cast<float*>(base + o_sc[k]);
       o->zero[k] = reinterpret_cast<uint8_t*>(base + o_z[k]);
-      quant_slot_layout(m, n, &o->w[0], &o->w[k], base + o_slot[k]);
+      quant_slot_layout(m, n, block, &o->w[0], &o->w[k], base + o_slot[k]);
     }
   }
   return off;

@@ -697,7 +697,7 @@ gptq_status launch_panels(const float* U, int64_t n, int block, float* panels,
 gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
                          const float* panel, int bits, int group, int64_t ngroups,
                          uint8_t* codes, float* scale, uint8_t* zero, float* Ehi,
-                         float* Elo, const SweepPrologue& pre, const SweepFar& far,
+                         float* Elo, int64_t epitch, const SweepPrologue& pre, const SweepFar& far,
                          float* loss_row, int32_t* info, const int32_t* rowgroup_perm,
                          const OutlierArgs* outl, cudaStream_t s) {
   constexpr size_t kSmem = SMEM_BYTES > QSMEM ? SMEM_BYTES : QSMEM;
@@ -731,9 +731,9 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
   const int64_t fc1 = far.c1 < n ? far.c1 : n;
   int fx = 0, nfar = 0;
   if (far.kw > 0 && far.c0 < fc1 && far.Ehi && far.Elo && far.Uhi && far.Ulo) {
-    if (far.kw % QK != 0 || far.kw > SB || (n % 4) != 0)
+    if (far.kw % QK != 0 || far.kw > kSuperBlocks * SB || far.kw > far.epitch || (n % 4) != 0)
       return fail(GPTQ_ERR_INVALID_ARG, "sweep far update: width %d", far.kw);
-    if (!make_trail_maps(&fm, Wp, m, n, far.Ehi, far.Elo, far.Uhi, far.Ulo))
+    if (!make_trail_maps(&fm, Wp, m, n, far.Ehi, far.Elo, far.kw, far.epitch, far.Uhi, far.Ulo))
       return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's far update");
     fx = (int)ceil_div(fc1 - far.c0, QN);
     nfar = fx * (int)ceil_div(m, QM);
@@ -751,8 +751,10 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
   if (kwp > 0) {
     if (kwp % SS != 0 || pre.kw > SB)
       return fail(GPTQ_ERR_INVALID_ARG, "sweep prologue: width %d", pre.kw);
-    if (!encode_tiled_2d(&tph, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Ehi, SB, mr, SB * 4, SS, RT) ||
-        !encode_tiled_2d(&tpl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Elo, SB, mr, SB * 4, SS, RT) ||
+    if (!encode_tiled_2d(&tph, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Ehi, SB, mr, pre.epitch * 4,
+                         SS, RT) ||
+        !encode_tiled_2d(&tpl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Elo, SB, mr, pre.epitch * 4,
+                         SS, RT) ||
         !encode_tiled_2d(&tuh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Uhi, n, n, n * 4, SS, RT) ||
         !encode_tiled_2d(&tul, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pre.Ulo, n, n, n * 4, SS, RT))
       return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's prologue");
@@ -762,8 +764,8 @@ gptq_status launch_sweep(float* Wp, int64_t m, int64_t n, int64_t j0, int bw,
     memset(&tuh, 0, sizeof(tuh));
     memset(&tul, 0, sizeof(tul));
   }
-  if (!encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ehi, SB, mr, SB * 4, SS, RT) ||
-      !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, SB * 4, SS, RT))
+  if (!encode_tiled_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ehi, SB, mr, epitch * 4, SS, RT) ||
+      !encode_tiled_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Elo, SB, mr, epitch * 4, SS, RT))
     return fail(GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the sweep's error output");
   const int nsweep = (int)ceil_div(m, RT);
   const unsigned grid = (unsigned)(nsweep + nfar);

@@ -110,10 +110,11 @@ bool encode_f32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t oute
 }  // namespace
 
 bool make_trail_maps(TrailMaps* maps, float* Wp, int64_t m, int64_t n, const float* Ehi,
-                     const float* Elo, const float* UhiT, const float* UloT) {
+                     const float* Elo, int64_t kw, int64_t epitch, const float* UhiT,
+                     const float* UloT) {
   const int64_t mr = error_rows(m);
-  return encode_f32(&maps->ahi, Ehi, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
-         encode_f32(&maps->alo, Elo, SWEEP_BLOCK_MAX, mr, SWEEP_BLOCK_MAX * 4, QK, QM) &&
+  return encode_f32(&maps->ahi, Ehi, kw, mr, epitch * 4, QK, QM) &&
+         encode_f32(&maps->alo, Elo, kw, mr, epitch * 4, QK, QM) &&
          encode_f32(&maps->bhi, UhiT, n, n, n * 4, QK, QN) &&
          encode_f32(&maps->blo, UloT, n, n, n * 4, QK, QN) &&
          encode_f32(&maps->c, Wp, n, mr, n * 4, 32, QM);

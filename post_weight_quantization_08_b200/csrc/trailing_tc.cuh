@@ -47,7 +47,8 @@ struct TrailMaps {
 // Tensor maps of the update Wp[:, c0:] −= (Ehi+Elo)·U (errors error_rows(m) ×
 // 128, UhiT/UloT the transposed TF32 split of U, Wp error_rows(m) × n).
 bool make_trail_maps(TrailMaps* maps, float* Wp, int64_t m, int64_t n, const float* Ehi,
-                     const float* Elo, const float* UhiT, const float* UloT);
+                     const float* Elo, int64_t kw, int64_t epitch, const float* UhiT,
+                     const float* UloT);
 
 namespace {
 
