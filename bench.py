@@ -371,17 +371,34 @@ def est_cost(p) -> float:
     return (2.0 / 3.0) * p.n ** 3 / 30e12 + 3.0 * p.m * p.n * p.n / 1e15
 
 
+def factor_workers(arg, nprobs, device):
+    """Most worker CTAs a factorisation may use: ``arg`` when given (0: every
+    SM but one); by default (-1) three quarters of the SMs when the step has
+    eight or more problems, so that sweeps of factorised problems run beside
+    the next factorisation, and every SM but one otherwise."""
+    if arg >= 0:
+        return int(arg)
+    if nprobs < 8:
+        return 0
+    return int(0.76 * torch.cuda.get_device_properties(device).multi_processor_count)
+
+
 class Job:
     """Device buffers of a list of problems (every layer of a stack), allocated
-    once.  The problems run on ``lanes`` streams: each lane takes its share one
-    after the other, the lanes side by side; problems go, most expensive first,
-    to the lane with the least work so far.  With ``static_groups`` the
-    quantize call fixes every group's parameters from the original weights
-    (gptq_quantize_static)."""
+    once, and the step's schedule.  Hessians and factorisations run on
+    ``lanes`` streams: each lane takes its share one after the other, the lanes
+    side by side; problems go, most expensive first, to the lane with the least
+    work so far.  Each problem's quantize then runs on one of ``qstreams``
+    streams as soon as its factorisation is done, the longest column sweeps
+    first: a quantize is a chain of dependent sweep launches that may hold
+    only a few CTAs (a down projection of 2048 rows: 16), so several of them
+    side by side fill the GPU where one alone would leave it mostly idle.
+    With ``static_groups`` the quantize call fixes every group's parameters
+    from the original weights (gptq_quantize_static)."""
 
     OUTS = ("qweight", "scale", "zero", "g_idx", "loss")
 
-    def __init__(self, probs, device, lanes, static_groups=False):
+    def __init__(self, probs, device, lanes, static_groups=False, qstreams=8):
         import post_weight_quantization_08_b200 as g
         self.g = g
         self.probs = probs
@@ -412,17 +429,22 @@ class Job:
                 "loss": torch.empty(m, dtype=torch.float32, device=device),
             })
         nl = max(1, min(int(lanes), len(probs)))
-        self.lanes = [{"s": torch.cuda.Stream(device=device),
-                       "cs": torch.cuda.Stream(device=device), "plan": [], "load": 0.0}
+        self.lanes = [{"s": torch.cuda.Stream(device=device), "plan": [], "load": 0.0}
                       for _ in range(nl)]
         for k in sorted(range(len(probs)), key=lambda k: -est_cost(probs[k])):
             lane = min(self.lanes, key=lambda ln: ln["load"])
             lane["plan"].append(k)
             lane["load"] += est_cost(probs[k])
+        self.cs = torch.cuda.Stream(device=device)            # host copies
+        nq = max(1, min(int(qstreams), len(probs)))
+        self.qs = [torch.cuda.Stream(device=device) for _ in range(nq)]
+        # quantize order: longest sweep chain (blocks) first, then most rows
+        self.qorder = sorted(range(len(probs)),
+                             key=lambda k: (-(-probs[k].n // probs[k].block), -probs[k].m))
 
-    def run_problem(self, it, s, x_ready=None, w_ready=None, host=None):
-        """One problem on stream ``s``; ``x_ready`` / ``w_ready``: events after
-        which X / W are in place; ``host``: pinned buffers for the results."""
+    def prepare_problem(self, it, s, x_ready=None):
+        """Hessian and factorisation of one problem on stream ``s``; ``x_ready``:
+        the event after which X is in place."""
         g, p = self.g, it["p"]
         if x_ready is not None:
             s.wait_event(x_ready)
@@ -431,6 +453,12 @@ class Job:
         g.gptq_hessian_accumulate(it["X"], it["H"], it["info_h"], s)
         g.gptq_prepare(it["H"], p.damp, p.order, it["perm"], it["U"], it["dead"],
                        it["info_p"], it["ws_p"], s)
+
+    def quantize_problem(self, it, s, w_ready=None, host=None):
+        """Quantize of one problem on stream ``s`` (its factorisation done);
+        ``w_ready``: the event after which W is in place; ``host``: pinned
+        buffers for the results."""
+        g, p = self.g, it["p"]
         if w_ready is not None:
             s.wait_event(w_ready)
         g.gptq_quantize(it["W"], it["U"], it["perm"], it["dead"], p.bits, p.group, p.block,
@@ -441,40 +469,55 @@ class Job:
                 for k in self.OUTS:
                     host[k].copy_(it[k], non_blocking=True)
 
+    def run_problem(self, it, s):
+        self.prepare_problem(it, s)
+        self.quantize_problem(it, s)
+
     def step(self, main, hosts=None):
-        """Fork the lanes off ``main`` and join them back.
+        """Fork the lanes and quantize streams off ``main`` and join them back.
 
         ``hosts``: per problem pinned input/output buffers (the end-to-end
-        step).  The host→device copies then run on one copy stream, in the
-        order the lanes need them: round r brings in the activations of every
-        lane's r-th problem, then their weights.  A problem starts once its
-        activations are in and quantizes once its weights are; its results go
-        back to the host on its lane's stream."""
+        step).  The host→device copies then run on one copy stream: every
+        problem's activations in the order the lanes need them (round r: each
+        lane's r-th problem), then the weights in quantize order.  A problem's
+        Hessian waits for its activations and its quantize for its weights;
+        its results go back to the host on its quantize stream."""
         fork = torch.cuda.Event()
         fork.record(main)
-        ready = {}
+        xr, wr = {}, {}
         if hosts is not None:
-            cs = self.lanes[0]["cs"]
-            cs.wait_event(fork)
+            self.cs.wait_event(fork)
             rounds = max(len(lane["plan"]) for lane in self.lanes)
-            with torch.cuda.stream(cs):
-                for r in range(rounds):
-                    batch = [lane["plan"][r] for lane in self.lanes if r < len(lane["plan"])]
-                    for key in ("X", "W"):
-                        for k in batch:
-                            self.items[k][key].copy_(hosts[k][key], non_blocking=True)
-                            e = torch.cuda.Event()
-                            e.record(cs)
-                            ready.setdefault(k, {})[key] = e
+            xorder = [lane["plan"][r] for r in range(rounds) for lane in self.lanes
+                      if r < len(lane["plan"])]
+            with torch.cuda.stream(self.cs):
+                for key, order, dst in (("X", xorder, xr), ("W", self.qorder, wr)):
+                    for k in order:
+                        self.items[k][key].copy_(hosts[k][key], non_blocking=True)
+                        e = torch.cuda.Event()
+                        e.record(self.cs)
+                        dst[k] = e
+        prepared = {}
         joins = []
         for lane in self.lanes:
             s = lane["s"]
             s.wait_event(fork)
             for k in lane["plan"]:
-                xr = ready[k]["X"] if hosts is not None else None
-                wr = ready[k]["W"] if hosts is not None else None
-                self.run_problem(self.items[k], s, xr, wr,
-                                 hosts[k] if hosts is not None else None)
+                self.prepare_problem(self.items[k], s, xr.get(k))
+                e = torch.cuda.Event()
+                e.record(s)
+                prepared[k] = e
+            e = torch.cuda.Event()
+            e.record(s)
+            joins.append(e)
+        for q, k in enumerate(self.qorder):
+            s = self.qs[q % len(self.qs)]
+            if q < len(self.qs):
+                s.wait_event(fork)
+            s.wait_event(prepared[k])
+            self.quantize_problem(self.items[k], s, wr.get(k),
+                                  hosts[k] if hosts is not None else None)
+        for s in self.qs:
             e = torch.cuda.Event()
             e.record(s)
             joins.append(e)
@@ -505,10 +548,10 @@ def run_ours(args, rank, world, local):
     probs = [p for l in range(nl)
              for p in problems_for(args.config, layer=layer_for_rank(rank) * nl + l, bits=bits,
                                    order=args.order)]
-    layer = Job(probs, device, args.lanes, args.static_groups)
+    layer = Job(probs, device, args.lanes, args.static_groups, args.qstreams)
     params = sum(p.params for p in probs)
-    if args.factor_workers:
-        g.lib().gptq_set_factor_workers(int(args.factor_workers))
+    workers = factor_workers(args.factor_workers, len(probs), device)
+    g.lib().gptq_set_factor_workers(workers)
     main = torch.cuda.Stream(device=device)     # non-default: graphs capture here
     torch.cuda.set_stream(main)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
@@ -641,8 +684,8 @@ def run_ours(args, rank, world, local):
         "config": {"workload": wl, "params_per_step_per_gpu": params,
                    "global_batch": len(probs) * world, "seq_len": probs[0].T,
                    "parallelism": f"independent layers x{world}",
-                   "lanes": len(layer.lanes),
-                   "factor_workers": args.factor_workers or "every SM but one",
+                   "lanes": len(layer.lanes), "qstreams": len(layer.qs),
+                   "factor_workers": workers or "every SM but one",
                    "l2": "flushed between timed steps (256 MB write)",
                    "launch": "CUDA graph replay per step" if graph is not None else "eager launches"},
         "e2e": {"value": round(total_params / (e2e_ms / 1e3), 1), "unit": "params/s",
@@ -1422,6 +1465,34 @@ def oracle_pass(probs, static_groups=False):
     return sum(p.params for p in probs)
 
 
+CPU_SAMPLE_ROWS = 1024
+
+
+def oracle_problem_seconds(p, static_groups=False, rows=CPU_SAMPLE_ROWS):
+    """Seconds the float64 oracle takes for one whole problem, from a bounded
+    sample: the Hessian and the factorisation in full, the oracle's layer pass
+    on the first `rows` rows (which factorises again), and the per-row part of
+    that pass scaled to all m rows (rows are independent given U).  Returns
+    (seconds, rows sampled)."""
+    from oracle import gptq as og
+    from oracle import static as ost
+    X = p.X.to(torch.float64).numpy()
+    W = p.W.to(torch.float64).numpy()
+    r = min(rows, p.m)
+    t0 = time.perf_counter()
+    H = og.hessian(X)
+    t1 = time.perf_counter()
+    og.prepare(H, p.damp, p.order)
+    t2 = time.perf_counter()
+    if static_groups:
+        ost.gptq_layer_static(W[:r], H, p.bits, p.group, p.block, p.damp, p.order)
+    else:
+        og.gptq_layer(W[:r], H, p.bits, p.group, p.block, p.damp, p.order)
+    t3 = time.perf_counter()
+    per_rows = max(0.0, (t3 - t2) - (t2 - t1))
+    return (t1 - t0) + (t2 - t1) + per_rows * p.m / r, r
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -1434,21 +1505,29 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(probs, budget_s: float = 12.0, static_groups=False):
-    """The float64 oracle on the host cores over whole problems of the step
-    (each with its Hessian, factorisation and sweep), one after the other in
-    the step's order, until ``budget_s`` has passed (at least one problem)."""
-    done, t0, count = 0, time.perf_counter(), 0
+    """The float64 oracle on the host cores over problems of the step, one after
+    the other in the step's order, until ``budget_s`` has passed (at least one
+    problem).  Small problems run whole; larger ones are a bounded sample
+    (oracle_problem_seconds: Hessian and factorisation in full, the per-row
+    pass on CPU_SAMPLE_ROWS rows scaled to all rows)."""
+    done, est, count = 0, 0.0, 0
+    t0 = time.perf_counter()
+    samples = []
     while True:
-        done += oracle_pass([probs[count % len(probs)]], static_groups)
+        p = probs[count % len(probs)]
+        sec, r = oracle_problem_seconds(p, static_groups)
+        done += p.params
+        est += sec
+        samples.append(f"{p.m}x{p.n}" + ("" if r >= p.m else f" ({r} of {p.m} rows)"))
         count += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or count >= 50:
+        if time.perf_counter() - t0 >= budget_s or count >= 50:
             break
-    names = sorted({f"{probs[k % len(probs)].m}x{probs[k % len(probs)].n}" for k in range(count)})
-    return {"value": round(done / el, 1), "unit": "params/s", "cores": blas_threads(),
+    el = time.perf_counter() - t0
+    return {"value": round(done / est, 1), "unit": "params/s", "cores": blas_threads(),
             "kind": "oracle",
-            "sample": (f"{count} whole problems of the step ({', '.join(names)}; "
-                       f"{el:.1f} s, float64 numpy)")}
+            "sample": (f"{count} problems of the step ({', '.join(sorted(set(samples)))}; "
+                       f"{el:.1f} s of float64 numpy): Hessian and factorisation in full, "
+                       f"the per-row pass scaled from the sampled rows to all rows")}
 
 
 def frontend_workload(frontend: str, cfg, bits: int, group: int, block: int) -> str:
@@ -1515,27 +1594,32 @@ def run_reference(args, rank, world):
     nl = stack_layers(args)
     probs = problems_for(args.config, layer=0, bits=bits, order=args.order)
     for k in range(args.warmup):
-        oracle_pass([probs[k % len(probs)]], args.static_groups)
+        oracle_problem_seconds(probs[k % len(probs)], args.static_groups)
     t0 = time.perf_counter()
-    params = 0
+    params, est = 0, 0.0
     for k in range(args.steps):
-        params += oracle_pass([probs[k % len(probs)]], args.static_groups)
+        p = probs[k % len(probs)]
+        sec, _ = oracle_problem_seconds(p, args.static_groups)
+        params += p.params
+        est += sec
     el = time.perf_counter() - t0
-    value = params / el
+    value = params / est
     cores = blas_threads()
     shapes = ", ".join(f"{p.m}x{p.n}" for p in probs)
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "params/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "ms_per_step": round(est * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded cone activations, N(0,0.02^2) weights)",
         "config": {"workload": workload_name(args.config, bits, args.order, args.static_groups,
                                              nl)},
         "cpu_baseline": {"value": round(value, 1), "unit": "params/s", "cores": cores,
                          "kind": "oracle",
-                         "sample": (f"per step one whole problem of a layer ({shapes}, in "
-                                    f"turn), {args.steps} timed steps on the host cores")},
+                         "sample": (f"per step one problem of a layer ({shapes}, in turn): "
+                                    f"Hessian and factorisation in full, the per-row pass on "
+                                    f"the first {CPU_SAMPLE_ROWS} rows scaled to all rows; "
+                                    f"{args.steps} timed steps ({el:.1f} s) on the host cores")},
         "e2e": {"value": round(value, 1), "unit": "params/s",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -1553,9 +1637,13 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=None,
                     help="decoder layers per step (default: every layer of the stack)")
     ap.add_argument("--lanes", type=int, default=4,
-                    help="streams the problems of a step are spread over")
-    ap.add_argument("--factor-workers", type=int, default=0,
-                    help="most worker CTAs a factorisation may use (0: every SM but one)")
+                    help="streams the Hessians and factorisations are spread over")
+    ap.add_argument("--qstreams", type=int, default=8,
+                    help="streams the quantize calls are spread over")
+    ap.add_argument("--factor-workers", type=int, default=-1,
+                    help="most worker CTAs a factorisation may use (0: every SM but one; "
+                         "default: three quarters of the SMs when a step has eight or more "
+                         "problems)")
     ap.add_argument("--profile-steps", type=int, default=2,
                     help="steps of the serialised per-kernel timing pass")
     ap.add_argument("--bits", type=int, default=None)
