@@ -183,6 +183,13 @@ prep_gather_kernel(const float* __restrict__ H, int64_t n, int64_t np,
 // over all banks and keeps every row 16-byte aligned.  Fragment layout of an
 // 8×8×4 product: lane = 4·g + t holds A[g][t], B[t][g] and C[g][2t], C[g][2t+1].
 constexpr int LDM = 68;
+// Worker groups of 4 warps per CTA, the launch's threads, and the shared
+// memory before the slot prefix: the chain's five tiles and 192 doubles, or
+// two tiles per worker group.
+constexpr int kGroups = 3;
+constexpr int kCholThreads = 128 * kGroups;
+constexpr int kTileDoubles = (5 * NB * LDM + 192 > 2 * kGroups * NB * LDM) ? 5 * NB * LDM + 192
+                                                                            : 2 * kGroups * NB * LDM;
 
 __device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
@@ -231,7 +238,7 @@ struct PanelOut {
   int* flag;
 };
 
-// Named barriers of the diagonal tile (0 is __syncthreads): 1 joins the six
+// Named barriers of the diagonal tile (0 is the chain's CTA-wide barrier): 1 joins the six
 // working warps (1–3, 5–7); 2 hands X and the next panel block from warp 0 to
 // them; 3 hands their finished trailing updates back to warp 0; 4 tells warp 4
 // that they have stored the panel of the step before; 5 joins warps 0–3 and
@@ -243,6 +250,13 @@ constexpr int kRest = 192, kHand = 224;     // 6 working warps; + warp 0
 
 __device__ __forceinline__ void bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// The chain runs on the first 256 threads of its CTA (the launch has
+// kCholThreads; the rest of the chain CTA leaves at once): barrier 0 with
+// that count stands for __syncthreads on the chain's path.
+constexpr int kChainThreads = 256;
+__device__ __forceinline__ void chain_sync() {
+  asm volatile("bar.sync 0, %0;" ::"n"(kChainThreads) : "memory");
 }
 __device__ __forceinline__ void bar_arrive(int id, int count) {
   __threadfence_block();
@@ -370,7 +384,7 @@ __device__ __forceinline__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM
     *s_stop = 0;
     *s_got = 0;
   }
-  __syncthreads();
+  chain_sync();
   if (warp == 0) {
     double l[36];
 #pragma unroll
@@ -536,7 +550,7 @@ __device__ __forceinline__ bool diag_tile_smem(double (*a)[LDM], double (*b)[LDM
       }
     }
   }
-  __syncthreads();
+  chain_sync();
   return *bad_s == 0;
 }
 
@@ -725,7 +739,9 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
 //   NN: y holds B (row q, column n):       C = X·Y.
 // With the row pitch LDM ≡ 4 (mod 16) doubles, every fragment load of either
 // layout touches each bank pair exactly twice (two wavefronts, no conflict).
-template <bool NT>
+// With NEG the products are subtracted (acc −= X·B): the accumulators start
+// from the tile being updated.
+template <bool NT, bool NEG>
 __device__ __forceinline__ void half_mm(const double (*x)[LDM], const double (*y)[LDM],
                                         double acc[4][4][2], int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
@@ -734,7 +750,7 @@ __device__ __forceinline__ void half_mm(const double (*x)[LDM], const double (*y
   for (int q = 0; q < NB; q += 4) {
     double a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = x[rb + 8 * i + g][q + t];
+    for (int i = 0; i < 4; ++i) a[i] = NEG ? -x[rb + 8 * i + g][q + t] : x[rb + 8 * i + g][q + t];
 #pragma unroll
     for (int j = 0; j < 4; ++j) b[j] = NT ? y[cb + 8 * j + g][q + t] : y[q + t][cb + 8 * j + g];
 #pragma unroll
@@ -745,33 +761,33 @@ __device__ __forceinline__ void half_mm(const double (*x)[LDM], const double (*y
 }
 
 // The part of a 64×64 output tile (leading dimension ld) that a lane's
-// accumulators cover, read ahead of the products (for C −= X·B).
-__device__ __forceinline__ void half_load_c(const double* out, int64_t ld, double2 (&c)[4][4],
-                                            int hw, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      c[i][j] = __ldcg(reinterpret_cast<const double2*>(out + (int64_t)(rb + 8 * i + g) * ld +
-                                                        cb + 8 * j + 2 * t));
-}
-
-// out = C, or out = c − C with c the values read by half_load_c.
-template <bool SUBTRACT>
-__device__ __forceinline__ void half_store(double* out, int64_t ld, const double acc[4][4][2],
-                                           const double2 (&c)[4][4], int hw, int lane) {
+// accumulators cover: into the accumulators (the start of C −= X·B), and
+// back out.
+__device__ __forceinline__ void half_load_acc(const double* out, int64_t ld, double acc[4][4][2],
+                                              int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      double2* p = reinterpret_cast<double2*>(out + (int64_t)(rb + 8 * i + g) * ld + cb + 8 * j + 2 * t);
-      *p = SUBTRACT ? make_double2(c[i][j].x - acc[i][j][0], c[i][j].y - acc[i][j][1])
-                    : make_double2(acc[i][j][0], acc[i][j][1]);
+      const double2 v = __ldcg(reinterpret_cast<const double2*>(out + (int64_t)(rb + 8 * i + g) * ld +
+                                                                cb + 8 * j + 2 * t));
+      acc[i][j][0] = v.x;
+      acc[i][j][1] = v.y;
     }
+}
+
+__device__ __forceinline__ void half_store(double* out, int64_t ld, const double acc[4][4][2],
+                                           int hw, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<double2*>(out + (int64_t)(rb + 8 * i + g) * ld + cb + 8 * j + 2 * t) =
+          make_double2(acc[i][j][0], acc[i][j][1]);
 }
 
 // One 64×64 float64 tile (leading dimension ld) into shared memory as it is,
@@ -970,16 +986,16 @@ __device__ bool half_wait(const WorkTask& t, int* abortp, int32_t* info, int* s_
   return ok;
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kCholThreads, 1)
 chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int64_t n, int64_t np, int N,
                        int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
   __shared__ int s_role, s_ok, s_bad, s_got, s_fail;
-  __shared__ int s_htask[2], s_hok[2];
-  __shared__ WorkTask s_hwt[2];
+  __shared__ int s_htask[kGroups], s_hok[kGroups];
+  __shared__ WorkTask s_hwt[kGroups];
   // the task numbering's slot prefix, after the tiles
-  int* prefix = reinterpret_cast<int*>(sm + 5 * NB * LDM + 192);
+  int* prefix = reinterpret_cast<int*>(sm + kTileDoubles);
   __shared__ volatile int s_stop;
   const CholSync S = sync_view(sync_base, N);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -991,6 +1007,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   if (*reinterpret_cast<volatile int32_t*>(info) != 0) return;
 
   if (s_role == 0) {
+    if (warp >= kChainThreads / 32) return;
     // ---- the critical chain: DIAG(k), then PANEL(k, k+1) and the last
     // update of tile (k+1, k+1), which stays in shared memory for DIAG(k+1).
     // Two buffers alternate as the diagonal tile and two as D (warp 4 clears
@@ -1011,7 +1028,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       s_bad = 0;
       s_fail = 0;
     }
-    __syncthreads();
+    chain_sync();
     for (int k = 0; k < N; ++k) {
       const int64_t base = (int64_t)k * NB;
       double (*a)[LDM] = (k & 1) ? t1 : t0;
@@ -1101,22 +1118,22 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
         }
         if (!ok && tid == 0) s_fail = 1;
       }
-      __syncthreads();
+      chain_sync();
       if (s_fail) return;
     }
     return;
   }
 
-  // ---- the workers: two independent halves of 4 warps (h = warp / 4), each
-  // claiming and computing its own tasks in numbering order, as two workers
-  // would.  One half's waits (its claim, its dependency poll, its tile
-  // copies and the release of its result) then run under the other half's
-  // float64 products.  Half h synchronises on named barrier 1 + h (128
-  // threads) and uses tiles 2h (x) and 2h + 1 (y).
+  // ---- the workers: kGroups independent groups of 4 warps (h = warp / 4),
+  // each claiming and computing its own tasks in numbering order, as that
+  // many workers would.  One group's waits (its claim, its dependency poll,
+  // its tile copies and the release of its result) then run under the other
+  // groups' float64 products.  Group h synchronises on named barrier 1 + h
+  // (128 threads) and uses tiles 2h (x) and 2h + 1 (y).
   const int h = warp >> 2, hw = warp & 3, ht = tid & 127, hbar = 1 + h;
   double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * h * NB * LDM);
   double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + (2 * h + 1) * NB * LDM);
-  // thread 0 of the half claims the next task before the current one's
+  // thread 0 of the group claims the next task before the current one's
   // products and decodes it after them (the atomic's round trip and the
   // decoding run while the other threads compute and store)
   int next = 0;
@@ -1133,27 +1150,34 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     half_copy(x, t.x, np, ht);
     half_copy(y, t.y, np, ht);
     asm volatile("cp.async.commit_group;" ::: "memory");
-    double2 cv[4][4];
-    if (t.subtract) half_load_c(t.out, np, cv, hw, lane);
+    // C −= X·B starts from C; out = X·B from zero
+    double acc[4][4][2];
+    if (t.subtract) {
+      half_load_acc(t.out, np, acc, hw, lane);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+    }
     copy_wait_all();
     bar_sync(hbar, 128);
     if (ht == 0) next = atomicAdd(&S.ctrl[0], 1);
-    double acc[4][4][2] = {};
-    if (t.nt)
-      half_mm<true>(x, y, acc, hw, lane);
-    else
-      half_mm<false>(x, y, acc, hw, lane);
+    if (t.nt) {
+      if (t.subtract) half_mm<true, true>(x, y, acc, hw, lane);
+      else half_mm<true, false>(x, y, acc, hw, lane);
+    } else {
+      if (t.subtract) half_mm<false, true>(x, y, acc, hw, lane);
+      else half_mm<false, false>(x, y, acc, hw, lane);
+    }
     if (ht == 0) {
       int c = next;
       if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
       s_htask[h] = c;                         // read after the barrier below
       if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
     }
-    if (t.subtract)
-      half_store<true>(t.out, np, acc, cv, hw, lane);
-    else
-      half_store<false>(t.out, np, acc, cv, hw, lane);
-    bar_sync(hbar, 128);                          // the half's stores are issued
+    half_store(t.out, np, acc, hw, lane);
+    bar_sync(hbar, 128);                          // the group's stores are issued
     if (ht == 0) st_release(t.flag, t.value);    // orders them (through the barrier) before the flag
   }
 }
@@ -1215,9 +1239,9 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   prep_ws_layout(n, &w, static_cast<char*>(ws));
   const int64_t np = ceil_div(n, NB) * NB;
   const int N = (int)(np / NB);
-  // five tiles and the chain's 8×8 pivot blocks, then the task numbering's
-  // slot prefix (N + kMLag + 1 ints)
-  const size_t tile_smem = (5 * NB * LDM + 192) * sizeof(double) +
+  // the tiles (the chain's five and its 8×8 pivot blocks, or two per worker
+  // group), then the task numbering's slot prefix (N + kMLag + 1 ints)
+  const size_t tile_smem = kTileDoubles * sizeof(double) +
                            sizeof(int) * (size_t)(task_slots(N) + 1);
   if (total_tasks(N) >= ((int64_t)1 << 31) || tile_smem > 227 * 1024)
     return fail(GPTQ_ERR_UNSUPPORTED, "gptq_prepare: n=%lld is too large for the factorisation",
@@ -1262,7 +1286,7 @@ extern "C" gptq_status gptq_prepare(const float* H, int64_t n, double damp,
   if (workers > ntasks) workers = ntasks;
   const int grid = 1 + workers;
   const uint32_t lim = g_wait_limit.load(std::memory_order_relaxed);
-  GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, 256, tile_smem, w.A, w.M, n, np,
+  GPTQ_LAUNCH(KK_CHOL, s, chol_persistent_kernel, grid, kCholThreads, tile_smem, w.A, w.M, n, np,
               N, ntasks, w.sync, info, lim != 0 ? lim : kSpinLimit);
   GPTQ_LAUNCH(KK_PREP_OUT, s, prep_out_kernel, (unsigned)ceil_div(n * n, 256), 256, 0,
               w.M, n, np, U);
