@@ -612,13 +612,17 @@ def run_ours(args, rank, world, local):
     # launch bracketed by CUDA events on its own stream
     # (problems one after the other on one stream, so that no kernel's
     # interval includes time spent waiting for the other problem's kernels)
+    # (nothing else runs beside a serialised kernel, so the factorisation gets
+    # every SM here, as it would alone)
     prof_steps = max(1, min(args.steps, args.profile_steps))
+    g.lib().gptq_set_factor_workers(0)
     g.gptq_profile_start(1 << 17)
     for _ in range(prof_steps):
         flush.fill_(1.0)
         layer.step_serial(main)
     torch.cuda.synchronize(device)
     kprof = g.gptq_profile_stop()
+    g.lib().gptq_set_factor_workers(workers)
 
     # ---- end to end: pinned host inputs in, packed results out, every step.
     # The copies are part of the captured step: one copy stream brings in the
@@ -687,6 +691,7 @@ def run_ours(args, rank, world, local):
                    "lanes": len(layer.lanes), "qstreams": len(layer.qs),
                    "factor_workers": workers or "every SM but one",
                    "l2": "flushed between timed steps (256 MB write)",
+                   "kernel_figures": "serialised eager pass, the factorisation on every SM",
                    "launch": "CUDA graph replay per step" if graph is not None else "eager launches"},
         "e2e": {"value": round(total_params / (e2e_ms / 1e3), 1), "unit": "params/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

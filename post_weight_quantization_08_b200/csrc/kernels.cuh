@@ -150,7 +150,8 @@ struct QuantWs {
   float* Ehi[2];    // error_rows(m) × ew scaled errors of a super-block, TF32 part
   float* Elo[2];    // remainder e − Ehi; two sets, alternating by super-block
   int ew;           // floats per row of the error buffers (error_width)
-  int32_t* pinv;    // n: processing position of each original column
+  int32_t* pinv;    // n + 1: processing position of each original column; pinv[n] = −1
+                    // when the processing order is the identity, else 0
   float* panels;    // pre-transposed U panels, one per block
   float* Uhi;       // n × n TF32 part of Uᵀ (tensor-core trailing update only)
   float* Ulo;       // n × n remainder, transposed likewise

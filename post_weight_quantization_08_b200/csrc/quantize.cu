@@ -37,7 +37,7 @@ size_t quant_ws_layout(int64_t m, int64_t n, int block, QuantWs* w, char* base) 
   const int ew = error_width(n, block);
   size_t o_e[4];
   for (int k = 0; k < 4; ++k) o_e[k] = take(sizeof(float) * mrows * (size_t)ew);
-  size_t o_pinv = take(sizeof(int32_t) * (size_t)n);
+  size_t o_pinv = take(sizeof(int32_t) * (size_t)(n + 1));
   size_t o_pan = take(panel_workspace_bytes(n, block));
   const bool tc = trailing_uses_tensor_cores(n, block);
   size_t o_uhi = tc ? take(sizeof(float) * (size_t)n * (size_t)n) : 0;
@@ -117,7 +117,8 @@ gptq_status side_stream_for(cudaStream_t s, SideStream** out) {
   return GPTQ_OK;
 }
 
-// pinv[perm[p]] = p and g_idx[perm[p]] = p / group (static groups: c / group).
+// pinv[perm[p]] = p and g_idx[perm[p]] = p / group (static groups: c / group);
+// pinv[n] (−1 before the launch) becomes 0 unless perm is the identity.
 __global__ void __launch_bounds__(256)
 pinv_kernel(const int32_t* __restrict__ perm, int64_t n, int group,
             int32_t* __restrict__ pinv, int32_t* __restrict__ g_idx, int static_groups,
@@ -125,6 +126,7 @@ pinv_kernel(const int32_t* __restrict__ perm, int64_t n, int group,
   const int64_t p = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (p >= n) return;
   const int32_t c = perm[p];
+  if (c != p) pinv[n] = 0;
   if (c < 0 || c >= n) { report(info, GPTQ_ERR_INVALID_ARG, p); return; }
   pinv[c] = (int32_t)p;
   if (g_idx) g_idx[c] = (int32_t)((static_groups ? c : p) / group);
@@ -167,22 +169,67 @@ static_params_kernel(const T* __restrict__ W, int64_t m, int64_t n,
   zero[r * ngroups + g] = (uint8_t)rintf(__fdiv_rn(-xmin, s));
 }
 
+// Eight consecutive elements of W as float32 (16- or 32-byte loads).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // Wp[r][p] = W[r][perm[p]] as float32; dead columns read as 0.  A CTA takes
-// `rpb` consecutive rows: they come into shared memory as they are (coalesced
-// 16-byte loads; rows of W are contiguous), and each thread then writes
-// consecutive processing positions of a row (coalesced stores), gathering
-// through perm from shared memory.  Rows longer than the staging area are
-// gathered from global memory instead (staged = 0).
+// `rpb` consecutive rows.
+//  * The processing order is the identity (*ident = −1) and `vec` (n a
+//    multiple of 8, W 16-byte and dead 8-byte aligned): a stream, eight consecutive elements
+//    a thread (one or two 16-byte loads, the eight dead flags in one 8-byte
+//    load, two 16-byte stores).
+//  * Otherwise the rows come into shared memory as they are (coalesced
+//    16-byte loads; rows of W are contiguous), and each thread then writes
+//    consecutive processing positions of a row (coalesced stores), gathering
+//    through perm from shared memory.  Rows longer than the staging area are
+//    gathered from global memory instead (staged = 0).
 template <typename T>
 __global__ void __launch_bounds__(256)
 ingest_kernel(const T* __restrict__ W, int64_t m, int64_t n,
               const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
-              float* __restrict__ Wp, int rpb, int staged, int32_t* info) {
+              float* __restrict__ Wp, int rpb, int staged, const int32_t* __restrict__ ident,
+              int vec, int32_t* info) {
   extern __shared__ __align__(16) unsigned char ig[];
   T* sw = reinterpret_cast<T*>(ig);
   const int64_t r0 = (int64_t)blockIdx.x * rpb;
   const int rows = (int)(m - r0 < rpb ? m - r0 : (int64_t)rpb);
   const int tid = threadIdx.x;
+  if (vec && *ident == -1) {
+    const int n8 = (int)(n >> 3);
+    for (int rl = 0; rl < rows; ++rl) {
+      const int64_t r = r0 + rl;
+      for (int k = tid; k < n8; k += 256) {
+        const int64_t c = (int64_t)k * 8;
+        float v[8];
+        load8(W + r * n + c, v);
+        const uint2 d = __ldg(reinterpret_cast<const uint2*>(dead + c));
+        const uint32_t dw[2] = {d.x, d.y};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (!isfinite(v[e])) { report(info, GPTQ_ERR_NONFINITE, r * n + c + e); v[e] = 0.f; }
+          if ((dw[e >> 2] >> (8 * (e & 3))) & 0xFFu) v[e] = 0.f;
+        }
+        float4* o = reinterpret_cast<float4*>(Wp + r * n + c);
+        o[0] = make_float4(v[0], v[1], v[2], v[3]);
+        o[1] = make_float4(v[4], v[5], v[6], v[7]);
+      }
+    }
+    return;
+  }
   const T* src = W + r0 * n;
   const int64_t elems = (int64_t)rows * n;
   if (staged) {
@@ -262,7 +309,57 @@ __device__ __forceinline__ uint32_t pack_code(const PackRow& a, int rl, int64_t 
   return q;
 }
 
-// Packing.  A CTA takes `rpb` consecutive rows: their codes (processing
+// Words of 32 consecutive codes (in processing order = original order) at
+// BITS bits each, LSB first: BITS words from 32 code bytes (each < 2^BITS).
+template <int BITS>
+__device__ __forceinline__ void pack32(const uint4 (&c)[2], uint32_t (&out)[BITS]) {
+  const uint32_t b[8] = {c[0].x, c[0].y, c[0].z, c[0].w, c[1].x, c[1].y, c[1].z, c[1].w};
+  if constexpr (BITS == 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[k] = b[k];
+  } else if constexpr (BITS == 4) {
+    // four bytes → 16 bits: byte pairs merged, then the two halves
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t lo = b[2 * k], hi = b[2 * k + 1];
+      lo |= lo >> 4;
+      hi |= hi >> 4;
+      out[k] = (lo & 0xFFu) | ((lo >> 8) & 0xFF00u) | ((hi & 0xFFu) << 16) | ((hi << 8) & 0xFF000000u);
+    }
+  } else if constexpr (BITS == 2) {
+    // four bytes → 8 bits
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t x = b[4 * k + q];
+        x |= x >> 6;
+        w |= ((x & 0xFu) | ((x >> 12) & 0xF0u)) << (8 * q);
+      }
+      out[k] = w;
+    }
+  } else {
+    // 3 bits: code j at bit 3j of a 96-bit string
+    uint64_t lo = 0, hi = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint64_t q = (b[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+      const int pos = 3 * j;
+      if (pos < 64) lo |= q << pos;
+      if (pos + 3 > 64) hi |= pos >= 64 ? q << (pos - 64) : q >> (64 - pos);
+    }
+    out[0] = (uint32_t)lo;
+    out[1] = (uint32_t)(lo >> 32);
+    out[2] = (uint32_t)hi;
+  }
+}
+
+// Packing.  With the identity as processing order, plain codes (no outlier
+// values, no dequantized copy) and `flat` (n a multiple of 32, qweight
+// 16-byte aligned), the codes of the CTA's rows and their words are two
+// contiguous streams: a thread turns 32 code bytes (two 16-byte loads) into
+// BITS words.  Otherwise a CTA takes `rpb` consecutive rows: their codes (processing
 // order, contiguous in the code array) come into shared memory with coalesced
 // 16-byte loads.  Then a warp walks a row's original columns in chunks: each
 // column's processing position pinv[c] (a coalesced load), its code from
@@ -276,11 +373,33 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t m, int64_t n,
             const float* __restrict__ scale, const uint8_t* __restrict__ zero,
             uint32_t* __restrict__ qweight, int64_t nwords,
             float* __restrict__ Qdq, const float* __restrict__ outv, int static_groups,
-            int rpb, int staged, int32_t* info) {
+            int rpb, int staged, int flat, int32_t* info) {
   extern __shared__ __align__(16) uint8_t sc[];
   const int64_t r0 = (int64_t)blockIdx.x * rpb;
   const int rows = (int)(m - r0 < rpb ? m - r0 : (int64_t)rpb);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (flat && pinv[n] == -1) {
+    // 32 codes → BITS words; the CTA's rows are contiguous in both arrays
+    const int chunks = (int)(((int64_t)rows * n) >> 5);
+    const uint4* in = reinterpret_cast<const uint4*>(codes + r0 * n);
+    uint32_t* out = qweight + r0 * nwords;
+    for (int k = tid; k < chunks; k += 256) {
+      const uint4 c[2] = {__ldg(in + 2 * k), __ldg(in + 2 * k + 1)};
+      uint32_t w[BITS];
+      pack32<BITS>(c, w);
+      if constexpr (BITS % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < BITS; q += 4)
+          *reinterpret_cast<uint4*>(out + (int64_t)k * BITS + q) = make_uint4(w[q], w[q + 1], w[q + 2], w[q + 3]);
+      } else if constexpr (BITS == 2) {
+        *reinterpret_cast<uint2*>(out + (int64_t)k * 2) = make_uint2(w[0], w[1]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < BITS; ++q) out[(int64_t)k * BITS + q] = w[q];
+      }
+    }
+    return;
+  }
   const uint8_t* src = codes + r0 * n;
   const int64_t bytes = (int64_t)rows * n;
   if (!staged) {
@@ -379,7 +498,7 @@ gptq_status quant_setup(const QuantWs& w, int64_t m, int64_t n, const float* U,
                         int32_t* info, cudaStream_t s, bool static_groups) {
   (void)m;
   GPTQ_CUDA(cudaMemsetAsync(info, 0, 2 * sizeof(int32_t), s));
-  GPTQ_CUDA(cudaMemsetAsync(w.pinv, 0xFF, sizeof(int32_t) * n, s));
+  GPTQ_CUDA(cudaMemsetAsync(w.pinv, 0xFF, sizeof(int32_t) * (n + 1), s));
   GPTQ_LAUNCH(KK_INGEST, s, pinv_kernel, (unsigned)ceil_div(n, 256), 256, 0, perm, n,
               group, w.pinv, g_idx, static_groups ? 1 : 0, info);
   gptq_status st = launch_panels(U, n, block, w.panels, s);
@@ -404,12 +523,16 @@ gptq_status quant_pass(const QuantWs& w, const void* W, int w_dtype, int64_t m, 
     const int staged = (int64_t)rpb * n * (int64_t)es <= 48 * 1024 ? 1 : 0;
     const size_t ism = staged ? align_up((size_t)rpb * (size_t)n * es, 16) : 0;
     const unsigned gin = (unsigned)ceil_div(m, rpb);
+    const int vec = (n % 8 == 0 && (reinterpret_cast<uintptr_t>(W) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(dead) & 7) == 0) ? 1 : 0;
     if (w_dtype == GPTQ_DTYPE_BF16)
       GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<__nv_bfloat16>, gin, 256, ism,
-                  static_cast<const __nv_bfloat16*>(W), m, n, perm, dead, w.Wp, rpb, staged, info);
+                  static_cast<const __nv_bfloat16*>(W), m, n, perm, dead, w.Wp, rpb, staged,
+                  w.pinv + n, vec, info);
     else
       GPTQ_LAUNCH(KK_INGEST, s, ingest_kernel<float>, gin, 256, ism,
-                  static_cast<const float*>(W), m, n, perm, dead, w.Wp, rpb, staged, info);
+                  static_cast<const float*>(W), m, n, perm, dead, w.Wp, rpb, staged,
+                  w.pinv + n, vec, info);
   }
 
   // padding rows of the working copy: zero, so that the last row box of
@@ -514,22 +637,24 @@ gptq_status quant_pack(const QuantWs& w, int64_t m, int64_t n, int bits, int gro
   const unsigned gpk = (unsigned)ceil_div(m, rpb);
   const int staged = (int64_t)rpb * n <= kPackStageMax ? 1 : 0;
   const size_t psm = staged ? align_up((size_t)rpb * (size_t)n, 16) : 0;
+  const int flat = (n % 32 == 0 && (reinterpret_cast<uintptr_t>(qweight) & 15) == 0 &&
+                    Qdq == nullptr && outl_vals == nullptr) ? 1 : 0;
   switch (bits) {
     case 2:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<2>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, flat, info);
       break;
     case 3:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<3>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, flat, info);
       break;
     case 4:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<4>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, flat, info);
       break;
     default:
       GPTQ_LAUNCH(KK_PACK, s, pack_kernel<8>, gpk, 256, psm, w.codes, m, n, w.pinv, group,
-                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, info);
+                  ngroups, rowgs, scale, zero, qweight, nwords, Qdq, outl_vals, sg, rpb, staged, flat, info);
       break;
   }
   return GPTQ_OK;

@@ -150,6 +150,38 @@ def test_identity_hessian_is_rtn():
     assert np.array_equal(q["zero"].cpu().numpy().astype(np.float32), z)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_identity_hessian_is_rtn_streamed(bits):
+    """The streamed ingest and pack (identity order, n a multiple of 32, no
+    dequantized copy): with H = I, codes, scales and zeros equal RTN bit for bit."""
+    import post_weight_quantization_08_b200 as g
+    n, m = 512, 70
+    W = gaussian_weights(m, n, 150 + bits)
+    H = torch.eye(n, dtype=torch.float32, device=DEV)
+    prep = g.prepare(H, 0.01, "natural")
+    q = g.quantize(W.to(DEV), prep, bits, 128, 128, want_qdq=False)
+    codes = P.unpack_rows(q["qweight"].cpu().numpy(), bits, n)
+    c, s, z, _ = ol.rtn(W.double().numpy(), bits, 128)
+    assert np.array_equal(codes, c)
+    assert np.array_equal(q["scale"].cpu().numpy(), s)
+    assert np.array_equal(q["zero"].cpu().numpy().astype(np.float32), z)
+
+
+@pytest.mark.parametrize("order", ["natural", "act"])
+@pytest.mark.parametrize("bits", [3, 4])
+def test_pack_paths_agree(order, bits):
+    """Asking for the dequantized copy switches the packer (and, for the
+    natural order, nothing else) to its gathering path: the words agree."""
+    import post_weight_quantization_08_b200 as g
+    X, W = _layer(512, 576, 130, 30 + bits)
+    H = g.hessian(X.to(DEV))
+    prep = g.prepare(H, 0.01, order)
+    a = g.quantize(W.to(DEV), prep, bits, 128, 128, want_qdq=False)
+    b = g.quantize(W.to(DEV), prep, bits, 128, 128, want_qdq=True)
+    for k in ("qweight", "scale", "zero", "g_idx", "loss_row"):
+        assert torch.equal(a[k], b[k]), k
+
+
 def test_dead_columns():
     X, W = _layer(300, 100, 20, 16)
     X[:, [3, 50]] = 0
