@@ -438,9 +438,9 @@ class Job:
         self.cs = torch.cuda.Stream(device=device)            # host copies
         nq = max(1, min(int(qstreams), len(probs)))
         self.qs = [torch.cuda.Stream(device=device) for _ in range(nq)]
-        # quantize order: longest sweep chain (blocks) first, then most rows
+        # quantize order: longest sweep chain (most blocks) first, then most rows
         self.qorder = sorted(range(len(probs)),
-                             key=lambda k: (-(-probs[k].n // probs[k].block), -probs[k].m))
+                             key=lambda k: ((-probs[k].n) // probs[k].block, -probs[k].m))
 
     def prepare_problem(self, it, s, x_ready=None):
         """Hessian and factorisation of one problem on stream ``s``; ``x_ready``:

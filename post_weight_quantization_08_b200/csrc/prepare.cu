@@ -1133,10 +1133,10 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   const int h = warp >> 2, hw = warp & 3, ht = tid & 127, hbar = 1 + h;
   double (*x)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + 2 * h * NB * LDM);
   double (*y)[LDM] = reinterpret_cast<double (*)[LDM]>(sm + (2 * h + 1) * NB * LDM);
-  // thread 0 of the group claims the next task before the current one's
-  // products and decodes it after them (the atomic's round trip and the
-  // decoding run while the other threads compute and store)
-  int next = 0;
+  // thread 0 of the group claims and decodes the next task while the current
+  // one's tiles land; during the current products the group then pulls the
+  // next output tile towards L2 (the trailing matrix does not fit there, so
+  // an update tile would otherwise come from DRAM on the critical path)
   if (ht == 0) {
     const int c = atomicAdd(&S.ctrl[0], 1);
     s_htask[h] = c;
@@ -1160,21 +1160,26 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
     }
+    if (ht == 0) {
+      int c = atomicAdd(&S.ctrl[0], 1);
+      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
+      s_htask[h] = c;                         // read at the top of the next round
+      if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
+    }
     copy_wait_all();
     bar_sync(hbar, 128);
-    if (ht == 0) next = atomicAdd(&S.ctrl[0], 1);
+    if (s_htask[h] < ntasks && s_hwt[h].subtract) {
+      // 64 rows × four 128-byte lines: two lines a thread
+      const double* o = s_hwt[h].out + (int64_t)(ht >> 1) * np + (ht & 1) * 32;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(o));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(o + 16));
+    }
     if (t.nt) {
       if (t.subtract) half_mm<true, true>(x, y, acc, hw, lane);
       else half_mm<true, false>(x, y, acc, hw, lane);
     } else {
       if (t.subtract) half_mm<false, true>(x, y, acc, hw, lane);
       else half_mm<false, false>(x, y, acc, hw, lane);
-    }
-    if (ht == 0) {
-      int c = next;
-      if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
-      s_htask[h] = c;                         // read after the barrier below
-      if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
     }
     half_store(t.out, np, acc, hw, lane);
     bar_sync(hbar, 128);                          // the group's stores are issued
