@@ -957,9 +957,11 @@ __device__ __forceinline__ bool deps_final(const WorkTask& t) {
   return ok;
 }
 
-// A worker half's bounded wait for every dependency of t (thread 0 of the
-// half polls; a fence after the final look gives the acquire the half's
-// tile loads need); false on abort or time-out (reported).
+// A worker group's bounded wait for every dependency of t (thread 0 of the
+// group polls; a fence after the final look gives the acquire the group's
+// tile loads need); false on abort or time-out (reported).  One barrier:
+// thread 0 writes *s_ok again only in the group's next wait, after two more
+// group barriers that every reader has passed.
 __device__ bool half_wait(const WorkTask& t, int* abortp, int32_t* info, int* s_ok, uint32_t spin,
                           int ht, int hbar) {
   if (ht == 0) {
@@ -981,9 +983,7 @@ __device__ bool half_wait(const WorkTask& t, int* abortp, int32_t* info, int* s_
     *s_ok = ok ? 1 : 0;
   }
   bar_sync(hbar, 128);
-  const bool ok = *s_ok != 0;
-  bar_sync(hbar, 128);
-  return ok;
+  return *s_ok != 0;
 }
 
 __global__ void __launch_bounds__(kCholThreads, 1)
@@ -1142,8 +1142,12 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     s_htask[h] = c;
     if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
   }
+  bar_sync(hbar, 128);
+  // Per task three group barriers: in the wait (the dependencies are final),
+  // after the copies (the tiles have landed; the next task is decoded), after
+  // the stores.  The next task's record is written before the second and read
+  // after the third.
   for (;;) {
-    bar_sync(hbar, 128);
     if (s_htask[h] >= ntasks) return;
     const WorkTask t = s_hwt[h];
     if (!half_wait(t, &S.ctrl[2], info, &s_hok[h], spin, ht, hbar)) return;
@@ -1183,7 +1187,10 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     }
     half_store(t.out, np, acc, hw, lane);
     bar_sync(hbar, 128);                          // the group's stores are issued
-    if (ht == 0) st_release(t.flag, t.value);    // orders them (through the barrier) before the flag
+    // a thread of the second warp publishes the result (the release orders the
+    // group's stores, through the barrier, before the flag) while thread 0
+    // polls the next task's dependencies
+    if (ht == 32) st_release(t.flag, t.value);
   }
 }
 
