@@ -232,12 +232,17 @@ def kernel_work(probs, block: int):
               tensor-core path, else the SIMT trailing update's bytes
     pack      bytes: codes 1 B + packed bits/8 B per element, scale/zero
     ingest    bytes: W in (2 or 4 B) + float32 out per element
+    prep_order  the min-pivot order only: flops n³/3 (the pivoted float64
+              elimination that produces it)
     """
-    w = {k: 0.0 for k in ("hessian", "cholesky", "sweep", "trailing", "pack", "ingest")}
+    w = {k: 0.0 for k in ("hessian", "cholesky", "sweep", "trailing", "pack", "ingest",
+                          "prep_order")}
     for p in probs:
         m, n, T = p.m, p.n, p.T
         w["hessian"] += T * n * (n + 1)
         w["cholesky"] += 2.0 * n ** 3 / 3.0
+        if p.order == "minpivot":
+            w["prep_order"] += n ** 3 / 3.0
         ng = -(-n // p.group)
         fused = n % 4 == 0 and n > block
         if fused:
@@ -249,7 +254,7 @@ def kernel_work(probs, block: int):
             w["sweep"] += 9 * m * bw + 4 * bw * bw + 5 * m * (-(-bw // p.group))
         w["pack"] += m * n + m * n * p.bits / 8 + 5 * m * ng
         w["ingest"] += m * n * (p.W.element_size() + 4)
-    units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s",
+    units = {"hessian": "TFLOP/s", "cholesky": "TFLOP/s", "prep_order": "TFLOP/s",
              "sweep": "GB/s", "trailing": "GB/s", "pack": "GB/s", "ingest": "GB/s"}
     return {k: (units[k], v) for k, v in w.items()}
 
