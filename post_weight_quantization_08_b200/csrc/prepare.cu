@@ -992,8 +992,8 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
                        int ntasks, int* sync_base, int32_t* info, uint32_t spin) {
   extern __shared__ double sm[];
   __shared__ int s_role, s_ok, s_bad, s_got, s_fail;
-  __shared__ int s_htask[kGroups], s_hok[kGroups];
-  __shared__ WorkTask s_hwt[kGroups];
+  __shared__ int s_htask[kGroups][2], s_hok[kGroups], s_hready[kGroups];
+  __shared__ WorkTask s_hwt[kGroups][2];
   // the task numbering's slot prefix, after the tiles
   int* prefix = reinterpret_cast<int*>(sm + kTileDoubles);
   __shared__ volatile int s_stop;
@@ -1139,18 +1139,27 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   // an update tile would otherwise come from DRAM on the critical path)
   if (ht == 0) {
     const int c = atomicAdd(&S.ctrl[0], 1);
-    s_htask[h] = c;
-    if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
+    s_htask[h][0] = c;
+    if (c < ntasks) s_hwt[h][0] = work_task(c, N, prefix, np, A, M, S);
   }
+  if (ht == 0) s_hready[h] = 0;
   bar_sync(hbar, 128);
-  // Per task three group barriers: in the wait (the dependencies are final),
+  // Per task two or three group barriers: in the wait (the dependencies are
+  // final; skipped when thread 0 saw them final during the task before),
   // after the copies (the tiles have landed; the next task is decoded), after
-  // the stores.  The next task's record is written before the second and read
-  // after the third.
-  for (;;) {
-    if (s_htask[h] >= ntasks) return;
-    const WorkTask t = s_hwt[h];
-    if (!half_wait(t, &S.ctrl[2], info, &s_hok[h], spin, ht, hbar)) return;
+  // the stores.  Task records alternate between two slots: round r reads slot
+  // r & 1 at its top and thread 0 writes the next one into the other slot
+  // before the second barrier; that slot's last readers (round r − 1) passed
+  // the second barrier of round r − 1 before.  The readiness flag is written
+  // before the third barrier and read after it.
+  for (int rd = 0;; rd ^= 1) {
+    if (s_htask[h][rd] >= ntasks) return;
+    const WorkTask t = s_hwt[h][rd];
+    if (!s_hready[h] && !half_wait(t, &S.ctrl[2], info, &s_hok[h], spin, ht, hbar)) return;
+    // the next task's number, claimed once this one can start: the atomic's
+    // round trip runs under the copies (it is decoded once they are issued)
+    int claimed = 0;
+    if (ht == 0) claimed = atomicAdd(&S.ctrl[0], 1);
     half_copy(x, t.x, np, ht);
     half_copy(y, t.y, np, ht);
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -1165,18 +1174,29 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
         for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
     }
     if (ht == 0) {
-      int c = atomicAdd(&S.ctrl[0], 1);
+      int c = claimed;
       if (*reinterpret_cast<volatile int*>(&S.ctrl[2])) c = ntasks;
-      s_htask[h] = c;                         // read at the top of the next round
-      if (c < ntasks) s_hwt[h] = work_task(c, N, prefix, np, A, M, S);
+      s_htask[h][rd ^ 1] = c;                 // read at the top of the next round
+      if (c < ntasks) s_hwt[h][rd ^ 1] = work_task(c, N, prefix, np, A, M, S);
     }
     copy_wait_all();
     bar_sync(hbar, 128);
-    if (s_htask[h] < ntasks && s_hwt[h].subtract) {
-      // 64 rows × four 128-byte lines: two lines a thread
-      const double* o = s_hwt[h].out + (int64_t)(ht >> 1) * np + (ht & 1) * 32;
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(o));
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(o + 16));
+    const bool more = s_htask[h][rd ^ 1] < ntasks;
+    const WorkTask& nx = s_hwt[h][rd ^ 1];
+    // thread 0 takes one look at the next task's dependencies, the loads in
+    // flight under the products
+    int nv[3] = {0, 0, 0};
+    if (ht == 0 && more) {
+#pragma unroll
+      for (int d = 0; d < 3; ++d)
+        if (d < nx.ndep) nv[d] = ld_relaxed(nx.dep[d]);
+    }
+    if (more && ht >= 64 && nx.subtract) {
+      // 64 rows × four 128-byte lines, by the group's last two warps (so that
+      // thread 0's fence below does not wait for them)
+      const double* o = nx.out + (int64_t)(ht - 64) * np;
+#pragma unroll
+      for (int l = 0; l < 4; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(o + 16 * l));
     }
     if (t.nt) {
       if (t.subtract) half_mm<true, true>(x, y, acc, hw, lane);
@@ -1184,6 +1204,15 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     } else {
       if (t.subtract) half_mm<false, true>(x, y, acc, hw, lane);
       else half_mm<false, false>(x, y, acc, hw, lane);
+    }
+    if (ht == 0) {
+      // every dependency already final: the acquire now (before this thread's
+      // stores, so the fence waits for nothing), and no wait next round
+      bool ready = more;
+#pragma unroll
+      for (int d = 0; d < 3; ++d) ready = ready && (d >= nx.ndep || nv[d] >= nx.target[d]);
+      if (ready) asm volatile("fence.acq_rel.gpu;" ::: "memory");
+      s_hready[h] = ready ? 1 : 0;
     }
     half_store(t.out, np, acc, hw, lane);
     bar_sync(hbar, 128);                          // the group's stores are issued
