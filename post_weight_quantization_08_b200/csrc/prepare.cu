@@ -790,18 +790,25 @@ __device__ __forceinline__ void half_store(double* out, int64_t ld, const double
           make_double2(acc[i][j][0], acc[i][j][1]);
 }
 
-// One 64×64 float64 tile (leading dimension ld) into shared memory as it is,
-// by a half's 128 threads: 16-byte cp.async through L2 only (tiles are
-// rewritten by other CTAs of the same launch).  The caller commits the group.
-__device__ __forceinline__ void half_copy(double (*dst)[LDM], const double* src, int64_t ld,
-                                          int ht) {
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int e = ht + 128 * k;             // 2048 chunks of 16 bytes
-    const int r = e >> 5, c = (e & 31) * 2;
-    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&dst[r][c]));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + (int64_t)r * ld + c)
-                 : "memory");
+// Two 64×64 float64 tiles (leading dimension ld) into shared memory as they
+// are, by the 96 threads of a group's last three warps (w = 0..95): 16-byte
+// cp.async through L2 only (tiles are rewritten by other CTAs of the same
+// launch).  The group's first warp meanwhile loads its part of the output
+// tile and its thread 0 decodes the next task.  The caller commits.
+__device__ __forceinline__ void group_copy2(double (*dx)[LDM], const double* sx,
+                                            double (*dy)[LDM], const double* sy, int64_t ld,
+                                            int w) {
+#pragma unroll 4
+  for (int k = 0; k < 43; ++k) {
+    const int e = w + 96 * k;               // 4096 chunks of 16 bytes
+    if (e < 4096) {
+      const int q = e & 2047, r = q >> 5, c = (q & 31) * 2;
+      double (*dst)[LDM] = (e < 2048) ? dx : dy;
+      const double* src = (e < 2048) ? sx : sy;
+      const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(&dst[r][c]));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
+                   "l"(src + (int64_t)r * ld + c) : "memory");
+    }
   }
 }
 
@@ -1160,9 +1167,10 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     // round trip runs under the copies (it is decoded once they are issued)
     int claimed = 0;
     if (ht == 0) claimed = atomicAdd(&S.ctrl[0], 1);
-    half_copy(x, t.x, np, ht);
-    half_copy(y, t.y, np, ht);
-    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (hw > 0) {
+      group_copy2(x, t.x, y, t.y, np, ht - 32);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
     // C −= X·B starts from C; out = X·B from zero
     double acc[4][4][2];
     if (t.subtract) {
