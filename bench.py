@@ -378,14 +378,14 @@ def est_cost(p) -> float:
 
 def factor_workers(arg, nprobs, device):
     """Most worker CTAs a factorisation may use: ``arg`` when given (0: every
-    SM but one); by default (-1) three quarters of the SMs when the step has
+    SM but one); by default (-1) three fifths of the SMs when the step has
     eight or more problems, so that sweeps of factorised problems run beside
     the next factorisation, and every SM but one otherwise."""
     if arg >= 0:
         return int(arg)
     if nprobs < 8:
         return 0
-    return int(0.76 * torch.cuda.get_device_properties(device).multi_processor_count)
+    return int(0.6 * torch.cuda.get_device_properties(device).multi_processor_count)
 
 
 class Job:
@@ -1659,7 +1659,7 @@ def main(argv=None):
                     help="streams the quantize calls are spread over")
     ap.add_argument("--factor-workers", type=int, default=-1,
                     help="most worker CTAs a factorisation may use (0: every SM but one; "
-                         "default: three quarters of the SMs when a step has eight or more "
+                         "default: three fifths of the SMs when a step has eight or more "
                          "problems)")
     ap.add_argument("--profile-steps", type=int, default=2,
                     help="steps of the serialised per-kernel timing pass")
