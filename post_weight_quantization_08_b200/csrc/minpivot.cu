@@ -47,41 +47,25 @@ mp_init_kernel(const float* __restrict__ H, int64_t n, int64_t ld, const double*
   S[a * ld + b] = v;
 }
 
-// Block-wide argmin of (value, −index): the smallest value, ties to the
-// larger index.  Returns the index (or −1 when every value is infinite).
-__device__ int block_argmin(double v, int idx, double* sv, int* si) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const double ov = __shfl_down_sync(0xffffffffu, v, o);
-    const int oi = __shfl_down_sync(0xffffffffu, idx, o);
-    if (ov < v || (ov == v && oi > idx)) { v = ov; idx = oi; }
-  }
-  if (lane == 0) { sv[warp] = v; si[warp] = idx; }
-  __syncthreads();
-  if (warp == 0) {
-    v = (lane < MP_THREADS / 32) ? sv[lane] : INFINITY;
-    idx = (lane < MP_THREADS / 32) ? si[lane] : -1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ov = __shfl_down_sync(0xffffffffu, v, o);
-      const int oi = __shfl_down_sync(0xffffffffu, idx, o);
-      if (ov < v || (ov == v && oi > idx)) { v = ov; idx = oi; }
-    }
-    if (lane == 0) { sv[0] = v; si[0] = (v < INFINITY) ? idx : -1; }
-  }
-  __syncthreads();
-  const int r = si[0];
-  __syncthreads();
-  return r;
+// (value, index) order of the pivot search: the smaller value, ties to the
+// larger index.  A total order, so any reduction order gives the same pivot.
+__device__ __forceinline__ bool mp_better(double ov, int oi, double v, int i) {
+  return ov < v || (ov == v && oi > i);
 }
 
 // One panel of pw ≤ MP_PANEL dependent steps in one CTA.  The Schur diagonal
 // d and, when they fit (lp_smem), the panel's factor columns live in shared
 // memory for the panel; d goes back to global memory at the end and the
 // columns are written to Lp (row i at i·MP_PANEL) for the trailing update.
-// The pivot is the diagonal entry itself (the factorisation's own, updated
-// value), so the only global reads per step are row j of S (and, without
+//
+// Thread t owns rows t, t + MP_THREADS, …: it alone updates their d and
+// panel columns, and while it does so it keeps the running pivot candidate
+// of its rows.  One barrier a step: each warp's best candidate goes to a
+// shared slot (two sets, alternating by step), and after the barrier every
+// thread reduces the slots itself.  The pivot value comes with the candidate
+// (the owner of row j sets d_j = ∞ during the same step); row j's panel
+// columns (written in earlier steps, before this step's barrier) are read in
+// place.  The only global reads per step are row j of S (and, without
 // lp_smem, the rows' panel columns), all issued before use.
 __global__ void __launch_bounds__(MP_THREADS, 1)
 mp_panel_kernel(const double* __restrict__ S, int64_t n, int64_t ld, double* __restrict__ dg,
@@ -91,37 +75,52 @@ mp_panel_kernel(const double* __restrict__ S, int64_t n, int64_t ld, double* __r
   double* d = smem;                                  // n
   double* lps = smem + ((n + 1) & ~int64_t(1));      // n rows of pw + 1 when lp_smem
   const int lds = pw + 1;                            // odd stride: no bank conflicts
-  __shared__ double sv[32];
-  __shared__ int si[32];
-  __shared__ double prow[MP_PANEL];
-  const int tid = threadIdx.x;
+  constexpr int NW = MP_THREADS / 32;
+  __shared__ double sv[2][NW];
+  __shared__ int si[2][NW];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (*reinterpret_cast<volatile int32_t*>(info) != 0) return;
   for (int64_t i = tid; i < n; i += MP_THREADS) d[i] = dg[i];
   if (lp_smem)
     for (int64_t e = tid; e < n * lds; e += MP_THREADS) lps[e] = 0.0;
   __syncthreads();
+  // the first candidate of this thread's rows
+  double bv = INFINITY;
+  int bi = -1;
+  for (int64_t i = tid; i < n; i += MP_THREADS) {
+    const double v = d[i];
+    if (v < INFINITY && mp_better(v, (int)i, bv, bi)) { bv = v; bi = (int)i; }
+  }
   const int steps = (int)((n - t0 < pw) ? (n - t0) : pw);
   for (int k = 0; k < steps; ++k) {
-    // the pivot: smallest remaining diagonal, ties to the larger index
-    double bv = INFINITY;
-    int bi = -1;
-    for (int64_t i = tid; i < n; i += MP_THREADS) {
-      const double v = d[i];
-      if (v < bv || (v == bv && (int)i > bi)) { bv = v; bi = (int)i; }
+    const int b = k & 1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_down_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_down_sync(0xffffffffu, bi, o);
+      if (mp_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
     }
-    const int j = block_argmin(bv, bi, sv, si);
-    const double piv = (j >= 0) ? d[j] : 0.0;
-    if (!(piv >= 2.2250738585072014e-308 && piv <= 1.7976931348623157e308)) {
+    if (lane == 0) { sv[b][warp] = bv; si[b][warp] = bi; }
+    __syncthreads();
+    double piv = sv[b][0];
+    int j = si[b][0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) {
+      const double ov = sv[b][w];
+      const int oi = si[b][w];
+      if (mp_better(ov, oi, piv, j)) { piv = ov; j = oi; }
+    }
+    if (!(piv < INFINITY)) j = -1;
+    if (j < 0 || !(piv >= 2.2250738585072014e-308 && piv <= 1.7976931348623157e308)) {
       if (tid == 0) report(info, GPTQ_ERR_NOT_PD, n - 1 - (t0 + k));   // uniform exit
       break;
     }
-    if (tid < MP_PANEL)
-      prow[tid] = (tid < k) ? (lp_smem ? lps[(int64_t)j * lds + tid]
-                                       : Lp[(int64_t)j * MP_PANEL + tid]) : 0.0;
     if (tid == 0) elim[t0 + k] = j;
-    __syncthreads();
     const double rp = 1.0 / sqrt(piv);
+    bv = INFINITY;
+    bi = -1;
     if (lp_smem) {
+      const double* lj = lps + (int64_t)j * lds;    // row j's panel columns, q < k
       // row j of S for all of this thread's rows first, then the sums
       constexpr int R = 8;                           // rows per thread per pass
       for (int64_t i0 = tid; i0 < n; i0 += (int64_t)R * MP_THREADS) {
@@ -134,26 +133,39 @@ mp_panel_kernel(const double* __restrict__ S, int64_t n, int64_t ld, double* __r
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           const int64_t i = i0 + (int64_t)r * MP_THREADS;
-          if (i >= n || i == j) continue;
+          if (i >= n) continue;
+          if (i == j) {                              // this thread owns the pivot row
+            d[i] = INFINITY;
+            lps[i * lds + k] = 0.0;
+            continue;
+          }
           const double di = d[i];
           if (!(di < INFINITY)) continue;
           const double* li = lps + i * lds;
           double c0 = sj[r], c1 = 0.0;
           int q = 0;
           for (; q + 1 < k; q += 2) {
-            c0 -= li[q] * prow[q];
-            c1 -= li[q + 1] * prow[q + 1];
+            c0 -= li[q] * lj[q];
+            c1 -= li[q + 1] * lj[q + 1];
           }
-          if (q < k) c0 -= li[q] * prow[q];
+          if (q < k) c0 -= li[q] * lj[q];
           const double l = (c0 + c1) * rp;
           lps[i * lds + k] = l;
-          d[i] = di - l * l;
+          const double dn = di - l * l;
+          d[i] = dn;
+          if (dn < INFINITY && mp_better(dn, (int)i, bv, bi)) { bv = dn; bi = (int)i; }
         }
       }
     } else {
+      const double* lj = Lp + (int64_t)j * MP_PANEL;
       for (int64_t i = tid; i < n; i += MP_THREADS) {
+        if (i == j) {
+          d[i] = INFINITY;
+          Lp[i * MP_PANEL + k] = 0.0;
+          continue;
+        }
         const double di = d[i];
-        if (i == j || !(di < INFINITY)) continue;
+        if (!(di < INFINITY)) continue;
         double c = S[(int64_t)j * ld + i];            // S is symmetric: row j
         const double2* li = reinterpret_cast<const double2*>(Lp + i * MP_PANEL);
 #pragma unroll
@@ -168,23 +180,19 @@ mp_panel_kernel(const double* __restrict__ S, int64_t n, int64_t ld, double* __r
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int s0 = 16 * h + 2 * q;
-            c -= ((s0 < k) ? lv[q].x : 0.0) * prow[s0];
-            c -= ((s0 + 1 < k) ? lv[q].y : 0.0) * prow[s0 + 1];
+            c -= ((s0 < k) ? lv[q].x : 0.0) * ((s0 < k) ? lj[s0] : 0.0);
+            c -= ((s0 + 1 < k) ? lv[q].y : 0.0) * ((s0 + 1 < k) ? lj[s0 + 1] : 0.0);
           }
         }
         const double l = c * rp;
         Lp[i * MP_PANEL + k] = l;
-        d[i] = di - l * l;
+        const double dn = di - l * l;
+        d[i] = dn;
+        if (dn < INFINITY && mp_better(dn, (int)i, bv, bi)) { bv = dn; bi = (int)i; }
       }
     }
-    __syncthreads();
-    if (tid == 0) {
-      if (lp_smem) lps[(int64_t)j * lds + k] = 0.0;
-      else Lp[(int64_t)j * MP_PANEL + k] = 0.0;
-      d[j] = INFINITY;
-    }
-    __syncthreads();
   }
+  __syncthreads();
   for (int64_t i = tid; i < n; i += MP_THREADS) dg[i] = d[i];
   if (lp_smem) {
     // the panel's columns out for the trailing update (zeros past pw)

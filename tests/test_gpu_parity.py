@@ -107,6 +107,51 @@ def test_min_pivot_identity_and_diagonal():
     assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("n", [1500, 3000])
+def test_min_pivot_block_diagonal(n):
+    """A block-diagonal H (blocks of 1–3 columns): every step of the GPU's order
+    takes a smallest Schur diagonal, checked along the order with the blocks'
+    own Schur complements (exact, cheap at any n).  n = 3000 runs the panel
+    with its factor columns in global memory (they no longer fit in shared
+    memory), n = 1500 with them in shared memory."""
+    import post_weight_quantization_08_b200 as g
+    rng = np.random.default_rng(n)
+    sizes = []
+    while sum(sizes) < n:
+        sizes.append(int(min(rng.integers(1, 4), n - sum(sizes))))
+    H = np.zeros((n, n))
+    blocks, owner = [], np.empty(n, dtype=np.int64)
+    c0 = 0
+    for b, sz in enumerate(sizes):
+        A = rng.standard_normal((sz, sz))
+        B = A @ A.T + np.diag(rng.uniform(0.5, 2.0, sz))
+        H[c0:c0 + sz, c0:c0 + sz] = B
+        blocks.append([list(range(c0, c0 + sz)), B.copy()])
+        owner[c0:c0 + sz] = b
+        c0 += sz
+    Ht = torch.tensor(H.astype(np.float32), device=DEV)
+    perm = g.prepare(Ht, 0.0, "minpivot")["perm"].cpu().numpy()
+    assert sorted(perm.tolist()) == list(range(n))
+    # the float32 H the GPU saw, in float64, block by block
+    H32 = H.astype(np.float32).astype(np.float64)
+    for blk in blocks:
+        cols = blk[0]
+        blk[1] = H32[np.ix_(cols, cols)].copy()
+    d = np.diag(H32).copy()
+    alive = np.ones(n, dtype=bool)
+    for t, j in enumerate(perm[::-1]):
+        dm = np.where(alive, d, np.inf).min()
+        assert alive[j] and d[j] <= dm + 1e-10 * abs(dm), (t, j, d[j], dm)
+        cols, S = blocks[owner[j]]
+        a = cols.index(j)
+        c = S[:, a].copy()
+        S -= np.outer(c, c) / c[a]
+        alive[j] = False
+        for q, col in enumerate(cols):
+            if alive[col]:
+                d[col] = S[q, q]
+
+
 def test_min_pivot_not_positive_definite():
     """A negative pivot is met at the first elimination step: processed last."""
     import post_weight_quantization_08_b200 as g
