@@ -125,8 +125,8 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 
 namespace gptq {
 
+// 2-D tiled TMA load of one box at (x = inner coordinate, y) into shared
 // memory, completing on `bar`.  The box lands in this CTA only.
-// memory, completing on `bar`.  No cluster multicast.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y,
                                             uint64_t* bar) {
   asm volatile(
