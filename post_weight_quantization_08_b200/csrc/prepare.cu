@@ -730,7 +730,7 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
   if (warp == 0) lower_syrk_group(tt, l, 4, lane);
 }
 
-// 64×64 float64 tile products C = X·B of a worker half (4 warps).  Warp w
+// 64×64 float64 tile products C = X·B of a worker group (4 warps).  Warp w
 // owns rows 32·(w/2) .. +32 and columns 32·(w%2) .. +32 of C: 4 × 4
 // accumulator blocks of 8×8.  X is held row-major (row r of C, column q of
 // the sum).  B comes in one of two layouts, both copied from global memory
@@ -742,7 +742,7 @@ __device__ __forceinline__ void lower_syrk(double (*tt)[LDM], const double (*l)[
 // With NEG the products are subtracted (acc −= X·B): the accumulators start
 // from the tile being updated.
 template <bool NT, bool NEG>
-__device__ __forceinline__ void half_mm(const double (*x)[LDM], const double (*y)[LDM],
+__device__ __forceinline__ void group_mm(const double (*x)[LDM], const double (*y)[LDM],
                                         double acc[4][4][2], int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
@@ -763,7 +763,7 @@ __device__ __forceinline__ void half_mm(const double (*x)[LDM], const double (*y
 // The part of a 64×64 output tile (leading dimension ld) that a lane's
 // accumulators cover: into the accumulators (the start of C −= X·B), and
 // back out.
-__device__ __forceinline__ void half_load_acc(const double* out, int64_t ld, double acc[4][4][2],
+__device__ __forceinline__ void group_load_acc(const double* out, int64_t ld, double acc[4][4][2],
                                               int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
@@ -778,7 +778,7 @@ __device__ __forceinline__ void half_load_acc(const double* out, int64_t ld, dou
     }
 }
 
-__device__ __forceinline__ void half_store(double* out, int64_t ld, const double acc[4][4][2],
+__device__ __forceinline__ void group_store(double* out, int64_t ld, const double acc[4][4][2],
                                            int hw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int rb = 32 * (hw >> 1), cb = 32 * (hw & 1);
@@ -969,7 +969,7 @@ __device__ __forceinline__ bool deps_final(const WorkTask& t) {
 // tile loads need); false on abort or time-out (reported).  One barrier:
 // thread 0 writes *s_ok again only in the group's next wait, after two more
 // group barriers that every reader has passed.
-__device__ bool half_wait(const WorkTask& t, int* abortp, int32_t* info, int* s_ok, uint32_t spin,
+__device__ bool group_wait_deps(const WorkTask& t, int* abortp, int32_t* info, int* s_ok, uint32_t spin,
                           int ht, int hbar) {
   if (ht == 0) {
     bool ok = false;
@@ -1162,7 +1162,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
   for (int rd = 0;; rd ^= 1) {
     if (s_htask[h][rd] >= ntasks) return;
     const WorkTask t = s_hwt[h][rd];
-    if (!s_hready[h] && !half_wait(t, &S.ctrl[2], info, &s_hok[h], spin, ht, hbar)) return;
+    if (!s_hready[h] && !group_wait_deps(t, &S.ctrl[2], info, &s_hok[h], spin, ht, hbar)) return;
     // the next task's number, claimed once this one can start: the atomic's
     // round trip runs under the copies (it is decoded once they are issued)
     int claimed = 0;
@@ -1174,7 +1174,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
     // C −= X·B starts from C; out = X·B from zero
     double acc[4][4][2];
     if (t.subtract) {
-      half_load_acc(t.out, np, acc, hw, lane);
+      group_load_acc(t.out, np, acc, hw, lane);
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -1207,11 +1207,11 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       for (int l = 0; l < 4; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(o + 16 * l));
     }
     if (t.nt) {
-      if (t.subtract) half_mm<true, true>(x, y, acc, hw, lane);
-      else half_mm<true, false>(x, y, acc, hw, lane);
+      if (t.subtract) group_mm<true, true>(x, y, acc, hw, lane);
+      else group_mm<true, false>(x, y, acc, hw, lane);
     } else {
-      if (t.subtract) half_mm<false, true>(x, y, acc, hw, lane);
-      else half_mm<false, false>(x, y, acc, hw, lane);
+      if (t.subtract) group_mm<false, true>(x, y, acc, hw, lane);
+      else group_mm<false, false>(x, y, acc, hw, lane);
     }
     if (ht == 0) {
       // every dependency already final: the acquire now (before this thread's
@@ -1222,7 +1222,7 @@ chol_persistent_kernel(double* __restrict__ A, double* __restrict__ M,
       if (ready) asm volatile("fence.acq_rel.gpu;" ::: "memory");
       s_hready[h] = ready ? 1 : 0;
     }
-    half_store(t.out, np, acc, hw, lane);
+    group_store(t.out, np, acc, hw, lane);
     bar_sync(hbar, 128);                          // the group's stores are issued
     // a thread of the second warp publishes the result (the release orders the
     // group's stores, through the barrier, before the flag) while thread 0
