@@ -376,6 +376,24 @@ def est_cost(p) -> float:
     return (2.0 / 3.0) * p.n ** 3 / 30e12 + 3.0 * p.m * p.n * p.n / 1e15
 
 
+def lane_plans(probs, lanes):
+    """Problems per lane for the Hessians and factorisations: most expensive
+    first (est_cost), each to the lane with the least work so far."""
+    nl = max(1, min(int(lanes), len(probs)))
+    plans, load = [[] for _ in range(nl)], [0.0] * nl
+    for k in sorted(range(len(probs)), key=lambda k: -est_cost(probs[k])):
+        ln = min(range(nl), key=lambda i: load[i])
+        plans[ln].append(k)
+        load[ln] += est_cost(probs[k])
+    return plans
+
+
+def quantize_order(probs):
+    """Order of the quantize calls: the longest sweep chain (most blocks)
+    first, then the most rows."""
+    return sorted(range(len(probs)), key=lambda k: ((-probs[k].n) // probs[k].block, -probs[k].m))
+
+
 def factor_workers(arg, nprobs, device):
     """Most worker CTAs a factorisation may use: ``arg`` when given (0: every
     SM but one); by default (-1) three fifths of the SMs when the step has
@@ -433,19 +451,12 @@ class Job:
                 "g_idx": torch.empty(n, dtype=torch.int32, device=device),
                 "loss": torch.empty(m, dtype=torch.float32, device=device),
             })
-        nl = max(1, min(int(lanes), len(probs)))
-        self.lanes = [{"s": torch.cuda.Stream(device=device), "plan": [], "load": 0.0}
-                      for _ in range(nl)]
-        for k in sorted(range(len(probs)), key=lambda k: -est_cost(probs[k])):
-            lane = min(self.lanes, key=lambda ln: ln["load"])
-            lane["plan"].append(k)
-            lane["load"] += est_cost(probs[k])
+        self.lanes = [{"s": torch.cuda.Stream(device=device), "plan": plan}
+                      for plan in lane_plans(probs, lanes)]
         self.cs = torch.cuda.Stream(device=device)            # host copies
         nq = max(1, min(int(qstreams), len(probs)))
         self.qs = [torch.cuda.Stream(device=device) for _ in range(nq)]
-        # quantize order: longest sweep chain (most blocks) first, then most rows
-        self.qorder = sorted(range(len(probs)),
-                             key=lambda k: ((-probs[k].n) // probs[k].block, -probs[k].m))
+        self.qorder = quantize_order(probs)
 
     def prepare_problem(self, it, s, x_ready=None):
         """Hessian and factorisation of one problem on stream ``s``; ``x_ready``:
