@@ -1611,8 +1611,9 @@ def run_reference_frontend(args, world):
 
 def run_reference(args, rank, world):
     """The oracle arm: each step one bounded sample of the same workload, the
-    float64 oracle over one whole problem of the step (Hessian, factorisation,
-    sweep), taking the step's problems in turn."""
+    float64 oracle on one problem of the step (its Hessian and factorisation in
+    full, the per-row pass on CPU_SAMPLE_ROWS rows scaled to all rows), taking
+    the step's problems in turn."""
     if rank != 0:
         return None
     if args.frontend != "gptq":
